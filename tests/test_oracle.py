@@ -1,0 +1,321 @@
+"""Pins for the CPU oracle, independent of the oracle's own code.
+
+Each test fixes a property the oracle must satisfy by a route other than the
+oracle itself: hand-built blocks whose values follow from the closed form
+d*sc*q - dmin*m, a full sweep of the fp16 scale field against numpy's binary16
+conversion, the installed ``gguf.quants.dequantize`` library routine on random
+blocks, exact rational brute force on tiny matmuls, and hand-worked tile maps
+(tests/golden/).  No GPU is needed.
+"""
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+Q8_0, Q4_K, Q6_K = oracle.Q8_0, oracle.Q4_K, oracle.Q6_K
+
+
+def bits(a):
+    return np.asarray(a, dtype=np.float32).view(np.uint32)
+
+
+# ----------------------------------------------------------------------------
+# block geometry (README "Codec reference" table)
+# ----------------------------------------------------------------------------
+def test_codec_table_matches_readme_and_gguf():
+    import gguf
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "codec_table.txt")) if l[0] != "#"]
+    assert len(rows) == 3
+    for name, vpb, _bits, bpb, tid in rows:
+        vpb, bpb, tid = int(vpb), int(bpb), int(tid)
+        assert oracle.block_info(tid) == (vpb, bpb)
+        assert synth.BLOCK_VALUES[tid] == vpb and synth.BLOCK_BYTES[tid] == bpb
+        gt = gguf.GGMLQuantizationType(tid)
+        assert gt.name.lower() == name
+        assert tuple(gguf.GGML_QUANT_SIZES[gt]) == (vpb, bpb)
+
+
+# ----------------------------------------------------------------------------
+# fp16 scale field: every binary16 pattern, through the q8_0 decoder with q=1
+# ----------------------------------------------------------------------------
+def test_fp16_scale_all_patterns():
+    pat = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    blocks = np.zeros((65536, 34), dtype=np.uint8)
+    blocks[:, 0:2] = pat.view(np.uint8).reshape(-1, 2)
+    blocks[:, 2:] = 1  # every code = +1  ->  y = d * 1 = d
+    y = oracle.dequantize(Q8_0, blocks.reshape(65536, 34), 32)[:, 0]
+    ref = pat.view(np.float16).astype(np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(y), nan)
+    assert np.array_equal(bits(y)[~nan], bits(ref)[~nan])   # incl. subnormals and -0.0
+
+
+# ----------------------------------------------------------------------------
+# q4_K hand-built blocks
+# ----------------------------------------------------------------------------
+def q4k_block(d=1.0, dmin=0.0, scale_bytes=None, qs=None):
+    b = np.zeros(144, dtype=np.uint8)
+    b[0:2] = np.array([d], dtype=np.float16).view(np.uint8)
+    b[2:4] = np.array([dmin], dtype=np.float16).view(np.uint8)
+    if scale_bytes is not None:
+        b[4:16] = scale_bytes
+    if qs is not None:
+        b[16:144] = qs
+    return b
+
+
+def test_q4k_codes_pass_through():
+    # d=1, dmin=0, every 6-bit scale code 1, every min code 0: y equals the code.
+    # Scale codes 0..3 are the low six bits of bytes 0..3; codes 4..7 take their
+    # low four bits from the low nibbles of bytes 8..11; min codes 0..3 live in
+    # bytes 4..7, min codes 4..7 in the high nibbles of bytes 8..11.
+    s = np.array([1, 1, 1, 1, 0, 0, 0, 0, 1, 1, 1, 1], dtype=np.uint8)
+    # value 64c + l is the low nibble of qs[32c + l], 64c + 32 + l its high nibble;
+    # choose both nibbles = l mod 16 so that value v carries code v mod 16.
+    qs = np.array([(l % 16) | ((l % 16) << 4) for c in range(4) for l in range(32)], dtype=np.uint8)
+    y = oracle.dequantize(Q4_K, q4k_block(1.0, 0.0, s, qs)[None], 256)[0]
+    assert np.array_equal(y, (np.arange(256) % 16).astype(np.float32))
+
+
+def _single_field(kind, j):
+    """Scale bytes with exactly one 6-bit code (scale or min of sub-block j) = 63."""
+    s = np.zeros(12, dtype=np.uint8)
+    if kind == "sc":
+        if j < 4:
+            s[j] = 63
+        else:
+            s[j + 4] = 0x0F      # low four bits
+            s[j - 4] = 0xC0      # bits 4..5 from the top two bits
+    else:
+        if j < 4:
+            s[j + 4] = 63
+        else:
+            s[j + 4] = 0xF0      # low four bits from the high nibble
+            s[j] = 0xC0          # bits 4..5
+    return s
+
+
+@pytest.mark.parametrize("kind", ["sc", "m"])
+@pytest.mark.parametrize("j", range(8))
+def test_q4k_single_field(kind, j):
+    # d = dmin = 1, all codes q = 1: y = sc_j - m_j, so only sub-block j moves.
+    blk = q4k_block(1.0, 1.0, _single_field(kind, j), np.full(128, 0x11, dtype=np.uint8))
+    y = oracle.dequantize(Q4_K, blk[None], 256)[0]
+    sub = np.zeros(256, dtype=np.int64)
+    for v in range(256):
+        sub[v] = 2 * (v // 64) + (v % 64) // 32
+    expect = np.where(sub == j, 63.0 if kind == "sc" else -63.0, 0.0).astype(np.float32)
+    assert np.array_equal(y, expect)
+
+
+def test_q4k_min_only():
+    # dmin = 1, every min code 63, every scale code 0, q = 0: y = -63 everywhere.
+    s = np.zeros(12, dtype=np.uint8)
+    for j in range(8):
+        s = s | _single_field("m", j)
+    y = oracle.dequantize(Q4_K, q4k_block(2.0, 1.0, s, np.zeros(128, np.uint8))[None], 256)[0]
+    assert np.array_equal(y, np.full(256, -63.0, dtype=np.float32))
+
+
+def test_q4k_scale_product_rounding():
+    # y = fp32(fp32(d)*sc)*q - fp32(dmin*m): with d = 1/3 in fp16, sc = 63, q = 15
+    # the two-rounding result is reproduced from numpy float32 scalars.
+    s = _single_field("sc", 2) | _single_field("m", 2)
+    d = np.float16(1.0 / 3.0)
+    dmin = np.float16(0.1)
+    blk = q4k_block(float(d), float(dmin), s, np.full(128, 0xFF, dtype=np.uint8))
+    y = oracle.dequantize(Q4_K, blk[None], 256)[0]
+    f = np.float32
+    expect = f(f(f(d) * f(63)) * f(15)) - f(f(dmin) * f(63))
+    assert bits(y[64 + 0]) == bits(expect)            # sub-block 2 = low nibbles of c = 1
+    assert bits(y[0]) == bits(f(f(f(d) * f(0)) * f(15)) - f(f(dmin) * f(0)))
+
+
+# ----------------------------------------------------------------------------
+# q6_K hand-built blocks
+# ----------------------------------------------------------------------------
+def q6k_block(codes, scales, d=1.0):
+    """codes: 256 ints in 0..63 placed by the q6_K layout; scales: 16 int8."""
+    b = np.zeros(210, dtype=np.uint8)
+    ql, qh = np.zeros(128, np.uint8), np.zeros(64, np.uint8)
+    for v in range(256):
+        h, t, l = v // 128, (v % 128) // 32, v % 32
+        c = int(codes[v])
+        ql[64 * h + 32 * (t & 1) + l] |= (c & 15) << (4 * (t >> 1))
+        qh[32 * h + l] |= (c >> 4) << (2 * t)
+    b[0:128], b[128:192] = ql, qh
+    b[192:208] = np.asarray(scales, dtype=np.int8).view(np.uint8)
+    b[208:210] = np.array([d], dtype=np.float16).view(np.uint8)
+    return b
+
+
+def test_q6k_all_codes():
+    codes = np.arange(256) % 64
+    y = oracle.dequantize(Q6_K, q6k_block(codes, np.ones(16))[None], 256)[0]
+    assert np.array_equal(y, (codes - 32).astype(np.float32))     # q spans -32..31
+
+
+def test_q6k_negative_scales():
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 64, 256)
+    scales = np.arange(16) - 8          # includes negative and zero scales
+    y = oracle.dequantize(Q6_K, q6k_block(codes, scales, d=0.5)[None], 256)[0]
+    expect = np.array([0.5 * scales[v // 16] * (codes[v] - 32) for v in range(256)], dtype=np.float32)
+    assert np.array_equal(y, expect)
+
+
+# ----------------------------------------------------------------------------
+# q8_0 hand-built blocks and zero blocks
+# ----------------------------------------------------------------------------
+def test_q8_0_all_codes():
+    b = np.zeros((8, 34), dtype=np.uint8)
+    b[:, 0:2] = np.array([1.0], dtype=np.float16).view(np.uint8)
+    b[:, 2:] = np.arange(256, dtype=np.uint32).astype(np.uint8).reshape(8, 32)
+    y = oracle.dequantize(Q8_0, b.reshape(1, 8 * 34), 256)[0]
+    assert np.array_equal(y, np.arange(256, dtype=np.uint32).astype(np.uint8).view(np.int8).astype(np.float32))
+
+
+def test_zero_blocks_signed_zero():
+    # q4_K and q8_0: 0*q - 0 = +0.0.  q6_K: code 0 means q = -32, (0*sc)*(-32) = -0.0.
+    y4 = oracle.dequantize(Q4_K, np.zeros((1, 144), np.uint8), 256)
+    y8 = oracle.dequantize(Q8_0, np.zeros((1, 34), np.uint8), 32)
+    y6 = oracle.dequantize(Q6_K, np.zeros((1, 210), np.uint8), 256)
+    assert np.all(bits(y4) == 0) and np.all(bits(y8) == 0)
+    assert np.all(bits(y6) == 0x80000000)
+
+
+# ----------------------------------------------------------------------------
+# library cross-check: gguf.quants.dequantize on seeded random blocks
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("qtype", [Q4_K, Q6_K, Q8_0])
+def test_matches_gguf_quants(qtype):
+    import gguf
+    k = 2048
+    w = synth.weights(qtype, 24, k, seed=11)
+    ref = gguf.quants.dequantize(w, gguf.GGMLQuantizationType(qtype)).astype(np.float32)
+    y = oracle.dequantize(qtype, w, k)
+    assert np.array_equal(bits(y), bits(ref))
+    # fully random bytes too (any fp16 d, any int8 scale), excluding NaN/inf scales
+    raw = np.random.default_rng(3).integers(0, 256, size=(64, synth.row_bytes(qtype, 256)), dtype=np.uint8)
+    ref = gguf.quants.dequantize(raw, gguf.GGMLQuantizationType(qtype)).astype(np.float32)
+    y = oracle.dequantize(qtype, raw, 256)
+    fin = np.isfinite(ref)
+    assert np.array_equal(np.isfinite(y), fin)
+    assert np.array_equal(bits(y)[fin], bits(ref)[fin])
+
+
+# ----------------------------------------------------------------------------
+# matmul: exact rational brute force and a library dot product
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("qtype,k", [(Q4_K, 256), (Q6_K, 512), (Q8_0, 256)])
+def test_matmul_brute_force(qtype, k):
+    import gguf
+    n, m = 5, 3
+    w = synth.weights(qtype, n, k, seed=21)
+    x = synth.activations(m, k, seed=22)
+    wd = gguf.quants.dequantize(w, gguf.GGMLQuantizationType(qtype)).astype(np.float32)
+    xf = oracle.bf16_to_f32(x)
+    y, a = oracle.matmul(qtype, w, k, x, absdot=True)
+    for i in range(m):
+        for j in range(n):
+            exact = sum(Fraction(float(xf[i, t])) * Fraction(float(wd[j, t])) for t in range(k))
+            aex = sum(abs(Fraction(float(xf[i, t])) * Fraction(float(wd[j, t]))) for t in range(k))
+            # fp64 sequential summation error bound: k * eps * sum|terms|
+            bound = k * 2.0 ** -53 * float(aex)
+            assert abs(y[i, j] - float(exact)) <= bound
+            assert abs(a[i, j] - float(aex)) <= bound
+
+
+@pytest.mark.parametrize("qtype", [Q4_K, Q6_K, Q8_0])
+def test_matmul_numpy_and_invariants(qtype):
+    import gguf
+    n, k, m = 37, 1024, 4
+    w = synth.weights(qtype, n, k, seed=31)
+    x = synth.activations(m, k, seed=32)
+    wd = gguf.quants.dequantize(w, gguf.GGMLQuantizationType(qtype)).astype(np.float64)
+    xf = oracle.bf16_to_f32(x).astype(np.float64)
+    y = oracle.matmul(qtype, w, k, x)
+    ref = xf @ wd.T
+    assert np.all(np.abs(y - ref) <= 2 * k * 2.0 ** -53 * (np.abs(xf) @ np.abs(wd).T))
+    # not transposed by mistake: a single nonzero activation picks one column of W
+    e = np.zeros((1, k), np.float32)
+    e[0, 7] = 1.0
+    ye = oracle.matmul(qtype, w, k, synth.f32_to_bf16_bits(e))
+    assert np.array_equal(ye[0], wd[:, 7])
+    # scaling x by 2 (exact in bf16) scales y by exactly 2
+    x2 = synth.f32_to_bf16_bits(2.0 * oracle.bf16_to_f32(x))
+    assert np.array_equal(oracle.matmul(qtype, w, k, x2), 2.0 * y)
+    # row independence: a row's result does not depend on the other rows
+    y1 = oracle.matmul(qtype, w, k, x[2:3])
+    assert np.array_equal(y1[0], y[2])
+    # the fp32 baseline stays within fp32 summation error of the fp64 value
+    y32 = oracle.matmul_f32(qtype, w, k, x)
+    _, a = oracle.matmul(qtype, w, k, x, absdot=True)
+    assert np.all(np.abs(y32 - y) <= (k + 1) * 2.0 ** -24 * a)
+
+
+# ----------------------------------------------------------------------------
+# MoE: sort, tile map (golden, hand-worked) and gather semantics
+# ----------------------------------------------------------------------------
+def _golden_tile_cases():
+    cases, cur = [], None
+    for line in open(os.path.join(GOLDEN, "tile_map_cases.txt")):
+        p = line.split()
+        if not p or p[0] == "#":
+            continue
+        if p[0] == "case":
+            cur = (int(p[1]), [int(s) for s in p[2].split(",")], [])
+            cases.append(cur)
+        else:
+            cur[2].append(tuple(int(v) for v in p[1:]))
+    return cases
+
+
+@pytest.mark.parametrize("case", _golden_tile_cases())
+def test_tile_map_golden(case):
+    n_experts, seg, expect = case
+    ids = np.repeat(np.arange(n_experts), seg).astype(np.uint32)
+    tiles = oracle.tile_map(ids, n_experts)
+    assert sorted(tiles) == sorted(expect)
+    assert len(tiles) <= oracle.map_capacity(len(ids), n_experts)
+
+
+def test_moe_sort_is_stable():
+    ids = np.array([[2, 0], [0, 1], [2, 1]], dtype=np.int32)   # 3 tokens, top-2
+    sids, pair = oracle.moe_sort(ids, 3)
+    assert sids.tolist() == [0, 0, 1, 1, 2, 2]
+    assert pair.tolist() == [1, 2, 3, 5, 0, 4]                  # equal experts keep pair order
+    x = np.arange(3 * 4, dtype=np.uint16).reshape(3, 4)
+    xs = oracle.gather_rows(x, pair, 2)
+    assert np.array_equal(xs, x[[0, 1, 1, 2, 0, 2]])
+
+
+def test_routing_distinct_experts():
+    r = synth.routing(512, 8, 2)
+    assert r.shape == (512, 2) and np.all(r[:, 0] != r[:, 1])
+    assert r.min() >= 0 and r.max() < 8
+
+
+def test_gather_single_expert_equals_matmul():
+    k, n, rows = 256, 16, 70
+    w = synth.weights(Q4_K, n, k, seed=41, experts=1)
+    x = synth.activations(rows, k, seed=42)
+    ids = np.zeros(rows, np.uint32)
+    tiles = oracle.tile_map(ids, 1)
+    assert tiles == [(0, 0, 64), (0, 64, 6)]
+    y = oracle.gather_qmm(Q4_K, w, k, x, tiles)
+    assert np.array_equal(y, oracle.matmul(Q4_K, w[0], k, x))
+
+
+def test_gather_uncovered_rows_unwritten():
+    k, n = 256, 8
+    w = synth.weights(Q8_0, n, k, seed=43, experts=2)
+    x = synth.activations(10, k, seed=44)
+    y = oracle.gather_qmm(Q8_0, w, k, x, [(1, 2, 3)])
+    assert np.all(np.isnan(y[:2])) and np.all(np.isnan(y[5:]))
+    assert np.array_equal(y[2:5], oracle.matmul(Q8_0, w[1], k, x[2:5]))
