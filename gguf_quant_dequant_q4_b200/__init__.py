@@ -1,0 +1,203 @@
+"""B200 (sm_100a) matrix products with GGUF block-quantized weights.
+
+A thin Python binding over the C ABI in ``include/kq.h`` (shared library
+``_lib/libkq.so``, built by ``python -m gguf_quant_dequant_q4_b200.build``).
+This module only marshals arguments: torch provides device memory and the
+current CUDA stream, every step of the computation runs in the library's
+kernels.  There is no CPU fallback; calling an op without the built library or
+without a CUDA device raises.
+
+Codecs (ggml type ids): ``Q8_0 = 8``, ``Q4_K = 12``, ``Q6_K = 14``.  Weights are
+wire bytes ``uint8 [N, row_bytes]`` ("transpose=True" layout: y = x @ W.T),
+activations ``bfloat16 [M, K]``, outputs ``float32``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+Q8_0, Q4_K, Q6_K = 8, 12, 14
+NAMES = {Q8_0: "q8_0", Q4_K: "q4_K", Q6_K: "q6_K"}
+_BLOCK = {Q8_0: (32, 34), Q4_K: (256, 144), Q6_K: (256, 210)}
+TILE_ROWS = 64
+
+DEV_BAD_EXPERT, DEV_BAD_ROWS, DEV_BAD_RANGE, DEV_UNSORTED = 0x1, 0x2, 0x4, 0x8
+DEV_TIMEOUT, DEV_TOO_MANY, DEV_X_RANGE = 0x10, 0x20, 0x40
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libkq.so")
+
+# Every entry point declared in include/kq.h: name -> (restype, argtypes)
+_vp, _i64, _i32, _int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
+SIGNATURES = {
+    "kq_block_info": (_int, [_int, ctypes.POINTER(_int), ctypes.POINTER(_int)]),
+    "kq_status_string": (ctypes.c_char_p, [_int]),
+    "kq_last_cuda_error": (_int, []),
+    "kq_read_device_status": (_int, [ctypes.POINTER(_i32), _int]),
+    "kq_dequantize": (_int, [_int, _vp, _i64, _i64, _vp, _vp]),
+    "kq_qmv": (_int, [_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp]),
+    "kq_qmm": (_int, [_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp]),
+    "kq_moe_sort": (_int, [_vp, _i64, _i32, _i32, _vp, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "kq_expert_tile_map": (_int, [_vp, _i64, _i32, _vp, _i64, _vp, _vp, _vp]),
+    "kq_gather_qmm": (_int, [_int, _vp, _i32, _i64, _i64, _vp, _i64, _vp, _vp, _i64, _vp, _vp, _vp]),
+}
+
+_lib = None
+
+
+class KQError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = lib().kq_status_string(status).decode()
+        if status == 4:
+            msg += f" (cudaError {lib().kq_last_cuda_error()})"
+        super().__init__(f"{what}: {msg} [status {status}]")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m gguf_quant_dequant_q4_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(l, name)
+            f.restype, f.argtypes = res, args
+        _lib = l
+    return _lib
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise KQError(rc, what)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+        if t is not None and not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+
+
+def block_info(qtype: int) -> tuple[int, int]:
+    v, b = _int(), _int()
+    _check(lib().kq_block_info(qtype, ctypes.byref(v), ctypes.byref(b)), "kq_block_info")
+    return v.value, b.value
+
+
+def row_bytes(qtype: int, k: int) -> int:
+    vpb, bpb = _BLOCK[qtype]
+    return k // vpb * bpb
+
+
+def read_device_status(clear: bool = False) -> int:
+    v = _i32()
+    _check(lib().kq_read_device_status(ctypes.byref(v), int(clear)), "kq_read_device_status")
+    return v.value
+
+
+def _bf16_bits(x: torch.Tensor) -> torch.Tensor:
+    if x.dtype == torch.bfloat16:
+        return x
+    if x.dtype in (torch.uint16, torch.int16):
+        return x
+    raise TypeError("activations must be bfloat16")
+
+
+def dequantize(w: torch.Tensor, qtype: int, k: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """fp32 [..., N, K] decode of wire bytes [..., N, row_bytes] (bit-exact)."""
+    rows = w.numel() // max(1, w.shape[-1]) if w.dim() else 0
+    if out is None:
+        out = torch.empty(*w.shape[:-1], k, dtype=torch.float32, device=w.device)
+    _need_cuda(w, out)
+    _check(lib().kq_dequantize(qtype, _ptr(w), rows, k, _ptr(out), _stream(stream)), "kq_dequantize")
+    return out
+
+
+def qmv(x: torch.Tensor, w: torch.Tensor, qtype: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y[M, N] = x[M, K] @ dequant(w[N, :]).T for 1 <= M <= 16."""
+    x = _bf16_bits(x)
+    m, k = x.shape
+    n = w.shape[0]
+    if out is None:
+        out = torch.empty(m, n, dtype=torch.float32, device=x.device)
+    _need_cuda(x, w, out)
+    _check(lib().kq_qmv(qtype, _ptr(w), n, k, _ptr(x), m, _ptr(out), _stream(stream)), "kq_qmv")
+    return out
+
+
+def qmm(x: torch.Tensor, w: torch.Tensor, qtype: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y[M, N] = x[M, K] @ dequant(w[N, :]).T on the tcgen05 tensor cores."""
+    x = _bf16_bits(x)
+    m, k = x.shape
+    n = w.shape[0]
+    if out is None:
+        out = torch.empty(m, n, dtype=torch.float32, device=x.device)
+    _need_cuda(x, w, out)
+    _check(lib().kq_qmm(qtype, _ptr(w), n, k, _ptr(x), m, _ptr(out), _stream(stream)), "kq_qmm")
+    return out
+
+
+def map_capacity(rows: int, n_experts: int) -> int:
+    return -(-rows // TILE_ROWS) + n_experts
+
+
+def moe_sort(topk_ids: torch.Tensor, n_experts: int, x: torch.Tensor | None = None, err: torch.Tensor | None = None,
+             stream=None):
+    """Stable sort of routed pairs by expert: (sorted_ids, sorted_pair, x_sorted)."""
+    t, top_k = topk_ids.shape
+    rows = t * top_k
+    dev = topk_ids.device
+    sids = torch.empty(rows, dtype=torch.int32, device=dev)
+    pair = torch.empty(rows, dtype=torch.int32, device=dev)
+    xs = None
+    k = 0
+    if x is not None:
+        x = _bf16_bits(x)
+        k = x.shape[1]
+        xs = torch.empty(rows, k, dtype=x.dtype, device=dev)
+    _need_cuda(topk_ids, x, xs, err)
+    _check(lib().kq_moe_sort(_ptr(topk_ids), t, top_k, n_experts, _ptr(x), k, _ptr(sids), _ptr(pair), _ptr(xs),
+                             _ptr(err), _stream(stream)), "kq_moe_sort")
+    return sids, pair, xs
+
+
+def expert_tile_map(sorted_ids: torch.Tensor, n_experts: int, cap: int | None = None,
+                    err: torch.Tensor | None = None, stream=None):
+    """(map int32 [cap, 3] of (expert, row_start, num_rows), count int32 [1])."""
+    rows = sorted_ids.numel()
+    cap = map_capacity(rows, n_experts) if cap is None else cap
+    m = torch.empty(cap, 3, dtype=torch.int32, device=sorted_ids.device)
+    c = torch.empty(1, dtype=torch.int32, device=sorted_ids.device)
+    _need_cuda(sorted_ids, err)
+    _check(lib().kq_expert_tile_map(_ptr(sorted_ids), rows, n_experts, _ptr(m), cap, _ptr(c), _ptr(err),
+                                    _stream(stream)), "kq_expert_tile_map")
+    return m, c
+
+
+def gather_qmm(x_sorted: torch.Tensor, w_bank: torch.Tensor, qtype: int, tile_map: torch.Tensor,
+               count: torch.Tensor, out: torch.Tensor | None = None, err: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """y[r] = x_sorted[r] @ dequant(w_bank[e(r)]).T for every row covered by a tile."""
+    x_sorted = _bf16_bits(x_sorted)
+    rows, k = x_sorted.shape
+    e, n = w_bank.shape[0], w_bank.shape[1]
+    if out is None:
+        out = torch.empty(rows, n, dtype=torch.float32, device=x_sorted.device)
+    _need_cuda(x_sorted, w_bank, tile_map, count, out, err)
+    _check(lib().kq_gather_qmm(qtype, _ptr(w_bank), e, n, k, _ptr(x_sorted), rows, _ptr(tile_map), _ptr(count),
+                               tile_map.shape[0], _ptr(out), _ptr(err), _stream(stream)), "kq_gather_qmm")
+    return out

@@ -1,0 +1,35 @@
+// Host-side declarations shared by the kq translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kq.h"
+
+namespace kq {
+
+// Number of SMs of the current device (cached per device).
+int device_sm_count();
+// Maximum opt-in dynamic shared memory per block of the current device.
+int device_smem_optin();
+// Records the launch error (if any) and maps it to a kq_status.
+int check_launch();
+int record_cuda(cudaError_t e);
+// Device address of the library-wide status word (bits KQ_DEV_*).
+int* device_status_ptr();
+
+int launch_dequantize(int type, const void* w, int64_t n_rows, int64_t k, float* out, cudaStream_t s);
+int launch_qmv(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int m, float* y,
+               cudaStream_t s);
+int launch_qmm(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int64_t m, float* y,
+               cudaStream_t s);
+int launch_gather_qmm(int type, const void* w_bank, int n_experts, int64_t n, int64_t k,
+                      const uint16_t* x_sorted, int64_t rows, const uint32_t* map, const uint32_t* count,
+                      int64_t cap, float* y, int32_t* err_flag, cudaStream_t s);
+int launch_moe_sort(const int32_t* topk_ids, int64_t n_tokens, int top_k, int n_experts, const uint16_t* x,
+                    int64_t k, uint32_t* sorted_ids, int32_t* sorted_pair, uint16_t* x_sorted,
+                    int32_t* err_flag, cudaStream_t s);
+int launch_tile_map(const uint32_t* sorted_ids, int64_t rows, int n_experts, uint32_t* map, int64_t cap,
+                    uint32_t* count, int32_t* err_flag, cudaStream_t s);
+
+}  // namespace kq

@@ -1,0 +1,746 @@
+// kq_qmm / kq_gather_qmm: prefill-shaped y = x . W^T on the tcgen05 tensor
+// cores, with W decoded from its GGUF wire blocks inside the kernel.
+//
+// mlx-kquant bindings.cpp `quantized_matmul` and `gather_qmm_seg` (segment-
+// walking gather GEMM over expert-sorted rows, map of (expert, row_start,
+// num_rows <= 64) tiles, uncovered rows left unwritten); README
+// "Performance": a single-pass matmul on the tensor units, per-expert-segment
+// GEMM for sorted MoE prefill.  hanzo-ml quantized/mod.rs notes that a GEMM
+// that re-reads the weight once per small row group wastes bandwidth; here
+// every weight tile is read and decoded once per 256 output rows.
+//
+// Tile: 128 weight rows (MMA M) x up to 256 activation rows (MMA N), K in
+// steps of 64.  One persistent CTA per SM, warp-specialized:
+//   warp 0      TMA producer: raw weight tiles (2-D box of wire bytes, 128
+//               rows x one 256-value block) and activation tiles (bf16,
+//               128B-swizzled, one 64-row box per map tile)
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator, masked stores
+//   warps 6..13 decoders: wire bytes -> bf16 A tile in the 128B-swizzled
+//               K-major layout the tensor core reads (thread = one row and
+//               one 32-value half of the 64-value step)
+// Accumulators are double-buffered in TMEM (2 x 256 columns) so the epilogue
+// of one tile overlaps the main loop of the next.  All waits are bounded; a
+// wait that runs out sets KQ_DEV_TIMEOUT and the CTA winds down, freeing its
+// TMEM.  No TMA multicast is used anywhere.
+#include <cuda.h>
+
+#include "kq_device.cuh"
+#include "kq_launch.h"
+
+namespace kq {
+namespace {
+
+constexpr int kThreads = 14 * 32;
+constexpr int kBM = 128;          // weight rows per tile (MMA M)
+constexpr int kBN = 256;          // activation rows per tile (MMA N max)
+constexpr int kBK = 64;           // K per pipeline step (one 128-byte swizzle row)
+constexpr int kRawStages = 2;     // raw weight stages, 256 values each
+constexpr int kBStages = 3;
+constexpr int kMaxTiles = 1024;   // map tiles a gather call may use
+constexpr uint32_t kHeader = 5120; // barriers, misc words, tile tables
+constexpr int kEpiWarp0 = 2, kDeqWarp0 = 6;
+
+template <int QT> struct QmmCodec;
+template <> struct QmmCodec<KQ_Q4_K> {
+    static constexpr int RAWB = 144, AST = 4;         // raw row bytes per stage, A stages
+};
+template <> struct QmmCodec<KQ_Q6_K> {
+    static constexpr int RAWB = 240, AST = 4;         // 210-byte block at offset 210b mod 16
+};
+template <> struct QmmCodec<KQ_Q8_0> {
+    static constexpr int RAWB = 272, AST = 3;         // eight 34-byte blocks
+};
+
+struct Smem {
+    static constexpr uint32_t kBars = 0;      // mbarriers
+    static constexpr uint32_t kMisc = 256;    // tmem base, abort flag, counts
+    static constexpr uint32_t kTiles = 512;   // sorted tile ids (u16) + per-expert tables
+};
+
+struct QmmParams {
+    int64_t n;            // weight rows per expert
+    int64_t m;            // activation rows (dense) / rows of x_sorted (gather)
+    int k;
+    int n_experts;        // 0 = dense qmm
+    int ntn;              // weight tiles per expert = ceil(n / 128)
+    int units;            // dense: ceil(m/256) * ntn
+    const uint32_t* map;
+    const uint32_t* count;
+    int64_t cap;
+    float* y;
+    int32_t* err;         // caller's flag (gather) or library status
+    int* status;
+};
+
+// ---------------------------------------------------------------- PTX glue
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t dtmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(dtmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+          "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+__device__ __forceinline__ uint32_t ldsu16(uint32_t a) {
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+
+// K-major operand in the 128-byte swizzle layout: rows of 128 bytes, groups of
+// 8 rows 1024 bytes apart (stride byte offset), start advanced by 32 bytes per
+// 16-element K slice.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFF) | (static_cast<uint64_t>(1) << 16) |
+           (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+           (static_cast<uint64_t>(2) << 61);
+}
+// kind::f16 instruction descriptor: D f32, A and B bf16, both K-major, M = 128.
+__device__ __forceinline__ uint32_t make_idesc(int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+// ------------------------------------------------------- bf16x2 arithmetic
+__device__ __forceinline__ uint32_t bsub2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t bfma2(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t bf16_bits(float f) { return __bfloat16_as_ushort(__float2bfloat16_rn(f)); }
+__device__ __forceinline__ float bf16_val(uint32_t b) { return __uint_as_float(b << 16); }
+__device__ __forceinline__ uint32_t dup(uint32_t b) { return b | (b << 16); }
+// A scale s split into two bf16 parts, s ~= hi + lo to 16 significant bits.
+__device__ __forceinline__ void split_scale(float s, uint32_t& hi2, uint32_t& lo2) {
+    const uint32_t h = bf16_bits(s);
+    hi2 = dup(h);
+    lo2 = dup(bf16_bits(s - bf16_val(h)));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+__device__ __forceinline__ float h16v(uint32_t h) { return __half2float(__ushort_as_half((unsigned short)h)); }
+
+// 32 bytes starting O bytes into the 16-byte aligned shared address `a`,
+// as 8 little-endian words (O even, compile time).
+template <int O>
+__device__ __forceinline__ void lds32B(uint32_t a, uint32_t (&w)[8]) {
+    uint32_t r[12];
+    const uint4 c0 = lds128(a), c1 = lds128(a + 16);
+    r[0] = c0.x; r[1] = c0.y; r[2] = c0.z; r[3] = c0.w;
+    r[4] = c1.x; r[5] = c1.y; r[6] = c1.z; r[7] = c1.w;
+    if constexpr (O != 0) {
+        const uint4 c2 = lds128(a + 32);
+        r[8] = c2.x; r[9] = c2.y; r[10] = c2.z; r[11] = c2.w;
+    } else {
+        r[8] = r[9] = r[10] = r[11] = 0;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        if constexpr ((O & 3) == 0) w[i] = r[(O >> 2) + i];
+        else w[i] = __byte_perm(r[(O >> 2) + i], r[(O >> 2) + i + 1], 0x5432);
+    }
+}
+
+// Store 16 bf16x2 words (32 consecutive K values, logical chunks 4p..4p+3 of
+// row r) into a 128B-swizzled A stage.
+__device__ __forceinline__ void store_a(uint32_t abase, int r, int p, const uint32_t (&o)[16]) {
+    const uint32_t rowb = abase + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+        const int c = 4 * p + cc;
+        sts128(rowb + ((c ^ (r & 7)) << 4), o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);
+    }
+}
+
+// ---------------------------------------------------------------- decoders
+// Each decoder turns 32 consecutive values (A step q in 0..3 of the raw
+// 256-value stage, half p) of one weight row into bf16:
+//   w = bf16( fp32(d*sc)*q - fp32(dmin*m) )  evaluated as
+//   t = q*s_lo - mm ; w = q*s_hi + t   in bf16x2 FMA (s = s_hi + s_lo exact to
+//   16 bits), so the result carries essentially one bf16 rounding.
+constexpr uint32_t kB128 = 0x43004300u;   // bf16 (128, 128)
+constexpr uint32_t kB160 = 0x43204320u;   // bf16 (160, 160)
+constexpr uint32_t kMagic = 0x43434343u;
+
+// q4_K: 144-byte block; values 64q + 32p .. are nibble p of qs[32q .. 32q+31]
+// with scale/min code j = 2q + p.
+__device__ __forceinline__ void dq_q4k(uint32_t row, int q, int p, uint32_t (&o)[16]) {
+    const uint4 h = lds128(row);
+    const int j = 2 * q + p;
+    const uint32_t s0 = h.y, s1 = h.z, s2 = h.w;   // bytes 0..3, 4..7, 8..11
+    int sc, m;
+    if (j < 4) {
+        sc = (s0 >> (8 * j)) & 63;
+        m = (s1 >> (8 * j)) & 63;
+    } else {
+        const int jj = j - 4;
+        const uint32_t b8 = (s2 >> (8 * jj)) & 0xff;
+        sc = (b8 & 15) | (((s0 >> (8 * jj + 6)) & 3) << 4);
+        m = (b8 >> 4) | (((s1 >> (8 * jj + 6)) & 3) << 4);
+    }
+    const float s = __fmul_rn(h16v(h.x & 0xffff), static_cast<float>(sc));
+    const float mm = __fmul_rn(h16v(h.x >> 16), static_cast<float>(m));
+    uint32_t shi, slo;
+    split_scale(s, shi, slo);
+    const uint32_t nmm = dup(bf16_bits(-mm));
+    const uint4 q0 = lds128(row + 16 + 32 * q), q1 = lds128(row + 32 + 32 * q);
+    const uint32_t wv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t nib = p ? ((wv[i] >> 4) & 0x0F0F0F0Fu) : (wv[i] & 0x0F0F0F0Fu);
+        const uint32_t v01 = bsub2(__byte_perm(nib, kMagic, 0x5140), kB128);   // (q0, q1) exact
+        const uint32_t v23 = bsub2(__byte_perm(nib, kMagic, 0x7362), kB128);
+        o[2 * i] = bfma2(v01, shi, bfma2(v01, slo, nmm));
+        o[2 * i + 1] = bfma2(v23, shi, bfma2(v23, slo, nmm));
+    }
+}
+
+// q6_K: 210-byte block starting O bytes into the staged row.  Values
+// 64q + 32p + l (l = 0..31) are h = q/2, quarter tq = 2(q&1) + p: low 4 bits
+// nibble tq>>1 of ql[64h + 32(tq&1) + l], high 2 bits bits 2tq of qh[32h + l],
+// scale sc[8h + 2tq + l/16].  y = fp32(d*sc) * (code - 32).
+template <int O>
+__device__ __forceinline__ void dq_q6k(uint32_t row, int q, int p, uint32_t (&o)[16]) {
+    const int h = q >> 1, tq = 2 * (q & 1) + p;
+    uint32_t QL[8], QH[8];
+    lds32B<O>(row + 64 * h + 32 * (tq & 1), QL);
+    lds32B<O>(row + 128 + 32 * h, QH);
+    const uint32_t scw = ldsu16(row + O + 192 + 8 * h + 2 * tq);
+    const float d = h16v(ldsu16(row + O + 208));
+    uint32_t shi[2], slo[2];
+    split_scale(__fmul_rn(d, static_cast<float>(static_cast<int8_t>(scw & 0xff))), shi[0], slo[0]);
+    split_scale(__fmul_rn(d, static_cast<float>(static_cast<int8_t>(scw >> 8))), shi[1], slo[1]);
+    const int lsh = 4 * (tq >> 1), hsh = 2 * tq;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t c4 = ((QL[i] >> lsh) & 0x0F0F0F0Fu) | (((QH[i] >> hsh) & 0x03030303u) << 4);
+        const uint32_t v01 = bsub2(__byte_perm(c4, kMagic, 0x5140), kB160);   // code - 32, exact
+        const uint32_t v23 = bsub2(__byte_perm(c4, kMagic, 0x7362), kB160);
+        const int sb = i >> 2;
+        o[2 * i] = bfma2(v01, shi[sb], bmul2(v01, slo[sb]));
+        o[2 * i + 1] = bfma2(v23, shi[sb], bmul2(v23, slo[sb]));
+    }
+}
+
+// q8_0: block BI (0..7) of the 272-byte stage row; qs starts 34*BI + 2.
+// y = fp32(d*q) rounded to bf16.
+template <int BI>
+__device__ __forceinline__ void dq_q8(uint32_t row, uint32_t (&o)[16]) {
+    constexpr int L = 34 * BI + 2;
+    uint32_t QW[8];
+    lds32B<(L & 15)>(row + (L & ~15), QW);
+    const float d = h16v(ldsu16(row + 34 * BI));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t u = QW[i] ^ 0x80808080u;   // q + 128
+        float f[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const uint32_t bits = __byte_perm(u, 0x4B000000u, 0x7650 + b);   // 2^23 + q + 128
+            f[b] = __fmul_rn(d, __uint_as_float(bits) - 8388736.0f);
+        }
+        o[2 * i] = pack_bf16x2(f[0], f[1]);
+        o[2 * i + 1] = pack_bf16x2(f[2], f[3]);
+    }
+}
+
+template <int QT>
+__device__ __forceinline__ void decode_step(uint32_t row, int q, int p, int o6, uint32_t (&o)[16]) {
+    if constexpr (QT == KQ_Q4_K) {
+        dq_q4k(row, q, p, o);
+    } else if constexpr (QT == KQ_Q6_K) {
+        switch (o6) {
+        case 0: dq_q6k<0>(row, q, p, o); break;
+        case 2: dq_q6k<2>(row, q, p, o); break;
+        case 4: dq_q6k<4>(row, q, p, o); break;
+        case 6: dq_q6k<6>(row, q, p, o); break;
+        case 8: dq_q6k<8>(row, q, p, o); break;
+        case 10: dq_q6k<10>(row, q, p, o); break;
+        case 12: dq_q6k<12>(row, q, p, o); break;
+        default: dq_q6k<14>(row, q, p, o); break;
+        }
+    } else {
+        switch (2 * q + p) {
+        case 0: dq_q8<0>(row, o); break;
+        case 1: dq_q8<1>(row, o); break;
+        case 2: dq_q8<2>(row, o); break;
+        case 3: dq_q8<3>(row, o); break;
+        case 4: dq_q8<4>(row, o); break;
+        case 5: dq_q8<5>(row, o); break;
+        case 6: dq_q8<6>(row, o); break;
+        default: dq_q8<7>(row, o); break;
+        }
+    }
+}
+
+// ------------------------------------------------------------- work units
+// A unit is (expert, up to 4 map tiles of that expert, one 128-row weight
+// tile).  Dense qmm: one pseudo-expert whose tiles are rows 64i..64i+63.
+struct Unit {
+    int e, ntile, nt;         // expert, weight tile, number of 64-row tiles
+    int rs[4], nr[4];         // row_start / num_rows of each tile
+};
+
+struct Pipe {
+    int idx = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void next(int n) {
+        if (++idx == n) {
+            idx = 0;
+            phase ^= 1;
+        }
+    }
+};
+
+template <int QT>
+__global__ void __launch_bounds__(kThreads, 1)
+    qmm_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
+               const QmmParams p) {
+    using C = QmmCodec<QT>;
+    constexpr int AST = C::AST;
+    constexpr uint32_t kRawBytes = kBM * C::RAWB;
+    constexpr uint32_t kABytes = kBM * kBK * 2;    // 16 KB
+    constexpr uint32_t kBBytes = kBN * kBK * 2;    // 32 KB
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t sb = smem_u32(smem);
+    // stage regions (1024-aligned): B stages, A stages, raw stages
+    const uint32_t base = (sb + kHeader + 1023) & ~1023u;
+    const uint32_t bst = base, ast = bst + kBStages * kBBytes, rst = ast + AST * kABytes;
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Smem::kBars);
+    uint64_t* raw_full = bars;
+    uint64_t* raw_empty = bars + 2;
+    uint64_t* a_full = bars + 4;
+    uint64_t* a_empty = bars + 8;
+    uint64_t* b_full = bars + 12;
+    uint64_t* b_empty = bars + 15;
+    uint64_t* acc_full = bars + 18;
+    uint64_t* acc_empty = bars + 20;
+    volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + Smem::kMisc);
+    // misc[0] tmem base, misc[1] abort, misc[2] number of chunks, misc[3] tiles
+    uint16_t* tiles = reinterpret_cast<uint16_t*>(smem + Smem::kTiles);          // sorted valid tile ids
+    int* cstart = reinterpret_cast<int*>(smem + Smem::kTiles + 2 * kMaxTiles);    // per expert chunk prefix [257]
+    int* tstart = cstart + 257;                                                  // per expert tile prefix [257]
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // ---- set-up: barriers, TMEM, work list
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&raw_full[i], 1);
+            mbar_init(&raw_empty[i], 8);
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 4);
+        }
+        for (int i = 0; i < AST; ++i) {
+            mbar_init(&a_full[i], 8);
+            mbar_init(&a_empty[i], 1);
+        }
+        for (int i = 0; i < kBStages; ++i) {
+            mbar_init(&b_full[i], 1);
+            mbar_init(&b_empty[i], 1);
+        }
+        misc[1] = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(sb + Smem::kMisc));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    int total_units;
+    if (p.n_experts == 0) {
+        total_units = p.units;
+    } else {
+        // Gather: validate the map, keep valid tiles, order them by
+        // (expert, row_start) and cut each expert's list into chunks of 4.
+        int cnt = static_cast<int>(*p.count);
+        if (cnt > p.cap || cnt < 0) {
+            if (tid == 0 && p.err) atomicOr(p.err, KQ_DEV_BAD_RANGE);
+            cnt = cnt < 0 ? 0 : static_cast<int>(p.cap);
+        }
+        if (cnt > kMaxTiles) {
+            if (tid == 0 && p.err) atomicOr(p.err, KQ_DEV_TOO_MANY);
+            cnt = kMaxTiles;
+        }
+        for (int e = tid; e < 257; e += kThreads) cstart[e] = tstart[e] = 0;
+        __syncthreads();
+        // validity and per-expert counts
+        for (int i = tid; i < cnt; i += kThreads) {
+            const uint32_t e = p.map[3 * i], rs = p.map[3 * i + 1], nr = p.map[3 * i + 2];
+            int bad = 0;
+            if (e >= static_cast<uint32_t>(p.n_experts)) bad |= KQ_DEV_BAD_EXPERT;
+            if (nr == 0 || nr > 64) bad |= KQ_DEV_BAD_ROWS;
+            if (static_cast<int64_t>(rs) + nr > p.m) bad |= KQ_DEV_BAD_RANGE;
+            if (bad) {
+                if (p.err) atomicOr(p.err, bad);
+            } else {
+                atomicAdd(&tstart[e + 1], 1);
+            }
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int tacc = 0, cacc = 0;
+            for (int e = 0; e < p.n_experts; ++e) {
+                const int te = tstart[e + 1];
+                tstart[e] = tacc;
+                cstart[e] = cacc;
+                tacc += te;
+                cacc += (te + 3) / 4;
+            }
+            tstart[p.n_experts] = tacc;
+            cstart[p.n_experts] = cacc;
+            misc[2] = cacc;
+        }
+        __syncthreads();
+        // place: rank of a valid tile among the valid tiles of its expert by row_start
+        for (int i = tid; i < cnt; i += kThreads) {
+            const uint32_t e = p.map[3 * i], rs = p.map[3 * i + 1], nr = p.map[3 * i + 2];
+            if (e >= static_cast<uint32_t>(p.n_experts) || nr == 0 || nr > 64 || static_cast<int64_t>(rs) + nr > p.m)
+                continue;
+            int rank = 0;
+            for (int j = 0; j < cnt; ++j) {
+                const uint32_t e2 = p.map[3 * j], rs2 = p.map[3 * j + 1], nr2 = p.map[3 * j + 2];
+                const bool ok2 = e2 == e && nr2 != 0 && nr2 <= 64 && static_cast<int64_t>(rs2) + nr2 <= p.m;
+                if (ok2 && (rs2 < rs || (rs2 == rs && j < i))) ++rank;
+            }
+            tiles[tstart[e] + rank] = static_cast<uint16_t>(i);
+        }
+        total_units = 0;   // read after the barrier below
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+    if (p.n_experts != 0) total_units = static_cast<int>(misc[2]) * p.ntn;
+
+    auto get_unit = [&](int u, Unit& U) {
+        if (p.n_experts == 0) {
+            const int mtiles = static_cast<int>((p.m + kBN - 1) / kBN);
+            const int mt = u % mtiles;
+            U.e = 0;
+            U.ntile = u / mtiles;
+            const int64_t r0 = static_cast<int64_t>(mt) * kBN;
+            const int64_t left = p.m - r0;
+            U.nt = static_cast<int>(left >= kBN ? 4 : (left + 63) / 64);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                U.rs[i] = static_cast<int>(r0 + 64 * i);
+                const int64_t ri = left - 64 * i;
+                U.nr[i] = ri <= 0 ? 0 : (ri >= 64 ? 64 : static_cast<int>(ri));
+            }
+        } else {
+            const int nch = static_cast<int>(misc[2]);
+            const int c = u % nch;
+            U.ntile = u / nch;
+            int lo = 0, hi = p.n_experts - 1;   // expert with cstart[e] <= c < cstart[e+1]
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (cstart[mid] <= c) lo = mid;
+                else hi = mid - 1;
+            }
+            U.e = lo;
+            const int first = tstart[lo] + 4 * (c - cstart[lo]);
+            const int left = tstart[lo + 1] - first;
+            U.nt = left >= 4 ? 4 : left;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (i < U.nt) {
+                    const int ti = tiles[first + i];
+                    U.rs[i] = static_cast<int>(p.map[3 * ti + 1]);
+                    U.nr[i] = static_cast<int>(p.map[3 * ti + 2]);
+                } else {
+                    U.rs[i] = 0;
+                    U.nr[i] = 0;
+                }
+            }
+        }
+    };
+    auto mma_n = [&](const Unit& U) { return 64 * (U.nt - 1) + ((U.nr[U.nt - 1] + 15) & ~15); };
+    auto aborted = [&]() { return misc[1] != 0; };
+    auto bwait = [&](uint64_t* bar, uint32_t parity) {
+        if (misc[1]) return false;
+        if (!mbar_wait(bar, parity, p.status)) {
+            misc[1] = 1;
+            return false;
+        }
+        return true;
+    };
+
+    const int ksteps = p.k / kBK;
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            Pipe rp, bp;
+            for (int u = blockIdx.x; u < total_units && !aborted(); u += gridDim.x) {
+                Unit U;
+                get_unit(u, U);
+                const int wrow = U.e * static_cast<int>(p.n) + U.ntile * kBM;
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    if ((ks & 3) == 0) {
+                        if (!bwait(&raw_empty[rp.idx], rp.phase ^ 1)) break;
+                        mbar_arrive_expect_tx(&raw_full[rp.idx], kRawBytes);
+                        const int blk = ks >> 2;
+                        int xc;
+                        if constexpr (QT == KQ_Q4_K) xc = 144 * blk;
+                        else if constexpr (QT == KQ_Q6_K) xc = (210 * blk) & ~15;
+                        else xc = 136 * blk;   // 2-byte elements
+                        tma_load_2d(rst + rp.idx * kRawBytes, &wmap, xc, wrow, &raw_full[rp.idx]);
+                        rp.next(kRawStages);
+                    }
+                    if (!bwait(&b_empty[bp.idx], bp.phase ^ 1)) break;
+                    mbar_arrive_expect_tx(&b_full[bp.idx], U.nt * 8192);
+                    for (int i = 0; i < U.nt; ++i)
+                        tma_load_2d(bst + bp.idx * kBBytes + i * 8192, &xmap, ks * kBK, U.rs[i], &b_full[bp.idx]);
+                    bp.next(kBStages);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            Pipe ap, bp, cp;
+            for (int u = blockIdx.x; u < total_units && !aborted(); u += gridDim.x) {
+                Unit U;
+                get_unit(u, U);
+                const uint32_t idesc = make_idesc(mma_n(U));
+                if (!bwait(&acc_empty[cp.idx], cp.phase ^ 1)) break;
+                tc_fence_after();
+                const uint32_t dt = tmem + cp.idx * 256;
+                bool ok = true;
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    if (!bwait(&a_full[ap.idx], ap.phase) || !bwait(&b_full[bp.idx], bp.phase)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_desc(ast + ap.idx * kABytes);
+                    const uint64_t bd = sw128_desc(bst + bp.idx * kBBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        tc_mma(dt, ad + 2 * kk, bd + 2 * kk, idesc, (ks | kk) != 0);
+                    tc_commit(&a_empty[ap.idx]);
+                    tc_commit(&b_empty[bp.idx]);
+                    ap.next(AST);
+                    bp.next(kBStages);
+                }
+                if (!ok) break;
+                tc_commit(&acc_full[cp.idx]);
+                cp.next(2);
+            }
+        }
+    } else if (warp < kDeqWarp0) {
+        // ------------------------------------------------ epilogue
+        const int q = warp & 3;   // TMEM lane quarter this warp may access
+        Pipe cp;
+        for (int u = blockIdx.x; u < total_units && !aborted(); u += gridDim.x) {
+            Unit U;
+            get_unit(u, U);
+            const int nmma = mma_n(U);
+            if (!bwait(&acc_full[cp.idx], cp.phase)) break;
+            tc_fence_after();
+            const int64_t nrow = static_cast<int64_t>(U.ntile) * kBM + 32 * q + lane;
+            const bool row_ok = nrow < p.n;
+            const uint32_t tbase = tmem + cp.idx * 256 + (static_cast<uint32_t>(32 * q) << 16);
+            for (int c0 = 0; c0 < nmma; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld16(tbase + c0, v);
+                const int ti = c0 >> 6;
+                const int r0 = c0 & 63;
+                if (row_ok) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        if (r0 + i < U.nr[ti]) {
+                            const int64_t tok = static_cast<int64_t>(U.rs[ti]) + r0 + i;
+                            p.y[tok * p.n + nrow] = __uint_as_float(v[i]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[cp.idx]);
+            cp.next(2);
+        }
+    } else {
+        // ------------------------------------------------ decoders
+        const int dt = tid - kDeqWarp0 * 32;   // 0..255
+        const int r = dt & 127, part = dt >> 7;
+        Pipe rp, ap;
+        for (int u = blockIdx.x; u < total_units && !aborted(); u += gridDim.x) {
+            bool ok = true;
+            for (int ks = 0; ks < ksteps; ++ks) {
+                if ((ks & 3) == 0 && !bwait(&raw_full[rp.idx], rp.phase)) {
+                    ok = false;
+                    break;
+                }
+                if (!bwait(&a_empty[ap.idx], ap.phase ^ 1)) {
+                    ok = false;
+                    break;
+                }
+                uint32_t o[16];
+                const uint32_t row = rst + rp.idx * kRawBytes + r * C::RAWB;
+                const int o6 = QT == KQ_Q6_K ? (210 * (ks >> 2)) & 15 : 0;
+                decode_step<QT>(row, ks & 3, part, o6, o);
+                store_a(ast + ap.idx * kABytes, r, part, o);
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&a_full[ap.idx]);
+                ap.next(AST);
+                if ((ks & 3) == 3) {
+                    if (lane == 0) mbar_arrive(&raw_empty[rp.idx]);
+                    rp.next(kRawStages);
+                }
+            }
+            if (!ok) break;
+        }
+    }
+
+    // ---- tear-down
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+    }
+}
+
+// ------------------------------------------------------------------ host
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled get_encoder() {
+    static EncodeTiled fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(ptr);
+    }
+    return fn;
+}
+
+int make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* ptr, uint64_t inner, uint64_t outer,
+             uint32_t box_in, uint32_t box_out, CUtensorMapSwizzle sw) {
+    EncodeTiled enc = get_encoder();
+    if (!enc) return KQ_ERR_CUDA;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner * esize};
+    const cuuint32_t box[2] = {box_in, box_out};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? KQ_OK : KQ_ERR_INVALID_ARG;
+}
+
+template <int QT>
+int launch_impl(const void* w, int64_t w_rows, int64_t n, int64_t k, const uint16_t* x, int64_t x_rows, int n_experts,
+                const uint32_t* map, const uint32_t* count, int64_t cap, float* y, int32_t* err, cudaStream_t s) {
+    using C = QmmCodec<QT>;
+    const int vpb = QT == KQ_Q8_0 ? 32 : 256, bpb = QT == KQ_Q4_K ? 144 : (QT == KQ_Q6_K ? 210 : 34);
+    const int64_t row_bytes = k / vpb * bpb;
+    if (k % 256 != 0) return KQ_ERR_UNSUPPORTED;        // 256-value raw stages
+    if (row_bytes % 16 != 0) return KQ_ERR_UNSUPPORTED;  // TMA row stride
+    CUtensorMap wmap, xmap;
+    int rc;
+    if constexpr (QT == KQ_Q8_0)
+        rc = make_map(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, w, row_bytes / 2, w_rows, C::RAWB / 2, kBM,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+    else
+        rc = make_map(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w, row_bytes, w_rows, C::RAWB, kBM,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc) return rc;
+    rc = make_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, k, x_rows, kBK, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+
+    QmmParams p{};
+    p.n = n;
+    p.m = x_rows;
+    p.k = static_cast<int>(k);
+    p.n_experts = n_experts;
+    p.ntn = static_cast<int>((n + kBM - 1) / kBM);
+    p.units = n_experts == 0 ? static_cast<int>((x_rows + kBN - 1) / kBN) * p.ntn : 0;
+    p.map = map;
+    p.count = count;
+    p.cap = cap;
+    p.y = y;
+    p.err = err;
+    p.status = device_status_ptr();
+    const uint32_t smem = kHeader + 1024 + kBStages * kBN * kBK * 2 + C::AST * kBM * kBK * 2 + kRawStages * kBM * C::RAWB;
+    auto kern = qmm_kernel<QT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return record_cuda(e);
+    int grid = device_sm_count();
+    if (n_experts == 0 && p.units < grid) grid = p.units;
+    if (grid < 1) return KQ_OK;
+    kern<<<grid, kThreads, smem, s>>>(wmap, xmap, p);
+    return check_launch();
+}
+
+}  // namespace
+
+int launch_qmm(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int64_t m, float* y,
+               cudaStream_t s) {
+    if (n == 0 || m == 0) return KQ_OK;
+    switch (type) {
+    case KQ_Q4_K: return launch_impl<KQ_Q4_K>(w, n, n, k, x, m, 0, nullptr, nullptr, 0, y, nullptr, s);
+    case KQ_Q6_K: return launch_impl<KQ_Q6_K>(w, n, n, k, x, m, 0, nullptr, nullptr, 0, y, nullptr, s);
+    default: return launch_impl<KQ_Q8_0>(w, n, n, k, x, m, 0, nullptr, nullptr, 0, y, nullptr, s);
+    }
+}
+
+int launch_gather_qmm(int type, const void* w_bank, int n_experts, int64_t n, int64_t k, const uint16_t* x_sorted,
+                      int64_t rows, const uint32_t* map, const uint32_t* count, int64_t cap, float* y,
+                      int32_t* err_flag, cudaStream_t s) {
+    if (n == 0 || rows == 0) return KQ_OK;
+    const int64_t wr = static_cast<int64_t>(n_experts) * n;
+    switch (type) {
+    case KQ_Q4_K:
+        return launch_impl<KQ_Q4_K>(w_bank, wr, n, k, x_sorted, rows, n_experts, map, count, cap, y, err_flag, s);
+    case KQ_Q6_K:
+        return launch_impl<KQ_Q6_K>(w_bank, wr, n, k, x_sorted, rows, n_experts, map, count, cap, y, err_flag, s);
+    default:
+        return launch_impl<KQ_Q8_0>(w_bank, wr, n, k, x_sorted, rows, n_experts, map, count, cap, y, err_flag, s);
+    }
+}
+
+}  // namespace kq

@@ -1,0 +1,682 @@
+// kq_qmv: y = x . W^T for 1 <= m <= 16 activation rows (decode shape).
+//
+// mlx-kquant bindings.cpp `quantized_matmul` (x @ dequant(w).T); README "How
+// it works": small row counts take a kernel that amortizes each weight read
+// over all rows (`verify_qmv`); hanzo-ml quantized/mod.rs: decode runs the
+// quantized matvec "straight out of the block format".
+//
+// The path is HBM-bound, so the design goal is to spend as few instructions
+// per weight as possible while reading every weight byte exactly once:
+//
+//  * Each CTA owns 16 weight rows and all of K.  Its row segments (several
+//    blocks per row) are streamed into a ring of shared-memory stages by 1-D
+//    bulk async copies (one per row, issued by warp 0, completion counted on
+//    an mbarrier), so many kilobytes per SM are in flight without registers.
+//  * The 8 warps split the blocks of a stage.  A warp decodes its 16 rows into
+//    m16n8k16 tensor-core A fragments whose entries are EXACT integers in
+//    binary16: the codes themselves (q6_K, q8_0) or code * 6-bit scale
+//    (q4_K, at most 945).  The activations, rounded once to binary16, are the
+//    B fragments (pre-permuted per CTA into a shared-memory "image" so each
+//    fragment is one 8-byte load).  The tensor core forms exact products and
+//    accumulates them in fp32, so the only rounding besides fp32 summation is
+//    x -> binary16.
+//  * Binary16 codes come from the exponent trick: OR-ing a 4/6/8-bit code
+//    into the mantissa of 1024.0 gives 1024 + code exactly.  The 1024 bias
+//    is removed exactly (q4_K: one HFMA2 that also applies the scale) or
+//    folded into a per-sub-block correction c * sum(x) in the epilogue.
+//  * q4_K (per-block scales d, dmin): each lane owns one 64-value group of a
+//    block, so it decodes only its own two 6-bit scale/min pairs; the MMA
+//    chain runs over the whole block and the min term sum_j m_j * X_j is one
+//    more MMA on (m_j) x (X_j split into two binary16 halves).
+//  * q6_K / q8_0 (per-16- or per-32-value scales): the chain stops at every
+//    sub-block.  For m <= 4 the 8 MMA columns are shared out as
+//    (token, sub-block slot) pairs, so one epilogue covers up to 8 sub-blocks
+//    instead of wasting 7 of 8 columns.
+//  * Partial sums of the 8 warps are combined in shared memory in a fixed
+//    order: no atomics, bitwise reproducible.
+#include "kq_device.cuh"
+#include "kq_launch.h"
+
+namespace kq {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kRows = 16;
+constexpr int kOffW = 128;   // barriers, abort flag and a zero word live below
+
+template <int QT> struct Codec;
+template <> struct Codec<KQ_Q4_K> {
+    static constexpr int VPB = 256, BPB = 144, G = 8, RS = 1168;  // RS = 16 mod 128
+    static constexpr int IMG = 544, XS = 0;   // B image bytes / fp32 sums per (token, block)
+};
+template <> struct Codec<KQ_Q6_K> {
+    static constexpr int VPB = 256, BPB = 210, G = 8, RS = 1680;
+    static constexpr int IMG = 1024, XS = 16;
+};
+template <> struct Codec<KQ_Q8_0> {
+    static constexpr int VPB = 32, BPB = 34, G = 64, RS = 2192;
+    static constexpr int IMG = 64, XS = 1;
+};
+
+struct QmvParams {
+    const uint8_t* w;
+    const uint16_t* x;
+    float* y;
+    int* status;
+    int64_t n, k, row_bytes;
+    int m, nblk, scb, ns, bulk;
+    uint32_t tokstride, off_img, off_x;
+};
+
+// binary16 constants
+constexpr uint32_t kH1024 = 0x64006400u;    // (1024, 1024)
+constexpr uint32_t kHm1024 = 0xE400E400u;   // (-1024, -1024)
+constexpr uint32_t kH1_16 = 0x2C002C00u;    // (1/16, 1/16)
+
+// Shared-memory loads are volatile so that they are never moved across the
+// mbarrier waits and __syncthreads that order them with the bulk copies.
+__device__ __forceinline__ uint32_t lds32c(uint32_t a) { return lds32(a); }
+__device__ __forceinline__ uint2 lds64c(uint32_t a) { return lds64(a); }
+__device__ __forceinline__ uint4 lds128c(uint32_t a) { return lds128(a); }
+__device__ __forceinline__ uint32_t ldsu16c(uint32_t a) {
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ int ldss8c(uint32_t a) {
+    int16_t v;
+    asm volatile("ld.shared.s8 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float ldsf32c(uint32_t a) { return __uint_as_float(lds32c(a)); }
+// 4 bytes at a 2-byte aligned address; `odd` = (a & 2) is warp-uniform.
+__device__ __forceinline__ uint32_t lds32c_a2(uint32_t a, bool odd) {
+    if (!odd) return lds32c(a);
+    return __byte_perm(lds32c(a - 2), lds32c(a + 2), 0x5432);
+}
+__device__ __forceinline__ void sts64(uint32_t a, uint32_t x, uint32_t y) {
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(x), "r"(y));
+}
+__device__ __forceinline__ void sts32(uint32_t a, uint32_t x) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(x));
+}
+__device__ __forceinline__ float h16(uint32_t h) { return __half2float(__ushort_as_half((unsigned short)h)); }
+
+// x (bf16) -> binary16, recording a range violation.
+__device__ __forceinline__ uint32_t f16pair(float a, float b, float& amax) {
+    amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
+    return pack_f16x2(a, b);
+}
+
+// ---------------------------------------------------------------------------
+// Activation images.  For block bl of the current super-chunk and token m the
+// image holds, for every MMA of that block and every lane column t, the two
+// B registers of lane (g = token, t) in binary16.
+// ---------------------------------------------------------------------------
+template <int QT>
+__device__ void build_image(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t xsum, float& amax);
+
+// q4_K: MMA (nib, u) of lane t uses values v = 64t + 32nib + 4u + {0,2 | 1,3};
+// the extra 32 bytes per block hold (Xhi, Xlo) of sub-blocks 2t and 2t+1.
+template <>
+__device__ void build_image<KQ_Q4_K>(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t, float& amax) {
+    const int items = p.m * nb * 4;
+    for (int it = threadIdx.x; it < items; it += kThreads) {
+        const int m = it / (nb * 4), rem = it % (nb * 4), bl = rem >> 2, t = rem & 3;
+        const uint16_t* xs = p.x + static_cast<int64_t>(m) * p.k + static_cast<int64_t>(blk0 + bl) * 256 + 64 * t;
+        const uint32_t base = img + m * p.tokstride + bl * 544;
+        float X[2] = {0.f, 0.f};
+#pragma unroll
+        for (int nib = 0; nib < 2; ++nib) {
+#pragma unroll
+            for (int uu = 0; uu < 2; ++uu) {
+                const uint4 r0 = ldg_nc_v4(xs + 32 * nib + 16 * uu);
+                const uint4 r1 = ldg_nc_v4(xs + 32 * nib + 16 * uu + 8);
+                const uint32_t wv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int u = 4 * uu + q;
+                    const float f0 = bf16lo_to_f32(wv[2 * q]), f1 = bf16hi_to_f32(wv[2 * q]);
+                    const float f2 = bf16lo_to_f32(wv[2 * q + 1]), f3 = bf16hi_to_f32(wv[2 * q + 1]);
+                    const uint32_t h02 = f16pair(f0, f2, amax), h13 = f16pair(f1, f3, amax);
+                    X[nib] += (h16(h02 & 0xffff) + h16(h13 & 0xffff)) + (h16(h02 >> 16) + h16(h13 >> 16));
+                    sts64(base + (nib * 8 + u) * 32 + t * 8, h02, h13);
+                }
+            }
+        }
+        uint32_t e[2];
+#pragma unroll
+        for (int nib = 0; nib < 2; ++nib) {
+            const __half hi = __float2half_rn(X[nib]);
+            const __half lo = __float2half_rn(X[nib] - __half2float(hi));
+            e[nib] = static_cast<uint32_t>(__half_as_ushort(hi)) | (static_cast<uint32_t>(__half_as_ushort(lo)) << 16);
+        }
+        sts64(base + 512 + t * 8, e[0], e[1]);
+    }
+}
+
+// q8_0: MMA h (0, 1) of lane t uses values v = 8t + 4h + {0,2 | 1,3};
+// X = sum of the block's 32 binary16 values.
+template <>
+__device__ void build_image<KQ_Q8_0>(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t xsum, float& amax) {
+    const int items = p.m * nb;
+    for (int it = threadIdx.x; it < items; it += kThreads) {
+        const int m = it / nb, bl = it % nb;
+        const uint16_t* xs = p.x + static_cast<int64_t>(m) * p.k + static_cast<int64_t>(blk0 + bl) * 32;
+        const uint32_t base = img + m * p.tokstride + bl * 64;
+        float X = 0.f;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const uint4 r = ldg_nc_v4(xs + 8 * t);
+            const uint32_t wv[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float f0 = bf16lo_to_f32(wv[2 * h]), f1 = bf16hi_to_f32(wv[2 * h]);
+                const float f2 = bf16lo_to_f32(wv[2 * h + 1]), f3 = bf16hi_to_f32(wv[2 * h + 1]);
+                const uint32_t h02 = f16pair(f0, f2, amax), h13 = f16pair(f1, f3, amax);
+                X += (h16(h02 & 0xffff) + h16(h13 & 0xffff)) + (h16(h02 >> 16) + h16(h13 >> 16));
+                sts64(base + h * 32 + t * 8, h02, h13);
+            }
+        }
+        sts32(xsum + (m * p.scb + bl) * 4, __float_as_uint(X));
+    }
+}
+
+// q6_K: sub-block j (16 values, j = 8h + 2tq + u) has a low-code MMA and a
+// high-code MMA; lane t uses values 16j + 4t + {0,2 | 1,3}.  The low-code B
+// is x (tq < 2) or x/16 (tq >= 2, where the code sits in the high nibble);
+// the high-code B is x (tq < 3) or x/4 (tq = 3).  X_j = sum of 16 values.
+template <>
+__device__ void build_image<KQ_Q6_K>(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t xsum, float& amax) {
+    const int items = p.m * nb * 16;
+    for (int it = threadIdx.x; it < items; it += kThreads) {
+        const int m = it / (nb * 16), rem = it % (nb * 16), bl = rem >> 4, j = rem & 15;
+        const int tq = (j & 7) >> 1;
+        const float slo = tq < 2 ? 1.0f : 0.0625f, shi = tq < 3 ? 1.0f : 0.25f;
+        const uint16_t* xs = p.x + static_cast<int64_t>(m) * p.k + static_cast<int64_t>(blk0 + bl) * 256 + 16 * j;
+        const uint32_t base = img + m * p.tokstride + bl * 1024 + j * 64;
+        const uint4 r0 = ldg_nc_v4(xs), r1 = ldg_nc_v4(xs + 8);
+        const uint32_t wv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+        float X = 0.f;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const float f0 = bf16lo_to_f32(wv[2 * t]), f1 = bf16hi_to_f32(wv[2 * t]);
+            const float f2 = bf16lo_to_f32(wv[2 * t + 1]), f3 = bf16hi_to_f32(wv[2 * t + 1]);
+            const uint32_t h02 = f16pair(f0, f2, amax), h13 = f16pair(f1, f3, amax);
+            X += (h16(h02 & 0xffff) + h16(h13 & 0xffff)) + (h16(h02 >> 16) + h16(h13 >> 16));
+            sts64(base + t * 8, pack_f16x2(f0 * slo, f2 * slo), pack_f16x2(f1 * slo, f3 * slo));
+            sts64(base + 32 + t * 8, pack_f16x2(f0 * shi, f2 * shi), pack_f16x2(f1 * shi, f3 * shi));
+        }
+        sts32(xsum + ((m * p.scb + bl) * 16 + j) * 4, __float_as_uint(X));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Per-warp block processing
+// ---------------------------------------------------------------------------
+template <int NT>
+struct Lane {
+    int g, t;
+    uint32_t tokb[NT];   // image base of the lane's B column (token) per n-tile
+    int tok[NT];         // token index (clamped) of that column
+};
+
+// q4_K, one superblock of 16 rows.  rowA/rowB: shared address of the block in
+// rows g and g+8.  imgb: offset of the block inside a token image.
+template <int NT>
+__device__ __forceinline__ void q4k_block(const Lane<NT>& L, uint32_t rowA, uint32_t rowB, uint32_t imgb,
+                                          float (&acc)[NT][4]) {
+    const int t = L.t;
+    const uint4 hA = lds128c(rowA), hB = lds128c(rowB);
+    const uint4 qA0 = lds128c(rowA + 16 + 32 * t), qA1 = lds128c(rowA + 32 + 32 * t);
+    const uint4 qB0 = lds128c(rowB + 16 + 32 * t), qB1 = lds128c(rowB + 32 + 32 * t);
+    // 6-bit scale/min codes of sub-blocks 2t, 2t+1 as (code_2t, code_2t+1) in
+    // bits 0..5 / 16..21.  For t < 2: sc = s[j] & 63, m = s[j+4] & 63.  For
+    // t >= 2 (j >= 4, jj = j-4): sc = (s[j+4] & 15) | (s[jj] >> 6) << 4 and
+    // m = (s[j+4] >> 4) | (s[j] >> 6) << 4.
+    const bool lo = t < 2;
+    const uint32_t jj0 = (2 * t) & 3;
+    const uint32_t sel = 0x4040u | jj0 | ((jj0 + 1) << 8);
+    const uint32_t mka = lo ? 0x003F003Fu : 0x000F000Fu, mkb = lo ? 0u : 0x00300030u;
+    uint32_t S_lo[2], B_lo[2], S_hi[2], B_hi[2], M_lo[2], M_hi[2];
+    float dd[2], dm[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const uint4 h = r ? hB : hA;
+        const uint32_t asc = lo ? h.y : h.w;
+        const uint32_t am = lo ? h.z : (h.w >> 4);
+        const uint32_t scp = (__byte_perm(asc, 0, sel) & mka) | ((__byte_perm(h.y, 0, sel) >> 2) & mkb);
+        const uint32_t mp = (__byte_perm(am, 0, sel) & mka) | ((__byte_perm(h.z, 0, sel) >> 2) & mkb);
+        const uint32_t scf = hsub2_u32(scp | kH1024, kH1024);   // (sc_2t, sc_2t+1) exact
+        const uint32_t mf = hsub2_u32(mp | kH1024, kH1024);
+        S_lo[r] = __byte_perm(scf, 0, 0x1010);
+        S_hi[r] = hmul2_u32(__byte_perm(scf, 0, 0x3232), kH1_16);
+        B_lo[r] = hmul2_u32(S_lo[r], kHm1024);   // -1024 sc
+        B_hi[r] = hmul2_u32(S_hi[r], kHm1024);   // -64 sc
+        M_lo[r] = __byte_perm(mf, 0, 0x1010);
+        M_hi[r] = __byte_perm(mf, 0, 0x3232);
+        dd[r] = h16(h.x & 0xffff);
+        dm[r] = h16(h.x >> 16);
+    }
+    const uint32_t wA[8] = {qA0.x, qA0.y, qA0.z, qA0.w, qA1.x, qA1.y, qA1.z, qA1.w};
+    const uint32_t wB[8] = {qB0.x, qB0.y, qB0.z, qB0.w, qB1.x, qB1.y, qB1.z, qB1.w};
+    float D[NT][4], Dm[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) D[nt][e] = Dm[nt][e] = 0.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const uint32_t a = wA[u], b = wB[u], a8 = a >> 8, b8 = b >> 8;
+        // low nibbles: 1024 + q, times sc, minus 1024 sc -> q*sc exactly
+        {
+            const uint32_t a0 = hfma2_u32(and_or(a, 0x000F000Fu, kH1024), S_lo[0], B_lo[0]);
+            const uint32_t a1 = hfma2_u32(and_or(b, 0x000F000Fu, kH1024), S_lo[1], B_lo[1]);
+            const uint32_t a2 = hfma2_u32(and_or(a8, 0x000F000Fu, kH1024), S_lo[0], B_lo[0]);
+            const uint32_t a3 = hfma2_u32(and_or(b8, 0x000F000Fu, kH1024), S_lo[1], B_lo[1]);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const uint2 bv = lds64c(L.tokb[nt] + imgb + u * 32 + t * 8);
+                mma_f16(D[nt], a0, a1, a2, a3, bv.x, bv.y);
+            }
+        }
+        // high nibbles: 1024 + 16q, times sc/16, minus 64 sc -> q*sc exactly
+        {
+            const uint32_t a0 = hfma2_u32(and_or(a, 0x00F000F0u, kH1024), S_hi[0], B_hi[0]);
+            const uint32_t a1 = hfma2_u32(and_or(b, 0x00F000F0u, kH1024), S_hi[1], B_hi[1]);
+            const uint32_t a2 = hfma2_u32(and_or(a8, 0x00F000F0u, kH1024), S_hi[0], B_hi[0]);
+            const uint32_t a3 = hfma2_u32(and_or(b8, 0x00F000F0u, kH1024), S_hi[1], B_hi[1]);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const uint2 bv = lds64c(L.tokb[nt] + imgb + (8 + u) * 32 + t * 8);
+                mma_f16(D[nt], a0, a1, a2, a3, bv.x, bv.y);
+            }
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const uint2 bv = lds64c(L.tokb[nt] + imgb + 512 + t * 8);
+        mma_f16(Dm[nt], M_lo[0], M_lo[1], M_hi[0], M_hi[1], bv.x, bv.y);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int r = e >> 1;
+            acc[nt][e] = fmaf(dd[r], D[nt][e], fmaf(-dm[r], Dm[nt][e], acc[nt][e]));
+        }
+    }
+}
+
+// Column bookkeeping for the slot variants (q6_K, q8_0): column c of n-tile nt
+// holds token c / S and sub-block slot c % S (S > 1), or token 8 nt + c.
+template <int S, int NT>
+__device__ __forceinline__ void col_info(int nt, int col, int m, int& tok, int& slot) {
+    if (S > 1) {
+        tok = col / S;
+        slot = col % S;
+    } else {
+        tok = 8 * nt + col;
+        slot = 0;
+    }
+    tok = tok < m ? tok : m - 1;
+}
+
+// q8_0: the warp's run of up to 8 consecutive 32-value blocks of one stage.
+// rowA/rowB: shared address of row g / g+8 of the stage; lb0: first local
+// block; nvalid: blocks present; imgb0 / xsb0: image/X offsets of lb0.
+template <int S, int NT>
+__device__ __forceinline__ void q8_run(const Lane<NT>& L, const QmvParams& p, uint32_t rowA, uint32_t rowB, int lb0,
+                                       int nvalid, uint32_t imgb0, uint32_t xsb0, uint32_t zero_addr,
+                                       float (&acc)[NT][4]) {
+    const int t = L.t;
+    float D[NT][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        if (i % S == 0) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) D[nt][e] = 0.f;
+        }
+        if (i < nvalid) {
+            const int lb = lb0 + i;
+            const uint32_t off = lb * 34 + 2 + 8 * t;
+            const bool odd = (off & 2) != 0;
+            const uint32_t a0w = lds32c_a2(rowA + off, odd), a1w = lds32c_a2(rowA + off + 4, odd);
+            const uint32_t b0w = lds32c_a2(rowB + off, odd), b1w = lds32c_a2(rowB + off + 4, odd);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t wa = h ? a1w : a0w, wb = h ? b1w : b0w;
+                // (byte ^ 0x80) in the mantissa of 1024: 1024 + q + 128 exactly
+                const uint32_t A0 = and_xor(wa, 0x00FF00FFu, 0x64806480u);
+                const uint32_t A1 = and_xor(wb, 0x00FF00FFu, 0x64806480u);
+                const uint32_t A2 = and_xor(wa >> 8, 0x00FF00FFu, 0x64806480u);
+                const uint32_t A3 = and_xor(wb >> 8, 0x00FF00FFu, 0x64806480u);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    uint32_t addr = L.tokb[nt] + imgb0 + i * 64 + h * 32 + t * 8;
+                    if (S > 1 && (L.g % S) != (i % S)) addr = zero_addr;
+                    const uint2 bv = lds64c(addr);
+                    mma_f16(D[nt], A0, A1, A2, A3, bv.x, bv.y);
+                }
+            }
+        }
+        if (i % S == S - 1 || i == 7) {
+            // epilogue: y += d * (D - 1152 X) per column's block
+            const int i0 = i - (i % S);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    int tok, slot;
+                    col_info<S, NT>(nt, 2 * t + (e & 1), p.m, tok, slot);
+                    const int ib = i0 + slot;
+                    if (ib < nvalid && ib <= i) {
+                        const uint32_t row = (e >> 1) ? rowB : rowA;
+                        const float d = h16(ldsu16c(row + (lb0 + ib) * 34));
+                        const float X = ldsf32c(xsb0 + (tok * p.scb + ib) * 4);
+                        acc[nt][e] = fmaf(d, fmaf(-1152.0f, X, D[nt][e]), acc[nt][e]);
+                    }
+                }
+            }
+        }
+    }
+}
+
+// q6_K: one 256-value block of 16 rows; sub-blocks in order j = 8h + 2tq + u.
+template <int S, int NT>
+__device__ __forceinline__ void q6k_block(const Lane<NT>& L, const QmvParams& p, uint32_t rowA, uint32_t rowB,
+                                          bool odd, uint32_t imgb, uint32_t xsb, uint32_t zero_addr,
+                                          float (&acc)[NT][4]) {
+    const int t = L.t;
+    const float dA = h16(ldsu16c(rowA + 208));
+    const float dB = h16(ldsu16c(rowB + 208));
+    // the lane's 4-byte pieces: ql[h][pp][u] and qh[h][u] for rows g and g+8
+    uint32_t QLA[8], QLB[8], QHA[4], QHB[4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t o = 64 * (i >> 2) + 32 * ((i >> 1) & 1) + 16 * (i & 1) + 4 * t;
+        QLA[i] = lds32c_a2(rowA + o, odd);
+        QLB[i] = lds32c_a2(rowB + o, odd);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t o = 128 + 32 * (i >> 1) + 16 * (i & 1) + 4 * t;
+        QHA[i] = lds32c_a2(rowA + o, odd);
+        QHB[i] = lds32c_a2(rowB + o, odd);
+    }
+    float D[NT][4];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const int h = j >> 3, tq = (j & 7) >> 1, u = j & 1, pp = tq & 1;
+        if (j % S == 0) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) D[nt][e] = 0.f;
+        }
+        const uint32_t la = QLA[4 * h + 2 * pp + u], lb = QLB[4 * h + 2 * pp + u];
+        const uint32_t ha = QHA[2 * h + u], hb = QHB[2 * h + u];
+        // low 4 bits: low nibble (tq < 2) -> 1024 + c, high nibble -> 1024 + 16c
+        const uint32_t mlo = tq < 2 ? 0x000F000Fu : 0x00F000F0u;
+        const uint32_t L0 = and_or(la, mlo, kH1024), L1 = and_or(lb, mlo, kH1024);
+        const uint32_t L2 = and_or(la >> 8, mlo, kH1024), L3 = and_or(lb >> 8, mlo, kH1024);
+        // high 2 bits (bits 2tq of each qh byte) moved to bits 4..5 (tq < 3):
+        // 1024 + 16c; tq = 3 stays at bits 6..7: 1024 + 64c with B = x/4.
+        uint32_t H0, H1, H2, H3;
+        if (tq == 3) {
+            H0 = and_or(ha, 0x00C000C0u, kH1024);
+            H1 = and_or(hb, 0x00C000C0u, kH1024);
+            H2 = and_or(ha >> 8, 0x00C000C0u, kH1024);
+            H3 = and_or(hb >> 8, 0x00C000C0u, kH1024);
+        } else {
+            const int sh = 4 - 2 * tq;   // 4, 2, 0: left shift for bytes 0/2
+            H0 = and_or(ha << sh, 0x00300030u, kH1024);
+            H1 = and_or(hb << sh, 0x00300030u, kH1024);
+            H2 = and_or(ha >> (8 - sh), 0x00300030u, kH1024);
+            H3 = and_or(hb >> (8 - sh), 0x00300030u, kH1024);
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const bool mine = !(S > 1) || (L.g % S) == (j % S);
+            const uint32_t a = L.tokb[nt] + imgb + j * 64 + t * 8;
+            const uint2 bl = lds64c(mine ? a : zero_addr);
+            const uint2 bh = lds64c(mine ? a + 32 : zero_addr);
+            mma_f16(D[nt], L0, L1, L2, L3, bl.x, bl.y);
+            mma_f16(D[nt], H0, H1, H2, H3, bh.x, bh.y);
+        }
+        if (j % S == S - 1) {
+            const int j0 = j - (S - 1);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    int tok, slot;
+                    col_info<S, NT>(nt, 2 * t + (e & 1), p.m, tok, slot);
+                    const int jj = j0 + slot;
+                    const int tqj = (jj & 7) >> 1;
+                    // bias of the two MMAs: 1024/sigma_lo + 1024/sigma_hi' + 32
+                    const float C = tqj < 2 ? 2080.0f : (tqj == 2 ? 1120.0f : 352.0f);
+                    const uint32_t row = (e >> 1) ? rowB : rowA;
+                    const float dr = (e >> 1) ? dB : dA;
+                    const int sc = ldss8c(row + 192 + jj);
+                    const float s = __fmul_rn(dr, static_cast<float>(sc));
+                    const float X = ldsf32c(xsb + (tok * p.scb * 16 + jj) * 4);
+                    acc[nt][e] = fmaf(s, fmaf(-C, X, D[nt][e]), acc[nt][e]);
+                }
+            }
+        }
+    }
+}
+
+template <int QT, int S, int NT>
+__global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const QmvParams p) {
+    using C = Codec<QT>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 64);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t zero_addr = sbase + 96;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRows;
+    const int rows_valid = static_cast<int>(p.n - row0 < kRows ? p.n - row0 : kRows);
+    const int nstages = cdiv(p.nblk, C::G);
+    const int spsc = p.scb / C::G;
+
+    if (tid == 0) {
+        for (int i = 0; i < p.ns; ++i) mbar_init(&full[i], 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (tid < 4) sts32(zero_addr + 4 * tid, 0u);
+    __syncthreads();
+
+    auto stage_addr = [&](int slot) { return sbase + kOffW + slot * (kRows * C::RS); };
+    auto issue = [&](int s) {   // warp 0
+        const int slot = s % p.ns, b0 = s * C::G;
+        const int nb = p.nblk - b0 < C::G ? p.nblk - b0 : C::G;
+        const uint32_t bytes = nb * C::BPB;
+        if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes * rows_valid);
+        __syncwarp();
+        if (lane < rows_valid)
+            bulk_g2s(smem + kOffW + slot * (kRows * C::RS) + lane * C::RS,
+                     p.w + (row0 + lane) * p.row_bytes + static_cast<int64_t>(b0) * C::BPB, bytes, &full[slot]);
+    };
+    auto sync_load = [&](int s) {   // all threads; any alignment (2-byte units)
+        const int slot = s % p.ns, b0 = s * C::G;
+        const int nb = p.nblk - b0 < C::G ? p.nblk - b0 : C::G;
+        const int half = nb * C::BPB / 2;
+        const uint32_t dst = stage_addr(slot);
+        for (int i = tid; i < rows_valid * half; i += kThreads) {
+            const int r = i / half, c = i % half;
+            const unsigned short v =
+                __ldg(reinterpret_cast<const unsigned short*>(p.w + (row0 + r) * p.row_bytes +
+                                                              static_cast<int64_t>(b0) * C::BPB) + c);
+            asm volatile("st.shared.u16 [%0], %1;" ::"r"(dst + r * C::RS + 2 * c), "h"(v));
+        }
+        __syncthreads();
+    };
+
+    int issued = 0;
+    if (p.bulk && warp == 0)
+        for (; issued < p.ns && issued < nstages; ++issued) issue(issued);
+
+    Lane<NT> L;
+    L.g = lane >> 2;
+    L.t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        int tok, slot;
+        col_info<S, NT>(nt, L.g, p.m, tok, slot);
+        L.tok[nt] = tok;
+        L.tokb[nt] = sbase + p.off_img + tok * p.tokstride;
+    }
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+    float amax = 0.f;
+    int s = 0;
+    for (; s < nstages; ++s) {
+        if (s % spsc == 0) {
+            const int blk0 = s * C::G;
+            const int nb = p.nblk - blk0 < p.scb ? p.nblk - blk0 : p.scb;
+            __syncthreads();
+            build_image<QT>(p, blk0, nb, sbase + p.off_img, sbase + p.off_x, amax);
+            __syncthreads();
+        }
+        const int slot = s % p.ns;
+        if (p.bulk) {
+            if (!mbar_wait(&full[slot], (s / p.ns) & 1, p.status)) *abort_flag = 1;
+        } else {
+            sync_load(s);
+        }
+        const int b0 = s * C::G;
+        const int nb = p.nblk - b0 < C::G ? p.nblk - b0 : C::G;
+        const int scbase = (s / spsc) * spsc * C::G;   // first block of the super-chunk
+        const uint32_t st = stage_addr(slot);
+        const uint32_t rowA = st + L.g * C::RS, rowB = rowA + 8 * C::RS;
+        if constexpr (QT == KQ_Q4_K) {
+            if (warp < nb) q4k_block<NT>(L, rowA + warp * 144, rowB + warp * 144, (b0 + warp - scbase) * 544, acc);
+        } else if constexpr (QT == KQ_Q6_K) {
+            if (warp < nb) {
+                const int lbi = b0 + warp - scbase;
+                q6k_block<S, NT>(L, p, rowA + warp * 210, rowB + warp * 210, (warp & 1) != 0, lbi * 1024,
+                                 sbase + p.off_x + lbi * 64, zero_addr, acc);
+            }
+        } else {
+            const int lb0 = 8 * warp;
+            if (lb0 < nb) {
+                const int nv = nb - lb0 < 8 ? nb - lb0 : 8;
+                const int lbi = b0 + lb0 - scbase;
+                q8_run<S, NT>(L, p, rowA, rowB, lb0, nv, lbi * 64, sbase + p.off_x + lbi * 4, zero_addr, acc);
+            }
+        }
+        __syncthreads();
+        if (*abort_flag) break;
+        if (p.bulk && warp == 0 && issued < nstages) issue(issued++);
+    }
+    if (*abort_flag) {
+        // wind down: let every copy still in flight land before the CTA exits
+        if (warp == 0 && lane == 0)
+            for (int q = s + 1; q < issued; ++q) mbar_wait(&full[q % p.ns], (q / p.ns) & 1, nullptr);
+        __syncthreads();
+        return;
+    }
+    if (amax >= 65504.0f) atomicOr(p.status, KQ_DEV_X_RANGE);
+
+    // ---- combine the 8 warps' partial sums (fixed order) and store y
+    float* red = reinterpret_cast<float*>(smem + kOffW);   // [warp][16 rows][16 cols]
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int r = L.g + 8 * (e >> 1), c = nt * 8 + 2 * L.t + (e & 1);
+            red[(warp * 16 + r) * 16 + c] = acc[nt][e];
+        }
+    }
+    __syncthreads();
+    const int ntok = p.m;
+    for (int i = tid; i < ntok * kRows; i += kThreads) {
+        const int tok = i / kRows, r = i % kRows;
+        if (r >= rows_valid) continue;
+        float sum = 0.f;
+        if (S > 1) {
+            for (int w = 0; w < kWarps; ++w)
+                for (int sl = 0; sl < S; ++sl) sum += red[(w * 16 + r) * 16 + tok * S + sl];
+        } else {
+            for (int w = 0; w < kWarps; ++w) sum += red[(w * 16 + r) * 16 + tok];
+        }
+        p.y[static_cast<int64_t>(tok) * p.n + row0 + r] = sum;
+    }
+}
+
+template <int QT>
+int launch_codec(const void* w, int64_t n, int64_t k, const uint16_t* x, int m, float* y, cudaStream_t st) {
+    using C = Codec<QT>;
+    QmvParams p{};
+    p.w = static_cast<const uint8_t*>(w);
+    p.x = x;
+    p.y = y;
+    p.status = device_status_ptr();
+    p.n = n;
+    p.k = k;
+    p.m = m;
+    p.nblk = static_cast<int>(k / C::VPB);
+    p.row_bytes = static_cast<int64_t>(p.nblk) * C::BPB;
+    p.bulk = (p.row_bytes % 16 == 0) && (reinterpret_cast<uintptr_t>(w) % 16 == 0);
+    const int optin = device_smem_optin();
+    const int nblk_g = cdiv(p.nblk, C::G) * C::G;
+    // Choose stage count and super-chunk size (blocks whose activation image
+    // is resident at once): as many blocks as fit, a multiple of G.
+    int ns = 3, scb = 0;
+    uint32_t tokstride = 0, off_img = 0, off_x = 0, total = 0;
+    for (; ns >= 2; --ns) {
+        const uint32_t wbytes = kOffW + ns * kRows * C::RS;
+        off_img = (wbytes + 127) & ~127u;
+        for (scb = nblk_g; scb >= C::G; scb -= C::G) {
+            const uint32_t base = scb * C::IMG;
+            tokstride = base + ((32u - (base & 127u)) & 127u);
+            off_x = off_img + m * tokstride;
+            total = off_x + m * scb * C::XS * 4;
+            if (total <= static_cast<uint32_t>(optin)) break;
+        }
+        if (scb >= C::G) break;
+    }
+    if (scb < C::G) return KQ_ERR_UNSUPPORTED;
+    p.ns = ns;
+    p.scb = scb;
+    p.tokstride = tokstride;
+    p.off_img = off_img;
+    p.off_x = off_x;
+    const int grid = cdiv(n, kRows);
+    auto launch = [&](auto kernel) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
+        if (e != cudaSuccess) return record_cuda(e);
+        kernel<<<grid, kThreads, total, st>>>(p);
+        return check_launch();
+    };
+    if constexpr (QT == KQ_Q4_K) {
+        return m > 8 ? launch(qmv_kernel<QT, 1, 2>) : launch(qmv_kernel<QT, 1, 1>);
+    } else {
+        if (m == 1) return launch(qmv_kernel<QT, 8, 1>);
+        if (m == 2) return launch(qmv_kernel<QT, 4, 1>);
+        if (m <= 4) return launch(qmv_kernel<QT, 2, 1>);
+        if (m <= 8) return launch(qmv_kernel<QT, 1, 1>);
+        return launch(qmv_kernel<QT, 1, 2>);
+    }
+}
+
+}  // namespace
+
+int launch_qmv(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int m, float* y,
+               cudaStream_t s) {
+    if (n == 0) return KQ_OK;
+    switch (type) {
+    case KQ_Q4_K: return launch_codec<KQ_Q4_K>(w, n, k, x, m, y, s);
+    case KQ_Q6_K: return launch_codec<KQ_Q6_K>(w, n, k, x, m, y, s);
+    default: return launch_codec<KQ_Q8_0>(w, n, k, x, m, y, s);
+    }
+}
+
+}  // namespace kq

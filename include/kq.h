@@ -1,0 +1,186 @@
+/*
+ * kq.h - C ABI of the B200 (sm_100a) library for matrix products with GGUF
+ * block-quantized weights: y = x . W^T where W is stored as q4_K, q6_K or
+ * q8_0 wire blocks.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every pointer argument is a DEVICE pointer (memory the caller allocated on
+ *    the current CUDA device, e.g. through torch), unless a comment says
+ *    "host".  The library allocates no device memory on any call below and
+ *    keeps no state other than the lazily created per-device kernel attribute
+ *    settings.  The caller owns every buffer.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every compute call is asynchronous on that stream: it only
+ *    validates its arguments on the host and enqueues kernels.  No call
+ *    synchronizes with the device.
+ *  - W is the codec's wire bytes for an [n, k] matrix, row-major, rows
+ *    contiguous: row r starts at byte r * row_bytes with
+ *    row_bytes = (k / values_per_block) * bytes_per_block.  This is the
+ *    "transpose=True" layout of the mlx-kquant `quantized_matmul` op
+ *    (bindings.cpp docstring: "uint8 K-quant wire bytes (laid out [N, K] when
+ *    transpose=True)") and of the README's "x @ dequant(w).T".
+ *  - Activations x are bfloat16 [m, k] row-major (passed as uint16_t bit
+ *    patterns).  They are converted to binary16 inside the kernels, so
+ *    |x| must stay below 65504 for qmv; bf16 is used as is by qmm/gather.
+ *  - Outputs y are fp32 [m, n] row-major.
+ *  - Return value: a kq_status.  A non-zero status means nothing was enqueued
+ *    (argument errors) or that the CUDA launch failed (KQ_ERR_CUDA; the
+ *    cudaError_t is available from kq_last_cuda_error()).  Nothing throws.
+ *  - Alignment: W, x, y and out must be 16-byte aligned, else
+ *    KQ_ERR_ALIGNMENT.  Weight rows whose byte length is not a multiple of 16
+ *    are accepted; they take a slower staging path.
+ *  - `k` must be a multiple of the codec's values_per_block, as the reference
+ *    requires ("last dim a multiple of the codec's bytes_per_block",
+ *    bindings.cpp `dequantize`); otherwise KQ_ERR_INVALID_ARG.
+ */
+#ifndef KQ_H
+#define KQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ggml / GGUF type ids of the supported codecs. */
+typedef enum {
+    KQ_Q8_0 = 8,   /* 32 values, 34 bytes: fp16 d, 32 x int8               */
+    KQ_Q4_K = 12,  /* 256 values, 144 bytes: fp16 d, fp16 dmin, 12 B packed
+                      6-bit scale/min codes, 128 B of 4-bit codes             */
+    KQ_Q6_K = 14   /* 256 values, 210 bytes: 128 B low nibbles, 64 B high
+                      2-bit pairs, 16 x int8 scales, fp16 d                   */
+} kq_type;
+
+typedef enum {
+    KQ_OK = 0,
+    KQ_ERR_INVALID_ARG = 1,   /* bad size, null pointer, bad capacity       */
+    KQ_ERR_UNSUPPORTED = 2,   /* unknown codec id                           */
+    KQ_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned           */
+    KQ_ERR_CUDA = 4,          /* a CUDA runtime call failed                 */
+    KQ_ERR_DEVICE_DATA = 5    /* reserved for device-side data errors       */
+} kq_status;
+
+/* Bits the kernels OR into a caller's int32 device error word (err_flag).
+ * The caller zeroes the word before the call and reads it afterwards. */
+#define KQ_DEV_BAD_EXPERT   0x1   /* tile or routing id >= n_experts           */
+#define KQ_DEV_BAD_ROWS     0x2   /* tile num_rows == 0 or > 64                */
+#define KQ_DEV_BAD_RANGE    0x4   /* tile rows past `rows`, count > cap        */
+#define KQ_DEV_UNSORTED     0x8   /* expert ids not ascending                  */
+#define KQ_DEV_TIMEOUT      0x10  /* a bounded pipeline wait ran out            */
+#define KQ_DEV_TOO_MANY     0x20  /* more tiles for one expert than supported   */
+#define KQ_DEV_X_RANGE      0x40  /* an activation is outside the binary16 range */
+
+/* Block geometry of a codec (host only).  Returns KQ_OK or
+ * KQ_ERR_UNSUPPORTED.  Source: mlx-kquant README, "Codec reference" table. */
+int kq_block_info(int type, int* values_per_block, int* bytes_per_block);
+
+/* Static, thread-safe description of a kq_status value. */
+const char* kq_status_string(int status);
+
+/* cudaError_t of the most recent KQ_ERR_CUDA on the calling host thread. */
+int kq_last_cuda_error(void);
+
+/* Library-wide device status word: bits KQ_DEV_* set by kernels that have no
+ * err_flag argument (kq_qmv, kq_qmm).  Host call, synchronous: it waits for
+ * the device.  `clear` != 0 resets the word after reading. */
+int kq_read_device_status(int32_t* host_status, int clear);
+
+/*
+ * kq_dequantize - decode wire bytes to fp32, bit-exactly.
+ * mlx-kquant bindings.cpp, `dequantize` ("Dequantize GGUF K-quant wire bytes
+ * to a float array"); hanzo-ml quantized/mod.rs, `QTensor::dequantize`
+ * (to_float into f32).
+ *   w    [n_rows, row_bytes] wire bytes
+ *   out  [n_rows, k] fp32; element (r, c) = decode of value c of row r,
+ *        computed in fp32 as (d*sc)*q - (dmin*m) (q4_K), (d*sc)*q (q6_K),
+ *        d*q (q8_0), each operation rounded separately (no FMA).
+ * n_rows >= 0; n_rows == 0 enqueues nothing.
+ */
+int kq_dequantize(int type, const void* w, int64_t n_rows, int64_t k, float* out, void* stream);
+
+/*
+ * kq_qmv - decode-shaped product y = x . W^T for 1 <= m <= 16 rows of x.
+ * mlx-kquant bindings.cpp, `quantized_matmul` (x @ dequant(w), transpose=True);
+ * README "How it works": small row counts take a weight-read-amortizing
+ * kernel (`verify_qmv`).  Every weight byte is read once for all m rows.
+ *   w [n, row_bytes], x [m, k] bf16, y [m, n] fp32.
+ * Arithmetic: quantization codes and integer scale products are exact in the
+ * tensor-core operands, activations are rounded to binary16, accumulation is
+ * fp32.  Results are deterministic (no atomics).
+ * m outside 1..16 -> KQ_ERR_INVALID_ARG.
+ */
+int kq_qmv(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int64_t m,
+           float* y, void* stream);
+
+/*
+ * kq_qmm - prefill-shaped product y = x . W^T for any m >= 1 on the
+ * tcgen05 tensor cores: W tiles are dequantized to bf16 in shared memory,
+ * x is read as bf16, products accumulate in fp32 in tensor memory.
+ * mlx-kquant bindings.cpp `quantized_matmul`; README "Performance"
+ * (single-pass matmul on the tensor units).
+ *   w [n, row_bytes], x [m, k] bf16, y [m, n] fp32.
+ */
+int kq_qmm(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int64_t m,
+           float* y, void* stream);
+
+/*
+ * kq_moe_sort - group routed (token, slot) pairs by expert for a sorted MoE
+ * prefill: a stable counting sort by expert id, plus the row gather of x.
+ * mlx-kquant README "Performance" (sorted MoE prefill batches route to a
+ * per-expert-segment GEMM) and bindings.cpp `gather_qmm_seg` ("rows
+ * pre-sorted by expert").
+ *   topk_ids    [n_tokens, top_k] int32 expert ids, each in [0, n_experts)
+ *   x           [n_tokens, k] bf16 (may be NULL when x_sorted is NULL)
+ *   sorted_ids  [n_tokens*top_k] uint32 out: expert id of sorted row r
+ *   sorted_pair [n_tokens*top_k] int32 out: token*top_k + slot of sorted row r
+ *   x_sorted    [n_tokens*top_k, k] bf16 out (nullable): x[sorted_pair/top_k]
+ *   err_flag    int32 device word (nullable): KQ_DEV_BAD_EXPERT on bad ids
+ * Pairs with equal expert id keep (token, slot) order.  1 <= n_experts <= 256.
+ */
+int kq_moe_sort(const int32_t* topk_ids, int64_t n_tokens, int32_t top_k, int32_t n_experts,
+                const uint16_t* x, int64_t k, uint32_t* sorted_ids, int32_t* sorted_pair,
+                uint16_t* x_sorted, int32_t* err_flag, void* stream);
+
+/*
+ * kq_expert_tile_map - build the tile map of a segment-walking gather GEMM on
+ * the device, without a host round trip.
+ * mlx-kquant bindings.cpp, `expert_tile_map`: tile each expert segment of
+ * the ascending id array into 64-row tiles (expert, row_start, num_rows)
+ * where only the last tile of a segment can be partial, plus the valid-tile
+ * count.  Tile order is unspecified (here: grouped by expert, ascending).
+ * Slots past the count are left untouched.
+ *   sorted_ids [rows] uint32 ascending expert ids
+ *   map        [cap, 3] uint32 out,  count [1] uint32 out
+ *   cap must be >= ceil(rows / 64) + n_experts, else KQ_ERR_INVALID_ARG.
+ *   err_flag (nullable): KQ_DEV_BAD_EXPERT (id >= n_experts),
+ *   KQ_DEV_UNSORTED (ids not ascending; the map is then unspecified).
+ */
+int kq_expert_tile_map(const uint32_t* sorted_ids, int64_t rows, int32_t n_experts,
+                       uint32_t* map, int64_t cap, uint32_t* count, int32_t* err_flag,
+                       void* stream);
+
+/*
+ * kq_gather_qmm - MoE segment GEMM: for every valid tile (e, start, n) of the
+ * map, y[r, :] = x_sorted[r, :] . dequant(W[e])^T for start <= r < start + n.
+ * mlx-kquant bindings.cpp, `gather_qmm_seg`: "valid tiles never span experts
+ * and must cover every x row exactly once (uncovered output rows are left
+ * unwritten)"; num_rows <= 64.  Each CTA owns one (expert, 128 weight rows)
+ * pair and streams all of that expert's tiles through the tensor cores, so
+ * each expert weight tile is decoded once per pass.
+ *   w_bank [n_experts, n, row_bytes], x_sorted [rows, k] bf16,
+ *   map [cap, 3], count [1] (device), y [rows, n] fp32.
+ *   err_flag (nullable): tiles with e >= n_experts (KQ_DEV_BAD_EXPERT),
+ *   num_rows 0 or > 64 (KQ_DEV_BAD_ROWS), rows past `rows` or count > cap
+ *   (KQ_DEV_BAD_RANGE) are skipped and flagged; they never fault.
+ */
+int kq_gather_qmm(int type, const void* w_bank, int32_t n_experts, int64_t n, int64_t k,
+                  const uint16_t* x_sorted, int64_t rows, const uint32_t* map,
+                  const uint32_t* count, int64_t cap, float* y, int32_t* err_flag,
+                  void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KQ_H */

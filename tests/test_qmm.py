@@ -1,0 +1,68 @@
+"""kq_qmm (tcgen05) vs the fp64 CPU oracle:
+max |y - ref| <= 2e-2 * ||x_row|| * ||w_row|| / sqrt(K)."""
+import numpy as np
+import pytest
+import torch
+
+import gguf_quant_dequant_q4_b200 as kq
+import oracle
+import synth
+from tests._util import check_qmm, dev_bf16, dev_u8, row_norms_w, row_norms_x
+
+pytestmark = pytest.mark.gpu
+CODECS = [kq.Q4_K, kq.Q6_K, kq.Q8_0]
+
+
+def run_full(qtype, n, k, m, seed=0):
+    w = synth.weights(qtype, n, k, seed=seed)
+    x = synth.activations(m, k, seed=seed + 1)
+    y = kq.qmm(dev_bf16(x), dev_u8(w), qtype).cpu().numpy()
+    ref = oracle.matmul(qtype, w, k, x)
+    return check_qmm(y, ref, row_norms_x(x), row_norms_w(qtype, w, k), k)
+
+
+@pytest.mark.parametrize("qtype", CODECS)
+@pytest.mark.parametrize("m,n", [(1, 128), (16, 130), (300, 200), (512, 384)])
+def test_small_shapes(qtype, m, n):
+    run_full(qtype, n, 2048, m, seed=m + n)
+
+
+@pytest.mark.parametrize("qtype", CODECS)
+def test_k4096_ragged(qtype):
+    run_full(qtype, 257, 4096, 513, seed=11)
+
+
+@pytest.mark.parametrize("qtype", [kq.Q4_K, kq.Q6_K])
+def test_c3_full_size_sampled(qtype):
+    m, n, k = 2048, 14336, 4096
+    w = synth.weights(qtype, n, k)
+    x = synth.activations(m, k)
+    y = kq.qmm(dev_bf16(x), dev_u8(w), qtype).cpu().numpy()
+    g = np.random.default_rng(123)
+    rows = np.sort(g.choice(m, 48, replace=False))
+    cols = np.sort(g.choice(n, 48, replace=False))
+    wn = row_norms_w(qtype, w, k)
+    xn = row_norms_x(x)
+    # all N for sampled activation rows, all M for sampled weight rows
+    ref_r = oracle.matmul(qtype, w, k, x[rows])
+    check_qmm(y[rows], ref_r, xn[rows], wn, k)
+    ref_c = oracle.matmul(qtype, w[cols], k, x)
+    check_qmm(y[:, cols], ref_c, xn, wn[cols], k)
+
+
+def test_matches_qmv_at_small_m():
+    n, k = 256, 4096
+    w = dev_u8(synth.weights(kq.Q4_K, n, k, seed=21))
+    x = dev_bf16(synth.activations(8, k, seed=22))
+    a = kq.qmm(x, w, kq.Q4_K).double()
+    b = kq.qmv(x, w, kq.Q4_K).double()
+    wn = torch.from_numpy(row_norms_w(kq.Q4_K, synth.weights(kq.Q4_K, n, k, seed=21), k)).cuda()
+    xn = x.float().norm(dim=1).double()
+    assert torch.all((a - b).abs() <= 2e-2 * xn[:, None] * wn[None, :] / np.sqrt(k))
+
+
+@pytest.mark.parametrize("qtype", CODECS)
+def test_deterministic(qtype):
+    w = dev_u8(synth.weights(qtype, 384, 2048, seed=1))
+    x = dev_bf16(synth.activations(300, 2048, seed=2))
+    assert torch.equal(kq.qmm(x, w, qtype), kq.qmm(x, w, qtype))
