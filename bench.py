@@ -476,6 +476,55 @@ def run_reference(args, dist: Dist) -> dict | None:
             "e2e": {"value": round(v, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ------------------------------------------------------------ profile cases
+CASES = ("qmv_q8_0", "qmv_q6_K", "qmv_q4_K_m1", "qmv_q4_K_m16", "dequant_q4_K", "qmm_q4_K", "qmm_q6_K",
+         "gather_q4_K")
+
+
+def run_case(name: str, iters: int) -> None:
+    """Run one kernel of the path `iters` times on its full-size workload,
+    untimed (for ncu captures: `ncu ... python bench.py --case NAME`)."""
+    import torch
+    import gguf_quant_dequant_q4_b200 as kq
+
+    dev = torch.device("cuda", 0)
+
+    def u8(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    def bf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    if name in ("qmv_q8_0", "qmv_q6_K"):
+        qt = Q8_0 if name == "qmv_q8_0" else Q6_K
+        w, x = u8(synth.weights(qt, 14336, 4096)), bf(synth.activations(1, 4096))
+        fn = lambda: kq.qmv(x, w, qt)
+    elif name.startswith("qmv_q4_K"):
+        m = 1 if name.endswith("m1") else 16
+        n, k = (4096, 4096) if m == 1 else (4096, 14336)
+        w, x = u8(synth.weights(Q4_K, n, k)), bf(synth.activations(m, k))
+        fn = lambda: kq.qmv(x, w, Q4_K)
+    elif name == "dequant_q4_K":
+        w = u8(synth.weights(Q4_K, 4096, 4096))
+        fn = lambda: kq.dequantize(w, Q4_K, 4096)
+    elif name.startswith("qmm"):
+        qt = Q4_K if name == "qmm_q4_K" else Q6_K
+        w, x = u8(synth.weights(qt, 14336, 4096)), bf(synth.activations(2048, 4096))
+        fn = lambda: kq.qmm(x, w, qt)
+    elif name == "gather_q4_K":
+        wb = u8(synth.weights(Q4_K, 14336, 4096, experts=8))
+        xt = bf(synth.activations(512, 4096))
+        sids, pair, xs = kq.moe_sort(torch.from_numpy(synth.routing(512, 8, 2)).to(dev), 8, xt)
+        tmap, cnt = kq.expert_tile_map(sids, 8)
+        fn = lambda: kq.gather_qmm(xs, wb, Q4_K, tmap, cnt)
+    else:
+        raise SystemExit(f"unknown case {name}; one of {CASES}")
+    for _ in range(iters):
+        fn()
+    torch.cuda.synchronize()
+    print(json.dumps({"case": name, "iters": iters, "status": "ok"}))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -484,7 +533,12 @@ def main(argv=None):
     ap.add_argument("--impl", default="kq", choices=["kq", "reference"])
     ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--case", choices=CASES, help="run one kernel untimed (profiling)")
+    ap.add_argument("--iters", type=int, default=3)
     args = ap.parse_args(argv)
+    if args.case:
+        run_case(args.case, args.iters)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     dist = Dist()

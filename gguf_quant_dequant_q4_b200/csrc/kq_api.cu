@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdlib>
 
 #include "../../include/kq.h"
 #include "kq_launch.h"
@@ -54,6 +55,14 @@ int record_cuda(cudaError_t e) {
 }
 
 int check_launch() { return record_cuda(cudaGetLastError()); }
+
+bool use_pdl() {
+    static const bool on = [] {
+        const char* v = std::getenv("KQ_NO_PDL");
+        return !(v && v[0] == '1');
+    }();
+    return on;
+}
 
 int device_sm_count() {
     const int d = current_device();

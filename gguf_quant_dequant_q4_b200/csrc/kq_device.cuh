@@ -16,11 +16,14 @@
 
 namespace kq {
 
-// Upper bound on the spin iterations of any wait on an mbarrier.  Each
-// iteration of try_wait already blocks for a hardware-defined interval, so
-// this bounds a wait at well over a second; a wait that runs out sets
-// KQ_DEV_TIMEOUT in the status word and the kernel winds down.
-constexpr uint32_t kSpinLimit = 1u << 24;
+// Upper bound on any wait on an mbarrier, in nanoseconds of %globaltimer.  A
+// wait that runs out sets KQ_DEV_TIMEOUT in the status word and the kernel
+// winds down instead of hanging.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Suspend-time hint of a blocking try_wait: the waiting thread sleeps until
+// the phase completes (or this many ns pass) instead of spinning, so warps
+// that wait do not take issue slots from warps that work.
+constexpr uint32_t kSuspendHintNs = 100000;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -59,11 +62,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
 // Bounded wait for the phase with the given parity to complete.  Returns
-// false (after recording KQ_DEV_TIMEOUT) if the spin limit is reached.
+// false (after recording KQ_DEV_TIMEOUT) once kWaitLimitNs have passed.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity)) return true;
+        if (global_ns() - t0 > kWaitLimitNs) break;
+    }
     if (status) atomicOr(status, KQ_DEV_TIMEOUT);
     return false;
 }

@@ -15,6 +15,9 @@ int device_smem_optin();
 // Records the launch error (if any) and maps it to a kq_status.
 int check_launch();
 int record_cuda(cudaError_t e);
+// Whether kernels are launched with programmatic dependent launch (PDL):
+// on unless the environment sets KQ_NO_PDL=1 (an A/B lever).
+bool use_pdl();
 // Device address of the library-wide status word (bits KQ_DEV_*).
 int* device_status_ptr();
 

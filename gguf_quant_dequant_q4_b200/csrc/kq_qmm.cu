@@ -16,9 +16,9 @@
 //               128B-swizzled, one 64-row box per map tile)
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
 //   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator, masked stores
-//   warps 6..13 decoders: wire bytes -> bf16 A tile in the 128B-swizzled
+//   warps 6..21 decoders: wire bytes -> bf16 A tile in the 128B-swizzled
 //               K-major layout the tensor core reads (thread = one row and
-//               one 32-value half of the 64-value step)
+//               one 16-value quarter of the 64-value step)
 // Accumulators are double-buffered in TMEM (2 x 256 columns) so the epilogue
 // of one tile overlaps the main loop of the next.  All waits are bounded; a
 // wait that runs out sets KQ_DEV_TIMEOUT and the CTA winds down, freeing its
@@ -31,7 +31,8 @@
 namespace kq {
 namespace {
 
-constexpr int kThreads = 14 * 32;
+constexpr int kDecWarps = 16;    // decoder warps (thread = row x 16-value part)
+constexpr int kThreads = (6 + kDecWarps) * 32;
 constexpr int kBM = 128;          // weight rows per tile (MMA M)
 constexpr int kBN = 256;          // activation rows per tile (MMA N max)
 constexpr int kBK = 64;           // K per pipeline step (one 128-byte swizzle row)
@@ -179,20 +180,29 @@ __device__ __forceinline__ void lds32B(uint32_t a, uint32_t (&w)[8]) {
     }
 }
 
-// Store 16 bf16x2 words (32 consecutive K values, logical chunks 4p..4p+3 of
-// row r) into a 128B-swizzled A stage.
-__device__ __forceinline__ void store_a(uint32_t abase, int r, int p, const uint32_t (&o)[16]) {
-    const uint32_t rowb = abase + (r >> 3) * 1024 + (r & 7) * 128;
+// 16 bytes starting O bytes after the 16-byte aligned shared address `a`, as 4
+// little-endian words (O even, compile time).
+template <int O>
+__device__ __forceinline__ void lds16B(uint32_t a, uint32_t (&w)[4]) {
+    if constexpr (O == 0) {
+        const uint4 c = lds128(a);
+        w[0] = c.x; w[1] = c.y; w[2] = c.z; w[3] = c.w;
+    } else {
+        const uint4 c0 = lds128(a), c1 = lds128(a + 16);
+        const uint32_t r[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-        const int c = 4 * p + cc;
-        sts128(rowb + ((c ^ (r & 7)) << 4), o[4 * cc], o[4 * cc + 1], o[4 * cc + 2], o[4 * cc + 3]);
+        for (int i = 0; i < 4; ++i) {
+            if constexpr ((O & 3) == 0) w[i] = r[(O >> 2) + i];
+            else w[i] = __byte_perm(r[(O >> 2) + i], r[(O >> 2) + i + 1], 0x5432);
+        }
     }
 }
 
 // ---------------------------------------------------------------- decoders
-// Each decoder turns 32 consecutive values (A step q in 0..3 of the raw
-// 256-value stage, half p) of one weight row into bf16:
+// A decoder thread owns one weight row r and one 16-value part p (0..3) of
+// every 64-value K step.  At the start of each raw stage (one 256-value block
+// row, four K steps q = 0..3) it decodes the scale terms of its four steps
+// once; each step then turns 16 wire values into 8 bf16x2 words:
 //   w = bf16( fp32(d*sc)*q - fp32(dmin*m) )  evaluated as
 //   t = q*s_lo - mm ; w = q*s_hi + t   in bf16x2 FMA (s = s_hi + s_lo exact to
 //   16 bits), so the result carries essentially one bf16 rounding.
@@ -200,76 +210,97 @@ constexpr uint32_t kB128 = 0x43004300u;   // bf16 (128, 128)
 constexpr uint32_t kB160 = 0x43204320u;   // bf16 (160, 160)
 constexpr uint32_t kMagic = 0x43434343u;
 
-// q4_K: 144-byte block; values 64q + 32p .. are nibble p of qs[32q .. 32q+31]
-// with scale/min code j = 2q + p.
-__device__ __forceinline__ void dq_q4k(uint32_t row, int q, int p, uint32_t (&o)[16]) {
+struct StageScales {
+    uint32_t hi[4], lo[4], nmm[4];
+    float d[4];
+};
+
+// q4_K: step q, part p covers values 64q + 16p .. +15: nibble p>>1 of
+// qs[32q + 16(p&1) ..], scale/min code j = 2q + (p>>1).
+__device__ __forceinline__ void q4k_scales(uint32_t row, int p, StageScales& S) {
     const uint4 h = lds128(row);
-    const int j = 2 * q + p;
-    const uint32_t s0 = h.y, s1 = h.z, s2 = h.w;   // bytes 0..3, 4..7, 8..11
-    int sc, m;
-    if (j < 4) {
-        sc = (s0 >> (8 * j)) & 63;
-        m = (s1 >> (8 * j)) & 63;
-    } else {
-        const int jj = j - 4;
-        const uint32_t b8 = (s2 >> (8 * jj)) & 0xff;
-        sc = (b8 & 15) | (((s0 >> (8 * jj + 6)) & 3) << 4);
-        m = (b8 >> 4) | (((s1 >> (8 * jj + 6)) & 3) << 4);
-    }
-    const float s = __fmul_rn(h16v(h.x & 0xffff), static_cast<float>(sc));
-    const float mm = __fmul_rn(h16v(h.x >> 16), static_cast<float>(m));
-    uint32_t shi, slo;
-    split_scale(s, shi, slo);
-    const uint32_t nmm = dup(bf16_bits(-mm));
-    const uint4 q0 = lds128(row + 16 + 32 * q), q1 = lds128(row + 32 + 32 * q);
-    const uint32_t wv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    const float d = h16v(h.x & 0xffff), dmin = h16v(h.x >> 16);
+    const int ph = p >> 1;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const uint32_t nib = p ? ((wv[i] >> 4) & 0x0F0F0F0Fu) : (wv[i] & 0x0F0F0F0Fu);
-        const uint32_t v01 = bsub2(__byte_perm(nib, kMagic, 0x5140), kB128);   // (q0, q1) exact
-        const uint32_t v23 = bsub2(__byte_perm(nib, kMagic, 0x7362), kB128);
-        o[2 * i] = bfma2(v01, shi, bfma2(v01, slo, nmm));
-        o[2 * i + 1] = bfma2(v23, shi, bfma2(v23, slo, nmm));
+    for (int q = 0; q < 4; ++q) {
+        const int j = 2 * q + ph;
+        int sc, m;
+        if (q < 2) {   // j < 4
+            sc = (h.y >> (8 * j)) & 63;
+            m = (h.z >> (8 * j)) & 63;
+        } else {
+            const int jj = j - 4;
+            const uint32_t b8 = (h.w >> (8 * jj)) & 0xff;
+            sc = (b8 & 15) | (((h.y >> (8 * jj + 6)) & 3) << 4);
+            m = (b8 >> 4) | (((h.z >> (8 * jj + 6)) & 3) << 4);
+        }
+        split_scale(__fmul_rn(d, static_cast<float>(sc)), S.hi[q], S.lo[q]);
+        S.nmm[q] = dup(bf16_bits(-__fmul_rn(dmin, static_cast<float>(m))));
     }
 }
 
-// q6_K: 210-byte block starting O bytes into the staged row.  Values
-// 64q + 32p + l (l = 0..31) are h = q/2, quarter tq = 2(q&1) + p: low 4 bits
-// nibble tq>>1 of ql[64h + 32(tq&1) + l], high 2 bits bits 2tq of qh[32h + l],
-// scale sc[8h + 2tq + l/16].  y = fp32(d*sc) * (code - 32).
-template <int O>
-__device__ __forceinline__ void dq_q6k(uint32_t row, int q, int p, uint32_t (&o)[16]) {
-    const int h = q >> 1, tq = 2 * (q & 1) + p;
-    uint32_t QL[8], QH[8];
-    lds32B<O>(row + 64 * h + 32 * (tq & 1), QL);
-    lds32B<O>(row + 128 + 32 * h, QH);
-    const uint32_t scw = ldsu16(row + O + 192 + 8 * h + 2 * tq);
-    const float d = h16v(ldsu16(row + O + 208));
-    uint32_t shi[2], slo[2];
-    split_scale(__fmul_rn(d, static_cast<float>(static_cast<int8_t>(scw & 0xff))), shi[0], slo[0]);
-    split_scale(__fmul_rn(d, static_cast<float>(static_cast<int8_t>(scw >> 8))), shi[1], slo[1]);
-    const int lsh = 4 * (tq >> 1), hsh = 2 * tq;
+__device__ __forceinline__ void q4k_step(uint32_t row, int q, int p, const StageScales& S, uint32_t (&o)[8]) {
+    const uint4 c = lds128(row + 16 + 32 * q + 16 * (p & 1));
+    const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
+    const uint32_t hi = S.hi[q], lo = S.lo[q], nmm = S.nmm[q];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t nib = (p >> 1) ? ((wv[i] >> 4) & 0x0F0F0F0Fu) : (wv[i] & 0x0F0F0F0Fu);
+        const uint32_t v01 = bsub2(__byte_perm(nib, kMagic, 0x5140), kB128);   // (q0, q1) exact
+        const uint32_t v23 = bsub2(__byte_perm(nib, kMagic, 0x7362), kB128);
+        o[2 * i] = bfma2(v01, hi, bfma2(v01, lo, nmm));
+        o[2 * i + 1] = bfma2(v23, hi, bfma2(v23, lo, nmm));
+    }
+}
+
+// q6_K (block at byte O of the staged row): step q, part p covers
+// h = q/2, quarter tq = 2(q&1) + (p>>1), l = 16(p&1) .. +15; low 4 bits nibble
+// tq>>1 of ql[64h + 32(tq&1) + l], high 2 bits bits 2tq of qh[32h + l],
+// scale sc[8h + 2tq + (p&1)].  y = fp32(d*sc) * (code - 32).
+template <int O>
+__device__ __forceinline__ void q6k_scales(uint32_t row, int p, StageScales& S) {
+    const float d = h16v(ldsu16(row + O + 208));
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int h = q >> 1, tq = 2 * (q & 1) + (p >> 1);
+        int16_t scv;
+        asm volatile("ld.shared.s8 %0, [%1];" : "=h"(scv) : "r"(row + O + 192 + 8 * h + 2 * tq + (p & 1)));
+        split_scale(__fmul_rn(d, static_cast<float>(scv)), S.hi[q], S.lo[q]);
+    }
+}
+
+template <int O>
+__device__ __forceinline__ void q6k_step(uint32_t row, int q, int p, const StageScales& S, uint32_t (&o)[8]) {
+    const int h = q >> 1, tq = 2 * (q & 1) + (p >> 1), sb = p & 1;
+    uint32_t QL[4], QH[4];
+    lds16B<O>(row + 64 * h + 32 * (tq & 1) + 16 * sb, QL);
+    lds16B<O>(row + 128 + 32 * h + 16 * sb, QH);
+    const int lsh = 4 * (tq >> 1), hsh = 2 * tq;
+    const uint32_t hi = S.hi[q], lo = S.lo[q];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
         const uint32_t c4 = ((QL[i] >> lsh) & 0x0F0F0F0Fu) | (((QH[i] >> hsh) & 0x03030303u) << 4);
         const uint32_t v01 = bsub2(__byte_perm(c4, kMagic, 0x5140), kB160);   // code - 32, exact
         const uint32_t v23 = bsub2(__byte_perm(c4, kMagic, 0x7362), kB160);
-        const int sb = i >> 2;
-        o[2 * i] = bfma2(v01, shi[sb], bmul2(v01, slo[sb]));
-        o[2 * i + 1] = bfma2(v23, shi[sb], bmul2(v23, slo[sb]));
+        o[2 * i] = bfma2(v01, hi, bmul2(v01, lo));
+        o[2 * i + 1] = bfma2(v23, hi, bmul2(v23, lo));
     }
 }
 
-// q8_0: block BI (0..7) of the 272-byte stage row; qs starts 34*BI + 2.
-// y = fp32(d*q) rounded to bf16.
-template <int BI>
-__device__ __forceinline__ void dq_q8(uint32_t row, uint32_t (&o)[16]) {
-    constexpr int L = 34 * BI + 2;
-    uint32_t QW[8];
-    lds32B<(L & 15)>(row + (L & ~15), QW);
-    const float d = h16v(ldsu16(row + 34 * BI));
+// q8_0 (eight 34-byte blocks per staged row): step q, part p covers block
+// bi = 2q + (p>>1), codes 16(p&1) .. +15.  y = fp32(d*q) rounded to bf16.
+__device__ __forceinline__ void q8_scales(uint32_t row, int p, StageScales& S) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int q = 0; q < 4; ++q) S.d[q] = h16v(ldsu16(row + 34 * (2 * q + (p >> 1))));
+}
+
+template <int BI, int SB>
+__device__ __forceinline__ void q8_step(uint32_t row, float d, uint32_t (&o)[8]) {
+    constexpr int L = 34 * BI + 2 + 16 * SB;
+    uint32_t QW[4];
+    lds16B<(L & 15)>(row + (L & ~15), QW);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
         const uint32_t u = QW[i] ^ 0x80808080u;   // q + 128
         float f[4];
 #pragma unroll
@@ -283,30 +314,60 @@ __device__ __forceinline__ void dq_q8(uint32_t row, uint32_t (&o)[16]) {
 }
 
 template <int QT>
-__device__ __forceinline__ void decode_step(uint32_t row, int q, int p, int o6, uint32_t (&o)[16]) {
+__device__ __forceinline__ void prep_scales(uint32_t row, int p, int o6, StageScales& S) {
     if constexpr (QT == KQ_Q4_K) {
-        dq_q4k(row, q, p, o);
+        q4k_scales(row, p, S);
     } else if constexpr (QT == KQ_Q6_K) {
         switch (o6) {
-        case 0: dq_q6k<0>(row, q, p, o); break;
-        case 2: dq_q6k<2>(row, q, p, o); break;
-        case 4: dq_q6k<4>(row, q, p, o); break;
-        case 6: dq_q6k<6>(row, q, p, o); break;
-        case 8: dq_q6k<8>(row, q, p, o); break;
-        case 10: dq_q6k<10>(row, q, p, o); break;
-        case 12: dq_q6k<12>(row, q, p, o); break;
-        default: dq_q6k<14>(row, q, p, o); break;
+        case 0: q6k_scales<0>(row, p, S); break;
+        case 2: q6k_scales<2>(row, p, S); break;
+        case 4: q6k_scales<4>(row, p, S); break;
+        case 6: q6k_scales<6>(row, p, S); break;
+        case 8: q6k_scales<8>(row, p, S); break;
+        case 10: q6k_scales<10>(row, p, S); break;
+        case 12: q6k_scales<12>(row, p, S); break;
+        default: q6k_scales<14>(row, p, S); break;
         }
     } else {
-        switch (2 * q + p) {
-        case 0: dq_q8<0>(row, o); break;
-        case 1: dq_q8<1>(row, o); break;
-        case 2: dq_q8<2>(row, o); break;
-        case 3: dq_q8<3>(row, o); break;
-        case 4: dq_q8<4>(row, o); break;
-        case 5: dq_q8<5>(row, o); break;
-        case 6: dq_q8<6>(row, o); break;
-        default: dq_q8<7>(row, o); break;
+        q8_scales(row, p, S);
+    }
+}
+
+template <int QT>
+__device__ __forceinline__ void decode_step(uint32_t row, int q, int p, int o6, const StageScales& S,
+                                            uint32_t (&o)[8]) {
+    if constexpr (QT == KQ_Q4_K) {
+        q4k_step(row, q, p, S, o);
+    } else if constexpr (QT == KQ_Q6_K) {
+        switch (o6) {
+        case 0: q6k_step<0>(row, q, p, S, o); break;
+        case 2: q6k_step<2>(row, q, p, S, o); break;
+        case 4: q6k_step<4>(row, q, p, S, o); break;
+        case 6: q6k_step<6>(row, q, p, S, o); break;
+        case 8: q6k_step<8>(row, q, p, S, o); break;
+        case 10: q6k_step<10>(row, q, p, S, o); break;
+        case 12: q6k_step<12>(row, q, p, S, o); break;
+        default: q6k_step<14>(row, q, p, S, o); break;
+        }
+    } else {
+        const float d = S.d[q];
+        switch (4 * q + p) {
+        case 0: q8_step<0, 0>(row, d, o); break;
+        case 1: q8_step<0, 1>(row, d, o); break;
+        case 2: q8_step<1, 0>(row, d, o); break;
+        case 3: q8_step<1, 1>(row, d, o); break;
+        case 4: q8_step<2, 0>(row, d, o); break;
+        case 5: q8_step<2, 1>(row, d, o); break;
+        case 6: q8_step<3, 0>(row, d, o); break;
+        case 7: q8_step<3, 1>(row, d, o); break;
+        case 8: q8_step<4, 0>(row, d, o); break;
+        case 9: q8_step<4, 1>(row, d, o); break;
+        case 10: q8_step<5, 0>(row, d, o); break;
+        case 11: q8_step<5, 1>(row, d, o); break;
+        case 12: q8_step<6, 0>(row, d, o); break;
+        case 13: q8_step<6, 1>(row, d, o); break;
+        case 14: q8_step<7, 0>(row, d, o); break;
+        default: q8_step<7, 1>(row, d, o); break;
         }
     }
 }
@@ -366,12 +427,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&raw_full[i], 1);
-            mbar_init(&raw_empty[i], 8);
+            mbar_init(&raw_empty[i], kDecWarps);
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_empty[i], 4);
         }
         for (int i = 0; i < AST; ++i) {
-            mbar_init(&a_full[i], 8);
+            mbar_init(&a_full[i], kDecWarps);
             mbar_init(&a_empty[i], 1);
         }
         for (int i = 0; i < kBStages; ++i) {
@@ -601,33 +662,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------ decoders
-        const int dt = tid - kDeqWarp0 * 32;   // 0..255
+        const int dt = tid - kDeqWarp0 * 32;   // 0..511
         const int r = dt & 127, part = dt >> 7;
+        // swizzled offsets of the thread's two 16-byte chunks (2p, 2p+1) in an A stage
+        const uint32_t rowb = (r >> 3) * 1024 + (r & 7) * 128;
+        const uint32_t so0 = rowb + (((2 * part) ^ (r & 7)) << 4), so1 = rowb + (((2 * part + 1) ^ (r & 7)) << 4);
         Pipe rp, ap;
+        StageScales S;
         for (int u = blockIdx.x; u < total_units && !aborted(); u += gridDim.x) {
             bool ok = true;
-            for (int ks = 0; ks < ksteps; ++ks) {
-                if ((ks & 3) == 0 && !bwait(&raw_full[rp.idx], rp.phase)) {
-                    ok = false;
-                    break;
-                }
-                if (!bwait(&a_empty[ap.idx], ap.phase ^ 1)) {
-                    ok = false;
-                    break;
-                }
-                uint32_t o[16];
+            for (int ks0 = 0; ks0 < ksteps && ok; ks0 += 4) {
                 const uint32_t row = rst + rp.idx * kRawBytes + r * C::RAWB;
-                const int o6 = QT == KQ_Q6_K ? (210 * (ks >> 2)) & 15 : 0;
-                decode_step<QT>(row, ks & 3, part, o6, o);
-                store_a(ast + ap.idx * kABytes, r, part, o);
-                fence_proxy_async();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&a_full[ap.idx]);
-                ap.next(AST);
-                if ((ks & 3) == 3) {
-                    if (lane == 0) mbar_arrive(&raw_empty[rp.idx]);
-                    rp.next(kRawStages);
+                const int o6 = QT == KQ_Q6_K ? (210 * (ks0 >> 2)) & 15 : 0;
+                if (!bwait(&raw_full[rp.idx], rp.phase)) {
+                    ok = false;
+                    break;
                 }
+                prep_scales<QT>(row, part, o6, S);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (!bwait(&a_empty[ap.idx], ap.phase ^ 1)) {
+                        ok = false;
+                        break;
+                    }
+                    uint32_t o[8];
+                    decode_step<QT>(row, q, part, o6, S, o);
+                    const uint32_t ab = ast + ap.idx * kABytes;
+                    sts128(ab + so0, o[0], o[1], o[2], o[3]);
+                    sts128(ab + so1, o[4], o[5], o[6], o[7]);
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&a_full[ap.idx]);
+                    ap.next(AST);
+                }
+                if (!ok) break;
+                if (lane == 0) mbar_arrive(&raw_empty[rp.idx]);
+                rp.next(kRawStages);
             }
             if (!ok) break;
         }

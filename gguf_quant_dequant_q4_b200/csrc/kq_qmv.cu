@@ -40,22 +40,28 @@
 namespace kq {
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = 32 * kWarps;
+constexpr int kCWarps = 16;                 // consumer warps
+constexpr int kProducerWarp = kCWarps;      // bulk-copy producer
+constexpr int kReducerWarp = kCWarps + 1;   // cross-warp reduction and stores
+constexpr int kThreads = 32 * (kCWarps + 2);
 constexpr int kRows = 16;
-constexpr int kOffW = 128;   // barriers, abort flag and a zero word live below
+constexpr int kOffW = 384;   // barriers, flags and a zero word live below
+constexpr int kMaxStages = 8;
 
 template <int QT> struct Codec;
+// Stage geometry is chosen per call: a stage is 16 rows x g blocks, g a
+// multiple of GA (so every per-row copy starts 16-byte aligned), as large as
+// shared memory allows; rows are padded to a stride of 16 mod 128 bytes.
 template <> struct Codec<KQ_Q4_K> {
-    static constexpr int VPB = 256, BPB = 144, G = 8, RS = 1168;  // RS = 16 mod 128
+    static constexpr int VPB = 256, BPB = 144, GA = 8;
     static constexpr int IMG = 544, XS = 0;   // B image bytes / fp32 sums per (token, block)
 };
 template <> struct Codec<KQ_Q6_K> {
-    static constexpr int VPB = 256, BPB = 210, G = 8, RS = 1680;
+    static constexpr int VPB = 256, BPB = 210, GA = 8;
     static constexpr int IMG = 1024, XS = 16;
 };
 template <> struct Codec<KQ_Q8_0> {
-    static constexpr int VPB = 32, BPB = 34, G = 64, RS = 2192;
+    static constexpr int VPB = 32, BPB = 34, GA = 8;
     static constexpr int IMG = 64, XS = 1;
 };
 
@@ -65,8 +71,8 @@ struct QmvParams {
     float* y;
     int* status;
     int64_t n, k, row_bytes;
-    int m, nblk, scb, ns, bulk;
-    uint32_t tokstride, off_img, off_x;
+    int m, nblk, scb, ns, bulk, g, rs;
+    uint32_t tokstride, off_img, off_x, off_pbuf, off_racc;
 };
 
 // binary16 constants
@@ -122,7 +128,7 @@ __device__ void build_image(const QmvParams& p, int blk0, int nb, uint32_t img, 
 template <>
 __device__ void build_image<KQ_Q4_K>(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t, float& amax) {
     const int items = p.m * nb * 4;
-    for (int it = threadIdx.x; it < items; it += kThreads) {
+    for (int it = threadIdx.x; it < items; it += kCWarps * 32) {
         const int m = it / (nb * 4), rem = it % (nb * 4), bl = rem >> 2, t = rem & 3;
         const uint16_t* xs = p.x + static_cast<int64_t>(m) * p.k + static_cast<int64_t>(blk0 + bl) * 256 + 64 * t;
         const uint32_t base = img + m * p.tokstride + bl * 544;
@@ -161,7 +167,7 @@ __device__ void build_image<KQ_Q4_K>(const QmvParams& p, int blk0, int nb, uint3
 template <>
 __device__ void build_image<KQ_Q8_0>(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t xsum, float& amax) {
     const int items = p.m * nb;
-    for (int it = threadIdx.x; it < items; it += kThreads) {
+    for (int it = threadIdx.x; it < items; it += kCWarps * 32) {
         const int m = it / nb, bl = it % nb;
         const uint16_t* xs = p.x + static_cast<int64_t>(m) * p.k + static_cast<int64_t>(blk0 + bl) * 32;
         const uint32_t base = img + m * p.tokstride + bl * 64;
@@ -185,15 +191,15 @@ __device__ void build_image<KQ_Q8_0>(const QmvParams& p, int blk0, int nb, uint3
 
 // q6_K: sub-block j (16 values, j = 8h + 2tq + u) has a low-code MMA and a
 // high-code MMA; lane t uses values 16j + 4t + {0,2 | 1,3}.  The low-code B
-// is x (tq < 2) or x/16 (tq >= 2, where the code sits in the high nibble);
-// the high-code B is x (tq < 3) or x/4 (tq = 3).  X_j = sum of 16 values.
+// is x/16 (tq < 2) or x/256 (tq >= 2, where the code sits in the high
+// nibble); the high-code B is x / 4^tq.  X_j = sum of the 16 values.
 template <>
 __device__ void build_image<KQ_Q6_K>(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t xsum, float& amax) {
     const int items = p.m * nb * 16;
-    for (int it = threadIdx.x; it < items; it += kThreads) {
+    for (int it = threadIdx.x; it < items; it += kCWarps * 32) {
         const int m = it / (nb * 16), rem = it % (nb * 16), bl = rem >> 4, j = rem & 15;
         const int tq = (j & 7) >> 1;
-        const float slo = tq < 2 ? 1.0f : 0.0625f, shi = tq < 3 ? 1.0f : 0.25f;
+        const float slo = tq < 2 ? 0.0625f : 0.00390625f, shi = 1.0f / static_cast<float>(1 << (2 * tq));
         const uint16_t* xs = p.x + static_cast<int64_t>(m) * p.k + static_cast<int64_t>(blk0 + bl) * 256 + 16 * j;
         const uint32_t base = img + m * p.tokstride + bl * 1024 + j * 64;
         const uint4 r0 = ldg_nc_v4(xs), r1 = ldg_nc_v4(xs + 8);
@@ -220,6 +226,7 @@ struct Lane {
     int g, t;
     uint32_t tokb[NT];   // image base of the lane's B column (token) per n-tile
     int tok[NT];         // token index (clamped) of that column
+    uint32_t bmask[8];   // slot variants: (1, 1) in binary16 if the lane's column has slot s, else 0
 };
 
 // q4_K, one superblock of 16 rows.  rowA/rowB: shared address of the block in
@@ -320,17 +327,17 @@ __device__ __forceinline__ void col_info(int nt, int col, int m, int& tok, int& 
     tok = tok < m ? tok : m - 1;
 }
 
-// q8_0: the warp's run of up to 8 consecutive 32-value blocks of one stage.
+// q8_0: the warp's run of up to RUN consecutive 32-value blocks of one stage.
 // rowA/rowB: shared address of row g / g+8 of the stage; lb0: first local
 // block; nvalid: blocks present; imgb0 / xsb0: image/X offsets of lb0.
-template <int S, int NT>
+template <int S, int NT, int RUN>
 __device__ __forceinline__ void q8_run(const Lane<NT>& L, const QmvParams& p, uint32_t rowA, uint32_t rowB, int lb0,
                                        int nvalid, uint32_t imgb0, uint32_t xsb0, uint32_t zero_addr,
                                        float (&acc)[NT][4]) {
     const int t = L.t;
     float D[NT][4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < RUN; ++i) {
         if (i % S == 0) {
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
@@ -353,14 +360,16 @@ __device__ __forceinline__ void q8_run(const Lane<NT>& L, const QmvParams& p, ui
                 const uint32_t A3 = and_xor(wb >> 8, 0x00FF00FFu, 0x64806480u);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    uint32_t addr = L.tokb[nt] + imgb0 + i * 64 + h * 32 + t * 8;
-                    if (S > 1 && (L.g % S) != (i % S)) addr = zero_addr;
-                    const uint2 bv = lds64c(addr);
+                    uint2 bv = lds64c(L.tokb[nt] + imgb0 + i * 64 + h * 32 + t * 8);
+                    if (S > 1) {   // only the columns of this block's slot see its activations
+                        bv.x = hmul2_u32(bv.x, L.bmask[i % S]);
+                        bv.y = hmul2_u32(bv.y, L.bmask[i % S]);
+                    }
                     mma_f16(D[nt], A0, A1, A2, A3, bv.x, bv.y);
                 }
             }
         }
-        if (i % S == S - 1 || i == 7) {
+        if (i % S == S - 1 || i == RUN - 1) {
             // epilogue: y += d * (D - 1152 X) per column's block
             const int i0 = i - (i % S);
 #pragma unroll
@@ -382,69 +391,67 @@ __device__ __forceinline__ void q8_run(const Lane<NT>& L, const QmvParams& p, ui
     }
 }
 
-// q6_K: one 256-value block of 16 rows; sub-blocks in order j = 8h + 2tq + u.
+// q6_K: half h (sub-blocks j = 8h + 2tq + u, 128 values) of one 256-value
+// block of 16 rows.  Two warps share a block, one half each.
 template <int S, int NT>
-__device__ __forceinline__ void q6k_block(const Lane<NT>& L, const QmvParams& p, uint32_t rowA, uint32_t rowB,
-                                          bool odd, uint32_t imgb, uint32_t xsb, uint32_t zero_addr,
-                                          float (&acc)[NT][4]) {
+__device__ __forceinline__ void q6k_half(const Lane<NT>& L, const QmvParams& p, uint32_t rowA, uint32_t rowB,
+                                         bool odd, int h, uint32_t imgb, uint32_t xsb, uint32_t zero_addr,
+                                         float (&acc)[NT][4]) {
     const int t = L.t;
     const float dA = h16(ldsu16c(rowA + 208));
     const float dB = h16(ldsu16c(rowB + 208));
     // the lane's 4-byte pieces: ql[h][pp][u] and qh[h][u] for rows g and g+8
-    uint32_t QLA[8], QLB[8], QHA[4], QHB[4];
+    uint32_t QLA[4], QLB[4], QHA[2], QHB[2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const uint32_t o = 64 * (i >> 2) + 32 * ((i >> 1) & 1) + 16 * (i & 1) + 4 * t;
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t o = 64 * h + 32 * (i >> 1) + 16 * (i & 1) + 4 * t;
         QLA[i] = lds32c_a2(rowA + o, odd);
         QLB[i] = lds32c_a2(rowB + o, odd);
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t o = 128 + 32 * (i >> 1) + 16 * (i & 1) + 4 * t;
+    for (int i = 0; i < 2; ++i) {
+        const uint32_t o = 128 + 32 * h + 16 * i + 4 * t;
         QHA[i] = lds32c_a2(rowA + o, odd);
         QHB[i] = lds32c_a2(rowB + o, odd);
     }
     float D[NT][4];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        const int h = j >> 3, tq = (j & 7) >> 1, u = j & 1, pp = tq & 1;
-        if (j % S == 0) {
+    for (int jl = 0; jl < 8; ++jl) {
+        const int tq = jl >> 1, u = jl & 1, pp = tq & 1;
+        const int j = 8 * h + jl;
+        if (jl % S == 0) {
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) D[nt][e] = 0.f;
         }
-        const uint32_t la = QLA[4 * h + 2 * pp + u], lb = QLB[4 * h + 2 * pp + u];
-        const uint32_t ha = QHA[2 * h + u], hb = QHB[2 * h + u];
-        // low 4 bits: low nibble (tq < 2) -> 1024 + c, high nibble -> 1024 + 16c
+        const uint32_t la = QLA[2 * pp + u], lb = QLB[2 * pp + u];
+        const uint32_t ha = QHA[u], hb = QHB[u];
+        // low 4 bits: low nibble (tq < 2) -> 1024 + c with B = x/16, high
+        // nibble (tq >= 2) -> 1024 + 16c with B = x/256
         const uint32_t mlo = tq < 2 ? 0x000F000Fu : 0x00F000F0u;
         const uint32_t L0 = and_or(la, mlo, kH1024), L1 = and_or(lb, mlo, kH1024);
         const uint32_t L2 = and_or(la >> 8, mlo, kH1024), L3 = and_or(lb >> 8, mlo, kH1024);
-        // high 2 bits (bits 2tq of each qh byte) moved to bits 4..5 (tq < 3):
-        // 1024 + 16c; tq = 3 stays at bits 6..7: 1024 + 64c with B = x/4.
-        uint32_t H0, H1, H2, H3;
-        if (tq == 3) {
-            H0 = and_or(ha, 0x00C000C0u, kH1024);
-            H1 = and_or(hb, 0x00C000C0u, kH1024);
-            H2 = and_or(ha >> 8, 0x00C000C0u, kH1024);
-            H3 = and_or(hb >> 8, 0x00C000C0u, kH1024);
-        } else {
-            const int sh = 4 - 2 * tq;   // 4, 2, 0: left shift for bytes 0/2
-            H0 = and_or(ha << sh, 0x00300030u, kH1024);
-            H1 = and_or(hb << sh, 0x00300030u, kH1024);
-            H2 = and_or(ha >> (8 - sh), 0x00300030u, kH1024);
-            H3 = and_or(hb >> (8 - sh), 0x00300030u, kH1024);
-        }
+        // high 2 bits, left at bits 2tq..2tq+1 of each byte: 1024 + 4^tq c with
+        // B = x / 4^tq (all B scalings are exact powers of two, none above 1)
+        const uint32_t mhi = 0x00030003u << (2 * tq);
+        const uint32_t H0 = and_or(ha, mhi, kH1024), H1 = and_or(hb, mhi, kH1024);
+        const uint32_t H2 = and_or(ha >> 8, mhi, kH1024), H3 = and_or(hb >> 8, mhi, kH1024);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            const bool mine = !(S > 1) || (L.g % S) == (j % S);
             const uint32_t a = L.tokb[nt] + imgb + j * 64 + t * 8;
-            const uint2 bl = lds64c(mine ? a : zero_addr);
-            const uint2 bh = lds64c(mine ? a + 32 : zero_addr);
+            uint2 bl = lds64c(a), bh = lds64c(a + 32);
+            if (S > 1) {   // only the columns of this sub-block's slot see its activations
+                const uint32_t mk = L.bmask[jl % S];
+                bl.x = hmul2_u32(bl.x, mk);
+                bl.y = hmul2_u32(bl.y, mk);
+                bh.x = hmul2_u32(bh.x, mk);
+                bh.y = hmul2_u32(bh.y, mk);
+            }
             mma_f16(D[nt], L0, L1, L2, L3, bl.x, bl.y);
             mma_f16(D[nt], H0, H1, H2, H3, bh.x, bh.y);
         }
-        if (j % S == S - 1) {
+        if (jl % S == S - 1) {
             const int j0 = j - (S - 1);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
@@ -454,12 +461,13 @@ __device__ __forceinline__ void q6k_block(const Lane<NT>& L, const QmvParams& p,
                     col_info<S, NT>(nt, 2 * t + (e & 1), p.m, tok, slot);
                     const int jj = j0 + slot;
                     const int tqj = (jj & 7) >> 1;
-                    // bias of the two MMAs: 1024/sigma_lo + 1024/sigma_hi' + 32
-                    const float C = tqj < 2 ? 2080.0f : (tqj == 2 ? 1120.0f : 352.0f);
+                    // D = (sum c x)/16 + bias X with bias = 1024/sigma_lo + 1024/4^tq;
+                    // sum (c - 32) x = 16 (D - (bias + 2) X)
+                    const float C = tqj == 0 ? 1090.0f : (tqj == 1 ? 322.0f : (tqj == 2 ? 70.0f : 22.0f));
                     const uint32_t row = (e >> 1) ? rowB : rowA;
                     const float dr = (e >> 1) ? dB : dA;
                     const int sc = ldss8c(row + 192 + jj);
-                    const float s = __fmul_rn(dr, static_cast<float>(sc));
+                    const float s = 16.0f * __fmul_rn(dr, static_cast<float>(sc));
                     const float X = ldsf32c(xsb + (tok * p.scb * 16 + jj) * 4);
                     acc[nt][e] = fmaf(s, fmaf(-C, X, D[nt][e]), acc[nt][e]);
                 }
@@ -472,143 +480,232 @@ template <int QT, int S, int NT>
 __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const QmvParams p) {
     using C = Codec<QT>;
     extern __shared__ __align__(1024) uint8_t smem[];
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 64);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);           // [kMaxStages]
+    uint64_t* empty = full + kMaxStages;                           // [kMaxStages]
+    uint64_t* red_full = full + 2 * kMaxStages;                    // [2]
+    uint64_t* red_empty = full + 2 * kMaxStages + 2;               // [2]
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 256);
+    volatile int* consumed = reinterpret_cast<volatile int*>(smem + 260);
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t zero_addr = sbase + 96;
+    const uint32_t zero_addr = sbase + 272;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRows;
-    const int rows_valid = static_cast<int>(p.n - row0 < kRows ? p.n - row0 : kRows);
-    const int nstages = cdiv(p.nblk, C::G);
-    const int spsc = p.scb / C::G;
+    // balanced contiguous row range of this CTA
+    const int64_t r0 = static_cast<int64_t>(blockIdx.x) * p.n / gridDim.x;
+    const int64_t r1 = static_cast<int64_t>(blockIdx.x + 1) * p.n / gridDim.x;
+    const int nrg = static_cast<int>((r1 - r0 + kRows - 1) / kRows);
+    const int nsc = cdiv(p.nblk, p.scb);
 
     if (tid == 0) {
-        for (int i = 0; i < p.ns; ++i) mbar_init(&full[i], 1);
+        for (int i = 0; i < p.ns; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], QT == KQ_Q4_K ? kCWarps / 2 : kCWarps);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&red_full[i], kCWarps);
+            mbar_init(&red_empty[i], 1);
+        }
         *abort_flag = 0;
+        *consumed = 0;
         fence_barrier_init();
     }
     if (tid < 4) sts32(zero_addr + 4 * tid, 0u);
+    // Programmatic dependent launch: the next kernel in the stream may start
+    // its prologue now.  This CTA's weight bytes are prefetched into L2 (a
+    // hint; L2 is coherent, so it is safe even if an earlier kernel is still
+    // writing them), then every thread waits for the earlier grids to finish
+    // before touching memory they might produce.  Without the launch
+    // attribute both instructions are no-ops.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (warp == kProducerWarp && p.bulk) {
+        const uint8_t* base = p.w + r0 * p.row_bytes;
+        const int64_t bytes = (r1 - r0) * p.row_bytes;
+        for (int64_t o = static_cast<int64_t>(lane) * 65536; o < bytes; o += 32 * 65536) {
+            const uint32_t sz = static_cast<uint32_t>(bytes - o < 65536 ? bytes - o : 65536);
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + o), "r"(sz) : "memory");
+        }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     __syncthreads();
 
-    auto stage_addr = [&](int slot) { return sbase + kOffW + slot * (kRows * C::RS); };
-    auto issue = [&](int s) {   // warp 0
-        const int slot = s % p.ns, b0 = s * C::G;
-        const int nb = p.nblk - b0 < C::G ? p.nblk - b0 : C::G;
-        const uint32_t bytes = nb * C::BPB;
-        if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes * rows_valid);
-        __syncwarp();
-        if (lane < rows_valid)
-            bulk_g2s(smem + kOffW + slot * (kRows * C::RS) + lane * C::RS,
-                     p.w + (row0 + lane) * p.row_bytes + static_cast<int64_t>(b0) * C::BPB, bytes, &full[slot]);
-    };
-    auto sync_load = [&](int s) {   // all threads; any alignment (2-byte units)
-        const int slot = s % p.ns, b0 = s * C::G;
-        const int nb = p.nblk - b0 < C::G ? p.nblk - b0 : C::G;
-        const int half = nb * C::BPB / 2;
-        const uint32_t dst = stage_addr(slot);
-        for (int i = tid; i < rows_valid * half; i += kThreads) {
-            const int r = i / half, c = i % half;
-            const unsigned short v =
-                __ldg(reinterpret_cast<const unsigned short*>(p.w + (row0 + r) * p.row_bytes +
-                                                              static_cast<int64_t>(b0) * C::BPB) + c);
-            asm volatile("st.shared.u16 [%0], %1;" ::"r"(dst + r * C::RS + 2 * c), "h"(v));
+    auto stages_in = [&](int sc) { return cdiv(min(p.scb, p.nblk - sc * p.scb), p.g); };
+    auto stage_addr = [&](int slot) { return sbase + kOffW + slot * (kRows * p.rs); };
+    auto bwait = [&](uint64_t* bar, uint32_t parity) {
+        if (*abort_flag) return false;
+        if (!mbar_wait(bar, parity, p.status)) {
+            *abort_flag = 1;
+            return false;
         }
-        __syncthreads();
+        return true;
     };
 
-    int issued = 0;
-    if (p.bulk && warp == 0)
-        for (; issued < p.ns && issued < nstages; ++issued) issue(issued);
-
-    Lane<NT> L;
-    L.g = lane >> 2;
-    L.t = lane & 3;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        int tok, slot;
-        col_info<S, NT>(nt, L.g, p.m, tok, slot);
-        L.tok[nt] = tok;
-        L.tokb[nt] = sbase + p.off_img + tok * p.tokstride;
-    }
-    float acc[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-    float amax = 0.f;
-    int s = 0;
-    for (; s < nstages; ++s) {
-        if (s % spsc == 0) {
-            const int blk0 = s * C::G;
-            const int nb = p.nblk - blk0 < p.scb ? p.nblk - blk0 : p.scb;
-            __syncthreads();
-            build_image<QT>(p, blk0, nb, sbase + p.off_img, sbase + p.off_x, amax);
-            __syncthreads();
-        }
-        const int slot = s % p.ns;
-        if (p.bulk) {
-            if (!mbar_wait(&full[slot], (s / p.ns) & 1, p.status)) *abort_flag = 1;
-        } else {
-            sync_load(s);
-        }
-        const int b0 = s * C::G;
-        const int nb = p.nblk - b0 < C::G ? p.nblk - b0 : C::G;
-        const int scbase = (s / spsc) * spsc * C::G;   // first block of the super-chunk
-        const uint32_t st = stage_addr(slot);
-        const uint32_t rowA = st + L.g * C::RS, rowB = rowA + 8 * C::RS;
-        if constexpr (QT == KQ_Q4_K) {
-            if (warp < nb) q4k_block<NT>(L, rowA + warp * 144, rowB + warp * 144, (b0 + warp - scbase) * 544, acc);
-        } else if constexpr (QT == KQ_Q6_K) {
-            if (warp < nb) {
-                const int lbi = b0 + warp - scbase;
-                q6k_block<S, NT>(L, p, rowA + warp * 210, rowB + warp * 210, (warp & 1) != 0, lbi * 1024,
-                                 sbase + p.off_x + lbi * 64, zero_addr, acc);
-            }
-        } else {
-            const int lb0 = 8 * warp;
-            if (lb0 < nb) {
-                const int nv = nb - lb0 < 8 ? nb - lb0 : 8;
-                const int lbi = b0 + lb0 - scbase;
-                q8_run<S, NT>(L, p, rowA, rowB, lb0, nv, lbi * 64, sbase + p.off_x + lbi * 4, zero_addr, acc);
+    if (warp == kProducerWarp) {
+        // ------------------------------------------------ W stage producer
+        int q = 0;   // global stage counter
+        bool ok = true;
+        for (int sc = 0; sc < nsc && ok; ++sc) {
+            const int nst = stages_in(sc);
+            for (int g = 0; g < nrg && ok; ++g) {
+                const int64_t row0 = r0 + static_cast<int64_t>(g) * kRows;
+                const int rv = static_cast<int>(r1 - row0 < kRows ? r1 - row0 : kRows);
+                for (int si = 0; si < nst; ++si, ++q) {
+                    const int slot = q % p.ns;
+                    const int b0 = sc * p.scb + si * p.g;
+                    const int nb = p.nblk - b0 < p.g ? p.nblk - b0 : p.g;
+                    const uint32_t bytes = nb * C::BPB;
+                    if (lane == 0) ok = bwait(&empty[slot], ((q / p.ns) & 1) ^ 1);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    const uint8_t* src = p.w + row0 * p.row_bytes + static_cast<int64_t>(b0) * C::BPB;
+                    if (p.bulk) {
+                        if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes * rv);
+                        __syncwarp();
+                        if (lane < rv)
+                            bulk_g2s(smem + kOffW + slot * (kRows * p.rs) + lane * p.rs, src + lane * p.row_bytes,
+                                     bytes, &full[slot]);
+                    } else {
+                        const int half = bytes / 2;
+                        const uint32_t dst = stage_addr(slot);
+                        for (int i = lane; i < rv * half; i += 32) {
+                            const int r = i / half, c = i % half;
+                            const unsigned short v =
+                                __ldg(reinterpret_cast<const unsigned short*>(src + r * p.row_bytes) + c);
+                            asm volatile("st.shared.u16 [%0], %1;" ::"r"(dst + r * p.rs + 2 * c), "h"(v));
+                        }
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&full[slot]);
+                    }
+                }
             }
         }
-        __syncthreads();
-        if (*abort_flag) break;
-        if (p.bulk && warp == 0 && issued < nstages) issue(issued++);
-    }
-    if (*abort_flag) {
-        // wind down: let every copy still in flight land before the CTA exits
-        if (warp == 0 && lane == 0)
-            for (int q = s + 1; q < issued; ++q) mbar_wait(&full[q % p.ns], (q / p.ns) & 1, nullptr);
-        __syncthreads();
-        return;
-    }
-    if (amax >= 65504.0f) atomicOr(p.status, KQ_DEV_X_RANGE);
-
-    // ---- combine the 8 warps' partial sums (fixed order) and store y
-    float* red = reinterpret_cast<float*>(smem + kOffW);   // [warp][16 rows][16 cols]
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int r = L.g + 8 * (e >> 1), c = nt * 8 + 2 * L.t + (e & 1);
-            red[(warp * 16 + r) * 16 + c] = acc[nt][e];
+        // wind down after an abort: let copies in flight land
+        if (*abort_flag && lane == 0)
+            for (int qq = *consumed; qq < q; ++qq) mbar_wait(&full[qq % p.ns], (qq / p.ns) & 1, nullptr);
+    } else if (warp == kReducerWarp) {
+        // ------------------------------------------------ cross-warp reducer
+        float* pbuf = reinterpret_cast<float*>(smem + p.off_pbuf);
+        float* racc = reinterpret_cast<float*>(smem + p.off_racc);
+        constexpr int PW = 32 * 4 * NT;   // floats per warp partial
+        int it = 0;
+        for (int sc = 0; sc < nsc; ++sc) {
+            for (int g = 0; g < nrg; ++g, ++it) {
+                const int b = it & 1;
+                if (!bwait(&red_full[b], (it >> 1) & 1)) break;
+                const int64_t row0 = r0 + static_cast<int64_t>(g) * kRows;
+                const int rv = static_cast<int>(r1 - row0 < kRows ? r1 - row0 : kRows);
+                const float* pb = pbuf + b * kCWarps * PW;
+                // outputs (token, row): 16 rows x m tokens
+                for (int o = lane; o < p.m * kRows; o += 32) {
+                    const int tok = o / kRows, r = o % kRows;
+                    float sum = 0.f;
+                    const int slots = S > 1 ? S : 1;
+                    for (int sl = 0; sl < slots; ++sl) {
+                        const int c = S > 1 ? tok * S + sl : tok;   // column within the 8 (or 16) of the tiles
+                        const int nt = c >> 3, cc = c & 7;
+                        const int ln = 4 * (r & 7) + (cc >> 1);
+                        const int e = 2 * (r >> 3) + (cc & 1);
+                        const int idx = ln * 4 * NT + nt * 4 + e;
+                        for (int w = 0; w < kCWarps; ++w) sum += pb[w * PW + idx];
+                    }
+                    float* ra = racc + (g * kRows + r) * 16 + tok;
+                    if (nsc > 1) {
+                        if (sc > 0) sum += *ra;
+                        *ra = sum;
+                    }
+                    if (sc == nsc - 1 && r < rv) p.y[static_cast<int64_t>(tok) * p.n + row0 + r] = sum;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&red_empty[b]);
+            }
+            if (*abort_flag) break;
         }
+    } else {
+        // ------------------------------------------------ consumers (16 warps)
+        Lane<NT> L;
+        L.g = lane >> 2;
+        L.t = lane & 3;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            int tok, slot;
+            col_info<S, NT>(nt, L.g, p.m, tok, slot);
+            L.tok[nt] = tok;
+            L.tokb[nt] = sbase + p.off_img + tok * p.tokstride;
+        }
+#pragma unroll
+        for (int sl = 0; sl < 8; ++sl) L.bmask[sl] = (S > 1 && (L.g % S) == sl) ? 0x3C003C00u : 0u;
+        // q4_K: two groups of 8 warps take alternate stages (a warp decodes a
+        // whole block); the other codecs share every stage among all 16 warps
+        const int grp = warp >> 3, wig = warp & 7;
+        float amax = 0.f;
+        float* pbuf = reinterpret_cast<float*>(smem + p.off_pbuf);
+        constexpr int PW = 32 * 4 * NT;
+        int q = 0, it = 0;
+        for (int sc = 0; sc < nsc && !*abort_flag; ++sc) {
+            const int blk0 = sc * p.scb;
+            const int nbsc = p.nblk - blk0 < p.scb ? p.nblk - blk0 : p.scb;
+            const int nst = stages_in(sc);
+            asm volatile("bar.sync 1, %0;" ::"r"(kCWarps * 32));
+            build_image<QT>(p, blk0, nbsc, sbase + p.off_img, sbase + p.off_x, amax);
+            asm volatile("bar.sync 1, %0;" ::"r"(kCWarps * 32));
+            for (int g = 0; g < nrg; ++g, ++it) {
+                float acc[NT][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+                bool ok = true;
+                for (int si = 0; si < nst; ++si, ++q) {
+                    const int slot = q % p.ns;
+                    if (QT == KQ_Q4_K && (q & 1) != grp) continue;
+                    if (!bwait(&full[slot], (q / p.ns) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    const int b0 = blk0 + si * p.g;
+                    const int nb = p.nblk - b0 < p.g ? p.nblk - b0 : p.g;
+                    const uint32_t st = stage_addr(slot);
+                    const uint32_t rowA = st + L.g * p.rs, rowB = rowA + 8 * p.rs;
+                    const int bl = si * p.g;   // first block of the stage within the super-chunk
+                    if constexpr (QT == KQ_Q4_K) {
+                        // group of 8 warps, a warp decodes whole blocks wig, wig + 8, ...
+                        for (int lb = wig; lb < nb; lb += 8)
+                            q4k_block<NT>(L, rowA + lb * 144, rowB + lb * 144, (bl + lb) * 544, acc);
+                    } else if constexpr (QT == KQ_Q6_K) {
+                        // half blocks: item i = (block i/2, half i%2)
+                        for (int it2 = warp; it2 < 2 * nb; it2 += kCWarps) {
+                            const int lb = it2 >> 1, lbi = bl + lb;
+                            q6k_half<S, NT>(L, p, rowA + lb * 210, rowB + lb * 210, (lb & 1) != 0, it2 & 1,
+                                            lbi * 1024, sbase + p.off_x + lbi * 64, zero_addr, acc);
+                        }
+                    } else {
+                        // runs of 4 consecutive blocks
+                        for (int lb0 = 4 * warp; lb0 < nb; lb0 += 4 * kCWarps) {
+                            const int nv = nb - lb0 < 4 ? nb - lb0 : 4;
+                            const int lbi = bl + lb0;
+                            q8_run<S, NT, 4>(L, p, rowA, rowB, lb0, nv, lbi * 64, sbase + p.off_x + lbi * 4,
+                                             zero_addr, acc);
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(&empty[slot]);
+                        if (warp == 0) *consumed = q + 1;
+                    }
+                }
+                if (!ok) break;
+                // hand the warp's partial sums of this row group to the reducer
+                const int b = it & 1;
+                if (!bwait(&red_empty[b], ((it >> 1) & 1) ^ 1)) break;
+                float* dst = pbuf + (b * kCWarps + warp) * PW + lane * 4 * NT;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    *reinterpret_cast<float4*>(dst + 4 * nt) = make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&red_full[b]);
+            }
+        }
+        if (amax >= 65504.0f) atomicOr(p.status, KQ_DEV_X_RANGE);
     }
     __syncthreads();
-    const int ntok = p.m;
-    for (int i = tid; i < ntok * kRows; i += kThreads) {
-        const int tok = i / kRows, r = i % kRows;
-        if (r >= rows_valid) continue;
-        float sum = 0.f;
-        if (S > 1) {
-            for (int w = 0; w < kWarps; ++w)
-                for (int sl = 0; sl < S; ++sl) sum += red[(w * 16 + r) * 16 + tok * S + sl];
-        } else {
-            for (int w = 0; w < kWarps; ++w) sum += red[(w * 16 + r) * 16 + tok];
-        }
-        p.y[static_cast<int64_t>(tok) * p.n + row0 + r] = sum;
-    }
 }
 
 template <int QT>
@@ -626,38 +723,87 @@ int launch_codec(const void* w, int64_t n, int64_t k, const uint16_t* x, int m, 
     p.row_bytes = static_cast<int64_t>(p.nblk) * C::BPB;
     p.bulk = (p.row_bytes % 16 == 0) && (reinterpret_cast<uintptr_t>(w) % 16 == 0);
     const int optin = device_smem_optin();
-    const int nblk_g = cdiv(p.nblk, C::G) * C::G;
-    // Choose stage count and super-chunk size (blocks whose activation image
-    // is resident at once): as many blocks as fit, a multiple of G.
-    int ns = 3, scb = 0;
-    uint32_t tokstride = 0, off_img = 0, off_x = 0, total = 0;
-    for (; ns >= 2; --ns) {
-        const uint32_t wbytes = kOffW + ns * kRows * C::RS;
-        off_img = (wbytes + 127) & ~127u;
-        for (scb = nblk_g; scb >= C::G; scb -= C::G) {
-            const uint32_t base = scb * C::IMG;
-            tokstride = base + ((32u - (base & 127u)) & 127u);
-            off_x = off_img + m * tokstride;
-            total = off_x + m * scb * C::XS * 4;
-            if (total <= static_cast<uint32_t>(optin)) break;
+    const int sms = device_sm_count();
+    // One persistent CTA per SM, each owning a contiguous range of rows.
+    const int64_t groups = (n + kRows - 1) / kRows;
+    const int grid = static_cast<int>(groups < sms ? groups : sms);
+    const int nt = (QT != KQ_Q4_K && m <= 4) ? 1 : (m > 8 ? 2 : 1);
+    const int64_t rpc = (n + grid - 1) / grid;
+    const int nrg = static_cast<int>((rpc + kRows - 1) / kRows);
+    const uint32_t pbuf_bytes = 2u * kCWarps * 32 * 4 * nt * 4;
+    // Pick the stage geometry: most bytes in flight (ns stages x 16 rows x g
+    // blocks), then more stages, subject to the shared-memory budget that the
+    // activation image, the partial-sum buffers and the barriers leave.
+    int ns = 0, g = 0, scb = 0, rs = 0;
+    uint32_t tokstride = 0, off_img = 0, off_x = 0, off_pbuf = 0, off_racc = 0, total = 0;
+    int64_t best = -1;
+    const int gmax = cdiv(p.nblk, C::GA) * C::GA;
+    for (int ns_try = 4; ns_try >= 2; --ns_try) {
+        for (int g_try = gmax; g_try >= C::GA; g_try -= C::GA) {
+            const int rs_try = ((g_try * C::BPB + 127) / 128) * 128 + 16;
+            const uint32_t wbytes = kOffW + ns_try * kRows * rs_try;
+            const uint32_t oi = (wbytes + 127) & ~127u;
+            const int scb_full = cdiv(p.nblk, g_try) * g_try;
+            // super-chunk: as many whole stages of blocks as the image allows
+            for (int scb_try = scb_full; scb_try >= g_try; scb_try -= g_try) {
+                const uint32_t base = scb_try * C::IMG;
+                const uint32_t ts = base + ((32u - (base & 127u)) & 127u);
+                const uint32_t ox = oi + m * ts;
+                const uint32_t op = (ox + m * scb_try * C::XS * 4 + 15) & ~15u;
+                const uint32_t orc = op + pbuf_bytes;
+                const uint32_t tot = orc + (scb_try < scb_full ? nrg * kRows * 16 * 4 : 0);
+                if (tot > static_cast<uint32_t>(optin)) continue;
+                const int64_t inflight = static_cast<int64_t>(ns_try) * kRows * g_try * C::BPB;
+                if (inflight > best) {
+                    best = inflight;
+                    ns = ns_try; g = g_try; scb = scb_try; rs = rs_try;
+                    tokstride = ts; off_img = oi; off_x = ox; off_pbuf = op; off_racc = orc; total = tot;
+                }
+                break;
+            }
         }
-        if (scb >= C::G) break;
     }
-    if (scb < C::G) return KQ_ERR_UNSUPPORTED;
+    if (best < 0) {
+        // the activation image of all m rows does not fit: split the rows
+        if (m == 1) return KQ_ERR_UNSUPPORTED;
+        const int m1 = m / 2;
+        const int rc = launch_codec<QT>(w, n, k, x, m1, y, st);
+        if (rc) return rc;
+        return launch_codec<QT>(w, n, k, x + static_cast<int64_t>(m1) * k, m - m1, y + static_cast<int64_t>(m1) * n, st);
+    }
     p.ns = ns;
+    p.g = g;
+    p.rs = rs;
     p.scb = scb;
     p.tokstride = tokstride;
     p.off_img = off_img;
     p.off_x = off_x;
-    const int grid = cdiv(n, kRows);
+    p.off_pbuf = off_pbuf;
+    p.off_racc = off_racc;
     auto launch = [&](auto kernel) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
         if (e != cudaSuccess) return record_cuda(e);
-        kernel<<<grid, kThreads, total, st>>>(p);
-        return check_launch();
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = total;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = use_pdl() ? 1 : 0;
+        return record_cuda(cudaLaunchKernelEx(&cfg, kernel, p));
     };
     if constexpr (QT == KQ_Q4_K) {
         return m > 8 ? launch(qmv_kernel<QT, 1, 2>) : launch(qmv_kernel<QT, 1, 1>);
+    } else if constexpr (QT == KQ_Q8_0) {
+        // runs of 4 blocks per warp: at most 4 sub-block slots per token
+        if (m == 1) return launch(qmv_kernel<QT, 4, 1>);
+        if (m == 2) return launch(qmv_kernel<QT, 4, 1>);
+        if (m <= 4) return launch(qmv_kernel<QT, 2, 1>);
+        if (m <= 8) return launch(qmv_kernel<QT, 1, 1>);
+        return launch(qmv_kernel<QT, 1, 2>);
     } else {
         if (m == 1) return launch(qmv_kernel<QT, 8, 1>);
         if (m == 2) return launch(qmv_kernel<QT, 4, 1>);
