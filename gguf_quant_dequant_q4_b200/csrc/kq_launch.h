@@ -24,6 +24,10 @@ int* device_status_ptr();
 int launch_dequantize(int type, const void* w, int64_t n_rows, int64_t k, float* out, cudaStream_t s);
 int launch_qmv(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int m, float* y,
                cudaStream_t s);
+// Staged decode kernel for few activation rows; KQ_ERR_UNSUPPORTED for shapes
+// it does not cover.
+int launch_qmv_stream(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int m, float* y,
+                      cudaStream_t s);
 int launch_qmm(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int64_t m, float* y,
                cudaStream_t s);
 int launch_gather_qmm(int type, const void* w_bank, int n_experts, int64_t n, int64_t k,

@@ -818,6 +818,8 @@ int launch_codec(const void* w, int64_t n, int64_t k, const uint16_t* x, int m, 
 int launch_qmv(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int m, float* y,
                cudaStream_t s) {
     if (n == 0) return KQ_OK;
+    const int rc = launch_qmv_stream(type, w, n, k, x, m, y, s);
+    if (rc != KQ_ERR_UNSUPPORTED) return rc;
     switch (type) {
     case KQ_Q4_K: return launch_codec<KQ_Q4_K>(w, n, k, x, m, y, s);
     case KQ_Q6_K: return launch_codec<KQ_Q6_K>(w, n, k, x, m, y, s);

@@ -1,0 +1,830 @@
+// kq_qmv for 1 <= m <= 2 (q8_0, q6_K) or m <= 16 (q4_K): y = x . W^T.
+//
+// mlx-kquant bindings.cpp `quantized_matmul` (x @ dequant(w).T) and README
+// "How it works" (small row counts take a kernel that amortizes each weight
+// read over all rows); hanzo-ml quantized/mod.rs (decode multiplies "straight
+// out of the block format").  Block layouts: mlx-kquant README, "Codec
+// reference"; gguf-py constants (q4_K 144 B, q6_K 210 B, q8_0 34 B).
+//
+// Streaming.  One CTA per SM owns a balanced contiguous range of rows.  A
+// producer warp streams 16-row stages (whole rows when they fit, else equal
+// row slices) into a ring of shared-memory slots with one 1-D bulk copy per
+// row; big contiguous copies are what keeps HBM busy.  Before the first
+// stage it copies the activation rows, so they land first.  16 consumer
+// warps split every stage into work items and release the slot through an
+// mbarrier; the producer never waits for anything else.
+//
+// Arithmetic is the exact-integer tensor-core scheme: a lane turns its codes
+// into binary16 integers (OR into the mantissa of 1024), the activations
+// rounded once to binary16 are the B operand of m16n8k16 MMAs, and the tensor
+// core accumulates exact products in fp32; per-block scales are applied in
+// fp32 once a block is complete.  The activation operand of every MMA is
+// precomputed per CTA into a shared-memory image in fragment order (one
+// 8-byte load per MMA); B lanes whose column does not receive a given word
+// read a zero block instead of being masked.  The lane-to-byte mappings:
+//
+//  * q8_0, item = 16 rows x 8 blocks: lane t owns blocks 2t and 2t+1 (68
+//    bytes, word aligned) and feeds one 32-bit word per MMA.  Words 0..8 hold
+//    codes of the even block only (its fp16 scale bytes and the odd block's
+//    get a zero activation), words 9..16 those of the odd block, so MMA
+//    column 2t + parity collects exactly lane t's block of that parity.
+//  * q6_K, item = 16 rows x 1 block: lane t takes quarter (h = t >> 1,
+//    lh = t & 1): 16-value runs l of half h for all four q.  Low nibbles,
+//    high nibbles and the four 2-bit fields are separate MMAs whose
+//    activations carry the power of two that puts every part in units of
+//    c6 / 16; columns 2t, 2t+1 hold sub-blocks q, q + 2 (two passes).
+//  * q4_K, item = 16 rows x 1 block: lane t owns values 64t..64t+63 and
+//    multiplies its 4-bit codes by the 6-bit scale exactly in binary16
+//    (q sc <= 945); one column per token; the min term is one more MMA on
+//    (m_j) x (X_j split into two binary16 halves).
+//
+// Partial sums of the 16 warps are combined in a fixed order by the last
+// warp to finish a row group: results are bitwise reproducible.
+#include "kq_device.cuh"
+#include "kq_launch.h"
+
+namespace kq {
+namespace {
+
+constexpr int kCW = 16;                  // consumer warps
+constexpr int kProd = kCW;               // producer warp
+constexpr int kThreads = 32 * (kCW + 1);
+constexpr int kRows = 16;
+constexpr int kMaxStages = 6;
+constexpr int kMaxGroups = 64;           // row groups per CTA (counters)
+constexpr uint32_t kHdr = 1024;          // barriers and counters
+
+struct SP {
+    const uint8_t* w;
+    const uint16_t* x;
+    float* y;
+    int* status;
+    int64_t n, k, row_bytes;
+    int m, nblk, g, spr, ns;
+    uint32_t rs;   // shared-memory stride of a stage row
+    uint32_t off_stage, off_img, img_tok, off_xs, xs_tok, off_zero, off_part, off_xraw;
+};
+
+constexpr uint32_t kH1024 = 0x64006400u;    // binary16 (1024, 1024)
+constexpr uint32_t kHm1024 = 0xE400E400u;   // (-1024, -1024)
+constexpr uint32_t kH1_16 = 0x2C002C00u;    // (1/16, 1/16)
+
+// Volatile so that the conversions stay next to the MMA that consumes them.
+__device__ __forceinline__ uint32_t vand_or(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm volatile("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t vand_xor(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm volatile("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t vhfma2(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm volatile("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ void sts64(uint32_t a, uint32_t x, uint32_t y) {
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(x), "r"(y));
+}
+__device__ __forceinline__ void sts32(uint32_t a, uint32_t x) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(x));
+}
+__device__ __forceinline__ int lds_s8(uint32_t a) {
+    int16_t v;
+    asm volatile("ld.shared.s8 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float h2f(uint32_t h) { return __half2float(__ushort_as_half(static_cast<unsigned short>(h))); }
+
+// Bounded spin on an mbarrier phase (no suspend hint: these waits are short
+// and a sleeping warp can wake up late).  False after the time limit, with
+// KQ_DEV_TIMEOUT recorded.
+__device__ __forceinline__ bool spin_wait(uint64_t* bar, uint32_t parity, int* status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (int i = 0;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255) == 255 && global_ns() - t0 > kWaitLimitNs) {
+            if (status) atomicOr(status, KQ_DEV_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Raw bf16 activations, copied into shared memory before the image is built.
+__device__ __forceinline__ uint32_t xaddr(const SP& p, uint32_t sb, int tok, int64_t i) {
+    return sb + p.off_xraw + 2u * static_cast<uint32_t>(tok * p.k + i);
+}
+__device__ __forceinline__ float xval(const SP& p, uint32_t sb, int tok, int64_t i) {
+    return __uint_as_float(lds_u16(xaddr(p, sb, tok, i)) << 16);
+}
+// Binary16 of a (power-of-two scaled) activation, tracking the range.
+__device__ __forceinline__ __half hx(float v, float& amax) {
+    amax = fmaxf(amax, fabsf(v));
+    return __float2half_rn(v);
+}
+__device__ __forceinline__ uint32_t hpair(__half lo, __half hi) {
+    return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+}
+
+// Lane roles in the m16n8k16 fragments (lane = 4 g + t): A rows g and g+8,
+// k-slots 2t, 2t+1, 2t+8, 2t+9; B column g; D columns 2t, 2t+1.
+struct Lane {
+    int g, t;
+};
+
+// ===========================================================================
+// q8_0
+// ===========================================================================
+template <int NT>
+struct Q8 {
+    static constexpr int kVPB = 32, kBPB = 34;
+    static constexpr int kItemBlocks = 8;
+    static constexpr uint32_t kItemImg = 17 * 32;   // image bytes per item (8 blocks) and token
+    static constexpr uint32_t kZero = kItemImg;
+    static constexpr int kAccPerLane = 2 * NT;
+
+    // rowA/rowB: shared address of the item (8 blocks) in rows g / g+8;
+    // gi: global item index (block 8 gi).
+    static __device__ __forceinline__ void item(const SP& p, uint32_t sb, const Lane& L, uint32_t rowA,
+                                                uint32_t rowB, int gi, float (&acc)[2 * NT]) {
+        const int t = L.t;
+        const bool act = (L.g >> 1) == t;   // B lanes whose column holds lane t's blocks
+        uint32_t bb[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const uint32_t img = sb + p.off_img + nt * p.img_tok + gi * kItemImg + 8 * t;
+            const uint32_t zero = sb + p.off_zero + 8 * t;
+            bb[nt][0] = (act && (L.g & 1) == 0) ? img : zero;
+            bb[nt][1] = (act && (L.g & 1) == 1) ? img : zero;
+        }
+        float D[NT][2][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) D[nt][c][e] = 0.f;
+        const uint32_t a0 = rowA + 68 * t, b0 = rowB + 68 * t;
+        float dE[2], dO[2];
+#pragma unroll
+        for (int mu = 0; mu < 17; ++mu) {
+            const uint32_t wa = lds32(a0 + 4 * mu), wb = lds32(b0 + 4 * mu);
+            if (mu == 0) {   // fp16 d of the even block: bytes 0..1 of the span
+                dE[0] = h2f(wa & 0xffff);
+                dE[1] = h2f(wb & 0xffff);
+            }
+            if (mu == 8) {   // the odd block's d: bytes 34..35
+                dO[0] = h2f(wa >> 16);
+                dO[1] = h2f(wb >> 16);
+            }
+            const int par = mu >= 9 ? 1 : 0;
+            // (byte ^ 0x80) in the mantissa of 1024: 1152 + code, exactly
+            const uint32_t A0 = vand_xor(wa, 0x00FF00FFu, 0x64806480u);
+            const uint32_t A1 = vand_xor(wb, 0x00FF00FFu, 0x64806480u);
+            const uint32_t A2 = vand_xor(wa >> 8, 0x00FF00FFu, 0x64806480u);
+            const uint32_t A3 = vand_xor(wb >> 8, 0x00FF00FFu, 0x64806480u);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const uint2 bv = lds64(bb[nt][par] + 32 * mu);
+                mma_f16(D[nt][mu & 1], A0, A1, A2, A3, bv.x, bv.y);
+            }
+        }
+        // y += d (D - 1152 X) for columns 2t (even block) and 2t+1 (odd block)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const uint2 xv = lds64(sb + p.off_xs + nt * p.xs_tok + 4 * (8 * gi + 2 * t));
+            const float X[2] = {__uint_as_float(xv.x), __uint_as_float(xv.y)};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = e >> 1, odd = e & 1;
+                const float Ds = D[nt][0][e] + D[nt][1][e];
+                const float d = odd ? dO[r] : dE[r];
+                acc[2 * nt + r] = fmaf(d, fmaf(-1152.0f, X[odd], Ds), acc[2 * nt + r]);
+            }
+        }
+    }
+
+    // Partial sums of this warp for a row group -> part[row][tok].
+    static __device__ __forceinline__ void store_part(const SP& p, const Lane& L, float (&acc)[2 * NT], float* part) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                float v = acc[2 * nt + r];
+                v += __shfl_xor_sync(0xffffffffu, v, 1);
+                v += __shfl_xor_sync(0xffffffffu, v, 2);
+                if (L.t == 0) part[(L.g + 8 * r) * p.m + nt] = v;
+            }
+    }
+
+    // Image entry (item, mu, t') = binary16 activations of the 4 raw bytes at
+    // offset 272 item + 68 t' + 4 mu of a row, as (byte0, byte2 | byte1,
+    // byte3); scale bytes get 0.  X[tok][block] = sum of its 32 activations.
+    static __device__ void build(const SP& p, uint32_t sb, float& amax) {
+        const int items = p.nblk / 8;
+        const int per_tok = items * 17 * 4;
+        for (int e = threadIdx.x; e < p.m * per_tok; e += kCW * 32) {
+            const int tok = e / per_tok, rem = e % per_tok;
+            const int it = rem / 68, mu = (rem % 68) >> 2, tt = rem & 3;
+            const int R0 = it * 272 + 68 * tt + 4 * mu;
+            __half h[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int R = R0 + b, blk = R / 34, o = R - 34 * blk;
+                h[b] = o >= 2 ? hx(xval(p, sb, tok, 32 * blk + o - 2), amax) : __float2half_rn(0.f);
+            }
+            sts64(sb + p.off_img + tok * p.img_tok + it * kItemImg + mu * 32 + tt * 8, hpair(h[0], h[2]),
+                  hpair(h[1], h[3]));
+        }
+        for (int e = threadIdx.x; e < p.m * p.nblk; e += kCW * 32) {
+            const int tok = e / p.nblk, blk = e % p.nblk;
+            const uint32_t xs = xaddr(p, sb, tok, 32 * blk);
+            float X = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint4 v = lds128(xs + 16 * c);
+                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    X += __half2float(__float2half_rn(bf16lo_to_f32(wv[q])));
+                    X += __half2float(__float2half_rn(bf16hi_to_f32(wv[q])));
+                }
+            }
+            sts32(sb + p.off_xs + tok * p.xs_tok + 4 * blk, __float_as_uint(X));
+        }
+    }
+};
+
+// ===========================================================================
+// q6_K
+// ===========================================================================
+template <int NT>
+struct Q6 {
+    static constexpr int kVPB = 256, kBPB = 210;
+    static constexpr int kItemBlocks = 1;
+    static constexpr uint32_t kBlkImg = 1024;   // image bytes per block and token
+    static constexpr uint32_t kZero = kBlkImg;
+    static constexpr int kAccPerLane = 2 * NT;
+
+    // 4 words of the 16-byte piece at shared address a (2-byte aligned when
+    // ODD: assembled from 5 aligned words).
+    template <bool ODD>
+    static __device__ __forceinline__ void piece(uint32_t a, uint32_t (&w)[4]) {
+        if constexpr (ODD) {
+            uint32_t u[5];
+#pragma unroll
+            for (int i = 0; i < 5; ++i) u[i] = lds32(a - 2 + 4 * i);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) w[i] = __byte_perm(u[i], u[i + 1], 0x5432);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) w[i] = lds32(a + 4 * i);
+        }
+    }
+
+    template <bool ODD>
+    static __device__ __forceinline__ void block(const SP& p, uint32_t sb, const Lane& L, uint32_t rowA,
+                                                 uint32_t rowB, int gb, float (&acc)[2 * NT]) {
+        const int t = L.t, h = t >> 1, lh = t & 1;
+        const bool act = (L.g >> 1) == t;
+        uint32_t bb[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const uint32_t img = sb + p.off_img + nt * p.img_tok + gb * kBlkImg + 8 * t;
+            const uint32_t zero = sb + p.off_zero + 8 * t;
+            bb[nt][0] = (act && (L.g & 1) == 0) ? img : zero;
+            bb[nt][1] = (act && (L.g & 1) == 1) ? img : zero;
+        }
+        // scales: sc[j], j = 8h + lh + 2q, and 16 d
+        float sc[2][4], d16[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const uint32_t row = r ? rowB : rowA;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) sc[r][q] = static_cast<float>(lds_s8(row + 192 + 8 * h + lh + 2 * q));
+            d16[r] = 16.0f * h2f(lds_u16(row + 208));
+        }
+        float D[2][2][NT][4];   // [pass qp][chain][n-tile][element]
+#pragma unroll
+        for (int qp = 0; qp < 2; ++qp)
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) D[qp][c][nt][e] = 0.f;
+        // ql pieces: low nibbles -> q = qp (slot 0, B = x/16), high nibbles ->
+        // q = qp + 2 (slot 1, B = x/256)
+#pragma unroll
+        for (int qp = 0; qp < 2; ++qp) {
+            uint32_t wa[4], wb[4];
+            piece<ODD>(rowA + 64 * h + 32 * qp + 16 * lh, wa);
+            piece<ODD>(rowB + 64 * h + 32 * qp + 16 * lh, wb);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t a8 = wa[k] >> 8, b8 = wb[k] >> 8;
+                const uint32_t L0 = vand_or(wa[k], 0x000F000Fu, kH1024), L1 = vand_or(wb[k], 0x000F000Fu, kH1024);
+                const uint32_t L2 = vand_or(a8, 0x000F000Fu, kH1024), L3 = vand_or(b8, 0x000F000Fu, kH1024);
+                const uint32_t H0 = vand_or(wa[k], 0x00F000F0u, kH1024), H1 = vand_or(wb[k], 0x00F000F0u, kH1024);
+                const uint32_t H2 = vand_or(a8, 0x00F000F0u, kH1024), H3 = vand_or(b8, 0x00F000F0u, kH1024);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const uint2 bl = lds64(bb[nt][0] + 32 * (16 * qp + k));
+                    const uint2 bh = lds64(bb[nt][1] + 32 * (16 * qp + 4 + k));
+                    mma_f16(D[qp][k & 1][nt], L0, L1, L2, L3, bl.x, bl.y);
+                    mma_f16(D[qp][k & 1][nt], H0, H1, H2, H3, bh.x, bh.y);
+                }
+            }
+        }
+        // qh piece: 2-bit field q at bits 2q -> 1024 + 4^q c, B = x / 4^q
+        {
+            uint32_t ha[4], hb[4];
+            piece<ODD>(rowA + 128 + 32 * h + 16 * lh, ha);
+            piece<ODD>(rowB + 128 + 32 * h + 16 * lh, hb);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t a8 = ha[k] >> 8, b8 = hb[k] >> 8;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t mk = 0x00030003u << (2 * q);
+                    const uint32_t A0 = vand_or(ha[k], mk, kH1024), A1 = vand_or(hb[k], mk, kH1024);
+                    const uint32_t A2 = vand_or(a8, mk, kH1024), A3 = vand_or(b8, mk, kH1024);
+                    const int qp = q & 1, sl = q >> 1;
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const uint2 bv = lds64(bb[nt][sl] + 32 * (16 * qp + 8 + 4 * sl + k));
+                        mma_f16(D[qp][(k >> 1) & 1][nt], A0, A1, A2, A3, bv.x, bv.y);
+                    }
+                }
+            }
+        }
+        // y += 16 d sc_j (D - C_q X_j), C_q = 1090, 322, 70, 22
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const uint4 xv = lds128(sb + p.off_xs + nt * p.xs_tok + gb * 64 + 16 * t);
+            const float Xq[4] = {__uint_as_float(xv.x), __uint_as_float(xv.y), __uint_as_float(xv.z),
+                                 __uint_as_float(xv.w)};
+#pragma unroll
+            for (int qp = 0; qp < 2; ++qp)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = e >> 1, q = qp + 2 * (e & 1);
+                    const float C = q == 0 ? 1090.0f : (q == 1 ? 322.0f : (q == 2 ? 70.0f : 22.0f));
+                    const float Ds = D[qp][0][nt][e] + D[qp][1][nt][e];
+                    const float s = __fmul_rn(d16[r], sc[r][q]);
+                    acc[2 * nt + r] = fmaf(s, fmaf(-C, Xq[q], Ds), acc[2 * nt + r]);
+                }
+        }
+    }
+
+    static __device__ __forceinline__ void item(const SP& p, uint32_t sb, const Lane& L, uint32_t rowA,
+                                                uint32_t rowB, int gb, float (&acc)[2 * NT]) {
+        if (gb & 1) block<true>(p, sb, L, rowA, rowB, gb, acc);
+        else block<false>(p, sb, L, rowA, rowB, gb, acc);
+    }
+
+    static __device__ __forceinline__ void store_part(const SP& p, const Lane& L, float (&acc)[2 * NT], float* part) {
+        Q8<NT>::store_part(p, L, acc, part);
+    }
+
+    // Image entry (block, E, t'): E = 16 qp + 4 kind + k; kind 0 = low nibble
+    // (q = qp, x/16), 1 = high nibble (q = qp + 2, x/256), 2 / 3 = 2-bit
+    // field q = qp / qp + 2 (x / 4^q).  Word k of quarter t' holds
+    // l = 16 lh + 4k + b, value v = 128 h + 32 q + l.
+    // X[tok][block][t'][q] = sum over the 16 l of binary16(x[v]).
+    static __device__ void build(const SP& p, uint32_t sb, float& amax) {
+        const int per_tok = p.nblk * 32 * 4;
+        for (int e = threadIdx.x; e < p.m * per_tok; e += kCW * 32) {
+            const int tok = e / per_tok, rem = e % per_tok;
+            const int blk = rem >> 7, E = (rem >> 2) & 31, tt = rem & 3;
+            const int h = tt >> 1, lh = tt & 1, qp = E >> 4, kind = (E >> 2) & 3, kk = E & 3;
+            const int q = qp + 2 * (kind & 1);
+            const float sc = kind == 0 ? 0.0625f : (kind == 1 ? 0.00390625f : 1.0f / static_cast<float>(1 << (2 * q)));
+            const int64_t v0 = static_cast<int64_t>(blk) * 256 + 128 * h + 32 * q + 16 * lh + 4 * kk;
+            const uint2 xr = lds64(xaddr(p, sb, tok, v0));
+            const float xf[4] = {bf16lo_to_f32(xr.x), bf16hi_to_f32(xr.x), bf16lo_to_f32(xr.y), bf16hi_to_f32(xr.y)};
+            __half hv[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) hv[b] = hx(xf[b] * sc, amax);
+            sts64(sb + p.off_img + tok * p.img_tok + blk * kBlkImg + E * 32 + tt * 8, hpair(hv[0], hv[2]),
+                  hpair(hv[1], hv[3]));
+        }
+        const int per_tok_x = p.nblk * 16;
+        for (int e = threadIdx.x; e < p.m * per_tok_x; e += kCW * 32) {
+            const int tok = e / per_tok_x, rem = e % per_tok_x;
+            const int blk = rem >> 4, tt = (rem >> 2) & 3, q = rem & 3;
+            const int h = tt >> 1, lh = tt & 1;
+            const uint32_t xs = xaddr(p, sb, tok, blk * 256 + 128 * h + 32 * q + 16 * lh);
+            float X = 0.f;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const uint4 v = lds128(xs + 16 * c);
+                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    X += __half2float(__float2half_rn(bf16lo_to_f32(wv[u])));
+                    X += __half2float(__float2half_rn(bf16hi_to_f32(wv[u])));
+                }
+            }
+            sts32(sb + p.off_xs + tok * p.xs_tok + (blk * 16 + tt * 4 + q) * 4, __float_as_uint(X));
+        }
+    }
+};
+
+// ===========================================================================
+// q4_K
+// ===========================================================================
+template <int NT>
+struct Q4 {
+    static constexpr int kVPB = 256, kBPB = 144;
+    static constexpr int kItemBlocks = 1;
+    static constexpr uint32_t kBlkImg = 544;
+    static constexpr uint32_t kZero = kBlkImg;
+    static constexpr int kAccPerLane = 4 * NT;
+
+    static __device__ __forceinline__ void item(const SP& p, uint32_t sb, const Lane& L, uint32_t rowA,
+                                                uint32_t rowB, int gb, float (&acc)[4 * NT]) {
+        const int t = L.t;
+        uint32_t bb[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int tok = 8 * nt + L.g;
+            bb[nt] = tok < p.m ? sb + p.off_img + tok * p.img_tok + gb * kBlkImg + 8 * t : sb + p.off_zero + 8 * t;
+        }
+        const uint4 hA = lds128(rowA), hB = lds128(rowB);
+        const uint4 qA0 = lds128(rowA + 16 + 32 * t), qA1 = lds128(rowA + 32 + 32 * t);
+        const uint4 qB0 = lds128(rowB + 16 + 32 * t), qB1 = lds128(rowB + 32 + 32 * t);
+        // 6-bit scale/min codes of sub-blocks 2t, 2t+1 as (code_2t, code_2t+1)
+        // in bits 0..5 / 16..21.  t < 2: sc = s[j] & 63, m = s[j+4] & 63;
+        // t >= 2 (j >= 4): sc = (s[j+4] & 15) | (s[j-4] >> 6) << 4,
+        // m = (s[j+4] >> 4) | (s[j] >> 6) << 4.
+        const bool lo = t < 2;
+        const uint32_t jj0 = (2 * t) & 3;
+        const uint32_t sel = 0x4040u | jj0 | ((jj0 + 1) << 8);
+        const uint32_t mka = lo ? 0x003F003Fu : 0x000F000Fu, mkb = lo ? 0u : 0x00300030u;
+        uint32_t S_lo[2], B_lo[2], S_hi[2], B_hi[2], M_lo[2], M_hi[2];
+        float dd[2], dm[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const uint4 hh = r ? hB : hA;
+            const uint32_t asc = lo ? hh.y : hh.w;
+            const uint32_t am = lo ? hh.z : (hh.w >> 4);
+            const uint32_t scp = (__byte_perm(asc, 0, sel) & mka) | ((__byte_perm(hh.y, 0, sel) >> 2) & mkb);
+            const uint32_t mp = (__byte_perm(am, 0, sel) & mka) | ((__byte_perm(hh.z, 0, sel) >> 2) & mkb);
+            const uint32_t scf = hsub2_u32(scp | kH1024, kH1024);   // (sc_2t, sc_2t+1) exactly
+            const uint32_t mf = hsub2_u32(mp | kH1024, kH1024);
+            S_lo[r] = __byte_perm(scf, 0, 0x1010);
+            S_hi[r] = hmul2_u32(__byte_perm(scf, 0, 0x3232), kH1_16);
+            B_lo[r] = hmul2_u32(S_lo[r], kHm1024);   // -1024 sc
+            B_hi[r] = hmul2_u32(S_hi[r], kHm1024);   // -64 sc
+            M_lo[r] = __byte_perm(mf, 0, 0x1010);
+            M_hi[r] = __byte_perm(mf, 0, 0x3232);
+            dd[r] = h2f(hh.x & 0xffff);
+            dm[r] = h2f(hh.x >> 16);
+        }
+        const uint32_t wA[8] = {qA0.x, qA0.y, qA0.z, qA0.w, qA1.x, qA1.y, qA1.z, qA1.w};
+        const uint32_t wB[8] = {qB0.x, qB0.y, qB0.z, qB0.w, qB1.x, qB1.y, qB1.z, qB1.w};
+        float D[4][NT][4], Dm[NT][4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) D[c][nt][e] = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const uint32_t a = wA[u], b = wB[u], a8 = a >> 8, b8 = b >> 8;
+            // low nibbles: (1024 + q) sc - 1024 sc = q sc exactly
+            const uint32_t a0 = vhfma2(vand_or(a, 0x000F000Fu, kH1024), S_lo[0], B_lo[0]);
+            const uint32_t a1 = vhfma2(vand_or(b, 0x000F000Fu, kH1024), S_lo[1], B_lo[1]);
+            const uint32_t a2 = vhfma2(vand_or(a8, 0x000F000Fu, kH1024), S_lo[0], B_lo[0]);
+            const uint32_t a3 = vhfma2(vand_or(b8, 0x000F000Fu, kH1024), S_lo[1], B_lo[1]);
+            // high nibbles: (1024 + 16 q) sc / 16 - 64 sc = q sc exactly
+            const uint32_t c0 = vhfma2(vand_or(a, 0x00F000F0u, kH1024), S_hi[0], B_hi[0]);
+            const uint32_t c1 = vhfma2(vand_or(b, 0x00F000F0u, kH1024), S_hi[1], B_hi[1]);
+            const uint32_t c2 = vhfma2(vand_or(a8, 0x00F000F0u, kH1024), S_hi[0], B_hi[0]);
+            const uint32_t c3 = vhfma2(vand_or(b8, 0x00F000F0u, kH1024), S_hi[1], B_hi[1]);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const uint2 bl = lds64(bb[nt] + u * 32);
+                const uint2 bh = lds64(bb[nt] + (8 + u) * 32);
+                mma_f16(D[u & 3][nt], a0, a1, a2, a3, bl.x, bl.y);
+                mma_f16(D[u & 3][nt], c0, c1, c2, c3, bh.x, bh.y);
+            }
+        }
+        // y += d D - dmin sum_j m_j X_j
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const uint2 bv = lds64(bb[nt] + 512);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) Dm[nt][e] = 0.f;
+            mma_f16(Dm[nt], M_lo[0], M_lo[1], M_hi[0], M_hi[1], bv.x, bv.y);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = e >> 1;
+                const float Ds = (D[0][nt][e] + D[1][nt][e]) + (D[2][nt][e] + D[3][nt][e]);
+                acc[4 * nt + e] = fmaf(dd[r], Ds, fmaf(-dm[r], Dm[nt][e], acc[4 * nt + e]));
+            }
+        }
+    }
+
+    static __device__ __forceinline__ void store_part(const SP& p, const Lane& L, float (&acc)[4 * NT], float* part) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int tok = 8 * nt + 2 * L.t + (e & 1);
+                if (tok < p.m) part[(L.g + 8 * (e >> 1)) * p.m + tok] = acc[4 * nt + e];
+            }
+    }
+
+    // Image per block and token: MMA (nib, u) of lane t uses values
+    // v = 64t + 32nib + 4u + {0,2 | 1,3}; the last 32 bytes hold (Xhi, Xlo)
+    // of sub-blocks 2t and 2t+1.
+    static __device__ void build(const SP& p, uint32_t sb, float& amax) {
+        const int items = p.m * p.nblk * 4;
+        for (int it = threadIdx.x; it < items; it += kCW * 32) {
+            const int tok = it / (p.nblk * 4), rem = it % (p.nblk * 4), bl = rem >> 2, t = rem & 3;
+            const uint32_t base = sb + p.off_img + tok * p.img_tok + bl * kBlkImg;
+            const uint32_t xs = xaddr(p, sb, tok, static_cast<int64_t>(bl) * 256 + 64 * t);
+            float X[2] = {0.f, 0.f};
+#pragma unroll
+            for (int nib = 0; nib < 2; ++nib) {
+#pragma unroll
+                for (int uu = 0; uu < 2; ++uu) {
+                    const uint4 r0 = lds128(xs + 2 * (32 * nib + 16 * uu));
+                    const uint4 r1 = lds128(xs + 2 * (32 * nib + 16 * uu + 8));
+                    const uint32_t wv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int u = 4 * uu + q;
+                        const __half f0 = hx(bf16lo_to_f32(wv[2 * q]), amax), f1 = hx(bf16hi_to_f32(wv[2 * q]), amax);
+                        const __half f2 = hx(bf16lo_to_f32(wv[2 * q + 1]), amax);
+                        const __half f3 = hx(bf16hi_to_f32(wv[2 * q + 1]), amax);
+                        X[nib] += (__half2float(f0) + __half2float(f1)) + (__half2float(f2) + __half2float(f3));
+                        sts64(base + (nib * 8 + u) * 32 + t * 8, hpair(f0, f2), hpair(f1, f3));
+                    }
+                }
+            }
+            uint32_t e[2];
+#pragma unroll
+            for (int nib = 0; nib < 2; ++nib) {
+                const __half hi = __float2half_rn(X[nib]);
+                const __half lo = __float2half_rn(X[nib] - __half2float(hi));
+                e[nib] = hpair(hi, lo);
+            }
+            sts64(base + 512 + t * 8, e[0], e[1]);
+        }
+    }
+};
+
+// ===========================================================================
+// Kernel
+// ===========================================================================
+template <class C>
+__global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);   // [kMaxStages]
+    uint64_t* empty = full + kMaxStages;                   // [kMaxStages]
+    uint64_t* xbar = full + 2 * kMaxStages;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 128);
+    int* grp_done = reinterpret_cast<int*>(smem + 256);   // [kMaxGroups]
+    const uint32_t sb = smem_u32(smem);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t r0 = static_cast<int64_t>(blockIdx.x) * p.n / gridDim.x;
+    const int64_t r1 = static_cast<int64_t>(blockIdx.x + 1) * p.n / gridDim.x;
+    const int nrg = cdiv(r1 - r0, kRows);
+    const uint32_t stage_bytes = kRows * p.rs;
+
+    if (tid == 0) {
+        for (int i = 0; i < p.ns; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kCW);
+        }
+        mbar_init(xbar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (tid < kMaxGroups) grp_done[tid] = 0;
+    __syncthreads();
+    // Programmatic dependent launch: the next kernel may start its prologue;
+    // this one waits for the earlier grids before it reads x or W.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    if (warp == kProd) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            const uint32_t row = 2u * static_cast<uint32_t>(p.k);
+            mbar_arrive_expect_tx(xbar, row * p.m);
+            for (int tok = 0; tok < p.m; ++tok)
+                bulk_g2s(smem + p.off_xraw + tok * row, p.x + static_cast<int64_t>(tok) * p.k, row, xbar);
+        }
+        int q = 0;
+        bool ok = true;
+        for (int rg = 0; rg < nrg && ok; ++rg) {
+            const int64_t row0 = r0 + static_cast<int64_t>(rg) * kRows;
+            const int rv = static_cast<int>(r1 - row0 < kRows ? r1 - row0 : kRows);
+            for (int st = 0; st < p.spr; ++st, ++q) {
+                const int slot = q % p.ns;
+                if (lane == 0 && q >= p.ns) ok = spin_wait(&empty[slot], ((q / p.ns) & 1) ^ 1, p.status);
+                ok = __shfl_sync(0xffffffffu, ok, 0) && !*abort_flag;
+                if (!ok) {
+                    *abort_flag = 1;
+                    break;
+                }
+                const int b0 = st * p.g;
+                const int nb = p.nblk - b0 < p.g ? p.nblk - b0 : p.g;
+                const uint32_t bytes = static_cast<uint32_t>(nb) * C::kBPB;
+                if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes * rv);
+                __syncwarp();
+                if (lane < rv)
+                    bulk_g2s(smem + p.off_stage + slot * stage_bytes + lane * p.rs,
+                             p.w + (row0 + lane) * p.row_bytes + static_cast<int64_t>(b0) * C::kBPB, bytes,
+                             &full[slot]);
+            }
+        }
+        // after an abort, let the copies in flight land before the CTA exits
+        if (!ok && lane == 0) {
+            spin_wait(xbar, 0, nullptr);
+            for (int qq = q - p.ns > 0 ? q - p.ns : 0; qq < q; ++qq)
+                spin_wait(&full[qq % p.ns], (qq / p.ns) & 1, nullptr);
+        }
+    } else {
+        // --------------------------------------------------------- consumers
+        Lane L;
+        L.g = lane >> 2;
+        L.t = lane & 3;
+        float amax = 0.f;
+        if (!spin_wait(xbar, 0, p.status)) *abort_flag = 1;
+        if (!*abort_flag) {
+            C::build(p, sb, amax);
+            for (uint32_t o = 4 * tid; o < C::kZero; o += 4 * kCW * 32) sts32(sb + p.off_zero + o, 0u);
+        }
+        if (amax >= 65504.0f) atomicOr(p.status, KQ_DEV_X_RANGE);
+        asm volatile("bar.sync 1, %0;" ::"r"(kCW * 32) : "memory");   // image ready (x copy now dead)
+        float* part = reinterpret_cast<float*>(smem + p.off_part);
+        const int items_per_row = p.nblk / C::kItemBlocks;
+        int q = 0;
+        for (int rg = 0; rg < nrg && !*abort_flag; ++rg) {
+            const int64_t row0 = r0 + static_cast<int64_t>(rg) * kRows;
+            const int rv = static_cast<int>(r1 - row0 < kRows ? r1 - row0 : kRows);
+            float acc[C::kAccPerLane];
+#pragma unroll
+            for (int i = 0; i < C::kAccPerLane; ++i) acc[i] = 0.f;
+            // items of the row group, round robin over warps across stages
+            bool ok = true;
+            for (int st = 0; st < p.spr; ++st, ++q) {
+                const int slot = q % p.ns;
+                const int i0 = st * p.g / C::kItemBlocks;
+                const int i1 = min(items_per_row, (st + 1) * p.g / C::kItemBlocks);
+                const int first = i0 + ((warp - i0) % kCW + kCW) % kCW;
+                // every warp waits for the stage, items or not, so that its
+                // release below always belongs to this fill of the slot
+                if (!spin_wait(&full[slot], (q / p.ns) & 1, p.status)) {
+                    *abort_flag = 1;
+                    ok = false;
+                } else {
+                    const uint32_t stg = sb + p.off_stage + slot * stage_bytes;
+                    const uint32_t rowA = stg + L.g * p.rs, rowB = rowA + 8 * p.rs;
+                    for (int it = first; it < i1; it += kCW) {
+                        const uint32_t off = static_cast<uint32_t>(it * C::kItemBlocks - st * p.g) * C::kBPB;
+                        C::item(p, sb, L, rowA + off, rowB + off, it, acc);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[slot]);
+                if (!ok) break;
+            }
+            if (!ok) break;
+            // partial sums -> shared memory; the last warp of the row group sums
+            // the 16 partials in warp order and stores y
+            float* pw = part + (rg * kCW + warp) * kRows * p.m;
+            C::store_part(p, L, acc, pw);
+            __threadfence_block();
+            __syncwarp();
+            int last = 0;
+            if (lane == 0) last = atomicAdd(&grp_done[rg], 1) == kCW - 1;
+            last = __shfl_sync(0xffffffffu, last, 0);
+            if (last) {
+                __threadfence_block();
+                for (int o = lane; o < kRows * p.m; o += 32) {
+                    const int tok = o / kRows, r = o % kRows;
+                    float sum = 0.f;
+                    for (int w = 0; w < kCW; ++w) sum += part[((rg * kCW + w) * kRows + r) * p.m + tok];
+                    if (r < rv) p.y[static_cast<int64_t>(tok) * p.n + row0 + r] = sum;
+                }
+            }
+        }
+    }
+    __syncthreads();
+}
+
+constexpr uint32_t align16(uint32_t v) { return (v + 15u) & ~15u; }
+
+template <class C>
+int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m, float* y, cudaStream_t st,
+                  uint32_t img_tok, uint32_t xs_tok) {
+    SP p{};
+    p.w = static_cast<const uint8_t*>(w);
+    p.x = x;
+    p.y = y;
+    p.status = device_status_ptr();
+    p.n = n;
+    p.k = k;
+    p.m = m;
+    p.nblk = static_cast<int>(k / C::kVPB);
+    p.row_bytes = static_cast<int64_t>(p.nblk) * C::kBPB;
+    if (p.row_bytes % 16 != 0) return KQ_ERR_UNSUPPORTED;
+    p.img_tok = img_tok;
+    p.xs_tok = xs_tok;
+    const int sms = device_sm_count();
+    const int64_t gmax = (n + 7) / 8;   // at least 8 rows per CTA
+    const int grid = static_cast<int>(sms < gmax ? sms : (gmax > 0 ? gmax : 1));
+    const int nrg_max = cdiv(cdiv(n, grid), kRows);
+    if (nrg_max > kMaxGroups) return KQ_ERR_UNSUPPORTED;
+    const uint32_t optin = static_cast<uint32_t>(device_smem_optin());
+    // fixed part of the layout
+    p.off_img = kHdr;
+    p.off_xs = align16(p.off_img + m * img_tok);
+    p.off_zero = align16(p.off_xs + m * xs_tok);
+    p.off_part = align16(p.off_zero + C::kZero);
+    p.off_xraw = p.off_part;   // the raw x copy is dead before any partial sum is written
+    const uint32_t part = static_cast<uint32_t>(nrg_max) * kCW * kRows * m * 4;
+    const uint32_t xraw = static_cast<uint32_t>(m) * static_cast<uint32_t>(k) * 2;
+    p.off_stage = (p.off_part + (part > xraw ? part : xraw) + 127u) & ~127u;
+    // stage geometry: whole rows if two or more stages fit, else the fewest
+    // equal row slices (a multiple of the item size, copies 16-byte sized)
+    // that do; the deepest ring that fits
+    const int ga = C::kItemBlocks * (C::kBPB % 16 == 0 ? 1 : 8 / C::kItemBlocks);
+    p.ns = 0;
+    for (int s = 1; s <= 16 && p.ns == 0; ++s) {
+        const int g = cdiv(cdiv(p.nblk, s), ga) * ga;
+        if (s > 1 && g >= p.nblk) continue;
+        const uint32_t rs = ((static_cast<uint32_t>(g) * C::kBPB + 127u) & ~127u) + 16;
+        for (int ns = kMaxStages; ns >= 2; --ns) {
+            if (p.off_stage + static_cast<uint32_t>(ns) * kRows * rs <= optin) {
+                p.ns = ns;
+                p.g = g;
+                p.rs = rs;
+                p.spr = cdiv(p.nblk, g);
+                break;
+            }
+        }
+    }
+    if (p.ns == 0) return KQ_ERR_UNSUPPORTED;
+    const uint32_t total = p.off_stage + static_cast<uint32_t>(p.ns) * kRows * p.rs;
+    auto kernel = qmv_stream_kernel<C>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
+    if (e != cudaSuccess) return record_cuda(e);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = total;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = use_pdl() ? 1 : 0;
+    return record_cuda(cudaLaunchKernelEx(&cfg, kernel, p));
+}
+
+}  // namespace
+
+// Staged qmv for the shapes it covers; KQ_ERR_UNSUPPORTED otherwise (the
+// caller then takes the general kernel).
+int launch_qmv_stream(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int m, float* y,
+                      cudaStream_t s) {
+    switch (type) {
+    case KQ_Q8_0: {
+        const int nblk = static_cast<int>(k / 32);
+        if (m > 2 || nblk % 8 != 0) return KQ_ERR_UNSUPPORTED;
+        const uint32_t it = (nblk / 8) * Q8<1>::kItemImg, xt = nblk * 4;
+        return m == 1 ? launch_stream<Q8<1>>(w, n, k, x, m, y, s, it, xt) : launch_stream<Q8<2>>(w, n, k, x, m, y, s, it, xt);
+    }
+    case KQ_Q6_K: {
+        const int nblk = static_cast<int>(k / 256);
+        if (m > 2 || nblk % 8 != 0) return KQ_ERR_UNSUPPORTED;
+        const uint32_t it = nblk * Q6<1>::kBlkImg, xt = nblk * 64;
+        return m == 1 ? launch_stream<Q6<1>>(w, n, k, x, m, y, s, it, xt) : launch_stream<Q6<2>>(w, n, k, x, m, y, s, it, xt);
+    }
+    case KQ_Q4_K: {
+        const int nblk = static_cast<int>(k / 256);
+        const uint32_t it = nblk * Q4<1>::kBlkImg;
+        if (m <= 8) return launch_stream<Q4<1>>(w, n, k, x, m, y, s, it, 0);
+        return launch_stream<Q4<2>>(w, n, k, x, m, y, s, it, 0);
+    }
+    default: return KQ_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace kq
