@@ -28,11 +28,11 @@
 //    codes of the even block only (its fp16 scale bytes and the odd block's
 //    get a zero activation), words 9..16 those of the odd block, so MMA
 //    column 2t + parity collects exactly lane t's block of that parity.
-//  * q6_K, item = 16 rows x 1 block: lane t takes quarter (h = t >> 1,
-//    lh = t & 1): 16-value runs l of half h for all four q.  Low nibbles,
-//    high nibbles and the four 2-bit fields are separate MMAs whose
-//    activations carry the power of two that puts every part in units of
-//    c6 / 16; columns 2t, 2t+1 hold sub-blocks q, q + 2 (two passes).
+//  * q6_K, item = 16 rows x 1 block: one MMA per 16-value sub-block j; the
+//    four lanes of a row read consecutive words of the same ql / qh pieces
+//    (no bank conflicts), merge nibble and 2-bit field into the 6-bit code
+//    with two LOP3s, and the MMA lands in column j mod 8: only the lanes of
+//    that column select their (preloaded) activations, the rest feed zeros.
 //  * q4_K, item = 16 rows x 1 block: lane t owns values 64t..64t+63 and
 //    multiplies its 4-bit codes by the 6-bit scale exactly in binary16
 //    (q sc <= 945); one column per token; the min term is one more MMA on
@@ -112,6 +112,20 @@ __device__ __forceinline__ bool spin_wait(uint64_t* bar, uint32_t parity, int* s
     for (int i = 0;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255) == 255 && global_ns() - t0 > kWaitLimitNs) {
+            if (status) atomicOr(status, KQ_DEV_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Bounded wait that lets the warp sleep until the phase completes (the
+// producer: it must not take issue slots from the decoding warps).
+__device__ __forceinline__ bool sleep_wait(uint64_t* bar, uint32_t parity, int* status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity)) return true;
+        if (global_ns() - t0 > kWaitLimitNs) {
             if (status) atomicOr(status, KQ_DEV_TIMEOUT);
             return false;
         }
@@ -266,122 +280,101 @@ struct Q8 {
 // ===========================================================================
 // q6_K
 // ===========================================================================
+// (a & m) | (b & ~m) in one LOP3.
+__device__ __forceinline__ uint32_t vbitsel(uint32_t a, uint32_t b, uint32_t m) {
+    uint32_t d;
+    asm volatile("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(d) : "r"(a), "r"(b), "r"(m));
+    return d;
+}
+
 template <int NT>
 struct Q6 {
     static constexpr int kVPB = 256, kBPB = 210;
     static constexpr int kItemBlocks = 1;
-    static constexpr uint32_t kBlkImg = 1024;   // image bytes per block and token
-    static constexpr uint32_t kZero = kBlkImg;
+    static constexpr uint32_t kBlkImg = 512;   // image bytes per block and token
+    static constexpr uint32_t kZero = 16;
     static constexpr int kAccPerLane = 2 * NT;
 
-    // 4 words of the 16-byte piece at shared address a (2-byte aligned when
-    // ODD: assembled from 5 aligned words).
+    // Word t of the 16-byte piece at shared address a (2-byte aligned when ODD).
     template <bool ODD>
-    static __device__ __forceinline__ void piece(uint32_t a, uint32_t (&w)[4]) {
-        if constexpr (ODD) {
-            uint32_t u[5];
-#pragma unroll
-            for (int i = 0; i < 5; ++i) u[i] = lds32(a - 2 + 4 * i);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) w[i] = __byte_perm(u[i], u[i + 1], 0x5432);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) w[i] = lds32(a + 4 * i);
-        }
+    static __device__ __forceinline__ uint32_t word(uint32_t a) {
+        if constexpr (ODD) return __byte_perm(lds32(a - 2), lds32(a + 2), 0x5432);
+        else return lds32(a);
     }
 
+    // One block of 16 rows.  Sub-block j = 8h + 2q + lh holds values
+    // v = 128h + 32q + l, l in [16 lh, 16 lh + 16); its 6-bit codes come from
+    // nibble q >> 1 of ql[64h + 32 (q & 1) + l] and bits 2q of qh[32h + l].
+    // One MMA per sub-block: lane t supplies l = 16 lh + 4t + {0..3} of both
+    // rows as 1024 + c6 (q < 2, activations x/16) or 1024 + 16 c6 (q >= 2,
+    // x/256), and the whole MMA lands in column j mod 8, i.e. lanes with
+    // g == j mod 8 supply the activations and all others zeros.
     template <bool ODD>
     static __device__ __forceinline__ void block(const SP& p, uint32_t sb, const Lane& L, uint32_t rowA,
                                                  uint32_t rowB, int gb, float (&acc)[2 * NT]) {
-        const int t = L.t, h = t >> 1, lh = t & 1;
-        const bool act = (L.g >> 1) == t;
-        uint32_t bb[NT][2];
+        const int t = L.t, g = L.g;
+        // activations of this lane's two columns (sub-blocks g and 8 + g)
+        uint2 xb[NT][2];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const uint32_t img = sb + p.off_img + nt * p.img_tok + gb * kBlkImg + 8 * t;
-            const uint32_t zero = sb + p.off_zero + 8 * t;
-            bb[nt][0] = (act && (L.g & 1) == 0) ? img : zero;
-            bb[nt][1] = (act && (L.g & 1) == 1) ? img : zero;
-        }
-        // scales: sc[j], j = 8h + lh + 2q, and 16 d
-        float sc[2][4], d16[2];
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const uint32_t row = r ? rowB : rowA;
+            for (int h = 0; h < 2; ++h)
+                xb[nt][h] = lds64(sb + p.off_img + nt * p.img_tok + gb * kBlkImg + (8 * h + g) * 32 + 8 * t);
+        const float d16[2] = {16.0f * h2f(lds_u16(rowA + 208)), 16.0f * h2f(lds_u16(rowB + 208))};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) sc[r][q] = static_cast<float>(lds_s8(row + 192 + 8 * h + lh + 2 * q));
-            d16[r] = 16.0f * h2f(lds_u16(row + 208));
-        }
-        float D[2][2][NT][4];   // [pass qp][chain][n-tile][element]
-#pragma unroll
-        for (int qp = 0; qp < 2; ++qp)
+        for (int h = 0; h < 2; ++h) {
+            float D[2][NT][4];   // chains by lh
 #pragma unroll
             for (int c = 0; c < 2; ++c)
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) D[qp][c][nt][e] = 0.f;
-        // ql pieces: low nibbles -> q = qp (slot 0, B = x/16), high nibbles ->
-        // q = qp + 2 (slot 1, B = x/256)
+                    for (int e = 0; e < 4; ++e) D[c][nt][e] = 0.f;
 #pragma unroll
-        for (int qp = 0; qp < 2; ++qp) {
-            uint32_t wa[4], wb[4];
-            piece<ODD>(rowA + 64 * h + 32 * qp + 16 * lh, wa);
-            piece<ODD>(rowB + 64 * h + 32 * qp + 16 * lh, wb);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t a8 = wa[k] >> 8, b8 = wb[k] >> 8;
-                const uint32_t L0 = vand_or(wa[k], 0x000F000Fu, kH1024), L1 = vand_or(wb[k], 0x000F000Fu, kH1024);
-                const uint32_t L2 = vand_or(a8, 0x000F000Fu, kH1024), L3 = vand_or(b8, 0x000F000Fu, kH1024);
-                const uint32_t H0 = vand_or(wa[k], 0x00F000F0u, kH1024), H1 = vand_or(wb[k], 0x00F000F0u, kH1024);
-                const uint32_t H2 = vand_or(a8, 0x00F000F0u, kH1024), H3 = vand_or(b8, 0x00F000F0u, kH1024);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const uint2 bl = lds64(bb[nt][0] + 32 * (16 * qp + k));
-                    const uint2 bh = lds64(bb[nt][1] + 32 * (16 * qp + 4 + k));
-                    mma_f16(D[qp][k & 1][nt], L0, L1, L2, L3, bl.x, bl.y);
-                    mma_f16(D[qp][k & 1][nt], H0, H1, H2, H3, bh.x, bh.y);
-                }
-            }
-        }
-        // qh piece: 2-bit field q at bits 2q -> 1024 + 4^q c, B = x / 4^q
-        {
-            uint32_t ha[4], hb[4];
-            piece<ODD>(rowA + 128 + 32 * h + 16 * lh, ha);
-            piece<ODD>(rowB + 128 + 32 * h + 16 * lh, hb);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t a8 = ha[k] >> 8, b8 = hb[k] >> 8;
+            for (int lh = 0; lh < 2; ++lh) {
+                const uint32_t o0 = 64 * h + 16 * lh + 4 * t, o1 = o0 + 32, oh = 128 + 32 * h + 16 * lh + 4 * t;
+                const uint32_t wa[2] = {word<ODD>(rowA + o0), word<ODD>(rowA + o1)};
+                const uint32_t wb[2] = {word<ODD>(rowB + o0), word<ODD>(rowB + o1)};
+                const uint32_t ha = word<ODD>(rowA + oh), hb = word<ODD>(rowB + oh);
+                // 2-bit fields moved next to their nibble: bits 4-5 (q < 2,
+                // after the low nibble) or 8-9 (q >= 2, after the high nibble);
+                // bytes 1 and 3 additionally shifted down by 8
+                const uint32_t sa02[2] = {ha << 4, ha << 2}, sa13[2] = {ha >> 4, ha >> 6};
+                const uint32_t sb02[2] = {hb << 4, hb << 2}, sb13[2] = {hb >> 4, hb >> 6};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const uint32_t mk = 0x00030003u << (2 * q);
-                    const uint32_t A0 = vand_or(ha[k], mk, kH1024), A1 = vand_or(hb[k], mk, kH1024);
-                    const uint32_t A2 = vand_or(a8, mk, kH1024), A3 = vand_or(b8, mk, kH1024);
-                    const int qp = q & 1, sl = q >> 1;
+                    const int qp = q & 1, hi = q >> 1, sh = (q == 0 || q == 2) ? 0 : 1;
+                    const uint32_t M1 = hi ? 0x00F000F0u : 0x000F000Fu, M2 = hi ? 0x03000300u : 0x00300030u;
+                    const uint32_t A0 = vbitsel(wa[qp], vand_or(sa02[sh], M2, kH1024), M1);
+                    const uint32_t A1 = vbitsel(wb[qp], vand_or(sb02[sh], M2, kH1024), M1);
+                    const uint32_t A2 = vbitsel(wa[qp] >> 8, vand_or(sa13[sh], M2, kH1024), M1);
+                    const uint32_t A3 = vbitsel(wb[qp] >> 8, vand_or(sb13[sh], M2, kH1024), M1);
+                    const int jj = 2 * q + lh;   // column of this MMA
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        const uint2 bv = lds64(bb[nt][sl] + 32 * (16 * qp + 8 + 4 * sl + k));
-                        mma_f16(D[qp][(k >> 1) & 1][nt], A0, A1, A2, A3, bv.x, bv.y);
+                        const uint32_t b0 = g == jj ? xb[nt][h].x : 0u, b1 = g == jj ? xb[nt][h].y : 0u;
+                        mma_f16(D[lh][nt], A0, A1, A2, A3, b0, b1);
                     }
                 }
             }
-        }
-        // y += 16 d sc_j (D - C_q X_j), C_q = 1090, 322, 70, 22
+            // columns 2t, 2t+1 = sub-blocks j = 8h + 2t + {0, 1} (q = t):
+            // y += 16 d sc_j (D - C X_j), C = 66 (q < 2) or 6 (q >= 2)
+            const float C = t < 2 ? 66.0f : 6.0f;
+            const int j0 = 8 * h + 2 * t;
+            const float sc[2][2] = {{static_cast<float>(lds_s8(rowA + 192 + j0)), static_cast<float>(lds_s8(rowA + 193 + j0))},
+                                    {static_cast<float>(lds_s8(rowB + 192 + j0)), static_cast<float>(lds_s8(rowB + 193 + j0))}};
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const uint4 xv = lds128(sb + p.off_xs + nt * p.xs_tok + gb * 64 + 16 * t);
-            const float Xq[4] = {__uint_as_float(xv.x), __uint_as_float(xv.y), __uint_as_float(xv.z),
-                                 __uint_as_float(xv.w)};
-#pragma unroll
-            for (int qp = 0; qp < 2; ++qp)
+            for (int nt = 0; nt < NT; ++nt) {
+                const uint2 xv = lds64(sb + p.off_xs + nt * p.xs_tok + (gb * 16 + j0) * 4);
+                const float X[2] = {__uint_as_float(xv.x), __uint_as_float(xv.y)};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int r = e >> 1, q = qp + 2 * (e & 1);
-                    const float C = q == 0 ? 1090.0f : (q == 1 ? 322.0f : (q == 2 ? 70.0f : 22.0f));
-                    const float Ds = D[qp][0][nt][e] + D[qp][1][nt][e];
-                    const float s = __fmul_rn(d16[r], sc[r][q]);
-                    acc[2 * nt + r] = fmaf(s, fmaf(-C, Xq[q], Ds), acc[2 * nt + r]);
+                    const int r = e >> 1, c = e & 1;
+                    const float Ds = D[0][nt][e] + D[1][nt][e];
+                    const float s = __fmul_rn(d16[r], sc[r][c]);
+                    acc[2 * nt + r] = fmaf(s, fmaf(-C, X[c], Ds), acc[2 * nt + r]);
                 }
+            }
         }
     }
 
@@ -395,33 +388,30 @@ struct Q6 {
         Q8<NT>::store_part(p, L, acc, part);
     }
 
-    // Image entry (block, E, t'): E = 16 qp + 4 kind + k; kind 0 = low nibble
-    // (q = qp, x/16), 1 = high nibble (q = qp + 2, x/256), 2 / 3 = 2-bit
-    // field q = qp / qp + 2 (x / 4^q).  Word k of quarter t' holds
-    // l = 16 lh + 4k + b, value v = 128 h + 32 q + l.
-    // X[tok][block][t'][q] = sum over the 16 l of binary16(x[v]).
+    // Image entry (block, j, t') = binary16 of x[v] / 16 (q < 2) or / 256
+    // (q >= 2) for l = 16 lh + 4 t' + {0, 2 | 1, 3}, j = 8h + 2q + lh.
+    // X[tok][block][j] = sum over the 16 l of binary16(x[v]).
     static __device__ void build(const SP& p, uint32_t sb, float& amax) {
-        const int per_tok = p.nblk * 32 * 4;
+        const int per_tok = p.nblk * 16 * 4;
         for (int e = threadIdx.x; e < p.m * per_tok; e += kCW * 32) {
             const int tok = e / per_tok, rem = e % per_tok;
-            const int blk = rem >> 7, E = (rem >> 2) & 31, tt = rem & 3;
-            const int h = tt >> 1, lh = tt & 1, qp = E >> 4, kind = (E >> 2) & 3, kk = E & 3;
-            const int q = qp + 2 * (kind & 1);
-            const float sc = kind == 0 ? 0.0625f : (kind == 1 ? 0.00390625f : 1.0f / static_cast<float>(1 << (2 * q)));
-            const int64_t v0 = static_cast<int64_t>(blk) * 256 + 128 * h + 32 * q + 16 * lh + 4 * kk;
+            const int blk = rem >> 6, j = (rem >> 2) & 15, tt = rem & 3;
+            const int h = j >> 3, q = (j >> 1) & 3, lh = j & 1;
+            const float sc = q < 2 ? 0.0625f : 0.00390625f;
+            const int64_t v0 = static_cast<int64_t>(blk) * 256 + 128 * h + 32 * q + 16 * lh + 4 * tt;
             const uint2 xr = lds64(xaddr(p, sb, tok, v0));
             const float xf[4] = {bf16lo_to_f32(xr.x), bf16hi_to_f32(xr.x), bf16lo_to_f32(xr.y), bf16hi_to_f32(xr.y)};
             __half hv[4];
 #pragma unroll
             for (int b = 0; b < 4; ++b) hv[b] = hx(xf[b] * sc, amax);
-            sts64(sb + p.off_img + tok * p.img_tok + blk * kBlkImg + E * 32 + tt * 8, hpair(hv[0], hv[2]),
+            sts64(sb + p.off_img + tok * p.img_tok + blk * kBlkImg + j * 32 + tt * 8, hpair(hv[0], hv[2]),
                   hpair(hv[1], hv[3]));
         }
         const int per_tok_x = p.nblk * 16;
         for (int e = threadIdx.x; e < p.m * per_tok_x; e += kCW * 32) {
             const int tok = e / per_tok_x, rem = e % per_tok_x;
-            const int blk = rem >> 4, tt = (rem >> 2) & 3, q = rem & 3;
-            const int h = tt >> 1, lh = tt & 1;
+            const int blk = rem >> 4, j = rem & 15;
+            const int h = j >> 3, q = (j >> 1) & 3, lh = j & 1;
             const uint32_t xs = xaddr(p, sb, tok, blk * 256 + 128 * h + 32 * q + 16 * lh);
             float X = 0.f;
 #pragma unroll
@@ -434,7 +424,7 @@ struct Q6 {
                     X += __half2float(__float2half_rn(bf16hi_to_f32(wv[u])));
                 }
             }
-            sts32(sb + p.off_xs + tok * p.xs_tok + (blk * 16 + tt * 4 + q) * 4, __float_as_uint(X));
+            sts32(sb + p.off_xs + tok * p.xs_tok + (blk * 16 + j) * 4, __float_as_uint(X));
         }
     }
 };
@@ -616,7 +606,9 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
     if (tid < kMaxGroups) grp_done[tid] = 0;
     __syncthreads();
     // Programmatic dependent launch: the next kernel may start its prologue;
-    // this one waits for the earlier grids before it reads x or W.
+    // this one waits for the earlier grids before it reads x or W.  (Asking L2
+    // for the first weight stages before the wait was measured to slow down
+    // the tail of the earlier grid more than it gained.)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
@@ -635,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
             const int rv = static_cast<int>(r1 - row0 < kRows ? r1 - row0 : kRows);
             for (int st = 0; st < p.spr; ++st, ++q) {
                 const int slot = q % p.ns;
-                if (lane == 0 && q >= p.ns) ok = spin_wait(&empty[slot], ((q / p.ns) & 1) ^ 1, p.status);
+                if (lane == 0 && q >= p.ns) ok = sleep_wait(&empty[slot], ((q / p.ns) & 1) ^ 1, p.status);
                 ok = __shfl_sync(0xffffffffu, ok, 0) && !*abort_flag;
                 if (!ok) {
                     *abort_flag = 1;
@@ -814,7 +806,7 @@ int launch_qmv_stream(int type, const void* w, int64_t n, int64_t k, const uint1
     case KQ_Q6_K: {
         const int nblk = static_cast<int>(k / 256);
         if (m > 2 || nblk % 8 != 0) return KQ_ERR_UNSUPPORTED;
-        const uint32_t it = nblk * Q6<1>::kBlkImg, xt = nblk * 64;
+        const uint32_t it = nblk * Q6<1>::kBlkImg, xt = nblk * 16 * 4;
         return m == 1 ? launch_stream<Q6<1>>(w, n, k, x, m, y, s, it, xt) : launch_stream<Q6<2>>(w, n, k, x, m, y, s, it, xt);
     }
     case KQ_Q4_K: {
