@@ -61,6 +61,7 @@ struct SP {
     int* status;
     int64_t n, k, row_bytes;
     int m, nblk, g, spr, ns;
+    int x_global;   // 1: build the image from x in global memory (no room for a raw copy)
     uint32_t rs;   // shared-memory stride of a stage row
     uint32_t off_stage, off_img, img_tok, off_xs, xs_tok, off_zero, off_part, off_xraw;
 };
@@ -544,14 +545,17 @@ struct Q4 {
         for (int it = threadIdx.x; it < items; it += kCW * 32) {
             const int tok = it / (p.nblk * 4), rem = it % (p.nblk * 4), bl = rem >> 2, t = rem & 3;
             const uint32_t base = sb + p.off_img + tok * p.img_tok + bl * kBlkImg;
-            const uint32_t xs = xaddr(p, sb, tok, static_cast<int64_t>(bl) * 256 + 64 * t);
+            const int64_t xi = static_cast<int64_t>(bl) * 256 + 64 * t;
+            const uint32_t xs = xaddr(p, sb, tok, xi);
+            const uint16_t* xg = p.x + static_cast<int64_t>(tok) * p.k + xi;
             float X[2] = {0.f, 0.f};
 #pragma unroll
             for (int nib = 0; nib < 2; ++nib) {
 #pragma unroll
                 for (int uu = 0; uu < 2; ++uu) {
-                    const uint4 r0 = lds128(xs + 2 * (32 * nib + 16 * uu));
-                    const uint4 r1 = lds128(xs + 2 * (32 * nib + 16 * uu + 8));
+                    const int o = 32 * nib + 16 * uu;
+                    const uint4 r0 = p.x_global ? ldg_nc_v4(xg + o) : lds128(xs + 2 * o);
+                    const uint4 r1 = p.x_global ? ldg_nc_v4(xg + o + 8) : lds128(xs + 2 * (o + 8));
                     const uint32_t wv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
@@ -615,10 +619,14 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
     if (warp == kProd) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
-            const uint32_t row = 2u * static_cast<uint32_t>(p.k);
-            mbar_arrive_expect_tx(xbar, row * p.m);
-            for (int tok = 0; tok < p.m; ++tok)
-                bulk_g2s(smem + p.off_xraw + tok * row, p.x + static_cast<int64_t>(tok) * p.k, row, xbar);
+            if (p.x_global) {
+                mbar_arrive(xbar);
+            } else {
+                const uint32_t row = 2u * static_cast<uint32_t>(p.k);
+                mbar_arrive_expect_tx(xbar, row * p.m);
+                for (int tok = 0; tok < p.m; ++tok)
+                    bulk_g2s(smem + p.off_xraw + tok * row, p.x + static_cast<int64_t>(tok) * p.k, row, xbar);
+            }
         }
         int q = 0;
         bool ok = true;
@@ -751,7 +759,11 @@ int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m,
     p.off_part = align16(p.off_zero + C::kZero);
     p.off_xraw = p.off_part;   // the raw x copy is dead before any partial sum is written
     const uint32_t part = static_cast<uint32_t>(nrg_max) * kCW * kRows * m * 4;
-    const uint32_t xraw = static_cast<uint32_t>(m) * static_cast<uint32_t>(k) * 2;
+    uint32_t xraw = static_cast<uint32_t>(m) * static_cast<uint32_t>(k) * 2;
+    // q4_K can build its image from global memory when the raw copy would
+    // crowd out the weight stages
+    p.x_global = (C::kBPB == 144 && p.off_part + xraw + 2u * kRows * 2048u > optin) ? 1 : 0;
+    if (p.x_global) xraw = 0;
     p.off_stage = (p.off_part + (part > xraw ? part : xraw) + 127u) & ~127u;
     // stage geometry: whole rows if two or more stages fit, else the fewest
     // equal row slices (a multiple of the item size, copies 16-byte sized)
