@@ -28,11 +28,12 @@
 //    codes of the even block only (its fp16 scale bytes and the odd block's
 //    get a zero activation), words 9..16 those of the odd block, so MMA
 //    column 2t + parity collects exactly lane t's block of that parity.
-//  * q6_K, item = 16 rows x 1 block: one MMA per 16-value sub-block j; the
-//    four lanes of a row read consecutive words of the same ql / qh pieces
-//    (no bank conflicts), merge nibble and 2-bit field into the 6-bit code
-//    with two LOP3s, and the MMA lands in column j mod 8: only the lanes of
-//    that column select their (preloaded) activations, the rest feed zeros.
+//  * q6_K, item = 16 rows x 1 block: lane t owns a quarter (half h, 16-value
+//    run lh) of the block for all four q; nibble and 2-bit field are merged
+//    into the 6-bit code with two LOP3s; columns 2t, 2t+1 hold its low- and
+//    high-nibble sub-blocks of the current pass.  The four lanes of a row read
+//    their words in a rotated order, which keeps the loads free of bank
+//    conflicts.
 //  * q4_K, item = 16 rows x 1 block: lane t owns values 64t..64t+63 and
 //    multiplies its 4-bit codes by the 6-bit scale exactly in binary16
 //    (q sc <= 945); one column per token; the min term is one more MMA on
@@ -293,87 +294,105 @@ struct Q6 {
     static constexpr int kVPB = 256, kBPB = 210;
     static constexpr int kItemBlocks = 1;
     static constexpr uint32_t kBlkImg = 512;   // image bytes per block and token
-    static constexpr uint32_t kZero = 16;
+    static constexpr uint32_t kZero = 512;
     static constexpr int kAccPerLane = 2 * NT;
 
-    // Word t of the 16-byte piece at shared address a (2-byte aligned when ODD).
+    // Word at shared address a (2-byte aligned when ODD).
     template <bool ODD>
     static __device__ __forceinline__ uint32_t word(uint32_t a) {
         if constexpr (ODD) return __byte_perm(lds32(a - 2), lds32(a + 2), 0x5432);
         else return lds32(a);
     }
 
-    // One block of 16 rows.  Sub-block j = 8h + 2q + lh holds values
-    // v = 128h + 32q + l, l in [16 lh, 16 lh + 16); its 6-bit codes come from
-    // nibble q >> 1 of ql[64h + 32 (q & 1) + l] and bits 2q of qh[32h + l].
-    // One MMA per sub-block: lane t supplies l = 16 lh + 4t + {0..3} of both
-    // rows as 1024 + c6 (q < 2, activations x/16) or 1024 + 16 c6 (q >= 2,
-    // x/256), and the whole MMA lands in column j mod 8, i.e. lanes with
-    // g == j mod 8 supply the activations and all others zeros.
+    // One block of 16 rows.  Lane t owns quarter (h = t >> 1, lh = t & 1):
+    // values v = 128h + 32q + l, l in [16 lh, 16 lh + 16), all four q, i.e.
+    // sub-blocks j = 8h + 2q + lh.  Its 6-bit codes come from nibble q >> 1 of
+    // ql[64h + 32 (q & 1) + l] and bits 2q of qh[32h + l].  For each pass
+    // qp = q & 1 and word k the lane feeds two MMAs: the low nibbles (q = qp,
+    // 1024 + c6, activations x/16) into column 2t and the high nibbles
+    // (q = qp + 2, 1024 + 16 c6, x/256) into column 2t + 1.  The four lanes of
+    // a row read their words in the order (k + t) mod 4, which spreads them over
+    // all 32 banks; the activation image follows the same order.
     template <bool ODD>
     static __device__ __forceinline__ void block(const SP& p, uint32_t sb, const Lane& L, uint32_t rowA,
                                                  uint32_t rowB, int gb, float (&acc)[2 * NT]) {
-        const int t = L.t, g = L.g;
-        // activations of this lane's two columns (sub-blocks g and 8 + g)
-        uint2 xb[NT][2];
+        const int t = L.t, h = t >> 1, lh = t & 1;
+        const bool act = (L.g >> 1) == t;   // B lanes whose columns hold lane t's sub-blocks
+        uint32_t bb[NT][2];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt < NT; ++nt) {
+            const uint32_t img = sb + p.off_img + nt * p.img_tok + gb * kBlkImg + 8 * t;
+            const uint32_t zero = sb + p.off_zero + 8 * t;
+            bb[nt][0] = (act && (L.g & 1) == 0) ? img : zero;
+            bb[nt][1] = (act && (L.g & 1) == 1) ? img : zero;
+        }
+        // scales of the lane's sub-blocks: sc[8h + 2q + lh], and 16 d
+        float sc[2][4], d16[2];
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-                xb[nt][h] = lds64(sb + p.off_img + nt * p.img_tok + gb * kBlkImg + (8 * h + g) * 32 + 8 * t);
-        const float d16[2] = {16.0f * h2f(lds_u16(rowA + 208)), 16.0f * h2f(lds_u16(rowB + 208))};
+        for (int r = 0; r < 2; ++r) {
+            const uint32_t row = r ? rowB : rowA;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            float D[2][NT][4];   // chains by lh
+            for (int q = 0; q < 4; ++q) sc[r][q] = static_cast<float>(lds_s8(row + 192 + 8 * h + lh + 2 * q));
+            d16[r] = 16.0f * h2f(lds_u16(row + 208));
+        }
+        // the lane's 4 qh words (rows g, g+8), in its rotated order
+        const uint32_t rot[4] = {4u * ((0 + t) & 3), 4u * ((1 + t) & 3), 4u * ((2 + t) & 3), 4u * ((3 + t) & 3)};
+        uint32_t ha[4], hb[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            ha[k] = word<ODD>(rowA + 128 + 32 * h + 16 * lh + rot[k]);
+            hb[k] = word<ODD>(rowB + 128 + 32 * h + 16 * lh + rot[k]);
+        }
+#pragma unroll
+        for (int qp = 0; qp < 2; ++qp) {
+            float D[2][NT][4];   // two chains (k parity)
 #pragma unroll
             for (int c = 0; c < 2; ++c)
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) D[c][nt][e] = 0.f;
+            // field qp (and qp + 2) of each qh byte moved next to its nibble:
+            // bits 4-5 (low nibble) / 8-9 (high nibble); bytes 1 and 3 also >> 8
+            constexpr int kSh[2] = {4, 2};
+            const int sh = kSh[qp];
 #pragma unroll
-            for (int lh = 0; lh < 2; ++lh) {
-                const uint32_t o0 = 64 * h + 16 * lh + 4 * t, o1 = o0 + 32, oh = 128 + 32 * h + 16 * lh + 4 * t;
-                const uint32_t wa[2] = {word<ODD>(rowA + o0), word<ODD>(rowA + o1)};
-                const uint32_t wb[2] = {word<ODD>(rowB + o0), word<ODD>(rowB + o1)};
-                const uint32_t ha = word<ODD>(rowA + oh), hb = word<ODD>(rowB + oh);
-                // 2-bit fields moved next to their nibble: bits 4-5 (q < 2,
-                // after the low nibble) or 8-9 (q >= 2, after the high nibble);
-                // bytes 1 and 3 additionally shifted down by 8
-                const uint32_t sa02[2] = {ha << 4, ha << 2}, sa13[2] = {ha >> 4, ha >> 6};
-                const uint32_t sb02[2] = {hb << 4, hb << 2}, sb13[2] = {hb >> 4, hb >> 6};
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t wa = word<ODD>(rowA + 64 * h + 32 * qp + 16 * lh + rot[k]);
+                const uint32_t wb = word<ODD>(rowB + 64 * h + 32 * qp + 16 * lh + rot[k]);
+                const uint32_t wa8 = wa >> 8, wb8 = wb >> 8;
+                const uint32_t sa02 = ha[k] << sh, sa13 = ha[k] >> (8 - sh);
+                const uint32_t sb02 = hb[k] << sh, sb13 = hb[k] >> (8 - sh);
+                // low nibble + field qp -> 1024 + c6
+                const uint32_t L0 = vbitsel(wa, vand_or(sa02, 0x00300030u, kH1024), 0x000F000Fu);
+                const uint32_t L1 = vbitsel(wb, vand_or(sb02, 0x00300030u, kH1024), 0x000F000Fu);
+                const uint32_t L2 = vbitsel(wa8, vand_or(sa13, 0x00300030u, kH1024), 0x000F000Fu);
+                const uint32_t L3 = vbitsel(wb8, vand_or(sb13, 0x00300030u, kH1024), 0x000F000Fu);
+                // high nibble + field qp + 2 -> 1024 + 16 c6
+                const uint32_t H0 = vbitsel(wa, vand_or(sa02, 0x03000300u, kH1024), 0x00F000F0u);
+                const uint32_t H1 = vbitsel(wb, vand_or(sb02, 0x03000300u, kH1024), 0x00F000F0u);
+                const uint32_t H2 = vbitsel(wa8, vand_or(sa13, 0x03000300u, kH1024), 0x00F000F0u);
+                const uint32_t H3 = vbitsel(wb8, vand_or(sb13, 0x03000300u, kH1024), 0x00F000F0u);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int qp = q & 1, hi = q >> 1, sh = (q == 0 || q == 2) ? 0 : 1;
-                    const uint32_t M1 = hi ? 0x00F000F0u : 0x000F000Fu, M2 = hi ? 0x03000300u : 0x00300030u;
-                    const uint32_t A0 = vbitsel(wa[qp], vand_or(sa02[sh], M2, kH1024), M1);
-                    const uint32_t A1 = vbitsel(wb[qp], vand_or(sb02[sh], M2, kH1024), M1);
-                    const uint32_t A2 = vbitsel(wa[qp] >> 8, vand_or(sa13[sh], M2, kH1024), M1);
-                    const uint32_t A3 = vbitsel(wb[qp] >> 8, vand_or(sb13[sh], M2, kH1024), M1);
-                    const int jj = 2 * q + lh;   // column of this MMA
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const uint32_t b0 = g == jj ? xb[nt][h].x : 0u, b1 = g == jj ? xb[nt][h].y : 0u;
-                        mma_f16(D[lh][nt], A0, A1, A2, A3, b0, b1);
-                    }
+                for (int nt = 0; nt < NT; ++nt) {
+                    const uint2 bl = lds64(bb[nt][0] + 32 * (8 * qp + k));
+                    const uint2 bh = lds64(bb[nt][1] + 32 * (8 * qp + 4 + k));
+                    mma_f16(D[k & 1][nt], L0, L1, L2, L3, bl.x, bl.y);
+                    mma_f16(D[k & 1][nt], H0, H1, H2, H3, bh.x, bh.y);
                 }
             }
-            // columns 2t, 2t+1 = sub-blocks j = 8h + 2t + {0, 1} (q = t):
-            // y += 16 d sc_j (D - C X_j), C = 66 (q < 2) or 6 (q >= 2)
-            const float C = t < 2 ? 66.0f : 6.0f;
-            const int j0 = 8 * h + 2 * t;
-            const float sc[2][2] = {{static_cast<float>(lds_s8(rowA + 192 + j0)), static_cast<float>(lds_s8(rowA + 193 + j0))},
-                                    {static_cast<float>(lds_s8(rowB + 192 + j0)), static_cast<float>(lds_s8(rowB + 193 + j0))}};
+            // columns 2t (q = qp, C = 66) and 2t + 1 (q = qp + 2, C = 6):
+            // y += 16 d sc_j (D - C X_j)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                const uint2 xv = lds64(sb + p.off_xs + nt * p.xs_tok + (gb * 16 + j0) * 4);
+                const uint2 xv = lds64(sb + p.off_xs + nt * p.xs_tok + ((gb * 4 + t) * 4 + 2 * qp) * 4);
                 const float X[2] = {__uint_as_float(xv.x), __uint_as_float(xv.y)};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int r = e >> 1, c = e & 1;
                     const float Ds = D[0][nt][e] + D[1][nt][e];
-                    const float s = __fmul_rn(d16[r], sc[r][c]);
-                    acc[2 * nt + r] = fmaf(s, fmaf(-C, X[c], Ds), acc[2 * nt + r]);
+                    const float s = __fmul_rn(d16[r], sc[r][qp + 2 * c]);
+                    acc[2 * nt + r] = fmaf(s, fmaf(c ? -6.0f : -66.0f, X[c], Ds), acc[2 * nt + r]);
                 }
             }
         }
@@ -389,30 +408,32 @@ struct Q6 {
         Q8<NT>::store_part(p, L, acc, part);
     }
 
-    // Image entry (block, j, t') = binary16 of x[v] / 16 (q < 2) or / 256
-    // (q >= 2) for l = 16 lh + 4 t' + {0, 2 | 1, 3}, j = 8h + 2q + lh.
-    // X[tok][block][j] = sum over the 16 l of binary16(x[v]).
+    // Image entry (block, E = 8 qp + 4 s + k, t'): binary16 of x[v] / 16
+    // (s = 0) or / 256 (s = 1) for q = qp + 2s, l = 16 lh + 4 ((k + t') mod 4)
+    // + {0, 2 | 1, 3}, v = 128h + 32q + l (h, lh of quarter t').
+    // X[tok][block][t'][qp][s] = sum over the 16 l of binary16(x[v]).
     static __device__ void build(const SP& p, uint32_t sb, float& amax) {
         const int per_tok = p.nblk * 16 * 4;
         for (int e = threadIdx.x; e < p.m * per_tok; e += kCW * 32) {
             const int tok = e / per_tok, rem = e % per_tok;
-            const int blk = rem >> 6, j = (rem >> 2) & 15, tt = rem & 3;
-            const int h = j >> 3, q = (j >> 1) & 3, lh = j & 1;
-            const float sc = q < 2 ? 0.0625f : 0.00390625f;
-            const int64_t v0 = static_cast<int64_t>(blk) * 256 + 128 * h + 32 * q + 16 * lh + 4 * tt;
+            const int blk = rem >> 6, E = (rem >> 2) & 15, tt = rem & 3;
+            const int h = tt >> 1, lh = tt & 1, qp = E >> 3, sl = (E >> 2) & 1, kk = E & 3;
+            const int q = qp + 2 * sl;
+            const float sc = sl ? 0.00390625f : 0.0625f;
+            const int64_t v0 = static_cast<int64_t>(blk) * 256 + 128 * h + 32 * q + 16 * lh + 4 * ((kk + tt) & 3);
             const uint2 xr = lds64(xaddr(p, sb, tok, v0));
             const float xf[4] = {bf16lo_to_f32(xr.x), bf16hi_to_f32(xr.x), bf16lo_to_f32(xr.y), bf16hi_to_f32(xr.y)};
             __half hv[4];
 #pragma unroll
             for (int b = 0; b < 4; ++b) hv[b] = hx(xf[b] * sc, amax);
-            sts64(sb + p.off_img + tok * p.img_tok + blk * kBlkImg + j * 32 + tt * 8, hpair(hv[0], hv[2]),
+            sts64(sb + p.off_img + tok * p.img_tok + blk * kBlkImg + E * 32 + tt * 8, hpair(hv[0], hv[2]),
                   hpair(hv[1], hv[3]));
         }
         const int per_tok_x = p.nblk * 16;
         for (int e = threadIdx.x; e < p.m * per_tok_x; e += kCW * 32) {
             const int tok = e / per_tok_x, rem = e % per_tok_x;
-            const int blk = rem >> 4, j = rem & 15;
-            const int h = j >> 3, q = (j >> 1) & 3, lh = j & 1;
+            const int blk = rem >> 4, tt = (rem >> 2) & 3, qp = (rem >> 1) & 1, sl = rem & 1;
+            const int h = tt >> 1, lh = tt & 1, q = qp + 2 * sl;
             const uint32_t xs = xaddr(p, sb, tok, blk * 256 + 128 * h + 32 * q + 16 * lh);
             float X = 0.f;
 #pragma unroll
@@ -425,7 +446,7 @@ struct Q6 {
                     X += __half2float(__float2half_rn(bf16hi_to_f32(wv[u])));
                 }
             }
-            sts32(sb + p.off_xs + tok * p.xs_tok + (blk * 16 + j) * 4, __float_as_uint(X));
+            sts32(sb + p.off_xs + tok * p.xs_tok + (blk * 16 + tt * 4 + qp * 2 + sl) * 4, __float_as_uint(X));
         }
     }
 };

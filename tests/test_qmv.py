@@ -51,6 +51,13 @@ def test_c2_q4K_4096x14336(m):
     run(kq.Q4_K, 4096, 14336, m, seed=synth.SEED_W)
 
 
+@pytest.mark.parametrize("m", [7, 9, 16])
+def test_q4K_long_k_many_tokens(m):
+    # an activation image of m x K that does not fit in shared memory at once:
+    # the decode kernel walks K in chunks (two images in turn); ragged N
+    run(kq.Q4_K, 200, 8192, m, seed=40 + m)
+
+
 @pytest.mark.parametrize("qtype", CODECS)
 def test_deterministic_and_row_independent(qtype):
     n, k = 200, 4096
