@@ -67,6 +67,14 @@ struct SP {
     uint32_t off_stage, off_img, img_tok, off_xs, xs_tok, off_zero, off_part, off_xraw;
 };
 
+// Row groups are walked with a partial last group (fewer than 16 rows) moved
+// to the front: its small stage lands first and its decode overlaps the full
+// stages still in flight instead of trailing the kernel.
+__device__ __forceinline__ int group_order(int rg, int nrg, int64_t rows) {
+    if (nrg < 2 || rows % kRows == 0) return rg;
+    return rg == 0 ? nrg - 1 : rg - 1;
+}
+
 constexpr uint32_t kH1024 = 0x64006400u;    // binary16 (1024, 1024)
 constexpr uint32_t kHm1024 = 0xE400E400u;   // (-1024, -1024)
 constexpr uint32_t kH1_16 = 0x2C002C00u;    // (1/16, 1/16)
@@ -652,7 +660,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
         int q = 0;
         bool ok = true;
         for (int rg = 0; rg < nrg && ok; ++rg) {
-            const int64_t row0 = r0 + static_cast<int64_t>(rg) * kRows;
+            const int64_t row0 = r0 + static_cast<int64_t>(group_order(rg, nrg, r1 - r0)) * kRows;
             const int rv = static_cast<int>(r1 - row0 < kRows ? r1 - row0 : kRows);
             for (int st = 0; st < p.spr; ++st, ++q) {
                 const int slot = q % p.ns;
@@ -696,7 +704,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
         const int items_per_row = p.nblk / C::kItemBlocks;
         int q = 0;
         for (int rg = 0; rg < nrg && !*abort_flag; ++rg) {
-            const int64_t row0 = r0 + static_cast<int64_t>(rg) * kRows;
+            const int64_t row0 = r0 + static_cast<int64_t>(group_order(rg, nrg, r1 - r0)) * kRows;
             const int rv = static_cast<int>(r1 - row0 < kRows ? r1 - row0 : kRows);
             float acc[C::kAccPerLane];
 #pragma unroll
