@@ -268,11 +268,11 @@ __device__ __forceinline__ void q4k_block(const Lane<NT>& L, uint32_t rowA, uint
     }
     const uint32_t wA[8] = {qA0.x, qA0.y, qA0.z, qA0.w, qA1.x, qA1.y, qA1.z, qA1.w};
     const uint32_t wB[8] = {qB0.x, qB0.y, qB0.z, qB0.w, qB1.x, qB1.y, qB1.z, qB1.w};
-    float D[NT][4], Dm[NT][4];
+    float D[2][NT][4], Dm[NT][4];   // two independent MMA chains (word parity)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) D[nt][e] = Dm[nt][e] = 0.f;
+        for (int e = 0; e < 4; ++e) D[0][nt][e] = D[1][nt][e] = Dm[nt][e] = 0.f;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
         const uint32_t a = wA[u], b = wB[u], a8 = a >> 8, b8 = b >> 8;
@@ -285,7 +285,7 @@ __device__ __forceinline__ void q4k_block(const Lane<NT>& L, uint32_t rowA, uint
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const uint2 bv = lds64c(L.tokb[nt] + imgb + u * 32 + t * 8);
-                mma_f16(D[nt], a0, a1, a2, a3, bv.x, bv.y);
+                mma_f16(D[u & 1][nt], a0, a1, a2, a3, bv.x, bv.y);
             }
         }
         // high nibbles: 1024 + 16q, times sc/16, minus 64 sc -> q*sc exactly
@@ -297,7 +297,7 @@ __device__ __forceinline__ void q4k_block(const Lane<NT>& L, uint32_t rowA, uint
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const uint2 bv = lds64c(L.tokb[nt] + imgb + (8 + u) * 32 + t * 8);
-                mma_f16(D[nt], a0, a1, a2, a3, bv.x, bv.y);
+                mma_f16(D[u & 1][nt], a0, a1, a2, a3, bv.x, bv.y);
             }
         }
     }
@@ -308,7 +308,7 @@ __device__ __forceinline__ void q4k_block(const Lane<NT>& L, uint32_t rowA, uint
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int r = e >> 1;
-            acc[nt][e] = fmaf(dd[r], D[nt][e], fmaf(-dm[r], Dm[nt][e], acc[nt][e]));
+            acc[nt][e] = fmaf(dd[r], D[0][nt][e] + D[1][nt][e], fmaf(-dm[r], Dm[nt][e], acc[nt][e]));
         }
     }
 }
