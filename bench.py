@@ -60,21 +60,31 @@ def peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def kernel_source_hash() -> str:
+# source files that define the kernel behind each roofline tag (the shared
+# device header and launch declarations included)
+KERNEL_SOURCES = {
+    "qmv_q8_0_m1_14336x4096": ("kq_qmv_stream.cu", "kq_device.cuh", "kq_launch.h"),
+    "qmv_q6_K_m1_14336x4096": ("kq_qmv_stream.cu", "kq_device.cuh", "kq_launch.h"),
+}
+
+
+def kernel_source_hash(tag: str | None = None) -> str:
+    """Hash of the kernel sources (of one roofline tag's kernel, or of all)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gguf_quant_dequant_q4_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    files = KERNEL_SOURCES.get(tag) if tag else None
+    for f in sorted(files or os.listdir(csrc)):
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(kernel_tag: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources (profiles/*.txt lines 'traffic <tag> <bytes> <hash>')."""
+    the current sources of that kernel (profiles/*.txt lines 'traffic <tag> <bytes> <hash>')."""
     d = os.path.join(ROOT, "profiles")
     if not os.path.isdir(d):
         return None
-    cur = kernel_source_hash()
+    cur = kernel_source_hash(kernel_tag)
     for f in sorted(os.listdir(d)):
         if not f.endswith((".txt", ".md")):
             continue
