@@ -37,21 +37,25 @@ constexpr int kBM = 128;          // weight rows per tile (MMA M)
 constexpr int kBN = 256;          // activation rows per tile (MMA N max)
 constexpr int kBK = 64;           // K per pipeline step (one 128-byte swizzle row)
 constexpr int kRawStages = 2;     // raw weight stages, 256 values each
-constexpr int kBStages = 3;
 constexpr int kMaxTiles = 1024;   // map tiles a gather call may use
 constexpr uint32_t kHeader = 5120; // barriers, misc words, tile tables
 constexpr int kEpiWarp0 = 2, kDeqWarp0 = 6;
 
 template <int QT> struct QmmCodec;
+// raw row bytes per stage, A (decoded) stages, B (activation) stages
 template <> struct QmmCodec<KQ_Q4_K> {
-    static constexpr int RAWB = 144, AST = 4;         // raw row bytes per stage, A stages
+    static constexpr int RAWB = 144, AST = 3, BST = 4;
 };
 template <> struct QmmCodec<KQ_Q6_K> {
-    static constexpr int RAWB = 240, AST = 4;         // 210-byte block at offset 210b mod 16
+    static constexpr int RAWB = 240, AST = 2, BST = 4;   // 210-byte block at offset 210b mod 16
 };
 template <> struct QmmCodec<KQ_Q8_0> {
-    static constexpr int RAWB = 272, AST = 3;         // eight 34-byte blocks
+    static constexpr int RAWB = 272, AST = 3, BST = 3;   // eight 34-byte blocks
 };
+template <int QT>
+constexpr bool fits_barriers() { return QmmCodec<QT>::AST <= 4 && QmmCodec<QT>::BST <= 4; }
+static_assert(fits_barriers<KQ_Q4_K>() && fits_barriers<KQ_Q6_K>() && fits_barriers<KQ_Q8_0>(),
+              "barrier table holds at most 4 A and 4 B stages");
 
 struct Smem {
     static constexpr uint32_t kBars = 0;      // mbarriers
@@ -65,7 +69,9 @@ struct QmmParams {
     int k;
     int n_experts;        // 0 = dense qmm
     int ntn;              // weight tiles per expert = ceil(n / 128)
-    int units;            // dense: ceil(m/256) * ntn
+    int units;            // dense: full units, then the tail's 64-row sub-units
+    int units_main;       // dense: units covered by whole rounds of the grid
+    int split;            // dense: sub-units per unit of the last round (1, 2 or 4)
     const uint32_t* map;
     const uint32_t* count;
     int64_t cap;
@@ -397,6 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                const QmmParams p) {
     using C = QmmCodec<QT>;
     constexpr int AST = C::AST;
+    constexpr int kBStages = C::BST;
     constexpr uint32_t kRawBytes = kBM * C::RAWB;
     constexpr uint32_t kABytes = kBM * kBK * 2;    // 16 KB
     constexpr uint32_t kBBytes = kBN * kBK * 2;    // 32 KB
@@ -412,9 +419,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* a_full = bars + 4;
     uint64_t* a_empty = bars + 8;
     uint64_t* b_full = bars + 12;
-    uint64_t* b_empty = bars + 15;
-    uint64_t* acc_full = bars + 18;
-    uint64_t* acc_empty = bars + 20;
+    uint64_t* b_empty = bars + 16;
+    uint64_t* acc_full = bars + 20;
+    uint64_t* acc_empty = bars + 22;
     volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + Smem::kMisc);
     // misc[0] tmem base, misc[1] abort, misc[2] number of chunks, misc[3] tiles
     uint16_t* tiles = reinterpret_cast<uint16_t*>(smem + Smem::kTiles);          // sorted valid tile ids
@@ -514,12 +521,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     auto get_unit = [&](int u, Unit& U) {
         if (p.n_experts == 0) {
+            // units below units_main: (256 activation rows, weight tile); the
+            // units of the last, partial round of the grid are split into
+            // `split` sub-units of 256/split rows so that they spread over
+            // more SMs (a sub-unit past the end of m has nt = 0: skipped)
             const int mtiles = static_cast<int>((p.m + kBN - 1) / kBN);
-            const int mt = u % mtiles;
+            int fu = u, sub = -1;
+            if (u >= p.units_main) {
+                fu = p.units_main + (u - p.units_main) / p.split;
+                sub = (u - p.units_main) % p.split;
+            }
+            const int mt = fu % mtiles;
             U.e = 0;
-            U.ntile = u / mtiles;
-            const int64_t r0 = static_cast<int64_t>(mt) * kBN;
-            const int64_t left = p.m - r0;
+            U.ntile = fu / mtiles;
+            int64_t r0 = static_cast<int64_t>(mt) * kBN;
+            int64_t left = p.m - r0;
+            if (sub >= 0) {
+                const int rows = kBN / p.split;
+                r0 += static_cast<int64_t>(rows) * sub;
+                left = left - static_cast<int64_t>(rows) * sub;
+                left = left < 0 ? 0 : (left > rows ? rows : left);
+            }
             U.nt = static_cast<int>(left >= kBN ? 4 : (left + 63) / 64);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -573,6 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int u = blockIdx.x; u < total_units && !aborted(); u += gridDim.x) {
                 Unit U;
                 get_unit(u, U);
+                if (U.nt == 0) continue;
                 const int wrow = U.e * static_cast<int>(p.n) + U.ntile * kBM;
                 for (int ks = 0; ks < ksteps; ++ks) {
                     if ((ks & 3) == 0) {
@@ -601,6 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int u = blockIdx.x; u < total_units && !aborted(); u += gridDim.x) {
                 Unit U;
                 get_unit(u, U);
+                if (U.nt == 0) continue;
                 const uint32_t idesc = make_idesc(mma_n(U));
                 if (!bwait(&acc_empty[cp.idx], cp.phase ^ 1)) break;
                 tc_fence_after();
@@ -634,6 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int u = blockIdx.x; u < total_units && !aborted(); u += gridDim.x) {
             Unit U;
             get_unit(u, U);
+            if (U.nt == 0) continue;
             const int nmma = mma_n(U);
             if (!bwait(&acc_full[cp.idx], cp.phase)) break;
             tc_fence_after();
@@ -645,13 +670,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld16(tbase + c0, v);
                 const int ti = c0 >> 6;
                 const int r0 = c0 & 63;
-                if (row_ok) {
+                const int nv = U.nr[ti] - r0;   // valid activation rows of this 16-column chunk
+                if (row_ok && nv > 0) {
+                    // y is written once and never read here: streaming stores
+                    float* yp = p.y + (static_cast<int64_t>(U.rs[ti]) + r0) * p.n + nrow;
+                    if (nv >= 16) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        if (r0 + i < U.nr[ti]) {
-                            const int64_t tok = static_cast<int64_t>(U.rs[ti]) + r0 + i;
-                            p.y[tok * p.n + nrow] = __uint_as_float(v[i]);
-                        }
+                        for (int i = 0; i < 16; ++i) __stcs(yp + i * p.n, __uint_as_float(v[i]));
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (i < nv) __stcs(yp + i * p.n, __uint_as_float(v[i]));
                     }
                 }
             }
@@ -670,6 +699,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         Pipe rp, ap;
         StageScales S;
         for (int u = blockIdx.x; u < total_units && !aborted(); u += gridDim.x) {
+            Unit U;
+            get_unit(u, U);
+            if (U.nt == 0) continue;
             bool ok = true;
             for (int ks0 = 0; ks0 < ksteps && ok; ks0 += 4) {
                 const uint32_t row = rst + rp.idx * kRawBytes + r * C::RAWB;
@@ -769,19 +801,29 @@ int launch_impl(const void* w, int64_t w_rows, int64_t n, int64_t k, const uint1
     p.n_experts = n_experts;
     p.ntn = static_cast<int>((n + kBM - 1) / kBM);
     p.units = n_experts == 0 ? static_cast<int>((x_rows + kBN - 1) / kBN) * p.ntn : 0;
+    p.units_main = p.units;
+    p.split = 1;
     p.map = map;
     p.count = count;
     p.cap = cap;
     p.y = y;
     p.err = err;
     p.status = device_status_ptr();
-    const uint32_t smem = kHeader + 1024 + kBStages * kBN * kBK * 2 + C::AST * kBM * kBK * 2 + kRawStages * kBM * C::RAWB;
+    const uint32_t smem = kHeader + 1024 + C::BST * kBN * kBK * 2 + C::AST * kBM * kBK * 2 + kRawStages * kBM * C::RAWB;
     auto kern = qmm_kernel<QT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return record_cuda(e);
     int grid = device_sm_count();
     if (n_experts == 0 && p.units < grid) grid = p.units;
     if (grid < 1) return KQ_OK;
+    if (n_experts == 0 && p.units > grid && p.units % grid != 0 && x_rows > 64) {
+        // the last, partial round: its units become sub-units, as many per
+        // unit as still fit in one round of the grid
+        const int tail = p.units % grid;
+        p.split = 4 * tail <= grid ? 4 : (2 * tail <= grid ? 2 : 1);
+        p.units_main = p.units - tail;
+        p.units = p.units_main + p.split * tail;
+    }
     kern<<<grid, kThreads, smem, s>>>(wmap, xmap, p);
     return check_launch();
 }

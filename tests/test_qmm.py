@@ -32,6 +32,18 @@ def test_k4096_ragged(qtype):
     run_full(qtype, 257, 4096, 513, seed=11)
 
 
+# (m, n) with more (256-row, 128-weight-row) units than SMs, so that the last
+# partial round of the grid is split: into four 64-row sub-units (m=300,
+# n=10240: 160 units, some sub-units past the end of m), into two 128-row
+# sub-units (m=200, n=25344: 198 units) and not at all (m=100, n=31744: 248
+# units); the split depends on the SM count, all three are covered on 148 SMs
+@pytest.mark.parametrize("qtype", CODECS)
+@pytest.mark.parametrize("m,n", [(300, 10240), (200, 25344), (100, 31744)])
+def test_last_round_split(qtype, m, n):
+    # a q6_K row of K values is a multiple of 16 bytes only when K % 2048 == 0
+    run_full(qtype, n, 2048 if qtype == kq.Q6_K else 256, m, seed=m + 7)
+
+
 @pytest.mark.parametrize("qtype", [kq.Q4_K, kq.Q6_K])
 def test_c3_full_size_sampled(qtype):
     m, n, k = 2048, 14336, 4096
