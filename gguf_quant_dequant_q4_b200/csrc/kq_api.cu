@@ -64,6 +64,14 @@ bool use_pdl() {
     return on;
 }
 
+bool use_pair_mma() {
+    static const bool on = [] {
+        const char* v = std::getenv("KQ_QMM_1SM");
+        return !(v && v[0] == '1');
+    }();
+    return on;
+}
+
 int device_sm_count() {
     const int d = current_device();
     if (!g_sm_count[d]) {

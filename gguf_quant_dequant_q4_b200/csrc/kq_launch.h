@@ -18,6 +18,9 @@ int record_cuda(cudaError_t e);
 // Whether kernels are launched with programmatic dependent launch (PDL):
 // on unless the environment sets KQ_NO_PDL=1 (an A/B lever).
 bool use_pdl();
+// Whether the prefill GEMM runs on CTA pairs (tcgen05 cta_group::2, 256
+// weight rows per tile): on unless the environment sets KQ_QMM_1SM=1.
+bool use_pair_mma();
 // Device address of the library-wide status word (bits KQ_DEV_*).
 int* device_status_ptr();
 

@@ -9,16 +9,24 @@
 // that re-reads the weight once per small row group wastes bandwidth; here
 // every weight tile is read and decoded once per 256 output rows.
 //
-// Tile: 128 weight rows (MMA M) x up to 256 activation rows (MMA N), K in
-// steps of 64.  One persistent CTA per SM, warp-specialized:
-//   warp 0      TMA producer: raw weight tiles (2-D box of wire bytes, 128
-//               rows x one 256-value block) and activation tiles (bf16,
-//               128B-swizzled, one 64-row box per map tile)
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+// Tile: 256 weight rows x up to 256 activation rows, K in steps of 64, on a
+// CTA pair (a cluster of two CTAs on neighbouring SMs, tcgen05 cta_group::2,
+// MMA M = 256): each CTA decodes its own 128 weight rows and loads half of
+// the activation rows, so a pair reads each activation tile once for 256
+// weight rows.  (With KQ_QMM_1SM=1 a single CTA takes 128 weight rows and all
+// 256 activation rows, MMA M = 128.)  Persistent, one CTA per SM,
+// warp-specialized:
+//   warp 0      activation producer: TMA of bf16 activation tiles
+//               (128B-swizzled, one 64-row box per map tile)
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer (in the
+//               first CTA of a pair; the full barriers it waits on live
+//               there, and its commits arrive on both CTAs' empty barriers)
 //   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator, masked stores
 //   warps 6..21 decoders: wire bytes -> bf16 A tile in the 128B-swizzled
 //               K-major layout the tensor core reads (thread = one row and
 //               one 16-value quarter of the 64-value step)
+//   warp 22     raw weight producer: TMA of wire-byte tiles (2-D box, 128
+//               rows x one 256-value block), with L2 prefetch ahead
 // Accumulators are double-buffered in TMEM (2 x 256 columns) so the epilogue
 // of one tile overlaps the main loop of the next.  All waits are bounded; a
 // wait that runs out sets KQ_DEV_TIMEOUT and the CTA winds down, freeing its
@@ -32,34 +40,31 @@ namespace kq {
 namespace {
 
 constexpr int kDecWarps = 16;    // decoder warps (thread = row x 16-value part)
-constexpr int kThreads = (6 + kDecWarps) * 32;
+constexpr int kThreads = (7 + kDecWarps) * 32;
 constexpr int kBM = 128;          // weight rows per tile (MMA M)
 constexpr int kBN = 256;          // activation rows per tile (MMA N max)
 constexpr int kBK = 64;           // K per pipeline step (one 128-byte swizzle row)
-constexpr int kRawStages = 2;     // raw weight stages, 256 values each
 constexpr int kMaxTiles = 1024;   // map tiles a gather call may use
 constexpr uint32_t kHeader = 5120; // barriers, misc words, tile tables
-constexpr int kEpiWarp0 = 2, kDeqWarp0 = 6;
+constexpr int kDeqWarp0 = 6;   // warps 0..5: producer, MMA, 4 epilogue
+constexpr int kRawWarp = kDeqWarp0 + kDecWarps;   // the raw weight producer
+constexpr int kRawAhead = 4;   // raw stages prefetched into L2 ahead of their load
 
 template <int QT> struct QmmCodec;
-// raw row bytes per stage, A (decoded) stages, B (activation) stages
+// raw row bytes per stage (one 256-value block column of 128 weight rows)
 template <> struct QmmCodec<KQ_Q4_K> {
-    static constexpr int RAWB = 144, AST = 3, BST = 4;
+    static constexpr int RAWB = 144;
 };
 template <> struct QmmCodec<KQ_Q6_K> {
-    static constexpr int RAWB = 240, AST = 2, BST = 4;   // 210-byte block at offset 210b mod 16
+    static constexpr int RAWB = 240;   // 210-byte block at offset 210b mod 16
 };
 template <> struct QmmCodec<KQ_Q8_0> {
-    static constexpr int RAWB = 272, AST = 3, BST = 3;   // eight 34-byte blocks
+    static constexpr int RAWB = 272;   // eight 34-byte blocks
 };
-template <int QT>
-constexpr bool fits_barriers() { return QmmCodec<QT>::AST <= 4 && QmmCodec<QT>::BST <= 4; }
-static_assert(fits_barriers<KQ_Q4_K>() && fits_barriers<KQ_Q6_K>() && fits_barriers<KQ_Q8_0>(),
-              "barrier table holds at most 4 A and 4 B stages");
 
 struct Smem {
-    static constexpr uint32_t kBars = 0;      // mbarriers
-    static constexpr uint32_t kMisc = 256;    // tmem base, abort flag, counts
+    static constexpr uint32_t kBars = 0;      // mbarriers (36)
+    static constexpr uint32_t kMisc = 384;    // tmem base, abort flag, counts
     static constexpr uint32_t kTiles = 512;   // sorted tile ids (u16) + per-expert tables
 };
 
@@ -91,15 +96,91 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// Arrive on `bar` once the MMAs issued so far complete; for a CTA pair the
+// arrival goes to the barrier at the same offset in both CTAs.
+template <int CG>
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+    if constexpr (CG == 2) {
+        asm volatile(
+            "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                smem_u32(bar)),
+            "h"(static_cast<uint16_t>(3))
+            : "memory");
+    } else {
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32(bar))
+                     : "memory");
+    }
+}
+template <int CG>
+__device__ __forceinline__ void tc_mma(uint32_t dtmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    if constexpr (CG == 2) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(dtmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(dtmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+            : "memory");
+    }
+}
+// All 512 TMEM columns (two 256-column accumulators), address written to
+// shared memory at `dst`; one whole warp, the same warp in both CTAs of a pair.
+template <int CG>
+__device__ __forceinline__ void tmem_alloc512(uint32_t dst) {
+    if constexpr (CG == 2) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(dst));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    } else {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(dst));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+}
+template <int CG>
+__device__ __forceinline__ void tmem_dealloc512(uint32_t tmem) {
+    if constexpr (CG == 2) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+    else asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+}
+// ---- CTA pairs (clusters of two)
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of this CTA's shared variable `saddr` in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_u32(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+// Arrive on an mbarrier given by its cluster shared-memory address (default
+// .release.cta semantics: the data it publishes is this CTA's shared memory,
+// read by the pair's tensor cores after the async-proxy fence, so no
+// cluster-scope fence is needed).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cl_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
+}
+// Prefetch of a tile into L2 (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y)
                  : "memory");
 }
-__device__ __forceinline__ void tc_mma(uint32_t dtmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+// Tiled load into this CTA's shared memory whose completion is counted on an
+// mbarrier of either CTA of the pair (cluster address), no multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(dtmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+        "%3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
         : "memory");
 }
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
@@ -128,9 +209,11 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
            (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
            (static_cast<uint64_t>(2) << 61);
 }
-// kind::f16 instruction descriptor: D f32, A and B bf16, both K-major, M = 128.
-__device__ __forceinline__ uint32_t make_idesc(int n) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | ((128u >> 4) << 24);
+// kind::f16 instruction descriptor: D f32, A and B bf16, both K-major, M =
+// 128 (one CTA) or 256 (a CTA pair).
+__device__ __forceinline__ uint32_t make_idesc(int n, int m) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(m >> 4) << 24);
 }
 
 // ------------------------------------------------------- bf16x2 arithmetic
@@ -397,31 +480,54 @@ struct Pipe {
     }
 };
 
-template <int QT>
+// Shared-memory stages per CTA: raw weight blocks (RST, 256 values each), A
+// (decoded weights, AST) and B (activations, BST), 64 values of K each.  A CTA
+// pair halves the activation stage.  Raw stages come from DRAM and have the
+// longest latency to cover.
+template <int QT, int CG> struct Stages;
+template <> struct Stages<KQ_Q4_K, 1> { static constexpr int RST = 3, AST = 3, BST = 3; };
+template <> struct Stages<KQ_Q6_K, 1> { static constexpr int RST = 3, AST = 2, BST = 3; };
+template <> struct Stages<KQ_Q8_0, 1> { static constexpr int RST = 3, AST = 2, BST = 2; };
+template <> struct Stages<KQ_Q4_K, 2> { static constexpr int RST = 4, AST = 4, BST = 5; };
+template <> struct Stages<KQ_Q6_K, 2> { static constexpr int RST = 3, AST = 3, BST = 5; };
+template <> struct Stages<KQ_Q8_0, 2> { static constexpr int RST = 3, AST = 3, BST = 4; };
+
+template <int QT, int CG>
+constexpr uint32_t smem_bytes() {
+    return kHeader + 1024 + Stages<QT, CG>::BST * (kBN / CG) * kBK * 2 + Stages<QT, CG>::AST * kBM * kBK * 2 +
+           Stages<QT, CG>::RST * kBM * QmmCodec<QT>::RAWB;
+}
+
+template <int QT, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
     qmm_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
                const QmmParams p) {
     using C = QmmCodec<QT>;
-    constexpr int AST = C::AST;
-    constexpr int kBStages = C::BST;
+    constexpr int RST = Stages<QT, CG>::RST;
+    constexpr int AST = Stages<QT, CG>::AST;
+    constexpr int BST = Stages<QT, CG>::BST;
+    static_assert(RST <= 4 && AST <= 4 && BST <= 8, "barrier table holds 4 raw, 4 A and 8 B stages");
+    static_assert(smem_bytes<QT, CG>() <= 232448, "shared memory per CTA");
+    constexpr int kBNc = kBN / CG;                    // activation rows of a B stage in this CTA
     constexpr uint32_t kRawBytes = kBM * C::RAWB;
-    constexpr uint32_t kABytes = kBM * kBK * 2;    // 16 KB
-    constexpr uint32_t kBBytes = kBN * kBK * 2;    // 32 KB
+    constexpr uint32_t kABytes = kBM * kBK * 2;      // 16 KB
+    constexpr uint32_t kBBytes = kBNc * kBK * 2;     // 32 KB (one CTA) or 16 KB (pair)
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sb = smem_u32(smem);
-    // stage regions (1024-aligned): B stages, A stages, raw stages
+    // stage regions (1024-aligned): B stages, A stages, raw stages; the same
+    // offsets in both CTAs of a pair, as the pair's MMA descriptors require
     const uint32_t base = (sb + kHeader + 1023) & ~1023u;
-    const uint32_t bst = base, ast = bst + kBStages * kBBytes, rst = ast + AST * kABytes;
+    const uint32_t bst = base, ast = bst + BST * kBBytes, rst = ast + AST * kABytes;
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Smem::kBars);
     uint64_t* raw_full = bars;
-    uint64_t* raw_empty = bars + 2;
-    uint64_t* a_full = bars + 4;
-    uint64_t* a_empty = bars + 8;
-    uint64_t* b_full = bars + 12;
-    uint64_t* b_empty = bars + 16;
-    uint64_t* acc_full = bars + 20;
-    uint64_t* acc_empty = bars + 22;
+    uint64_t* raw_empty = bars + 4;
+    uint64_t* a_full = bars + 8;
+    uint64_t* a_empty = bars + 12;
+    uint64_t* b_full = bars + 16;
+    uint64_t* b_empty = bars + 24;
+    uint64_t* acc_full = bars + 32;
+    uint64_t* acc_empty = bars + 34;
     volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + Smem::kMisc);
     // misc[0] tmem base, misc[1] abort, misc[2] number of chunks, misc[3] tiles
     uint16_t* tiles = reinterpret_cast<uint16_t*>(smem + Smem::kTiles);          // sorted valid tile ids
@@ -429,36 +535,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* tstart = cstart + 257;                                                  // per expert tile prefix [257]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = CG == 2 ? cluster_ctarank() : 0;   // 0 = the pair's MMA-issuing CTA
+    // full barriers the pair's MMA waits on live in CTA 0 of the pair
+    auto lead = [&](uint64_t* bar) { return CG == 2 ? mapa_u32(smem_u32(bar), 0) : smem_u32(bar); };
 
     // ---- set-up: barriers, TMEM, work list
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < RST; ++i) {
             mbar_init(&raw_full[i], 1);
             mbar_init(&raw_empty[i], kDecWarps);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], 4);
+            mbar_init(&acc_empty[i], 4 * CG);
         }
         for (int i = 0; i < AST; ++i) {
-            mbar_init(&a_full[i], kDecWarps);
+            mbar_init(&a_full[i], kDecWarps * CG);
             mbar_init(&a_empty[i], 1);
         }
-        for (int i = 0; i < kBStages; ++i) {
+        for (int i = 0; i < BST; ++i) {
             mbar_init(&b_full[i], 1);
             mbar_init(&b_empty[i], 1);
         }
         misc[1] = 0;
         fence_barrier_init();
     }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(sb + Smem::kMisc));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-    }
+    if (warp == 1) tmem_alloc512<CG>(sb + Smem::kMisc);
     int total_units;
     if (p.n_experts == 0) {
         total_units = p.units;
     } else {
         // Gather: validate the map, keep valid tiles, order them by
         // (expert, row_start) and cut each expert's list into chunks of 4.
+        // Both CTAs of a pair build the same tables.
         int cnt = static_cast<int>(*p.count);
         if (cnt > p.cap || cnt < 0) {
             if (tid == 0 && p.err) atomicOr(p.err, KQ_DEV_BAD_RANGE);
@@ -503,21 +612,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t e = p.map[3 * i], rs = p.map[3 * i + 1], nr = p.map[3 * i + 2];
             if (e >= static_cast<uint32_t>(p.n_experts) || nr == 0 || nr > 64 || static_cast<int64_t>(rs) + nr > p.m)
                 continue;
-            int rank = 0;
+            int rk = 0;
             for (int j = 0; j < cnt; ++j) {
                 const uint32_t e2 = p.map[3 * j], rs2 = p.map[3 * j + 1], nr2 = p.map[3 * j + 2];
                 const bool ok2 = e2 == e && nr2 != 0 && nr2 <= 64 && static_cast<int64_t>(rs2) + nr2 <= p.m;
-                if (ok2 && (rs2 < rs || (rs2 == rs && j < i))) ++rank;
+                if (ok2 && (rs2 < rs || (rs2 == rs && j < i))) ++rk;
             }
-            tiles[tstart[e] + rank] = static_cast<uint16_t>(i);
+            tiles[tstart[e] + rk] = static_cast<uint16_t>(i);
         }
         total_units = 0;   // read after the barrier below
     }
     tc_fence_before();
-    __syncthreads();
+    // the pair's barriers and TMEM are set up before any CTA of it goes on
+    if constexpr (CG == 2) cluster_sync();
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
     if (p.n_experts != 0) total_units = static_cast<int>(misc[2]) * p.ntn;
+    // a unit is processed by one CTA (CG = 1) or one CTA pair (CG = 2)
+    const int u0 = static_cast<int>(blockIdx.x) / CG, ustep = static_cast<int>(gridDim.x) / CG;
 
     auto get_unit = [&](int u, Unit& U) {
         if (p.n_experts == 0) {
@@ -576,7 +689,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     };
-    auto mma_n = [&](const Unit& U) { return 64 * (U.nt - 1) + ((U.nr[U.nt - 1] + 15) & ~15); };
+    // MMA N: one CTA trims it to the rows present; a pair splits N evenly
+    // between its CTAs (CTA r holds B rows [rN/2, (r+1)N/2)), so N is 128
+    // (one 64-row tile per CTA) or 256 (two per CTA)
+    auto mma_n = [&](const Unit& U) {
+        if constexpr (CG == 2) return U.nt <= 2 ? 128 : 256;
+        else return 64 * (U.nt - 1) + ((U.nr[U.nt - 1] + 15) & ~15);
+    };
     auto aborted = [&]() { return misc[1] != 0; };
     auto bwait = [&](uint64_t* bar, uint32_t parity) {
         if (misc[1]) return false;
@@ -588,50 +707,91 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     const int ksteps = p.k / kBK;
+    const int wtile_rows = kBM * CG;   // weight rows of a unit
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ activation producer
         if (lane == 0) {
-            Pipe rp, bp;
-            for (int u = blockIdx.x; u < total_units && !aborted(); u += gridDim.x) {
+            Pipe bp;
+            for (int u = u0; u < total_units && !aborted(); u += ustep) {
                 Unit U;
                 get_unit(u, U);
                 if (U.nt == 0) continue;
-                const int wrow = U.e * static_cast<int>(p.n) + U.ntile * kBM;
+                // this CTA's activation tiles of the unit: [t0, t1), at 64-row slots from 0
+                int t0 = 0, t1 = U.nt;
+                if constexpr (CG == 2) {
+                    const int tpc = mma_n(U) / 128;
+                    t0 = static_cast<int>(rank) * tpc;
+                    t1 = t0 + tpc < U.nt ? t0 + tpc : U.nt;
+                }
                 for (int ks = 0; ks < ksteps; ++ks) {
-                    if ((ks & 3) == 0) {
-                        if (!bwait(&raw_empty[rp.idx], rp.phase ^ 1)) break;
-                        mbar_arrive_expect_tx(&raw_full[rp.idx], kRawBytes);
-                        const int blk = ks >> 2;
-                        int xc;
-                        if constexpr (QT == KQ_Q4_K) xc = 144 * blk;
-                        else if constexpr (QT == KQ_Q6_K) xc = (210 * blk) & ~15;
-                        else xc = 136 * blk;   // 2-byte elements
-                        tma_load_2d(rst + rp.idx * kRawBytes, &wmap, xc, wrow, &raw_full[rp.idx]);
-                        rp.next(kRawStages);
-                    }
                     if (!bwait(&b_empty[bp.idx], bp.phase ^ 1)) break;
-                    mbar_arrive_expect_tx(&b_full[bp.idx], U.nt * 8192);
-                    for (int i = 0; i < U.nt; ++i)
-                        tma_load_2d(bst + bp.idx * kBBytes + i * 8192, &xmap, ks * kBK, U.rs[i], &b_full[bp.idx]);
-                    bp.next(kBStages);
+                    const uint32_t dst = bst + bp.idx * kBBytes;
+                    if constexpr (CG == 2) {
+                        // both CTAs' bytes land on CTA 0's full barrier; CTA 0
+                        // expects the unit's total
+                        if (rank == 0) mbar_arrive_expect_tx(&b_full[bp.idx], U.nt * 8192);
+                        const uint32_t fb = lead(&b_full[bp.idx]);
+                        for (int i = t0; i < t1; ++i) tma_load_2d_pair(dst + (i - t0) * 8192, &xmap, ks * kBK, U.rs[i], fb);
+                    } else {
+                        mbar_arrive_expect_tx(&b_full[bp.idx], U.nt * 8192);
+                        for (int i = t0; i < t1; ++i) tma_load_2d(dst + i * 8192, &xmap, ks * kBK, U.rs[i], &b_full[bp.idx]);
+                    }
+                    bp.next(BST);
+                }
+            }
+        }
+    } else if (warp == kRawWarp) {
+        // ------------------------------------------------ raw weight producer
+        // One 256-value block column of this CTA's 128 weight rows per stage,
+        // straight from the wire bytes; the block kRawAhead stages ahead is
+        // prefetched into L2 so that the load it later issues finds it there.
+        if (lane == 0) {
+            Pipe rp;
+            const int nblk = ksteps / 4;
+            auto xcol = [&](int blk) {
+                if constexpr (QT == KQ_Q4_K) return 144 * blk;
+                else if constexpr (QT == KQ_Q6_K) return (210 * blk) & ~15;
+                else return 136 * blk;   // 2-byte elements
+            };
+            for (int u = u0; u < total_units && !aborted(); u += ustep) {
+                Unit U;
+                get_unit(u, U);
+                if (U.nt == 0) continue;
+                const int wrow = U.e * static_cast<int>(p.n) + U.ntile * wtile_rows + kBM * static_cast<int>(rank);
+                for (int b = 0; b < kRawAhead && b < nblk; ++b) tma_prefetch_2d(&wmap, xcol(b), wrow);
+                for (int blk = 0; blk < nblk; ++blk) {
+                    if (blk + kRawAhead < nblk) tma_prefetch_2d(&wmap, xcol(blk + kRawAhead), wrow);
+                    if (!bwait(&raw_empty[rp.idx], rp.phase ^ 1)) break;
+                    mbar_arrive_expect_tx(&raw_full[rp.idx], kRawBytes);
+                    tma_load_2d(rst + rp.idx * kRawBytes, &wmap, xcol(blk), wrow, &raw_full[rp.idx]);
+                    rp.next(RST);
                 }
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // ------------------------------------------------ MMA issuer (CTA 0 of a pair)
+        if (lane == 0 && rank == 0) {
             Pipe ap, bp, cp;
-            for (int u = blockIdx.x; u < total_units && !aborted(); u += gridDim.x) {
+            for (int u = u0; u < total_units && !aborted(); u += ustep) {
                 Unit U;
                 get_unit(u, U);
                 if (U.nt == 0) continue;
-                const uint32_t idesc = make_idesc(mma_n(U));
+                const uint32_t idesc = make_idesc(mma_n(U), kBM * CG);
                 if (!bwait(&acc_empty[cp.idx], cp.phase ^ 1)) break;
                 tc_fence_after();
                 const uint32_t dt = tmem + cp.idx * 256;
                 bool ok = true;
+                // The issue loop is on the critical path of the tensor pipe:
+                // a stage seen complete is polled once, before the last MMA
+                // of the previous stage, and the bounded wait runs only when
+                // a stage is not ready yet.
+                bool ra = false, rb = false;
                 for (int ks = 0; ks < ksteps; ++ks) {
-                    if (!bwait(&a_full[ap.idx], ap.phase) || !bwait(&b_full[bp.idx], bp.phase)) {
+                    if (!ra && !mbar_try_wait(&a_full[ap.idx], ap.phase) && !bwait(&a_full[ap.idx], ap.phase)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!rb && !mbar_try_wait(&b_full[bp.idx], bp.phase) && !bwait(&b_full[bp.idx], bp.phase)) {
                         ok = false;
                         break;
                     }
@@ -639,15 +799,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t ad = sw128_desc(ast + ap.idx * kABytes);
                     const uint64_t bd = sw128_desc(bst + bp.idx * kBBytes);
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
-                        tc_mma(dt, ad + 2 * kk, bd + 2 * kk, idesc, (ks | kk) != 0);
-                    tc_commit(&a_empty[ap.idx]);
-                    tc_commit(&b_empty[bp.idx]);
-                    ap.next(AST);
-                    bp.next(kBStages);
+                    for (int kk = 0; kk < kBK / 16 - 1; ++kk)
+                        tc_mma<CG>(dt, ad + 2 * kk, bd + 2 * kk, idesc, (ks | kk) != 0);
+                    Pipe an = ap, bn = bp;
+                    an.next(AST);
+                    bn.next(BST);
+                    ra = ks + 1 < ksteps && mbar_try_wait(&a_full[an.idx], an.phase);
+                    rb = ks + 1 < ksteps && mbar_try_wait(&b_full[bn.idx], bn.phase);
+                    tc_mma<CG>(dt, ad + 2 * (kBK / 16 - 1), bd + 2 * (kBK / 16 - 1), idesc, 1);
+                    tc_commit<CG>(&a_empty[ap.idx]);
+                    tc_commit<CG>(&b_empty[bp.idx]);
+                    ap = an;
+                    bp = bn;
                 }
                 if (!ok) break;
-                tc_commit(&acc_full[cp.idx]);
+                tc_commit<CG>(&acc_full[cp.idx]);
                 cp.next(2);
             }
         }
@@ -655,23 +821,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ epilogue
         const int q = warp & 3;   // TMEM lane quarter this warp may access
         Pipe cp;
-        for (int u = blockIdx.x; u < total_units && !aborted(); u += gridDim.x) {
+        for (int u = u0; u < total_units && !aborted(); u += ustep) {
             Unit U;
             get_unit(u, U);
             if (U.nt == 0) continue;
             const int nmma = mma_n(U);
             if (!bwait(&acc_full[cp.idx], cp.phase)) break;
             tc_fence_after();
-            const int64_t nrow = static_cast<int64_t>(U.ntile) * kBM + 32 * q + lane;
+            const int64_t nrow = static_cast<int64_t>(U.ntile) * wtile_rows + kBM * static_cast<int>(rank) + 32 * q + lane;
             const bool row_ok = nrow < p.n;
             const uint32_t tbase = tmem + cp.idx * 256 + (static_cast<uint32_t>(32 * q) << 16);
             for (int c0 = 0; c0 < nmma; c0 += 16) {
-                uint32_t v[16];
-                tmem_ld16(tbase + c0, v);
                 const int ti = c0 >> 6;
                 const int r0 = c0 & 63;
                 const int nv = U.nr[ti] - r0;   // valid activation rows of this 16-column chunk
-                if (row_ok && nv > 0) {
+                if (nv <= 0) continue;          // warp-uniform
+                uint32_t v[16];
+                tmem_ld16(tbase + c0, v);
+                if (row_ok) {
                     // y is written once and never read here: streaming stores
                     float* yp = p.y + (static_cast<int64_t>(U.rs[ti]) + r0) * p.n + nrow;
                     if (nv >= 16) {
@@ -686,7 +853,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[cp.idx]);
+            if (lane == 0) {
+                if constexpr (CG == 2) mbar_arrive_remote(lead(&acc_empty[cp.idx]));
+                else mbar_arrive(&acc_empty[cp.idx]);
+            }
             cp.next(2);
         }
     } else {
@@ -698,7 +868,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t so0 = rowb + (((2 * part) ^ (r & 7)) << 4), so1 = rowb + (((2 * part + 1) ^ (r & 7)) << 4);
         Pipe rp, ap;
         StageScales S;
-        for (int u = blockIdx.x; u < total_units && !aborted(); u += gridDim.x) {
+        for (int u = u0; u < total_units && !aborted(); u += ustep) {
             Unit U;
             get_unit(u, U);
             if (U.nt == 0) continue;
@@ -724,23 +894,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                     sts128(ab + so1, o[4], o[5], o[6], o[7]);
                     fence_proxy_async();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&a_full[ap.idx]);
+                    if (lane == 0) {
+                        if constexpr (CG == 2) mbar_arrive_remote(lead(&a_full[ap.idx]));
+                        else mbar_arrive(&a_full[ap.idx]);
+                    }
                     ap.next(AST);
                 }
                 if (!ok) break;
                 if (lane == 0) mbar_arrive(&raw_empty[rp.idx]);
-                rp.next(kRawStages);
+                rp.next(RST);
             }
             if (!ok) break;
         }
     }
 
-    // ---- tear-down
+    // ---- tear-down: neither CTA of a pair leaves while the other may still
+    // read its shared memory or signal its barriers
+    __syncwarp();
     tc_fence_before();
-    __syncthreads();
+    if constexpr (CG == 2) cluster_sync();
+    else __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+        tmem_dealloc512<CG>(tmem);
     }
 }
 
@@ -774,6 +950,75 @@ int make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* ptr,
     return r == CUDA_SUCCESS ? KQ_OK : KQ_ERR_INVALID_ARG;
 }
 
+// Launch with units of 128 (one CTA) or 256 (a CTA pair) weight rows; a pair
+// is a cluster of two CTAs on neighbouring SMs.
+template <int QT, int CG>
+int launch_cg(const CUtensorMap& wmap, const CUtensorMap& xmap, QmmParams p, cudaStream_t s) {
+    constexpr uint32_t smem = smem_bytes<QT, CG>();
+    auto kern = qmm_kernel<QT, CG>;
+    static bool attr_set[64] = {false};
+    static int slots[64] = {0};   // CTAs of this kernel resident at once, per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return record_cuda(e);
+        int n = device_sm_count();
+        if (CG == 2) {
+            cudaLaunchConfig_t q = {};
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = 2;
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            q.gridDim = dim3(2 * (n / 2), 1, 1);
+            q.blockDim = dim3(kThreads, 1, 1);
+            q.dynamicSmemBytes = smem;
+            q.attrs = at;
+            q.numAttrs = 1;
+            int clusters = 0;
+            e = cudaOccupancyMaxActiveClusters(&clusters, kern, &q);
+            if (e != cudaSuccess) return record_cuda(e);
+            n = 2 * clusters;
+        }
+        if (n < CG) return KQ_ERR_UNSUPPORTED;
+        slots[dev] = n;
+        attr_set[dev] = true;
+    }
+    const int groups = slots[dev] / CG;   // CTAs or CTA pairs resident at once
+    p.ntn = static_cast<int>((p.n + kBM * CG - 1) / (kBM * CG));
+    p.units = p.n_experts == 0 ? static_cast<int>((p.m + kBN - 1) / kBN) * p.ntn : 0;
+    p.units_main = p.units;
+    p.split = 1;
+    int ng = groups;
+    if (p.n_experts == 0 && p.units < ng) ng = p.units;
+    if (ng < 1) return KQ_OK;
+    if (p.n_experts == 0 && p.units > ng && p.units % ng != 0 && p.m > 64) {
+        // the last, partial round: its units become sub-units, as many per
+        // unit as still fit in one round of the grid
+        const int tail = p.units % ng;
+        p.split = 4 * tail <= ng ? 4 : (2 * tail <= ng ? 2 : 1);
+        p.units_main = p.units - tail;
+        p.units = p.units_main + p.split * tail;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = CG;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(ng * CG), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = at;
+    cfg.numAttrs = CG == 2 ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, wmap, xmap, p);
+    if (e != cudaSuccess) return record_cuda(e);
+    return check_launch();
+}
+
 template <int QT>
 int launch_impl(const void* w, int64_t w_rows, int64_t n, int64_t k, const uint16_t* x, int64_t x_rows, int n_experts,
                 const uint32_t* map, const uint32_t* count, int64_t cap, float* y, int32_t* err, cudaStream_t s) {
@@ -799,33 +1044,13 @@ int launch_impl(const void* w, int64_t w_rows, int64_t n, int64_t k, const uint1
     p.m = x_rows;
     p.k = static_cast<int>(k);
     p.n_experts = n_experts;
-    p.ntn = static_cast<int>((n + kBM - 1) / kBM);
-    p.units = n_experts == 0 ? static_cast<int>((x_rows + kBN - 1) / kBN) * p.ntn : 0;
-    p.units_main = p.units;
-    p.split = 1;
     p.map = map;
     p.count = count;
     p.cap = cap;
     p.y = y;
     p.err = err;
     p.status = device_status_ptr();
-    const uint32_t smem = kHeader + 1024 + C::BST * kBN * kBK * 2 + C::AST * kBM * kBK * 2 + kRawStages * kBM * C::RAWB;
-    auto kern = qmm_kernel<QT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return record_cuda(e);
-    int grid = device_sm_count();
-    if (n_experts == 0 && p.units < grid) grid = p.units;
-    if (grid < 1) return KQ_OK;
-    if (n_experts == 0 && p.units > grid && p.units % grid != 0 && x_rows > 64) {
-        // the last, partial round: its units become sub-units, as many per
-        // unit as still fit in one round of the grid
-        const int tail = p.units % grid;
-        p.split = 4 * tail <= grid ? 4 : (2 * tail <= grid ? 2 : 1);
-        p.units_main = p.units - tail;
-        p.units = p.units_main + p.split * tail;
-    }
-    kern<<<grid, kThreads, smem, s>>>(wmap, xmap, p);
-    return check_launch();
+    return use_pair_mma() ? launch_cg<QT, 2>(wmap, xmap, p, s) : launch_cg<QT, 1>(wmap, xmap, p, s);
 }
 
 }  // namespace
