@@ -481,21 +481,24 @@ struct Pipe {
 };
 
 // Shared-memory stages per CTA: raw weight blocks (RST, 256 values each), A
-// (decoded weights, AST) and B (activations, BST), 64 values of K each.  A CTA
-// pair halves the activation stage.  Raw stages come from DRAM and have the
-// longest latency to cover.
+// (decoded weights, AST) and B (activations, BST), KPS steps of 64 values of K
+// each.  A CTA pair halves the activation stage.  Raw stages come from DRAM
+// and have the longest latency to cover.  Every stage boundary costs the MMA
+// issuing thread a wait and a release, which the shallow MMA queue does not
+// hide, so where shared memory allows a stage holds two K steps.
 template <int QT, int CG> struct Stages;
-template <> struct Stages<KQ_Q4_K, 1> { static constexpr int RST = 3, AST = 3, BST = 3; };
-template <> struct Stages<KQ_Q6_K, 1> { static constexpr int RST = 3, AST = 2, BST = 3; };
-template <> struct Stages<KQ_Q8_0, 1> { static constexpr int RST = 3, AST = 2, BST = 2; };
-template <> struct Stages<KQ_Q4_K, 2> { static constexpr int RST = 4, AST = 4, BST = 5; };
-template <> struct Stages<KQ_Q6_K, 2> { static constexpr int RST = 3, AST = 3, BST = 5; };
-template <> struct Stages<KQ_Q8_0, 2> { static constexpr int RST = 3, AST = 3, BST = 4; };
+template <> struct Stages<KQ_Q4_K, 1> { static constexpr int RST = 3, AST = 3, BST = 3, KPS = 1; };
+template <> struct Stages<KQ_Q6_K, 1> { static constexpr int RST = 3, AST = 2, BST = 3, KPS = 1; };
+template <> struct Stages<KQ_Q8_0, 1> { static constexpr int RST = 3, AST = 2, BST = 2, KPS = 1; };
+template <> struct Stages<KQ_Q4_K, 2> { static constexpr int RST = 3, AST = 2, BST = 3, KPS = 2; };
+template <> struct Stages<KQ_Q6_K, 2> { static constexpr int RST = 2, AST = 2, BST = 3, KPS = 2; };
+template <> struct Stages<KQ_Q8_0, 2> { static constexpr int RST = 3, AST = 3, BST = 4, KPS = 1; };
 
 template <int QT, int CG>
 constexpr uint32_t smem_bytes() {
-    return kHeader + 1024 + Stages<QT, CG>::BST * (kBN / CG) * kBK * 2 + Stages<QT, CG>::AST * kBM * kBK * 2 +
-           Stages<QT, CG>::RST * kBM * QmmCodec<QT>::RAWB;
+    using S = Stages<QT, CG>;
+    return kHeader + 1024 + S::BST * S::KPS * (kBN / CG) * kBK * 2 + S::AST * S::KPS * kBM * kBK * 2 +
+           S::RST * kBM * QmmCodec<QT>::RAWB;
 }
 
 template <int QT, int CG>
@@ -506,12 +509,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int RST = Stages<QT, CG>::RST;
     constexpr int AST = Stages<QT, CG>::AST;
     constexpr int BST = Stages<QT, CG>::BST;
+    constexpr int KPS = Stages<QT, CG>::KPS;   // 64-value K steps per A/B stage
     static_assert(RST <= 4 && AST <= 4 && BST <= 8, "barrier table holds 4 raw, 4 A and 8 B stages");
+    static_assert(KPS == 1 || KPS == 2, "a raw stage (4 K steps) holds whole A/B stages");
     static_assert(smem_bytes<QT, CG>() <= 232448, "shared memory per CTA");
     constexpr int kBNc = kBN / CG;                    // activation rows of a B stage in this CTA
     constexpr uint32_t kRawBytes = kBM * C::RAWB;
-    constexpr uint32_t kABytes = kBM * kBK * 2;      // 16 KB
-    constexpr uint32_t kBBytes = kBNc * kBK * 2;     // 32 KB (one CTA) or 16 KB (pair)
+    constexpr uint32_t kAAtom = kBM * kBK * 2;       // 16 KB: one K step of A
+    constexpr uint32_t kBAtom = kBNc * kBK * 2;      // 32 KB (one CTA) or 16 KB (pair): one K step of B
+    constexpr uint32_t kABytes = KPS * kAAtom;
+    constexpr uint32_t kBBytes = KPS * kBAtom;
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sb = smem_u32(smem);
     // stage regions (1024-aligned): B stages, A stages, raw stages; the same
@@ -707,6 +714,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     const int ksteps = p.k / kBK;
+    const int nstages = ksteps / KPS;   // A/B stages per unit (ksteps is a multiple of 4)
     const int wtile_rows = kBM * CG;   // weight rows of a unit
     if (warp == 0) {
         // ------------------------------------------------ activation producer
@@ -723,18 +731,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                     t0 = static_cast<int>(rank) * tpc;
                     t1 = t0 + tpc < U.nt ? t0 + tpc : U.nt;
                 }
-                for (int ks = 0; ks < ksteps; ++ks) {
+                for (int st = 0; st < nstages; ++st) {
                     if (!bwait(&b_empty[bp.idx], bp.phase ^ 1)) break;
                     const uint32_t dst = bst + bp.idx * kBBytes;
                     if constexpr (CG == 2) {
                         // both CTAs' bytes land on CTA 0's full barrier; CTA 0
                         // expects the unit's total
-                        if (rank == 0) mbar_arrive_expect_tx(&b_full[bp.idx], U.nt * 8192);
+                        if (rank == 0) mbar_arrive_expect_tx(&b_full[bp.idx], KPS * U.nt * 8192);
                         const uint32_t fb = lead(&b_full[bp.idx]);
-                        for (int i = t0; i < t1; ++i) tma_load_2d_pair(dst + (i - t0) * 8192, &xmap, ks * kBK, U.rs[i], fb);
+#pragma unroll
+                        for (int a = 0; a < KPS; ++a)
+                            for (int i = t0; i < t1; ++i)
+                                tma_load_2d_pair(dst + a * kBAtom + (i - t0) * 8192, &xmap, (st * KPS + a) * kBK, U.rs[i], fb);
                     } else {
-                        mbar_arrive_expect_tx(&b_full[bp.idx], U.nt * 8192);
-                        for (int i = t0; i < t1; ++i) tma_load_2d(dst + i * 8192, &xmap, ks * kBK, U.rs[i], &b_full[bp.idx]);
+                        mbar_arrive_expect_tx(&b_full[bp.idx], KPS * U.nt * 8192);
+#pragma unroll
+                        for (int a = 0; a < KPS; ++a)
+                            for (int i = t0; i < t1; ++i)
+                                tma_load_2d(dst + a * kBAtom + i * 8192, &xmap, (st * KPS + a) * kBK, U.rs[i], &b_full[bp.idx]);
                     }
                     bp.next(BST);
                 }
@@ -781,12 +795,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t dt = tmem + cp.idx * 256;
                 bool ok = true;
-                // The issue loop is on the critical path of the tensor pipe:
-                // a stage seen complete is polled once, before the last MMA
-                // of the previous stage, and the bounded wait runs only when
-                // a stage is not ready yet.
-                bool ra = false, rb = false;
-                for (int ks = 0; ks < ksteps; ++ks) {
+                // The issue loop is on the critical path of the tensor pipe
+                // (the MMA queue is shallow: whatever this thread does between
+                // two MMAs can leave the pipe idle), so the bookkeeping of a
+                // stage sits between the MMAs of the next one: the previous
+                // stage's release (commit) after the first MMA, the poll of
+                // the next stage after the second.  The bounded wait runs
+                // only when a stage is not complete yet.
+                bool ra = false, rb = false;   // stage seen complete by the poll
+                int pa = -1, pb = -1;          // stages whose release is pending
+                for (int st = 0; st < nstages; ++st) {
                     if (!ra && !mbar_try_wait(&a_full[ap.idx], ap.phase) && !bwait(&a_full[ap.idx], ap.phase)) {
                         ok = false;
                         break;
@@ -798,19 +816,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const uint64_t ad = sw128_desc(ast + ap.idx * kABytes);
                     const uint64_t bd = sw128_desc(bst + bp.idx * kBBytes);
-#pragma unroll
-                    for (int kk = 0; kk < kBK / 16 - 1; ++kk)
-                        tc_mma<CG>(dt, ad + 2 * kk, bd + 2 * kk, idesc, (ks | kk) != 0);
+                    tc_mma<CG>(dt, ad, bd, idesc, st != 0);
+                    if (pa >= 0) {
+                        tc_commit<CG>(&a_empty[pa]);
+                        tc_commit<CG>(&b_empty[pb]);
+                    }
+                    tc_mma<CG>(dt, ad + 2, bd + 2, idesc, 1);
                     Pipe an = ap, bn = bp;
                     an.next(AST);
                     bn.next(BST);
-                    ra = ks + 1 < ksteps && mbar_try_wait(&a_full[an.idx], an.phase);
-                    rb = ks + 1 < ksteps && mbar_try_wait(&b_full[bn.idx], bn.phase);
-                    tc_mma<CG>(dt, ad + 2 * (kBK / 16 - 1), bd + 2 * (kBK / 16 - 1), idesc, 1);
-                    tc_commit<CG>(&a_empty[ap.idx]);
-                    tc_commit<CG>(&b_empty[bp.idx]);
+                    ra = st + 1 < nstages && mbar_try_wait(&a_full[an.idx], an.phase);
+                    rb = st + 1 < nstages && mbar_try_wait(&b_full[bn.idx], bn.phase);
+                    // descriptor start addresses advance 32 bytes (2 units) per
+                    // 16-value K slice inside an atom, one atom per K step
+#pragma unroll
+                    for (int kk = 2; kk < KPS * (kBK / 16); ++kk) {
+                        const int a = kk / (kBK / 16), sl = kk % (kBK / 16);
+                        tc_mma<CG>(dt, ad + (a * kAAtom >> 4) + 2 * sl, bd + (a * kBAtom >> 4) + 2 * sl, idesc, 1);
+                    }
+                    pa = ap.idx;
+                    pb = bp.idx;
                     ap = an;
                     bp = bn;
+                }
+                if (pa >= 0) {
+                    tc_commit<CG>(&a_empty[pa]);
+                    tc_commit<CG>(&b_empty[pb]);
                 }
                 if (!ok) break;
                 tc_commit<CG>(&acc_full[cp.idx]);
@@ -883,22 +914,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 prep_scales<QT>(row, part, o6, S);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    if (!bwait(&a_empty[ap.idx], ap.phase ^ 1)) {
+                    const int a = q % KPS;   // K step within the A stage
+                    if (a == 0 && !bwait(&a_empty[ap.idx], ap.phase ^ 1)) {
                         ok = false;
                         break;
                     }
                     uint32_t o[8];
                     decode_step<QT>(row, q, part, o6, S, o);
-                    const uint32_t ab = ast + ap.idx * kABytes;
+                    const uint32_t ab = ast + ap.idx * kABytes + a * kAAtom;
                     sts128(ab + so0, o[0], o[1], o[2], o[3]);
                     sts128(ab + so1, o[4], o[5], o[6], o[7]);
-                    fence_proxy_async();
-                    __syncwarp();
-                    if (lane == 0) {
-                        if constexpr (CG == 2) mbar_arrive_remote(lead(&a_full[ap.idx]));
-                        else mbar_arrive(&a_full[ap.idx]);
+                    if (a == KPS - 1) {
+                        fence_proxy_async();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if constexpr (CG == 2) mbar_arrive_remote(lead(&a_full[ap.idx]));
+                            else mbar_arrive(&a_full[ap.idx]);
+                        }
+                        ap.next(AST);
                     }
-                    ap.next(AST);
                 }
                 if (!ok) break;
                 if (lane == 0) mbar_arrive(&raw_empty[rp.idx]);
