@@ -145,21 +145,7 @@ __device__ __forceinline__ void tmem_dealloc512(uint32_t tmem) {
     if constexpr (CG == 2) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, 512;" ::"r"(tmem));
     else asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
 }
-// ---- CTA pairs (clusters of two)
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// Address of this CTA's shared variable `saddr` in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t mapa_u32(uint32_t saddr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-    return r;
-}
+// ---- CTA pairs (clusters of two): cluster helpers are in kq_device.cuh
 // Arrive on an mbarrier given by its cluster shared-memory address (default
 // .release.cta semantics: the data it publishes is this CTA's shared memory,
 // read by the pair's tensor cores after the async-proxy fence, so no

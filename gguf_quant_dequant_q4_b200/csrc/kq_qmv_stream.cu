@@ -60,12 +60,18 @@ struct SP {
     const uint16_t* x;
     float* y;
     int* status;
-    int64_t n, k, row_bytes;
-    int m, nblk, g, spr, ns;
-    int x_global;   // 1: build the image from x in global memory (no room for a raw copy)
+    int64_t n, k, row_bytes;   // k: values of K this CTA covers (its slice)
+    int m, nblk, g, spr, ns;   // nblk: blocks of the slice
+    // x_global 1: build the image from x in global memory (no room for a raw
+    // copy); ks: CTAs of a cluster splitting K (q4_K; 1: no split; the token
+    // stride of x is then ks k).  Packed: a larger parameter block was
+    // measured to slow the kernel down.
+    uint32_t x_global : 8, ks : 8;
     uint32_t rs;   // shared-memory stride of a stage row
     uint32_t off_stage, off_img, img_tok, off_xs, xs_tok, off_zero, off_part, off_xraw;
+    uint32_t off_red;   // split: receive slots of the cluster reduction
 };
+static_assert(sizeof(SP) == 120, "kernel parameter block size");
 
 // Row groups are walked with a partial last group (fewer than 16 rows) moved
 // to the front: its small stage lands first and its decode overlaps the full
@@ -252,7 +258,7 @@ struct Q8 {
     // Image entry (item, mu, t') = binary16 activations of the 4 raw bytes at
     // offset 272 item + 68 t' + 4 mu of a row, as (byte0, byte2 | byte1,
     // byte3); scale bytes get 0.  X[tok][block] = sum of its 32 activations.
-    static __device__ void build(const SP& p, uint32_t sb, float& amax) {
+    static __device__ void build(const SP& p, uint32_t sb, float& amax, int64_t xoff) {
         const int items = p.nblk / 8;
         const int per_tok = items * 17 * 4;
         for (int e = threadIdx.x; e < p.m * per_tok; e += kCW * 32) {
@@ -420,7 +426,7 @@ struct Q6 {
     // (s = 0) or / 256 (s = 1) for q = qp + 2s, l = 16 lh + 4 ((k + t') mod 4)
     // + {0, 2 | 1, 3}, v = 128h + 32q + l (h, lh of quarter t').
     // X[tok][block][t'][qp][s] = sum over the 16 l of binary16(x[v]).
-    static __device__ void build(const SP& p, uint32_t sb, float& amax) {
+    static __device__ void build(const SP& p, uint32_t sb, float& amax, int64_t xoff) {
         const int per_tok = p.nblk * 16 * 4;
         for (int e = threadIdx.x; e < p.m * per_tok; e += kCW * 32) {
             const int tok = e / per_tok, rem = e % per_tok;
@@ -569,14 +575,14 @@ struct Q4 {
     // Image per block and token: MMA (nib, u) of lane t uses values
     // v = 64t + 32nib + 4u + {0,2 | 1,3}; the last 32 bytes hold (Xhi, Xlo)
     // of sub-blocks 2t and 2t+1.
-    static __device__ void build(const SP& p, uint32_t sb, float& amax) {
+    static __device__ void build(const SP& p, uint32_t sb, float& amax, int64_t xoff) {
         const int items = p.m * p.nblk * 4;
         for (int it = threadIdx.x; it < items; it += kCW * 32) {
             const int tok = it / (p.nblk * 4), rem = it % (p.nblk * 4), bl = rem >> 2, t = rem & 3;
             const uint32_t base = sb + p.off_img + tok * p.img_tok + bl * kBlkImg;
             const int64_t xi = static_cast<int64_t>(bl) * 256 + 64 * t;
             const uint32_t xs = xaddr(p, sb, tok, xi);
-            const uint16_t* xg = p.x + static_cast<int64_t>(tok) * p.k + xi;
+            const uint16_t* xg = p.x + static_cast<int64_t>(tok) * p.k * p.ks + xoff + xi;
             float X[2] = {0.f, 0.f};
 #pragma unroll
             for (int nib = 0; nib < 2; ++nib) {
@@ -612,20 +618,29 @@ struct Q4 {
 // ===========================================================================
 // Kernel
 // ===========================================================================
-template <class C>
+// SPLIT: the launch is in clusters of p.ks CTAs that split K (compiled out
+// otherwise, so the unsplit kernel carries none of it).
+template <class C, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);   // [kMaxStages]
     uint64_t* empty = full + kMaxStages;                   // [kMaxStages]
     uint64_t* xbar = full + 2 * kMaxStages;
+    uint64_t* pfree = xbar + 1;                            // [2] partial-sum slots released
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 128);
     int* grp_done = reinterpret_cast<int*>(smem + 256);   // [kMaxGroups]
     const uint32_t sb = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t r0 = static_cast<int64_t>(blockIdx.x) * p.n / gridDim.x;
-    const int64_t r1 = static_cast<int64_t>(blockIdx.x + 1) * p.n / gridDim.x;
+    // A cluster of p.ks CTAs owns a balanced contiguous range of rows; CTA
+    // `rank` of it covers blocks [rank nblk, (rank + 1) nblk) of every row.
+    const int ks = SPLIT ? p.ks : 1;
+    const int rank = SPLIT ? static_cast<int>(cluster_ctarank()) : 0;
+    const int ncl = static_cast<int>(gridDim.x) / ks, cl = static_cast<int>(blockIdx.x) / ks;
+    const int64_t r0 = static_cast<int64_t>(cl) * p.n / ncl;
+    const int64_t r1 = static_cast<int64_t>(cl + 1) * p.n / ncl;
     const int nrg = cdiv(r1 - r0, kRows);
     const uint32_t stage_bytes = kRows * p.rs;
+    const int64_t kb0 = static_cast<int64_t>(rank) * p.nblk;   // first block of the slice
 
     if (tid == 0) {
         for (int i = 0; i < p.ns; ++i) {
@@ -633,6 +648,10 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
             mbar_init(&empty[i], kCW);
         }
         mbar_init(xbar, 1);
+        if (SPLIT) {
+            mbar_init(&pfree[0], 1);
+            mbar_init(&pfree[1], 1);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -654,7 +673,8 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
                 const uint32_t row = 2u * static_cast<uint32_t>(p.k);
                 mbar_arrive_expect_tx(xbar, row * p.m);
                 for (int tok = 0; tok < p.m; ++tok)
-                    bulk_g2s(smem + p.off_xraw + tok * row, p.x + static_cast<int64_t>(tok) * p.k, row, xbar);
+                    bulk_g2s(smem + p.off_xraw + tok * row, p.x + static_cast<int64_t>(tok) * p.k * ks + kb0 * C::kVPB,
+                             row, xbar);
             }
         }
         int q = 0;
@@ -677,7 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
                 __syncwarp();
                 if (lane < rv)
                     bulk_g2s(smem + p.off_stage + slot * stage_bytes + lane * p.rs,
-                             p.w + (row0 + lane) * p.row_bytes + static_cast<int64_t>(b0) * C::kBPB, bytes,
+                             p.w + (row0 + lane) * p.row_bytes + (kb0 + b0) * C::kBPB, bytes,
                              &full[slot]);
             }
         }
@@ -695,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
         float amax = 0.f;
         if (!spin_wait(xbar, 0, p.status)) *abort_flag = 1;
         if (!*abort_flag) {
-            C::build(p, sb, amax);
+            C::build(p, sb, amax, kb0 * C::kVPB);
             for (uint32_t o = 4 * tid; o < C::kZero; o += 4 * kCW * 32) sts32(sb + p.off_zero + o, 0u);
         }
         if (amax >= 65504.0f) atomicOr(p.status, KQ_DEV_X_RANGE);
@@ -715,7 +735,10 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
                 const int slot = q % p.ns;
                 const int i0 = st * p.g / C::kItemBlocks;
                 const int i1 = min(items_per_row, (st + 1) * p.g / C::kItemBlocks);
-                const int first = i0 + ((warp - i0) % kCW + kCW) % kCW;
+                // items continue the round robin of the previous row groups, so
+                // that rows with fewer items than warps still spread over all
+                const int rot = SPLIT ? rg * items_per_row : 0;
+                const int first = i0 + ((warp - i0 - rot) % kCW + kCW) % kCW;
                 // every warp waits for the stage, items or not, so that its
                 // release below always belongs to this fill of the slot
                 if (!spin_wait(&full[slot], (q / p.ns) & 1, p.status)) {
@@ -735,8 +758,17 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
             }
             if (!ok) break;
             // partial sums -> shared memory; the last warp of the row group sums
-            // the 16 partials in warp order and stores y
-            float* pw = part + (rg * kCW + warp) * kRows * p.m;
+            // the 16 partials in warp order and stores y (or, when the cluster
+            // splits K, this CTA's share of y for the cluster reduction).  With
+            // two slots, row group rg reuses the slot of rg - 2 once its sum is done.
+            const int pslot = SPLIT ? (rg & 1) : rg;
+            if (SPLIT && rg >= 2) {
+                if (!spin_wait(&pfree[rg & 1], ((rg >> 1) - 1) & 1, p.status)) {
+                    *abort_flag = 1;
+                    break;
+                }
+            }
+            float* pw = part + (pslot * kCW + warp) * kRows * p.m;
             C::store_part(p, L, acc, pw);
             __threadfence_block();
             __syncwarp();
@@ -745,55 +777,161 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
             last = __shfl_sync(0xffffffffu, last, 0);
             if (last) {
                 __threadfence_block();
-                for (int o = lane; o < kRows * p.m; o += 32) {
-                    const int tok = o / kRows, r = o % kRows;
-                    float sum = 0.f;
-                    for (int w = 0; w < kCW; ++w) sum += part[((rg * kCW + w) * kRows + r) * p.m + tok];
-                    if (r < rv) p.y[static_cast<int64_t>(tok) * p.n + row0 + r] = sum;
+                // split: the sum of this slice goes to the CTA that owns the
+                // row group (rg mod ks), into its receive slot for this rank
+                const uint32_t recv = sb + p.off_red +
+                                      4u * static_cast<uint32_t>(((rg / ks) * ks + rank) * kRows * p.m);
+                const uint32_t dst = SPLIT ? mapa_u32(recv, static_cast<uint32_t>(rg % ks)) : 0u;
+                if constexpr (SPLIT) {
+                    // element f = r m + tok of the row group, four per 16-byte
+                    // load, the 16 partials added in warp order
+                    const int nv4 = kRows * p.m / 4;
+                    const uint32_t pbase = sb + p.off_part + 16u * static_cast<uint32_t>(pslot * kCW * nv4);
+                    for (int f4 = lane; f4 < nv4; f4 += 32) {
+                        float sum[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                        for (int w = 0; w < kCW; ++w) {
+                            const uint4 v = lds128(pbase + 16u * static_cast<uint32_t>(w * nv4 + f4));
+                            sum[0] += __uint_as_float(v.x);
+                            sum[1] += __uint_as_float(v.y);
+                            sum[2] += __uint_as_float(v.z);
+                            sum[3] += __uint_as_float(v.w);
+                        }
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) st_cluster_f32(dst + 16u * f4 + 4u * c, sum[c]);
+                    }
+                } else {
+                    for (int o = lane; o < kRows * p.m; o += 32) {
+                        const int tok = o / kRows, r = o % kRows;
+                        float sum = 0.f;
+                        for (int w = 0; w < kCW; ++w) sum += part[((pslot * kCW + w) * kRows + r) * p.m + tok];
+                        if (r < rv) p.y[static_cast<int64_t>(tok) * p.n + row0 + r] = sum;
+                    }
                 }
+                __syncwarp();
+                if (SPLIT && lane == 0) mbar_arrive(&pfree[rg & 1]);
             }
         }
     }
-    __syncthreads();
+    if constexpr (SPLIT) {
+        // Every CTA of the cluster has pushed its slice sums of every row
+        // group to the row group's owner; the owner adds them in slice order.
+        // Nothing touches another CTA's shared memory after this barrier.
+        __syncwarp();
+        cluster_sync();
+        if (!*abort_flag) {
+            for (int rg = rank; rg < nrg; rg += ks) {
+                const int64_t row0 = r0 + static_cast<int64_t>(group_order(rg, nrg, r1 - r0)) * kRows;
+                const int rv = static_cast<int>(r1 - row0 < kRows ? r1 - row0 : kRows);
+                const float* recv = reinterpret_cast<const float*>(smem + p.off_red) + (rg / ks) * ks * kRows * p.m;
+                for (int f = tid; f < kRows * p.m; f += kThreads) {
+                    const int r = f / p.m, tok = f - r * p.m;
+                    if (r >= rv) continue;
+                    float sum = 0.f;
+                    for (int j = 0; j < ks; ++j) sum += recv[j * kRows * p.m + f];
+                    p.y[static_cast<int64_t>(tok) * p.n + row0 + r] = sum;
+                }
+            }
+        }
+    } else {
+        __syncthreads();
+    }
 }
 
 constexpr uint32_t align16(uint32_t v) { return (v + 15u) & ~15u; }
 
+// CTAs of this kernel resident at once when launched in clusters of ks
+// (one CTA per SM; clusters are placed within a GPC, so for ks > 2 fewer
+// than all SMs can be used), cached per device.
+template <class C>
+int resident_ctas(int ks, uint32_t smem) {
+    static int cache[64][4] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    const int slot = ks == 1 ? 0 : (ks == 2 ? 1 : (ks == 4 ? 2 : 3));
+    if (cache[dev][slot]) return cache[dev][slot];
+    const int sms = device_sm_count();
+    int n = sms;
+    if constexpr (C::kBPB != 144) {
+        if (ks > 1) return 0;
+    } else if (ks > 1) {
+        // the query needs the launch's shared-memory size to be allowed
+        if (cudaFuncSetAttribute(qmv_stream_kernel<C, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return 0;
+        }
+        cudaLaunchConfig_t q{};
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = ks;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        q.gridDim = dim3(sms / ks * ks);
+        q.blockDim = dim3(kThreads);
+        q.dynamicSmemBytes = smem;
+        q.attrs = at;
+        q.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, qmv_stream_kernel<C, true>, &q) != cudaSuccess) {
+            cudaGetLastError();
+            clusters = 0;
+        }
+        n = clusters * ks;
+    }
+    cache[dev][slot] = n;
+    return n;
+}
+
+// ks: CTAs of a cluster that split K (1, 2, 4, 8; a divisor of the block
+// count), each covering nblk / ks blocks of every row of the cluster's rows.
 template <class C>
 int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m, float* y, cudaStream_t st,
-                  uint32_t img_tok, uint32_t xs_tok) {
+                  uint32_t img_tok, uint32_t xs_tok, int ks = 1) {
     SP p{};
     p.w = static_cast<const uint8_t*>(w);
     p.x = x;
     p.y = y;
     p.status = device_status_ptr();
     p.n = n;
-    p.k = k;
     p.m = m;
-    p.nblk = static_cast<int>(k / C::kVPB);
-    p.row_bytes = static_cast<int64_t>(p.nblk) * C::kBPB;
+    const int nblk_all = static_cast<int>(k / C::kVPB);
+    if (ks < 1 || nblk_all % ks != 0) return KQ_ERR_UNSUPPORTED;
+    p.ks = ks;
+    p.nblk = nblk_all / ks;
+    p.k = static_cast<int64_t>(p.nblk) * C::kVPB;
+    p.row_bytes = static_cast<int64_t>(nblk_all) * C::kBPB;
     if (p.row_bytes % 16 != 0) return KQ_ERR_UNSUPPORTED;
+    if ((static_cast<int64_t>(p.nblk) * C::kBPB) % 16 != 0) return KQ_ERR_UNSUPPORTED;   // slice copies
     p.img_tok = img_tok;
     p.xs_tok = xs_tok;
-    const int sms = device_sm_count();
-    const int64_t gmax = (n + 7) / 8;   // at least 8 rows per CTA
-    const int grid = static_cast<int>(sms < gmax ? sms : (gmax > 0 ? gmax : 1));
-    const int nrg_max = cdiv(cdiv(n, grid), kRows);
-    if (nrg_max > kMaxGroups) return KQ_ERR_UNSUPPORTED;
     const uint32_t optin = static_cast<uint32_t>(device_smem_optin());
+    const int slots = resident_ctas<C>(ks, optin);
+    const int64_t gmax = (n + 7) / 8;   // at least 8 rows per cluster
+    int64_t ncl = slots / ks;
+    if (ncl > gmax) ncl = gmax;
+    if (ncl < 1) return KQ_ERR_UNSUPPORTED;
+    const int grid = static_cast<int>(ncl) * ks;
+    const int nrg_max = cdiv(cdiv(n, ncl), kRows);
+    if (nrg_max > kMaxGroups) return KQ_ERR_UNSUPPORTED;
     // fixed part of the layout
     p.off_img = kHdr;
     p.off_xs = align16(p.off_img + m * img_tok);
     p.off_zero = align16(p.off_xs + m * xs_tok);
     p.off_part = align16(p.off_zero + C::kZero);
     p.off_xraw = p.off_part;   // the raw x copy is dead before any partial sum is written
-    const uint32_t part = static_cast<uint32_t>(nrg_max) * kCW * kRows * m * 4;
-    uint32_t xraw = static_cast<uint32_t>(m) * static_cast<uint32_t>(k) * 2;
+    // split: two row-group slots of partial sums, reused in turn
+    const uint32_t part = static_cast<uint32_t>(ks > 1 ? 2 : nrg_max) * kCW * kRows * m * 4;
+    // receive slots of the row groups this CTA owns: ceil(nrg / ks) x ks slices
+    const uint32_t red = ks > 1 ? static_cast<uint32_t>(cdiv(nrg_max, ks) * ks) * kRows * m * 4 : 0;
+    uint32_t xraw = static_cast<uint32_t>(m) * static_cast<uint32_t>(p.k) * 2;
     // q4_K can build its image from global memory when the raw copy would
     // crowd out the weight stages
-    p.x_global = (C::kBPB == 144 && p.off_part + xraw + 2u * kRows * 2048u > optin) ? 1 : 0;
+    p.x_global = (C::kBPB == 144 && p.off_part + xraw + red + 2u * kRows * 2048u > optin) ? 1 : 0;
     if (p.x_global) xraw = 0;
-    p.off_stage = (p.off_part + (part > xraw ? part : xraw) + 127u) & ~127u;
+    p.off_red = align16(p.off_part + (part > xraw ? part : xraw));
+    p.off_stage = (p.off_red + red + 127u) & ~127u;
     // stage geometry: whole rows if two or more stages fit, else the fewest
     // equal row slices (a multiple of the item size, copies 16-byte sized)
     // that do; the deepest ring that fits
@@ -815,7 +953,12 @@ int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m,
     }
     if (p.ns == 0) return KQ_ERR_UNSUPPORTED;
     const uint32_t total = p.off_stage + static_cast<uint32_t>(p.ns) * kRows * p.rs;
-    auto kernel = qmv_stream_kernel<C>;
+    auto kernel = qmv_stream_kernel<C, false>;
+    if constexpr (C::kBPB == 144) {   // the K split is built for q4_K only
+        if (ks > 1) kernel = qmv_stream_kernel<C, true>;
+    } else if (ks > 1) {
+        return KQ_ERR_UNSUPPORTED;
+    }
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
     if (e != cudaSuccess) return record_cuda(e);
     cudaLaunchConfig_t cfg{};
@@ -823,11 +966,22 @@ int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m,
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = total;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (use_pdl()) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (ks > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = ks;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = use_pdl() ? 1 : 0;
+    cfg.numAttrs = na;
     return record_cuda(cudaLaunchKernelEx(&cfg, kernel, p));
 }
 
@@ -851,10 +1005,24 @@ int launch_qmv_stream(int type, const void* w, int64_t n, int64_t k, const uint1
         return m == 1 ? launch_stream<Q6<1>>(w, n, k, x, m, y, s, it, xt) : launch_stream<Q6<2>>(w, n, k, x, m, y, s, it, xt);
     }
     case KQ_Q4_K: {
+        // From M = 4 the activation image of a whole row crowds out the
+        // weight stages (and from M = 8 it no longer fits): K is then split
+        // over a cluster of 4 (else 2) CTAs, each covering a slice of at least
+        // 7 blocks.  Below M = 4 the split's cluster reduction costs more than
+        // it saves (measured).
         const int nblk = static_cast<int>(k / 256);
-        const uint32_t it = nblk * Q4<1>::kBlkImg;
-        if (m <= 8) return launch_stream<Q4<1>>(w, n, k, x, m, y, s, it, 0);
-        return launch_stream<Q4<2>>(w, n, k, x, m, y, s, it, 0);
+        int ks = 1;
+        if (m >= 4) {
+            if (nblk % 4 == 0 && nblk / 4 >= 7) ks = 4;
+            else if (nblk % 2 == 0 && nblk / 2 >= 7) ks = 2;
+        }
+        for (;;) {
+            const uint32_t it = (nblk / ks) * Q4<1>::kBlkImg;
+            const int rc = m <= 8 ? launch_stream<Q4<1>>(w, n, k, x, m, y, s, it, 0, ks)
+                                  : launch_stream<Q4<2>>(w, n, k, x, m, y, s, it, 0, ks);
+            if (rc != KQ_ERR_UNSUPPORTED || ks == 1) return rc;
+            ks = 1;
+        }
     }
     default: return KQ_ERR_UNSUPPORTED;
     }

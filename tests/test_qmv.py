@@ -58,6 +58,17 @@ def test_q4K_long_k_many_tokens(m):
     run(kq.Q4_K, 200, 8192, m, seed=40 + m)
 
 
+# q4_K from M = 4 splits K over a cluster of CTAs (4 CTAs when the slices
+# keep >= 7 blocks, else 2) and reduces the slices through the CTAs' shared
+# memory: clusters with fewer than 16 rows and a ragged row group (n = 37),
+# several row groups per cluster so that the two partial-sum slots are reused
+# (n = 2647), and the 2-CTA split (K = 3584: 14 blocks)
+@pytest.mark.parametrize("n,k,m", [(37, 7168, 4), (37, 7168, 12), (2647, 7168, 5), (300, 3584, 8),
+                                   (300, 3584, 16)])
+def test_q4K_split_k(n, k, m):
+    run(kq.Q4_K, n, k, m, seed=n + m)
+
+
 @pytest.mark.parametrize("qtype", CODECS)
 def test_deterministic_and_row_independent(qtype):
     n, k = 200, 4096
