@@ -1017,7 +1017,10 @@ int launch_qmv_stream(int type, const void* w, int64_t n, int64_t k, const uint1
             else if (nblk % 2 == 0 && nblk / 2 >= 7) ks = 2;
         }
         for (;;) {
-            const uint32_t it = (nblk / ks) * Q4<1>::kBlkImg;
+            // per-token image stride 32 bytes past a multiple of 128: the 8
+            // tokens of an MMA's B fragment then read disjoint banks
+            uint32_t it = (nblk / ks) * Q4<1>::kBlkImg;
+            it += (32u - it % 128u + 128u) % 128u;
             const int rc = m <= 8 ? launch_stream<Q4<1>>(w, n, k, x, m, y, s, it, 0, ks)
                                   : launch_stream<Q4<2>>(w, n, k, x, m, y, s, it, 0, ks);
             if (rc != KQ_ERR_UNSUPPORTED || ks == 1) return rc;
