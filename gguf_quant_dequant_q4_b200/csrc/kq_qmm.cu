@@ -453,6 +453,10 @@ __device__ __forceinline__ void decode_step(uint32_t row, int q, int p, int o6, 
 struct Unit {
     int e, ntile, nt;         // expert, weight tile, number of 64-row tiles
     int rs[4], nr[4];         // row_start / num_rows of each tile
+    // cont: the tiles are one run of rows [rs0, rs0 + rows) (full tiles back
+    // to back, only the last one partial), as in every dense unit and in the
+    // units of a map that tiles each expert segment in order
+    int cont, rs0, rows;
 };
 
 struct Pipe {
@@ -681,12 +685,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
+        U.cont = 1;
+#pragma unroll
+        for (int i = 1; i < 4; ++i)
+            if (i < U.nt && (U.nr[i - 1] != 64 || U.rs[i] != U.rs[i - 1] + 64)) U.cont = 0;
+        U.rs0 = U.rs[0];
+        U.rows = U.nt > 0 ? 64 * (U.nt - 1) + U.nr[U.nt - 1] : 0;
     };
-    // MMA N: one CTA trims it to the rows present; a pair splits N evenly
-    // between its CTAs (CTA r holds B rows [rN/2, (r+1)N/2)), so N is 128
-    // (one 64-row tile per CTA) or 256 (two per CTA)
+    // MMA N: one CTA trims it to the rows present.  A pair splits N evenly
+    // between its CTAs (CTA r holds B rows [rN/2, (r+1)N/2)): a run of rows
+    // takes N = rows rounded up to 32 (each CTA then holds a multiple of 16
+    // rows, loaded as 64-row boxes from the run's start), tiles that are not
+    // one run keep whole tiles per CTA, N = 128 (one each) or 256 (two each).
     auto mma_n = [&](const Unit& U) {
-        if constexpr (CG == 2) return U.nt <= 2 ? 128 : 256;
+        if constexpr (CG == 2) return U.cont ? (U.rows + 31) & ~31 : (U.nt <= 2 ? 128 : 256);
         else return 64 * (U.nt - 1) + ((U.nr[U.nt - 1] + 15) & ~15);
     };
     auto aborted = [&]() { return misc[1] != 0; };
@@ -712,10 +724,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (U.nt == 0) continue;
                 // this CTA's activation tiles of the unit: [t0, t1), at 64-row slots from 0
                 int t0 = 0, t1 = U.nt;
+                // a run of rows (pair): this CTA's rows start at `cr`; boxes
+                // (64 rows each, slots from 0) are loaded while they start
+                // inside the run, rows past it are never stored
+                int cr = 0, cb = 0, boxes = U.nt;
                 if constexpr (CG == 2) {
-                    const int tpc = mma_n(U) / 128;
-                    t0 = static_cast<int>(rank) * tpc;
-                    t1 = t0 + tpc < U.nt ? t0 + tpc : U.nt;
+                    if (U.cont) {
+                        const int half = mma_n(U) / 2;
+                        cr = static_cast<int>(rank) * half;
+                        boxes = 0;
+                        for (int r = 0; r < 2; ++r)
+                            for (int b = 0; 64 * b < half; ++b) {
+                                const bool in = r * half + 64 * b < U.rows;
+                                boxes += in;
+                                if (r == static_cast<int>(rank)) cb += in;
+                            }
+                    } else {
+                        const int tpc = mma_n(U) / 128;
+                        t0 = static_cast<int>(rank) * tpc;
+                        t1 = t0 + tpc < U.nt ? t0 + tpc : U.nt;
+                    }
                 }
                 for (int st = 0; st < nstages; ++st) {
                     if (!bwait(&b_empty[bp.idx], bp.phase ^ 1)) break;
@@ -723,12 +751,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if constexpr (CG == 2) {
                         // both CTAs' bytes land on CTA 0's full barrier; CTA 0
                         // expects the unit's total
-                        if (rank == 0) mbar_arrive_expect_tx(&b_full[bp.idx], KPS * U.nt * 8192);
+                        if (rank == 0) mbar_arrive_expect_tx(&b_full[bp.idx], KPS * boxes * 8192);
                         const uint32_t fb = lead(&b_full[bp.idx]);
+                        if (U.cont) {
 #pragma unroll
-                        for (int a = 0; a < KPS; ++a)
-                            for (int i = t0; i < t1; ++i)
-                                tma_load_2d_pair(dst + a * kBAtom + (i - t0) * 8192, &xmap, (st * KPS + a) * kBK, U.rs[i], fb);
+                            for (int a = 0; a < KPS; ++a)
+                                for (int b = 0; b < cb; ++b)
+                                    tma_load_2d_pair(dst + a * kBAtom + b * 8192, &xmap, (st * KPS + a) * kBK,
+                                                     U.rs0 + cr + 64 * b, fb);
+                        } else {
+#pragma unroll
+                            for (int a = 0; a < KPS; ++a)
+                                for (int i = t0; i < t1; ++i)
+                                    tma_load_2d_pair(dst + a * kBAtom + (i - t0) * 8192, &xmap, (st * KPS + a) * kBK,
+                                                     U.rs[i], fb);
+                        }
                     } else {
                         mbar_arrive_expect_tx(&b_full[bp.idx], KPS * U.nt * 8192);
 #pragma unroll
@@ -849,15 +886,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool row_ok = nrow < p.n;
             const uint32_t tbase = tmem + cp.idx * 256 + (static_cast<uint32_t>(32 * q) << 16);
             for (int c0 = 0; c0 < nmma; c0 += 16) {
-                const int ti = c0 >> 6;
-                const int r0 = c0 & 63;
-                const int nv = U.nr[ti] - r0;   // valid activation rows of this 16-column chunk
+                // activation row of column c0 and the valid rows of this
+                // 16-column chunk (column j is B row j: a run's row rs0 + j,
+                // else row j % 64 of tile j / 64)
+                int nv;
+                int64_t ar;
+                if (CG == 2 && U.cont) {
+                    nv = U.rows - c0;
+                    ar = static_cast<int64_t>(U.rs0) + c0;
+                } else {
+                    const int ti = c0 >> 6, r0 = c0 & 63;
+                    nv = U.nr[ti] - r0;
+                    ar = static_cast<int64_t>(U.rs[ti]) + r0;
+                }
                 if (nv <= 0) continue;          // warp-uniform
                 uint32_t v[16];
                 tmem_ld16(tbase + c0, v);
                 if (row_ok) {
                     // y is written once and never read here: streaming stores
-                    float* yp = p.y + (static_cast<int64_t>(U.rs[ti]) + r0) * p.n + nrow;
+                    float* yp = p.y + ar * p.n + nrow;
                     if (nv >= 16) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i) __stcs(yp + i * p.n, __uint_as_float(v[i]));

@@ -126,3 +126,20 @@ def test_c4_full_size_sampled():
         rr = np.nonzero(ref_ids == e)[0]
         ref = oracle.matmul(kq.Q4_K, w[e][cols], k, xs_ref[rr])
         check_qmm(y[rr][:, cols], ref, xn[rr], row_norms_w(kq.Q4_K, w[e][cols], k), k)
+
+
+@pytest.mark.parametrize("qtype", [kq.Q4_K, kq.Q8_0])
+def test_gather_row_runs_and_split_tiles(qtype):
+    # expert 0: one run of 202 rows over four tiles; expert 1: a 5-row run (the
+    # second CTA of a pair then holds no row); expert 2: two tiles that are not
+    # adjacent (rows 271..279 belong to no tile and stay unwritten)
+    n, k, rows = 300, 1024, 300
+    tiles = [(0, 0, 64), (0, 64, 64), (0, 128, 64), (0, 192, 10), (1, 202, 5), (2, 207, 64), (2, 280, 20)]
+    w, x, y, e = run_gather(qtype, 3, n, k, tiles[::-1], rows, seed=11)
+    assert e == 0
+    assert np.all(np.isnan(y[271:280]))
+    ref = oracle.gather_qmm(qtype, w, k, x, tiles)
+    xn = row_norms_x(x)
+    for ex, (lo, hi) in enumerate([(0, 202), (202, 207), (207, 300)]):
+        r = np.array([i for i in range(lo, hi) if not 271 <= i < 280])
+        check_qmm(y[r], ref[r], xn[r], row_norms_w(qtype, w[ex], k), k)
