@@ -24,6 +24,18 @@ and states the MoE semantics in plain numpy:
                    hanzo-ml quantized/mod.rs, ``indexed_moe_forward`` CPU
                    fallback that groups rows per expert and runs one
                    quantized matmul per expert).
+* ``gather_qmv``   decode-shaped MoE product, one output row per (token,
+                   slot) pair: y[p] = x[row(p)] @ dequant(w[ids[p]]).T
+                   (bindings.cpp, ``gather_qmv_kq``: "one activation row per
+                   expert slot", x [T, R, K], indices [T, R], output
+                   [T, R, N]; with one activation row per token the same
+                   product feeds the gate/up projections of
+                   ``moe_glu_gather_kq``).
+* ``inverse_order`` / ``gather_mix``  unsort and score mix of expert-sorted
+                   rows: out[t] = sum_s scores[t, s] * y[inv_order[t k + s]]
+                   (bindings.cpp, ``gather_mix``: f32 accumulation; hanzo-ml
+                   quantized/mod.rs ``moe_combine``: the per-slot outputs
+                   reduced by the router weights).
 """
 from __future__ import annotations
 
@@ -188,3 +200,53 @@ def gather_qmm(qtype: int, w_bank: np.ndarray, k: int, x_sorted: np.ndarray, til
         else:
             y[s:s + c] = r
     return (y, a) if absdot else y
+
+
+def gather_qmv(qtype: int, w_bank: np.ndarray, k: int, x_bf16: np.ndarray, ids: np.ndarray,
+               x_per_token: bool = False, absdot: bool = False):
+    """fp64 y[P, N] for the P = T * top_k (token, slot) pairs of ids [T, top_k]:
+    y[p] = x[p] @ dequant(w_bank[ids.flat[p]]).T, or x[p // top_k] when x holds
+    one row per token.  Rows of pairs whose id is out of range are NaN
+    (left unwritten).  Each row is independent; rows of one expert are simply
+    computed together."""
+    ids = np.asarray(ids, dtype=np.int64)
+    top_k = ids.shape[-1] if ids.ndim > 1 else 1
+    flat = ids.reshape(-1)
+    x = np.asarray(x_bf16, dtype=np.uint16).reshape(-1, k)
+    rows = np.arange(flat.size) // top_k if x_per_token else np.arange(flat.size)
+    n = w_bank.shape[1]
+    y = np.full((flat.size, n), np.nan)
+    a = np.full((flat.size, n), np.nan) if absdot else None
+    for e in range(w_bank.shape[0]):
+        sel = np.nonzero(flat == e)[0]
+        if sel.size == 0:
+            continue
+        r = matmul(qtype, w_bank[e], k, x[rows[sel]], absdot=absdot)
+        if absdot:
+            y[sel], a[sel] = r
+        else:
+            y[sel] = r
+    return (y, a) if absdot else y
+
+
+def inverse_order(sorted_pair: np.ndarray) -> np.ndarray:
+    """inv[sorted_pair[r]] = r: the sorted row of every (token, slot) pair."""
+    sp = np.asarray(sorted_pair, dtype=np.int64)
+    inv = np.empty(sp.size, dtype=np.int32)
+    inv[sp] = np.arange(sp.size, dtype=np.int32)
+    return inv
+
+
+def gather_mix(y: np.ndarray, inv_order: np.ndarray, scores: np.ndarray) -> np.ndarray:
+    """out[t] = sum over s = 0, 1, .. of scores[t, s] * y[inv_order[t k + s]], in
+    fp32: each product rounded to fp32, then added to the running fp32 sum
+    (which starts at zero), slots in ascending order."""
+    y = np.asarray(y, dtype=np.float32)
+    sc = np.asarray(scores, dtype=np.float32)
+    t, kk = sc.shape
+    inv = np.asarray(inv_order, dtype=np.int64).reshape(t, kk)
+    out = np.zeros((t, y.shape[1]), dtype=np.float32)
+    for s in range(kk):
+        prod = (sc[:, s:s + 1] * y[inv[:, s]]).astype(np.float32)
+        out = (out + prod).astype(np.float32)
+    return out

@@ -319,3 +319,85 @@ def test_gather_uncovered_rows_unwritten():
     y = oracle.gather_qmm(Q8_0, w, k, x, [(1, 2, 3)])
     assert np.all(np.isnan(y[:2])) and np.all(np.isnan(y[5:]))
     assert np.array_equal(y[2:5], oracle.matmul(Q8_0, w[1], k, x[2:5]))
+
+
+# ----------------------------------------------------------------------------
+# decode MoE: gather_qmv (one output row per (token, slot) pair) and the
+# unsort + score mix gather_mix
+# ----------------------------------------------------------------------------
+def test_gather_qmv_one_hot_picks_expert_columns():
+    # Two q8_0 experts of hand-built blocks (d = 1, so W = the int8 codes) and a
+    # third expert of q8_0 blocks with d = 0.5.  A one-hot activation row at
+    # column c returns column c of the routed expert's matrix, so every output
+    # follows from the closed form d * q without the oracle's decoder.
+    n, k = 4, 64
+    codes = np.arange(3 * n * k, dtype=np.int64).reshape(3, n, k) % 251 - 125
+    d = [1.0, 1.0, 0.5]
+    w = np.zeros((3, n, 2 * 34), dtype=np.uint8)
+    for e in range(3):
+        for b in range(2):
+            w[e, :, 34 * b:34 * b + 2] = np.array([d[e]], dtype=np.float16).view(np.uint8)
+            w[e, :, 34 * b + 2:34 * b + 34] = codes[e, :, 32 * b:32 * b + 32].astype(np.int8).view(np.uint8)
+    ids = np.array([[2, 0], [1, 2], [0, 1]], dtype=np.int32)      # 3 tokens, top-2
+    cols = [5, 40, 63, 0, 33, 17]                                 # one per pair
+    x = np.zeros((6, k), np.float32)
+    for p, c in enumerate(cols):
+        x[p, c] = 1.0
+    y = oracle.gather_qmv(Q8_0, w, k, synth.f32_to_bf16_bits(x), ids)
+    for p, c in enumerate(cols):
+        e = ids.reshape(-1)[p]
+        assert np.array_equal(y[p], d[e] * codes[e, :, c].astype(np.float64))
+
+
+def test_gather_qmv_reductions():
+    # all pairs on one expert: the plain product; one activation row per token:
+    # the per-pair product with that row repeated for every slot; a bad id
+    # leaves its row unwritten
+    n, k, t, top_k = 9, 512, 3, 2
+    w = synth.weights(Q6_K, n, k, seed=51, experts=3)
+    xp = synth.activations(t * top_k, k, seed=52)
+    same = np.ones((t, top_k), np.int32)
+    assert np.array_equal(oracle.gather_qmv(Q6_K, w, k, xp, same), oracle.matmul(Q6_K, w[1], k, xp))
+    ids = np.array([[0, 2], [2, 1], [1, 0]], np.int32)
+    xt = synth.activations(t, k, seed=53)
+    a = oracle.gather_qmv(Q6_K, w, k, xt, ids, x_per_token=True)
+    b = oracle.gather_qmv(Q6_K, w, k, np.repeat(xt, top_k, axis=0), ids)
+    assert np.array_equal(a, b)
+    bad = ids.copy()
+    bad[1, 0] = 7
+    yb = oracle.gather_qmv(Q6_K, w, k, xp, bad)
+    assert np.all(np.isnan(yb[2])) and np.array_equal(np.delete(yb, 2, 0), np.delete(oracle.gather_qmv(Q6_K, w, k, xp, ids), 2, 0))
+
+
+def test_inverse_order_and_gather_mix_unsort():
+    ids = np.array([[2, 0], [0, 1], [2, 1]], dtype=np.int32)
+    _, pair = oracle.moe_sort(ids, 3)
+    inv = oracle.inverse_order(pair)
+    assert inv.tolist() == [4, 0, 1, 2, 5, 3]                    # worked by hand from the sort above
+    # top-1 with score 1: the mix is the unsort permutation, exactly
+    y = np.random.default_rng(5).standard_normal((6, 8)).astype(np.float32)
+    out = oracle.gather_mix(y, inv, np.ones((6, 1), np.float32))
+    assert np.array_equal(out, y[inv])
+
+
+def test_gather_mix_exact_values_and_order():
+    # exactly representable products and sums: out[0] = 0.5*y[1] + 0.25*y[0]
+    y = np.array([[4.0, -8.0], [2.0, 6.0], [1.0, 1.0]], np.float32)
+    inv = np.array([1, 0, 2, 1], np.int32)                       # 2 tokens, top-2
+    sc = np.array([[0.5, 0.25], [2.0, -1.0]], np.float32)
+    out = oracle.gather_mix(y, inv, sc)
+    assert out.tolist() == [[2.0, 1.0], [0.0, -4.0]]
+    # fp32 rounding at every step, slots in ascending order: 1e8 + 1 rounds back
+    # to 1e8 in fp32 (its spacing there is 8), so the result is 0, not the exact 1
+    y = np.array([[1e8], [1.0], [-1e8]], np.float32)
+    out = oracle.gather_mix(y, np.array([0, 1, 2], np.int32), np.ones((1, 3), np.float32))
+    assert out[0, 0] == 0.0
+    out = oracle.gather_mix(y, np.array([0, 2, 1], np.int32), np.ones((1, 3), np.float32))
+    assert out[0, 0] == 1.0
+    # a product is rounded to fp32 before it is added (no fused multiply-add):
+    # (1 + 2^-12)^2 = 1 + 2^-11 + 2^-24 rounds to 1 + 2^-11 in fp32, so adding
+    # -(1 + 2^-11) gives 0 (a fused form would keep 2^-24)
+    a = np.float32(1 + 2.0 ** -12)
+    y = np.array([[a], [-(1 + 2.0 ** -11)]], np.float32)
+    out = oracle.gather_mix(y, np.array([0, 1], np.int32), np.array([[a, 1.0]], np.float32))
+    assert out[0, 0] == 0.0
