@@ -17,8 +17,9 @@ The JSON line also carries:
                 the kernels, device -> host copy of the result, all timed
   cpu_baseline  the CPU oracle on a bounded sample of the workload (rank 0)
   rows          every other row of the hot path (dequantize, qmv at M up to
-                16, tcgen05 qmm, MoE sort + tile map + gather) on its own
-                workload: kernel time, GB/s or TFLOP/s, roofline fraction
+                16, tcgen05 qmm, MoE sort + tile map + gather, the unsort +
+                score mix, the decode MoE gather_qmv) on its own workload:
+                kernel time, GB/s or TFLOP/s, roofline fraction
   clocks        SM clock median and throttle reasons sampled while timing
 
 With --gpus N under torchrun every rank runs an independent replica of the
@@ -423,6 +424,36 @@ def measure_rows(kq, torch, dev, pk, args) -> dict:
     t = time_graph(torch, route, 8, s)
     launches += 3 * (8 + 3)
     rows["c4_moe_sort_and_tile_map"] = {"us": round(t * 1e3, 2), "launches_per_call": 3}
+    # c4 epilogue: unsort + score mix of the 1024 expert-sorted output rows
+    _, _, _, inv = kq.moe_sort(ids, e, with_inverse=True)
+    sc = torch.rand(tok, topk, device=dev)
+    mixo = torch.empty(tok, n, device=dev)
+    ys = [y] + [torch.randn_like(y) for _ in range(ncopies(y.numel() * 4 + mixo.numel() * 4) - 1)]
+    t = time_graph(torch, lambda i: kq.gather_mix(ys[i % len(ys)], inv, sc, out=mixo), reps, s)
+    launches += reps + 3
+    mb = (tok * topk + tok) * n * 4
+    rows["c4_gather_mix_t512_top2_n14336"] = {"kernel_us": round(t * 1e3, 2), "GB/s": round(mb / (t / 1e3) / 1e9, 1),
+                                             "frac_hbm": round(mb / (t / 1e3) / 1e9 / pk["hbm_gbs"], 4), "bytes": mb}
+    del ys, mixo, y
+    # decode MoE: gather_qmv on the same q4_K bank, 1 and 4 tokens routed
+    # top-2, one activation row per token (the gate/up product); the weight
+    # bytes are those of the distinct experts routed.  Rotating copies of the
+    # whole bank keep the experts' bytes out of L2 between launches.
+    ebytes = synth.row_bytes(Q4_K, k) * n
+    banks = [wb] + [wb.clone() for _ in range(ncopies(2 * ebytes) - 1)]
+    for tk in (1, 4):
+        rid = torch.from_numpy(synth.routing(tk, e, topk, seed=9)).to(dev)
+        distinct = int(torch.unique(rid).numel())
+        xd = bf(synth.activations(tk, k, seed=10))
+        yd = torch.empty(tk * topk, n, device=dev)
+        t = time_graph(torch, lambda i: kq.gather_qmv(xd, banks[i % len(banks)], Q4_K, rid, x_per_token=True,
+                                                      out=yd), reps, s)
+        launches += reps + 3
+        gbs = distinct * ebytes / (t / 1e3) / 1e9
+        rows[f"decode_moe_gather_qmv_q4K_8x14336x4096_t{tk}_top2"] = {
+            "kernel_us": round(t * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
+            "bytes": distinct * ebytes, "experts_read": distinct}
+    del banks
     rows["_launches"] = launches
     return rows
 
@@ -488,7 +519,7 @@ def run_reference(args, dist: Dist) -> dict | None:
 
 # ------------------------------------------------------------ profile cases
 CASES = ("qmv_q8_0", "qmv_q6_K", "qmv_q4_K_m1", "qmv_q4_K_m16", "dequant_q4_K", "qmm_q4_K", "qmm_q6_K",
-         "gather_q4_K")
+         "gather_q4_K", "gather_qmv_q4_K", "gather_mix")
 
 
 def run_case(name: str, iters: int) -> None:
@@ -527,6 +558,17 @@ def run_case(name: str, iters: int) -> None:
         sids, pair, xs = kq.moe_sort(torch.from_numpy(synth.routing(512, 8, 2)).to(dev), 8, xt)
         tmap, cnt = kq.expert_tile_map(sids, 8)
         fn = lambda: kq.gather_qmm(xs, wb, Q4_K, tmap, cnt)
+    elif name == "gather_qmv_q4_K":
+        wb = u8(synth.weights(Q4_K, 14336, 4096, experts=8))
+        xd = bf(synth.activations(4, 4096, seed=10))
+        rid = torch.from_numpy(synth.routing(4, 8, 2, seed=9)).to(dev)
+        fn = lambda: kq.gather_qmv(xd, wb, Q4_K, rid, x_per_token=True)
+    elif name == "gather_mix":
+        ids = torch.from_numpy(synth.routing(512, 8, 2)).to(dev)
+        _, _, _, inv = kq.moe_sort(ids, 8, with_inverse=True)
+        yy = torch.randn(1024, 14336, device=dev)
+        sc = torch.rand(512, 2, device=dev)
+        fn = lambda: kq.gather_mix(yy, inv, sc)
     else:
         raise SystemExit(f"unknown case {name}; one of {CASES}")
     for _ in range(iters):

@@ -39,9 +39,11 @@ SIGNATURES = {
     "kq_dequantize": (_int, [_int, _vp, _i64, _i64, _vp, _vp]),
     "kq_qmv": (_int, [_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp]),
     "kq_qmm": (_int, [_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp]),
-    "kq_moe_sort": (_int, [_vp, _i64, _i32, _i32, _vp, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "kq_moe_sort": (_int, [_vp, _i64, _i32, _i32, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "kq_expert_tile_map": (_int, [_vp, _i64, _i32, _vp, _i64, _vp, _vp, _vp]),
     "kq_gather_qmm": (_int, [_int, _vp, _i32, _i64, _i64, _vp, _i64, _vp, _vp, _i64, _vp, _vp, _vp]),
+    "kq_gather_qmv": (_int, [_int, _vp, _i32, _i64, _i64, _vp, _i32, _vp, _i64, _i32, _vp, _vp, _vp]),
+    "kq_gather_mix": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _vp, _vp]),
 }
 
 _lib = None
@@ -156,13 +158,15 @@ def map_capacity(rows: int, n_experts: int) -> int:
 
 
 def moe_sort(topk_ids: torch.Tensor, n_experts: int, x: torch.Tensor | None = None, err: torch.Tensor | None = None,
-             stream=None):
-    """Stable sort of routed pairs by expert: (sorted_ids, sorted_pair, x_sorted)."""
+             stream=None, with_inverse: bool = False):
+    """Stable sort of routed pairs by expert: (sorted_ids, sorted_pair, x_sorted),
+    plus inv_order (the sorted row of every pair) when with_inverse is set."""
     t, top_k = topk_ids.shape
     rows = t * top_k
     dev = topk_ids.device
     sids = torch.empty(rows, dtype=torch.int32, device=dev)
     pair = torch.empty(rows, dtype=torch.int32, device=dev)
+    inv = torch.empty(rows, dtype=torch.int32, device=dev) if with_inverse else None
     xs = None
     k = 0
     if x is not None:
@@ -170,9 +174,9 @@ def moe_sort(topk_ids: torch.Tensor, n_experts: int, x: torch.Tensor | None = No
         k = x.shape[1]
         xs = torch.empty(rows, k, dtype=x.dtype, device=dev)
     _need_cuda(topk_ids, x, xs, err)
-    _check(lib().kq_moe_sort(_ptr(topk_ids), t, top_k, n_experts, _ptr(x), k, _ptr(sids), _ptr(pair), _ptr(xs),
-                             _ptr(err), _stream(stream)), "kq_moe_sort")
-    return sids, pair, xs
+    _check(lib().kq_moe_sort(_ptr(topk_ids), t, top_k, n_experts, _ptr(x), k, _ptr(sids), _ptr(pair), _ptr(inv),
+                             _ptr(xs), _ptr(err), _stream(stream)), "kq_moe_sort")
+    return (sids, pair, xs, inv) if with_inverse else (sids, pair, xs)
 
 
 def expert_tile_map(sorted_ids: torch.Tensor, n_experts: int, cap: int | None = None,
@@ -200,4 +204,34 @@ def gather_qmm(x_sorted: torch.Tensor, w_bank: torch.Tensor, qtype: int, tile_ma
     _need_cuda(x_sorted, w_bank, tile_map, count, out, err)
     _check(lib().kq_gather_qmm(qtype, _ptr(w_bank), e, n, k, _ptr(x_sorted), rows, _ptr(tile_map), _ptr(count),
                                tile_map.shape[0], _ptr(out), _ptr(err), _stream(stream)), "kq_gather_qmm")
+    return out
+
+
+def gather_qmv(x: torch.Tensor, w_bank: torch.Tensor, qtype: int, ids: torch.Tensor, x_per_token: bool = False,
+               out: torch.Tensor | None = None, err: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Decode MoE product, one row per (token, slot) pair p = t * top_k + s:
+    y[p] = x[p] @ dequant(w_bank[ids[t, s]]).T (x [T*top_k, K]), or
+    x[t] @ ... with x_per_token (x [T, K]).  ids int32 [T, top_k]."""
+    x = _bf16_bits(x)
+    t, top_k = ids.shape
+    k = x.shape[-1]
+    e, n = w_bank.shape[0], w_bank.shape[1]
+    if out is None:
+        out = torch.empty(t * top_k, n, dtype=torch.float32, device=x.device)
+    _need_cuda(x, w_bank, ids, out, err)
+    _check(lib().kq_gather_qmv(qtype, _ptr(w_bank), e, n, k, _ptr(x), int(bool(x_per_token)), _ptr(ids), t, top_k,
+                               _ptr(out), _ptr(err), _stream(stream)), "kq_gather_qmv")
+    return out
+
+
+def gather_mix(y: torch.Tensor, inv_order: torch.Tensor, scores: torch.Tensor, out: torch.Tensor | None = None,
+               err: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out[t] = sum_s scores[t, s] * y[inv_order[t * top_k + s]] (fp32, slots in order)."""
+    rows, n = y.shape
+    t, top_k = scores.shape
+    if out is None:
+        out = torch.empty(t, n, dtype=torch.float32, device=y.device)
+    _need_cuda(y, inv_order, scores, out, err)
+    _check(lib().kq_gather_mix(_ptr(y), rows, n, _ptr(inv_order), _ptr(scores), t, top_k, _ptr(out), _ptr(err),
+                               _stream(stream)), "kq_gather_mix")
     return out

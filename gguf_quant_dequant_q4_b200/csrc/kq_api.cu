@@ -173,8 +173,8 @@ int kq_qmm(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int
 }
 
 int kq_moe_sort(const int32_t* topk_ids, int64_t n_tokens, int32_t top_k, int32_t n_experts, const uint16_t* x,
-                int64_t k, uint32_t* sorted_ids, int32_t* sorted_pair, uint16_t* x_sorted, int32_t* err_flag,
-                void* stream) {
+                int64_t k, uint32_t* sorted_ids, int32_t* sorted_pair, int32_t* inv_order, uint16_t* x_sorted,
+                int32_t* err_flag, void* stream) {
     if (n_tokens < 0 || top_k < 1 || n_experts < 1 || n_experts > 256) return KQ_ERR_INVALID_ARG;
     if (n_tokens * top_k > (int64_t(1) << 30)) return KQ_ERR_INVALID_ARG;
     if (n_tokens == 0) return KQ_OK;
@@ -183,8 +183,8 @@ int kq_moe_sort(const int32_t* topk_ids, int64_t n_tokens, int32_t top_k, int32_
         if (!x || k <= 0 || k % 8 != 0) return KQ_ERR_INVALID_ARG;
         if (!aligned16(x) || !aligned16(x_sorted)) return KQ_ERR_ALIGNMENT;
     }
-    return launch_moe_sort(topk_ids, n_tokens, top_k, n_experts, x, k, sorted_ids, sorted_pair, x_sorted, err_flag,
-                           static_cast<cudaStream_t>(stream));
+    return launch_moe_sort(topk_ids, n_tokens, top_k, n_experts, x, k, sorted_ids, sorted_pair, inv_order, x_sorted,
+                           err_flag, static_cast<cudaStream_t>(stream));
 }
 
 int kq_expert_tile_map(const uint32_t* sorted_ids, int64_t rows, int32_t n_experts, uint32_t* map, int64_t cap,
@@ -207,6 +207,35 @@ int kq_gather_qmm(int type, const void* w_bank, int32_t n_experts, int64_t n, in
     if (!x_sorted || !map || !count || !y) return KQ_ERR_INVALID_ARG;
     if (!aligned16(x_sorted) || !aligned16(y)) return KQ_ERR_ALIGNMENT;
     return launch_gather_qmm(type, w_bank, n_experts, n, k, x_sorted, rows, map, count, cap, y, err_flag,
+                             static_cast<cudaStream_t>(stream));
+}
+
+int kq_gather_qmv(int type, const void* w_bank, int32_t n_experts, int64_t n, int64_t k, const uint16_t* x,
+                  int32_t x_per_token, const int32_t* ids, int64_t n_tokens, int32_t top_k, float* y,
+                  int32_t* err_flag, void* stream) {
+    if (n_experts < 1 || n_experts > 256 || n_tokens < 0 || top_k < 1) return KQ_ERR_INVALID_ARG;
+    int rc = check_weights(type, w_bank, n, k);
+    if (rc) return rc;
+    if (n_tokens * top_k > 8192) return KQ_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(n_experts) * n > (int64_t(1) << 31) - 1) return KQ_ERR_INVALID_ARG;
+    if (n == 0 || n_tokens == 0) return KQ_OK;
+    if (!x || !ids || !y) return KQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y)) return KQ_ERR_ALIGNMENT;
+    const int pairs = static_cast<int>(n_tokens * top_k);
+    // distinct experts per token bound the pairs of one expert by n_tokens
+    const int m_cap = n_tokens < 16 ? static_cast<int>(n_tokens) : 16;
+    return launch_gather_qmv(type, w_bank, n_experts, n, k, x, x_per_token ? top_k : 1, ids, pairs, m_cap, y,
+                             err_flag, static_cast<cudaStream_t>(stream));
+}
+
+int kq_gather_mix(const float* y, int64_t rows, int64_t n, const int32_t* inv_order, const float* scores,
+                  int64_t n_tokens, int32_t top_k, float* out, int32_t* err_flag, void* stream) {
+    if (rows < 0 || n < 0 || n % 4 != 0 || n_tokens < 0 || top_k < 1 || top_k > 64) return KQ_ERR_INVALID_ARG;
+    if (n_tokens > (int64_t(1) << 31) - 1 || rows > (int64_t(1) << 31) - 1) return KQ_ERR_INVALID_ARG;
+    if (n == 0 || n_tokens == 0) return KQ_OK;
+    if (!inv_order || !scores || !out || (rows > 0 && !y)) return KQ_ERR_INVALID_ARG;
+    if ((y && !aligned16(y)) || !aligned16(out)) return KQ_ERR_ALIGNMENT;
+    return launch_gather_mix(y, rows, n, inv_order, scores, n_tokens, top_k, out, err_flag,
                              static_cast<cudaStream_t>(stream));
 }
 

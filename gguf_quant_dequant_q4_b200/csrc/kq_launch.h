@@ -31,14 +31,21 @@ int launch_qmv(int type, const void* w, int64_t n, int64_t k, const uint16_t* x,
 // it does not cover.
 int launch_qmv_stream(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int m, float* y,
                       cudaStream_t s);
+// Decode MoE product (one output row per (token, slot) pair) on the staged
+// kernel; KQ_ERR_UNSUPPORTED for shapes it does not cover.
+int launch_gather_qmv(int type, const void* w_bank, int n_experts, int64_t n, int64_t k, const uint16_t* x,
+                      int xdiv, const int32_t* ids, int pairs, int m_cap, float* y, int32_t* err_flag,
+                      cudaStream_t s);
 int launch_qmm(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int64_t m, float* y,
                cudaStream_t s);
 int launch_gather_qmm(int type, const void* w_bank, int n_experts, int64_t n, int64_t k,
                       const uint16_t* x_sorted, int64_t rows, const uint32_t* map, const uint32_t* count,
                       int64_t cap, float* y, int32_t* err_flag, cudaStream_t s);
 int launch_moe_sort(const int32_t* topk_ids, int64_t n_tokens, int top_k, int n_experts, const uint16_t* x,
-                    int64_t k, uint32_t* sorted_ids, int32_t* sorted_pair, uint16_t* x_sorted,
-                    int32_t* err_flag, cudaStream_t s);
+                    int64_t k, uint32_t* sorted_ids, int32_t* sorted_pair, int32_t* inv_order,
+                    uint16_t* x_sorted, int32_t* err_flag, cudaStream_t s);
+int launch_gather_mix(const float* y, int64_t rows, int64_t n, const int32_t* inv_order, const float* scores,
+                      int64_t n_tokens, int top_k, float* out, int32_t* err_flag, cudaStream_t s);
 int launch_tile_map(const uint32_t* sorted_ids, int64_t rows, int n_experts, uint32_t* map, int64_t cap,
                     uint32_t* count, int32_t* err_flag, cudaStream_t s);
 

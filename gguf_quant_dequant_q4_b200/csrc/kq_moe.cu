@@ -23,7 +23,8 @@ constexpr int kMaxExperts = 256;
 // their (token, slot) order.
 __global__ void __launch_bounds__(kSortThreads) moe_sort_kernel(const int32_t* __restrict__ ids, int rows, int n_experts,
                                                                  uint32_t* __restrict__ sorted_ids,
-                                                                 int32_t* __restrict__ sorted_pair, int32_t* err) {
+                                                                 int32_t* __restrict__ sorted_pair,
+                                                                 int32_t* __restrict__ inv, int32_t* err) {
     __shared__ int base[kMaxExperts];
     __shared__ int wcount[kSortThreads / 32][kMaxExperts];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -69,6 +70,9 @@ __global__ void __launch_bounds__(kSortThreads) moe_sort_kernel(const int32_t* _
             for (int w = 0; w < warp; ++w) pos += wcount[w][e];
             sorted_ids[pos] = static_cast<uint32_t>(e);
             sorted_pair[pos] = i;
+            if (inv) inv[i] = pos;
+        } else if (inv && i < rows) {
+            inv[i] = -1;
         }
         __syncthreads();
         // advance the per-expert bases by this chunk's counts
@@ -138,14 +142,43 @@ __global__ void __launch_bounds__(1024) tile_map_kernel(const uint32_t* __restri
     }
 }
 
+// out[t, c..c+3] = sum over s of scores[t, s] * y[inv[t k + s], c..c+3]:
+// one thread per (token, 4 columns), 16-byte loads and stores, fp32 product
+// then sum per slot in ascending order (explicitly rounded, never fused).
+__global__ void __launch_bounds__(256) gather_mix_kernel(const float* __restrict__ y, int64_t rows, int64_t n4,
+                                                          const int32_t* __restrict__ inv,
+                                                          const float* __restrict__ scores, int64_t n_tokens,
+                                                          int top_k, float* __restrict__ out, int32_t* err) {
+    const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    for (int64_t t = blockIdx.y; t < n_tokens; t += gridDim.y) {
+        if (c >= n4) continue;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < top_k; ++s) {
+            const int64_t r = __ldg(inv + t * top_k + s);
+            if (r < 0 || r >= rows) {
+                if (c == 0 && err) atomicOr(err, KQ_DEV_BAD_RANGE);
+                continue;
+            }
+            const float sc = __ldg(scores + t * top_k + s);
+            const float4 v = __ldcs(reinterpret_cast<const float4*>(y + r * n4 * 4) + c);
+            acc.x = __fadd_rn(acc.x, __fmul_rn(sc, v.x));
+            acc.y = __fadd_rn(acc.y, __fmul_rn(sc, v.y));
+            acc.z = __fadd_rn(acc.z, __fmul_rn(sc, v.z));
+            acc.w = __fadd_rn(acc.w, __fmul_rn(sc, v.w));
+        }
+        __stcs(reinterpret_cast<float4*>(out + t * n4 * 4) + c, acc);
+    }
+}
+
 }  // namespace
 
 int launch_moe_sort(const int32_t* topk_ids, int64_t n_tokens, int top_k, int n_experts, const uint16_t* x,
-                    int64_t k, uint32_t* sorted_ids, int32_t* sorted_pair, uint16_t* x_sorted, int32_t* err_flag,
-                    cudaStream_t s) {
+                    int64_t k, uint32_t* sorted_ids, int32_t* sorted_pair, int32_t* inv_order, uint16_t* x_sorted,
+                    int32_t* err_flag, cudaStream_t s) {
     const int rows = static_cast<int>(n_tokens * top_k);
     if (rows == 0) return KQ_OK;
-    moe_sort_kernel<<<1, kSortThreads, 0, s>>>(topk_ids, rows, n_experts, sorted_ids, sorted_pair, err_flag);
+    moe_sort_kernel<<<1, kSortThreads, 0, s>>>(topk_ids, rows, n_experts, sorted_ids, sorted_pair, inv_order,
+                                                err_flag);
     int rc = check_launch();
     if (rc || !x_sorted) return rc;
     int grid = (rows + 7) / 8;
@@ -159,6 +192,17 @@ int launch_tile_map(const uint32_t* sorted_ids, int64_t rows, int n_experts, uin
                     uint32_t* count, int32_t* err_flag, cudaStream_t s) {
     (void)cap;
     tile_map_kernel<<<1, 1024, 0, s>>>(sorted_ids, static_cast<int>(rows), n_experts, map, count, err_flag);
+    return check_launch();
+}
+
+int launch_gather_mix(const float* y, int64_t rows, int64_t n, const int32_t* inv_order, const float* scores,
+                      int64_t n_tokens, int top_k, float* out, int32_t* err_flag, cudaStream_t s) {
+    const int64_t n4 = n / 4;
+    const int64_t bx = (n4 + 255) / 256;
+    if (bx > 65535) return KQ_ERR_INVALID_ARG;
+    const int64_t by = n_tokens < 65535 ? n_tokens : 65535;
+    gather_mix_kernel<<<dim3(static_cast<unsigned>(bx), static_cast<unsigned>(by)), 256, 0, s>>>(
+        y, rows, n4, inv_order, scores, n_tokens, top_k, out, err_flag);
     return check_launch();
 }
 

@@ -41,6 +41,9 @@
 //
 // Partial sums of the 16 warps are combined in a fixed order by the last
 // warp to finish a row group: results are bitwise reproducible.
+#include <algorithm>
+#include <type_traits>
+
 #include "kq_device.cuh"
 #include "kq_launch.h"
 
@@ -72,6 +75,23 @@ struct SP {
     uint32_t off_red;   // split: receive slots of the cluster reduction
 };
 static_assert(sizeof(SP) == 120, "kernel parameter block size");
+
+// Gather mode (decode MoE, one output row per (token, slot) pair): the pairs
+// of an expert-id list are grouped by expert into "virtual experts" of at most
+// m pairs (ascending expert id, pairs in (token, slot) order, an expert with
+// more than m pairs takes several); the CTAs of a launch are spread evenly
+// over virtual experts [vbase, vbase + vcount), each CTA covering a
+// contiguous range of its expert's rows.  x row of pair q: q / xdiv; y row:
+// q.  A separate parameter type, so that the dense kernels keep their block.
+struct SPG : SP {
+    const int32_t* ids;   // [pairs] expert id of every (token, slot) pair
+    int32_t* err;         // caller's device flag word (nullable)
+    int pairs, xdiv, n_experts, vbase, vcount;
+};
+constexpr uint32_t kGList = 512;     // gather: pair list of the CTA (16 ints)
+constexpr uint32_t kGMisc = 576;     // gather: expert, pairs present, row range
+constexpr uint32_t kGCount = 1024;   // gather: pairs per expert (256 ints)
+constexpr uint32_t kGHdr = 2048;     // gather header size
 
 // Row groups are walked with a partial last group (fewer than 16 rows) moved
 // to the front: its small stage lands first and its decode overlaps the full
@@ -620,8 +640,100 @@ struct Q4 {
 // ===========================================================================
 // SPLIT: the launch is in clusters of p.ks CTAs that split K (compiled out
 // otherwise, so the unsplit kernel carries none of it).
-template <class C, bool SPLIT>
-__global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
+// Gather mode, all threads: this CTA's virtual expert (its expert, pairs and
+// row range) from the id list.  False when the launch has no virtual expert
+// for this CTA.
+__device__ bool gather_setup(const SPG& p, uint8_t* smem, int64_t& r0, int64_t& r1, int& ge, int& gm) {
+    int* cnt = reinterpret_cast<int*>(smem + kGCount);
+    int* glist = reinterpret_cast<int*>(smem + kGList);
+    volatile int* gmisc = reinterpret_cast<volatile int*>(smem + kGMisc);
+    volatile long long* grange = reinterpret_cast<volatile long long*>(smem + kGMisc + 16);
+    const int tid = threadIdx.x;
+    for (int e = tid; e < p.n_experts; e += kThreads) cnt[e] = 0;
+    __syncthreads();
+    int bad = 0;
+    for (int q = tid; q < p.pairs; q += kThreads) {
+        const int e = p.ids[q];
+        if (e < 0 || e >= p.n_experts) bad = 1;
+        else atomicAdd(&cnt[e], 1);
+    }
+    if (bad && p.err) atomicOr(p.err, KQ_DEV_BAD_EXPERT);
+    __syncthreads();
+    if (tid < 32) {
+        const int lane = tid;
+        // virtual experts per expert, lane l holding experts 8l .. 8l + 7
+        int loc[8], sum = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = 8 * lane + i;
+            loc[i] = e < p.n_experts ? (cnt[e] + p.m - 1) / p.m : 0;
+            sum += loc[i];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        const int vj = min(p.vcount, total - p.vbase);
+        if (lane == 0) gmisc[0] = -1;
+        __syncwarp();
+        if (vj > 0) {
+            // CTA c serves virtual expert floor(c vj / G); the CTAs of one
+            // virtual expert split its rows evenly
+            const int64_t G = gridDim.x, c = blockIdx.x;
+            const int vl = static_cast<int>(c * vj / G);
+            const int64_t cf = (static_cast<int64_t>(vl) * G + vj - 1) / vj;
+            const int64_t cn = (static_cast<int64_t>(vl + 1) * G + vj - 1) / vj - cf;
+            const int v = p.vbase + vl;
+            const int excl = incl - sum;
+            if (v >= excl && v < incl) {
+                int acc = excl, e = -1, b = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (e < 0 && v < acc + loc[i]) {
+                        e = 8 * lane + i;
+                        b = v - acc;
+                    }
+                    acc += loc[i];
+                }
+                gmisc[0] = e;
+                gmisc[1] = b;
+                gmisc[2] = min(p.m, cnt[e] - b * p.m);
+                grange[0] = (c - cf) * p.n / cn;
+                grange[1] = (c - cf + 1) * p.n / cn;
+            }
+        }
+        __syncwarp();
+        // the pairs of the virtual expert: ranks [b m, b m + present) among
+        // the pairs of expert e, in (token, slot) order
+        const int e = gmisc[0];
+        if (e >= 0) {
+            const int lo = gmisc[1] * p.m, hi = lo + gmisc[2];
+            int seen = 0;
+            for (int q0 = 0; q0 < p.pairs && seen < hi; q0 += 32) {
+                const int q = q0 + lane;
+                const bool hit = q < p.pairs && p.ids[q] == e;
+                const unsigned bal = __ballot_sync(0xffffffffu, hit);
+                const int rk = seen + __popc(bal & ((1u << lane) - 1u));
+                if (hit && rk >= lo && rk < hi) glist[rk - lo] = q;
+                seen += __popc(bal);
+            }
+        }
+    }
+    __syncthreads();
+    ge = gmisc[0];
+    if (ge < 0) return false;
+    gm = gmisc[2];
+    r0 = grange[0];
+    r1 = grange[1];
+    return true;
+}
+
+template <class C, bool SPLIT, class P = SP>
+__global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
+    constexpr bool GATHER = !std::is_same<P, SP>::value;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);   // [kMaxStages]
     uint64_t* empty = full + kMaxStages;                   // [kMaxStages]
@@ -636,9 +748,8 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
     const int ks = SPLIT ? p.ks : 1;
     const int rank = SPLIT ? static_cast<int>(cluster_ctarank()) : 0;
     const int ncl = static_cast<int>(gridDim.x) / ks, cl = static_cast<int>(blockIdx.x) / ks;
-    const int64_t r0 = static_cast<int64_t>(cl) * p.n / ncl;
-    const int64_t r1 = static_cast<int64_t>(cl + 1) * p.n / ncl;
-    const int nrg = cdiv(r1 - r0, kRows);
+    int64_t r0 = static_cast<int64_t>(cl) * p.n / ncl;
+    int64_t r1 = static_cast<int64_t>(cl + 1) * p.n / ncl;
     const uint32_t stage_bytes = kRows * p.rs;
     const int64_t kb0 = static_cast<int64_t>(rank) * p.nblk;   // first block of the slice
 
@@ -648,7 +759,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
             mbar_init(&empty[i], kCW);
         }
         mbar_init(xbar, 1);
-        if (SPLIT) {
+        if (SPLIT || GATHER) {
             mbar_init(&pfree[0], 1);
             mbar_init(&pfree[1], 1);
         }
@@ -663,6 +774,17 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
     // the tail of the earlier grid more than it gained.)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // gather: the expert's weights, the pairs present (x rows gathered and y
+    // rows scattered through the pair list) and the row range
+    const uint8_t* wbase = p.w;
+    int gm = p.m;
+    const int* glist = reinterpret_cast<const int*>(smem + kGList);
+    if constexpr (GATHER) {
+        int ge = 0;
+        if (!gather_setup(p, smem, r0, r1, ge, gm)) return;
+        wbase = p.w + static_cast<int64_t>(ge) * p.n * p.row_bytes;
+    }
+    const int nrg = cdiv(r1 - r0, kRows);
 
     if (warp == kProd) {
         // ---------------------------------------------------------- producer
@@ -672,9 +794,12 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
             } else {
                 const uint32_t row = 2u * static_cast<uint32_t>(p.k);
                 mbar_arrive_expect_tx(xbar, row * p.m);
-                for (int tok = 0; tok < p.m; ++tok)
-                    bulk_g2s(smem + p.off_xraw + tok * row, p.x + static_cast<int64_t>(tok) * p.k * ks + kb0 * C::kVPB,
-                             row, xbar);
+                for (int tok = 0; tok < p.m; ++tok) {
+                    // gather: token slots past the pairs present repeat the last pair's row
+                    int64_t xr = tok;
+                    if constexpr (GATHER) xr = glist[tok < gm ? tok : gm - 1] / p.xdiv;
+                    bulk_g2s(smem + p.off_xraw + tok * row, p.x + xr * p.k * ks + kb0 * C::kVPB, row, xbar);
+                }
             }
         }
         int q = 0;
@@ -697,7 +822,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
                 __syncwarp();
                 if (lane < rv)
                     bulk_g2s(smem + p.off_stage + slot * stage_bytes + lane * p.rs,
-                             p.w + (row0 + lane) * p.row_bytes + (kb0 + b0) * C::kBPB, bytes,
+                             wbase + (row0 + lane) * p.row_bytes + (kb0 + b0) * C::kBPB, bytes,
                              &full[slot]);
             }
         }
@@ -760,9 +885,12 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
             // partial sums -> shared memory; the last warp of the row group sums
             // the 16 partials in warp order and stores y (or, when the cluster
             // splits K, this CTA's share of y for the cluster reduction).  With
-            // two slots, row group rg reuses the slot of rg - 2 once its sum is done.
-            const int pslot = SPLIT ? (rg & 1) : rg;
-            if (SPLIT && rg >= 2) {
+            // two slots (K split, gather), row group rg reuses the slot of rg - 2
+            // once its sum is done; gather also reuses the two arrival counters,
+            // so a CTA may own any number of rows.
+            constexpr bool kReuse = SPLIT || GATHER;
+            const int pslot = kReuse ? (rg & 1) : rg;
+            if (kReuse && rg >= 2) {
                 if (!spin_wait(&pfree[rg & 1], ((rg >> 1) - 1) & 1, p.status)) {
                     *abort_flag = 1;
                     break;
@@ -773,7 +901,8 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
             __threadfence_block();
             __syncwarp();
             int last = 0;
-            if (lane == 0) last = atomicAdd(&grp_done[rg], 1) == kCW - 1;
+            int* gdone = &grp_done[GATHER ? (rg & 1) : rg];
+            if (lane == 0) last = atomicAdd(gdone, 1) == kCW - 1;
             last = __shfl_sync(0xffffffffu, last, 0);
             if (last) {
                 __threadfence_block();
@@ -805,11 +934,18 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const SP p) {
                         const int tok = o / kRows, r = o % kRows;
                         float sum = 0.f;
                         for (int w = 0; w < kCW; ++w) sum += part[((pslot * kCW + w) * kRows + r) * p.m + tok];
-                        if (r < rv) p.y[static_cast<int64_t>(tok) * p.n + row0 + r] = sum;
+                        if constexpr (GATHER) {
+                            if (r < rv && tok < gm) p.y[static_cast<int64_t>(glist[tok]) * p.n + row0 + r] = sum;
+                        } else {
+                            if (r < rv) p.y[static_cast<int64_t>(tok) * p.n + row0 + r] = sum;
+                        }
                     }
                 }
                 __syncwarp();
-                if (SPLIT && lane == 0) mbar_arrive(&pfree[rg & 1]);
+                // the slot's next row group counts from zero; it starts only
+                // after the release below
+                if (GATHER && lane == 0) *gdone = 0;
+                if (kReuse && lane == 0) mbar_arrive(&pfree[rg & 1]);
             }
         }
     }
@@ -884,11 +1020,19 @@ int resident_ctas(int ks, uint32_t smem) {
     return n;
 }
 
+// Gather-mode arguments (decode MoE); see SPG.
+struct GatherArgs {
+    const int32_t* ids;
+    int32_t* err;
+    int pairs, xdiv, n_experts;
+};
+
 // ks: CTAs of a cluster that split K (1, 2, 4, 8; a divisor of the block
 // count), each covering nblk / ks blocks of every row of the cluster's rows.
+// ga: gather mode (ks = 1), n the rows of one expert.
 template <class C>
 int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m, float* y, cudaStream_t st,
-                  uint32_t img_tok, uint32_t xs_tok, int ks = 1) {
+                  uint32_t img_tok, uint32_t xs_tok, int ks = 1, const GatherArgs* ga = nullptr) {
     SP p{};
     p.w = static_cast<const uint8_t*>(w);
     p.x = x;
@@ -897,7 +1041,7 @@ int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m,
     p.n = n;
     p.m = m;
     const int nblk_all = static_cast<int>(k / C::kVPB);
-    if (ks < 1 || nblk_all % ks != 0) return KQ_ERR_UNSUPPORTED;
+    if (ks < 1 || nblk_all % ks != 0 || (ga && ks != 1)) return KQ_ERR_UNSUPPORTED;
     p.ks = ks;
     p.nblk = nblk_all / ks;
     p.k = static_cast<int64_t>(p.nblk) * C::kVPB;
@@ -908,59 +1052,73 @@ int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m,
     p.xs_tok = xs_tok;
     const uint32_t optin = static_cast<uint32_t>(device_smem_optin());
     const int slots = resident_ctas<C>(ks, optin);
-    const int64_t gmax = (n + 7) / 8;   // at least 8 rows per cluster
-    int64_t ncl = slots / ks;
-    if (ncl > gmax) ncl = gmax;
-    if (ncl < 1) return KQ_ERR_UNSUPPORTED;
-    const int grid = static_cast<int>(ncl) * ks;
-    const int nrg_max = cdiv(cdiv(n, ncl), kRows);
-    if (nrg_max > kMaxGroups) return KQ_ERR_UNSUPPORTED;
-    // fixed part of the layout
-    p.off_img = kHdr;
-    p.off_xs = align16(p.off_img + m * img_tok);
-    p.off_zero = align16(p.off_xs + m * xs_tok);
-    p.off_part = align16(p.off_zero + C::kZero);
-    p.off_xraw = p.off_part;   // the raw x copy is dead before any partial sum is written
-    // split: two row-group slots of partial sums, reused in turn
-    const uint32_t part = static_cast<uint32_t>(ks > 1 ? 2 : nrg_max) * kCW * kRows * m * 4;
-    // receive slots of the row groups this CTA owns: ceil(nrg / ks) x ks slices
-    const uint32_t red = ks > 1 ? static_cast<uint32_t>(cdiv(nrg_max, ks) * ks) * kRows * m * 4 : 0;
-    uint32_t xraw = static_cast<uint32_t>(m) * static_cast<uint32_t>(p.k) * 2;
-    // q4_K can build its image from global memory when the raw copy would
-    // crowd out the weight stages
-    p.x_global = (C::kBPB == 144 && p.off_part + xraw + red + 2u * kRows * 2048u > optin) ? 1 : 0;
-    if (p.x_global) xraw = 0;
-    p.off_red = align16(p.off_part + (part > xraw ? part : xraw));
-    p.off_stage = (p.off_red + red + 127u) & ~127u;
-    // stage geometry: whole rows if two or more stages fit, else the fewest
-    // equal row slices (a multiple of the item size, copies 16-byte sized)
-    // that do; the deepest ring that fits
-    const int ga = C::kItemBlocks * (C::kBPB % 16 == 0 ? 1 : 8 / C::kItemBlocks);
-    p.ns = 0;
-    for (int s = 1; s <= 16 && p.ns == 0; ++s) {
-        const int g = cdiv(cdiv(p.nblk, s), ga) * ga;
-        if (s > 1 && g >= p.nblk) continue;
-        const uint32_t rs = ((static_cast<uint32_t>(g) * C::kBPB + 127u) & ~127u) + 16;
-        for (int ns = kMaxStages; ns >= 2; --ns) {
-            if (p.off_stage + static_cast<uint32_t>(ns) * kRows * rs <= optin) {
-                p.ns = ns;
-                p.g = g;
-                p.rs = rs;
-                p.spr = cdiv(p.nblk, g);
-                break;
+    // Shared-memory layout for at most nrg_max row groups per CTA (gather
+    // mode: any number, in two reused slots); the total size, or 0 when it
+    // does not fit.
+    auto layout = [&](int nrg_max) -> uint32_t {
+        if (!ga && nrg_max > kMaxGroups) return 0;
+        // fixed part of the layout
+        p.off_img = ga ? kGHdr : kHdr;
+        p.off_xs = align16(p.off_img + m * img_tok);
+        p.off_zero = align16(p.off_xs + m * xs_tok);
+        p.off_part = align16(p.off_zero + C::kZero);
+        p.off_xraw = p.off_part;   // the raw x copy is dead before any partial sum is written
+        // split: two row-group slots of partial sums, reused in turn
+        const uint32_t part = static_cast<uint32_t>(ks > 1 || ga ? 2 : nrg_max) * kCW * kRows * m * 4;
+        // receive slots of the row groups this CTA owns: ceil(nrg / ks) x ks slices
+        const uint32_t red = ks > 1 ? static_cast<uint32_t>(cdiv(nrg_max, ks) * ks) * kRows * m * 4 : 0;
+        uint32_t xraw = static_cast<uint32_t>(m) * static_cast<uint32_t>(p.k) * 2;
+        // q4_K can build its image from global memory when the raw copy would
+        // crowd out the weight stages (not in gather mode, whose x rows are
+        // gathered by the copy)
+        p.x_global = (C::kBPB == 144 && p.off_part + xraw + red + 2u * kRows * 2048u > optin) ? 1 : 0;
+        if (p.x_global && ga) return 0;
+        if (p.x_global) xraw = 0;
+        p.off_red = align16(p.off_part + (part > xraw ? part : xraw));
+        p.off_stage = (p.off_red + red + 127u) & ~127u;
+        // stage geometry: whole rows if two or more stages fit, else the fewest
+        // equal row slices (a multiple of the item size, copies 16-byte sized)
+        // that do; the deepest ring that fits
+        const int ga_blk = C::kItemBlocks * (C::kBPB % 16 == 0 ? 1 : 8 / C::kItemBlocks);
+        p.ns = 0;
+        for (int s = 1; s <= 16 && p.ns == 0; ++s) {
+            const int g = cdiv(cdiv(p.nblk, s), ga_blk) * ga_blk;
+            if (s > 1 && g >= p.nblk) continue;
+            const uint32_t rs = ((static_cast<uint32_t>(g) * C::kBPB + 127u) & ~127u) + 16;
+            for (int ns = kMaxStages; ns >= 2; --ns) {
+                if (p.off_stage + static_cast<uint32_t>(ns) * kRows * rs <= optin) {
+                    p.ns = ns;
+                    p.g = g;
+                    p.rs = rs;
+                    p.spr = cdiv(p.nblk, g);
+                    break;
+                }
             }
         }
+        if (p.ns == 0) return 0;
+        return p.off_stage + static_cast<uint32_t>(p.ns) * kRows * p.rs;
+    };
+    int grid = 0, launches = 1, vcount = 0;
+    uint32_t total = 0;
+    if (!ga) {
+        const int64_t gmax = (n + 7) / 8;   // at least 8 rows per cluster
+        int64_t ncl = slots / ks;
+        if (ncl > gmax) ncl = gmax;
+        if (ncl < 1) return KQ_ERR_UNSUPPORTED;
+        grid = static_cast<int>(ncl) * ks;
+        total = layout(cdiv(cdiv(n, ncl), kRows));
+    } else {
+        // Every CTA takes one virtual expert, any number of its rows; a
+        // launch serves up to one virtual expert per CTA, and there are
+        // enough launches for the most virtual experts the pairs can form.
+        grid = slots;
+        total = layout(2);
+        vcount = grid;
+        if (total == 0) return KQ_ERR_UNSUPPORTED;
+        const int64_t vmax = std::min<int64_t>(ga->pairs, cdiv(ga->pairs, m) + std::min(ga->n_experts, ga->pairs));
+        launches = static_cast<int>(cdiv(vmax, vcount));
     }
-    if (p.ns == 0) return KQ_ERR_UNSUPPORTED;
-    const uint32_t total = p.off_stage + static_cast<uint32_t>(p.ns) * kRows * p.rs;
-    auto kernel = qmv_stream_kernel<C, false>;
-    if constexpr (C::kBPB == 144) {   // the K split is built for q4_K only
-        if (ks > 1) kernel = qmv_stream_kernel<C, true>;
-    } else if (ks > 1) {
-        return KQ_ERR_UNSUPPORTED;
-    }
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
-    if (e != cudaSuccess) return record_cuda(e);
+    if (total == 0) return KQ_ERR_UNSUPPORTED;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
@@ -982,6 +1140,33 @@ int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m,
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
+    if (ga) {
+        auto kernel = qmv_stream_kernel<C, false, SPG>;
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
+        if (e != cudaSuccess) return record_cuda(e);
+        SPG g{};
+        static_cast<SP&>(g) = p;
+        g.ids = ga->ids;
+        g.err = ga->err;
+        g.pairs = ga->pairs;
+        g.xdiv = ga->xdiv;
+        g.n_experts = ga->n_experts;
+        g.vcount = vcount;
+        for (int j = 0; j < launches; ++j) {
+            g.vbase = j * vcount;
+            const int rc = record_cuda(cudaLaunchKernelEx(&cfg, kernel, g));
+            if (rc) return rc;
+        }
+        return KQ_OK;
+    }
+    auto kernel = qmv_stream_kernel<C, false>;
+    if constexpr (C::kBPB == 144) {   // the K split is built for q4_K only
+        if (ks > 1) kernel = qmv_stream_kernel<C, true>;
+    } else if (ks > 1) {
+        return KQ_ERR_UNSUPPORTED;
+    }
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
+    if (e != cudaSuccess) return record_cuda(e);
     return record_cuda(cudaLaunchKernelEx(&cfg, kernel, p));
 }
 
@@ -1026,6 +1211,44 @@ int launch_qmv_stream(int type, const void* w, int64_t n, int64_t k, const uint1
             if (rc != KQ_ERR_UNSUPPORTED || ks == 1) return rc;
             ks = 1;
         }
+    }
+    default: return KQ_ERR_UNSUPPORTED;
+    }
+}
+
+// Decode MoE product on the staged kernel: at most m_cap pairs of one expert
+// per virtual expert (q8_0 and q6_K take up to 2 activation rows, q4_K up to
+// 16 while the activation image fits; fewer when shared memory requires).
+int launch_gather_qmv(int type, const void* w_bank, int n_experts, int64_t n, int64_t k, const uint16_t* x,
+                      int xdiv, const int32_t* ids, int pairs, int m_cap, float* y, int32_t* err_flag,
+                      cudaStream_t s) {
+    GatherArgs ga{ids, err_flag, pairs, xdiv, n_experts};
+    const int nblk = static_cast<int>(k / (type == KQ_Q8_0 ? 32 : 256));
+    int rc = KQ_ERR_UNSUPPORTED;
+    switch (type) {
+    case KQ_Q8_0: {
+        if (nblk % 8 != 0) return KQ_ERR_UNSUPPORTED;
+        const uint32_t it = (nblk / 8) * Q8<1>::kItemImg, xt = nblk * 4;
+        rc = m_cap >= 2 ? launch_stream<Q8<2>>(w_bank, n, k, x, 2, y, s, it, xt, 1, &ga) : KQ_ERR_UNSUPPORTED;
+        if (rc == KQ_ERR_UNSUPPORTED) rc = launch_stream<Q8<1>>(w_bank, n, k, x, 1, y, s, it, xt, 1, &ga);
+        return rc;
+    }
+    case KQ_Q6_K: {
+        if (nblk % 8 != 0) return KQ_ERR_UNSUPPORTED;
+        const uint32_t it = nblk * Q6<1>::kBlkImg, xt = nblk * 16 * 4;
+        rc = m_cap >= 2 ? launch_stream<Q6<2>>(w_bank, n, k, x, 2, y, s, it, xt, 1, &ga) : KQ_ERR_UNSUPPORTED;
+        if (rc == KQ_ERR_UNSUPPORTED) rc = launch_stream<Q6<1>>(w_bank, n, k, x, 1, y, s, it, xt, 1, &ga);
+        return rc;
+    }
+    case KQ_Q4_K: {
+        uint32_t it = nblk * Q4<1>::kBlkImg;
+        it += (32u - it % 128u + 128u) % 128u;
+        for (int m = m_cap < 16 ? m_cap : 16; m >= 1; --m) {
+            rc = m <= 8 ? launch_stream<Q4<1>>(w_bank, n, k, x, m, y, s, it, 0, 1, &ga)
+                        : launch_stream<Q4<2>>(w_bank, n, k, x, m, y, s, it, 0, 1, &ga);
+            if (rc != KQ_ERR_UNSUPPORTED) return rc;
+        }
+        return rc;
     }
     default: return KQ_ERR_UNSUPPORTED;
     }

@@ -134,13 +134,16 @@ int kq_qmm(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int
  *   x           [n_tokens, k] bf16 (may be NULL when x_sorted is NULL)
  *   sorted_ids  [n_tokens*top_k] uint32 out: expert id of sorted row r
  *   sorted_pair [n_tokens*top_k] int32 out: token*top_k + slot of sorted row r
+ *   inv_order   [n_tokens*top_k] int32 out (nullable): the sorted row of pair
+ *               token*top_k + slot (the inverse permutation, as
+ *               kq_gather_mix takes it); -1 for a pair with a bad id
  *   x_sorted    [n_tokens*top_k, k] bf16 out (nullable): x[sorted_pair/top_k]
  *   err_flag    int32 device word (nullable): KQ_DEV_BAD_EXPERT on bad ids
  * Pairs with equal expert id keep (token, slot) order.  1 <= n_experts <= 256.
  */
 int kq_moe_sort(const int32_t* topk_ids, int64_t n_tokens, int32_t top_k, int32_t n_experts,
                 const uint16_t* x, int64_t k, uint32_t* sorted_ids, int32_t* sorted_pair,
-                uint16_t* x_sorted, int32_t* err_flag, void* stream);
+                int32_t* inv_order, uint16_t* x_sorted, int32_t* err_flag, void* stream);
 
 /*
  * kq_expert_tile_map - build the tile map of a segment-walking gather GEMM on
@@ -178,6 +181,50 @@ int kq_gather_qmm(int type, const void* w_bank, int32_t n_experts, int64_t n, in
                   const uint16_t* x_sorted, int64_t rows, const uint32_t* map,
                   const uint32_t* count, int64_t cap, float* y, int32_t* err_flag,
                   void* stream);
+
+/*
+ * kq_gather_qmv - decode-shaped MoE product with one output row per
+ * (token, slot) pair: y[p, :] = x[row(p), :] . dequant(W[ids[p]])^T for the
+ * p = token*top_k + slot pairs of ids [n_tokens, top_k].
+ * mlx-kquant bindings.cpp, `gather_qmv_kq` ("gathered matvec for K-quant
+ * expert stacks (the MoE down projection); one activation row per expert
+ * slot": x [T, R, K], w (n_experts, N, bytes_per_row), indices [T, R],
+ * output [T, R, N]).  With x_per_token != 0 x holds one row per token,
+ * row(p) = p / top_k, which is the gate/up product of `moe_glu_gather_kq`
+ * before its GLU; else row(p) = p.
+ *   w_bank [n_experts, n, row_bytes], x [n_tokens*top_k or n_tokens, k] bf16,
+ *   ids [n_tokens*top_k] int32, y [n_tokens*top_k, n] fp32.
+ * No host round trip: the pairs are grouped by expert on the device and each
+ * routed expert's weights are read once for all of its pairs (in batches of
+ * up to 2 (q8_0, q6_K) or 16 (q4_K) activation rows; an expert with more
+ * pairs than a batch is streamed once per batch).  Arithmetic as kq_qmv.
+ * Limits: 1 <= n_experts <= 256, 1 <= n_tokens*top_k <= 8192; k % 256 == 0
+ * (q8_0, q4_K) or k % 2048 == 0 (q6_K), else KQ_ERR_UNSUPPORTED.
+ *   err_flag (nullable): KQ_DEV_BAD_EXPERT for ids outside [0, n_experts);
+ *   the rows of those pairs are left unwritten.
+ */
+int kq_gather_qmv(int type, const void* w_bank, int32_t n_experts, int64_t n, int64_t k,
+                  const uint16_t* x, int32_t x_per_token, const int32_t* ids, int64_t n_tokens,
+                  int32_t top_k, float* y, int32_t* err_flag, void* stream);
+
+/*
+ * kq_gather_mix - unsort and score mix of expert-sorted MoE outputs:
+ * out[t, :] = sum over s = 0 .. top_k-1 of scores[t, s] * y[inv_order[t*top_k + s], :].
+ * mlx-kquant bindings.cpp, `gather_mix` (fused unsort and score mix for
+ * sorted-prefill MoE, f32 accumulation, N a multiple of 4); hanzo-ml
+ * quantized/mod.rs `moe_combine` (the per-slot outputs reduced by the router
+ * weights).  fp32 throughout, in a fixed order: each product rounded to
+ * fp32, then added to the running sum (which starts at 0), slots ascending;
+ * no fused multiply-add, so results are bit-reproducible.
+ *   y [rows, n] fp32 (e.g. kq_gather_qmm's output), inv_order
+ *   [n_tokens*top_k] int32 (kq_moe_sort's), scores [n_tokens, top_k] fp32,
+ *   out [n_tokens, n] fp32.  n % 4 == 0, else KQ_ERR_INVALID_ARG.
+ *   err_flag (nullable): KQ_DEV_BAD_RANGE for an inv_order entry outside
+ *   [0, rows); that term is left out of the sum.
+ */
+int kq_gather_mix(const float* y, int64_t rows, int64_t n, const int32_t* inv_order,
+                  const float* scores, int64_t n_tokens, int32_t top_k, float* out,
+                  int32_t* err_flag, void* stream);
 
 #ifdef __cplusplus
 }

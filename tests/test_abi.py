@@ -29,7 +29,8 @@ def declared_symbols():
 
 def test_header_declares_the_path():
     syms = declared_symbols()
-    for s in ("kq_dequantize", "kq_qmv", "kq_qmm", "kq_moe_sort", "kq_expert_tile_map", "kq_gather_qmm"):
+    for s in ("kq_dequantize", "kq_qmv", "kq_qmm", "kq_moe_sort", "kq_expert_tile_map", "kq_gather_qmm",
+              "kq_gather_qmv", "kq_gather_mix"):
         assert s in syms
 
 
@@ -86,12 +87,12 @@ def test_dequantize_argument_checks(lib):
 
 def test_moe_argument_checks(lib):
     s = lib.kq_moe_sort
-    assert s(A, 4, 0, 8, None, 0, A, A, None, None, None) == INVALID      # top_k < 1
-    assert s(A, 4, 2, 0, None, 0, A, A, None, None, None) == INVALID      # no experts
-    assert s(A, 4, 2, 257, None, 0, A, A, None, None, None) == INVALID
-    assert s(A, 4, 2, 8, None, 64, A, A, A, None, None) == INVALID        # x_sorted without x
-    assert s(A, 4, 2, 8, A, 60, A, A, A, None, None) == INVALID           # k % 8
-    assert s(A, 0, 2, 8, None, 0, A, A, None, None, None) == OK
+    assert s(A, 4, 0, 8, None, 0, A, A, None, None, None, None) == INVALID      # top_k < 1
+    assert s(A, 4, 2, 0, None, 0, A, A, None, None, None, None) == INVALID      # no experts
+    assert s(A, 4, 2, 257, None, 0, A, A, None, None, None, None) == INVALID
+    assert s(A, 4, 2, 8, None, 64, A, A, None, A, None, None) == INVALID        # x_sorted without x
+    assert s(A, 4, 2, 8, A, 60, A, A, A, A, None, None) == INVALID              # k % 8
+    assert s(A, 0, 2, 8, None, 0, A, A, A, None, None, None) == OK
     t = lib.kq_expert_tile_map
     assert t(A, 1024, 8, A, 23, A, None, None) == INVALID                 # cap < ceil(1024/64) + 8
     assert t(A, 1024, 8, None, 24, A, None, None) == INVALID
@@ -101,6 +102,28 @@ def test_moe_argument_checks(lib):
     assert g(kq.Q4_K, A, 8, 64, 256, None, 10, A, A, 8, A, None, None) == INVALID
     assert g(kq.Q4_K, A, 8, 64, 256, MIS, 10, A, A, 8, A, None, None) == ALIGN
     assert g(kq.Q4_K, A, 8, 64, 256, A, 0, A, A, 8, A, None, None) == OK
+
+
+def test_decode_moe_argument_checks(lib):
+    g = lib.kq_gather_qmv
+    assert g(3, A, 8, 64, 256, A, 0, A, 1, 2, A, None, None) == UNSUPPORTED      # unknown codec
+    assert g(kq.Q4_K, A, 0, 64, 256, A, 0, A, 1, 2, A, None, None) == INVALID    # no experts
+    assert g(kq.Q4_K, A, 257, 64, 256, A, 0, A, 1, 2, A, None, None) == INVALID
+    assert g(kq.Q4_K, A, 8, 64, 250, A, 0, A, 1, 2, A, None, None) == INVALID    # K not a block multiple
+    assert g(kq.Q4_K, A, 8, 64, 256, A, 0, A, 1, 0, A, None, None) == INVALID    # top_k < 1
+    assert g(kq.Q4_K, A, 8, 64, 256, A, 0, A, 4097, 2, A, None, None) == INVALID  # more than 8192 pairs
+    assert g(kq.Q4_K, A, 8, 64, 256, None, 0, A, 1, 2, A, None, None) == INVALID
+    assert g(kq.Q4_K, A, 8, 64, 256, A, 0, None, 1, 2, A, None, None) == INVALID
+    assert g(kq.Q4_K, A, 8, 64, 256, MIS, 0, A, 1, 2, A, None, None) == ALIGN
+    assert g(kq.Q4_K, A, 8, 64, 256, A, 0, A, 1, 2, MIS, None, None) == ALIGN
+    assert g(kq.Q4_K, A, 8, 64, 256, A, 0, A, 0, 2, A, None, None) == OK         # no tokens
+    m = lib.kq_gather_mix
+    assert m(A, 8, 6, A, A, 4, 2, A, None, None) == INVALID                      # n % 4
+    assert m(A, 8, 8, A, A, 4, 0, A, None, None) == INVALID                      # top_k < 1
+    assert m(A, 8, 8, None, A, 4, 2, A, None, None) == INVALID
+    assert m(A, 8, 8, A, A, 4, 2, MIS, None, None) == ALIGN
+    assert m(MIS, 8, 8, A, A, 4, 2, A, None, None) == ALIGN
+    assert m(A, 8, 8, A, A, 0, 2, A, None, None) == OK
 
 
 def test_binding_fails_loudly_without_library(monkeypatch):
