@@ -18,7 +18,8 @@ The JSON line also carries:
   cpu_baseline  the CPU oracle on a bounded sample of the workload (rank 0)
   rows          every other row of the hot path (dequantize, qmv at M up to
                 16, tcgen05 qmm, MoE sort + tile map + gather, the unsort +
-                score mix, the decode MoE gather_qmv) on its own workload:
+                score mix, the decode MoE gather_qmv and gate/up GLU) on its
+                own workload:
                 kernel time, GB/s or TFLOP/s, roofline fraction
   clocks        SM clock median and throttle reasons sampled while timing
 
@@ -453,6 +454,16 @@ def measure_rows(kq, torch, dev, pk, args) -> dict:
         rows[f"decode_moe_gather_qmv_q4K_8x14336x4096_t{tk}_top2"] = {
             "kernel_us": round(t * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
             "bytes": distinct * ebytes, "experts_read": distinct}
+        # the fused gate/up GLU on the same routing: two banks (gate = the
+        # rotating copies, up = the next copy), each routed expert read once
+        yg = torch.empty(tk * topk, n, device=dev)
+        t = time_graph(torch, lambda i: kq.moe_glu_gather(xd, banks[i % len(banks)], banks[(i + 1) % len(banks)],
+                                                          Q4_K, rid, out=yg), reps, s)
+        launches += reps + 3
+        gbs = 2 * distinct * ebytes / (t / 1e3) / 1e9
+        rows[f"decode_moe_glu_gather_q4K_2x8x14336x4096_t{tk}_top2"] = {
+            "kernel_us": round(t * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
+            "bytes": 2 * distinct * ebytes, "experts_read": distinct}
     del banks
     rows["_launches"] = launches
     return rows

@@ -44,7 +44,10 @@ SIGNATURES = {
     "kq_gather_qmm": (_int, [_int, _vp, _i32, _i64, _i64, _vp, _i64, _vp, _vp, _i64, _vp, _vp, _vp]),
     "kq_gather_qmv": (_int, [_int, _vp, _i32, _i64, _i64, _vp, _i32, _vp, _i64, _i32, _vp, _vp, _vp]),
     "kq_gather_mix": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _i32, _vp, _vp, _vp]),
+    "kq_moe_glu_gather": (_int, [_int, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _i32, _i32, ctypes.c_float,
+                                 _vp, _vp, _vp]),
 }
+ACT_SILU, ACT_GELU_TANH, ACT_SILU_LIMIT = 0, 1, 2
 
 _lib = None
 
@@ -234,4 +237,20 @@ def gather_mix(y: torch.Tensor, inv_order: torch.Tensor, scores: torch.Tensor, o
     _need_cuda(y, inv_order, scores, out, err)
     _check(lib().kq_gather_mix(_ptr(y), rows, n, _ptr(inv_order), _ptr(scores), t, top_k, _ptr(out), _ptr(err),
                                _stream(stream)), "kq_gather_mix")
+    return out
+
+
+def moe_glu_gather(x: torch.Tensor, gate_bank: torch.Tensor, up_bank: torch.Tensor, qtype: int, ids: torch.Tensor,
+                   act: int = ACT_SILU, limit: float = 0.0, out: torch.Tensor | None = None,
+                   err: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out[t * top_k + s] = act(x[t] @ dequant(gate[e]).T, x[t] @ dequant(up[e]).T), e = ids[t, s]."""
+    x = _bf16_bits(x)
+    t, top_k = ids.shape
+    k = x.shape[-1]
+    e, n = gate_bank.shape[0], gate_bank.shape[1]
+    if out is None:
+        out = torch.empty(t * top_k, n, dtype=torch.float32, device=x.device)
+    _need_cuda(x, gate_bank, up_bank, ids, out, err)
+    _check(lib().kq_moe_glu_gather(qtype, _ptr(gate_bank), _ptr(up_bank), e, n, k, _ptr(x), _ptr(ids), t, top_k,
+                                   act, limit, _ptr(out), _ptr(err), _stream(stream)), "kq_moe_glu_gather")
     return out

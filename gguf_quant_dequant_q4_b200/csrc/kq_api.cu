@@ -224,7 +224,28 @@ int kq_gather_qmv(int type, const void* w_bank, int32_t n_experts, int64_t n, in
     const int pairs = static_cast<int>(n_tokens * top_k);
     // distinct experts per token bound the pairs of one expert by n_tokens
     const int m_cap = n_tokens < 16 ? static_cast<int>(n_tokens) : 16;
-    return launch_gather_qmv(type, w_bank, n_experts, n, k, x, x_per_token ? top_k : 1, ids, pairs, m_cap, y,
+    return launch_gather_qmv(type, w_bank, nullptr, 0, 0.f, n_experts, n, k, x, x_per_token ? top_k : 1, ids, pairs,
+                             m_cap, y, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+int kq_moe_glu_gather(int type, const void* gate_bank, const void* up_bank, int32_t n_experts, int64_t n, int64_t k,
+                      const uint16_t* x, const int32_t* ids, int64_t n_tokens, int32_t top_k, int32_t act,
+                      float limit, float* out, int32_t* err_flag, void* stream) {
+    if (n_experts < 1 || n_experts > 256 || n_tokens < 0 || top_k < 1) return KQ_ERR_INVALID_ARG;
+    if (act < KQ_ACT_SILU || act > KQ_ACT_SILU_LIMIT) return KQ_ERR_INVALID_ARG;
+    if (act == KQ_ACT_SILU_LIMIT && !(limit > 0.f)) return KQ_ERR_INVALID_ARG;
+    int rc = check_weights(type, gate_bank, n, k);
+    if (rc) return rc;
+    rc = check_weights(type, up_bank, n, k);
+    if (rc) return rc;
+    if (n_tokens * top_k > 8192) return KQ_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(n_experts) * n > (int64_t(1) << 31) - 1) return KQ_ERR_INVALID_ARG;
+    if (n == 0 || n_tokens == 0) return KQ_OK;
+    if (!x || !ids || !out) return KQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(out)) return KQ_ERR_ALIGNMENT;
+    const int pairs = static_cast<int>(n_tokens * top_k);
+    const int m_cap = n_tokens < 16 ? static_cast<int>(n_tokens) : 16;
+    return launch_gather_qmv(type, gate_bank, up_bank, act, limit, n_experts, n, k, x, top_k, ids, pairs, m_cap, out,
                              err_flag, static_cast<cudaStream_t>(stream));
 }
 

@@ -32,10 +32,11 @@ int launch_qmv(int type, const void* w, int64_t n, int64_t k, const uint16_t* x,
 int launch_qmv_stream(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int m, float* y,
                       cudaStream_t s);
 // Decode MoE product (one output row per (token, slot) pair) on the staged
-// kernel; KQ_ERR_UNSUPPORTED for shapes it does not cover.
-int launch_gather_qmv(int type, const void* w_bank, int n_experts, int64_t n, int64_t k, const uint16_t* x,
-                      int xdiv, const int32_t* ids, int pairs, int m_cap, float* y, int32_t* err_flag,
-                      cudaStream_t s);
+// kernel; with w_bank2 (the up bank) the GLU act(x W^T) * (x W2^T) of each
+// pair.  KQ_ERR_UNSUPPORTED for shapes it does not cover.
+int launch_gather_qmv(int type, const void* w_bank, const void* w_bank2, int act, float limit, int n_experts,
+                      int64_t n, int64_t k, const uint16_t* x, int xdiv, const int32_t* ids, int pairs, int m_cap,
+                      float* y, int32_t* err_flag, cudaStream_t s);
 int launch_qmm(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int64_t m, float* y,
                cudaStream_t s);
 int launch_gather_qmm(int type, const void* w_bank, int n_experts, int64_t n, int64_t k,

@@ -88,6 +88,16 @@ struct SPG : SP {
     int32_t* err;         // caller's device flag word (nullable)
     int pairs, xdiv, n_experts, vbase, vcount;
 };
+// GLU mode (decode MoE gate/up pair, one activation row per token): the
+// gate bank is w, the up bank w2; logical row group 2g + h of a CTA is its
+// row group g of the gate (h = 0) or up (h = 1) matrix.  The gate sums wait
+// in a small buffer for the up sums of the same rows, and act(gate) * up is
+// stored.
+struct SPGLU : SPG {
+    const uint8_t* w2;
+    int act;       // 0: silu, 1: gelu (tanh form), 2: silu with limit
+    float limit;
+};
 constexpr uint32_t kGList = 512;     // gather: pair list of the CTA (16 ints)
 constexpr uint32_t kGMisc = 576;     // gather: expert, pairs present, row range
 constexpr uint32_t kGCount = 1024;   // gather: pairs per expert (256 ints)
@@ -731,9 +741,24 @@ __device__ bool gather_setup(const SPG& p, uint8_t* smem, int64_t& r0, int64_t& 
     return true;
 }
 
+// act(g) * u of the GLU epilogue, in fp32: silu(g) = g / (1 + e^-g); gelu in
+// its tanh form 0.5 g (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3))); silu with
+// limit: silu(min(g, L)) * clamp(u, -L, L).
+__device__ __forceinline__ float glu_act(int act, float limit, float g, float u) {
+    if (act == 2) {
+        g = fminf(g, limit);
+        u = fminf(fmaxf(u, -limit), limit);
+    }
+    float a;
+    if (act == 1) a = 0.5f * g * (1.0f + tanhf(0.7978845608028654f * (g + 0.044715f * g * g * g)));
+    else a = g / (1.0f + expf(-g));
+    return a * u;
+}
+
 template <class C, bool SPLIT, class P = SP>
 __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
     constexpr bool GATHER = !std::is_same<P, SP>::value;
+    constexpr bool GLU = std::is_same<P, SPGLU>::value;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);   // [kMaxStages]
     uint64_t* empty = full + kMaxStages;                   // [kMaxStages]
@@ -777,14 +802,17 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
     // gather: the expert's weights, the pairs present (x rows gathered and y
     // rows scattered through the pair list) and the row range
     const uint8_t* wbase = p.w;
+    const uint8_t* wbase2 = nullptr;
     int gm = p.m;
     const int* glist = reinterpret_cast<const int*>(smem + kGList);
     if constexpr (GATHER) {
         int ge = 0;
         if (!gather_setup(p, smem, r0, r1, ge, gm)) return;
         wbase = p.w + static_cast<int64_t>(ge) * p.n * p.row_bytes;
+        if constexpr (GLU) wbase2 = p.w2 + static_cast<int64_t>(ge) * p.n * p.row_bytes;
     }
     const int nrg = cdiv(r1 - r0, kRows);
+    const int nlg = GLU ? 2 * nrg : nrg;   // logical row groups (GLU: gate and up)
 
     if (warp == kProd) {
         // ---------------------------------------------------------- producer
@@ -804,9 +832,11 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
         }
         int q = 0;
         bool ok = true;
-        for (int rg = 0; rg < nrg && ok; ++rg) {
-            const int64_t row0 = r0 + static_cast<int64_t>(group_order(rg, nrg, r1 - r0)) * kRows;
+        for (int rg = 0; rg < nlg && ok; ++rg) {
+            const int gi = GLU ? rg >> 1 : rg;
+            const int64_t row0 = r0 + static_cast<int64_t>(group_order(gi, nrg, r1 - r0)) * kRows;
             const int rv = static_cast<int>(r1 - row0 < kRows ? r1 - row0 : kRows);
+            const uint8_t* wsrc = (GLU && (rg & 1)) ? wbase2 : wbase;
             for (int st = 0; st < p.spr; ++st, ++q) {
                 const int slot = q % p.ns;
                 if (lane == 0 && q >= p.ns) ok = sleep_wait(&empty[slot], ((q / p.ns) & 1) ^ 1, p.status);
@@ -822,7 +852,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
                 __syncwarp();
                 if (lane < rv)
                     bulk_g2s(smem + p.off_stage + slot * stage_bytes + lane * p.rs,
-                             wbase + (row0 + lane) * p.row_bytes + (kb0 + b0) * C::kBPB, bytes,
+                             wsrc + (row0 + lane) * p.row_bytes + (kb0 + b0) * C::kBPB, bytes,
                              &full[slot]);
             }
         }
@@ -848,8 +878,9 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
         float* part = reinterpret_cast<float*>(smem + p.off_part);
         const int items_per_row = p.nblk / C::kItemBlocks;
         int q = 0;
-        for (int rg = 0; rg < nrg && !*abort_flag; ++rg) {
-            const int64_t row0 = r0 + static_cast<int64_t>(group_order(rg, nrg, r1 - r0)) * kRows;
+        for (int rg = 0; rg < nlg && !*abort_flag; ++rg) {
+            const int gi = GLU ? rg >> 1 : rg;
+            const int64_t row0 = r0 + static_cast<int64_t>(group_order(gi, nrg, r1 - r0)) * kRows;
             const int rv = static_cast<int>(r1 - row0 < kRows ? r1 - row0 : kRows);
             float acc[C::kAccPerLane];
 #pragma unroll
@@ -934,7 +965,13 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
                         const int tok = o / kRows, r = o % kRows;
                         float sum = 0.f;
                         for (int w = 0; w < kCW; ++w) sum += part[((pslot * kCW + w) * kRows + r) * p.m + tok];
-                        if constexpr (GATHER) {
+                        if constexpr (GLU) {
+                            // gate sums wait behind the two partial slots for the up sums
+                            float* gbuf = part + 2 * kCW * kRows * p.m;
+                            if ((rg & 1) == 0) gbuf[o] = sum;
+                            else if (r < rv && tok < gm)
+                                p.y[static_cast<int64_t>(glist[tok]) * p.n + row0 + r] = glu_act(p.act, p.limit, gbuf[o], sum);
+                        } else if constexpr (GATHER) {
                             if (r < rv && tok < gm) p.y[static_cast<int64_t>(glist[tok]) * p.n + row0 + r] = sum;
                         } else {
                             if (r < rv) p.y[static_cast<int64_t>(tok) * p.n + row0 + r] = sum;
@@ -1025,6 +1062,9 @@ struct GatherArgs {
     const int32_t* ids;
     int32_t* err;
     int pairs, xdiv, n_experts;
+    const void* w2;   // GLU mode: the up bank (w is the gate bank)
+    int act;
+    float limit;
 };
 
 // ks: CTAs of a cluster that split K (1, 2, 4, 8; a divisor of the block
@@ -1064,7 +1104,8 @@ int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m,
         p.off_part = align16(p.off_zero + C::kZero);
         p.off_xraw = p.off_part;   // the raw x copy is dead before any partial sum is written
         // split: two row-group slots of partial sums, reused in turn
-        const uint32_t part = static_cast<uint32_t>(ks > 1 || ga ? 2 : nrg_max) * kCW * kRows * m * 4;
+        uint32_t part = static_cast<uint32_t>(ks > 1 || ga ? 2 : nrg_max) * kCW * kRows * m * 4;
+        if (ga && ga->w2) part += kRows * m * 4;   // GLU: the gate sums of a row group
         // receive slots of the row groups this CTA owns: ceil(nrg / ks) x ks slices
         const uint32_t red = ks > 1 ? static_cast<uint32_t>(cdiv(nrg_max, ks) * ks) * kRows * m * 4 : 0;
         uint32_t xraw = static_cast<uint32_t>(m) * static_cast<uint32_t>(p.k) * 2;
@@ -1141,10 +1182,7 @@ int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m,
     cfg.attrs = attr;
     cfg.numAttrs = na;
     if (ga) {
-        auto kernel = qmv_stream_kernel<C, false, SPG>;
-        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
-        if (e != cudaSuccess) return record_cuda(e);
-        SPG g{};
+        SPGLU g{};
         static_cast<SP&>(g) = p;
         g.ids = ga->ids;
         g.err = ga->err;
@@ -1152,9 +1190,18 @@ int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m,
         g.xdiv = ga->xdiv;
         g.n_experts = ga->n_experts;
         g.vcount = vcount;
+        g.w2 = static_cast<const uint8_t*>(ga->w2);
+        g.act = ga->act;
+        g.limit = ga->limit;
+        auto kg = qmv_stream_kernel<C, false, SPG>;
+        auto kglu = qmv_stream_kernel<C, false, SPGLU>;
+        cudaError_t e = ga->w2 ? cudaFuncSetAttribute(kglu, cudaFuncAttributeMaxDynamicSharedMemorySize, total)
+                               : cudaFuncSetAttribute(kg, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
+        if (e != cudaSuccess) return record_cuda(e);
         for (int j = 0; j < launches; ++j) {
             g.vbase = j * vcount;
-            const int rc = record_cuda(cudaLaunchKernelEx(&cfg, kernel, g));
+            const int rc = ga->w2 ? record_cuda(cudaLaunchKernelEx(&cfg, kglu, g))
+                                  : record_cuda(cudaLaunchKernelEx(&cfg, kg, static_cast<const SPG&>(g)));
             if (rc) return rc;
         }
         return KQ_OK;
@@ -1219,10 +1266,10 @@ int launch_qmv_stream(int type, const void* w, int64_t n, int64_t k, const uint1
 // Decode MoE product on the staged kernel: at most m_cap pairs of one expert
 // per virtual expert (q8_0 and q6_K take up to 2 activation rows, q4_K up to
 // 16 while the activation image fits; fewer when shared memory requires).
-int launch_gather_qmv(int type, const void* w_bank, int n_experts, int64_t n, int64_t k, const uint16_t* x,
-                      int xdiv, const int32_t* ids, int pairs, int m_cap, float* y, int32_t* err_flag,
-                      cudaStream_t s) {
-    GatherArgs ga{ids, err_flag, pairs, xdiv, n_experts};
+int launch_gather_qmv(int type, const void* w_bank, const void* w_bank2, int act, float limit, int n_experts,
+                      int64_t n, int64_t k, const uint16_t* x, int xdiv, const int32_t* ids, int pairs, int m_cap,
+                      float* y, int32_t* err_flag, cudaStream_t s) {
+    GatherArgs ga{ids, err_flag, pairs, xdiv, n_experts, w_bank2, act, limit};
     const int nblk = static_cast<int>(k / (type == KQ_Q8_0 ? 32 : 256));
     int rc = KQ_ERR_UNSUPPORTED;
     switch (type) {

@@ -207,6 +207,34 @@ int kq_gather_qmv(int type, const void* w_bank, int32_t n_experts, int64_t n, in
                   const uint16_t* x, int32_t x_per_token, const int32_t* ids, int64_t n_tokens,
                   int32_t top_k, float* y, int32_t* err_flag, void* stream);
 
+/* GLU activations of kq_moe_glu_gather. */
+#define KQ_ACT_SILU        0   /* silu(g) * u, silu(g) = g / (1 + exp(-g))          */
+#define KQ_ACT_GELU_TANH   1   /* gelu(g) * u, gelu in its tanh approximation:
+                                  0.5 g (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3)))   */
+#define KQ_ACT_SILU_LIMIT  2   /* silu(min(g, limit)) * clamp(u, -limit, limit)     */
+
+/*
+ * kq_moe_glu_gather - decode MoE gate/up products and their GLU in one
+ * dispatch: out[p, :] = act(x[t, :] . dequant(Wg[e])^T, x[t, :] . dequant(Wu[e])^T)
+ * for the pairs p = t*top_k + s of ids [n_tokens, top_k], e = ids[p].
+ * mlx-kquant bindings.cpp, `moe_glu_gather_kq` ("gate and up expert matvecs
+ * share each activation load and the GLU epilogue act(g) * u is applied in
+ * the same dispatch"; act 'silu' (default), 'gelu' (tanh approx),
+ * 'silu_limit' (requires limit > 0); x [T, K], gate_w and up_w
+ * (n_experts, N, bytes_per_row), indices [T, R], output [T, R, N]).
+ * Each routed expert's gate and up rows are streamed once; every CTA takes
+ * 16 gate rows, then the same 16 up rows, and applies act in fp32 to the
+ * two fp32 sums (arithmetic of the sums as kq_qmv).
+ *   gate_bank, up_bank [n_experts, n, row_bytes], x [n_tokens, k] bf16,
+ *   ids [n_tokens*top_k] int32, out [n_tokens*top_k, n] fp32.
+ *   act one of KQ_ACT_*; KQ_ACT_SILU_LIMIT needs limit > 0.
+ * Limits and errors as kq_gather_qmv.
+ */
+int kq_moe_glu_gather(int type, const void* gate_bank, const void* up_bank, int32_t n_experts,
+                      int64_t n, int64_t k, const uint16_t* x, const int32_t* ids, int64_t n_tokens,
+                      int32_t top_k, int32_t act, float limit, float* out, int32_t* err_flag,
+                      void* stream);
+
 /*
  * kq_gather_mix - unsort and score mix of expert-sorted MoE outputs:
  * out[t, :] = sum over s = 0 .. top_k-1 of scores[t, s] * y[inv_order[t*top_k + s], :].

@@ -31,6 +31,9 @@ and states the MoE semantics in plain numpy:
                    [T, R, N]; with one activation row per token the same
                    product feeds the gate/up projections of
                    ``moe_glu_gather_kq``).
+* ``moe_glu_gather`` act(x W_g^T) * (x W_u^T) per pair from the fp64 gate
+                   and up products, act silu, gelu (tanh form) or silu with
+                   a limit (bindings.cpp, ``moe_glu_gather_kq``).
 * ``inverse_order`` / ``gather_mix``  unsort and score mix of expert-sorted
                    rows: out[t] = sum_s scores[t, s] * y[inv_order[t k + s]]
                    (bindings.cpp, ``gather_mix``: f32 accumulation; hanzo-ml
@@ -250,3 +253,33 @@ def gather_mix(y: np.ndarray, inv_order: np.ndarray, scores: np.ndarray) -> np.n
         prod = (sc[:, s:s + 1] * y[inv[:, s]]).astype(np.float32)
         out = (out + prod).astype(np.float32)
     return out
+
+
+ACT_SILU, ACT_GELU_TANH, ACT_SILU_LIMIT = 0, 1, 2
+
+
+def glu(act: int, g: np.ndarray, u: np.ndarray, limit: float = 0.0) -> np.ndarray:
+    """act(g) * u in fp64: silu(g) = g / (1 + exp(-g)); gelu in the tanh form
+    0.5 g (1 + tanh(sqrt(2 / pi) (g + 0.044715 g^3))); silu with limit L:
+    silu(min(g, L)) * clip(u, -L, L)."""
+    g = np.asarray(g, dtype=np.float64)
+    u = np.asarray(u, dtype=np.float64)
+    if act == ACT_SILU_LIMIT:
+        g = np.minimum(g, limit)
+        u = np.clip(u, -limit, limit)
+    if act == ACT_GELU_TANH:
+        a = 0.5 * g * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (g + 0.044715 * g ** 3)))
+    else:
+        with np.errstate(over="ignore"):   # exp(-g) = inf for g << 0 gives silu = -0
+            a = g / (1.0 + np.exp(-g))
+    return a * u
+
+
+def moe_glu_gather(qtype: int, gate_bank: np.ndarray, up_bank: np.ndarray, k: int, x_bf16: np.ndarray,
+                   ids: np.ndarray, act: int = ACT_SILU, limit: float = 0.0):
+    """(out, g, u, ag, au): out[p] = act(g[p], u[p]) with the fp64 per-pair
+    products g = x[t] @ dequant(gate[e]).T and u = x[t] @ dequant(up[e]).T
+    (one activation row per token), and their sums of |x w| (ag, au)."""
+    g, ag = gather_qmv(qtype, gate_bank, k, x_bf16, ids, x_per_token=True, absdot=True)
+    u, au = gather_qmv(qtype, up_bank, k, x_bf16, ids, x_per_token=True, absdot=True)
+    return glu(act, g, u, limit), g, u, ag, au

@@ -30,7 +30,7 @@ def declared_symbols():
 def test_header_declares_the_path():
     syms = declared_symbols()
     for s in ("kq_dequantize", "kq_qmv", "kq_qmm", "kq_moe_sort", "kq_expert_tile_map", "kq_gather_qmm",
-              "kq_gather_qmv", "kq_gather_mix"):
+              "kq_gather_qmv", "kq_gather_mix", "kq_moe_glu_gather"):
         assert s in syms
 
 
@@ -117,6 +117,12 @@ def test_decode_moe_argument_checks(lib):
     assert g(kq.Q4_K, A, 8, 64, 256, MIS, 0, A, 1, 2, A, None, None) == ALIGN
     assert g(kq.Q4_K, A, 8, 64, 256, A, 0, A, 1, 2, MIS, None, None) == ALIGN
     assert g(kq.Q4_K, A, 8, 64, 256, A, 0, A, 0, 2, A, None, None) == OK         # no tokens
+    f = lib.kq_moe_glu_gather
+    assert f(kq.Q4_K, A, A, 8, 64, 256, A, A, 1, 2, 3, 0.0, A, None, None) == INVALID    # unknown act
+    assert f(kq.Q4_K, A, A, 8, 64, 256, A, A, 1, 2, 2, 0.0, A, None, None) == INVALID    # limit must be > 0
+    assert f(kq.Q4_K, A, None, 8, 64, 256, A, A, 1, 2, 0, 0.0, A, None, None) == INVALID  # null up bank
+    assert f(kq.Q4_K, A, MIS, 8, 64, 256, A, A, 1, 2, 0, 0.0, A, None, None) == ALIGN
+    assert f(kq.Q4_K, A, A, 8, 64, 256, A, A, 0, 2, 2, 1.0, A, None, None) == OK
     m = lib.kq_gather_mix
     assert m(A, 8, 6, A, A, 4, 2, A, None, None) == INVALID                      # n % 4
     assert m(A, 8, 8, A, A, 4, 0, A, None, None) == INVALID                      # top_k < 1

@@ -159,3 +159,48 @@ def test_prefill_moe_end_to_end_mix():
     out = kq.gather_mix(y, inv, torch.from_numpy(sc).cuda()).cpu().numpy()
     ref = oracle.gather_mix(y.cpu().numpy(), inv.cpu().numpy(), sc)
     assert np.array_equal(out.view(np.uint32), ref.view(np.uint32))
+
+
+def check_glu(y, out, g, u, ag, au, act):
+    """|y - out| within the propagated qmv bound: the gate and up sums each
+    carry at most 1e-3 * sum|x w|, and act is 1.2-Lipschitz in g (silu, gelu
+    and their limited forms) and linear in u; plus fp32 rounding of act."""
+    dg, du = 1e-3 * ag, 1e-3 * au
+    a = np.abs(oracle.glu(act, g, np.ones_like(g), limit=4.0))
+    tol = 1.2 * dg * (np.abs(u) + du) + (a + 1.2 * dg) * du + 1e-5 * np.abs(out) + 1e-30
+    err = np.abs(y.astype(np.float64) - out)
+    assert np.all(np.isfinite(y))
+    worst = float(np.max(err / tol))
+    assert worst <= 1.0, f"error / bound = {worst:.3f}"
+
+
+@pytest.mark.parametrize("qtype", [kq.Q4_K, kq.Q6_K, kq.Q8_0])
+@pytest.mark.parametrize("act", [kq.ACT_SILU, kq.ACT_GELU_TANH, kq.ACT_SILU_LIMIT])
+def test_moe_glu_gather_vs_oracle(qtype, act):
+    tokens, top_k, experts, n, k = 3, 2, 5, 333, 2048
+    wg = synth.weights(qtype, n, k, seed=101, experts=experts)
+    wu = synth.weights(qtype, n, k, seed=102, experts=experts)
+    ids = synth.routing(tokens, experts, top_k, seed=103)
+    x = synth.activations(tokens, k, seed=104)
+    # scale x so that the products reach the region where the activations bend
+    x = synth.f32_to_bf16_bits(oracle.bf16_to_f32(x) * 40.0)
+    out = torch.full((tokens * top_k, n), float("nan"), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kq.moe_glu_gather(dev_bf16(x), dev_u8(wg), dev_u8(wu), qtype, torch.from_numpy(ids).cuda(), act=act, limit=4.0,
+                      out=out, err=err)
+    assert int(err.item()) == 0
+    ref, g, u, ag, au = oracle.moe_glu_gather(qtype, wg, wu, k, x, ids, act=act, limit=4.0)
+    assert np.mean(np.abs(g) > 1.0) > 0.2          # the activations are exercised off their linear part
+    check_glu(out.cpu().numpy(), ref, g, u, ag, au, act)
+
+
+def test_moe_glu_gather_full_bank_sampled():
+    experts, n, k, tokens, top_k = 8, 14336, 4096, 4, 2
+    wg = synth.weights(kq.Q4_K, n, k, experts=experts, seed=0)
+    wu = synth.weights(kq.Q4_K, n, k, experts=experts, seed=1)
+    ids = synth.routing(tokens, experts, top_k, seed=5)
+    x = synth.activations(tokens, k, seed=6)
+    y = kq.moe_glu_gather(dev_bf16(x), dev_u8(wg), dev_u8(wu), kq.Q4_K, torch.from_numpy(ids).cuda()).cpu().numpy()
+    cols = np.sort(np.random.default_rng(8).choice(n, 16, replace=False))
+    ref, g, u, ag, au = oracle.moe_glu_gather(kq.Q4_K, wg[:, cols], wu[:, cols], k, x, ids)
+    check_glu(y[:, cols], ref, g, u, ag, au, kq.ACT_SILU)

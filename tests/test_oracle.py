@@ -401,3 +401,47 @@ def test_gather_mix_exact_values_and_order():
     y = np.array([[a], [-(1 + 2.0 ** -11)]], np.float32)
     out = oracle.gather_mix(y, np.array([0, 1], np.int32), np.array([[a, 1.0]], np.float32))
     assert out[0, 0] == 0.0
+
+
+def test_glu_activations():
+    import math
+    from scipy.special import expit
+    g = np.linspace(-12, 12, 2401)
+    u = np.random.default_rng(9).standard_normal(g.size)
+    one = np.ones_like(g)
+    # odd-part identities of both activations: a(g) - a(-g) = g
+    for act in (oracle.ACT_SILU, oracle.ACT_GELU_TANH):
+        assert np.allclose(oracle.glu(act, g, one) - oracle.glu(act, -g, one), g, rtol=0, atol=1e-12)
+    # silu against the library logistic function
+    assert np.allclose(oracle.glu(oracle.ACT_SILU, g, u), g * expit(g) * u, rtol=1e-14, atol=1e-300)
+    # the tanh form stays within 1e-3 of the exact gelu g * Phi(g) (Phi from erf)
+    exact = np.array([0.5 * v * (1 + math.erf(v / math.sqrt(2))) for v in g])
+    assert np.max(np.abs(oracle.glu(oracle.ACT_GELU_TANH, g, one) - exact)) < 1e-3
+    # silu with a limit: the gate is capped from above, the up value clipped both ways
+    lim = 3.0
+    out = oracle.glu(oracle.ACT_SILU_LIMIT, g, 10 * u, limit=lim)
+    assert np.allclose(out, oracle.glu(oracle.ACT_SILU, np.minimum(g, lim), np.clip(10 * u, -lim, lim)))
+    assert np.all(np.abs(out) <= lim * lim * expit(lim) + 1e-12)
+
+
+def test_moe_glu_gather_one_hot():
+    # q8_0 hand blocks (d = 1): a one-hot token row returns one column of each
+    # routed expert's gate and up matrix, so g and u are the int8 codes there
+    n, k, e = 3, 32, 2
+    gc = (np.arange(e * n * k).reshape(e, n, k) % 17 - 8).astype(np.int8)
+    uc = (np.arange(e * n * k).reshape(e, n, k) % 13 - 6).astype(np.int8)
+    def bank(c):
+        w = np.zeros((e, n, 34), np.uint8)
+        w[:, :, 0:2] = np.array([1.0], np.float16).view(np.uint8)
+        w[:, :, 2:] = c.view(np.uint8)
+        return w
+    x = np.zeros((2, k), np.float32)
+    x[0, 4] = 1.0
+    x[1, 30] = 1.0
+    ids = np.array([[1, 0], [0, 1]], np.int32)
+    out, g, u, _, _ = oracle.moe_glu_gather(Q8_0, bank(gc), bank(uc), k, synth.f32_to_bf16_bits(x), ids)
+    for p in range(4):
+        t, ex, c = p // 2, ids.reshape(-1)[p], (4, 30)[p // 2]
+        assert np.array_equal(g[p], gc[ex, :, c].astype(np.float64))
+        assert np.array_equal(u[p], uc[ex, :, c].astype(np.float64))
+        assert np.array_equal(out[p], oracle.glu(oracle.ACT_SILU, g[p], u[p]))
