@@ -34,6 +34,10 @@ and states the MoE semantics in plain numpy:
 * ``moe_glu_gather`` act(x W_g^T) * (x W_u^T) per pair from the fp64 gate
                    and up products, act silu, gelu (tanh form) or silu with
                    a limit (bindings.cpp, ``moe_glu_gather_kq``).
+* ``quantize``     float -> wire bytes (bindings.cpp, ``quantize``: encode a
+                   float weight tensor into GGUF K-quant wire bytes): q8_0 by
+                   ggml's absmax rule, q4_K / q6_K by min/max and absmax
+                   scales in fixed fp32 steps (see kq_oracle.c).
 * ``inverse_order`` / ``gather_mix``  unsort and score mix of expert-sorted
                    rows: out[t] = sum_s scores[t, s] * y[inv_order[t k + s]]
                    (bindings.cpp, ``gather_mix``: f32 accumulation; hanzo-ml
@@ -80,6 +84,8 @@ def _load():
         lib.oracle_matmul_f64.argtypes = [ctypes.c_int, ip, i64, i64, ip, i64, ip, ip]
         lib.oracle_matmul_f32.argtypes = [ctypes.c_int, ip, i64, i64, ip, i64, ip]
         lib.oracle_threads.restype = ctypes.c_int
+        lib.oracle_quantize.argtypes = [ctypes.c_int, ip, i64, i64, ip]
+        lib.oracle_float_to_half.argtypes = [ip, i64, ip]
         _lib = lib
     return _lib
 
@@ -283,3 +289,25 @@ def moe_glu_gather(qtype: int, gate_bank: np.ndarray, up_bank: np.ndarray, k: in
     g, ag = gather_qmv(qtype, gate_bank, k, x_bf16, ids, x_per_token=True, absdot=True)
     u, au = gather_qmv(qtype, up_bank, k, x_bf16, ids, x_per_token=True, absdot=True)
     return glu(act, g, u, limit), g, u, ag, au
+
+
+def float_to_half_bits(x: np.ndarray) -> np.ndarray:
+    """binary32 -> binary16 bits, round to nearest even (the encoder's rounding)."""
+    x = np.ascontiguousarray(x, dtype=np.float32).reshape(-1)
+    out = np.empty(x.size, dtype=np.uint16)
+    _load().oracle_float_to_half(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def quantize(qtype: int, w: np.ndarray) -> np.ndarray:
+    """fp32 [..., K] -> wire bytes [..., row_bytes] (fixed fp32 steps)."""
+    vpb, bpb = block_info(qtype)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    k = w.shape[-1]
+    if k % vpb:
+        raise ValueError("K must be a multiple of the block size")
+    rows = int(np.prod(w.shape[:-1]))
+    out = np.empty(w.shape[:-1] + (k // vpb * bpb,), dtype=np.uint8)
+    if _load().oracle_quantize(qtype, _ptr(w), rows, k, _ptr(out)):
+        raise RuntimeError("oracle_quantize failed")
+    return out

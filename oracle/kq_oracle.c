@@ -22,6 +22,16 @@
  *    docstring, transpose=True, mlx-kquant bindings.cpp; README "Using
  *    K-quant ops directly").  The reference value accumulates in fp64; an
  *    fp32 sequential-k variant is provided for timing only.
+ *  - quantize: float -> wire bytes ("quantize" op docstring, mlx-kquant
+ *    bindings.cpp: encode a float weight tensor into GGUF K-quant wire bytes;
+ *    hanzo-ml quantized/mod.rs QTensor::quantize).  The pages give no
+ *    encoding search.  q8_0 follows ggml's published rule (absmax / 127,
+ *    round half away from zero), pinned against gguf.quants.quantize.  q4_K
+ *    and q6_K take the plainest reading: per sub-block min/max (q4_K) or
+ *    absmax (q6_K) scales, 6-bit / int8 scale codes against an fp16 super-
+ *    block scale, then the codes; every step below is one fp32 operation
+ *    in a fixed order.  Those two are pinned by round-trip error bounds, not
+ *    against ggml's own (search-based) encoder.
  *
  * Parity pins for every function live in tests/test_oracle.py.
  */
@@ -254,4 +264,162 @@ int oracle_threads(void) {
         }
     }
     return t;
+}
+
+
+/* ------------------------------------------------------------------ encoder */
+
+/* binary32 -> binary16, round to nearest, ties to even (IEEE-754 default).
+ * Written from the binary16 definition: normal numbers 2^(e-15) (1 + f/1024)
+ * for 1 <= e <= 30, subnormals 2^-14 (f / 1024); the 11-bit significand of
+ * |v| is rounded with rintf (default rounding mode: nearest, ties to even);
+ * a carry into bit 11 moves to the next binade; from 65520 on (the midpoint
+ * between 65504 and 2^16) the result is infinity. */
+static uint16_t float_to_half(float v) {
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    float a = fabsf(v);
+    if (isnan(v)) return (uint16_t)(sign | 0x7e00u);
+    if (a >= 65520.0f) return (uint16_t)(sign | 0x7c00u);
+    if (a < ldexpf(1.0f, -14)) {                       /* subnormal range (and zero) */
+        float m = rintf(ldexpf(a, 24));                /* units of 2^-24, exact scaling */
+        return (uint16_t)(sign | (uint16_t)m);         /* m == 1024 is the smallest normal */
+    }
+    int e;
+    frexpf(a, &e);                                     /* a = f * 2^e, f in [0.5, 1) */
+    e -= 1;                                            /* a in [2^e, 2^(e+1)) */
+    float m = rintf(ldexpf(a, 10 - e));                /* significand in [1024, 2048] */
+    if (m >= 2048.0f) {
+        m = 1024.0f;
+        e += 1;
+    }
+    return (uint16_t)(sign | (uint16_t)((e + 15) << 10) | (uint16_t)(m - 1024.0f));
+}
+
+int oracle_float_to_half(const float* in, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = float_to_half(in[i]);
+    return 0;
+}
+
+static int clampi(float v, int lo, int hi) {
+    int q = (int)v;
+    return q < lo ? lo : (q > hi ? hi : q);
+}
+
+static void wr16(uint8_t* p, uint16_t h) {
+    p[0] = (uint8_t)(h & 0xff);
+    p[1] = (uint8_t)(h >> 8);
+}
+
+/* q8_0: d = max|x| / 127, codes round(x * (1/d)) (half away from zero),
+ * d stored as binary16. */
+static void qz_q8_0(const float* x, uint8_t* b) {
+    float amax = 0.0f;
+    for (int i = 0; i < 32; ++i) {
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    float d = amax / 127.0f;
+    float id = d == 0.0f ? 0.0f : 1.0f / d;
+    wr16(b, float_to_half(d));
+    for (int i = 0; i < 32; ++i) {
+        float p = x[i] * id;
+        b[2 + i] = (uint8_t)(int8_t)clampi(roundf(p), -128, 127);
+    }
+}
+
+/* q4_K: sub-block j (values 32j..32j+31) spans [lo_j, hi_j] with
+ * lo_j = min(0, min x) and hi_j = max x; its scale is (hi_j - lo_j) / 15 and
+ * its min -lo_j.  The super-block scales d = max scale / 63 and
+ * dmin = max min / 63 are stored as binary16; the 6-bit codes are the
+ * rounded ratios to the stored values; each value's 4-bit code is
+ * round((x + dmin*m_j) / (d*sc_j)), using the decoder's own products. */
+static void qz_q4k(const float* x, uint8_t* b) {
+    float sc_f[8], mn_f[8], smax = 0.0f, mmax = 0.0f;
+    for (int j = 0; j < 8; ++j) {
+        float lo = 0.0f, hi = x[32 * j];
+        for (int i = 0; i < 32; ++i) {
+            float v = x[32 * j + i];
+            if (v < lo) lo = v;
+            if (v > hi) hi = v;
+        }
+        sc_f[j] = (hi - lo) / 15.0f;
+        mn_f[j] = -lo;
+        if (sc_f[j] > smax) smax = sc_f[j];
+        if (mn_f[j] > mmax) mmax = mn_f[j];
+    }
+    uint16_t hd = float_to_half(smax / 63.0f), hm = float_to_half(mmax / 63.0f);
+    float df = half_to_float(hd), dmf = half_to_float(hm);
+    int sc[8], m[8];
+    for (int j = 0; j < 8; ++j) {
+        sc[j] = df > 0.0f ? clampi(roundf(sc_f[j] / df), 0, 63) : 0;
+        m[j] = dmf > 0.0f ? clampi(roundf(mn_f[j] / dmf), 0, 63) : 0;
+    }
+    memset(b, 0, 144);
+    wr16(b, hd);
+    wr16(b + 2, hm);
+    uint8_t* s = b + 4;
+    for (int j = 0; j < 4; ++j) {
+        s[j] = (uint8_t)(sc[j] | ((sc[j + 4] >> 4) << 6));
+        s[j + 4] = (uint8_t)(m[j] | ((m[j + 4] >> 4) << 6));
+        s[j + 8] = (uint8_t)((sc[j + 4] & 0x0f) | ((m[j + 4] & 0x0f) << 4));
+    }
+    uint8_t* qs = b + 16;
+    for (int v = 0; v < 256; ++v) {
+        int j = v / 32;
+        float ds = df * (float)sc[j];
+        float dm = dmf * (float)m[j];
+        int q = ds > 0.0f ? clampi(roundf((x[v] + dm) / ds), 0, 15) : 0;
+        int c = v / 64, w = v % 64;
+        if (w < 32) qs[32 * c + w] |= (uint8_t)q;
+        else qs[32 * c + w - 32] |= (uint8_t)(q << 4);
+    }
+}
+
+/* q6_K: sub-block j (values 16j..16j+15) has scale max|x| / 31; the
+ * super-block scale d = max scale / 127 is stored as binary16, the int8
+ * scale codes are the rounded ratios to it, and each value's 6-bit code is
+ * round(x / (d*sc_j)) + 32, clamped to 0..63. */
+static void qz_q6k(const float* x, uint8_t* b) {
+    float s_f[16], smax = 0.0f;
+    for (int j = 0; j < 16; ++j) {
+        float a = 0.0f;
+        for (int i = 0; i < 16; ++i) {
+            float v = fabsf(x[16 * j + i]);
+            if (v > a) a = v;
+        }
+        s_f[j] = a / 31.0f;
+        if (s_f[j] > smax) smax = s_f[j];
+    }
+    uint16_t hd = float_to_half(smax / 127.0f);
+    float df = half_to_float(hd);
+    int sc[16];
+    for (int j = 0; j < 16; ++j) sc[j] = df > 0.0f ? clampi(roundf(s_f[j] / df), -128, 127) : 0;
+    memset(b, 0, 210);
+    uint8_t *ql = b, *qh = b + 128;
+    for (int v = 0; v < 256; ++v) {
+        int j = v / 16;
+        float ds = df * (float)sc[j];
+        int q = ds > 0.0f ? clampi(roundf(x[v] / ds), -32, 31) : 0;
+        int c = q + 32;
+        int h = v / 128, t = (v % 128) / 32, l = v % 32;
+        ql[64 * h + l + 32 * (t & 1)] |= (uint8_t)((c & 0x0f) << (4 * (t >> 1)));
+        qh[32 * h + l] |= (uint8_t)((c >> 4) << (2 * t));
+    }
+    for (int j = 0; j < 16; ++j) b[192 + j] = (uint8_t)(int8_t)sc[j];
+    wr16(b + 208, hd);
+}
+
+int oracle_quantize(int type, const float* x, int64_t n_rows, int64_t k, uint8_t* out) {
+    int vpb, bpb;
+    if (oracle_block_info(type, &vpb, &bpb) || k % vpb) return 1;
+    int64_t nb = n_rows * (k / vpb);
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < nb; ++i) {
+        const float* xb = x + i * vpb;
+        uint8_t* ob = out + i * bpb;
+        if (type == T_Q8_0) qz_q8_0(xb, ob);
+        else if (type == T_Q4_K) qz_q4k(xb, ob);
+        else qz_q6k(xb, ob);
+    }
+    return 0;
 }

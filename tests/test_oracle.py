@@ -445,3 +445,140 @@ def test_moe_glu_gather_one_hot():
         assert np.array_equal(g[p], gc[ex, :, c].astype(np.float64))
         assert np.array_equal(u[p], uc[ex, :, c].astype(np.float64))
         assert np.array_equal(out[p], oracle.glu(oracle.ACT_SILU, g[p], u[p]))
+
+
+# ----------------------------------------------------------------------------
+# encoder: float -> wire bytes
+# ----------------------------------------------------------------------------
+def test_float_to_half_matches_numpy():
+    g = np.random.default_rng(21)
+    bits32 = g.integers(0, 2**32, 200000, dtype=np.uint64).astype(np.uint32)
+    x = bits32.view(np.float32)
+    x = x[np.isfinite(x)]
+    # ties: binary16 midpoints in every binade, subnormal range, overflow edge
+    h = np.arange(0, 0x7c00, 7, dtype=np.uint16)
+    lo = h.view(np.float16).astype(np.float32)
+    hi = (h + 1).view(np.float16).astype(np.float32)
+    ties = ((lo.astype(np.float64) + hi.astype(np.float64)) / 2).astype(np.float32)
+    edge = np.array([65504, 65519.99, 65520, 65536, 1e-8, 2.0**-24, 2.0**-25, 3 * 2.0**-26, 0.0, -0.0],
+                    np.float32)
+    for v in (x, ties, -ties, edge, -edge):
+        with np.errstate(over="ignore"):
+            ref = v.astype(np.float16).view(np.uint16)
+        assert np.array_equal(oracle.float_to_half_bits(v), ref)
+
+
+def test_quantize_q8_0_matches_gguf():
+    import gguf
+    g = np.random.default_rng(22)
+    w = (g.standard_normal((40, 512)) * g.uniform(1e-3, 10, (40, 1))).astype(np.float32)
+    w[3, :32] = 0.0                                     # an all-zero block
+    w[4, :32] = np.arange(32) - 15.5                    # x * (1/d) lands on halves
+    w[5, 32:64] = 127.0 * np.sign(np.arange(32) - 16)   # codes at the extremes
+    ref = gguf.quants.quantize(w, gguf.GGMLQuantizationType.Q8_0)
+    assert np.array_equal(oracle.quantize(Q8_0, w), ref)
+
+
+def _canonical_q4k(g, nblk):
+    """q4_K blocks that the encoder must reproduce exactly: d = 2^-8,
+    dmin = 2^-9, 6-bit codes with 63 present, every sub-block using codes 0
+    and 15 (so its range is exactly 15 d sc_j and its min exactly -dmin m_j)."""
+    blocks = np.zeros((nblk, 144), np.uint8)
+    for b in range(nblk):
+        sc = g.integers(1, 64, 8)
+        m = g.integers(0, 64, 8)
+        sc[g.integers(8)] = 63
+        m[g.integers(8)] = 63
+        q = g.integers(0, 16, 256)
+        for j in range(8):
+            pos = g.choice(32, 2, replace=False)
+            q[32 * j + pos[0]], q[32 * j + pos[1]] = 0, 15
+        blk = blocks[b]
+        blk[0:2] = np.array([2.0 ** -8], np.float16).view(np.uint8)
+        blk[2:4] = np.array([2.0 ** -9], np.float16).view(np.uint8)
+        s = blk[4:16]
+        for j in range(4):                              # the layout the decoder reads
+            s[j] = sc[j] | ((sc[j + 4] >> 4) << 6)
+            s[j + 4] = m[j] | ((m[j + 4] >> 4) << 6)
+            s[j + 8] = (sc[j + 4] & 15) | ((m[j + 4] & 15) << 4)
+        for c in range(4):
+            for l in range(32):
+                blk[16 + 32 * c + l] = q[64 * c + l] | (q[64 * c + 32 + l] << 4)
+    return blocks
+
+
+def _canonical_q6k(g, nblk):
+    """q6_K blocks the encoder must reproduce exactly: d = 2^-10, int8 scales
+    in 1..127 with 127 present, codes q in -31..31 with +-31 in every
+    sub-block (so max|x| is exactly 31 d sc_j)."""
+    blocks = np.zeros((nblk, 210), np.uint8)
+    for b in range(nblk):
+        sc = g.integers(1, 128, 16)
+        sc[g.integers(16)] = 127
+        q = g.integers(-31, 32, 256)
+        for j in range(16):
+            q[16 * j + g.integers(16)] = 31 if g.integers(2) else -31
+        c = q + 32
+        blk = blocks[b]
+        for v in range(256):
+            h, t, l = v // 128, (v % 128) // 32, v % 32
+            blk[64 * h + l + 32 * (t & 1)] |= (c[v] & 15) << (4 * (t >> 1))
+            blk[128 + 32 * h + l] |= (c[v] >> 4) << (2 * t)
+        blk[192:208] = sc.astype(np.int8).view(np.uint8)
+        blk[208:210] = np.array([2.0 ** -10], np.float16).view(np.uint8)
+    return blocks
+
+
+@pytest.mark.parametrize("qtype", [Q4_K, Q6_K])
+def test_quantize_reproduces_canonical_blocks(qtype):
+    g = np.random.default_rng(23)
+    blocks = (_canonical_q4k if qtype == Q4_K else _canonical_q6k)(g, 24)
+    x = oracle.dequantize(qtype, blocks.reshape(1, -1), 24 * 256)
+    assert np.array_equal(oracle.quantize(qtype, x).reshape(24, -1), blocks)
+
+
+def test_quantize_zero_blocks():
+    z = np.zeros((1, 256), np.float32)
+    assert np.all(oracle.quantize(Q4_K, z) == 0)
+    assert np.all(oracle.quantize(Q8_0, z) == 0)
+    # q6_K: d = 0 and scales 0, every code q = 0 stored as 32 = 0b10_0000: low
+    # nibbles 0, each 2-bit high field 2, so every qh byte is 0b10101010
+    b = oracle.quantize(Q6_K, z)[0]
+    assert np.all(b[:128] == 0) and np.all(b[128:192] == 0xAA) and np.all(b[192:] == 0)
+
+
+@pytest.mark.parametrize("qtype", [Q4_K, Q6_K, Q8_0])
+def test_quantize_round_trip_bound(qtype):
+    # per-value error of decode(encode(x)) within the bound that follows from
+    # the sub-block range and the binary16 super-block scales, computed from x
+    # alone; and at most a few per cent of values beyond half a quantization
+    # step (only values clipped at the top of a sub-block's range)
+    g = np.random.default_rng(24)
+    x = (g.standard_normal((16, 1024)) * g.uniform(1e-2, 3, (16, 1))).astype(np.float32)
+    y = oracle.dequantize(qtype, oracle.quantize(qtype, x), 1024).astype(np.float64)
+    err = np.abs(y - x)
+    xs = x.astype(np.float64)
+    eps = 1e-6 * np.abs(xs).max()
+    if qtype == Q8_0:
+        a = np.abs(xs.reshape(-1, 32)).max(axis=1, keepdims=True)
+        assert np.all(err.reshape(-1, 32) <= a / 254 * (1 + 2.0 ** -10) + a * 2.0 ** -11 + eps)
+        return
+    sb = xs.reshape(-1, 256)
+    if qtype == Q4_K:
+        sub = sb.reshape(-1, 8, 32)
+        lo, hi = np.minimum(sub.min(axis=2), 0), sub.max(axis=2)
+        s = (hi - lo) / 15
+        df = s.max(axis=1, keepdims=True) / 63 * (1 + 2.0 ** -10)
+        dmf = (-lo).max(axis=1, keepdims=True) / 63 * (1 + 2.0 ** -10)
+        half = s / 2 + df / 4
+        bound = half + 7.5 * df + dmf / 2
+        e = err.reshape(-1, 8, 32)
+    else:
+        sub = sb.reshape(-1, 16, 16)
+        s = np.abs(sub).max(axis=2) / 31
+        df = s.max(axis=1, keepdims=True) / 127 * (1 + 2.0 ** -10)
+        half = s / 2 + df / 4
+        bound = half + 15.5 * df
+        e = err.reshape(-1, 16, 16)
+    assert np.all(e <= bound[..., None] + eps)
+    assert np.mean(e > half[..., None] + eps) < 0.05
