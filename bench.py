@@ -16,7 +16,7 @@ The JSON line also carries:
                 host -> device copy of the step's weights and activations,
                 the kernels, device -> host copy of the result, all timed
   cpu_baseline  the CPU oracle on a bounded sample of the workload (rank 0)
-  rows          every other row of the hot path (dequantize, qmv at M up to
+  rows          every other row of the hot path (the encoder, dequantize, qmv at M up to
                 16, tcgen05 qmm, MoE sort + tile map + gather, the unsort +
                 score mix, the decode MoE gather_qmv and gate/up GLU) on its
                 own workload:
@@ -374,6 +374,19 @@ def measure_rows(kq, torch, dev, pk, args) -> dict:
                                                 "frac_hbm": round(db / (t / 1e3) / 1e9 / pk["hbm_gbs"], 4),
                                                 "bytes": db}
     del Ws, out
+    # the encoder on the c0 shape: fp32 4096 x 4096 -> wire bytes of each codec
+    # (rotating fp32 copies larger than L2 between launches)
+    wf = [torch.randn(4096, 4096, device=dev) * 0.02 for _ in range(ncopies(4096 * 4096 * 4))]
+    for qt, nm in ((Q4_K, "q4K"), (Q6_K, "q6K"), (Q8_0, "q8_0")):
+        qo = torch.empty(4096, synth.row_bytes(qt, 4096), dtype=torch.uint8, device=dev)
+        t = time_graph(torch, lambda i: kq.quantize(wf[i % len(wf)], qt, out=qo), reps, s)
+        launches += reps + 3
+        qb = 4096 * 4096 * 4 + qo.numel()
+        rows[f"quantize_{nm}_4096x4096_from_fp32"] = {"kernel_us": round(t * 1e3, 2),
+                                                     "GB/s": round(qb / (t / 1e3) / 1e9, 1),
+                                                     "frac_hbm": round(qb / (t / 1e3) / 1e9 / pk["hbm_gbs"], 4),
+                                                     "bytes": qb}
+    del wf
     # c2: q4_K qmv 4096x14336, M in {1, 4, 8, 16}
     w = synth.weights(Q4_K, 4096, 14336)
     cp = ncopies(w.nbytes)
@@ -530,7 +543,7 @@ def run_reference(args, dist: Dist) -> dict | None:
 
 # ------------------------------------------------------------ profile cases
 CASES = ("qmv_q8_0", "qmv_q6_K", "qmv_q4_K_m1", "qmv_q4_K_m16", "dequant_q4_K", "qmm_q4_K", "qmm_q6_K",
-         "gather_q4_K", "gather_qmv_q4_K", "gather_mix")
+         "gather_q4_K", "gather_qmv_q4_K", "gather_mix", "quantize_q4_K", "quantize_q6_K", "quantize_q8_0")
 
 
 def run_case(name: str, iters: int) -> None:
@@ -574,6 +587,10 @@ def run_case(name: str, iters: int) -> None:
         xd = bf(synth.activations(4, 4096, seed=10))
         rid = torch.from_numpy(synth.routing(4, 8, 2, seed=9)).to(dev)
         fn = lambda: kq.gather_qmv(xd, wb, Q4_K, rid, x_per_token=True)
+    elif name.startswith("quantize_"):
+        qt = {"quantize_q4_K": Q4_K, "quantize_q6_K": Q6_K, "quantize_q8_0": Q8_0}[name]
+        wf = torch.randn(4096, 4096, device=dev) * 0.02
+        fn = lambda: kq.quantize(wf, qt)
     elif name == "gather_mix":
         ids = torch.from_numpy(synth.routing(512, 8, 2)).to(dev)
         _, _, _, inv = kq.moe_sort(ids, 8, with_inverse=True)

@@ -37,6 +37,7 @@ SIGNATURES = {
     "kq_last_cuda_error": (_int, []),
     "kq_read_device_status": (_int, [ctypes.POINTER(_i32), _int]),
     "kq_dequantize": (_int, [_int, _vp, _i64, _i64, _vp, _vp]),
+    "kq_quantize": (_int, [_int, _vp, _i64, _i64, _vp, _vp]),
     "kq_qmv": (_int, [_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp]),
     "kq_qmm": (_int, [_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp]),
     "kq_moe_sort": (_int, [_vp, _i64, _i32, _i32, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
@@ -129,6 +130,19 @@ def dequantize(w: torch.Tensor, qtype: int, k: int, out: torch.Tensor | None = N
         out = torch.empty(*w.shape[:-1], k, dtype=torch.float32, device=w.device)
     _need_cuda(w, out)
     _check(lib().kq_dequantize(qtype, _ptr(w), rows, k, _ptr(out), _stream(stream)), "kq_dequantize")
+    return out
+
+
+def quantize(w: torch.Tensor, qtype: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Wire bytes uint8 [..., row_bytes] of fp32 weights [..., K]."""
+    if w.dtype != torch.float32:
+        raise TypeError("weights must be float32")
+    k = w.shape[-1]
+    rows = w.numel() // max(1, k)
+    if out is None:
+        out = torch.empty(*w.shape[:-1], row_bytes(qtype, k), dtype=torch.uint8, device=w.device)
+    _need_cuda(w, out)
+    _check(lib().kq_quantize(qtype, _ptr(w), rows, k, _ptr(out), _stream(stream)), "kq_quantize")
     return out
 
 

@@ -152,6 +152,16 @@ int kq_dequantize(int type, const void* w, int64_t n_rows, int64_t k, float* out
     return launch_dequantize(type, w, n_rows, k, out, static_cast<cudaStream_t>(stream));
 }
 
+int kq_quantize(int type, const float* w, int64_t n_rows, int64_t k, void* out, void* stream) {
+    int vpb, bpb;
+    if (block_geometry(type, &vpb, &bpb)) return KQ_ERR_UNSUPPORTED;
+    if (k <= 0 || k % vpb != 0 || n_rows < 0) return KQ_ERR_INVALID_ARG;
+    if (n_rows == 0) return KQ_OK;
+    if (!w || !out) return KQ_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(out)) return KQ_ERR_ALIGNMENT;
+    return launch_quantize(type, w, n_rows, k, out, static_cast<cudaStream_t>(stream));
+}
+
 int kq_qmv(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int64_t m, float* y, void* stream) {
     int rc = check_weights(type, w, n, k);
     if (rc) return rc;

@@ -24,6 +24,7 @@ bool use_pair_mma();
 // Device address of the library-wide status word (bits KQ_DEV_*).
 int* device_status_ptr();
 
+int launch_quantize(int type, const float* x, int64_t n_rows, int64_t k, void* out, cudaStream_t s);
 int launch_dequantize(int type, const void* w, int64_t n_rows, int64_t k, float* out, cudaStream_t s);
 int launch_qmv(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int m, float* y,
                cudaStream_t s);

@@ -100,6 +100,24 @@ int kq_read_device_status(int32_t* host_status, int clear);
 int kq_dequantize(int type, const void* w, int64_t n_rows, int64_t k, float* out, void* stream);
 
 /*
+ * kq_quantize - encode fp32 weights into wire bytes (the step before the
+ * products).  mlx-kquant bindings.cpp, `quantize` ("Encode a float weight
+ * tensor into GGUF K-quant wire bytes"; last dim a multiple of the codec's
+ * block); hanzo-ml quantized/mod.rs `QTensor::quantize`.
+ *   w    [n_rows, k] fp32, finite (scales must stay in binary16 range)
+ *   out  [n_rows, row_bytes] wire bytes
+ * The pages give no encoding search; this one is fixed step by step in fp32:
+ * q8_0 d = max|x|/127, codes round(x * (1/d)) (ggml's rule, identical bytes);
+ * q4_K per 32 values scale (max - min(0, min))/15 and min -min(0, min x),
+ * 6-bit codes against binary16 d = max scale/63 and dmin = max min/63,
+ * codes round((x + dmin*m)/(d*sc)); q6_K per 16 values scale max|x|/31, int8
+ * codes against binary16 d = max scale/127, codes round(x/(d*sc)) + 32.
+ * Rounding is to nearest with ties away from zero.  The importance matrix
+ * of the pages' op is not supported.  n_rows == 0 enqueues nothing.
+ */
+int kq_quantize(int type, const float* w, int64_t n_rows, int64_t k, void* out, void* stream);
+
+/*
  * kq_qmv - decode-shaped product y = x . W^T for 1 <= m <= 16 rows of x.
  * mlx-kquant bindings.cpp, `quantized_matmul` (x @ dequant(w), transpose=True);
  * README "How it works": small row counts take a weight-read-amortizing

@@ -76,6 +76,17 @@ def test_matmul_argument_checks(lib, fn):
         assert f(kq.Q4_K, A, 16, 256, A, 17, A, None) == INVALID
 
 
+def test_quantize_argument_checks(lib):
+    f = lib.kq_quantize
+    assert f(5, A, 4, 256, A, None) == UNSUPPORTED
+    assert f(kq.Q4_K, A, 4, 255, A, None) == INVALID
+    assert f(kq.Q4_K, A, -1, 256, A, None) == INVALID
+    assert f(kq.Q4_K, None, 4, 256, A, None) == INVALID
+    assert f(kq.Q4_K, A, 4, 256, MIS, None) == ALIGN
+    assert f(kq.Q8_0, MIS, 4, 32, A, None) == ALIGN
+    assert f(kq.Q6_K, None, 0, 256, None, None) == OK
+
+
 def test_dequantize_argument_checks(lib):
     f = lib.kq_dequantize
     assert f(5, A, 4, 256, A, None) == UNSUPPORTED
