@@ -58,7 +58,7 @@ _BUILD = os.path.join(_HERE, "_build")
 _LIB_PATH = os.path.join(_BUILD, "liboracle.so")
 _lib = None
 
-Q8_0, Q4_K, Q6_K = 8, 12, 14
+Q4_0, Q8_0, Q4_K, Q5_K, Q6_K = 2, 8, 12, 13, 14
 TILE_ROWS = 64
 
 

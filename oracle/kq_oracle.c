@@ -1,5 +1,6 @@
 /*
- * CPU oracle for GGUF block-quantized weights (q4_K, q6_K, q8_0).
+ * CPU oracle for GGUF block-quantized weights (q4_K, q6_K, q8_0; decoders also
+ * for q5_K and q4_0).
  *
  * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
  * cpu_baseline / reference leg of bench.py may load this library.  It shares
@@ -11,7 +12,8 @@
  *  - dequantize: wire bytes -> float ("dequantize" op docstring, mlx-kquant
  *    bindings.cpp; "QTensor::dequantize -> to_float into f32", hanzo-ml
  *    quantized/mod.rs).  Block sizes: mlx-kquant README, "Codec reference"
- *    table (q4_k 256 values / 144 B, q6_k 256 / 210 B, q8_0 32 / 34 B).  The
+ *    table (q4_k 256 values / 144 B, q5_k 256 / 176 B, q6_k 256 / 210 B, q8_0
+ *    32 / 34 B, q4_0 32 / 18 B).  The
  *    field layout inside a block is not printed on the pages; the pages say
  *    the codecs are ggml's (README, "Acknowledgements") and that the scalar
  *    decoder is bit-exact against the gguf.quants reference (README, "How it
@@ -40,8 +42,10 @@
 #include <stdlib.h>
 #include <string.h>
 
+#define T_Q4_0 2
 #define T_Q8_0 8
 #define T_Q4_K 12
+#define T_Q5_K 13
 #define T_Q6_K 14
 
 /* IEEE-754 binary16 -> binary32, exact for every input (subnormals, +-0,
@@ -139,11 +143,49 @@ static void dq_q8_0(const uint8_t* b, float* out) {
     for (int i = 0; i < 32; ++i) out[i] = d * (float)qs[i];
 }
 
+/* q5_K block (176 B): d and dmin (fp16) at 0 and 2, the 12 packed 6-bit
+ * scale/min bytes at 4 (packed as in q4_K), qh[32] at 16, qs[128] at 48.
+ * Value 64c + l (c = 0..3, l = 0..31) is the low nibble of qs[32c + l] plus 16
+ * times bit 2c of qh[l], in sub-block 2c; value 64c + 32 + l is the high nibble
+ * of the same byte plus 16 times bit 2c + 1 of qh[l], in sub-block 2c + 1.
+ * y = fp32(fp32(d) * sc) * q - fp32(fp32(dmin) * m), q in 0..31. */
+static void dq_q5k(const uint8_t* b, float* out) {
+    float d = half_to_float(rd16(b)), dmin = half_to_float(rd16(b + 2));
+    const uint8_t* s = b + 4;
+    const uint8_t* qh = b + 16;
+    const uint8_t* qs = b + 48;
+    for (int c = 0; c < 4; ++c) {
+        for (int half = 0; half < 2; ++half) {
+            int j = 2 * c + half, sc, m;
+            q4k_scale_min(s, j, &sc, &m);
+            float dl = d * (float)sc, ml = dmin * (float)m;
+            for (int l = 0; l < 32; ++l) {
+                int nib = half ? (qs[32 * c + l] >> 4) : (qs[32 * c + l] & 15);
+                int q = nib + 16 * ((qh[l] >> j) & 1);
+                out[64 * c + 32 * half + l] = dl * (float)q - ml;
+            }
+        }
+    }
+}
+
+/* q4_0 block (18 B): d (fp16) at 0, qs[16] at 2.  Value l (l = 0..15) is the
+ * low nibble of qs[l] minus 8, value 16 + l the high nibble minus 8;
+ * y = fp32(d) * q. */
+static void dq_q4_0(const uint8_t* b, float* out) {
+    float d = half_to_float(rd16(b));
+    for (int l = 0; l < 16; ++l) {
+        out[l] = d * (float)((b[2 + l] & 15) - 8);
+        out[16 + l] = d * (float)((b[2 + l] >> 4) - 8);
+    }
+}
+
 int oracle_block_info(int type, int* values, int* bytes) {
     switch (type) {
     case T_Q4_K: *values = 256; *bytes = 144; return 0;
     case T_Q6_K: *values = 256; *bytes = 210; return 0;
     case T_Q8_0: *values = 32; *bytes = 34; return 0;
+    case T_Q5_K: *values = 256; *bytes = 176; return 0;
+    case T_Q4_0: *values = 32; *bytes = 18; return 0;
     default: return -1;
     }
 }
@@ -156,6 +198,8 @@ static void dq_row(int type, const uint8_t* row, int64_t k, float* out) {
         float* o = out + b * vpb;
         if (type == T_Q4_K) dq_q4k(blk, o);
         else if (type == T_Q6_K) dq_q6k(blk, o);
+        else if (type == T_Q5_K) dq_q5k(blk, o);
+        else if (type == T_Q4_0) dq_q4_0(blk, o);
         else dq_q8_0(blk, o);
     }
 }
@@ -412,6 +456,7 @@ static void qz_q6k(const float* x, uint8_t* b) {
 int oracle_quantize(int type, const float* x, int64_t n_rows, int64_t k, uint8_t* out) {
     int vpb, bpb;
     if (oracle_block_info(type, &vpb, &bpb) || k % vpb) return 1;
+    if (type != T_Q8_0 && type != T_Q4_K && type != T_Q6_K) return 1;   /* encoders of the three codecs */
     int64_t nb = n_rows * (k / vpb);
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < nb; ++i) {

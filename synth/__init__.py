@@ -6,7 +6,8 @@ CPU oracle (``oracle/``) and the CUDA library are fed the very same bytes.
 
 Block field positions follow the GGUF/ggml wire layout whose per-codec sizes
 are printed in the mlx-kquant README (METADATA page), "Codec reference" table:
-q4_K 144 B / 256 values, q6_K 210 B / 256 values, q8_0 34 B / 32 values.
+q4_K 144 B / 256 values, q5_K 176 B / 256, q6_K 210 B / 256 values, q8_0 34 B /
+32 values, q4_0 18 B / 32.
 
 Distributions (one ``numpy.random.Generator(PCG64(seed))`` stream per tensor):
 
@@ -16,16 +17,19 @@ Distributions (one ``numpy.random.Generator(PCG64(seed))`` stream per tensor):
 * q6_K: ``ql``/``qh`` uniform bytes, int8 sub-scales uniform in [-64, 63],
   ``d = fp16(|N(0,1)| * 1e-3)``.
 * q8_0: int8 codes uniform in [-128, 127], ``d = fp16(|N(0,1)| * 1e-3)``.
+* q5_K (176 B): as q4_K for ``d, dmin``, the scale bytes and the nibbles, plus
+  uniform bytes for the 32 high-bit bytes ``qh``.
+* q4_0 (18 B): ``d = fp16(|N(0,1)| * 1e-3)``, uniform nibble bytes.
 * activations: bf16 (round-to-nearest-even) of N(0,1), returned as uint16 bits.
 """
 from __future__ import annotations
 
 import numpy as np
 
-Q8_0, Q4_K, Q6_K = 8, 12, 14
-NAMES = {Q8_0: "q8_0", Q4_K: "q4_K", Q6_K: "q6_K"}
-BLOCK_VALUES = {Q8_0: 32, Q4_K: 256, Q6_K: 256}
-BLOCK_BYTES = {Q8_0: 34, Q4_K: 144, Q6_K: 210}
+Q4_0, Q8_0, Q4_K, Q5_K, Q6_K = 2, 8, 12, 13, 14
+NAMES = {Q4_0: "q4_0", Q8_0: "q8_0", Q4_K: "q4_K", Q5_K: "q5_K", Q6_K: "q6_K"}
+BLOCK_VALUES = {Q4_0: 32, Q8_0: 32, Q4_K: 256, Q5_K: 256, Q6_K: 256}
+BLOCK_BYTES = {Q4_0: 18, Q8_0: 34, Q4_K: 144, Q5_K: 176, Q6_K: 210}
 
 SEED_W, SEED_X, SEED_ROUTE = 0, 1, 2
 
@@ -51,13 +55,13 @@ def weights(qtype: int, n: int, k: int, seed: int = SEED_W, experts: int = 0) ->
     nblk = (experts or 1) * n * (k // BLOCK_VALUES[qtype])
     bpb = BLOCK_BYTES[qtype]
     blocks = g.integers(0, 256, size=(nblk, bpb), dtype=np.uint8)
-    if qtype == Q4_K:
+    if qtype in (Q4_K, Q5_K):
         dd = _scale_f16(g, 2 * nblk).reshape(nblk, 2)
         blocks[:, 0:4] = dd.view(np.uint8).reshape(nblk, 4)
     elif qtype == Q6_K:
         blocks[:, 192:208] = g.integers(-64, 64, size=(nblk, 16), dtype=np.int8).view(np.uint8)
         blocks[:, 208:210] = _scale_f16(g, nblk).view(np.uint8).reshape(nblk, 2)
-    elif qtype == Q8_0:
+    elif qtype in (Q8_0, Q4_0):
         blocks[:, 0:2] = _scale_f16(g, nblk).view(np.uint8).reshape(nblk, 2)
     else:
         raise ValueError(qtype)

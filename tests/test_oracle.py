@@ -18,6 +18,7 @@ import synth
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 Q8_0, Q4_K, Q6_K = oracle.Q8_0, oracle.Q4_K, oracle.Q6_K
+Q5_K, Q4_0 = oracle.Q5_K, oracle.Q4_0
 
 
 def bits(a):
@@ -30,7 +31,7 @@ def bits(a):
 def test_codec_table_matches_readme_and_gguf():
     import gguf
     rows = [l.split() for l in open(os.path.join(GOLDEN, "codec_table.txt")) if l[0] != "#"]
-    assert len(rows) == 3
+    assert len(rows) == 5
     for name, vpb, _bits, bpb, tid in rows:
         vpb, bpb, tid = int(vpb), int(bpb), int(tid)
         assert oracle.block_info(tid) == (vpb, bpb)
@@ -192,7 +193,7 @@ def test_zero_blocks_signed_zero():
 # ----------------------------------------------------------------------------
 # library cross-check: gguf.quants.dequantize on seeded random blocks
 # ----------------------------------------------------------------------------
-@pytest.mark.parametrize("qtype", [Q4_K, Q6_K, Q8_0])
+@pytest.mark.parametrize("qtype", [Q4_K, Q6_K, Q8_0, Q5_K, Q4_0])
 def test_matches_gguf_quants(qtype):
     import gguf
     k = 2048
@@ -212,7 +213,7 @@ def test_matches_gguf_quants(qtype):
 # ----------------------------------------------------------------------------
 # matmul: exact rational brute force and a library dot product
 # ----------------------------------------------------------------------------
-@pytest.mark.parametrize("qtype,k", [(Q4_K, 256), (Q6_K, 512), (Q8_0, 256)])
+@pytest.mark.parametrize("qtype,k", [(Q4_K, 256), (Q6_K, 512), (Q8_0, 256), (Q5_K, 256), (Q4_0, 256)])
 def test_matmul_brute_force(qtype, k):
     import gguf
     n, m = 5, 3
@@ -582,3 +583,41 @@ def test_quantize_round_trip_bound(qtype):
         e = err.reshape(-1, 16, 16)
     assert np.all(e <= bound[..., None] + eps)
     assert np.mean(e > half[..., None] + eps) < 0.05
+
+
+
+# ----------------------------------------------------------------------------
+# q5_K and q4_0 hand-built blocks
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("bit", range(8))
+def test_q5k_high_bit(bit):
+    # d = 1, dmin = 0, every scale code 1, every nibble 0, qh bytes with only
+    # bit `bit` set: sub-block `bit` reads 16 everywhere, every other value 0
+    b = np.zeros(176, np.uint8)
+    b[0:2] = np.array([1.0], np.float16).view(np.uint8)
+    b[4:16] = [1, 1, 1, 1, 0, 0, 0, 0, 1, 1, 1, 1]
+    b[16:48] = 1 << bit
+    y = oracle.dequantize(Q5_K, b[None], 256)[0]
+    sub = np.array([2 * (v // 64) + (v % 64) // 32 for v in range(256)])
+    assert np.array_equal(y, np.where(sub == bit, 16.0, 0.0).astype(np.float32))
+
+
+def test_q5k_codes_and_min():
+    # nibbles l mod 16 in both halves, high bits all set, d = 1, dmin = 1,
+    # scale codes 1, min codes 3: y = (code + 16) - 3
+    b = np.zeros(176, np.uint8)
+    b[0:4] = np.array([1.0, 1.0], np.float16).view(np.uint8)
+    b[4:16] = [1, 1, 1, 1, 3, 3, 3, 3, 0x31, 0x31, 0x31, 0x31]
+    b[16:48] = 0xFF
+    b[48:176] = [(l % 16) | ((l % 16) << 4) for c in range(4) for l in range(32)]
+    y = oracle.dequantize(Q5_K, b[None], 256)[0]
+    assert np.array_equal(y, (np.arange(256) % 16 + 16 - 3).astype(np.float32))
+
+
+def test_q4_0_all_codes():
+    b = np.zeros((1, 18), np.uint8)
+    b[0, 0:2] = np.array([0.5], np.float16).view(np.uint8)
+    b[0, 2:] = [l | ((15 - l) << 4) for l in range(16)]
+    y = oracle.dequantize(Q4_0, b, 32)[0]
+    expect = np.concatenate([np.arange(16) - 8, (15 - np.arange(16)) - 8]) * 0.5
+    assert np.array_equal(y, expect.astype(np.float32))
