@@ -49,6 +49,7 @@ import synth  # noqa: E402
 
 METRIC = "qmv effective weight GB/s (% of HBM peak); qmm/gather_qmm TFLOP/s (% bf16 peak)"
 Q8_0, Q4_K, Q6_K = synth.Q8_0, synth.Q4_K, synth.Q6_K
+Q5_K, Q4_0 = synth.Q5_K, synth.Q4_0
 L2_BYTES = 126 * 2**20
 
 
@@ -387,6 +388,37 @@ def measure_rows(kq, torch, dev, pk, args) -> dict:
                                                      "frac_hbm": round(qb / (t / 1e3) / 1e9 / pk["hbm_gbs"], 4),
                                                      "bytes": qb}
     del wf
+    # q5_K and q4_0 (no decode kernel of their own): dequantize 4096 x 4096,
+    # qmv M=1 on the c1 shape (exact fp32 decode-and-dot kernel) and qmm on the c3 shape
+    for qt, nm in ((Q5_K, "q5K"), (Q4_0, "q4_0")):
+        w = synth.weights(qt, 4096, 4096)
+        cp = ncopies(w.nbytes)
+        Ws = [u8(w) for _ in range(cp)]
+        out = torch.empty(4096, 4096, device=dev)
+        t = time_graph(torch, lambda i: kq.dequantize(Ws[i % cp], qt, 4096, out=out), reps, s)
+        launches += reps + 3
+        db = w.nbytes + 4096 * 4096 * 4
+        rows[f"dequantize_{nm}_4096x4096_fp32"] = {"kernel_us": round(t * 1e3, 2), "GB/s": round(db / (t / 1e3) / 1e9, 1),
+                                                  "frac_hbm": round(db / (t / 1e3) / 1e9 / pk["hbm_gbs"], 4), "bytes": db}
+        del Ws, out
+        w = synth.weights(qt, 14336, 4096)
+        cp = ncopies(w.nbytes)
+        Ws = [u8(w) for _ in range(cp)]
+        x1 = bf(synth.activations(1, 4096))
+        y1 = torch.empty(1, 14336, device=dev)
+        t = time_graph(torch, lambda i: kq.qmv(x1, Ws[i % cp], qt, out=y1), reps, s)
+        launches += reps + 3
+        gbs = w.nbytes / (t / 1e3) / 1e9
+        rows[f"qmv_{nm}_m1_14336x4096"] = {"kernel_us": round(t * 1e3, 2), "GB/s": round(gbs, 1),
+                                                  "frac_hbm": round(gbs / pk["hbm_gbs"], 4), "bytes": w.nbytes}
+        xq = bf(synth.activations(2048, 4096))
+        yq = torch.empty(2048, 14336, device=dev)
+        t = time_graph(torch, lambda i: kq.qmm(xq, Ws[i % cp], qt, out=yq), 8, s)
+        launches += 8 + 3
+        tf = 2 * 2048 * 14336 * 4096 / (t / 1e3) / 1e12
+        rows[f"qmm_{nm}_2048x14336x4096"] = {"kernel_us": round(t * 1e3, 2), "TFLOP/s": round(tf, 1),
+                                             "frac_bf16": round(tf / pk["bf16_tflops"], 4)}
+        del Ws, xq, yq
     # c2: q4_K qmv 4096x14336, M in {1, 4, 8, 16}
     w = synth.weights(Q4_K, 4096, 14336)
     cp = ncopies(w.nbytes)

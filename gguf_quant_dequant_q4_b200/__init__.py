@@ -7,7 +7,8 @@ current CUDA stream, every step of the computation runs in the library's
 kernels.  There is no CPU fallback; calling an op without the built library or
 without a CUDA device raises.
 
-Codecs (ggml type ids): ``Q8_0 = 8``, ``Q4_K = 12``, ``Q6_K = 14``.  Weights are
+Codecs (ggml type ids): ``Q4_0 = 2``, ``Q8_0 = 8``, ``Q4_K = 12``, ``Q5_K = 13``,
+``Q6_K = 14`` (q5_K and q4_0: dequantize and the tensor-core products).  Weights are
 wire bytes ``uint8 [N, row_bytes]`` ("transpose=True" layout: y = x @ W.T),
 activations ``bfloat16 [M, K]``, outputs ``float32``.
 """
@@ -18,9 +19,9 @@ import os
 
 import torch
 
-Q8_0, Q4_K, Q6_K = 8, 12, 14
-NAMES = {Q8_0: "q8_0", Q4_K: "q4_K", Q6_K: "q6_K"}
-_BLOCK = {Q8_0: (32, 34), Q4_K: (256, 144), Q6_K: (256, 210)}
+Q4_0, Q8_0, Q4_K, Q5_K, Q6_K = 2, 8, 12, 13, 14
+NAMES = {Q4_0: "q4_0", Q8_0: "q8_0", Q4_K: "q4_K", Q5_K: "q5_K", Q6_K: "q6_K"}
+_BLOCK = {Q4_0: (32, 18), Q8_0: (32, 34), Q4_K: (256, 144), Q5_K: (256, 176), Q6_K: (256, 210)}
 TILE_ROWS = 64
 
 DEV_BAD_EXPERT, DEV_BAD_ROWS, DEV_BAD_RANGE, DEV_UNSORTED = 0x1, 0x2, 0x4, 0x8

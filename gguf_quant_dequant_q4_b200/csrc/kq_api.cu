@@ -32,6 +32,8 @@ int block_geometry(int type, int* vpb, int* bpb) {
     case KQ_Q4_K: *vpb = 256; *bpb = 144; return KQ_OK;
     case KQ_Q6_K: *vpb = 256; *bpb = 210; return KQ_OK;
     case KQ_Q8_0: *vpb = 32; *bpb = 34; return KQ_OK;
+    case KQ_Q5_K: *vpb = 256; *bpb = 176; return KQ_OK;
+    case KQ_Q4_0: *vpb = 32; *bpb = 18; return KQ_OK;
     default: return KQ_ERR_UNSUPPORTED;
     }
 }

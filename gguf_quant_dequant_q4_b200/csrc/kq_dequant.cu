@@ -10,6 +10,7 @@
 // decodes one 256-value superblock (q4_K, q6_K) or eight 32-value blocks
 // (q8_0) per step, every lane producing 8 consecutive outputs stored as two
 // 16-byte streaming stores, so a warp writes 1 KB contiguously.
+#include "kq_decode.cuh"
 #include "kq_device.cuh"
 #include "kq_launch.h"
 
@@ -103,6 +104,20 @@ __device__ __forceinline__ void dq_q8_0(const uint8_t* blk, float* out, int part
     store8(out + 8 * part, v);
 }
 
+// q5_K superblock b: lane i writes values 8i..8i+7 (decode in kq_decode.cuh).
+__device__ __forceinline__ void dq_q5k(const uint8_t* blk, float* out, int lane) {
+    float v[8];
+    decode8_q5k(blk, lane, v);
+    store8(out + 8 * lane, v);
+}
+
+// q4_0: lane i handles block (i >> 2) of the warp's eight, values 8(i&3)..+7.
+__device__ __forceinline__ void dq_q4_0(const uint8_t* blk, float* out, int part) {
+    float v[8];
+    decode8_q4_0(blk, part, v);
+    store8(out + 8 * part, v);
+}
+
 template <int QT>
 __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict__ w, int64_t nblocks,
                                                       float* __restrict__ out) {
@@ -113,11 +128,16 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
         for (int64_t b = warp; b < nblocks; b += nwarps) dq_q4k(w + b * 144, out + b * 256, lane);
     } else if constexpr (QT == KQ_Q6_K) {
         for (int64_t b = warp; b < nblocks; b += nwarps) dq_q6k(w + b * 210, out + b * 256, lane);
+    } else if constexpr (QT == KQ_Q5_K) {
+        for (int64_t b = warp; b < nblocks; b += nwarps) dq_q5k(w + b * 176, out + b * 256, lane);
     } else {
         const int64_t units = (nblocks + 7) / 8;
         for (int64_t u = warp; u < units; u += nwarps) {
             const int64_t b = u * 8 + (lane >> 2);
-            if (b < nblocks) dq_q8_0(w + b * 34, out + b * 32, lane & 3);
+            if (b < nblocks) {
+                if constexpr (QT == KQ_Q4_0) dq_q4_0(w + b * 18, out + b * 32, lane & 3);
+                else dq_q8_0(w + b * 34, out + b * 32, lane & 3);
+            }
         }
     }
 }
@@ -125,10 +145,11 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
 }  // namespace
 
 int launch_dequantize(int type, const void* w, int64_t n_rows, int64_t k, float* out, cudaStream_t s) {
-    const int vpb = type == KQ_Q8_0 ? 32 : 256;
+    const bool small = type == KQ_Q8_0 || type == KQ_Q4_0;   // 32-value blocks, eight per warp
+    const int vpb = small ? 32 : 256;
     const int64_t nblocks = n_rows * (k / vpb);
     if (nblocks == 0) return KQ_OK;
-    const int64_t units = type == KQ_Q8_0 ? (nblocks + 7) / 8 : nblocks;
+    const int64_t units = small ? (nblocks + 7) / 8 : nblocks;
     const int sms = device_sm_count();
     int64_t grid = (units + 7) / 8;
     if (grid > static_cast<int64_t>(sms) * 16) grid = static_cast<int64_t>(sms) * 16;
@@ -136,7 +157,10 @@ int launch_dequantize(int type, const void* w, int64_t n_rows, int64_t k, float*
     switch (type) {
     case KQ_Q4_K: dequant_kernel<KQ_Q4_K><<<static_cast<int>(grid), 256, 0, s>>>(wb, nblocks, out); break;
     case KQ_Q6_K: dequant_kernel<KQ_Q6_K><<<static_cast<int>(grid), 256, 0, s>>>(wb, nblocks, out); break;
-    default: dequant_kernel<KQ_Q8_0><<<static_cast<int>(grid), 256, 0, s>>>(wb, nblocks, out); break;
+    case KQ_Q5_K: dequant_kernel<KQ_Q5_K><<<static_cast<int>(grid), 256, 0, s>>>(wb, nblocks, out); break;
+    case KQ_Q4_0: dequant_kernel<KQ_Q4_0><<<static_cast<int>(grid), 256, 0, s>>>(wb, nblocks, out); break;
+    case KQ_Q8_0: dequant_kernel<KQ_Q8_0><<<static_cast<int>(grid), 256, 0, s>>>(wb, nblocks, out); break;
+    default: return KQ_ERR_UNSUPPORTED;
     }
     return check_launch();
 }

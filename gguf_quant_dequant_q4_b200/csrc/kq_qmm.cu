@@ -61,6 +61,12 @@ template <> struct QmmCodec<KQ_Q6_K> {
 template <> struct QmmCodec<KQ_Q8_0> {
     static constexpr int RAWB = 272;   // eight 34-byte blocks
 };
+template <> struct QmmCodec<KQ_Q5_K> {
+    static constexpr int RAWB = 176;
+};
+template <> struct QmmCodec<KQ_Q4_0> {
+    static constexpr int RAWB = 144;   // eight 18-byte blocks
+};
 
 struct Smem {
     static constexpr uint32_t kBars = 0;      // mbarriers (36)
@@ -362,6 +368,54 @@ __device__ __forceinline__ void q6k_step(uint32_t row, int q, int p, const Stage
     }
 }
 
+// q5_K: as q4_K with the codes at 48 and the fifth bit of value 64q + 16p + i
+// in bit 2q + (p>>1) of qh[16(p&1) + i] (codes 0..31, exact in the same
+// bf16 trick).
+__device__ __forceinline__ void q5k_step(uint32_t row, int q, int p, const StageScales& S, uint32_t (&o)[8]) {
+    const uint4 c = lds128(row + 48 + 32 * q + 16 * (p & 1));
+    const uint4 hbits = lds128(row + 16 + 16 * (p & 1));
+    const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
+    const uint32_t hv[4] = {hbits.x, hbits.y, hbits.z, hbits.w};
+    const int j = 2 * q + (p >> 1);
+    const uint32_t hi = S.hi[q], lo = S.lo[q], nmm = S.nmm[q];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t nib = (p >> 1) ? ((wv[i] >> 4) & 0x0F0F0F0Fu) : (wv[i] & 0x0F0F0F0Fu);
+        const uint32_t code = nib | (((hv[i] >> j) & 0x01010101u) << 4);
+        const uint32_t v01 = bsub2(__byte_perm(code, kMagic, 0x5140), kB128);   // (q0, q1) exact
+        const uint32_t v23 = bsub2(__byte_perm(code, kMagic, 0x7362), kB128);
+        o[2 * i] = bfma2(v01, hi, bfma2(v01, lo, nmm));
+        o[2 * i + 1] = bfma2(v23, hi, bfma2(v23, lo, nmm));
+    }
+}
+
+// q4_0 (eight 18-byte blocks per staged row): step q, part p covers block
+// bi = 2q + (p>>1), values 16(p&1) .. +15: the low (p&1 = 0) or high nibbles
+// of its 16 code bytes.  y = fp32(d*(q-8)) rounded to bf16.
+__device__ __forceinline__ void q40_scales(uint32_t row, int p, StageScales& S) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) S.d[q] = h16v(ldsu16(row + 18 * (2 * q + (p >> 1))));
+}
+
+template <int BI, int SB>
+__device__ __forceinline__ void q40_step(uint32_t row, float d, uint32_t (&o)[8]) {
+    constexpr int L = 18 * BI + 2;
+    uint32_t QW[4];
+    lds16B<(L & 15)>(row + (L & ~15), QW);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t u = (QW[i] >> (4 * SB)) & 0x0F0F0F0Fu;
+        float f[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const uint32_t bits = __byte_perm(u, 0x4B000000u, 0x7650 + b);   // 2^23 + code
+            f[b] = __fmul_rn(d, __uint_as_float(bits) - 8388616.0f);        // code - 8, exact
+        }
+        o[2 * i] = pack_bf16x2(f[0], f[1]);
+        o[2 * i + 1] = pack_bf16x2(f[2], f[3]);
+    }
+}
+
 // q8_0 (eight 34-byte blocks per staged row): step q, part p covers block
 // bi = 2q + (p>>1), codes 16(p&1) .. +15.  y = fp32(d*q) rounded to bf16.
 __device__ __forceinline__ void q8_scales(uint32_t row, int p, StageScales& S) {
@@ -390,8 +444,10 @@ __device__ __forceinline__ void q8_step(uint32_t row, float d, uint32_t (&o)[8])
 
 template <int QT>
 __device__ __forceinline__ void prep_scales(uint32_t row, int p, int o6, StageScales& S) {
-    if constexpr (QT == KQ_Q4_K) {
-        q4k_scales(row, p, S);
+    if constexpr (QT == KQ_Q4_K || QT == KQ_Q5_K) {
+        q4k_scales(row, p, S);   // the same header
+    } else if constexpr (QT == KQ_Q4_0) {
+        q40_scales(row, p, S);
     } else if constexpr (QT == KQ_Q6_K) {
         switch (o6) {
         case 0: q6k_scales<0>(row, p, S); break;
@@ -413,6 +469,28 @@ __device__ __forceinline__ void decode_step(uint32_t row, int q, int p, int o6, 
                                             uint32_t (&o)[8]) {
     if constexpr (QT == KQ_Q4_K) {
         q4k_step(row, q, p, S, o);
+    } else if constexpr (QT == KQ_Q5_K) {
+        q5k_step(row, q, p, S, o);
+    } else if constexpr (QT == KQ_Q4_0) {
+        const float d = S.d[q];
+        switch (4 * q + p) {
+        case 0: q40_step<0, 0>(row, d, o); break;
+        case 1: q40_step<0, 1>(row, d, o); break;
+        case 2: q40_step<1, 0>(row, d, o); break;
+        case 3: q40_step<1, 1>(row, d, o); break;
+        case 4: q40_step<2, 0>(row, d, o); break;
+        case 5: q40_step<2, 1>(row, d, o); break;
+        case 6: q40_step<3, 0>(row, d, o); break;
+        case 7: q40_step<3, 1>(row, d, o); break;
+        case 8: q40_step<4, 0>(row, d, o); break;
+        case 9: q40_step<4, 1>(row, d, o); break;
+        case 10: q40_step<5, 0>(row, d, o); break;
+        case 11: q40_step<5, 1>(row, d, o); break;
+        case 12: q40_step<6, 0>(row, d, o); break;
+        case 13: q40_step<6, 1>(row, d, o); break;
+        case 14: q40_step<7, 0>(row, d, o); break;
+        default: q40_step<7, 1>(row, d, o); break;
+        }
     } else if constexpr (QT == KQ_Q6_K) {
         switch (o6) {
         case 0: q6k_step<0>(row, q, p, S, o); break;
@@ -483,6 +561,10 @@ template <> struct Stages<KQ_Q8_0, 1> { static constexpr int RST = 3, AST = 2, B
 template <> struct Stages<KQ_Q4_K, 2> { static constexpr int RST = 3, AST = 2, BST = 3, KPS = 2; };
 template <> struct Stages<KQ_Q6_K, 2> { static constexpr int RST = 2, AST = 2, BST = 3, KPS = 2; };
 template <> struct Stages<KQ_Q8_0, 2> { static constexpr int RST = 3, AST = 3, BST = 4, KPS = 1; };
+template <> struct Stages<KQ_Q5_K, 1> { static constexpr int RST = 3, AST = 2, BST = 3, KPS = 1; };
+template <> struct Stages<KQ_Q5_K, 2> { static constexpr int RST = 2, AST = 2, BST = 3, KPS = 2; };
+template <> struct Stages<KQ_Q4_0, 1> { static constexpr int RST = 3, AST = 3, BST = 3, KPS = 1; };
+template <> struct Stages<KQ_Q4_0, 2> { static constexpr int RST = 3, AST = 2, BST = 3, KPS = 2; };
 
 template <int QT, int CG>
 constexpr uint32_t smem_bytes() {
@@ -786,7 +868,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             Pipe rp;
             const int nblk = ksteps / 4;
             auto xcol = [&](int blk) {
-                if constexpr (QT == KQ_Q4_K) return 144 * blk;
+                if constexpr (QT == KQ_Q4_K || QT == KQ_Q4_0) return 144 * blk;
+                else if constexpr (QT == KQ_Q5_K) return 176 * blk;
                 else if constexpr (QT == KQ_Q6_K) return (210 * blk) & ~15;
                 else return 136 * blk;   // 2-byte elements
             };
@@ -1090,7 +1173,8 @@ template <int QT>
 int launch_impl(const void* w, int64_t w_rows, int64_t n, int64_t k, const uint16_t* x, int64_t x_rows, int n_experts,
                 const uint32_t* map, const uint32_t* count, int64_t cap, float* y, int32_t* err, cudaStream_t s) {
     using C = QmmCodec<QT>;
-    const int vpb = QT == KQ_Q8_0 ? 32 : 256, bpb = QT == KQ_Q4_K ? 144 : (QT == KQ_Q6_K ? 210 : 34);
+    const int vpb = (QT == KQ_Q8_0 || QT == KQ_Q4_0) ? 32 : 256;
+    const int bpb = QT == KQ_Q4_K ? 144 : QT == KQ_Q5_K ? 176 : QT == KQ_Q6_K ? 210 : QT == KQ_Q4_0 ? 18 : 34;
     const int64_t row_bytes = k / vpb * bpb;
     if (k % 256 != 0) return KQ_ERR_UNSUPPORTED;        // 256-value raw stages
     if (row_bytes % 16 != 0) return KQ_ERR_UNSUPPORTED;  // TMA row stride
@@ -1128,7 +1212,10 @@ int launch_qmm(int type, const void* w, int64_t n, int64_t k, const uint16_t* x,
     switch (type) {
     case KQ_Q4_K: return launch_impl<KQ_Q4_K>(w, n, n, k, x, m, 0, nullptr, nullptr, 0, y, nullptr, s);
     case KQ_Q6_K: return launch_impl<KQ_Q6_K>(w, n, n, k, x, m, 0, nullptr, nullptr, 0, y, nullptr, s);
-    default: return launch_impl<KQ_Q8_0>(w, n, n, k, x, m, 0, nullptr, nullptr, 0, y, nullptr, s);
+    case KQ_Q8_0: return launch_impl<KQ_Q8_0>(w, n, n, k, x, m, 0, nullptr, nullptr, 0, y, nullptr, s);
+    case KQ_Q5_K: return launch_impl<KQ_Q5_K>(w, n, n, k, x, m, 0, nullptr, nullptr, 0, y, nullptr, s);
+    case KQ_Q4_0: return launch_impl<KQ_Q4_0>(w, n, n, k, x, m, 0, nullptr, nullptr, 0, y, nullptr, s);
+    default: return KQ_ERR_UNSUPPORTED;
     }
 }
 
@@ -1142,8 +1229,13 @@ int launch_gather_qmm(int type, const void* w_bank, int n_experts, int64_t n, in
         return launch_impl<KQ_Q4_K>(w_bank, wr, n, k, x_sorted, rows, n_experts, map, count, cap, y, err_flag, s);
     case KQ_Q6_K:
         return launch_impl<KQ_Q6_K>(w_bank, wr, n, k, x_sorted, rows, n_experts, map, count, cap, y, err_flag, s);
-    default:
+    case KQ_Q8_0:
         return launch_impl<KQ_Q8_0>(w_bank, wr, n, k, x_sorted, rows, n_experts, map, count, cap, y, err_flag, s);
+    case KQ_Q5_K:
+        return launch_impl<KQ_Q5_K>(w_bank, wr, n, k, x_sorted, rows, n_experts, map, count, cap, y, err_flag, s);
+    case KQ_Q4_0:
+        return launch_impl<KQ_Q4_0>(w_bank, wr, n, k, x_sorted, rows, n_experts, map, count, cap, y, err_flag, s);
+    default: return KQ_ERR_UNSUPPORTED;
     }
 }
 

@@ -823,7 +823,11 @@ int launch_qmv(int type, const void* w, int64_t n, int64_t k, const uint16_t* x,
     switch (type) {
     case KQ_Q4_K: return launch_codec<KQ_Q4_K>(w, n, k, x, m, y, s);
     case KQ_Q6_K: return launch_codec<KQ_Q6_K>(w, n, k, x, m, y, s);
-    default: return launch_codec<KQ_Q8_0>(w, n, k, x, m, y, s);
+    case KQ_Q8_0: return launch_codec<KQ_Q8_0>(w, n, k, x, m, y, s);
+    // exact fp32 decode-and-dot kernel
+    case KQ_Q5_K:
+    case KQ_Q4_0: return launch_qmv_exact(type, w, n, k, x, m, y, s);
+    default: return KQ_ERR_UNSUPPORTED;
     }
 }
 

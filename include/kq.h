@@ -45,9 +45,12 @@ extern "C" {
 
 /* ggml / GGUF type ids of the supported codecs. */
 typedef enum {
+    KQ_Q4_0 = 2,   /* 32 values, 18 bytes: fp16 d, 16 B of 4-bit codes (q-8) */
     KQ_Q8_0 = 8,   /* 32 values, 34 bytes: fp16 d, 32 x int8               */
     KQ_Q4_K = 12,  /* 256 values, 144 bytes: fp16 d, fp16 dmin, 12 B packed
                       6-bit scale/min codes, 128 B of 4-bit codes             */
+    KQ_Q5_K = 13,  /* 256 values, 176 bytes: as q4_K plus 32 B of fifth bits
+                      (qh) before the 128 B of 4-bit codes                    */
     KQ_Q6_K = 14   /* 256 values, 210 bytes: 128 B low nibbles, 64 B high
                       2-bit pairs, 16 x int8 scales, fp16 d                   */
 } kq_type;
@@ -87,14 +90,14 @@ int kq_last_cuda_error(void);
 int kq_read_device_status(int32_t* host_status, int clear);
 
 /*
- * kq_dequantize - decode wire bytes to fp32, bit-exactly.
+ * kq_dequantize - decode wire bytes to fp32, bit-exactly (all five codecs).
  * mlx-kquant bindings.cpp, `dequantize` ("Dequantize GGUF K-quant wire bytes
  * to a float array"); hanzo-ml quantized/mod.rs, `QTensor::dequantize`
  * (to_float into f32).
  *   w    [n_rows, row_bytes] wire bytes
  *   out  [n_rows, k] fp32; element (r, c) = decode of value c of row r,
- *        computed in fp32 as (d*sc)*q - (dmin*m) (q4_K), (d*sc)*q (q6_K),
- *        d*q (q8_0), each operation rounded separately (no FMA).
+ *        computed in fp32 as (d*sc)*q - (dmin*m) (q4_K, q5_K), (d*sc)*q
+ *        (q6_K), d*q (q8_0, q4_0), each operation rounded separately (no FMA).
  * n_rows >= 0; n_rows == 0 enqueues nothing.
  */
 int kq_dequantize(int type, const void* w, int64_t n_rows, int64_t k, float* out, void* stream);
@@ -119,6 +122,8 @@ int kq_quantize(int type, const float* w, int64_t n_rows, int64_t k, void* out, 
 
 /*
  * kq_qmv - decode-shaped product y = x . W^T for 1 <= m <= 16 rows of x.
+ * (q5_K and q4_0 take a plainer kernel: every weight decoded exactly to
+ * fp32 and multiplied by the activations with fp32 FMAs; k % 256 == 0.)
  * mlx-kquant bindings.cpp, `quantized_matmul` (x @ dequant(w), transpose=True);
  * README "How it works": small row counts take a weight-read-amortizing
  * kernel (`verify_qmv`).  Every weight byte is read once for all m rows.

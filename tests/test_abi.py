@@ -47,6 +47,8 @@ def test_block_info_and_status_strings(lib):
     assert kq.block_info(kq.Q4_K) == (256, 144)
     assert kq.block_info(kq.Q6_K) == (256, 210)
     assert kq.block_info(kq.Q8_0) == (32, 34)
+    assert kq.block_info(kq.Q5_K) == (256, 176)
+    assert kq.block_info(kq.Q4_0) == (32, 18)
     v = ctypes.c_int()
     assert lib.kq_block_info(3, ctypes.byref(v), None) == UNSUPPORTED
     for s in range(6):
@@ -85,6 +87,7 @@ def test_quantize_argument_checks(lib):
     assert f(kq.Q4_K, A, 4, 256, MIS, None) == ALIGN
     assert f(kq.Q8_0, MIS, 4, 32, A, None) == ALIGN
     assert f(kq.Q6_K, None, 0, 256, None, None) == OK
+    assert f(kq.Q5_K, A, 4, 256, A, None) == UNSUPPORTED              # no encoder for q5_K / q4_0
 
 
 def test_dequantize_argument_checks(lib):
