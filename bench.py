@@ -63,11 +63,12 @@ def peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-# source files that define the kernel behind each roofline tag (the shared
-# device header and launch declarations included)
+# source files that define the device code of the kernel behind each roofline
+# tag (its translation unit and the shared device header; host-only launch
+# declarations do not change what the kernel does)
 KERNEL_SOURCES = {
-    "qmv_q8_0_m1_14336x4096": ("kq_qmv_stream.cu", "kq_device.cuh", "kq_launch.h"),
-    "qmv_q6_K_m1_14336x4096": ("kq_qmv_stream.cu", "kq_device.cuh", "kq_launch.h"),
+    "qmv_q8_0_m1_14336x4096": ("kq_qmv_stream.cu", "kq_device.cuh"),
+    "qmv_q6_K_m1_14336x4096": ("kq_qmv_stream.cu", "kq_device.cuh"),
 }
 
 
