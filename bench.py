@@ -576,7 +576,8 @@ def run_reference(args, dist: Dist) -> dict | None:
 
 # ------------------------------------------------------------ profile cases
 CASES = ("qmv_q8_0", "qmv_q6_K", "qmv_q4_K_m1", "qmv_q4_K_m16", "dequant_q4_K", "qmm_q4_K", "qmm_q6_K",
-         "gather_q4_K", "gather_qmv_q4_K", "gather_mix", "quantize_q4_K", "quantize_q6_K", "quantize_q8_0")
+         "gather_q4_K", "gather_qmv_q4_K", "gather_mix", "quantize_q4_K", "quantize_q6_K", "quantize_q8_0",
+         "glu_q4_K", "qmv_q5_K", "qmv_q4_0", "dequant_q5_K")
 
 
 def run_case(name: str, iters: int) -> None:
@@ -624,6 +625,19 @@ def run_case(name: str, iters: int) -> None:
         qt = {"quantize_q4_K": Q4_K, "quantize_q6_K": Q6_K, "quantize_q8_0": Q8_0}[name]
         wf = torch.randn(4096, 4096, device=dev) * 0.02
         fn = lambda: kq.quantize(wf, qt)
+    elif name == "glu_q4_K":
+        wg = u8(synth.weights(Q4_K, 14336, 4096, experts=8))
+        wu = u8(synth.weights(Q4_K, 14336, 4096, experts=8, seed=1))
+        xd = bf(synth.activations(4, 4096, seed=10))
+        rid = torch.from_numpy(synth.routing(4, 8, 2, seed=9)).to(dev)
+        fn = lambda: kq.moe_glu_gather(xd, wg, wu, Q4_K, rid)
+    elif name in ("qmv_q5_K", "qmv_q4_0"):
+        qt = Q5_K if name == "qmv_q5_K" else Q4_0
+        w, x = u8(synth.weights(qt, 14336, 4096)), bf(synth.activations(1, 4096))
+        fn = lambda: kq.qmv(x, w, qt)
+    elif name == "dequant_q5_K":
+        w = u8(synth.weights(Q5_K, 4096, 4096))
+        fn = lambda: kq.dequantize(w, Q5_K, 4096)
     elif name == "gather_mix":
         ids = torch.from_numpy(synth.routing(512, 8, 2)).to(dev)
         _, _, _, inv = kq.moe_sort(ids, 8, with_inverse=True)
