@@ -69,3 +69,12 @@ def test_gather_vs_oracle(qtype):
     for e in range(experts):
         r = np.nonzero(ids == e)[0]
         check_qmm(y[r], ref[r], xn[r], row_norms_w(qtype, w[e], k), k)
+
+
+def test_q4_0_qmv_needs_whole_256_value_steps():
+    # q4_0 rows of 96 values: dequantize works, the decode product refuses
+    w = synth.weights(kq.Q4_0, 8, 96, seed=12)
+    d = kq.dequantize(dev_u8(w), kq.Q4_0, 96).cpu().numpy()
+    assert np.array_equal(d.view(np.uint32), oracle.dequantize(kq.Q4_0, w, 96).view(np.uint32))
+    with pytest.raises(kq.KQError, match="unsupported"):
+        kq.qmv(dev_bf16(synth.activations(1, 96)), dev_u8(w), kq.Q4_0)

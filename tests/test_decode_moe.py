@@ -204,3 +204,23 @@ def test_moe_glu_gather_full_bank_sampled():
     cols = np.sort(np.random.default_rng(8).choice(n, 16, replace=False))
     ref, g, u, ag, au = oracle.moe_glu_gather(kq.Q4_K, wg[:, cols], wu[:, cols], k, x, ids)
     check_glu(y[:, cols], ref, g, u, ag, au, kq.ACT_SILU)
+
+
+def test_decode_moe_edge_cases():
+    # one pair; zero tokens (nothing enqueued); top-8 mix over the smallest N
+    w = synth.weights(kq.Q4_K, 64, 256, seed=1, experts=2)
+    x = synth.activations(1, 256, seed=2)
+    ids = np.array([[1]], np.int32)
+    y, e = run_gather_qmv(kq.Q4_K, w, 256, x, ids)
+    assert e == 0
+    check_pairs(kq.Q4_K, w, 256, x, ids, y)
+    empty = torch.empty(0, 2, dtype=torch.int32, device="cuda")
+    out = kq.gather_qmv(dev_bf16(x), dev_u8(w), kq.Q4_K, empty)
+    assert out.shape == (0, 64)
+    g = np.random.default_rng(3)
+    yv = g.standard_normal((24, 4)).astype(np.float32)
+    inv = g.permutation(24).astype(np.int32)
+    sc = g.random((3, 8)).astype(np.float32)
+    o = kq.gather_mix(torch.from_numpy(yv).cuda(), torch.from_numpy(inv).cuda(), torch.from_numpy(sc).cuda())
+    ref = oracle.gather_mix(yv, inv, sc)
+    assert np.array_equal(o.cpu().numpy().view(np.uint32), ref.view(np.uint32))

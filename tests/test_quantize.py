@@ -55,3 +55,10 @@ def test_quantize_full_size_and_round_trip(qtype):
     step = {kq.Q4_K: 1 / 15, kq.Q6_K: 1 / 31, kq.Q8_0: 1 / 127}[qtype]
     amax = np.abs(w).max()
     assert np.abs(d - w).max() <= amax * step     # a coarse bound; the exact ones are in the oracle pins
+
+
+def test_quantize_empty_and_unsupported_codec():
+    z = torch.empty(0, 256, dtype=torch.float32, device="cuda")
+    assert kq.quantize(z, kq.Q4_K).shape == (0, 144)
+    with pytest.raises(kq.KQError, match="unsupported"):
+        kq.quantize(torch.zeros(1, 256, device="cuda"), kq.Q5_K)
