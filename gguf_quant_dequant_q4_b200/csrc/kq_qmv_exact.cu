@@ -17,7 +17,6 @@ namespace kq {
 namespace {
 
 constexpr int kWarpsPerCta = 8;
-constexpr int kU = 4;   // 256-value steps whose loads are issued together
 
 template <int QT, int MT>
 __global__ void __launch_bounds__(kWarpsPerCta * 32) qmv_exact_kernel(const uint8_t* __restrict__ w, int64_t n,
@@ -31,45 +30,26 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qmv_exact_kernel(const uint
         float acc[MT];
 #pragma unroll
         for (int t = 0; t < MT; ++t) acc[t] = 0.f;
-        // kU steps of 256 values at a time: every raw load of the kU blocks
-        // is issued before the first decode, so that each lane has several
-        // independent loads in flight
-        for (int64_t v0 = 0; v0 < k; v0 += kU * 256) {
-            const int steps = static_cast<int>((k - v0) / 256 < kU ? (k - v0) / 256 : kU);
-            RawQ5K r5[kU];
-            RawQ40 r4[kU];
-            int64_t col[kU];
-#pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                if (u < steps) {
-                    const int64_t vs = v0 + 256 * u;
-                    if constexpr (QT == KQ_Q5_K) {
-                        r5[u] = load_q5k(row + (vs / 256) * 176, lane);
-                        col[u] = vs + 8 * lane;
-                    } else {
-                        const int64_t b = vs / 32 + (lane >> 2);
-                        r4[u] = load_q4_0(row + b * 18, lane & 3);
-                        col[u] = b * 32 + 8 * (lane & 3);
-                    }
-                }
+        for (int64_t v0 = 0; v0 < k; v0 += 256) {
+            float wv[8];
+            int64_t col;   // first of the lane's 8 values
+            if constexpr (QT == KQ_Q5_K) {
+                decode8_q5k(row + (v0 / 256) * 176, lane, wv);
+                col = v0 + 8 * lane;
+            } else {
+                const int64_t b = v0 / 32 + (lane >> 2);
+                decode8_q4_0(row + b * 18, lane & 3, wv);
+                col = b * 32 + 8 * (lane & 3);
             }
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                if (u < steps) {
-                    float wv[8];
-                    if constexpr (QT == KQ_Q5_K) decode_q5k(r5[u], lane, wv);
-                    else decode_q4_0(r4[u], lane & 3, wv);
+            for (int t = 0; t < MT; ++t) {
+                if (t < m) {
+                    const uint4 xr = __ldg(reinterpret_cast<const uint4*>(x + t * k + col));
+                    const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
 #pragma unroll
-                    for (int t = 0; t < MT; ++t) {
-                        if (t < m) {
-                            const uint4 xr = __ldg(reinterpret_cast<const uint4*>(x + t * k + col[u]));
-                            const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                acc[t] = fmaf(wv[2 * i], __uint_as_float(xw[i] << 16), acc[t]);
-                                acc[t] = fmaf(wv[2 * i + 1], __uint_as_float(xw[i] & 0xffff0000u), acc[t]);
-                            }
-                        }
+                    for (int i = 0; i < 4; ++i) {
+                        acc[t] = fmaf(wv[2 * i], __uint_as_float(xw[i] << 16), acc[t]);
+                        acc[t] = fmaf(wv[2 * i + 1], __uint_as_float(xw[i] & 0xffff0000u), acc[t]);
                     }
                 }
             }
