@@ -289,6 +289,7 @@ __device__ __forceinline__ void lds16B(uint32_t a, uint32_t (&w)[4]) {
 //   16 bits), so the result carries essentially one bf16 rounding.
 constexpr uint32_t kB128 = 0x43004300u;   // bf16 (128, 128)
 constexpr uint32_t kB160 = 0x43204320u;   // bf16 (160, 160)
+constexpr uint32_t kB136 = 0x43084308u;   // bf16 (136, 136)
 constexpr uint32_t kMagic = 0x43434343u;
 
 struct StageScales {
@@ -391,28 +392,25 @@ __device__ __forceinline__ void q5k_step(uint32_t row, int q, int p, const Stage
 
 // q4_0 (eight 18-byte blocks per staged row): step q, part p covers block
 // bi = 2q + (p>>1), values 16(p&1) .. +15: the low (p&1 = 0) or high nibbles
-// of its 16 code bytes.  y = fp32(d*(q-8)) rounded to bf16.
+// of its 16 code bytes.  code - 8 is exact in bf16 (the 128 + code trick,
+// minus 136), multiplied by d split into two bf16 parts as in q6_K.
 __device__ __forceinline__ void q40_scales(uint32_t row, int p, StageScales& S) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) S.d[q] = h16v(ldsu16(row + 18 * (2 * q + (p >> 1))));
+    for (int q = 0; q < 4; ++q) split_scale(h16v(ldsu16(row + 18 * (2 * q + (p >> 1)))), S.hi[q], S.lo[q]);
 }
 
 template <int BI, int SB>
-__device__ __forceinline__ void q40_step(uint32_t row, float d, uint32_t (&o)[8]) {
+__device__ __forceinline__ void q40_step(uint32_t row, uint32_t hi, uint32_t lo, uint32_t (&o)[8]) {
     constexpr int L = 18 * BI + 2;
     uint32_t QW[4];
     lds16B<(L & 15)>(row + (L & ~15), QW);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const uint32_t u = (QW[i] >> (4 * SB)) & 0x0F0F0F0Fu;
-        float f[4];
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const uint32_t bits = __byte_perm(u, 0x4B000000u, 0x7650 + b);   // 2^23 + code
-            f[b] = __fmul_rn(d, __uint_as_float(bits) - 8388616.0f);        // code - 8, exact
-        }
-        o[2 * i] = pack_bf16x2(f[0], f[1]);
-        o[2 * i + 1] = pack_bf16x2(f[2], f[3]);
+        const uint32_t v01 = bsub2(__byte_perm(u, kMagic, 0x5140), kB136);   // code - 8, exact
+        const uint32_t v23 = bsub2(__byte_perm(u, kMagic, 0x7362), kB136);
+        o[2 * i] = bfma2(v01, hi, bmul2(v01, lo));
+        o[2 * i + 1] = bfma2(v23, hi, bmul2(v23, lo));
     }
 }
 
@@ -472,24 +470,24 @@ __device__ __forceinline__ void decode_step(uint32_t row, int q, int p, int o6, 
     } else if constexpr (QT == KQ_Q5_K) {
         q5k_step(row, q, p, S, o);
     } else if constexpr (QT == KQ_Q4_0) {
-        const float d = S.d[q];
+        const uint32_t hi = S.hi[q], lo = S.lo[q];
         switch (4 * q + p) {
-        case 0: q40_step<0, 0>(row, d, o); break;
-        case 1: q40_step<0, 1>(row, d, o); break;
-        case 2: q40_step<1, 0>(row, d, o); break;
-        case 3: q40_step<1, 1>(row, d, o); break;
-        case 4: q40_step<2, 0>(row, d, o); break;
-        case 5: q40_step<2, 1>(row, d, o); break;
-        case 6: q40_step<3, 0>(row, d, o); break;
-        case 7: q40_step<3, 1>(row, d, o); break;
-        case 8: q40_step<4, 0>(row, d, o); break;
-        case 9: q40_step<4, 1>(row, d, o); break;
-        case 10: q40_step<5, 0>(row, d, o); break;
-        case 11: q40_step<5, 1>(row, d, o); break;
-        case 12: q40_step<6, 0>(row, d, o); break;
-        case 13: q40_step<6, 1>(row, d, o); break;
-        case 14: q40_step<7, 0>(row, d, o); break;
-        default: q40_step<7, 1>(row, d, o); break;
+        case 0: q40_step<0, 0>(row, hi, lo, o); break;
+        case 1: q40_step<0, 1>(row, hi, lo, o); break;
+        case 2: q40_step<1, 0>(row, hi, lo, o); break;
+        case 3: q40_step<1, 1>(row, hi, lo, o); break;
+        case 4: q40_step<2, 0>(row, hi, lo, o); break;
+        case 5: q40_step<2, 1>(row, hi, lo, o); break;
+        case 6: q40_step<3, 0>(row, hi, lo, o); break;
+        case 7: q40_step<3, 1>(row, hi, lo, o); break;
+        case 8: q40_step<4, 0>(row, hi, lo, o); break;
+        case 9: q40_step<4, 1>(row, hi, lo, o); break;
+        case 10: q40_step<5, 0>(row, hi, lo, o); break;
+        case 11: q40_step<5, 1>(row, hi, lo, o); break;
+        case 12: q40_step<6, 0>(row, hi, lo, o); break;
+        case 13: q40_step<6, 1>(row, hi, lo, o); break;
+        case 14: q40_step<7, 0>(row, hi, lo, o); break;
+        default: q40_step<7, 1>(row, hi, lo, o); break;
         }
     } else if constexpr (QT == KQ_Q6_K) {
         switch (o6) {
