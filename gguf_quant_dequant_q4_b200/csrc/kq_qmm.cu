@@ -551,13 +551,15 @@ struct Pipe {
 // each.  A CTA pair halves the activation stage.  Raw stages come from DRAM
 // and have the longest latency to cover.  Every stage boundary costs the MMA
 // issuing thread a wait and a release, which the shallow MMA queue does not
-// hide, so where shared memory allows a stage holds two K steps.
+// hide, so where shared memory allows a stage holds two K steps.  The split
+// between A and B stages is measured per codec: q4_K pairs are faster with
+// three B stages, q6_K pairs (the heavier decoder) with three A stages.
 template <int QT, int CG> struct Stages;
 template <> struct Stages<KQ_Q4_K, 1> { static constexpr int RST = 3, AST = 3, BST = 3, KPS = 1; };
 template <> struct Stages<KQ_Q6_K, 1> { static constexpr int RST = 3, AST = 2, BST = 3, KPS = 1; };
 template <> struct Stages<KQ_Q8_0, 1> { static constexpr int RST = 3, AST = 2, BST = 2, KPS = 1; };
 template <> struct Stages<KQ_Q4_K, 2> { static constexpr int RST = 3, AST = 2, BST = 3, KPS = 2; };
-template <> struct Stages<KQ_Q6_K, 2> { static constexpr int RST = 2, AST = 2, BST = 3, KPS = 2; };
+template <> struct Stages<KQ_Q6_K, 2> { static constexpr int RST = 2, AST = 3, BST = 2, KPS = 2; };
 template <> struct Stages<KQ_Q8_0, 2> { static constexpr int RST = 3, AST = 3, BST = 4, KPS = 1; };
 template <> struct Stages<KQ_Q5_K, 1> { static constexpr int RST = 3, AST = 2, BST = 3, KPS = 1; };
 template <> struct Stages<KQ_Q5_K, 2> { static constexpr int RST = 2, AST = 2, BST = 3, KPS = 2; };
