@@ -228,7 +228,7 @@ int kq_gather_qmv(int type, const void* w_bank, int32_t n_experts, int64_t n, in
     if (n_experts < 1 || n_experts > 256 || n_tokens < 0 || top_k < 1) return KQ_ERR_INVALID_ARG;
     int rc = check_weights(type, w_bank, n, k);
     if (rc) return rc;
-    if (n_tokens * top_k > 8192) return KQ_ERR_INVALID_ARG;
+    if (n_tokens > 8192 || n_tokens * top_k > 8192) return KQ_ERR_INVALID_ARG;
     if (static_cast<int64_t>(n_experts) * n > (int64_t(1) << 31) - 1) return KQ_ERR_INVALID_ARG;
     if (n == 0 || n_tokens == 0) return KQ_OK;
     if (!x || !ids || !y) return KQ_ERR_INVALID_ARG;
@@ -250,7 +250,7 @@ int kq_moe_glu_gather(int type, const void* gate_bank, const void* up_bank, int3
     if (rc) return rc;
     rc = check_weights(type, up_bank, n, k);
     if (rc) return rc;
-    if (n_tokens * top_k > 8192) return KQ_ERR_INVALID_ARG;
+    if (n_tokens > 8192 || n_tokens * top_k > 8192) return KQ_ERR_INVALID_ARG;
     if (static_cast<int64_t>(n_experts) * n > (int64_t(1) << 31) - 1) return KQ_ERR_INVALID_ARG;
     if (n == 0 || n_tokens == 0) return KQ_OK;
     if (!x || !ids || !out) return KQ_ERR_INVALID_ARG;

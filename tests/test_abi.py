@@ -126,6 +126,7 @@ def test_decode_moe_argument_checks(lib):
     assert g(kq.Q4_K, A, 8, 64, 250, A, 0, A, 1, 2, A, None, None) == INVALID    # K not a block multiple
     assert g(kq.Q4_K, A, 8, 64, 256, A, 0, A, 1, 0, A, None, None) == INVALID    # top_k < 1
     assert g(kq.Q4_K, A, 8, 64, 256, A, 0, A, 4097, 2, A, None, None) == INVALID  # more than 8192 pairs
+    assert g(kq.Q4_K, A, 8, 64, 256, A, 0, A, 2**62, 4, A, None, None) == INVALID  # no overflow of the count
     assert g(kq.Q4_K, A, 8, 64, 256, None, 0, A, 1, 2, A, None, None) == INVALID
     assert g(kq.Q4_K, A, 8, 64, 256, A, 0, None, 1, 2, A, None, None) == INVALID
     assert g(kq.Q4_K, A, 8, 64, 256, MIS, 0, A, 1, 2, A, None, None) == ALIGN
@@ -140,6 +141,7 @@ def test_decode_moe_argument_checks(lib):
     m = lib.kq_gather_mix
     assert m(A, 8, 6, A, A, 4, 2, A, None, None) == INVALID                      # n % 4
     assert m(A, 8, 8, A, A, 4, 0, A, None, None) == INVALID                      # top_k < 1
+    assert m(A, 8, 8, A, A, 4, 65, A, None, None) == INVALID                     # top_k > 64
     assert m(A, 8, 8, None, A, 4, 2, A, None, None) == INVALID
     assert m(A, 8, 8, A, A, 4, 2, MIS, None, None) == ALIGN
     assert m(MIS, 8, 8, A, A, 4, 2, A, None, None) == ALIGN
