@@ -17,7 +17,8 @@
 // 256 activation rows, MMA M = 128.)  Persistent, one CTA per SM,
 // warp-specialized:
 //   warp 0      activation producer: TMA of bf16 activation tiles
-//               (128B-swizzled, one 64-row box per map tile)
+//               (128B-swizzled 64-row boxes: over the CTA's half of a unit's
+//               run of rows, or one per map tile when the tiles are not one run)
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer (in the
 //               first CTA of a pair; the full barriers it waits on live
 //               there, and its commits arrive on both CTAs' empty barriers)
@@ -48,7 +49,7 @@ constexpr int kMaxTiles = 1024;   // map tiles a gather call may use
 constexpr uint32_t kHeader = 5120; // barriers, misc words, tile tables
 constexpr int kDeqWarp0 = 6;   // warps 0..5: producer, MMA, 4 epilogue
 constexpr int kRawWarp = kDeqWarp0 + kDecWarps;   // the raw weight producer
-constexpr int kRawAhead = 4;   // raw stages prefetched into L2 ahead of their load
+constexpr int kRawAhead = 2;   // raw stages prefetched into L2 ahead of their load (measured: 1-2 best)
 
 template <int QT> struct QmmCodec;
 // raw row bytes per stage (one 256-value block column of 128 weight rows)
