@@ -71,3 +71,23 @@ def test_reference_arm_json(monkeypatch, capsys):
 def test_cpu_sample_is_bounded():
     r = bench.cpu_sample(seconds=0.0)       # one pass of the oracle on c1
     assert r["kind"] == "oracle" and r["value"] > 0 and r["cores"] >= 1
+
+
+def test_traffic_keyed_by_kernel_device_sources(tmp_path, monkeypatch):
+    # the roofline's DRAM traffic is reported only while the sources of the
+    # profiled kernel are the ones the counters were taken on; a host-only
+    # launch header does not count, a change to the kernel's file does
+    csrc = tmp_path / "gguf_quant_dequant_q4_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for f in ("kq_qmv_stream.cu", "kq_device.cuh", "kq_launch.h"):
+        (csrc / f).write_text(f"// {f}\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    tag = "qmv_q6_K_m1_14336x4096"
+    h = bench.kernel_source_hash(tag)
+    (tmp_path / "profiles" / "p.txt").write_text(f"summary\ntraffic {tag} 48223488 {h}\n")
+    assert bench.profiled_traffic(tag) == 48223488
+    (csrc / "kq_launch.h").write_text("// a new host declaration\n")
+    assert bench.profiled_traffic(tag) == 48223488
+    (csrc / "kq_qmv_stream.cu").write_text("// the kernel changed\n")
+    assert bench.profiled_traffic(tag) is None
