@@ -1,7 +1,8 @@
 /*
  * kq.h - C ABI of the B200 (sm_100a) library for matrix products with GGUF
- * block-quantized weights: y = x . W^T where W is stored as q4_K, q6_K or
- * q8_0 wire blocks.
+ * block-quantized weights: y = x . W^T where W is stored as q4_K, q6_K,
+ * q8_0, q5_K or q4_0 wire blocks, plus the encoder that writes such blocks,
+ * the MoE routing helpers and the MoE epilogues.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -21,15 +22,19 @@
  *    (bindings.cpp docstring: "uint8 K-quant wire bytes (laid out [N, K] when
  *    transpose=True)") and of the README's "x @ dequant(w).T".
  *  - Activations x are bfloat16 [m, k] row-major (passed as uint16_t bit
- *    patterns).  They are converted to binary16 inside the kernels, so
- *    |x| must stay below 65504 for qmv; bf16 is used as is by qmm/gather.
+ *    patterns).  The decode kernels of q4_K, q6_K and q8_0 (kq_qmv,
+ *    kq_gather_qmv, kq_moe_glu_gather) convert them to binary16, so |x| must
+ *    stay below 65504 there (KQ_DEV_X_RANGE flags it); qmm/gather use bf16 as
+ *    is, and the q5_K / q4_0 qmv widens it to fp32 exactly.
  *  - Outputs y are fp32 [m, n] row-major.
  *  - Return value: a kq_status.  A non-zero status means nothing was enqueued
  *    (argument errors) or that the CUDA launch failed (KQ_ERR_CUDA; the
  *    cudaError_t is available from kq_last_cuda_error()).  Nothing throws.
  *  - Alignment: W, x, y and out must be 16-byte aligned, else
  *    KQ_ERR_ALIGNMENT.  Weight rows whose byte length is not a multiple of 16
- *    are accepted; they take a slower staging path.
+ *    are accepted by kq_dequantize and kq_qmv (a slower staging path);
+ *    kq_qmm / kq_gather_qmm need k % 256 == 0 and 16-byte multiple rows
+ *    (KQ_ERR_UNSUPPORTED otherwise).
  *  - `k` must be a multiple of the codec's values_per_block, as the reference
  *    requires ("last dim a multiple of the codec's bytes_per_block",
  *    bindings.cpp `dequantize`); otherwise KQ_ERR_INVALID_ARG.
