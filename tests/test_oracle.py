@@ -418,6 +418,22 @@ def test_glu_activations():
     # the tanh form stays within 1e-3 of the exact gelu g * Phi(g) (Phi from erf)
     exact = np.array([0.5 * v * (1 + math.erf(v / math.sqrt(2))) for v in g])
     assert np.max(np.abs(oracle.glu(oracle.ACT_GELU_TANH, g, one) - exact)) < 1e-3
+    # and it is exactly the tanh form: torch's own float64 implementation of
+    # gelu(approximate="tanh") agrees to 1e-14 absolutely everywhere and to
+    # 1e-12 relative where the value is not a cancellation residue of
+    # 1 + tanh (|gelu| > 1e-2); a wrong constant such as 0.8 for sqrt(2/pi),
+    # or 0.0447 for 0.044715, is off by more than 1e-5 absolute and 1e-3
+    # relative
+    import torch
+    ref = torch.nn.functional.gelu(torch.from_numpy(g), approximate="tanh").numpy()
+    got = oracle.glu(oracle.ACT_GELU_TANH, g, one)
+    big = np.abs(ref) > 1e-2
+    assert np.max(np.abs(got - ref)[big] / np.abs(ref[big])) < 1e-12
+    assert np.max(np.abs(got - ref)) < 1e-14
+    # two points worked by hand from the definition, to 1e-15
+    for v, want in ((1.0, 0.5 * (1 + math.tanh(math.sqrt(2 / math.pi) * 1.044715))),
+                    (-2.0, -1.0 * (1 + math.tanh(math.sqrt(2 / math.pi) * (-2.0 - 0.35772))))):
+        assert abs(float(oracle.glu(oracle.ACT_GELU_TANH, np.array([v]), np.ones(1))[0]) - want) <= 1e-15 * abs(want)
     # silu with a limit: the gate is capped from above, the up value clipped both ways
     lim = 3.0
     out = oracle.glu(oracle.ACT_SILU_LIMIT, g, 10 * u, limit=lim)
