@@ -218,4 +218,28 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1,
 
 __host__ __device__ constexpr int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
+// ------------------------------------------- activation scaling (decode)
+// The decode kernels round activations to binary16 for the tensor cores.
+// Binary16 covers magnitudes 2^-14 .. 65504 at full precision only, so each
+// token's activations are first multiplied by an exact power of two 2^s that
+// brings its largest magnitude into [2^T, 2^(T+1)); the inverse 2^-s is
+// applied to that token's fp32 sums.  `mx` is the bf16 bit pattern of the
+// largest |x| (non-negative values order as their bit patterns).  s = 0 for
+// an all-zero or non-finite token; s is clamped to [-126, 126] so that both
+// 2^s and 2^-s are normal fp32 numbers.
+__device__ __forceinline__ int xscale_exp(uint32_t mx, int T) {
+    if (mx == 0 || mx >= 0x7F80u) return 0;
+    const int s = T - (static_cast<int>(mx >> 7) - 127);
+    return s < -126 ? -126 : (s > 126 ? 126 : s);
+}
+// 2^s for -126 <= s <= 126, exactly.
+__device__ __forceinline__ float exp2_int(int s) { return __uint_as_float(static_cast<uint32_t>(127 + s) << 23); }
+// Largest |x| of 8 bf16 values (a 16-byte chunk) folded into `mx` as a pair
+// of 16-bit bit patterns.
+__device__ __forceinline__ uint32_t absmax8_bf16(uint32_t mx, uint4 v) {
+    const uint32_t a = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+    const uint32_t b = __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu);
+    return __vmaxu2(mx, __vmaxu2(a, b));
+}
+
 }  // namespace kq

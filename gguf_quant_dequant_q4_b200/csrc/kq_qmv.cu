@@ -20,10 +20,13 @@
 //    fragment is one 8-byte load).  The tensor core forms exact products and
 //    accumulates them in fp32, so the only rounding besides fp32 summation is
 //    x -> binary16.
-//  * Binary16 codes come from the exponent trick: OR-ing a 4/6/8-bit code
-//    into the mantissa of 1024.0 gives 1024 + code exactly.  The 1024 bias
-//    is removed exactly (q4_K: one HFMA2 that also applies the scale) or
-//    folded into a per-sub-block correction c * sum(x) in the epilogue.
+//  * Binary16 codes: q4_K ORs its 4-bit code into the mantissa of 1024.0
+//    (1024 + code, exactly) and removes the 1024 with the HFMA2 that also
+//    applies its scale; q6_K and q8_0 put the code's bits in the mantissa with
+//    exponent field 0, a subnormal code x 2^-24 (exact; the tensor core keeps
+//    subnormal operands exact), and the codec's own offset (32, 128) is
+//    removed in the fp32 epilogue with a per-sub-block sum of the activation
+//    operands; the 2^24 goes into the per-block scale.
 //  * q4_K (per-block scales d, dmin): each lane owns one 64-value group of a
 //    block, so it decodes only its own two 6-bit scale/min pairs; the MMA
 //    chain runs over the whole block and the min term sum_j m_j * X_j is one
@@ -32,6 +35,10 @@
 //    sub-block.  For m <= 4 the 8 MMA columns are shared out as
 //    (token, sub-block slot) pairs, so one epilogue covers up to 8 sub-blocks
 //    instead of wasting 7 of 8 columns.
+//  * Activation range: before the binary16 rounding each token's activations
+//    (per super-chunk of K) are multiplied by a power of two that puts their
+//    largest magnitude at 2^T; the warps multiply their partial sums by the
+//    inverse, so the relative precision does not depend on the scale of x.
 //  * Partial sums of the 8 warps are combined in shared memory in a fixed
 //    order: no atomics, bitwise reproducible.
 #include "kq_device.cuh"
@@ -45,23 +52,28 @@ constexpr int kProducerWarp = kCWarps;      // bulk-copy producer
 constexpr int kReducerWarp = kCWarps + 1;   // cross-warp reduction and stores
 constexpr int kThreads = 32 * (kCWarps + 2);
 constexpr int kRows = 16;
-constexpr int kOffW = 384;   // barriers, flags and a zero word live below
+constexpr int kOffW = 512;   // barriers, flags, a zero word and the activation scales live below
+constexpr int kXMax = 320;   // largest |x| per token, bf16 bits, two buffers of 16 words
+constexpr int kXInv = 448;   // inverse activation scale per token (16 floats)
 constexpr int kMaxStages = 8;
 
 template <int QT> struct Codec;
 // Stage geometry is chosen per call: a stage is 16 rows x g blocks, g a
 // multiple of GA (so every per-row copy starts 16-byte aligned), as large as
 // shared memory allows; rows are padded to a stride of 16 mod 128 bytes.
+// XT: target exponent of the scaled activations (largest magnitude in
+// [2^XT, 2^(XT+1))): q4_K keeps its 32-value sums inside binary16 range,
+// q6_K and q8_0 keep their smallest operands (x/256, x/64) normal.
 template <> struct Codec<KQ_Q4_K> {
-    static constexpr int VPB = 256, BPB = 144, GA = 8;
+    static constexpr int VPB = 256, BPB = 144, GA = 8, XT = 9;
     static constexpr int IMG = 544, XS = 0;   // B image bytes / fp32 sums per (token, block)
 };
 template <> struct Codec<KQ_Q6_K> {
-    static constexpr int VPB = 256, BPB = 210, GA = 8;
+    static constexpr int VPB = 256, BPB = 210, GA = 8, XT = 14;
     static constexpr int IMG = 1024, XS = 16;
 };
 template <> struct Codec<KQ_Q8_0> {
-    static constexpr int VPB = 32, BPB = 34, GA = 8;
+    static constexpr int VPB = 32, BPB = 34, GA = 8, XT = 14;
     static constexpr int IMG = 64, XS = 1;
 };
 
@@ -79,6 +91,7 @@ struct QmvParams {
 constexpr uint32_t kH1024 = 0x64006400u;    // (1024, 1024)
 constexpr uint32_t kHm1024 = 0xE400E400u;   // (-1024, -1024)
 constexpr uint32_t kH1_16 = 0x2C002C00u;    // (1/16, 1/16)
+constexpr float kTwo24 = 16777216.0f;        // 2^24: a subnormal code's unit is 2^-24
 
 // Shared-memory loads are volatile so that they are never moved across the
 // mbarrier waits and __syncthreads that order them with the bulk copies.
@@ -95,7 +108,6 @@ __device__ __forceinline__ int ldss8c(uint32_t a) {
     asm volatile("ld.shared.s8 %0, [%1];" : "=h"(v) : "r"(a));
     return v;
 }
-__device__ __forceinline__ float ldsf32c(uint32_t a) { return __uint_as_float(lds32c(a)); }
 // 4 bytes at a 2-byte aligned address; `odd` = (a & 2) is warp-uniform.
 __device__ __forceinline__ uint32_t lds32c_a2(uint32_t a, bool odd) {
     if (!odd) return lds32c(a);
@@ -109,29 +121,61 @@ __device__ __forceinline__ void sts32(uint32_t a, uint32_t x) {
 }
 __device__ __forceinline__ float h16(uint32_t h) { return __half2float(__ushort_as_half((unsigned short)h)); }
 
-// x (bf16) -> binary16, recording a range violation.
-__device__ __forceinline__ uint32_t f16pair(float a, float b, float& amax) {
-    amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
-    return pack_f16x2(a, b);
+// Scaled bf16 pair -> binary16 pair, and the two binary16 values back as floats.
+__device__ __forceinline__ uint32_t f16pair(float a, float b, float S) { return pack_f16x2(a * S, b * S); }
+__device__ __forceinline__ float f16sum(uint32_t h) { return h16(h & 0xffff) + h16(h >> 16); }
+// Scale 2^s of token m for the codec's target exponent (see xscale_exp).
+template <int QT>
+__device__ __forceinline__ float tok_scale(const uint32_t* xm, int m) {
+    return exp2_int(xscale_exp(xm[m], Codec<QT>::XT));
+}
+
+// Largest |x| of every token over values [v0, v0 + nv) of K, as bf16 bit
+// patterns, by atomic max into xm[token] (zeroed beforehand).  All consumer
+// warps take part: 16 / m warps per token, each lane loading up to eight
+// 16-byte chunks before it reduces, so the loads overlap.
+__device__ void x_range(const QmvParams& p, int64_t v0, int nv, uint32_t* xm) {
+    constexpr int U = 8;
+    const int chunks = nv / 8;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wpt = p.m < kCWarps ? kCWarps / p.m : 1;
+    const int m = warp / wpt, slot = warp % wpt;
+    if (m >= p.m) return;   // warp-uniform
+    uint32_t mx = 0;
+    for (int c0 = slot * 32 * U; c0 < chunks; c0 += wpt * 32 * U) {
+        uint4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int c = c0 + 32 * u + lane;
+            v[u] = c < chunks ? ldg_nc_v4(p.x + static_cast<int64_t>(m) * p.k + v0 + 8 * c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) mx = absmax8_bf16(mx, v[u]);
+    }
+    mx = __reduce_max_sync(0xffffffffu, max(mx & 0xFFFFu, mx >> 16));
+    if (lane == 0 && mx) atomicMax(&xm[m], mx);
 }
 
 // ---------------------------------------------------------------------------
 // Activation images.  For block bl of the current super-chunk and token m the
 // image holds, for every MMA of that block and every lane column t, the two
-// B registers of lane (g = token, t) in binary16.
+// B registers of lane (g = token, t) in binary16 (of the scaled activations).
 // ---------------------------------------------------------------------------
 template <int QT>
-__device__ void build_image(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t xsum, float& amax);
+__device__ void build_image(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t xsum, const uint32_t* xm);
 
 // q4_K: MMA (nib, u) of lane t uses values v = 64t + 32nib + 4u + {0,2 | 1,3};
-// the extra 32 bytes per block hold (Xhi, Xlo) of sub-blocks 2t and 2t+1.
+// the extra 32 bytes per block hold (Xhi, Xlo) of sub-blocks 2t and 2t+1, the
+// sums of their binary16 operands split into two binary16 parts.
 template <>
-__device__ void build_image<KQ_Q4_K>(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t, float& amax) {
+__device__ void build_image<KQ_Q4_K>(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t,
+                                     const uint32_t* xm) {
     const int items = p.m * nb * 4;
     for (int it = threadIdx.x; it < items; it += kCWarps * 32) {
         const int m = it / (nb * 4), rem = it % (nb * 4), bl = rem >> 2, t = rem & 3;
         const uint16_t* xs = p.x + static_cast<int64_t>(m) * p.k + static_cast<int64_t>(blk0 + bl) * 256 + 64 * t;
         const uint32_t base = img + m * p.tokstride + bl * 544;
+        const float S = tok_scale<KQ_Q4_K>(xm, m);
         float X[2] = {0.f, 0.f};
 #pragma unroll
         for (int nib = 0; nib < 2; ++nib) {
@@ -145,8 +189,8 @@ __device__ void build_image<KQ_Q4_K>(const QmvParams& p, int blk0, int nb, uint3
                     const int u = 4 * uu + q;
                     const float f0 = bf16lo_to_f32(wv[2 * q]), f1 = bf16hi_to_f32(wv[2 * q]);
                     const float f2 = bf16lo_to_f32(wv[2 * q + 1]), f3 = bf16hi_to_f32(wv[2 * q + 1]);
-                    const uint32_t h02 = f16pair(f0, f2, amax), h13 = f16pair(f1, f3, amax);
-                    X[nib] += (h16(h02 & 0xffff) + h16(h13 & 0xffff)) + (h16(h02 >> 16) + h16(h13 >> 16));
+                    const uint32_t h02 = f16pair(f0, f2, S), h13 = f16pair(f1, f3, S);
+                    X[nib] += f16sum(h02) + f16sum(h13);
                     sts64(base + (nib * 8 + u) * 32 + t * 8, h02, h13);
                 }
             }
@@ -163,14 +207,16 @@ __device__ void build_image<KQ_Q4_K>(const QmvParams& p, int blk0, int nb, uint3
 }
 
 // q8_0: MMA h (0, 1) of lane t uses values v = 8t + 4h + {0,2 | 1,3};
-// X = sum of the block's 32 binary16 values.
+// X = 128 2^-24 (= 2^-17) times the sum of the block's 32 binary16 operands.
 template <>
-__device__ void build_image<KQ_Q8_0>(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t xsum, float& amax) {
+__device__ void build_image<KQ_Q8_0>(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t xsum,
+                                     const uint32_t* xm) {
     const int items = p.m * nb;
     for (int it = threadIdx.x; it < items; it += kCWarps * 32) {
         const int m = it / nb, bl = it % nb;
         const uint16_t* xs = p.x + static_cast<int64_t>(m) * p.k + static_cast<int64_t>(blk0 + bl) * 32;
         const uint32_t base = img + m * p.tokstride + bl * 64;
+        const float S = tok_scale<KQ_Q8_0>(xm, m);
         float X = 0.f;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
@@ -180,41 +226,47 @@ __device__ void build_image<KQ_Q8_0>(const QmvParams& p, int blk0, int nb, uint3
             for (int h = 0; h < 2; ++h) {
                 const float f0 = bf16lo_to_f32(wv[2 * h]), f1 = bf16hi_to_f32(wv[2 * h]);
                 const float f2 = bf16lo_to_f32(wv[2 * h + 1]), f3 = bf16hi_to_f32(wv[2 * h + 1]);
-                const uint32_t h02 = f16pair(f0, f2, amax), h13 = f16pair(f1, f3, amax);
-                X += (h16(h02 & 0xffff) + h16(h13 & 0xffff)) + (h16(h02 >> 16) + h16(h13 >> 16));
+                const uint32_t h02 = f16pair(f0, f2, S), h13 = f16pair(f1, f3, S);
+                X += f16sum(h02) + f16sum(h13);
                 sts64(base + h * 32 + t * 8, h02, h13);
             }
         }
-        sts32(xsum + (m * p.scb + bl) * 4, __float_as_uint(X));
+        sts32(xsum + (m * p.scb + bl) * 4, __float_as_uint(X * 7.62939453125e-06f));
     }
 }
 
 // q6_K: sub-block j (16 values, j = 8h + 2tq + u) has a low-code MMA and a
 // high-code MMA; lane t uses values 16j + 4t + {0,2 | 1,3}.  The low-code B
-// is x/16 (tq < 2) or x/256 (tq >= 2, where the code sits in the high
-// nibble); the high-code B is x / 4^tq.  X_j = sum of the 16 values.
+// is a = x/16 (tq < 2) or x/256 (tq >= 2, where the code sits in the high
+// nibble); the high-code B is x / 4^tq (x scaled, then rounded to binary16).
+// The MMAs give D = 2^-24 sum c x / 16 with c the 6-bit code, so
+// sum (c - 32) x = 16 2^24 (D - X) with X = 2^-24 * 32 * sum x / 16, stored
+// from the low-code operands: 2^-19 sum a (tq < 2) or 2^-15 sum a.
 template <>
-__device__ void build_image<KQ_Q6_K>(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t xsum, float& amax) {
+__device__ void build_image<KQ_Q6_K>(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t xsum,
+                                     const uint32_t* xm) {
     const int items = p.m * nb * 16;
     for (int it = threadIdx.x; it < items; it += kCWarps * 32) {
         const int m = it / (nb * 16), rem = it % (nb * 16), bl = rem >> 4, j = rem & 15;
         const int tq = (j & 7) >> 1;
-        const float slo = tq < 2 ? 0.0625f : 0.00390625f, shi = 1.0f / static_cast<float>(1 << (2 * tq));
+        const float S = tok_scale<KQ_Q6_K>(xm, m);
+        const float slo = S * (tq < 2 ? 0.0625f : 0.00390625f), shi = S * exp2_int(-2 * tq);
         const uint16_t* xs = p.x + static_cast<int64_t>(m) * p.k + static_cast<int64_t>(blk0 + bl) * 256 + 16 * j;
         const uint32_t base = img + m * p.tokstride + bl * 1024 + j * 64;
         const uint4 r0 = ldg_nc_v4(xs), r1 = ldg_nc_v4(xs + 8);
         const uint32_t wv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-        float X = 0.f;
+        float A = 0.f;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
             const float f0 = bf16lo_to_f32(wv[2 * t]), f1 = bf16hi_to_f32(wv[2 * t]);
             const float f2 = bf16lo_to_f32(wv[2 * t + 1]), f3 = bf16hi_to_f32(wv[2 * t + 1]);
-            const uint32_t h02 = f16pair(f0, f2, amax), h13 = f16pair(f1, f3, amax);
-            X += (h16(h02 & 0xffff) + h16(h13 & 0xffff)) + (h16(h02 >> 16) + h16(h13 >> 16));
-            sts64(base + t * 8, pack_f16x2(f0 * slo, f2 * slo), pack_f16x2(f1 * slo, f3 * slo));
-            sts64(base + 32 + t * 8, pack_f16x2(f0 * shi, f2 * shi), pack_f16x2(f1 * shi, f3 * shi));
+            const uint32_t a02 = f16pair(f0, f2, slo), a13 = f16pair(f1, f3, slo);
+            A += f16sum(a02) + f16sum(a13);
+            sts64(base + t * 8, a02, a13);
+            sts64(base + 32 + t * 8, f16pair(f0, f2, shi), f16pair(f1, f3, shi));
         }
-        sts32(xsum + ((m * p.scb + bl) * 16 + j) * 4, __float_as_uint(X));
+        sts32(xsum + ((m * p.scb + bl) * 16 + j) * 4,
+              __float_as_uint(A * (tq < 2 ? 1.9073486328125e-06f : 3.0517578125e-05f)));
     }
 }
 
@@ -353,11 +405,11 @@ __device__ __forceinline__ void q8_run(const Lane<NT>& L, const QmvParams& p, ui
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const uint32_t wa = h ? a1w : a0w, wb = h ? b1w : b0w;
-                // (byte ^ 0x80) in the mantissa of 1024: 1024 + q + 128 exactly
-                const uint32_t A0 = and_xor(wa, 0x00FF00FFu, 0x64806480u);
-                const uint32_t A1 = and_xor(wb, 0x00FF00FFu, 0x64806480u);
-                const uint32_t A2 = and_xor(wa >> 8, 0x00FF00FFu, 0x64806480u);
-                const uint32_t A3 = and_xor(wb >> 8, 0x00FF00FFu, 0x64806480u);
+                // byte ^ 0x80 = q + 128 as a binary16 subnormal: (q + 128) 2^-24
+                const uint32_t A0 = and_xor(wa, 0x00FF00FFu, 0x00800080u);
+                const uint32_t A1 = and_xor(wb, 0x00FF00FFu, 0x00800080u);
+                const uint32_t A2 = and_xor(wa >> 8, 0x00FF00FFu, 0x00800080u);
+                const uint32_t A3 = and_xor(wb >> 8, 0x00FF00FFu, 0x00800080u);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     uint2 bv = lds64c(L.tokb[nt] + imgb0 + i * 64 + h * 32 + t * 8);
@@ -370,7 +422,8 @@ __device__ __forceinline__ void q8_run(const Lane<NT>& L, const QmvParams& p, ui
             }
         }
         if (i % S == S - 1 || i == RUN - 1) {
-            // epilogue: y += d * (D - 1152 X) per column's block
+            // epilogue: y += 2^24 d (D - X) per column's block (D = 2^-24
+            // sum (q + 128) x, X = 2^-17 sum x)
             const int i0 = i - (i % S);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
@@ -381,9 +434,9 @@ __device__ __forceinline__ void q8_run(const Lane<NT>& L, const QmvParams& p, ui
                     const int ib = i0 + slot;
                     if (ib < nvalid && ib <= i) {
                         const uint32_t row = (e >> 1) ? rowB : rowA;
-                        const float d = h16(ldsu16c(row + (lb0 + ib) * 34));
-                        const float X = ldsf32c(xsb0 + (tok * p.scb + ib) * 4);
-                        acc[nt][e] = fmaf(d, fmaf(-1152.0f, X, D[nt][e]), acc[nt][e]);
+                        const float d = h16(ldsu16c(row + (lb0 + ib) * 34)) * kTwo24;
+                        const float X = __uint_as_float(lds32c(xsb0 + (tok * p.scb + ib) * 4));
+                        acc[nt][e] = fmaf(d, D[nt][e] - X, acc[nt][e]);
                     }
                 }
             }
@@ -427,16 +480,15 @@ __device__ __forceinline__ void q6k_half(const Lane<NT>& L, const QmvParams& p, 
         }
         const uint32_t la = QLA[2 * pp + u], lb = QLB[2 * pp + u];
         const uint32_t ha = QHA[u], hb = QHB[u];
-        // low 4 bits: low nibble (tq < 2) -> 1024 + c with B = x/16, high
-        // nibble (tq >= 2) -> 1024 + 16c with B = x/256
+        // low 4 bits as binary16 subnormals: low nibble c (tq < 2) -> c 2^-24
+        // with B = x/16, high nibble (tq >= 2) -> 16 c 2^-24 with B = x/256
         const uint32_t mlo = tq < 2 ? 0x000F000Fu : 0x00F000F0u;
-        const uint32_t L0 = and_or(la, mlo, kH1024), L1 = and_or(lb, mlo, kH1024);
-        const uint32_t L2 = and_or(la >> 8, mlo, kH1024), L3 = and_or(lb >> 8, mlo, kH1024);
-        // high 2 bits, left at bits 2tq..2tq+1 of each byte: 1024 + 4^tq c with
-        // B = x / 4^tq (all B scalings are exact powers of two, none above 1)
+        const uint32_t L0 = la & mlo, L1 = lb & mlo, L2 = (la >> 8) & mlo, L3 = (lb >> 8) & mlo;
+        // high 2 bits h, left at bits 2tq..2tq+1 of each byte: 4^tq h 2^-24,
+        // with B = x / 4^tq (all B scalings are exact powers of two, none
+        // above 1).  The two MMAs sum 2^-24 c6 x / 16.
         const uint32_t mhi = 0x00030003u << (2 * tq);
-        const uint32_t H0 = and_or(ha, mhi, kH1024), H1 = and_or(hb, mhi, kH1024);
-        const uint32_t H2 = and_or(ha >> 8, mhi, kH1024), H3 = and_or(hb >> 8, mhi, kH1024);
+        const uint32_t H0 = ha & mhi, H1 = hb & mhi, H2 = (ha >> 8) & mhi, H3 = (hb >> 8) & mhi;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const uint32_t a = L.tokb[nt] + imgb + j * 64 + t * 8;
@@ -460,16 +512,13 @@ __device__ __forceinline__ void q6k_half(const Lane<NT>& L, const QmvParams& p, 
                     int tok, slot;
                     col_info<S, NT>(nt, 2 * t + (e & 1), p.m, tok, slot);
                     const int jj = j0 + slot;
-                    const int tqj = (jj & 7) >> 1;
-                    // D = (sum c x)/16 + bias X with bias = 1024/sigma_lo + 1024/4^tq;
-                    // sum (c - 32) x = 16 (D - (bias + 2) X)
-                    const float C = tqj == 0 ? 1090.0f : (tqj == 1 ? 322.0f : (tqj == 2 ? 70.0f : 22.0f));
+                    // sum (c - 32) x = 16 2^24 (D - X), X from the image build
                     const uint32_t row = (e >> 1) ? rowB : rowA;
                     const float dr = (e >> 1) ? dB : dA;
                     const int sc = ldss8c(row + 192 + jj);
-                    const float s = 16.0f * __fmul_rn(dr, static_cast<float>(sc));
-                    const float X = ldsf32c(xsb + (tok * p.scb * 16 + jj) * 4);
-                    acc[nt][e] = fmaf(s, fmaf(-C, X, D[nt][e]), acc[nt][e]);
+                    const float s = 268435456.0f * __fmul_rn(dr, static_cast<float>(sc));   // 16 2^24 d sc
+                    const float X = __uint_as_float(lds32c(xsb + (tok * p.scb * 16 + jj) * 4));
+                    acc[nt][e] = fmaf(s, D[nt][e] - X, acc[nt][e]);
                 }
             }
         }
@@ -509,6 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const QmvParams p) {
         fence_barrier_init();
     }
     if (tid < 4) sts32(zero_addr + 4 * tid, 0u);
+    if (tid < 32) reinterpret_cast<uint32_t*>(smem + kXMax)[tid] = 0u;
     // Programmatic dependent launch: the next kernel in the stream may start
     // its prologue now.  This CTA's weight bytes are prefetched into L2 (a
     // hint; L2 is coherent, so it is safe even if an earlier kernel is still
@@ -635,17 +685,29 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const QmvParams p) {
         // q4_K: two groups of 8 warps take alternate stages (a warp decodes a
         // whole block); the other codecs share every stage among all 16 warps
         const int grp = warp >> 3, wig = warp & 7;
-        float amax = 0.f;
         float* pbuf = reinterpret_cast<float*>(smem + p.off_pbuf);
+        float* xinv = reinterpret_cast<float*>(smem + kXInv);
         constexpr int PW = 32 * 4 * NT;
         int q = 0, it = 0;
-        for (int sc = 0; sc < nsc && !*abort_flag; ++sc) {
+        // every consumer thread passes the same barriers, aborted or not
+        for (int sc = 0; sc < nsc; ++sc) {
             const int blk0 = sc * p.scb;
             const int nbsc = p.nblk - blk0 < p.scb ? p.nblk - blk0 : p.scb;
             const int nst = stages_in(sc);
+            // the super-chunk's activation scales (two buffers of maxima: the
+            // other one is cleared for the next super-chunk), then its image
+            uint32_t* xm = reinterpret_cast<uint32_t*>(smem + kXMax) + 16 * (sc & 1);
             asm volatile("bar.sync 1, %0;" ::"r"(kCWarps * 32));
-            build_image<QT>(p, blk0, nbsc, sbase + p.off_img, sbase + p.off_x, amax);
+            if (!*abort_flag) x_range(p, static_cast<int64_t>(blk0) * C::VPB, nbsc * C::VPB, xm);
+            if (tid < 16) xm[16 * (1 - 2 * (sc & 1)) + tid] = 0u;
             asm volatile("bar.sync 1, %0;" ::"r"(kCWarps * 32));
+            if (tid < p.m) {
+                if (xm[tid] >= 0x7F80u) atomicOr(p.status, KQ_DEV_X_RANGE);   // Inf or NaN
+                xinv[tid] = exp2_int(-xscale_exp(xm[tid], C::XT));
+            }
+            if (!*abort_flag) build_image<QT>(p, blk0, nbsc, sbase + p.off_img, sbase + p.off_x, xm);
+            asm volatile("bar.sync 1, %0;" ::"r"(kCWarps * 32));
+            if (*abort_flag) continue;
             for (int g = 0; g < nrg; ++g, ++it) {
                 float acc[NT][4];
 #pragma unroll
@@ -692,7 +754,16 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const QmvParams p) {
                     }
                 }
                 if (!ok) break;
-                // hand the warp's partial sums of this row group to the reducer
+                // hand the warp's partial sums of this row group, unscaled, to
+                // the reducer
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        int tok, slot;
+                        col_info<S, NT>(nt, 2 * L.t + (e & 1), p.m, tok, slot);
+                        acc[nt][e] *= xinv[tok];
+                    }
                 const int b = it & 1;
                 if (!bwait(&red_empty[b], ((it >> 1) & 1) ^ 1)) break;
                 float* dst = pbuf + (b * kCWarps + warp) * PW + lane * 4 * NT;
@@ -703,7 +774,6 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const QmvParams p) {
                 if (lane == 0) mbar_arrive(&red_full[b]);
             }
         }
-        if (amax >= 65504.0f) atomicOr(p.status, KQ_DEV_X_RANGE);
     }
     __syncthreads();
 }

@@ -18,7 +18,16 @@
 // into binary16 integers (OR into the mantissa of 1024), the activations
 // rounded once to binary16 are the B operand of m16n8k16 MMAs, and the tensor
 // core accumulates exact products in fp32; per-block scales are applied in
-// fp32 once a block is complete.  The activation operand of every MMA is
+// fp32 once a block is complete.  Before that rounding each token's
+// activations are scaled by a power of two that puts its largest magnitude
+// at 2^T (T per codec), and the inverse scale is applied to its fp32 sums, so
+// the relative precision does not depend on the activations' magnitude.  The
+// q8_0 and q6_K codes enter the MMA as binary16 subnormals (the code's bits in
+// the mantissa, exponent field 0: code x 2^-24, exact; the tensor core keeps
+// subnormal operands exact), so the only offset left is the codec's own (128
+// for q8_0's unsigned view of the int8 code, 32 for q6_K), removed in the fp32
+// epilogue with sums of the very binary16 activation operands the MMAs
+// consumed; the 2^24 goes into the per-block scale.  The activation operand of every MMA is
 // precomputed per CTA into a shared-memory image in fragment order (one
 // 8-byte load per MMA); B lanes whose column does not receive a given word
 // read a zero block instead of being masked.  The lane-to-byte mappings:
@@ -51,6 +60,7 @@ namespace kq {
 namespace {
 
 constexpr int kCW = 16;                  // consumer warps
+static_assert((kCW & (kCW - 1)) == 0, "warp round robin uses a power-of-two mask");
 constexpr int kProd = kCW;               // producer warp
 constexpr int kThreads = 32 * (kCW + 1);
 constexpr int kRows = 16;
@@ -100,6 +110,8 @@ struct SPGLU : SPG {
 };
 constexpr uint32_t kGList = 512;     // gather: pair list of the CTA (16 ints)
 constexpr uint32_t kGMisc = 576;     // gather: expert, pairs present, row range
+constexpr uint32_t kXMax = 640;      // largest |x| per token (bf16 bits, 16 words)
+constexpr uint32_t kXInv = 704;      // inverse activation scale per token (16 floats)
 constexpr uint32_t kGCount = 1024;   // gather: pairs per expert (256 ints)
 constexpr uint32_t kGHdr = 2048;     // gather header size
 
@@ -114,6 +126,7 @@ __device__ __forceinline__ int group_order(int rg, int nrg, int64_t rows) {
 constexpr uint32_t kH1024 = 0x64006400u;    // binary16 (1024, 1024)
 constexpr uint32_t kHm1024 = 0xE400E400u;   // (-1024, -1024)
 constexpr uint32_t kH1_16 = 0x2C002C00u;    // (1/16, 1/16)
+constexpr float kTwo24 = 16777216.0f;        // 2^24: a subnormal code's unit is 2^-24
 
 // Volatile so that the conversions stay next to the MMA that consumes them.
 __device__ __forceinline__ uint32_t vand_or(uint32_t a, uint32_t b, uint32_t c) {
@@ -185,10 +198,11 @@ __device__ __forceinline__ uint32_t xaddr(const SP& p, uint32_t sb, int tok, int
 __device__ __forceinline__ float xval(const SP& p, uint32_t sb, int tok, int64_t i) {
     return __uint_as_float(lds_u16(xaddr(p, sb, tok, i)) << 16);
 }
-// Binary16 of a (power-of-two scaled) activation, tracking the range.
-__device__ __forceinline__ __half hx(float v, float& amax) {
-    amax = fmaxf(amax, fabsf(v));
-    return __float2half_rn(v);
+// Binary16 of an activation times its token's power-of-two scale.
+__device__ __forceinline__ __half hx(float v, float scale) { return __float2half_rn(v * scale); }
+// Scale 2^s of token `tok` (see xscale_exp) for a codec with target exponent T.
+__device__ __forceinline__ float tok_scale(const uint32_t* xmax, int tok, int T) {
+    return exp2_int(xscale_exp(xmax[tok], T));
 }
 __device__ __forceinline__ uint32_t hpair(__half lo, __half hi) {
     return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
@@ -210,6 +224,11 @@ struct Q8 {
     static constexpr uint32_t kItemImg = 17 * 32;   // image bytes per item (8 blocks) and token
     static constexpr uint32_t kZero = kItemImg;
     static constexpr int kAccPerLane = 2 * NT;
+    // scaled activations below 2^15: the 1152 + code operands and the
+    // 32-value sums X stay far inside fp32 and binary16 range
+    static constexpr int kXT = 14;
+    // token of accumulator i (acc[2 nt + r]: token nt, row g + 8 r)
+    static __device__ __forceinline__ int acc_tok(const Lane&, int i) { return i >> 1; }
 
     // rowA/rowB: shared address of the item (8 blocks) in rows g / g+8;
     // gi: global item index (block 8 gi).
@@ -238,26 +257,27 @@ struct Q8 {
         for (int mu = 0; mu < 17; ++mu) {
             const uint32_t wa = lds32(a0 + 4 * mu), wb = lds32(b0 + 4 * mu);
             if (mu == 0) {   // fp16 d of the even block: bytes 0..1 of the span
-                dE[0] = h2f(wa & 0xffff);
-                dE[1] = h2f(wb & 0xffff);
+                dE[0] = h2f(wa & 0xffff) * kTwo24;
+                dE[1] = h2f(wb & 0xffff) * kTwo24;
             }
             if (mu == 8) {   // the odd block's d: bytes 34..35
-                dO[0] = h2f(wa >> 16);
-                dO[1] = h2f(wb >> 16);
+                dO[0] = h2f(wa >> 16) * kTwo24;
+                dO[1] = h2f(wb >> 16) * kTwo24;
             }
             const int par = mu >= 9 ? 1 : 0;
-            // (byte ^ 0x80) in the mantissa of 1024: 1152 + code, exactly
-            const uint32_t A0 = vand_xor(wa, 0x00FF00FFu, 0x64806480u);
-            const uint32_t A1 = vand_xor(wb, 0x00FF00FFu, 0x64806480u);
-            const uint32_t A2 = vand_xor(wa >> 8, 0x00FF00FFu, 0x64806480u);
-            const uint32_t A3 = vand_xor(wb >> 8, 0x00FF00FFu, 0x64806480u);
+            // byte ^ 0x80 = 128 + code as a binary16 subnormal: (128 + code) 2^-24
+            const uint32_t A0 = vand_xor(wa, 0x00FF00FFu, 0x00800080u);
+            const uint32_t A1 = vand_xor(wb, 0x00FF00FFu, 0x00800080u);
+            const uint32_t A2 = vand_xor(wa >> 8, 0x00FF00FFu, 0x00800080u);
+            const uint32_t A3 = vand_xor(wb >> 8, 0x00FF00FFu, 0x00800080u);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const uint2 bv = lds64(bb[nt][par] + 32 * mu);
                 mma_f16(D[nt][mu & 1], A0, A1, A2, A3, bv.x, bv.y);
             }
         }
-        // y += d (D - 1152 X) for columns 2t (even block) and 2t+1 (odd block)
+        // D = 2^-24 sum (128 + code) a;  y += 2^24 d (D - 2^-17 X), X = sum a,
+        // for columns 2t (even block) and 2t+1 (odd block)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const uint2 xv = lds64(sb + p.off_xs + nt * p.xs_tok + 4 * (8 * gi + 2 * t));
@@ -266,8 +286,7 @@ struct Q8 {
             for (int e = 0; e < 4; ++e) {
                 const int r = e >> 1, odd = e & 1;
                 const float Ds = D[nt][0][e] + D[nt][1][e];
-                const float d = odd ? dO[r] : dE[r];
-                acc[2 * nt + r] = fmaf(d, fmaf(-1152.0f, X[odd], Ds), acc[2 * nt + r]);
+                acc[2 * nt + r] = fmaf(odd ? dO[r] : dE[r], Ds - X[odd], acc[2 * nt + r]);
             }
         }
     }
@@ -285,21 +304,23 @@ struct Q8 {
             }
     }
 
-    // Image entry (item, mu, t') = binary16 activations of the 4 raw bytes at
-    // offset 272 item + 68 t' + 4 mu of a row, as (byte0, byte2 | byte1,
-    // byte3); scale bytes get 0.  X[tok][block] = sum of its 32 activations.
-    static __device__ void build(const SP& p, uint32_t sb, float& amax, int64_t xoff) {
+    // Image entry (item, mu, t') = binary16 of the scaled activations of the 4
+    // raw bytes at offset 272 item + 68 t' + 4 mu of a row, as (byte0, byte2 |
+    // byte1, byte3); scale bytes get 0.  X[tok][block] = 2^-17 (= 128 2^-24)
+    // times the sum of the block's 32 binary16 operands.
+    static __device__ void build(const SP& p, uint32_t sb, const uint32_t* xmax, int64_t xoff) {
         const int items = p.nblk / 8;
         const int per_tok = items * 17 * 4;
         for (int e = threadIdx.x; e < p.m * per_tok; e += kCW * 32) {
             const int tok = e / per_tok, rem = e % per_tok;
             const int it = rem / 68, mu = (rem % 68) >> 2, tt = rem & 3;
             const int R0 = it * 272 + 68 * tt + 4 * mu;
+            const float S = tok_scale(xmax, tok, kXT);
             __half h[4];
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
                 const int R = R0 + b, blk = R / 34, o = R - 34 * blk;
-                h[b] = o >= 2 ? hx(xval(p, sb, tok, 32 * blk + o - 2), amax) : __float2half_rn(0.f);
+                h[b] = o >= 2 ? hx(xval(p, sb, tok, 32 * blk + o - 2), S) : __float2half_rn(0.f);
             }
             sts64(sb + p.off_img + tok * p.img_tok + it * kItemImg + mu * 32 + tt * 8, hpair(h[0], h[2]),
                   hpair(h[1], h[3]));
@@ -307,6 +328,7 @@ struct Q8 {
         for (int e = threadIdx.x; e < p.m * p.nblk; e += kCW * 32) {
             const int tok = e / p.nblk, blk = e % p.nblk;
             const uint32_t xs = xaddr(p, sb, tok, 32 * blk);
+            const float S = tok_scale(xmax, tok, kXT);
             float X = 0.f;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -314,11 +336,11 @@ struct Q8 {
                 const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    X += __half2float(__float2half_rn(bf16lo_to_f32(wv[q])));
-                    X += __half2float(__float2half_rn(bf16hi_to_f32(wv[q])));
+                    X += __half2float(hx(bf16lo_to_f32(wv[q]), S));
+                    X += __half2float(hx(bf16hi_to_f32(wv[q]), S));
                 }
             }
-            sts32(sb + p.off_xs + tok * p.xs_tok + 4 * blk, __float_as_uint(X));
+            sts32(sb + p.off_xs + tok * p.xs_tok + 4 * blk, __float_as_uint(X * 7.62939453125e-06f));
         }
     }
 };
@@ -340,6 +362,10 @@ struct Q6 {
     static constexpr uint32_t kBlkImg = 512;   // image bytes per block and token
     static constexpr uint32_t kZero = 512;
     static constexpr int kAccPerLane = 2 * NT;
+    // scaled activations below 2^15: the x/16 and x/256 operands stay normal
+    // binary16 numbers down to 2^-22 of the token's largest magnitude
+    static constexpr int kXT = 14;
+    static __device__ __forceinline__ int acc_tok(const Lane&, int i) { return i >> 1; }
 
     // Word at shared address a (2-byte aligned when ODD).
     template <bool ODD>
@@ -377,7 +403,7 @@ struct Q6 {
             const uint32_t row = r ? rowB : rowA;
 #pragma unroll
             for (int q = 0; q < 4; ++q) sc[r][q] = static_cast<float>(lds_s8(row + 192 + 8 * h + lh + 2 * q));
-            d16[r] = 16.0f * h2f(lds_u16(row + 208));
+            d16[r] = 268435456.0f * h2f(lds_u16(row + 208));   // 2^28 d = 16 d 2^24
         }
         // the lane's 4 qh words (rows g, g+8), in its rotated order
         const uint32_t rot[4] = {4u * ((0 + t) & 3), 4u * ((1 + t) & 3), 4u * ((2 + t) & 3), 4u * ((3 + t) & 3)};
@@ -407,16 +433,16 @@ struct Q6 {
                 const uint32_t wa8 = wa >> 8, wb8 = wb >> 8;
                 const uint32_t sa02 = ha[k] << sh, sa13 = ha[k] >> (8 - sh);
                 const uint32_t sb02 = hb[k] << sh, sb13 = hb[k] >> (8 - sh);
-                // low nibble + field qp -> 1024 + c6
-                const uint32_t L0 = vbitsel(wa, vand_or(sa02, 0x00300030u, kH1024), 0x000F000Fu);
-                const uint32_t L1 = vbitsel(wb, vand_or(sb02, 0x00300030u, kH1024), 0x000F000Fu);
-                const uint32_t L2 = vbitsel(wa8, vand_or(sa13, 0x00300030u, kH1024), 0x000F000Fu);
-                const uint32_t L3 = vbitsel(wb8, vand_or(sb13, 0x00300030u, kH1024), 0x000F000Fu);
-                // high nibble + field qp + 2 -> 1024 + 16 c6
-                const uint32_t H0 = vbitsel(wa, vand_or(sa02, 0x03000300u, kH1024), 0x00F000F0u);
-                const uint32_t H1 = vbitsel(wb, vand_or(sb02, 0x03000300u, kH1024), 0x00F000F0u);
-                const uint32_t H2 = vbitsel(wa8, vand_or(sa13, 0x03000300u, kH1024), 0x00F000F0u);
-                const uint32_t H3 = vbitsel(wb8, vand_or(sb13, 0x03000300u, kH1024), 0x00F000F0u);
+                // low nibble + field qp -> c6 as a subnormal (c6 2^-24)
+                const uint32_t L0 = vbitsel(wa, vand_or(sa02, 0x00300030u, 0u), 0x000F000Fu);
+                const uint32_t L1 = vbitsel(wb, vand_or(sb02, 0x00300030u, 0u), 0x000F000Fu);
+                const uint32_t L2 = vbitsel(wa8, vand_or(sa13, 0x00300030u, 0u), 0x000F000Fu);
+                const uint32_t L3 = vbitsel(wb8, vand_or(sb13, 0x00300030u, 0u), 0x000F000Fu);
+                // high nibble + field qp + 2 -> 16 c6 as a subnormal
+                const uint32_t H0 = vbitsel(wa, vand_or(sa02, 0x03000300u, 0u), 0x00F000F0u);
+                const uint32_t H1 = vbitsel(wb, vand_or(sb02, 0x03000300u, 0u), 0x00F000F0u);
+                const uint32_t H2 = vbitsel(wa8, vand_or(sa13, 0x03000300u, 0u), 0x00F000F0u);
+                const uint32_t H3 = vbitsel(wb8, vand_or(sb13, 0x03000300u, 0u), 0x00F000F0u);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const uint2 bl = lds64(bb[nt][0] + 32 * (8 * qp + k));
@@ -425,8 +451,10 @@ struct Q6 {
                     mma_f16(D[k & 1][nt], H0, H1, H2, H3, bh.x, bh.y);
                 }
             }
-            // columns 2t (q = qp, C = 66) and 2t + 1 (q = qp + 2, C = 6):
-            // y += 16 d sc_j (D - C X_j)
+            // column 2t: D = 2^-24 sum c a with a = x/16, column 2t + 1:
+            // D = 2^-24 sum 16 c a with a = x/256; both are 2^-24 sum c x / 16,
+            // and sum (c - 32) x = 16 2^24 (D - X) with X the stored offset sum
+            // (2^-19 sum a, resp. 2^-15 sum a): y += 2^28 d sc_j (D - X)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const uint2 xv = lds64(sb + p.off_xs + nt * p.xs_tok + ((gb * 4 + t) * 4 + 2 * qp) * 4);
@@ -435,8 +463,7 @@ struct Q6 {
                 for (int e = 0; e < 4; ++e) {
                     const int r = e >> 1, c = e & 1;
                     const float Ds = D[0][nt][e] + D[1][nt][e];
-                    const float s = __fmul_rn(d16[r], sc[r][qp + 2 * c]);
-                    acc[2 * nt + r] = fmaf(s, fmaf(c ? -6.0f : -66.0f, X[c], Ds), acc[2 * nt + r]);
+                    acc[2 * nt + r] = fmaf(__fmul_rn(d16[r], sc[r][qp + 2 * c]), Ds - X[c], acc[2 * nt + r]);
                 }
             }
         }
@@ -452,24 +479,26 @@ struct Q6 {
         Q8<NT>::store_part(p, L, acc, part);
     }
 
-    // Image entry (block, E = 8 qp + 4 s + k, t'): binary16 of x[v] / 16
-    // (s = 0) or / 256 (s = 1) for q = qp + 2s, l = 16 lh + 4 ((k + t') mod 4)
-    // + {0, 2 | 1, 3}, v = 128h + 32q + l (h, lh of quarter t').
-    // X[tok][block][t'][qp][s] = sum over the 16 l of binary16(x[v]).
-    static __device__ void build(const SP& p, uint32_t sb, float& amax, int64_t xoff) {
+    // Image entry (block, E = 8 qp + 4 s + k, t'): binary16 of x[v] S / 16
+    // (s = 0) or x[v] S / 256 (s = 1), S the token's scale, for q = qp + 2s,
+    // l = 16 lh + 4 ((k + t') mod 4) + {0, 2 | 1, 3}, v = 128h + 32q + l (h,
+    // lh of quarter t').  X[tok][block][t'][qp][s] = the sum over the 16 l of
+    // those binary16 operands times 2^-19 (s = 0) or 2^-15 (s = 1): 32 2^-24
+    // and 32 16 2^-24, the code offset in the MMA's units.
+    static __device__ void build(const SP& p, uint32_t sb, const uint32_t* xmax, int64_t xoff) {
         const int per_tok = p.nblk * 16 * 4;
         for (int e = threadIdx.x; e < p.m * per_tok; e += kCW * 32) {
             const int tok = e / per_tok, rem = e % per_tok;
             const int blk = rem >> 6, E = (rem >> 2) & 15, tt = rem & 3;
             const int h = tt >> 1, lh = tt & 1, qp = E >> 3, sl = (E >> 2) & 1, kk = E & 3;
             const int q = qp + 2 * sl;
-            const float sc = sl ? 0.00390625f : 0.0625f;
+            const float sc = tok_scale(xmax, tok, kXT) * (sl ? 0.00390625f : 0.0625f);
             const int64_t v0 = static_cast<int64_t>(blk) * 256 + 128 * h + 32 * q + 16 * lh + 4 * ((kk + tt) & 3);
             const uint2 xr = lds64(xaddr(p, sb, tok, v0));
             const float xf[4] = {bf16lo_to_f32(xr.x), bf16hi_to_f32(xr.x), bf16lo_to_f32(xr.y), bf16hi_to_f32(xr.y)};
             __half hv[4];
 #pragma unroll
-            for (int b = 0; b < 4; ++b) hv[b] = hx(xf[b] * sc, amax);
+            for (int b = 0; b < 4; ++b) hv[b] = hx(xf[b], sc);
             sts64(sb + p.off_img + tok * p.img_tok + blk * kBlkImg + E * 32 + tt * 8, hpair(hv[0], hv[2]),
                   hpair(hv[1], hv[3]));
         }
@@ -479,6 +508,7 @@ struct Q6 {
             const int blk = rem >> 4, tt = (rem >> 2) & 3, qp = (rem >> 1) & 1, sl = rem & 1;
             const int h = tt >> 1, lh = tt & 1, q = qp + 2 * sl;
             const uint32_t xs = xaddr(p, sb, tok, blk * 256 + 128 * h + 32 * q + 16 * lh);
+            const float sc = tok_scale(xmax, tok, kXT) * (sl ? 0.00390625f : 0.0625f);
             float X = 0.f;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
@@ -486,10 +516,11 @@ struct Q6 {
                 const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    X += __half2float(__float2half_rn(bf16lo_to_f32(wv[u])));
-                    X += __half2float(__float2half_rn(bf16hi_to_f32(wv[u])));
+                    X += __half2float(hx(bf16lo_to_f32(wv[u]), sc));
+                    X += __half2float(hx(bf16hi_to_f32(wv[u]), sc));
                 }
             }
+            X *= sl ? 3.0517578125e-05f : 1.9073486328125e-06f;   // 2^-15, 2^-19
             sts32(sb + p.off_xs + tok * p.xs_tok + (blk * 16 + tt * 4 + qp * 2 + sl) * 4, __float_as_uint(X));
         }
     }
@@ -505,6 +536,11 @@ struct Q4 {
     static constexpr uint32_t kBlkImg = 544;
     static constexpr uint32_t kZero = kBlkImg;
     static constexpr int kAccPerLane = 4 * NT;
+    // scaled activations below 2^10: a sub-block sum X_j (32 values) stays
+    // below 2^15, inside the binary16 range of its two-part split
+    static constexpr int kXT = 9;
+    // acc[4 nt + e]: token 8 nt + 2t + (e & 1), row g + 8 (e >> 1)
+    static __device__ __forceinline__ int acc_tok(const Lane& L, int i) { return 8 * (i >> 2) + 2 * L.t + (i & 1); }
 
     static __device__ __forceinline__ void item(const SP& p, uint32_t sb, const Lane& L, uint32_t rowA,
                                                 uint32_t rowB, int gb, float (&acc)[4 * NT]) {
@@ -602,13 +638,14 @@ struct Q4 {
             }
     }
 
-    // Image per block and token: MMA (nib, u) of lane t uses values
-    // v = 64t + 32nib + 4u + {0,2 | 1,3}; the last 32 bytes hold (Xhi, Xlo)
-    // of sub-blocks 2t and 2t+1.
-    static __device__ void build(const SP& p, uint32_t sb, float& amax, int64_t xoff) {
+    // Image per block and token: MMA (nib, u) of lane t uses the scaled
+    // values v = 64t + 32nib + 4u + {0,2 | 1,3}; the last 32 bytes hold (Xhi,
+    // Xlo) of sub-blocks 2t and 2t+1, the sums of their binary16 operands.
+    static __device__ void build(const SP& p, uint32_t sb, const uint32_t* xmax, int64_t xoff) {
         const int items = p.m * p.nblk * 4;
         for (int it = threadIdx.x; it < items; it += kCW * 32) {
             const int tok = it / (p.nblk * 4), rem = it % (p.nblk * 4), bl = rem >> 2, t = rem & 3;
+            const float S = tok_scale(xmax, tok, kXT);
             const uint32_t base = sb + p.off_img + tok * p.img_tok + bl * kBlkImg;
             const int64_t xi = static_cast<int64_t>(bl) * 256 + 64 * t;
             const uint32_t xs = xaddr(p, sb, tok, xi);
@@ -625,9 +662,9 @@ struct Q4 {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const int u = 4 * uu + q;
-                        const __half f0 = hx(bf16lo_to_f32(wv[2 * q]), amax), f1 = hx(bf16hi_to_f32(wv[2 * q]), amax);
-                        const __half f2 = hx(bf16lo_to_f32(wv[2 * q + 1]), amax);
-                        const __half f3 = hx(bf16hi_to_f32(wv[2 * q + 1]), amax);
+                        const __half f0 = hx(bf16lo_to_f32(wv[2 * q]), S), f1 = hx(bf16hi_to_f32(wv[2 * q]), S);
+                        const __half f2 = hx(bf16lo_to_f32(wv[2 * q + 1]), S);
+                        const __half f3 = hx(bf16hi_to_f32(wv[2 * q + 1]), S);
                         X[nib] += (__half2float(f0) + __half2float(f1)) + (__half2float(f2) + __half2float(f3));
                         sts64(base + (nib * 8 + u) * 32 + t * 8, hpair(f0, f2), hpair(f1, f3));
                     }
@@ -741,6 +778,36 @@ __device__ bool gather_setup(const SPG& p, uint8_t* smem, int64_t& r0, int64_t& 
     return true;
 }
 
+// Largest |x| of every token of this CTA's activation slice, as bf16 bit
+// patterns, by atomic max into xmax[tok] (zeroed beforehand).  All consumer
+// warps take part: 16 / m warps per token, each lane loading up to eight
+// 16-byte chunks before it reduces, so the loads overlap.
+__device__ void x_range(const SP& p, uint32_t sb, int64_t xoff, uint32_t* xmax) {
+    constexpr int U = 8;
+    const int chunks = static_cast<int>(p.k / 8);   // 16-byte chunks per token
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wpt = p.m < kCW ? kCW / p.m : 1;      // warps per token
+    const int tok = warp / wpt, slot = warp % wpt;
+    if (tok >= p.m) return;   // warp-uniform
+    uint32_t mx = 0;
+    for (int c0 = slot * 32 * U; c0 < chunks; c0 += wpt * 32 * U) {
+        uint4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int c = c0 + 32 * u + lane;
+            if (c < chunks)
+                v[u] = p.x_global ? ldg_nc_v4(p.x + static_cast<int64_t>(tok) * p.k * p.ks + xoff + 8 * c)
+                                  : lds128(xaddr(p, sb, tok, 8 * c));
+            else
+                v[u] = make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) mx = absmax8_bf16(mx, v[u]);
+    }
+    mx = __reduce_max_sync(0xffffffffu, max(mx & 0xFFFFu, mx >> 16));
+    if (lane == 0 && mx) atomicMax(&xmax[tok], mx);
+}
+
 // act(g) * u of the GLU epilogue, in fp32: silu(g) = g / (1 + e^-g); gelu in
 // its tanh form 0.5 g (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3))); silu with
 // limit: silu(min(g, L)) * clamp(u, -L, L).
@@ -791,7 +858,9 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
         *abort_flag = 0;
         fence_barrier_init();
     }
+    uint32_t* xmax = reinterpret_cast<uint32_t*>(smem + kXMax);   // [16]
     if (tid < kMaxGroups) grp_done[tid] = 0;
+    if (tid < 16) xmax[tid] = 0;
     __syncthreads();
     // Programmatic dependent launch: the next kernel may start its prologue;
     // this one waits for the earlier grids before it reads x or W.  (Asking L2
@@ -830,7 +899,10 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
                 }
             }
         }
-        int q = 0;
+        // ring position: stage q goes to slot q mod ns, whose previous fill
+        // (phase parity ^ 1) must have been released first
+        int q = 0, slot = 0;
+        uint32_t phase = 0;
         bool ok = true;
         for (int rg = 0; rg < nlg && ok; ++rg) {
             const int gi = GLU ? rg >> 1 : rg;
@@ -838,8 +910,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
             const int rv = static_cast<int>(r1 - row0 < kRows ? r1 - row0 : kRows);
             const uint8_t* wsrc = (GLU && (rg & 1)) ? wbase2 : wbase;
             for (int st = 0; st < p.spr; ++st, ++q) {
-                const int slot = q % p.ns;
-                if (lane == 0 && q >= p.ns) ok = sleep_wait(&empty[slot], ((q / p.ns) & 1) ^ 1, p.status);
+                if (lane == 0 && q >= p.ns) ok = sleep_wait(&empty[slot], phase ^ 1, p.status);
                 ok = __shfl_sync(0xffffffffu, ok, 0) && !*abort_flag;
                 if (!ok) {
                     *abort_flag = 1;
@@ -854,6 +925,10 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
                     bulk_g2s(smem + p.off_stage + slot * stage_bytes + lane * p.rs,
                              wsrc + (row0 + lane) * p.row_bytes + (kb0 + b0) * C::kBPB, bytes,
                              &full[slot]);
+                if (++slot == p.ns) {
+                    slot = 0;
+                    phase ^= 1;
+                }
             }
         }
         // after an abort, let the copies in flight land before the CTA exits
@@ -867,17 +942,26 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
         Lane L;
         L.g = lane >> 2;
         L.t = lane & 3;
-        float amax = 0.f;
         if (!spin_wait(xbar, 0, p.status)) *abort_flag = 1;
+        // the tokens' activation scales, then the image
+        if (!*abort_flag) x_range(p, sb, kb0 * C::kVPB, xmax);
+        asm volatile("bar.sync 1, %0;" ::"r"(kCW * 32) : "memory");
+        // inverse scale of each token, applied to the partial sums before
+        // they leave the warp
+        const float* xinv = reinterpret_cast<const float*>(smem + kXInv);
+        if (tid < p.m) {
+            if (xmax[tid] >= 0x7F80u) atomicOr(p.status, KQ_DEV_X_RANGE);   // Inf or NaN
+            reinterpret_cast<float*>(smem + kXInv)[tid] = exp2_int(-xscale_exp(xmax[tid], C::kXT));
+        }
         if (!*abort_flag) {
-            C::build(p, sb, amax, kb0 * C::kVPB);
+            C::build(p, sb, xmax, kb0 * C::kVPB);
             for (uint32_t o = 4 * tid; o < C::kZero; o += 4 * kCW * 32) sts32(sb + p.off_zero + o, 0u);
         }
-        if (amax >= 65504.0f) atomicOr(p.status, KQ_DEV_X_RANGE);
         asm volatile("bar.sync 1, %0;" ::"r"(kCW * 32) : "memory");   // image ready (x copy now dead)
         float* part = reinterpret_cast<float*>(smem + p.off_part);
         const int items_per_row = p.nblk / C::kItemBlocks;
-        int q = 0;
+        int slot = 0;   // ring slot and fill parity of the next stage
+        uint32_t phase = 0;
         for (int rg = 0; rg < nlg && !*abort_flag; ++rg) {
             const int gi = GLU ? rg >> 1 : rg;
             const int64_t row0 = r0 + static_cast<int64_t>(group_order(gi, nrg, r1 - r0)) * kRows;
@@ -887,17 +971,16 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
             for (int i = 0; i < C::kAccPerLane; ++i) acc[i] = 0.f;
             // items of the row group, round robin over warps across stages
             bool ok = true;
-            for (int st = 0; st < p.spr; ++st, ++q) {
-                const int slot = q % p.ns;
+            for (int st = 0; st < p.spr; ++st) {
                 const int i0 = st * p.g / C::kItemBlocks;
                 const int i1 = min(items_per_row, (st + 1) * p.g / C::kItemBlocks);
                 // items continue the round robin of the previous row groups, so
                 // that rows with fewer items than warps still spread over all
                 const int rot = SPLIT ? rg * items_per_row : 0;
-                const int first = i0 + ((warp - i0 - rot) % kCW + kCW) % kCW;
+                const int first = i0 + ((warp - i0 - rot) & (kCW - 1));
                 // every warp waits for the stage, items or not, so that its
                 // release below always belongs to this fill of the slot
-                if (!spin_wait(&full[slot], (q / p.ns) & 1, p.status)) {
+                if (!spin_wait(&full[slot], phase, p.status)) {
                     *abort_flag = 1;
                     ok = false;
                 } else {
@@ -910,6 +993,10 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[slot]);
+                if (++slot == p.ns) {
+                    slot = 0;
+                    phase ^= 1;
+                }
                 if (!ok) break;
             }
             if (!ok) break;
@@ -928,6 +1015,11 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
                 }
             }
             float* pw = part + (pslot * kCW + warp) * kRows * p.m;
+#pragma unroll
+            for (int i = 0; i < C::kAccPerLane; ++i) {
+                const int tok = C::acc_tok(L, i);
+                acc[i] *= xinv[tok < p.m ? tok : p.m - 1];
+            }
             C::store_part(p, L, acc, pw);
             __threadfence_block();
             __syncwarp();

@@ -22,10 +22,13 @@
  *    (bindings.cpp docstring: "uint8 K-quant wire bytes (laid out [N, K] when
  *    transpose=True)") and of the README's "x @ dequant(w).T".
  *  - Activations x are bfloat16 [m, k] row-major (passed as uint16_t bit
- *    patterns).  The decode kernels of q4_K, q6_K and q8_0 (kq_qmv,
- *    kq_gather_qmv, kq_moe_glu_gather) convert them to binary16, so |x| must
- *    stay below 65504 there (KQ_DEV_X_RANGE flags it); qmm/gather use bf16 as
- *    is, and the q5_K / q4_0 qmv widens it to fp32 exactly.
+ *    patterns), any finite value.  The decode kernels of q4_K, q6_K and q8_0
+ *    (kq_qmv, kq_gather_qmv, kq_moe_glu_gather) scale each activation row by
+ *    a power of two taken from its largest magnitude, round it to binary16
+ *    and apply the inverse scale to the fp32 sums, so their relative error
+ *    does not depend on the magnitude of x; a non-finite activation sets
+ *    KQ_DEV_X_RANGE (its outputs are then NaN or infinite).  qmm/gather use
+ *    bf16 as is, and the q5_K / q4_0 qmv widens it to fp32 exactly.
  *  - Outputs y are fp32 [m, n] row-major.
  *  - Return value: a kq_status.  A non-zero status means nothing was enqueued
  *    (argument errors) or that the CUDA launch failed (KQ_ERR_CUDA; the
@@ -77,7 +80,7 @@ typedef enum {
 #define KQ_DEV_UNSORTED     0x8   /* expert ids not ascending                  */
 #define KQ_DEV_TIMEOUT      0x10  /* a bounded pipeline wait ran out            */
 #define KQ_DEV_TOO_MANY     0x20  /* more tiles for one expert than supported   */
-#define KQ_DEV_X_RANGE      0x40  /* an activation is outside the binary16 range */
+#define KQ_DEV_X_RANGE      0x40  /* an activation is infinite or NaN         */
 
 /* Block geometry of a codec (host only).  Returns KQ_OK or
  * KQ_ERR_UNSUPPORTED.  Source: mlx-kquant README, "Codec reference" table. */
@@ -134,8 +137,9 @@ int kq_quantize(int type, const float* w, int64_t n_rows, int64_t k, void* out, 
  * kernel (`verify_qmv`).  Every weight byte is read once for all m rows.
  *   w [n, row_bytes], x [m, k] bf16, y [m, n] fp32.
  * Arithmetic: quantization codes and integer scale products are exact in the
- * tensor-core operands, activations are rounded to binary16, accumulation is
- * fp32.  Results are deterministic (no atomics).
+ * tensor-core operands, activations (scaled by a power of two per row) are
+ * rounded to binary16, accumulation is fp32.  Results are deterministic (no
+ * atomics).
  * m outside 1..16 -> KQ_ERR_INVALID_ARG.
  */
 int kq_qmv(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int64_t m,

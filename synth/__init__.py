@@ -80,6 +80,26 @@ def activations(m: int, k: int, seed: int = SEED_X) -> np.ndarray:
     return f32_to_bf16_bits(rng(seed).standard_normal((m, k), dtype=np.float32))
 
 
+def activations_scaled(scales, k: int, seed: int = SEED_X) -> np.ndarray:
+    """bf16 activations [len(scales), k] as uint16 bits, row i drawn from
+    N(0, scales[i]^2): rows of very different magnitude in one batch."""
+    g = rng(seed)
+    rows = [np.float32(sc) * g.standard_normal(k, dtype=np.float32) for sc in scales]
+    return f32_to_bf16_bits(np.stack(rows))
+
+
+def activations_outliers(m: int, k: int, small: float, big: float, per_row: int,
+                         seed: int = SEED_X) -> np.ndarray:
+    """bf16 activations [m, k] as uint16 bits: N(0, small^2) values with
+    `per_row` entries per row replaced by +-big at seeded positions."""
+    g = rng(seed)
+    x = np.float32(small) * g.standard_normal((m, k), dtype=np.float32)
+    for i in range(m):
+        pos = g.choice(k, per_row, replace=False)
+        x[i, pos] = np.float32(big) * np.where(g.random(per_row) < 0.5, -1.0, 1.0).astype(np.float32)
+    return f32_to_bf16_bits(x)
+
+
 def routing(tokens: int, n_experts: int, top_k: int, seed: int = SEED_ROUTE) -> np.ndarray:
     """int32 [tokens, top_k]: the first top_k entries of a seeded permutation
     of 0..n_experts-1 per token (distinct experts, uniformly at random)."""
