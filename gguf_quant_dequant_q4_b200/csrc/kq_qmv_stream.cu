@@ -110,8 +110,6 @@ struct SPGLU : SPG {
 };
 constexpr uint32_t kGList = 512;     // gather: pair list of the CTA (16 ints)
 constexpr uint32_t kGMisc = 576;     // gather: expert, pairs present, row range
-constexpr uint32_t kXMax = 640;      // largest |x| per token (bf16 bits, 16 words)
-constexpr uint32_t kXInv = 704;      // inverse activation scale per token (16 floats)
 constexpr uint32_t kGCount = 1024;   // gather: pairs per expert (256 ints)
 constexpr uint32_t kGHdr = 2048;     // gather header size
 
@@ -146,6 +144,9 @@ __device__ __forceinline__ uint32_t vhfma2(uint32_t a, uint32_t b, uint32_t c) {
 }
 __device__ __forceinline__ void sts64(uint32_t a, uint32_t x, uint32_t y) {
     asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(x), "r"(y));
+}
+__device__ __forceinline__ void sts8(uint32_t a, uint32_t x) {
+    asm volatile("st.shared.u8 [%0], %1;" ::"r"(a), "r"(x));
 }
 __device__ __forceinline__ void sts32(uint32_t a, uint32_t x) {
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(x));
@@ -198,12 +199,8 @@ __device__ __forceinline__ uint32_t xaddr(const SP& p, uint32_t sb, int tok, int
 __device__ __forceinline__ float xval(const SP& p, uint32_t sb, int tok, int64_t i) {
     return __uint_as_float(lds_u16(xaddr(p, sb, tok, i)) << 16);
 }
-// Binary16 of an activation times its token's power-of-two scale.
+// Binary16 of an activation times its power-of-two scale.
 __device__ __forceinline__ __half hx(float v, float scale) { return __float2half_rn(v * scale); }
-// Scale 2^s of token `tok` (see xscale_exp) for a codec with target exponent T.
-__device__ __forceinline__ float tok_scale(const uint32_t* xmax, int tok, int T) {
-    return exp2_int(xscale_exp(xmax[tok], T));
-}
 __device__ __forceinline__ uint32_t hpair(__half lo, __half hi) {
     return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
 }
@@ -224,11 +221,10 @@ struct Q8 {
     static constexpr uint32_t kItemImg = 17 * 32;   // image bytes per item (8 blocks) and token
     static constexpr uint32_t kZero = kItemImg;
     static constexpr int kAccPerLane = 2 * NT;
-    // scaled activations below 2^15: the 1152 + code operands and the
-    // 32-value sums X stay far inside fp32 and binary16 range
+    // a block's scaled activations stay below 2^15: far inside binary16
     static constexpr int kXT = 14;
-    // token of accumulator i (acc[2 nt + r]: token nt, row g + 8 r)
-    static __device__ __forceinline__ int acc_tok(const Lane&, int i) { return i >> 1; }
+    // the build needs every block's scale before it writes the image
+    static constexpr bool kTwoPhase = true;
 
     // rowA/rowB: shared address of the item (8 blocks) in rows g / g+8;
     // gi: global item index (block 8 gi).
@@ -276,17 +272,19 @@ struct Q8 {
                 mma_f16(D[nt][mu & 1], A0, A1, A2, A3, bv.x, bv.y);
             }
         }
-        // D = 2^-24 sum (128 + code) a;  y += 2^24 d (D - 2^-17 X), X = sum a,
-        // for columns 2t (even block) and 2t+1 (odd block)
+        // D = 2^-24 sum (128 + code) a with a = x 2^s (s per token and block);
+        // y += 2^(24-s) d (D - 2^-17 X), X = sum a, for columns 2t (even
+        // block) and 2t+1 (odd block)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            const uint2 xv = lds64(sb + p.off_xs + nt * p.xs_tok + 4 * (8 * gi + 2 * t));
+            const uint4 xv = lds128(sb + p.off_xs + nt * p.xs_tok + 16 * (4 * gi + t));
             const float X[2] = {__uint_as_float(xv.x), __uint_as_float(xv.y)};
+            const float iv[2] = {__uint_as_float(xv.z), __uint_as_float(xv.w)};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int r = e >> 1, odd = e & 1;
                 const float Ds = D[nt][0][e] + D[nt][1][e];
-                acc[2 * nt + r] = fmaf(odd ? dO[r] : dE[r], Ds - X[odd], acc[2 * nt + r]);
+                acc[2 * nt + r] = fmaf((odd ? dO[r] : dE[r]) * iv[odd], Ds - X[odd], acc[2 * nt + r]);
             }
         }
     }
@@ -304,44 +302,67 @@ struct Q8 {
             }
     }
 
-    // Image entry (item, mu, t') = binary16 of the scaled activations of the 4
-    // raw bytes at offset 272 item + 68 t' + 4 mu of a row, as (byte0, byte2 |
-    // byte1, byte3); scale bytes get 0.  X[tok][block] = 2^-17 (= 128 2^-24)
-    // times the sum of the block's 32 binary16 operands.
-    static __device__ void build(const SP& p, uint32_t sb, const uint32_t* xmax, int64_t xoff) {
-        const int items = p.nblk / 8;
-        const int per_tok = items * 17 * 4;
-        for (int e = threadIdx.x; e < p.m * per_tok; e += kCW * 32) {
-            const int tok = e / per_tok, rem = e % per_tok;
-            const int it = rem / 68, mu = (rem % 68) >> 2, tt = rem & 3;
-            const int R0 = it * 272 + 68 * tt + 4 * mu;
-            const float S = tok_scale(xmax, tok, kXT);
-            __half h[4];
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const int R = R0 + b, blk = R / 34, o = R - 34 * blk;
-                h[b] = o >= 2 ? hx(xval(p, sb, tok, 32 * blk + o - 2), S) : __float2half_rn(0.f);
-            }
-            sts64(sb + p.off_img + tok * p.img_tok + it * kItemImg + mu * 32 + tt * 8, hpair(h[0], h[2]),
-                  hpair(h[1], h[3]));
-        }
+    // Phase 1, one thread per (token, block): the block's scale 2^s from its
+    // largest |x|, then X = 2^-17 (= 128 2^-24) times the sum of the block's
+    // 32 binary16 operands and 2^-s, stored as {X_even, X_odd, 2^-s_even,
+    // 2^-s_odd} per block pair.  Returns whether this thread met a
+    // non-finite activation.
+    static __device__ bool build_scales(const SP& p, uint32_t sb, int64_t xoff) {
+        bool bad = false;
         for (int e = threadIdx.x; e < p.m * p.nblk; e += kCW * 32) {
             const int tok = e / p.nblk, blk = e % p.nblk;
             const uint32_t xs = xaddr(p, sb, tok, 32 * blk);
-            const float S = tok_scale(xmax, tok, kXT);
+            uint4 v[4];
+            uint32_t mx = 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                v[c] = lds128(xs + 16 * c);
+                mx = absmax8_bf16(mx, v[c]);
+            }
+            mx = max(mx & 0xFFFFu, mx >> 16);
+            bad |= mx >= 0x7F80u;
+            const int se = xscale_exp(mx, kXT);
+            const float S = exp2_int(se);
             float X = 0.f;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const uint4 v = lds128(xs + 16 * c);
-                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+                const uint32_t wv[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     X += __half2float(hx(bf16lo_to_f32(wv[q]), S));
                     X += __half2float(hx(bf16hi_to_f32(wv[q]), S));
                 }
             }
-            sts32(sb + p.off_xs + tok * p.xs_tok + 4 * blk, __float_as_uint(X * 7.62939453125e-06f));
+            const uint32_t xo = sb + p.off_xs + tok * p.xs_tok + 16 * (blk >> 1) + 4 * (blk & 1);
+            sts32(xo, __float_as_uint(X * 7.62939453125e-06f));
+            sts32(xo + 8, __float_as_uint(exp2_int(-se)));
         }
+        return bad;
+    }
+    // Phase 2: image entry (item, mu, t') = binary16 of the scaled activations
+    // of the 4 raw bytes at offset 272 item + 68 t' + 4 mu of a row, as
+    // (byte0, byte2 | byte1, byte3); scale bytes get 0.  A block's 2^s is read
+    // back from its stored 2^-s (powers of two: the bit patterns of 2^k and
+    // 2^-k add up to 254 << 23).
+    static __device__ bool build(const SP& p, uint32_t sb, int64_t xoff) {
+        const int items = p.nblk / 8;
+        const int per_tok = items * 17 * 4;
+        for (int e = threadIdx.x; e < p.m * per_tok; e += kCW * 32) {
+            const int tok = e / per_tok, rem = e % per_tok;
+            const int it = rem / 68, mu = (rem % 68) >> 2, tt = rem & 3;
+            const int R0 = it * 272 + 68 * tt + 4 * mu;
+            __half h[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int R = R0 + b, blk = R / 34, o = R - 34 * blk;
+                const uint32_t ib = lds32(sb + p.off_xs + tok * p.xs_tok + 16 * (blk >> 1) + 4 * (blk & 1) + 8);
+                const float S = __uint_as_float(0x7F000000u - ib);
+                h[b] = o >= 2 ? hx(xval(p, sb, tok, 32 * blk + o - 2), S) : __float2half_rn(0.f);
+            }
+            sts64(sb + p.off_img + tok * p.img_tok + it * kItemImg + mu * 32 + tt * 8, hpair(h[0], h[2]),
+                  hpair(h[1], h[3]));
+        }
+        return false;
     }
 };
 
@@ -362,10 +383,10 @@ struct Q6 {
     static constexpr uint32_t kBlkImg = 512;   // image bytes per block and token
     static constexpr uint32_t kZero = 512;
     static constexpr int kAccPerLane = 2 * NT;
-    // scaled activations below 2^15: the x/16 and x/256 operands stay normal
-    // binary16 numbers down to 2^-22 of the token's largest magnitude
+    // a run's scaled activations below 2^15: its x/16 and x/256 operands stay
+    // normal binary16 numbers down to 2^-22 of the run's largest magnitude
     static constexpr int kXT = 14;
-    static __device__ __forceinline__ int acc_tok(const Lane&, int i) { return i >> 1; }
+    static constexpr bool kTwoPhase = false;
 
     // Word at shared address a (2-byte aligned when ODD).
     template <bool ODD>
@@ -451,19 +472,22 @@ struct Q6 {
                     mma_f16(D[k & 1][nt], H0, H1, H2, H3, bh.x, bh.y);
                 }
             }
-            // column 2t: D = 2^-24 sum c a with a = x/16, column 2t + 1:
-            // D = 2^-24 sum 16 c a with a = x/256; both are 2^-24 sum c x / 16,
-            // and sum (c - 32) x = 16 2^24 (D - X) with X the stored offset sum
-            // (2^-19 sum a, resp. 2^-15 sum a): y += 2^28 d sc_j (D - X)
+            // column 2t: D = 2^-24 sum c a with a = x 2^s/16, column 2t + 1:
+            // D = 2^-24 sum 16 c a with a = x 2^s/256 (s per 16-value run);
+            // both are 2^-24 2^s sum c x / 16, and sum (c - 32) x =
+            // 16 2^24 2^-s (D - X) with X the stored offset sum (2^-19 sum a,
+            // resp. 2^-15 sum a): y += 2^28 d sc_j 2^-s (D - X)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                const uint2 xv = lds64(sb + p.off_xs + nt * p.xs_tok + ((gb * 4 + t) * 4 + 2 * qp) * 4);
+                const uint4 xv = lds128(sb + p.off_xs + nt * p.xs_tok + ((gb * 4 + t) * 2 + qp) * 16);
                 const float X[2] = {__uint_as_float(xv.x), __uint_as_float(xv.y)};
+                const float iv[2] = {__uint_as_float(xv.z), __uint_as_float(xv.w)};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int r = e >> 1, c = e & 1;
                     const float Ds = D[0][nt][e] + D[1][nt][e];
-                    acc[2 * nt + r] = fmaf(__fmul_rn(d16[r], sc[r][qp + 2 * c]), Ds - X[c], acc[2 * nt + r]);
+                    acc[2 * nt + r] =
+                        fmaf(__fmul_rn(d16[r], sc[r][qp + 2 * c]) * iv[c], Ds - X[c], acc[2 * nt + r]);
                 }
             }
         }
@@ -479,50 +503,49 @@ struct Q6 {
         Q8<NT>::store_part(p, L, acc, part);
     }
 
-    // Image entry (block, E = 8 qp + 4 s + k, t'): binary16 of x[v] S / 16
-    // (s = 0) or x[v] S / 256 (s = 1), S the token's scale, for q = qp + 2s,
-    // l = 16 lh + 4 ((k + t') mod 4) + {0, 2 | 1, 3}, v = 128h + 32q + l (h,
-    // lh of quarter t').  X[tok][block][t'][qp][s] = the sum over the 16 l of
-    // those binary16 operands times 2^-19 (s = 0) or 2^-15 (s = 1): 32 2^-24
-    // and 32 16 2^-24, the code offset in the MMA's units.
-    static __device__ void build(const SP& p, uint32_t sb, const uint32_t* xmax, int64_t xoff) {
-        const int per_tok = p.nblk * 16 * 4;
+    // One thread per 16-value run (token, block, quarter t' = (h, lh), qp,
+    // s): q = qp + 2s, values v = 128h + 32q + 16 lh + l, l = 0..15.  Its
+    // scale 2^e puts the run's largest |x| at 2^14; image entry (block,
+    // E = 8 qp + 4 s + k, t') = binary16 of x[v] 2^e / 16 (s = 0) or / 256
+    // (s = 1) for l = 4 ((k + t') mod 4) + {0, 2 | 1, 3}; the run's
+    // {X_s=0, X_s=1, 2^-e_s=0, 2^-e_s=1} per (block, t', qp), X = the sum of
+    // the 16 binary16 operands times 2^-19 (s = 0) or 2^-15 (s = 1): 32 2^-24
+    // and 32 16 2^-24, the code offset in the MMA's units.  Returns whether
+    // this thread met a non-finite activation.
+    static __device__ bool build(const SP& p, uint32_t sb, int64_t xoff) {
+        bool bad = false;
+        const int per_tok = p.nblk * 16;
         for (int e = threadIdx.x; e < p.m * per_tok; e += kCW * 32) {
             const int tok = e / per_tok, rem = e % per_tok;
-            const int blk = rem >> 6, E = (rem >> 2) & 15, tt = rem & 3;
-            const int h = tt >> 1, lh = tt & 1, qp = E >> 3, sl = (E >> 2) & 1, kk = E & 3;
-            const int q = qp + 2 * sl;
-            const float sc = tok_scale(xmax, tok, kXT) * (sl ? 0.00390625f : 0.0625f);
-            const int64_t v0 = static_cast<int64_t>(blk) * 256 + 128 * h + 32 * q + 16 * lh + 4 * ((kk + tt) & 3);
-            const uint2 xr = lds64(xaddr(p, sb, tok, v0));
-            const float xf[4] = {bf16lo_to_f32(xr.x), bf16hi_to_f32(xr.x), bf16lo_to_f32(xr.y), bf16hi_to_f32(xr.y)};
-            __half hv[4];
-#pragma unroll
-            for (int b = 0; b < 4; ++b) hv[b] = hx(xf[b], sc);
-            sts64(sb + p.off_img + tok * p.img_tok + blk * kBlkImg + E * 32 + tt * 8, hpair(hv[0], hv[2]),
-                  hpair(hv[1], hv[3]));
-        }
-        const int per_tok_x = p.nblk * 16;
-        for (int e = threadIdx.x; e < p.m * per_tok_x; e += kCW * 32) {
-            const int tok = e / per_tok_x, rem = e % per_tok_x;
             const int blk = rem >> 4, tt = (rem >> 2) & 3, qp = (rem >> 1) & 1, sl = rem & 1;
             const int h = tt >> 1, lh = tt & 1, q = qp + 2 * sl;
             const uint32_t xs = xaddr(p, sb, tok, blk * 256 + 128 * h + 32 * q + 16 * lh);
-            const float sc = tok_scale(xmax, tok, kXT) * (sl ? 0.00390625f : 0.0625f);
+            const uint4 v0 = lds128(xs), v1 = lds128(xs + 16);
+            uint32_t mx = absmax8_bf16(0u, v0);
+            mx = absmax8_bf16(mx, v1);
+            mx = max(mx & 0xFFFFu, mx >> 16);
+            bad |= mx >= 0x7F80u;
+            const int se = xscale_exp(mx, kXT);
+            const float sc = exp2_int(se) * (sl ? 0.00390625f : 0.0625f);
+            const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            __half hv[16];
             float X = 0.f;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const uint4 v = lds128(xs + 16 * c);
-                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    X += __half2float(hx(bf16lo_to_f32(wv[u]), sc));
-                    X += __half2float(hx(bf16hi_to_f32(wv[u]), sc));
-                }
+            for (int u = 0; u < 8; ++u) {
+                hv[2 * u] = hx(bf16lo_to_f32(wv[u]), sc);
+                hv[2 * u + 1] = hx(bf16hi_to_f32(wv[u]), sc);
+                X += __half2float(hv[2 * u]) + __half2float(hv[2 * u + 1]);
             }
-            X *= sl ? 3.0517578125e-05f : 1.9073486328125e-06f;   // 2^-15, 2^-19
-            sts32(sb + p.off_xs + tok * p.xs_tok + (blk * 16 + tt * 4 + qp * 2 + sl) * 4, __float_as_uint(X));
+            const uint32_t img = sb + p.off_img + tok * p.img_tok + blk * kBlkImg + (8 * qp + 4 * sl) * 32 + tt * 8;
+            // values 4g .. 4g+3 go to entry k = (g - t') mod 4
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+                sts64(img + ((g - tt) & 3) * 32, hpair(hv[4 * g], hv[4 * g + 2]), hpair(hv[4 * g + 1], hv[4 * g + 3]));
+            const uint32_t xo = sb + p.off_xs + tok * p.xs_tok + ((blk * 4 + tt) * 2 + qp) * 16 + 4 * sl;
+            sts32(xo, __float_as_uint(X * (sl ? 3.0517578125e-05f : 1.9073486328125e-06f)));   // 2^-15, 2^-19
+            sts32(xo + 8, __float_as_uint(exp2_int(-se)));
         }
+        return bad;
     }
 };
 
@@ -536,11 +559,10 @@ struct Q4 {
     static constexpr uint32_t kBlkImg = 544;
     static constexpr uint32_t kZero = kBlkImg;
     static constexpr int kAccPerLane = 4 * NT;
-    // scaled activations below 2^10: a sub-block sum X_j (32 values) stays
-    // below 2^15, inside the binary16 range of its two-part split
+    // a block's scaled activations below 2^10: a sub-block sum X_j (32
+    // values) stays below 2^15, inside the binary16 range of its two-part split
     static constexpr int kXT = 9;
-    // acc[4 nt + e]: token 8 nt + 2t + (e & 1), row g + 8 (e >> 1)
-    static __device__ __forceinline__ int acc_tok(const Lane& L, int i) { return 8 * (i >> 2) + 2 * L.t + (i & 1); }
+    static constexpr bool kTwoPhase = false;
 
     static __device__ __forceinline__ void item(const SP& p, uint32_t sb, const Lane& L, uint32_t rowA,
                                                 uint32_t rowB, int gb, float (&acc)[4 * NT]) {
@@ -584,9 +606,12 @@ struct Q4 {
         }
         const uint32_t wA[8] = {qA0.x, qA0.y, qA0.z, qA0.w, qA1.x, qA1.y, qA1.z, qA1.w};
         const uint32_t wB[8] = {qB0.x, qB0.y, qB0.z, qB0.w, qB1.x, qB1.y, qB1.z, qB1.w};
-        float D[4][NT][4], Dm[NT][4];
+        // independent MMA chains: four for one n-tile, two per n-tile for two
+        // (the same MMAs in flight, fewer accumulator registers)
+        constexpr int CH = NT == 1 ? 4 : 2;
+        float D[CH][NT][4], Dm[NT][4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < CH; ++c)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -608,22 +633,28 @@ struct Q4 {
             for (int nt = 0; nt < NT; ++nt) {
                 const uint2 bl = lds64(bb[nt] + u * 32);
                 const uint2 bh = lds64(bb[nt] + (8 + u) * 32);
-                mma_f16(D[u & 3][nt], a0, a1, a2, a3, bl.x, bl.y);
-                mma_f16(D[u & 3][nt], c0, c1, c2, c3, bh.x, bh.y);
+                mma_f16(D[u % CH][nt], a0, a1, a2, a3, bl.x, bl.y);
+                mma_f16(D[u % CH][nt], c0, c1, c2, c3, bh.x, bh.y);
             }
         }
-        // y += d D - dmin sum_j m_j X_j
+        // y += 2^-s (d D - dmin sum_j m_j X_j), 2^-s of this block for the
+        // column's token: tokens 2t, 2t + 1 of the n-tile, one 2-byte load
+        // from the [block][16 tokens] table of biased exponents 127 - s
+        // (entries past m are never stored)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const uint2 bv = lds64(bb[nt] + 512);
+            const uint32_t eb = lds_u16(sb + p.off_xs + 16 * gb + 8 * nt + 2 * t);
+            const float iv[2] = {__uint_as_float((eb & 0xFFu) << 23), __uint_as_float((eb >> 8) << 23)};
 #pragma unroll
             for (int e = 0; e < 4; ++e) Dm[nt][e] = 0.f;
             mma_f16(Dm[nt], M_lo[0], M_lo[1], M_hi[0], M_hi[1], bv.x, bv.y);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int r = e >> 1;
-                const float Ds = (D[0][nt][e] + D[1][nt][e]) + (D[2][nt][e] + D[3][nt][e]);
-                acc[4 * nt + e] = fmaf(dd[r], Ds, fmaf(-dm[r], Dm[nt][e], acc[4 * nt + e]));
+                float Ds = D[0][nt][e] + D[1][nt][e];
+                if constexpr (CH == 4) Ds = (D[0][nt][e] + D[1][nt][e]) + (D[2][nt][e] + D[3][nt][e]);
+                acc[4 * nt + e] = fmaf(iv[e & 1], fmaf(dd[r], Ds, -dm[r] * Dm[nt][e]), acc[4 * nt + e]);
             }
         }
     }
@@ -641,23 +672,41 @@ struct Q4 {
     // Image per block and token: MMA (nib, u) of lane t uses the scaled
     // values v = 64t + 32nib + 4u + {0,2 | 1,3}; the last 32 bytes hold (Xhi,
     // Xlo) of sub-blocks 2t and 2t+1, the sums of their binary16 operands.
-    static __device__ void build(const SP& p, uint32_t sb, const uint32_t* xmax, int64_t xoff) {
-        const int items = p.m * p.nblk * 4;
+    // One thread per 64 values (token, block, t); the four threads of a block
+    // are neighbouring lanes and agree on the block's scale 2^s (largest |x|
+    // at 2^9) by two shuffles; 127 - s (the biased exponent of 2^-s) goes to
+    // the [block][16 tokens] byte table.
+    // Returns whether this thread met a non-finite activation.
+    static __device__ bool build(const SP& p, uint32_t sb, int64_t xoff) {
+        bool bad = false;
+        const int items = p.m * p.nblk * 4;   // a multiple of 4: a block's lanes are all in or all out
         for (int it = threadIdx.x; it < items; it += kCW * 32) {
             const int tok = it / (p.nblk * 4), rem = it % (p.nblk * 4), bl = rem >> 2, t = rem & 3;
-            const float S = tok_scale(xmax, tok, kXT);
             const uint32_t base = sb + p.off_img + tok * p.img_tok + bl * kBlkImg;
             const int64_t xi = static_cast<int64_t>(bl) * 256 + 64 * t;
             const uint32_t xs = xaddr(p, sb, tok, xi);
             const uint16_t* xg = p.x + static_cast<int64_t>(tok) * p.k * p.ks + xoff + xi;
+            uint4 r[8];
+            uint32_t mx = 0;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                r[c] = p.x_global ? ldg_nc_v4(xg + 8 * c) : lds128(xs + 16 * c);
+                mx = absmax8_bf16(mx, r[c]);
+            }
+            mx = max(mx & 0xFFFFu, mx >> 16);
+            const unsigned grp = __activemask();
+            mx = max(mx, __shfl_xor_sync(grp, mx, 1));
+            mx = max(mx, __shfl_xor_sync(grp, mx, 2));
+            bad |= mx >= 0x7F80u;
+            const int se = xscale_exp(mx, kXT);
+            const float S = exp2_int(se);
+            if (t == 0) sts8(sb + p.off_xs + 16 * bl + tok, static_cast<uint32_t>(127 - se));
             float X[2] = {0.f, 0.f};
 #pragma unroll
             for (int nib = 0; nib < 2; ++nib) {
 #pragma unroll
                 for (int uu = 0; uu < 2; ++uu) {
-                    const int o = 32 * nib + 16 * uu;
-                    const uint4 r0 = p.x_global ? ldg_nc_v4(xg + o) : lds128(xs + 2 * o);
-                    const uint4 r1 = p.x_global ? ldg_nc_v4(xg + o + 8) : lds128(xs + 2 * (o + 8));
+                    const uint4 r0 = r[4 * nib + 2 * uu], r1 = r[4 * nib + 2 * uu + 1];
                     const uint32_t wv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
@@ -679,6 +728,7 @@ struct Q4 {
             }
             sts64(base + 512 + t * 8, e[0], e[1]);
         }
+        return bad;
     }
 };
 
@@ -778,36 +828,6 @@ __device__ bool gather_setup(const SPG& p, uint8_t* smem, int64_t& r0, int64_t& 
     return true;
 }
 
-// Largest |x| of every token of this CTA's activation slice, as bf16 bit
-// patterns, by atomic max into xmax[tok] (zeroed beforehand).  All consumer
-// warps take part: 16 / m warps per token, each lane loading up to eight
-// 16-byte chunks before it reduces, so the loads overlap.
-__device__ void x_range(const SP& p, uint32_t sb, int64_t xoff, uint32_t* xmax) {
-    constexpr int U = 8;
-    const int chunks = static_cast<int>(p.k / 8);   // 16-byte chunks per token
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int wpt = p.m < kCW ? kCW / p.m : 1;      // warps per token
-    const int tok = warp / wpt, slot = warp % wpt;
-    if (tok >= p.m) return;   // warp-uniform
-    uint32_t mx = 0;
-    for (int c0 = slot * 32 * U; c0 < chunks; c0 += wpt * 32 * U) {
-        uint4 v[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int c = c0 + 32 * u + lane;
-            if (c < chunks)
-                v[u] = p.x_global ? ldg_nc_v4(p.x + static_cast<int64_t>(tok) * p.k * p.ks + xoff + 8 * c)
-                                  : lds128(xaddr(p, sb, tok, 8 * c));
-            else
-                v[u] = make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) mx = absmax8_bf16(mx, v[u]);
-    }
-    mx = __reduce_max_sync(0xffffffffu, max(mx & 0xFFFFu, mx >> 16));
-    if (lane == 0 && mx) atomicMax(&xmax[tok], mx);
-}
-
 // act(g) * u of the GLU epilogue, in fp32: silu(g) = g / (1 + e^-g); gelu in
 // its tanh form 0.5 g (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3))); silu with
 // limit: silu(min(g, L)) * clamp(u, -L, L).
@@ -858,9 +878,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
         *abort_flag = 0;
         fence_barrier_init();
     }
-    uint32_t* xmax = reinterpret_cast<uint32_t*>(smem + kXMax);   // [16]
     if (tid < kMaxGroups) grp_done[tid] = 0;
-    if (tid < 16) xmax[tid] = 0;
     __syncthreads();
     // Programmatic dependent launch: the next kernel may start its prologue;
     // this one waits for the earlier grids before it reads x or W.  (Asking L2
@@ -943,20 +961,18 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
         L.g = lane >> 2;
         L.t = lane & 3;
         if (!spin_wait(xbar, 0, p.status)) *abort_flag = 1;
-        // the tokens' activation scales, then the image
-        if (!*abort_flag) x_range(p, sb, kb0 * C::kVPB, xmax);
-        asm volatile("bar.sync 1, %0;" ::"r"(kCW * 32) : "memory");
-        // inverse scale of each token, applied to the partial sums before
-        // they leave the warp
-        const float* xinv = reinterpret_cast<const float*>(smem + kXInv);
-        if (tid < p.m) {
-            if (xmax[tid] >= 0x7F80u) atomicOr(p.status, KQ_DEV_X_RANGE);   // Inf or NaN
-            reinterpret_cast<float*>(smem + kXInv)[tid] = exp2_int(-xscale_exp(xmax[tid], C::kXT));
+        // the activation image with its per-block scales (q8_0: the scales
+        // first, the image entries of a block read them)
+        bool bad = false;
+        if constexpr (C::kTwoPhase) {
+            if (!*abort_flag) bad = C::build_scales(p, sb, kb0 * C::kVPB);
+            asm volatile("bar.sync 1, %0;" ::"r"(kCW * 32) : "memory");
         }
         if (!*abort_flag) {
-            C::build(p, sb, xmax, kb0 * C::kVPB);
+            bad |= C::build(p, sb, kb0 * C::kVPB);
             for (uint32_t o = 4 * tid; o < C::kZero; o += 4 * kCW * 32) sts32(sb + p.off_zero + o, 0u);
         }
+        if (bad) atomicOr(p.status, KQ_DEV_X_RANGE);   // an activation is Inf or NaN
         asm volatile("bar.sync 1, %0;" ::"r"(kCW * 32) : "memory");   // image ready (x copy now dead)
         float* part = reinterpret_cast<float*>(smem + p.off_part);
         const int items_per_row = p.nblk / C::kItemBlocks;
@@ -1015,11 +1031,6 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
                 }
             }
             float* pw = part + (pslot * kCW + warp) * kRows * p.m;
-#pragma unroll
-            for (int i = 0; i < C::kAccPerLane; ++i) {
-                const int tok = C::acc_tok(L, i);
-                acc[i] *= xinv[tok < p.m ? tok : p.m - 1];
-            }
             C::store_part(p, L, acc, pw);
             __threadfence_block();
             __syncwarp();
@@ -1309,6 +1320,10 @@ int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m,
     return record_cuda(cudaLaunchKernelEx(&cfg, kernel, p));
 }
 
+// q4_K keeps its inverse scales in one [block][16 tokens] byte table in the
+// per-token X region: the per-token stride that makes m of them hold it.
+uint32_t q4_inv_tok(int nblk, int m) { return align16(static_cast<uint32_t>(cdiv(nblk * 16, m))); }
+
 }  // namespace
 
 // Staged qmv for the shapes it covers; KQ_ERR_UNSUPPORTED otherwise (the
@@ -1319,13 +1334,13 @@ int launch_qmv_stream(int type, const void* w, int64_t n, int64_t k, const uint1
     case KQ_Q8_0: {
         const int nblk = static_cast<int>(k / 32);
         if (m > 2 || nblk % 8 != 0) return KQ_ERR_UNSUPPORTED;
-        const uint32_t it = (nblk / 8) * Q8<1>::kItemImg, xt = nblk * 4;
+        const uint32_t it = (nblk / 8) * Q8<1>::kItemImg, xt = nblk * 8;
         return m == 1 ? launch_stream<Q8<1>>(w, n, k, x, m, y, s, it, xt) : launch_stream<Q8<2>>(w, n, k, x, m, y, s, it, xt);
     }
     case KQ_Q6_K: {
         const int nblk = static_cast<int>(k / 256);
         if (m > 2 || nblk % 8 != 0) return KQ_ERR_UNSUPPORTED;
-        const uint32_t it = nblk * Q6<1>::kBlkImg, xt = nblk * 16 * 4;
+        const uint32_t it = nblk * Q6<1>::kBlkImg, xt = nblk * 32 * 4;
         return m == 1 ? launch_stream<Q6<1>>(w, n, k, x, m, y, s, it, xt) : launch_stream<Q6<2>>(w, n, k, x, m, y, s, it, xt);
     }
     case KQ_Q4_K: {
@@ -1345,8 +1360,8 @@ int launch_qmv_stream(int type, const void* w, int64_t n, int64_t k, const uint1
             // tokens of an MMA's B fragment then read disjoint banks
             uint32_t it = (nblk / ks) * Q4<1>::kBlkImg;
             it += (32u - it % 128u + 128u) % 128u;
-            const int rc = m <= 8 ? launch_stream<Q4<1>>(w, n, k, x, m, y, s, it, 0, ks)
-                                  : launch_stream<Q4<2>>(w, n, k, x, m, y, s, it, 0, ks);
+            const int rc = m <= 8 ? launch_stream<Q4<1>>(w, n, k, x, m, y, s, it, q4_inv_tok(nblk / ks, m), ks)
+                                  : launch_stream<Q4<2>>(w, n, k, x, m, y, s, it, q4_inv_tok(nblk / ks, m), ks);
             if (rc != KQ_ERR_UNSUPPORTED || ks == 1) return rc;
             ks = 1;
         }
@@ -1367,14 +1382,14 @@ int launch_gather_qmv(int type, const void* w_bank, const void* w_bank2, int act
     switch (type) {
     case KQ_Q8_0: {
         if (nblk % 8 != 0) return KQ_ERR_UNSUPPORTED;
-        const uint32_t it = (nblk / 8) * Q8<1>::kItemImg, xt = nblk * 4;
+        const uint32_t it = (nblk / 8) * Q8<1>::kItemImg, xt = nblk * 8;
         rc = m_cap >= 2 ? launch_stream<Q8<2>>(w_bank, n, k, x, 2, y, s, it, xt, 1, &ga) : KQ_ERR_UNSUPPORTED;
         if (rc == KQ_ERR_UNSUPPORTED) rc = launch_stream<Q8<1>>(w_bank, n, k, x, 1, y, s, it, xt, 1, &ga);
         return rc;
     }
     case KQ_Q6_K: {
         if (nblk % 8 != 0) return KQ_ERR_UNSUPPORTED;
-        const uint32_t it = nblk * Q6<1>::kBlkImg, xt = nblk * 16 * 4;
+        const uint32_t it = nblk * Q6<1>::kBlkImg, xt = nblk * 32 * 4;
         rc = m_cap >= 2 ? launch_stream<Q6<2>>(w_bank, n, k, x, 2, y, s, it, xt, 1, &ga) : KQ_ERR_UNSUPPORTED;
         if (rc == KQ_ERR_UNSUPPORTED) rc = launch_stream<Q6<1>>(w_bank, n, k, x, 1, y, s, it, xt, 1, &ga);
         return rc;
@@ -1383,8 +1398,8 @@ int launch_gather_qmv(int type, const void* w_bank, const void* w_bank2, int act
         uint32_t it = nblk * Q4<1>::kBlkImg;
         it += (32u - it % 128u + 128u) % 128u;
         for (int m = m_cap < 16 ? m_cap : 16; m >= 1; --m) {
-            rc = m <= 8 ? launch_stream<Q4<1>>(w_bank, n, k, x, m, y, s, it, 0, 1, &ga)
-                        : launch_stream<Q4<2>>(w_bank, n, k, x, m, y, s, it, 0, 1, &ga);
+            rc = m <= 8 ? launch_stream<Q4<1>>(w_bank, n, k, x, m, y, s, it, q4_inv_tok(nblk, m), 1, &ga)
+                        : launch_stream<Q4<2>>(w_bank, n, k, x, m, y, s, it, q4_inv_tok(nblk, m), 1, &ga);
             if (rc != KQ_ERR_UNSUPPORTED) return rc;
         }
         return rc;
