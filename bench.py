@@ -539,6 +539,94 @@ def cpu_sample(seconds: float = 10.0) -> dict:
             "cpu": _cpu_model()}
 
 
+def cpu_baseline_configs(min_seconds: float = 0.3) -> dict:
+    """The oracle's fp32 product (as it stands) on every configuration, once on
+    one host thread and once on all host cores; c0-c2 in full, c3 / c4 on a
+    fixed subset of activation rows with the per-call time extrapolated by
+    the row ratio (labelled).  About 15 s of CPU work."""
+    import oracle
+    out = {}
+
+    def timed(fn):
+        n, t0 = 0, time.perf_counter()
+        while True:
+            fn()
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= min_seconds:
+                return el / n
+
+    def both(fn):
+        res = {}
+        for label, t in (("1_thread", 1), ("all_cores", 0)):
+            oracle.set_threads(t)
+            res[label] = (timed(fn), oracle.threads())
+        oracle.set_threads(0)
+        return res
+
+    def gbs_entry(nbytes, fn, note=None):
+        r = both(fn)
+        e = {f"{lab}_GB/s": round(nbytes / t / 1e9, 3) for lab, (t, _) in r.items()}
+        e["cores"] = r["all_cores"][1]
+        if note:
+            e["sample"] = note
+        return e
+
+    # c0: q4_K qmv 4096 x 4096, M = 1, and its full dequantize to fp32
+    w = synth.weights(Q4_K, 4096, 4096)
+    x = synth.activations(1, 4096)
+    out["c0_qmv_q4K_m1_4096x4096"] = gbs_entry(w.nbytes, lambda: oracle.matmul_f32(Q4_K, w, 4096, x))
+    out["c0_dequantize_q4K_4096x4096_fp32"] = gbs_entry(w.nbytes + 4096 * 4096 * 4,
+                                                        lambda: oracle.dequantize(Q4_K, w, 4096))
+    # c1: q8_0 + q6_K qmv 14336 x 4096, M = 1
+    w8, w6 = synth.weights(Q8_0, 14336, 4096), synth.weights(Q6_K, 14336, 4096)
+    x = synth.activations(1, 4096)
+    out["c1_qmv_q8_0_q6K_m1_14336x4096"] = gbs_entry(
+        w8.nbytes + w6.nbytes, lambda: (oracle.matmul_f32(Q8_0, w8, 4096, x), oracle.matmul_f32(Q6_K, w6, 4096, x)))
+    del w8, w6
+    # c2: q4_K qmv 4096 x 14336, M in {1, 4, 8, 16}
+    w = synth.weights(Q4_K, 4096, 14336)
+    xa = synth.activations(16, 14336)
+    for m in (1, 4, 8, 16):
+        xm = xa[:m]
+        out[f"c2_qmv_q4K_m{m}_4096x14336"] = gbs_entry(w.nbytes, lambda: oracle.matmul_f32(Q4_K, w, 14336, xm))
+    # c3: qmm 2048 x 14336 x 4096 (q4_K, q6_K): 32 of the 2048 activation rows
+    sub = 32
+    xs = synth.activations(2048, 4096)[:sub]
+    for qt, nm in ((Q4_K, "q4K"), (Q6_K, "q6K")):
+        w = synth.weights(qt, 14336, 4096)
+        r = both(lambda: oracle.matmul_f32(qt, w, 4096, xs))
+        e = {}
+        for lab, (t, _) in r.items():
+            full = t * 2048 / sub
+            e[f"{lab}_TFLOP/s"] = round(2 * 2048 * 14336 * 4096 / full / 1e12, 6)
+            e[f"{lab}_extrapolated_ms_per_call"] = round(full * 1e3, 1)
+        e["cores"] = r["all_cores"][1]
+        e["sample"] = f"{sub} of 2048 activation rows, per-call time extrapolated x{2048 // sub}"
+        out[f"c3_qmm_{nm}_2048x14336x4096"] = e
+    del w
+    # c4: gather q4_K, 8 experts x 14336 x 4096, 512 tokens top-2 (1024 rows):
+    # every expert's first 4 sorted rows (32 of 1024)
+    e_, tok, topk = 8, 512, 2
+    wb = synth.weights(Q4_K, 14336, 4096, experts=e_)
+    ids = synth.routing(tok, e_, topk)
+    srt, pair = oracle.moe_sort(ids, e_)
+    xt = synth.activations(tok, 4096)
+    per = 4
+    groups = [(ex, xt[pair[srt == ex][:per] // topk]) for ex in range(e_) if np.any(srt == ex)]
+    rows = sum(g[1].shape[0] for g in groups)
+    r = both(lambda: [oracle.matmul_f32(Q4_K, wb[ex], 4096, xg) for ex, xg in groups])
+    e = {}
+    for lab, (t, _) in r.items():
+        full = t * (tok * topk) / rows
+        e[f"{lab}_TFLOP/s"] = round(2 * tok * topk * 14336 * 4096 / full / 1e12, 6)
+        e[f"{lab}_extrapolated_ms_per_call"] = round(full * 1e3, 1)
+    e["cores"] = r["all_cores"][1]
+    e["sample"] = f"{rows} of {tok * topk} sorted rows ({per} per expert), per-call time extrapolated"
+    out["c4_gather_qmm_q4K_8x14336x4096_t512_top2"] = e
+    return out
+
+
 def _cpu_model() -> str:
     try:
         for line in open("/proc/cpuinfo"):
@@ -675,7 +763,8 @@ def main(argv=None):
         dist.init("nccl")
         res = run_kq(args, dist)
         if res is not None and dist.rank == 0 and not args.no_cpu:
-            res["cpu_baseline"] = cpu_sample(10.0)
+            res["cpu_baseline"] = cpu_sample(5.0)
+            res["cpu_baseline"]["configs"] = cpu_baseline_configs()
     if dist.rank == 0 and res is not None:
         print(json.dumps(res), flush=True)
     dist.close()

@@ -84,6 +84,7 @@ def _load():
         lib.oracle_matmul_f64.argtypes = [ctypes.c_int, ip, i64, i64, ip, i64, ip, ip]
         lib.oracle_matmul_f32.argtypes = [ctypes.c_int, ip, i64, i64, ip, i64, ip]
         lib.oracle_threads.restype = ctypes.c_int
+        lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_quantize.argtypes = [ctypes.c_int, ip, i64, i64, ip]
         lib.oracle_float_to_half.argtypes = [ip, i64, ip]
         _lib = lib
@@ -103,6 +104,11 @@ def block_info(qtype: int) -> tuple[int, int]:
 
 def threads() -> int:
     return _load().oracle_threads()
+
+
+def set_threads(n: int) -> None:
+    """Thread count of the parallel loops (0: all host cores)."""
+    _load().oracle_set_threads(int(n))
 
 
 def _check_w(qtype: int, w: np.ndarray, k: int) -> np.ndarray:

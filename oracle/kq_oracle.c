@@ -294,6 +294,18 @@ int oracle_matmul_f32(int type, const uint8_t* w, int64_t n, int64_t k, const ui
     return fail ? -2 : 0;
 }
 
+/* Thread count of the parallel loops (the timed baseline runs once on one
+ * thread and once on all host cores); n <= 0 restores the default. */
+void oracle_set_threads(int n) {
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    extern int omp_get_num_procs(void);
+    omp_set_num_threads(n > 0 ? n : omp_get_num_procs());
+#else
+    (void)n;
+#endif
+}
+
 /* Number of OpenMP threads the parallel loops above use. */
 int oracle_threads(void) {
     int t = 1;
