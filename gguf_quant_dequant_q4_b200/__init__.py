@@ -37,6 +37,7 @@ SIGNATURES = {
     "kq_status_string": (ctypes.c_char_p, [_int]),
     "kq_last_cuda_error": (_int, []),
     "kq_read_device_status": (_int, [ctypes.POINTER(_i32), _int]),
+    "kq_set_wait_limit": (_int, [_i64]),
     "kq_dequantize": (_int, [_int, _vp, _i64, _i64, _vp, _vp]),
     "kq_quantize": (_int, [_int, _vp, _i64, _i64, _vp, _vp]),
     "kq_qmv": (_int, [_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp]),
@@ -114,6 +115,12 @@ def read_device_status(clear: bool = False) -> int:
     v = _i32()
     _check(lib().kq_read_device_status(ctypes.byref(v), int(clear)), "kq_read_device_status")
     return v.value
+
+
+def set_wait_limit(ns: int = 0) -> None:
+    """Time limit (ns) of the staged decode kernel's pipeline waits; 0 restores
+    the default (2 s).  For fault-handling tests."""
+    _check(lib().kq_set_wait_limit(int(ns)), "kq_set_wait_limit")
 
 
 def _bf16_bits(x: torch.Tensor) -> torch.Tensor:

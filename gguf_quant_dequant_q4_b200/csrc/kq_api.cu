@@ -136,7 +136,12 @@ int kq_read_device_status(int32_t* host_status, int clear) {
     if (!host_status) return KQ_ERR_INVALID_ARG;
     int* p = device_status_ptr();
     if (!p) return KQ_ERR_CUDA;
-    int rc = record_cuda(cudaMemcpy(host_status, p, sizeof(int32_t), cudaMemcpyDeviceToHost));
+    // every stream of the device, blocking or not, has finished its kernels
+    // before the word is read (a plain copy would order with the legacy
+    // default stream only)
+    int rc = record_cuda(cudaDeviceSynchronize());
+    if (rc) return rc;
+    rc = record_cuda(cudaMemcpy(host_status, p, sizeof(int32_t), cudaMemcpyDeviceToHost));
     if (rc) return rc;
     if (clear) {
         const int32_t zero = 0;
@@ -144,6 +149,8 @@ int kq_read_device_status(int32_t* host_status, int clear) {
     }
     return rc;
 }
+
+int kq_set_wait_limit(int64_t ns) { return set_stream_wait_limit(ns > 0 ? static_cast<uint64_t>(ns) : 0); }
 
 int kq_dequantize(int type, const void* w, int64_t n_rows, int64_t k, float* out, void* stream) {
     int rc = check_weights(type, w, n_rows, k);

@@ -38,6 +38,9 @@ int launch_qmv_stream(int type, const void* w, int64_t n, int64_t k, const uint1
 int launch_gather_qmv(int type, const void* w_bank, const void* w_bank2, int act, float limit, int n_experts,
                       int64_t n, int64_t k, const uint16_t* x, int xdiv, const int32_t* ids, int pairs, int m_cap,
                       float* y, int32_t* err_flag, cudaStream_t s);
+// Pipeline wait limit (ns; 0 = the default) of the staged decode kernel on
+// the current device.
+int set_stream_wait_limit(uint64_t ns);
 // q5_K / q4_0 decode product: exact fp32 decode and fp32 dot (k % 256 == 0).
 int launch_qmv_exact(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int m, float* y,
                      cudaStream_t s);

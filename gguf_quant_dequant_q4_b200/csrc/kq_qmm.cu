@@ -45,7 +45,7 @@ constexpr int kThreads = (7 + kDecWarps) * 32;
 constexpr int kBM = 128;          // weight rows per tile (MMA M)
 constexpr int kBN = 256;          // activation rows per tile (MMA N max)
 constexpr int kBK = 64;           // K per pipeline step (one 128-byte swizzle row)
-constexpr int kMaxTiles = 1024;   // map tiles a gather call may use
+constexpr int kMaxTiles = 1024;   // map tiles one gather launch takes (a window of the map)
 constexpr uint32_t kHeader = 5120; // barriers, misc words, tile tables
 constexpr int kDeqWarp0 = 6;   // warps 0..5: producer, MMA, 4 epilogue
 constexpr int kRawWarp = kDeqWarp0 + kDecWarps;   // the raw weight producer
@@ -87,6 +87,7 @@ struct QmmParams {
     const uint32_t* map;
     const uint32_t* count;
     int64_t cap;
+    int64_t win0;         // gather: first map tile of this launch's window of kMaxTiles
     float* y;
     int32_t* err;         // caller's flag (gather) or library status
     int* status;
@@ -645,27 +646,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (p.n_experts == 0) {
         total_units = p.units;
     } else {
-        // Gather: validate the map, keep valid tiles, order them by
-        // (expert, row_start) and cut each expert's list into chunks of 4.
+        // Gather: this launch takes the window [win0, win0 + kMaxTiles) of
+        // the map's first `count` tiles (a larger map is served by further
+        // launches).  Validate the window, keep its valid tiles, group them by
+        // expert in map order and cut each expert's list into chunks of 4.
         // Both CTAs of a pair build the same tables.
-        int cnt = static_cast<int>(*p.count);
-        if (cnt > p.cap || cnt < 0) {
-            if (tid == 0 && p.err) atomicOr(p.err, KQ_DEV_BAD_RANGE);
-            cnt = cnt < 0 ? 0 : static_cast<int>(p.cap);
+        int64_t cnt = static_cast<int64_t>(*p.count);
+        if (cnt > p.cap) {
+            if (tid == 0 && p.win0 == 0 && p.err) atomicOr(p.err, KQ_DEV_BAD_RANGE);
+            cnt = p.cap;
         }
-        if (cnt > kMaxTiles) {
-            if (tid == 0 && p.err) atomicOr(p.err, KQ_DEV_TOO_MANY);
-            cnt = kMaxTiles;
-        }
+        const int wn = static_cast<int>(cnt - p.win0 < 0 ? 0 : (cnt - p.win0 < kMaxTiles ? cnt - p.win0 : kMaxTiles));
+        const uint32_t* wmap_t = p.map + 3 * p.win0;   // the window's tiles
         for (int e = tid; e < 257; e += kThreads) cstart[e] = tstart[e] = 0;
         __syncthreads();
         // validity and per-expert counts
-        for (int i = tid; i < cnt; i += kThreads) {
-            const uint32_t e = p.map[3 * i], rs = p.map[3 * i + 1], nr = p.map[3 * i + 2];
+        auto tile_ok = [&](int i, uint32_t& e) {
+            e = wmap_t[3 * i];
+            const uint32_t rs = wmap_t[3 * i + 1], nr = wmap_t[3 * i + 2];
             int bad = 0;
             if (e >= static_cast<uint32_t>(p.n_experts)) bad |= KQ_DEV_BAD_EXPERT;
             if (nr == 0 || nr > 64) bad |= KQ_DEV_BAD_ROWS;
             if (static_cast<int64_t>(rs) + nr > p.m) bad |= KQ_DEV_BAD_RANGE;
+            return bad;
+        };
+        for (int i = tid; i < wn; i += kThreads) {
+            uint32_t e;
+            const int bad = tile_ok(i, e);
             if (bad) {
                 if (p.err) atomicOr(p.err, bad);
             } else {
@@ -673,32 +680,49 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncthreads();
+        // first slot of every expert's list (tstart), and a running fill
+        // pointer per expert (cstart, turned into the chunk prefix below)
         if (tid == 0) {
-            int tacc = 0, cacc = 0;
+            int tacc = 0;
             for (int e = 0; e < p.n_experts; ++e) {
                 const int te = tstart[e + 1];
                 tstart[e] = tacc;
-                cstart[e] = cacc;
+                cstart[e] = tacc;
                 tacc += te;
-                cacc += (te + 3) / 4;
             }
             tstart[p.n_experts] = tacc;
-            cstart[p.n_experts] = cacc;
-            misc[2] = cacc;
         }
         __syncthreads();
-        // place: rank of a valid tile among the valid tiles of its expert by row_start
-        for (int i = tid; i < cnt; i += kThreads) {
-            const uint32_t e = p.map[3 * i], rs = p.map[3 * i + 1], nr = p.map[3 * i + 2];
-            if (e >= static_cast<uint32_t>(p.n_experts) || nr == 0 || nr > 64 || static_cast<int64_t>(rs) + nr > p.m)
-                continue;
-            int rk = 0;
-            for (int j = 0; j < cnt; ++j) {
-                const uint32_t e2 = p.map[3 * j], rs2 = p.map[3 * j + 1], nr2 = p.map[3 * j + 2];
-                const bool ok2 = e2 == e && nr2 != 0 && nr2 <= 64 && static_cast<int64_t>(rs2) + nr2 <= p.m;
-                if (ok2 && (rs2 < rs || (rs2 == rs && j < i))) ++rk;
+        // place: one warp walks the window in map order, 32 tiles at a time;
+        // a valid tile goes to its expert's next free slot (lanes of one
+        // expert in a step ranked among themselves), so each expert's list
+        // keeps map order, which is row order for kq_expert_tile_map's maps
+        if (warp == 0) {
+            for (int i0 = 0; i0 < wn; i0 += 32) {
+                const int i = i0 + lane;
+                uint32_t e = 0xFFFFFFFFu;
+                if (i < wn && tile_ok(i, e) != 0) e = 0xFFFFFFFFu;
+                const unsigned same = __match_any_sync(0xffffffffu, e);
+                const unsigned below = same & ((1u << lane) - 1u);
+                int pos = 0;
+                if (e != 0xFFFFFFFFu) pos = cstart[e] + __popc(below);
+                __syncwarp();
+                if (e != 0xFFFFFFFFu) {
+                    tiles[pos] = static_cast<uint16_t>(i);
+                    if (below == 0) cstart[e] += __popc(same);
+                }
+                __syncwarp();
             }
-            tiles[tstart[e] + rk] = static_cast<uint16_t>(i);
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int cacc = 0;
+            for (int e = 0; e < p.n_experts; ++e) {
+                cstart[e] = cacc;
+                cacc += (tstart[e + 1] - tstart[e] + 3) / 4;
+            }
+            cstart[p.n_experts] = cacc;
+            misc[2] = cacc;
         }
         total_units = 0;   // read after the barrier below
     }
@@ -760,8 +784,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 4; ++i) {
                 if (i < U.nt) {
                     const int ti = tiles[first + i];
-                    U.rs[i] = static_cast<int>(p.map[3 * ti + 1]);
-                    U.nr[i] = static_cast<int>(p.map[3 * ti + 2]);
+                    U.rs[i] = static_cast<int>(p.map[3 * (p.win0 + ti) + 1]);
+                    U.nr[i] = static_cast<int>(p.map[3 * (p.win0 + ti) + 2]);
                 } else {
                     U.rs[i] = 0;
                     U.nr[i] = 0;
@@ -1165,8 +1189,14 @@ int launch_cg(const CUtensorMap& wmap, const CUtensorMap& xmap, QmmParams p, cud
     cfg.stream = s;
     cfg.attrs = at;
     cfg.numAttrs = CG == 2 ? 1 : 0;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, wmap, xmap, p);
-    if (e != cudaSuccess) return record_cuda(e);
+    // gather: one launch per window of kMaxTiles map slots (the valid-tile
+    // count is on the device; a window past it has no units)
+    const int64_t windows = p.n_experts == 0 ? 1 : (p.cap + kMaxTiles - 1) / kMaxTiles;
+    for (int64_t w = 0; w < (windows > 0 ? windows : 1); ++w) {
+        p.win0 = w * kMaxTiles;
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, wmap, xmap, p);
+        if (e != cudaSuccess) return record_cuda(e);
+    }
     return check_launch();
 }
 

@@ -163,32 +163,49 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
 }
 __device__ __forceinline__ float h2f(uint32_t h) { return __half2float(__ushort_as_half(static_cast<unsigned short>(h))); }
 
+// Time limit of the pipeline waits of this kernel, per device (default
+// kWaitLimitNs; kq_set_wait_limit shortens it for fault-handling tests).  Read
+// only once a wait has not completed at its first poll.
+__device__ uint64_t g_wait_ns = kWaitLimitNs;
+__device__ __forceinline__ uint64_t wait_limit() { return *static_cast<volatile uint64_t*>(&g_wait_ns); }
+
 // Bounded spin on an mbarrier phase (no suspend hint: these waits are short
 // and a sleeping warp can wake up late).  False after the time limit, with
-// KQ_DEV_TIMEOUT recorded.
+// KQ_DEV_TIMEOUT recorded.  Under a limit shorter than the default (a test's)
+// the time is taken at every poll and a completion seen after the limit
+// counts as run out, so the first wait that is not complete at once runs out.
 __device__ __forceinline__ bool spin_wait(uint64_t* bar, uint32_t parity, int* status) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_ns();
+    const uint64_t t0 = global_ns(), limit = wait_limit();
+    const bool strict = limit < kWaitLimitNs;
     for (int i = 0;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255) == 255 && global_ns() - t0 > kWaitLimitNs) {
-            if (status) atomicOr(status, KQ_DEV_TIMEOUT);
-            return false;
+        const bool done = mbar_try_wait(bar, parity);
+        if (done && !strict) return true;
+        if (strict || (i & 255) == 255) {
+            if (global_ns() - t0 > limit) {
+                if (status) atomicOr(status, KQ_DEV_TIMEOUT);
+                return false;
+            }
+            if (done) return true;
         }
     }
 }
 
 // Bounded wait that lets the warp sleep until the phase completes (the
-// producer: it must not take issue slots from the decoding warps).
-__device__ __forceinline__ bool sleep_wait(uint64_t* bar, uint32_t parity, int* status) {
+// producer: it must not take issue slots from the decoding warps).  `limit`
+// is the time limit (the pipeline's, or kWaitLimitNs for the wind-down).
+__device__ __forceinline__ bool sleep_wait(uint64_t* bar, uint32_t parity, int* status, uint64_t limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
+    const bool strict = limit < kWaitLimitNs;   // as in spin_wait
     for (;;) {
-        if (mbar_try_wait_sleep(bar, parity)) return true;
-        if (global_ns() - t0 > kWaitLimitNs) {
+        const bool done = mbar_try_wait_sleep(bar, parity);
+        if (done && !strict) return true;
+        if (global_ns() - t0 > limit) {
             if (status) atomicOr(status, KQ_DEV_TIMEOUT);
             return false;
         }
+        if (done) return true;
     }
 }
 
@@ -928,7 +945,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
             const int rv = static_cast<int>(r1 - row0 < kRows ? r1 - row0 : kRows);
             const uint8_t* wsrc = (GLU && (rg & 1)) ? wbase2 : wbase;
             for (int st = 0; st < p.spr; ++st, ++q) {
-                if (lane == 0 && q >= p.ns) ok = sleep_wait(&empty[slot], phase ^ 1, p.status);
+                if (lane == 0 && q >= p.ns) ok = sleep_wait(&empty[slot], phase ^ 1, p.status, wait_limit());
                 ok = __shfl_sync(0xffffffffu, ok, 0) && !*abort_flag;
                 if (!ok) {
                     *abort_flag = 1;
@@ -949,11 +966,14 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
                 }
             }
         }
-        // after an abort, let the copies in flight land before the CTA exits
-        if (!ok && lane == 0) {
-            spin_wait(xbar, 0, nullptr);
+        // The copies this warp issued land before the CTA exits, also when a
+        // consumer gave up on a wait after the last stage was issued: the x
+        // copy and the latest fill of every slot (each slot's last phase, so
+        // a completed wait returns at once), with the full time limit.
+        if (lane == 0) {
+            sleep_wait(xbar, 0, nullptr, kWaitLimitNs);
             for (int qq = q - p.ns > 0 ? q - p.ns : 0; qq < q; ++qq)
-                spin_wait(&full[qq % p.ns], (qq / p.ns) & 1, nullptr);
+                sleep_wait(&full[qq % p.ns], (qq / p.ns) & 1, nullptr, kWaitLimitNs);
         }
     } else {
         // --------------------------------------------------------- consumers
@@ -1325,6 +1345,13 @@ int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m,
 uint32_t q4_inv_tok(int nblk, int m) { return align16(static_cast<uint32_t>(cdiv(nblk * 16, m))); }
 
 }  // namespace
+
+// Pipeline wait limit of the staged decode kernel on the current device
+// (ns == 0: the default).
+int set_stream_wait_limit(uint64_t ns) {
+    const uint64_t v = ns ? ns : kWaitLimitNs;
+    return record_cuda(cudaMemcpyToSymbol(g_wait_ns, &v, sizeof(v)));
+}
 
 // Staged qmv for the shapes it covers; KQ_ERR_UNSUPPORTED otherwise (the
 // caller then takes the general kernel).

@@ -79,7 +79,7 @@ typedef enum {
 #define KQ_DEV_BAD_RANGE    0x4   /* tile rows past `rows`, count > cap        */
 #define KQ_DEV_UNSORTED     0x8   /* expert ids not ascending                  */
 #define KQ_DEV_TIMEOUT      0x10  /* a bounded pipeline wait ran out            */
-#define KQ_DEV_TOO_MANY     0x20  /* more tiles for one expert than supported   */
+#define KQ_DEV_TOO_MANY     0x20  /* reserved: not set by this version         */
 #define KQ_DEV_X_RANGE      0x40  /* an activation is infinite or NaN         */
 
 /* Block geometry of a codec (host only).  Returns KQ_OK or
@@ -93,9 +93,25 @@ const char* kq_status_string(int status);
 int kq_last_cuda_error(void);
 
 /* Library-wide device status word: bits KQ_DEV_* set by kernels that have no
- * err_flag argument (kq_qmv, kq_qmm).  Host call, synchronous: it waits for
- * the device.  `clear` != 0 resets the word after reading. */
+ * err_flag argument (kq_qmv, kq_qmm).  Host call, synchronous: it first waits
+ * for all work on the current device (every stream, cudaDeviceSynchronize),
+ * then reads the word.  `clear` != 0 resets the word after reading.  The word
+ * is shared by every call and stream of the device: a bit cannot be traced to
+ * the call that set it. */
 int kq_read_device_status(int32_t* host_status, int clear);
+
+/*
+ * kq_set_wait_limit - time limit, in ns, of every pipeline wait of the staged
+ * decode kernel (kq_qmv at m <= 2 for q8_0 / q6_K and q4_K shapes it covers,
+ * kq_gather_qmv, kq_moe_glu_gather) on the current device; ns <= 0 restores
+ * the default of 2 s.  Host call, synchronous.  A wait that runs out sets
+ * KQ_DEV_TIMEOUT in the library status word and the kernel winds down
+ * (letting its own copies land) without finishing: its outputs are then
+ * incomplete.  A short limit exists so that fault-handling tests can make a
+ * wait run out on purpose; production code has no reason to call it.
+ * No counterpart on the pages (the failure handling of this library).
+ */
+int kq_set_wait_limit(int64_t ns);
 
 /*
  * kq_dequantize - decode wire bytes to fp32, bit-exactly (all five codecs).
@@ -202,7 +218,10 @@ int kq_expert_tile_map(const uint32_t* sorted_ids, int64_t rows, int32_t n_exper
  * and must cover every x row exactly once (uncovered output rows are left
  * unwritten)"; num_rows <= 64.  Each CTA owns one (expert, 128 weight rows)
  * pair and streams all of that expert's tiles through the tensor cores, so
- * each expert weight tile is decoded once per pass.
+ * each expert weight tile is decoded once per pass.  Any number of tiles:
+ * the map is taken in windows of 1024 slots, one kernel launch per window
+ * (ceil(cap / 1024) launches; a window past the device-side count has no
+ * work), and an expert's tiles are grouped in map order within a window.
  *   w_bank [n_experts, n, row_bytes], x_sorted [rows, k] bf16,
  *   map [cap, 3], count [1] (device), y [rows, n] fp32.
  *   err_flag (nullable): tiles with e >= n_experts (KQ_DEV_BAD_EXPERT),

@@ -143,3 +143,35 @@ def test_gather_row_runs_and_split_tiles(qtype):
     for ex, (lo, hi) in enumerate([(0, 202), (202, 207), (207, 300)]):
         r = np.array([i for i in range(lo, hi) if not 271 <= i < 280])
         check_qmm(y[r], ref[r], xn[r], row_norms_w(qtype, w[ex], k), k)
+
+
+@pytest.mark.parametrize("shuffle", [False, True])
+def test_gather_more_than_1024_tiles(shuffle):
+    # 70 000 sorted rows over 3 experts: 1096 map tiles, more than one launch
+    # window of 1024 map slots; the device-built map (grouped by expert, rows
+    # in order) and the same tiles shuffled; every row against the oracle, no
+    # flag raised
+    experts, n, k, rows = 3, 64, 256, 70000
+    ids = np.repeat(np.arange(experts), [30001, 25000, 14999]).astype(np.uint32)
+    if shuffle:
+        tiles = oracle.tile_map(ids, experts)
+        assert len(tiles) > 1024
+        tiles = [tiles[i] for i in np.random.default_rng(21).permutation(len(tiles))]
+        w, x, y, e = run_gather(kq.Q4_K, experts, n, k, tiles, rows, seed=20)
+    else:
+        w = synth.weights(kq.Q4_K, n, k, seed=20, experts=experts)
+        x = synth.activations(rows, k, seed=21)
+        m, c = kq.expert_tile_map(torch.from_numpy(ids.view(np.int32)).cuda(), experts)
+        tiles = tiles_of(m, c)
+        assert len(tiles) > 1024
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        out = torch.full((rows, n), float("nan"), device="cuda")
+        kq.gather_qmm(dev_bf16(x), dev_u8(w), kq.Q4_K, m, c, out=out, err=err)
+        y, e = out.cpu().numpy(), int(err.item())
+    assert e == 0
+    assert np.all(np.isfinite(y))
+    ref = oracle.gather_qmm(kq.Q4_K, w, k, x, tiles)
+    xn = row_norms_x(x)
+    for ex in range(experts):
+        r = np.nonzero(ids == ex)[0]
+        check_qmm(y[r], ref[r], xn[r], row_norms_w(kq.Q4_K, w[ex], k), k)
