@@ -451,6 +451,20 @@ def measure_rows(kq, torch, dev, pk, args) -> dict:
                                                "frac_bf16_sustained": round(tf / pk["bf16_tflops_sustained"], 4)}
         del Ws
     del y, xq
+    # q6_K qmm with rows that are not a 16-byte multiple (K = 11008: 9030-byte
+    # rows, the flat view of the weights), M = 2048, N = 14336
+    k6 = 11008
+    xq = bf(synth.activations(m, k6))
+    y = torch.empty(m, n, device=dev)
+    w = synth.weights(Q6_K, n, k6)
+    cp = ncopies(w.nbytes + m * k6 * 2)
+    Ws = [u8(w) for _ in range(cp)]
+    t = time_graph(torch, lambda i: kq.qmm(xq, Ws[i % cp], Q6_K, out=y), 8, s)
+    launches += 8 + 3
+    tf = 2 * m * n * k6 / (t / 1e3) / 1e12
+    rows["qmm_q6K_2048x14336x11008_unaligned_rows"] = {"kernel_us": round(t * 1e3, 2), "TFLOP/s": round(tf, 1),
+                                                       "frac_bf16": round(tf / pk["bf16_tflops"], 4)}
+    del Ws, y, xq
     # c4: MoE sort + tile map + gather, 8 experts x 14336 x 4096 q4_K, 512 tokens top-2
     e, n, k, tok, topk = 8, 14336, 4096, 512, 2
     wb = u8(synth.weights(Q4_K, n, k, experts=e))

@@ -88,6 +88,7 @@ struct QmmParams {
     const uint32_t* count;
     int64_t cap;
     int64_t win0;         // gather: first map tile of this launch's window of kMaxTiles
+    int64_t row_bytes;    // flat raw view (rows not a 16-byte multiple): bytes per weight row
     float* y;
     int32_t* err;         // caller's flag (gather) or library status
     int* status;
@@ -99,6 +100,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
             dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+// Rank-1 tiled load (the flat byte view of the weights); x a multiple of 16.
+__device__ __forceinline__ void tma_load_1d(uint32_t dst, const CUtensorMap* map, int x, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.1d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2}], [%3];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(smem_u32(bar))
         : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -371,6 +380,47 @@ __device__ __forceinline__ void q6k_step(uint32_t row, int q, int p, const Stage
     }
 }
 
+// The same q6_K step for a block at a run-time offset O (even, 0..14) of its
+// 16-byte aligned window, as in the flat raw view where every weight row has
+// its own offset: 16 bytes from five 4-byte loads joined by byte permutes
+// with a per-thread selector (no divergence between threads of one warp).
+__device__ __forceinline__ void lds16B_rt(uint32_t a, int O, uint32_t (&w)[4]) {
+    const uint32_t base = a + static_cast<uint32_t>(O & ~3);
+    const uint32_t sel = (O & 2) ? 0x5432u : 0x3210u;
+    uint32_t r[5];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) r[i] = lds32(base + 4 * i);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = __byte_perm(r[i], r[i + 1], sel);
+}
+__device__ __forceinline__ void q6k_scales_rt(uint32_t row, int O, int p, StageScales& S) {
+    const float d = h16v(ldsu16(row + O + 208));
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int h = q >> 1, tq = 2 * (q & 1) + (p >> 1);
+        int16_t scv;
+        asm volatile("ld.shared.s8 %0, [%1];" : "=h"(scv) : "r"(row + O + 192 + 8 * h + 2 * tq + (p & 1)));
+        split_scale(__fmul_rn(d, static_cast<float>(scv)), S.hi[q], S.lo[q]);
+    }
+}
+__device__ __forceinline__ void q6k_step_rt(uint32_t row, int O, int q, int p, const StageScales& S,
+                                            uint32_t (&o)[8]) {
+    const int h = q >> 1, tq = 2 * (q & 1) + (p >> 1), sb = p & 1;
+    uint32_t QL[4], QH[4];
+    lds16B_rt(row + 64 * h + 32 * (tq & 1) + 16 * sb, O, QL);
+    lds16B_rt(row + 128 + 32 * h + 16 * sb, O, QH);
+    const int lsh = 4 * (tq >> 1), hsh = 2 * tq;
+    const uint32_t hi = S.hi[q], lo = S.lo[q];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t c4 = ((QL[i] >> lsh) & 0x0F0F0F0Fu) | (((QH[i] >> hsh) & 0x03030303u) << 4);
+        const uint32_t v01 = bsub2(__byte_perm(c4, kMagic, 0x5140), kB160);   // code - 32, exact
+        const uint32_t v23 = bsub2(__byte_perm(c4, kMagic, 0x7362), kB160);
+        o[2 * i] = bfma2(v01, hi, bmul2(v01, lo));
+        o[2 * i + 1] = bfma2(v23, hi, bmul2(v23, lo));
+    }
+}
+
 // q5_K: as q4_K with the codes at 48 and the fifth bit of value 64q + 16p + i
 // in bit 2q + (p>>1) of qh[16(p&1) + i] (codes 0..31, exact in the same
 // bf16 trick).
@@ -568,27 +618,46 @@ template <> struct Stages<KQ_Q5_K, 2> { static constexpr int RST = 2, AST = 2, B
 template <> struct Stages<KQ_Q4_0, 1> { static constexpr int RST = 3, AST = 3, BST = 3, KPS = 1; };
 template <> struct Stages<KQ_Q4_0, 2> { static constexpr int RST = 3, AST = 2, BST = 3, KPS = 2; };
 
-template <int QT, int CG>
+// The flat raw view (q6_K rows that are not a 16-byte multiple) loads each
+// row's 240-byte window with its own tensor copy, whose shared-memory
+// destination must be 128-byte aligned: rows of raw stages are then 256
+// bytes apart, and fewer stages fit (two of each).
+template <int QT, int CG, bool FLAT> struct StagesOf : Stages<QT, CG> {
+    static constexpr int RAWB = QmmCodec<QT>::RAWB;
+};
+template <int CG> struct StagesOf<KQ_Q6_K, CG, true> {
+    static constexpr int RST = 2, AST = 2, BST = CG == 2 ? 2 : 3, KPS = Stages<KQ_Q6_K, CG>::KPS;
+    static constexpr int RAWB = 256;
+};
+
+template <int QT, int CG, bool FLAT = false>
 constexpr uint32_t smem_bytes() {
-    using S = Stages<QT, CG>;
+    using S = StagesOf<QT, CG, FLAT>;
     return kHeader + 1024 + S::BST * S::KPS * (kBN / CG) * kBK * 2 + S::AST * S::KPS * kBM * kBK * 2 +
-           S::RST * kBM * QmmCodec<QT>::RAWB;
+           S::RST * kBM * S::RAWB;
 }
 
-template <int QT, int CG>
+// FLAT (q6_K only): the weight rows are not a 16-byte multiple, so the raw
+// tensor map is a rank-1 view of all the weight bytes; the raw producer loads
+// each row's 16-byte aligned window of a block separately, and each decoder
+// thread takes its row's offset in the window at run time.
+template <int QT, int CG, bool FLAT = false>
 __global__ void __launch_bounds__(kThreads, 1)
     qmm_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
                const QmmParams p) {
+    static_assert(!FLAT || QT == KQ_Q6_K, "the flat raw view serves q6_K");
     using C = QmmCodec<QT>;
-    constexpr int RST = Stages<QT, CG>::RST;
-    constexpr int AST = Stages<QT, CG>::AST;
-    constexpr int BST = Stages<QT, CG>::BST;
-    constexpr int KPS = Stages<QT, CG>::KPS;   // 64-value K steps per A/B stage
+    using SO = StagesOf<QT, CG, FLAT>;
+    constexpr int RST = SO::RST;
+    constexpr int AST = SO::AST;
+    constexpr int BST = SO::BST;
+    constexpr int KPS = SO::KPS;     // 64-value K steps per A/B stage
+    constexpr int RAWB = SO::RAWB;   // shared-memory bytes of a raw stage row
     static_assert(RST <= 4 && AST <= 4 && BST <= 8, "barrier table holds 4 raw, 4 A and 8 B stages");
     static_assert(KPS == 1 || KPS == 2, "a raw stage (4 K steps) holds whole A/B stages");
-    static_assert(smem_bytes<QT, CG>() <= 232448, "shared memory per CTA");
+    static_assert(smem_bytes<QT, CG, FLAT>() <= 232448, "shared memory per CTA");
     constexpr int kBNc = kBN / CG;                    // activation rows of a B stage in this CTA
-    constexpr uint32_t kRawBytes = kBM * C::RAWB;
+    constexpr uint32_t kRawBytes = kBM * RAWB;
     constexpr uint32_t kAAtom = kBM * kBK * 2;       // 16 KB: one K step of A
     constexpr uint32_t kBAtom = kBNc * kBK * 2;      // 32 KB (one CTA) or 16 KB (pair): one K step of B
     constexpr uint32_t kABytes = KPS * kAAtom;
@@ -889,7 +958,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         // One 256-value block column of this CTA's 128 weight rows per stage,
         // straight from the wire bytes; the block kRawAhead stages ahead is
         // prefetched into L2 so that the load it later issues finds it there.
-        if (lane == 0) {
+        if constexpr (FLAT) {
+            // flat view: lane l loads the windows of rows l, l + 32, l + 64,
+            // l + 96 (240 bytes each, from the 16-byte boundary at or below
+            // the block's first byte, into a 256-byte slot: a tensor copy's
+            // shared-memory destination is 128-byte aligned; past the end of
+            // the weights the tensor map fills zeros); lane 0 waits and sets
+            // the byte count
+            Pipe rp;
+            const int nblk = ksteps / 4;
+            for (int u = u0; u < total_units && !aborted(); u += ustep) {
+                Unit U;
+                get_unit(u, U);
+                if (U.nt == 0) continue;
+                const int64_t wrow = static_cast<int64_t>(U.e) * p.n + U.ntile * wtile_rows + kBM * static_cast<int>(rank);
+                bool ok = true;
+                for (int blk = 0; blk < nblk; ++blk) {
+                    if (lane == 0) {
+                        ok = bwait(&raw_empty[rp.idx], rp.phase ^ 1);
+                        // 128 windows of C::RAWB (240) bytes land in 256-byte slots
+                        if (ok) mbar_arrive_expect_tx(&raw_full[rp.idx], kBM * C::RAWB);
+                    }
+                    if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+#pragma unroll
+                    for (int j = 0; j < kBM / 32; ++j) {
+                        const int r = lane + 32 * j;
+                        const int64_t b0 = (wrow + r) * p.row_bytes + 210 * blk;
+                        tma_load_1d(rst + rp.idx * kRawBytes + r * RAWB, &wmap, static_cast<int>(b0 & ~int64_t(15)),
+                                    &raw_full[rp.idx]);
+                    }
+                    rp.next(RST);
+                }
+                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            }
+        } else if (lane == 0) {
             Pipe rp;
             const int nblk = ksteps / 4;
             auto xcol = [&](int blk) {
@@ -1045,14 +1147,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             get_unit(u, U);
             if (U.nt == 0) continue;
             bool ok = true;
+            // flat view: this thread's row starts at rbyte (its window offset
+            // moves with every block)
+            int64_t rbyte = 0;
+            if constexpr (FLAT)
+                rbyte = (static_cast<int64_t>(U.e) * p.n + U.ntile * wtile_rows + kBM * static_cast<int>(rank) + r) *
+                        p.row_bytes;
             for (int ks0 = 0; ks0 < ksteps && ok; ks0 += 4) {
-                const uint32_t row = rst + rp.idx * kRawBytes + r * C::RAWB;
-                const int o6 = QT == KQ_Q6_K ? (210 * (ks0 >> 2)) & 15 : 0;
+                const uint32_t row = rst + rp.idx * kRawBytes + r * RAWB;
+                const int o6 = QT != KQ_Q6_K ? 0
+                               : FLAT        ? static_cast<int>((rbyte + 210 * (ks0 >> 2)) & 15)
+                                             : (210 * (ks0 >> 2)) & 15;
                 if (!bwait(&raw_full[rp.idx], rp.phase)) {
                     ok = false;
                     break;
                 }
-                prep_scales<QT>(row, part, o6, S);
+                if constexpr (FLAT) q6k_scales_rt(row, o6, part, S);
+                else prep_scales<QT>(row, part, o6, S);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const int a = q % KPS;   // K step within the A stage
@@ -1061,7 +1172,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     uint32_t o[8];
-                    decode_step<QT>(row, q, part, o6, S, o);
+                    if constexpr (FLAT) q6k_step_rt(row, o6, q, part, S, o);
+                    else decode_step<QT>(row, q, part, o6, S, o);
                     const uint32_t ab = ast + ap.idx * kABytes + a * kAAtom;
                     sts128(ab + so0, o[0], o[1], o[2], o[3]);
                     sts128(ab + so1, o[4], o[5], o[6], o[7]);
@@ -1125,12 +1237,27 @@ int make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* ptr,
     return r == CUDA_SUCCESS ? KQ_OK : KQ_ERR_INVALID_ARG;
 }
 
+// Rank-1 byte map over `bytes` bytes at w (16-byte aligned), boxes of `box`
+// bytes (a multiple of 16); reads past the end are zero-filled.
+int make_map_1d(CUtensorMap* m, const void* w, uint64_t bytes, uint32_t box) {
+    EncodeTiled enc = get_encoder();
+    if (!enc) return KQ_ERR_CUDA;
+    const cuuint64_t dims[1] = {bytes};
+    const cuuint64_t strides[1] = {bytes};   // unused at rank 1
+    const cuuint32_t boxd[1] = {box};
+    const cuuint32_t estr[1] = {1};
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, const_cast<void*>(w), dims, strides, boxd, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? KQ_OK : KQ_ERR_INVALID_ARG;
+}
+
 // Launch with units of 128 (one CTA) or 256 (a CTA pair) weight rows; a pair
 // is a cluster of two CTAs on neighbouring SMs.
-template <int QT, int CG>
+template <int QT, int CG, bool FLAT = false>
 int launch_cg(const CUtensorMap& wmap, const CUtensorMap& xmap, QmmParams p, cudaStream_t s) {
-    constexpr uint32_t smem = smem_bytes<QT, CG>();
-    auto kern = qmm_kernel<QT, CG>;
+    constexpr uint32_t smem = smem_bytes<QT, CG, FLAT>();
+    auto kern = qmm_kernel<QT, CG, FLAT>;
     static bool attr_set[64] = {false};
     static int slots[64] = {0};   // CTAs of this kernel resident at once, per device
     int dev = 0;
@@ -1208,10 +1335,16 @@ int launch_impl(const void* w, int64_t w_rows, int64_t n, int64_t k, const uint1
     const int bpb = QT == KQ_Q4_K ? 144 : QT == KQ_Q5_K ? 176 : QT == KQ_Q6_K ? 210 : QT == KQ_Q4_0 ? 18 : 34;
     const int64_t row_bytes = k / vpb * bpb;
     if (k % 256 != 0) return KQ_ERR_UNSUPPORTED;        // 256-value raw stages
-    if (row_bytes % 16 != 0) return KQ_ERR_UNSUPPORTED;  // TMA row stride
+    // rows that are not a 16-byte multiple (q6_K with K / 256 not a multiple
+    // of 8) take the flat raw view: a rank-1 map over all the weight bytes,
+    // whose coordinates (bytes, 32-bit) must cover the last tile's rows
+    const bool flat = row_bytes % 16 != 0;
+    if (flat && (QT != KQ_Q6_K || (w_rows + 2 * kBM) * row_bytes >= (int64_t(1) << 31))) return KQ_ERR_UNSUPPORTED;
     CUtensorMap wmap, xmap;
     int rc;
-    if constexpr (QT == KQ_Q8_0)
+    if (flat)
+        rc = make_map_1d(&wmap, w, static_cast<uint64_t>(w_rows * row_bytes), C::RAWB);
+    else if constexpr (QT == KQ_Q8_0)
         rc = make_map(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, w, row_bytes / 2, w_rows, C::RAWB / 2, kBM,
                       CU_TENSOR_MAP_SWIZZLE_NONE);
     else
@@ -1232,6 +1365,10 @@ int launch_impl(const void* w, int64_t w_rows, int64_t n, int64_t k, const uint1
     p.y = y;
     p.err = err;
     p.status = device_status_ptr();
+    p.row_bytes = row_bytes;
+    if constexpr (QT == KQ_Q6_K) {
+        if (flat) return use_pair_mma() ? launch_cg<QT, 2, true>(wmap, xmap, p, s) : launch_cg<QT, 1, true>(wmap, xmap, p, s);
+    }
     return use_pair_mma() ? launch_cg<QT, 2>(wmap, xmap, p, s) : launch_cg<QT, 1>(wmap, xmap, p, s);
 }
 

@@ -175,3 +175,17 @@ def test_gather_more_than_1024_tiles(shuffle):
     for ex in range(experts):
         r = np.nonzero(ids == ex)[0]
         check_qmm(y[r], ref[r], xn[r], row_norms_w(kq.Q4_K, w[ex], k), k)
+
+
+def test_gather_q6K_rows_not_16_byte_multiple():
+    # K = 11008: 9030-byte rows; three experts' segments through the flat view
+    experts, n, k = 3, 200, 11008
+    ids = np.sort(np.random.default_rng(31).integers(0, experts, 300)).astype(np.uint32)
+    tiles = oracle.tile_map(ids, experts)
+    w, x, y, e = run_gather(kq.Q6_K, experts, n, k, tiles, len(ids), seed=32)
+    assert e == 0
+    ref = oracle.gather_qmm(kq.Q6_K, w, k, x, tiles)
+    xn = row_norms_x(x)
+    for ex in range(experts):
+        r = np.nonzero(ids == ex)[0]
+        check_qmm(y[r], ref[r], xn[r], row_norms_w(kq.Q6_K, w[ex], k), k)

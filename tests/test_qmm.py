@@ -78,3 +78,28 @@ def test_deterministic(qtype):
     w = dev_u8(synth.weights(qtype, 384, 2048, seed=1))
     x = dev_bf16(synth.activations(300, 2048, seed=2))
     assert torch.equal(kq.qmm(x, w, qtype), kq.qmm(x, w, qtype))
+
+
+# q6_K rows that are not a 16-byte multiple (K / 256 not a multiple of 8: 210
+# bytes per block) take the flat view of the weights, each row's window loaded
+# on its own and decoded at its own byte offset: K = 768 (630-byte rows),
+# K = 11008 (9030-byte rows), ragged M and N, several units and the last-round
+# split
+@pytest.mark.parametrize("m,n,k", [(70, 130, 768), (300, 257, 11008), (200, 25344, 768)])
+def test_q6K_rows_not_16_byte_multiple(m, n, k):
+    assert synth.row_bytes(kq.Q6_K, k) % 16 != 0
+    run_full(kq.Q6_K, n, k, m, seed=k + m)
+
+
+def test_q6K_k11008_large_sampled():
+    m, n, k = 1024, 14336, 11008
+    w = synth.weights(kq.Q6_K, n, k, seed=3)
+    x = synth.activations(m, k, seed=4)
+    y = kq.qmm(dev_bf16(x), dev_u8(w), kq.Q6_K).cpu().numpy()
+    g = np.random.default_rng(5)
+    rows = np.sort(g.choice(m, 16, replace=False))
+    cols = np.sort(g.choice(n, 16, replace=False))
+    wn = row_norms_w(kq.Q6_K, w, k)
+    xn = row_norms_x(x)
+    check_qmm(y[rows], oracle.matmul(kq.Q6_K, w, k, x[rows]), xn[rows], wn, k)
+    check_qmm(y[:, cols], oracle.matmul(kq.Q6_K, w[cols], k, x), xn, wn[cols], k)
