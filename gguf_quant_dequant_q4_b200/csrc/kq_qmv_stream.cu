@@ -405,11 +405,16 @@ struct Q6 {
     static constexpr int kXT = 14;
     static constexpr bool kTwoPhase = false;
 
-    // Word at shared address a (2-byte aligned when ODD).
-    template <bool ODD>
+    // Word at shared address a: 4-byte aligned (MODE 0), 2 bytes past a
+    // 4-byte boundary (MODE 1), or either, per thread (MODE 2: rows at their
+    // own offsets, when a row is not a 16-byte multiple).
+    template <int MODE>
     static __device__ __forceinline__ uint32_t word(uint32_t a) {
-        if constexpr (ODD) return __byte_perm(lds32(a - 2), lds32(a + 2), 0x5432);
-        else return lds32(a);
+        if constexpr (MODE == 1) return __byte_perm(lds32(a - 2), lds32(a + 2), 0x5432);
+        else if constexpr (MODE == 2) {
+            const uint32_t al = a & ~3u;
+            return __byte_perm(lds32(al), lds32(al + 4), (a & 2u) ? 0x5432u : 0x3210u);
+        } else return lds32(a);
     }
 
     // One block of 16 rows.  Lane t owns quarter (h = t >> 1, lh = t & 1):
@@ -421,7 +426,7 @@ struct Q6 {
     // (q = qp + 2, 1024 + 16 c6, x/256) into column 2t + 1.  The four lanes of
     // a row read their words in the order (k + t) mod 4, which spreads them over
     // all 32 banks; the activation image follows the same order.
-    template <bool ODD>
+    template <int ODD>
     static __device__ __forceinline__ void block(const SP& p, uint32_t sb, const Lane& L, uint32_t rowA,
                                                  uint32_t rowB, int gb, float (&acc)[2 * NT]) {
         const int t = L.t, h = t >> 1, lh = t & 1;
@@ -512,8 +517,13 @@ struct Q6 {
 
     static __device__ __forceinline__ void item(const SP& p, uint32_t sb, const Lane& L, uint32_t rowA,
                                                 uint32_t rowB, int gb, float (&acc)[2 * NT]) {
-        if (gb & 1) block<true>(p, sb, L, rowA, rowB, gb, acc);
-        else block<false>(p, sb, L, rowA, rowB, gb, acc);
+        if (gb & 1) block<1>(p, sb, L, rowA, rowB, gb, acc);
+        else block<0>(p, sb, L, rowA, rowB, gb, acc);
+    }
+    // rows A and B at their own byte offsets (rows not a 16-byte multiple)
+    static __device__ __forceinline__ void item_rt(const SP& p, uint32_t sb, const Lane& L, uint32_t rowA,
+                                                   uint32_t rowB, int gb, float (&acc)[2 * NT]) {
+        block<2>(p, sb, L, rowA, rowB, gb, acc);
     }
 
     static __device__ __forceinline__ void store_part(const SP& p, const Lane& L, float (&acc)[2 * NT], float* part) {
@@ -845,6 +855,18 @@ __device__ bool gather_setup(const SPG& p, uint8_t* smem, int64_t& r0, int64_t& 
     return true;
 }
 
+// The weight bank a stage is read from (GLU: gate or up) and its size.
+template <class P>
+__device__ __forceinline__ const uint8_t* bank_of(const P& p, bool up) {
+    if constexpr (std::is_same<P, SPGLU>::value) return up ? p.w2 : p.w;
+    else return p.w;
+}
+template <class P>
+__device__ __forceinline__ int64_t bank_bytes(const P& p) {
+    if constexpr (std::is_same<P, SP>::value) return p.n * p.row_bytes;
+    else return static_cast<int64_t>(p.n_experts) * p.n * p.row_bytes;
+}
+
 // act(g) * u of the GLU epilogue, in fp32: silu(g) = g / (1 + e^-g); gelu in
 // its tanh form 0.5 g (1 + tanh(sqrt(2/pi) (g + 0.044715 g^3))); silu with
 // limit: silu(min(g, L)) * clamp(u, -L, L).
@@ -954,12 +976,44 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
                 const int b0 = st * p.g;
                 const int nb = p.nblk - b0 < p.g ? p.nblk - b0 : p.g;
                 const uint32_t bytes = static_cast<uint32_t>(nb) * C::kBPB;
-                if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes * rv);
-                __syncwarp();
-                if (lane < rv)
-                    bulk_g2s(smem + p.off_stage + slot * stage_bytes + lane * p.rs,
-                             wsrc + (row0 + lane) * p.row_bytes + (kb0 + b0) * C::kBPB, bytes,
-                             &full[slot]);
+                bool rt = false;
+                if constexpr (C::kBPB == 210 && GATHER) rt = (p.row_bytes & 15) != 0;
+                if (rt) {
+                    // rows that are not a 16-byte multiple (decode MoE q6_K):
+                    // each row's span is copied from the 16-byte boundary at or
+                    // below its first byte, so it lands at its own offset in
+                    // the slot; the copy stops at the last 16-byte boundary of
+                    // the bank and the bytes after it (the bank's last row only)
+                    // are stored one by one before the stage is announced
+                    const uint8_t* bank = bank_of(p, GLU && (rg & 1));
+                    const int64_t lim = bank_bytes(p) & ~int64_t(15);
+                    uint32_t nb16 = 0;
+                    if (lane < rv) {
+                        const int64_t a0 = (wsrc - bank) + (row0 + lane) * p.row_bytes + (kb0 + b0) * C::kBPB;
+                        const int64_t s0 = a0 & ~int64_t(15), end = a0 + bytes;
+                        const int64_t ce = ((end + 15) & ~int64_t(15)) < lim ? ((end + 15) & ~int64_t(15)) : lim;
+                        nb16 = ce > s0 ? static_cast<uint32_t>(ce - s0) : 0u;
+                        uint8_t* dst = smem + p.off_stage + slot * stage_bytes + lane * p.rs;
+                        for (int64_t b = ce > a0 ? ce : a0; b < end; ++b)
+                            asm volatile("st.shared.u8 [%0], %1;" ::"r"(smem_u32(dst + (b - s0))),
+                                         "r"(static_cast<uint32_t>(__ldg(bank + b))));
+                    }
+                    const uint32_t tx = __reduce_add_sync(0xffffffffu, nb16);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_expect_tx(&full[slot], tx);
+                    __syncwarp();
+                    if (nb16) {
+                        const int64_t a0 = (wsrc - bank) + (row0 + lane) * p.row_bytes + (kb0 + b0) * C::kBPB;
+                        bulk_g2s(smem + p.off_stage + slot * stage_bytes + lane * p.rs, bank + (a0 & ~int64_t(15)),
+                                 nb16, &full[slot]);
+                    }
+                } else {
+                    if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes * rv);
+                    __syncwarp();
+                    if (lane < rv)
+                        bulk_g2s(smem + p.off_stage + slot * stage_bytes + lane * p.rs,
+                                 wsrc + (row0 + lane) * p.row_bytes + (kb0 + b0) * C::kBPB, bytes, &full[slot]);
+                }
                 if (++slot == p.ns) {
                     slot = 0;
                     phase ^= 1;
@@ -1021,10 +1075,26 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
                     ok = false;
                 } else {
                     const uint32_t stg = sb + p.off_stage + slot * stage_bytes;
-                    const uint32_t rowA = stg + L.g * p.rs, rowB = rowA + 8 * p.rs;
+                    uint32_t rowA = stg + L.g * p.rs, rowB = rowA + 8 * p.rs;
+                    bool rt = false;
+                    if constexpr (C::kBPB == 210 && GATHER) {
+                        // rows that are not a 16-byte multiple sit at their own
+                        // offsets in the slot (see the producer)
+                        if (p.row_bytes & 15) {
+                            rt = true;
+                            const int64_t ab = (wbase - p.w) + static_cast<int64_t>(st * p.g) * C::kBPB;
+                            rowA += static_cast<uint32_t>((ab + (row0 + L.g) * p.row_bytes) & 15);
+                            rowB += static_cast<uint32_t>((ab + (row0 + L.g + 8) * p.row_bytes) & 15);
+                        }
+                    }
                     for (int it = first; it < i1; it += kCW) {
                         const uint32_t off = static_cast<uint32_t>(it * C::kItemBlocks - st * p.g) * C::kBPB;
-                        C::item(p, sb, L, rowA + off, rowB + off, it, acc);
+                        if constexpr (C::kBPB == 210 && GATHER) {
+                            if (rt) C::item_rt(p, sb, L, rowA + off, rowB + off, it, acc);
+                            else C::item(p, sb, L, rowA + off, rowB + off, it, acc);
+                        } else {
+                            C::item(p, sb, L, rowA + off, rowB + off, it, acc);
+                        }
                     }
                 }
                 __syncwarp();
@@ -1209,8 +1279,11 @@ int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m,
     p.nblk = nblk_all / ks;
     p.k = static_cast<int64_t>(p.nblk) * C::kVPB;
     p.row_bytes = static_cast<int64_t>(nblk_all) * C::kBPB;
-    if (p.row_bytes % 16 != 0) return KQ_ERR_UNSUPPORTED;
-    if ((static_cast<int64_t>(p.nblk) * C::kBPB) % 16 != 0) return KQ_ERR_UNSUPPORTED;   // slice copies
+    // rows that are not a 16-byte multiple: q6_K decode MoE only (each row's
+    // copy starts at a 16-byte boundary, the row at its offset past it)
+    const bool unaligned = p.row_bytes % 16 != 0;
+    if (unaligned && !(ga && C::kBPB == 210)) return KQ_ERR_UNSUPPORTED;
+    if (!unaligned && (static_cast<int64_t>(p.nblk) * C::kBPB) % 16 != 0) return KQ_ERR_UNSUPPORTED;   // slice copies
     p.img_tok = img_tok;
     p.xs_tok = xs_tok;
     const uint32_t optin = static_cast<uint32_t>(device_smem_optin());
@@ -1248,7 +1321,7 @@ int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m,
         for (int s = 1; s <= 16 && p.ns == 0; ++s) {
             const int g = cdiv(cdiv(p.nblk, s), ga_blk) * ga_blk;
             if (s > 1 && g >= p.nblk) continue;
-            const uint32_t rs = ((static_cast<uint32_t>(g) * C::kBPB + 127u) & ~127u) + 16;
+            const uint32_t rs = ((static_cast<uint32_t>(g) * C::kBPB + (unaligned ? 32u : 0u) + 127u) & ~127u) + 16;
             for (int ns = kMaxStages; ns >= 2; --ns) {
                 if (p.off_stage + static_cast<uint32_t>(ns) * kRows * rs <= optin) {
                     p.ns = ns;
@@ -1414,8 +1487,7 @@ int launch_gather_qmv(int type, const void* w_bank, const void* w_bank2, int act
         if (rc == KQ_ERR_UNSUPPORTED) rc = launch_stream<Q8<1>>(w_bank, n, k, x, 1, y, s, it, xt, 1, &ga);
         return rc;
     }
-    case KQ_Q6_K: {
-        if (nblk % 8 != 0) return KQ_ERR_UNSUPPORTED;
+    case KQ_Q6_K: {   // any k % 256 == 0 (rows that are not a 16-byte multiple included)
         const uint32_t it = nblk * Q6<1>::kBlkImg, xt = nblk * 32 * 4;
         rc = m_cap >= 2 ? launch_stream<Q6<2>>(w_bank, n, k, x, 2, y, s, it, xt, 1, &ga) : KQ_ERR_UNSUPPORTED;
         if (rc == KQ_ERR_UNSUPPORTED) rc = launch_stream<Q6<1>>(w_bank, n, k, x, 1, y, s, it, xt, 1, &ga);

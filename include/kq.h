@@ -35,8 +35,8 @@
  *    cudaError_t is available from kq_last_cuda_error()).  Nothing throws.
  *  - Alignment: W, x, y and out must be 16-byte aligned, else
  *    KQ_ERR_ALIGNMENT.  Weight rows whose byte length is not a multiple of 16
- *    are accepted by kq_dequantize and kq_qmv (a slower staging path);
- *    kq_qmm / kq_gather_qmm need k % 256 == 0 and 16-byte multiple rows
+ *    (q6_K with k / 256 not a multiple of 8) are accepted everywhere, on
+ *    slower copy paths; kq_qmm / kq_gather_qmm need k % 256 == 0
  *    (KQ_ERR_UNSUPPORTED otherwise).
  *  - `k` must be a multiple of the codec's values_per_block, as the reference
  *    requires ("last dim a multiple of the codec's bytes_per_block",
@@ -249,8 +249,10 @@ int kq_gather_qmm(int type, const void* w_bank, int32_t n_experts, int64_t n, in
  * routed expert's weights are read once for all of its pairs (in batches of
  * up to 2 (q8_0, q6_K) or 16 (q4_K) activation rows; an expert with more
  * pairs than a batch is streamed once per batch).  Arithmetic as kq_qmv.
- * Limits: 1 <= n_experts <= 256, 1 <= n_tokens*top_k <= 8192; k % 256 == 0
- * (q8_0, q4_K) or k % 2048 == 0 (q6_K), else KQ_ERR_UNSUPPORTED.
+ * Limits: 1 <= n_experts <= 256, 1 <= n_tokens*top_k <= 8192; k % 256 == 0,
+ * else KQ_ERR_UNSUPPORTED (q6_K rows that are not a 16-byte multiple, k / 256
+ * not a multiple of 8, take a slower copy path: each row is staged from the
+ * 16-byte boundary below it and decoded at its own byte offset).
  *   err_flag (nullable): KQ_DEV_BAD_EXPERT for ids outside [0, n_experts);
  *   the rows of those pairs are left unwritten.
  */

@@ -224,3 +224,34 @@ def test_decode_moe_edge_cases():
     o = kq.gather_mix(torch.from_numpy(yv).cuda(), torch.from_numpy(inv).cuda(), torch.from_numpy(sc).cuda())
     ref = oracle.gather_mix(yv, inv, sc)
     assert np.array_equal(o.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("k,n", [(768, 201), (11008, 257)])
+def test_gather_qmv_q6K_rows_not_16_byte_multiple(k, n):
+    # q6_K rows of 630 / 9030 bytes: staged from the 16-byte boundary below
+    # each row and decoded at the row's own offset; the bank's size is not a
+    # multiple of 16 either, so its last row ends past the last 16-byte
+    # boundary (every expert is routed, the last one included)
+    tokens, top_k, experts = 4, 2, 4
+    assert synth.row_bytes(kq.Q6_K, k) % 16 != 0 and (experts * n * synth.row_bytes(kq.Q6_K, k)) % 16 != 0
+    w = synth.weights(kq.Q6_K, n, k, seed=k, experts=experts)
+    ids = np.array([[0, 3], [1, 2], [3, 1], [2, 0]], np.int32)
+    x = synth.activations(tokens * top_k, k, seed=k + 1)
+    y, e = run_gather_qmv(kq.Q6_K, w, k, x, ids)
+    assert e == 0
+    check_pairs(kq.Q6_K, w, k, x, ids, y)
+    xt = synth.activations(tokens, k, seed=k + 2)
+    y, e = run_gather_qmv(kq.Q6_K, w, k, xt, ids, x_per_token=True)
+    assert e == 0
+    check_pairs(kq.Q6_K, w, k, xt, ids, y, x_per_token=True)
+
+
+def test_moe_glu_gather_q6K_k11008():
+    tokens, top_k, experts, n, k = 3, 2, 4, 129, 11008
+    wg = synth.weights(kq.Q6_K, n, k, seed=111, experts=experts)
+    wu = synth.weights(kq.Q6_K, n, k, seed=112, experts=experts)
+    ids = np.array([[3, 0], [1, 3], [2, 1]], np.int32)
+    x = synth.activations(tokens, k, seed=113)
+    out = kq.moe_glu_gather(dev_bf16(x), dev_u8(wg), dev_u8(wu), kq.Q6_K, torch.from_numpy(ids).cuda())
+    ref, g, u, ag, au = oracle.moe_glu_gather(kq.Q6_K, wg, wu, k, x, ids)
+    check_glu(out.cpu().numpy(), ref, g, u, ag, au, kq.ACT_SILU)
