@@ -801,7 +801,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     else __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
-    if (p.n_experts != 0) total_units = static_cast<int>(misc[2]) * p.ntn;
+    // gather: units are (chunk of <= 4 map tiles, weight tile); as for dense
+    // qmm, the units of the last, partial round of the grid are split, here
+    // into sub-units of one or two map tiles, so that they spread over more
+    // CTAs (every thread derives the same split from the chunk count)
+    int g_main = 0, g_split = 1;
+    if (p.n_experts != 0) {
+        total_units = static_cast<int>(misc[2]) * p.ntn;
+        const int ng = static_cast<int>(gridDim.x) / CG;
+        g_main = total_units;
+        const int tail = total_units % ng;
+        if (total_units > ng && tail != 0) {
+            g_split = 4 * tail <= ng ? 4 : (2 * tail <= ng ? 2 : 1);
+            g_main = total_units - tail;
+            total_units = g_main + g_split * tail;
+        }
+    }
     // a unit is processed by one CTA (CG = 1) or one CTA pair (CG = 2)
     const int u0 = static_cast<int>(blockIdx.x) / CG, ustep = static_cast<int>(gridDim.x) / CG;
 
@@ -837,8 +852,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         } else {
             const int nch = static_cast<int>(misc[2]);
-            const int c = u % nch;
-            U.ntile = u / nch;
+            int fu = u, sub = -1;
+            if (u >= g_main) {
+                fu = g_main + (u - g_main) / g_split;
+                sub = (u - g_main) % g_split;
+            }
+            const int c = fu % nch;
+            U.ntile = fu / nch;
             int lo = 0, hi = p.n_experts - 1;   // expert with cstart[e] <= c < cstart[e+1]
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
@@ -846,8 +866,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 else hi = mid - 1;
             }
             U.e = lo;
-            const int first = tstart[lo] + 4 * (c - cstart[lo]);
-            const int left = tstart[lo + 1] - first;
+            int first = tstart[lo] + 4 * (c - cstart[lo]);
+            int left = tstart[lo + 1] - first;
+            if (sub >= 0) {   // sub-unit: tiles [sub * per, sub * per + per) of the chunk
+                const int per = 4 / g_split;
+                first += sub * per;
+                left -= sub * per;
+                left = left < 0 ? 0 : (left > per ? per : left);
+            }
             U.nt = left >= 4 ? 4 : left;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
