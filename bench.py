@@ -389,8 +389,9 @@ def measure_rows(kq, torch, dev, pk, args) -> dict:
                                                      "frac_hbm": round(qb / (t / 1e3) / 1e9 / pk["hbm_gbs"], 4),
                                                      "bytes": qb}
     del wf
-    # q5_K and q4_0 (no decode kernel of their own): dequantize 4096 x 4096,
-    # qmv M=1 on the c1 shape (exact fp32 decode-and-dot kernel) and qmm on the c3 shape
+    # q5_K and q4_0: dequantize 4096 x 4096; qmv M = 1, 2 on the c1 shape (the
+    # staged decode kernel); gather_qmv, one token routed top-2 over a bank of
+    # 4 such experts; qmm on the c3 shape
     for qt, nm in ((Q5_K, "q5K"), (Q4_0, "q4_0")):
         w = synth.weights(qt, 4096, 4096)
         cp = ncopies(w.nbytes)
@@ -405,13 +406,28 @@ def measure_rows(kq, torch, dev, pk, args) -> dict:
         w = synth.weights(qt, 14336, 4096)
         cp = ncopies(w.nbytes)
         Ws = [u8(w) for _ in range(cp)]
-        x1 = bf(synth.activations(1, 4096))
-        y1 = torch.empty(1, 14336, device=dev)
-        t = time_graph(torch, lambda i: kq.qmv(x1, Ws[i % cp], qt, out=y1), reps, s)
+        for m in (1, 2):
+            xm = bf(synth.activations(m, 4096))
+            ym = torch.empty(m, 14336, device=dev)
+            t = time_graph(torch, lambda i: kq.qmv(xm, Ws[i % cp], qt, out=ym), reps, s)
+            launches += reps + 3
+            gbs = w.nbytes / (t / 1e3) / 1e9
+            rows[f"qmv_{nm}_m{m}_14336x4096"] = {"kernel_us": round(t * 1e3, 2), "GB/s": round(gbs, 1),
+                                                 "frac_hbm": round(gbs / pk["hbm_gbs"], 4), "bytes": w.nbytes}
+        bank0 = torch.stack([Ws[i % cp] for i in range(4)])
+        qbanks = [bank0] + [bank0.clone() for _ in range(ncopies(2 * w.nbytes) - 1)]
+        rid = torch.from_numpy(synth.routing(1, 4, 2, seed=9)).to(dev)
+        distinct = int(torch.unique(rid).numel())
+        xg = bf(synth.activations(1, 4096, seed=10))
+        yg = torch.empty(2, 14336, device=dev)
+        t = time_graph(torch, lambda i: kq.gather_qmv(xg, qbanks[i % len(qbanks)], qt, rid, x_per_token=True,
+                                                      out=yg), reps, s)
         launches += reps + 3
-        gbs = w.nbytes / (t / 1e3) / 1e9
-        rows[f"qmv_{nm}_m1_14336x4096"] = {"kernel_us": round(t * 1e3, 2), "GB/s": round(gbs, 1),
-                                                  "frac_hbm": round(gbs / pk["hbm_gbs"], 4), "bytes": w.nbytes}
+        gbs = distinct * w.nbytes / (t / 1e3) / 1e9
+        rows[f"decode_moe_gather_qmv_{nm}_4x14336x4096_t1_top2"] = {
+            "kernel_us": round(t * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
+            "bytes": distinct * w.nbytes, "experts_read": distinct}
+        del qbanks, bank0
         xq = bf(synth.activations(2048, 4096))
         yq = torch.empty(2048, 14336, device=dev)
         t = time_graph(torch, lambda i: kq.qmm(xq, Ws[i % cp], qt, out=yq), 8, s)

@@ -3,7 +3,7 @@
 // mlx-kquant bindings.cpp `quantized_matmul` (x @ dequant(w).T); README "How
 // it works": small row counts take a kernel that amortizes each weight read
 // over all rows (`verify_qmv`); hanzo-ml quantized/mod.rs: decode runs the
-// quantized matvec "straight out of the block format".
+// quantized matvec directly on the packed blocks.
 //
 // The path is HBM-bound, so the design goal is to spend as few instructions
 // per weight as possible while reading every weight byte exactly once:
@@ -66,15 +66,15 @@ template <int QT> struct Codec;
 // q6_K and q8_0 keep their smallest operands (x/256, x/64) normal.
 template <> struct Codec<KQ_Q4_K> {
     static constexpr int VPB = 256, BPB = 144, GA = 8, XT = 9;
-    static constexpr int IMG = 544, XS = 0;   // B image bytes / fp32 sums per (token, block)
+    static constexpr int IMG = 544;   // B image bytes per (token, block)
 };
 template <> struct Codec<KQ_Q6_K> {
     static constexpr int VPB = 256, BPB = 210, GA = 8, XT = 14;
-    static constexpr int IMG = 1024, XS = 16;
+    static constexpr int IMG = 1024;
 };
 template <> struct Codec<KQ_Q8_0> {
     static constexpr int VPB = 32, BPB = 34, GA = 8, XT = 14;
-    static constexpr int IMG = 64, XS = 1;
+    static constexpr int IMG = 64;
 };
 
 struct QmvParams {
@@ -84,7 +84,7 @@ struct QmvParams {
     int* status;
     int64_t n, k, row_bytes;
     int m, nblk, scb, ns, bulk, g, rs;
-    uint32_t tokstride, off_img, off_x, off_pbuf, off_racc;
+    uint32_t tokstride, off_img, off_pbuf, off_racc;
 };
 
 // binary16 constants
@@ -162,14 +162,13 @@ __device__ void x_range(const QmvParams& p, int64_t v0, int nv, uint32_t* xm) {
 // B registers of lane (g = token, t) in binary16 (of the scaled activations).
 // ---------------------------------------------------------------------------
 template <int QT>
-__device__ void build_image(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t xsum, const uint32_t* xm);
+__device__ void build_image(const QmvParams& p, int blk0, int nb, uint32_t img, const uint32_t* xm);
 
 // q4_K: MMA (nib, u) of lane t uses values v = 64t + 32nib + 4u + {0,2 | 1,3};
 // the extra 32 bytes per block hold (Xhi, Xlo) of sub-blocks 2t and 2t+1, the
 // sums of their binary16 operands split into two binary16 parts.
 template <>
-__device__ void build_image<KQ_Q4_K>(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t,
-                                     const uint32_t* xm) {
+__device__ void build_image<KQ_Q4_K>(const QmvParams& p, int blk0, int nb, uint32_t img, const uint32_t* xm) {
     const int items = p.m * nb * 4;
     for (int it = threadIdx.x; it < items; it += kCWarps * 32) {
         const int m = it / (nb * 4), rem = it % (nb * 4), bl = rem >> 2, t = rem & 3;
@@ -206,18 +205,15 @@ __device__ void build_image<KQ_Q4_K>(const QmvParams& p, int blk0, int nb, uint3
     }
 }
 
-// q8_0: MMA h (0, 1) of lane t uses values v = 8t + 4h + {0,2 | 1,3};
-// X = 128 2^-24 (= 2^-17) times the sum of the block's 32 binary16 operands.
+// q8_0: MMA h (0, 1) of lane t uses values v = 8t + 4h + {0,2 | 1,3}.
 template <>
-__device__ void build_image<KQ_Q8_0>(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t xsum,
-                                     const uint32_t* xm) {
+__device__ void build_image<KQ_Q8_0>(const QmvParams& p, int blk0, int nb, uint32_t img, const uint32_t* xm) {
     const int items = p.m * nb;
     for (int it = threadIdx.x; it < items; it += kCWarps * 32) {
         const int m = it / nb, bl = it % nb;
         const uint16_t* xs = p.x + static_cast<int64_t>(m) * p.k + static_cast<int64_t>(blk0 + bl) * 32;
         const uint32_t base = img + m * p.tokstride + bl * 64;
         const float S = tok_scale<KQ_Q8_0>(xm, m);
-        float X = 0.f;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
             const uint4 r = ldg_nc_v4(xs + 8 * t);
@@ -226,12 +222,9 @@ __device__ void build_image<KQ_Q8_0>(const QmvParams& p, int blk0, int nb, uint3
             for (int h = 0; h < 2; ++h) {
                 const float f0 = bf16lo_to_f32(wv[2 * h]), f1 = bf16hi_to_f32(wv[2 * h]);
                 const float f2 = bf16lo_to_f32(wv[2 * h + 1]), f3 = bf16hi_to_f32(wv[2 * h + 1]);
-                const uint32_t h02 = f16pair(f0, f2, S), h13 = f16pair(f1, f3, S);
-                X += f16sum(h02) + f16sum(h13);
-                sts64(base + h * 32 + t * 8, h02, h13);
+                sts64(base + h * 32 + t * 8, f16pair(f0, f2, S), f16pair(f1, f3, S));
             }
         }
-        sts32(xsum + (m * p.scb + bl) * 4, __float_as_uint(X * 7.62939453125e-06f));
     }
 }
 
@@ -239,12 +232,10 @@ __device__ void build_image<KQ_Q8_0>(const QmvParams& p, int blk0, int nb, uint3
 // high-code MMA; lane t uses values 16j + 4t + {0,2 | 1,3}.  The low-code B
 // is a = x/16 (tq < 2) or x/256 (tq >= 2, where the code sits in the high
 // nibble); the high-code B is x / 4^tq (x scaled, then rounded to binary16).
-// The MMAs give D = 2^-24 sum c x / 16 with c the 6-bit code, so
-// sum (c - 32) x = 16 2^24 (D - X) with X = 2^-24 * 32 * sum x / 16, stored
-// from the low-code operands: 2^-19 sum a (tq < 2) or 2^-15 sum a.
+// With the high 2 bits centred (h - 2) the MMAs give D = 2^-24 sum (c - 32)
+// x / 16, c the 6-bit code.
 template <>
-__device__ void build_image<KQ_Q6_K>(const QmvParams& p, int blk0, int nb, uint32_t img, uint32_t xsum,
-                                     const uint32_t* xm) {
+__device__ void build_image<KQ_Q6_K>(const QmvParams& p, int blk0, int nb, uint32_t img, const uint32_t* xm) {
     const int items = p.m * nb * 16;
     for (int it = threadIdx.x; it < items; it += kCWarps * 32) {
         const int m = it / (nb * 16), rem = it % (nb * 16), bl = rem >> 4, j = rem & 15;
@@ -255,18 +246,13 @@ __device__ void build_image<KQ_Q6_K>(const QmvParams& p, int blk0, int nb, uint3
         const uint32_t base = img + m * p.tokstride + bl * 1024 + j * 64;
         const uint4 r0 = ldg_nc_v4(xs), r1 = ldg_nc_v4(xs + 8);
         const uint32_t wv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-        float A = 0.f;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
             const float f0 = bf16lo_to_f32(wv[2 * t]), f1 = bf16hi_to_f32(wv[2 * t]);
             const float f2 = bf16lo_to_f32(wv[2 * t + 1]), f3 = bf16hi_to_f32(wv[2 * t + 1]);
-            const uint32_t a02 = f16pair(f0, f2, slo), a13 = f16pair(f1, f3, slo);
-            A += f16sum(a02) + f16sum(a13);
-            sts64(base + t * 8, a02, a13);
+            sts64(base + t * 8, f16pair(f0, f2, slo), f16pair(f1, f3, slo));
             sts64(base + 32 + t * 8, f16pair(f0, f2, shi), f16pair(f1, f3, shi));
         }
-        sts32(xsum + ((m * p.scb + bl) * 16 + j) * 4,
-              __float_as_uint(A * (tq < 2 ? 1.9073486328125e-06f : 3.0517578125e-05f)));
     }
 }
 
@@ -381,10 +367,10 @@ __device__ __forceinline__ void col_info(int nt, int col, int m, int& tok, int& 
 
 // q8_0: the warp's run of up to RUN consecutive 32-value blocks of one stage.
 // rowA/rowB: shared address of row g / g+8 of the stage; lb0: first local
-// block; nvalid: blocks present; imgb0 / xsb0: image/X offsets of lb0.
+// block; nvalid: blocks present; imgb0: image offset of lb0.
 template <int S, int NT, int RUN>
 __device__ __forceinline__ void q8_run(const Lane<NT>& L, const QmvParams& p, uint32_t rowA, uint32_t rowB, int lb0,
-                                       int nvalid, uint32_t imgb0, uint32_t xsb0, uint32_t zero_addr,
+                                       int nvalid, uint32_t imgb0, uint32_t zero_addr,
                                        float (&acc)[NT][4]) {
     const int t = L.t;
     float D[NT][4];
@@ -405,11 +391,12 @@ __device__ __forceinline__ void q8_run(const Lane<NT>& L, const QmvParams& p, ui
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const uint32_t wa = h ? a1w : a0w, wb = h ? b1w : b0w;
-                // byte ^ 0x80 = q + 128 as a binary16 subnormal: (q + 128) 2^-24
-                const uint32_t A0 = and_xor(wa, 0x00FF00FFu, 0x00800080u);
-                const uint32_t A1 = and_xor(wb, 0x00FF00FFu, 0x00800080u);
-                const uint32_t A2 = and_xor(wa >> 8, 0x00FF00FFu, 0x00800080u);
-                const uint32_t A3 = and_xor(wb >> 8, 0x00FF00FFu, 0x00800080u);
+                // byte ^ 0x80 = q + 128 as a binary16 subnormal, less 128 2^-24:
+                // the signed code as the subnormal q 2^-24 (exact)
+                const uint32_t A0 = hsub2_u32(and_xor(wa, 0x00FF00FFu, 0x00800080u), 0x00800080u);
+                const uint32_t A1 = hsub2_u32(and_xor(wb, 0x00FF00FFu, 0x00800080u), 0x00800080u);
+                const uint32_t A2 = hsub2_u32(and_xor(wa >> 8, 0x00FF00FFu, 0x00800080u), 0x00800080u);
+                const uint32_t A3 = hsub2_u32(and_xor(wb >> 8, 0x00FF00FFu, 0x00800080u), 0x00800080u);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     uint2 bv = lds64c(L.tokb[nt] + imgb0 + i * 64 + h * 32 + t * 8);
@@ -422,8 +409,7 @@ __device__ __forceinline__ void q8_run(const Lane<NT>& L, const QmvParams& p, ui
             }
         }
         if (i % S == S - 1 || i == RUN - 1) {
-            // epilogue: y += 2^24 d (D - X) per column's block (D = 2^-24
-            // sum (q + 128) x, X = 2^-17 sum x)
+            // epilogue: y += 2^24 d D per column's block (D = 2^-24 sum q x)
             const int i0 = i - (i % S);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
@@ -435,8 +421,7 @@ __device__ __forceinline__ void q8_run(const Lane<NT>& L, const QmvParams& p, ui
                     if (ib < nvalid && ib <= i) {
                         const uint32_t row = (e >> 1) ? rowB : rowA;
                         const float d = h16(ldsu16c(row + (lb0 + ib) * 34)) * kTwo24;
-                        const float X = __uint_as_float(lds32c(xsb0 + (tok * p.scb + ib) * 4));
-                        acc[nt][e] = fmaf(d, D[nt][e] - X, acc[nt][e]);
+                        acc[nt][e] = fmaf(d, D[nt][e], acc[nt][e]);
                     }
                 }
             }
@@ -448,7 +433,7 @@ __device__ __forceinline__ void q8_run(const Lane<NT>& L, const QmvParams& p, ui
 // block of 16 rows.  Two warps share a block, one half each.
 template <int S, int NT>
 __device__ __forceinline__ void q6k_half(const Lane<NT>& L, const QmvParams& p, uint32_t rowA, uint32_t rowB,
-                                         bool odd, int h, uint32_t imgb, uint32_t xsb, uint32_t zero_addr,
+                                         bool odd, int h, uint32_t imgb, uint32_t zero_addr,
                                          float (&acc)[NT][4]) {
     const int t = L.t;
     const float dA = h16(ldsu16c(rowA + 208));
@@ -484,11 +469,13 @@ __device__ __forceinline__ void q6k_half(const Lane<NT>& L, const QmvParams& p, 
         // with B = x/16, high nibble (tq >= 2) -> 16 c 2^-24 with B = x/256
         const uint32_t mlo = tq < 2 ? 0x000F000Fu : 0x00F000F0u;
         const uint32_t L0 = la & mlo, L1 = lb & mlo, L2 = (la >> 8) & mlo, L3 = (lb >> 8) & mlo;
-        // high 2 bits h, left at bits 2tq..2tq+1 of each byte: 4^tq h 2^-24,
-        // with B = x / 4^tq (all B scalings are exact powers of two, none
-        // above 1).  The two MMAs sum 2^-24 c6 x / 16.
-        const uint32_t mhi = 0x00030003u << (2 * tq);
-        const uint32_t H0 = ha & mhi, H1 = hb & mhi, H2 = (ha >> 8) & mhi, H3 = (hb >> 8) & mhi;
+        // high 2 bits h, left at bits 2tq..2tq+1 of each byte, less 2 (the
+        // code offset 32 = 16 2): 4^tq (h - 2) 2^-24 (exact), with B =
+        // x / 4^tq (all B scalings are exact powers of two, none above 1).
+        // The two MMAs sum 2^-24 (c6 - 32) x / 16.
+        const uint32_t mhi = 0x00030003u << (2 * tq), off = 0x00020002u << (2 * tq);
+        const uint32_t H0 = hsub2_u32(ha & mhi, off), H1 = hsub2_u32(hb & mhi, off);
+        const uint32_t H2 = hsub2_u32((ha >> 8) & mhi, off), H3 = hsub2_u32((hb >> 8) & mhi, off);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const uint32_t a = L.tokb[nt] + imgb + j * 64 + t * 8;
@@ -512,13 +499,12 @@ __device__ __forceinline__ void q6k_half(const Lane<NT>& L, const QmvParams& p, 
                     int tok, slot;
                     col_info<S, NT>(nt, 2 * t + (e & 1), p.m, tok, slot);
                     const int jj = j0 + slot;
-                    // sum (c - 32) x = 16 2^24 (D - X), X from the image build
+                    // sum (c - 32) x = 16 2^24 D
                     const uint32_t row = (e >> 1) ? rowB : rowA;
                     const float dr = (e >> 1) ? dB : dA;
                     const int sc = ldss8c(row + 192 + jj);
                     const float s = 268435456.0f * __fmul_rn(dr, static_cast<float>(sc));   // 16 2^24 d sc
-                    const float X = __uint_as_float(lds32c(xsb + (tok * p.scb * 16 + jj) * 4));
-                    acc[nt][e] = fmaf(s, D[nt][e] - X, acc[nt][e]);
+                    acc[nt][e] = fmaf(s, D[nt][e], acc[nt][e]);
                 }
             }
         }
@@ -705,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const QmvParams p) {
                 if (xm[tid] >= 0x7F80u) atomicOr(p.status, KQ_DEV_X_RANGE);   // Inf or NaN
                 xinv[tid] = exp2_int(-xscale_exp(xm[tid], C::XT));
             }
-            if (!*abort_flag) build_image<QT>(p, blk0, nbsc, sbase + p.off_img, sbase + p.off_x, xm);
+            if (!*abort_flag) build_image<QT>(p, blk0, nbsc, sbase + p.off_img, xm);
             asm volatile("bar.sync 1, %0;" ::"r"(kCWarps * 32));
             if (*abort_flag) continue;
             for (int g = 0; g < nrg; ++g, ++it) {
@@ -736,15 +722,14 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_kernel(const QmvParams p) {
                         for (int it2 = warp; it2 < 2 * nb; it2 += kCWarps) {
                             const int lb = it2 >> 1, lbi = bl + lb;
                             q6k_half<S, NT>(L, p, rowA + lb * 210, rowB + lb * 210, (lb & 1) != 0, it2 & 1,
-                                            lbi * 1024, sbase + p.off_x + lbi * 64, zero_addr, acc);
+                                            lbi * 1024, zero_addr, acc);
                         }
                     } else {
                         // runs of 4 consecutive blocks
                         for (int lb0 = 4 * warp; lb0 < nb; lb0 += 4 * kCWarps) {
                             const int nv = nb - lb0 < 4 ? nb - lb0 : 4;
                             const int lbi = bl + lb0;
-                            q8_run<S, NT, 4>(L, p, rowA, rowB, lb0, nv, lbi * 64, sbase + p.off_x + lbi * 4,
-                                             zero_addr, acc);
+                            q8_run<S, NT, 4>(L, p, rowA, rowB, lb0, nv, lbi * 64, zero_addr, acc);
                         }
                     }
                     __syncwarp();
@@ -805,7 +790,7 @@ int launch_codec(const void* w, int64_t n, int64_t k, const uint16_t* x, int m, 
     // blocks), then more stages, subject to the shared-memory budget that the
     // activation image, the partial-sum buffers and the barriers leave.
     int ns = 0, g = 0, scb = 0, rs = 0;
-    uint32_t tokstride = 0, off_img = 0, off_x = 0, off_pbuf = 0, off_racc = 0, total = 0;
+    uint32_t tokstride = 0, off_img = 0, off_pbuf = 0, off_racc = 0, total = 0;
     int64_t best = -1;
     const int gmax = cdiv(p.nblk, C::GA) * C::GA;
     for (int ns_try = 4; ns_try >= 2; --ns_try) {
@@ -818,8 +803,7 @@ int launch_codec(const void* w, int64_t n, int64_t k, const uint16_t* x, int m, 
             for (int scb_try = scb_full; scb_try >= g_try; scb_try -= g_try) {
                 const uint32_t base = scb_try * C::IMG;
                 const uint32_t ts = base + ((32u - (base & 127u)) & 127u);
-                const uint32_t ox = oi + m * ts;
-                const uint32_t op = (ox + m * scb_try * C::XS * 4 + 15) & ~15u;
+                const uint32_t op = (oi + m * ts + 15) & ~15u;
                 const uint32_t orc = op + pbuf_bytes;
                 const uint32_t tot = orc + (scb_try < scb_full ? nrg * kRows * 16 * 4 : 0);
                 if (tot > static_cast<uint32_t>(optin)) continue;
@@ -827,7 +811,7 @@ int launch_codec(const void* w, int64_t n, int64_t k, const uint16_t* x, int m, 
                 if (inflight > best) {
                     best = inflight;
                     ns = ns_try; g = g_try; scb = scb_try; rs = rs_try;
-                    tokstride = ts; off_img = oi; off_x = ox; off_pbuf = op; off_racc = orc; total = tot;
+                    tokstride = ts; off_img = oi; off_pbuf = op; off_racc = orc; total = tot;
                 }
                 break;
             }
@@ -847,7 +831,6 @@ int launch_codec(const void* w, int64_t n, int64_t k, const uint16_t* x, int m, 
     p.scb = scb;
     p.tokstride = tokstride;
     p.off_img = off_img;
-    p.off_x = off_x;
     p.off_pbuf = off_pbuf;
     p.off_racc = off_racc;
     auto launch = [&](auto kernel) {

@@ -137,6 +137,15 @@ __device__ __forceinline__ uint32_t vand_xor(uint32_t a, uint32_t b, uint32_t c)
     asm volatile("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
     return d;
 }
+// a - b per binary16 half.  On codes held as subnormals (integer multiples
+// of 2^-24 below 2^-14 in magnitude) the difference is exact: it centres a
+// code on the format's offset before the MMA, so that a large activation
+// meets a zero weight as an exact zero.
+__device__ __forceinline__ uint32_t vhsub2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm volatile("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
 __device__ __forceinline__ uint32_t vhfma2(uint32_t a, uint32_t b, uint32_t c) {
     uint32_t d;
     asm volatile("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
@@ -222,6 +231,25 @@ __device__ __forceinline__ uint32_t hpair(__half lo, __half hi) {
     return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
 }
 
+// Scales of the 32-value blocks (q8_0, q4_0), one thread per (token, block):
+// 2^s from the block's largest |x| (its scaled values below 2^(xt+1)), stored
+// as 2^-s at 4 bytes per block in block order.  Returns whether this thread
+// met a non-finite activation.
+__device__ __forceinline__ bool block_scales(const SP& p, uint32_t sb, int xt) {
+    bool bad = false;
+    for (int e = threadIdx.x; e < p.m * p.nblk; e += kCW * 32) {
+        const int tok = e / p.nblk, blk = e % p.nblk;
+        const uint32_t xs = xaddr(p, sb, tok, 32 * blk);
+        uint32_t mx = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) mx = absmax8_bf16(mx, lds128(xs + 16 * c));
+        mx = max(mx & 0xFFFFu, mx >> 16);
+        bad |= mx >= 0x7F80u;
+        sts32(sb + p.off_xs + tok * p.xs_tok + 4 * blk, __float_as_uint(exp2_int(-xscale_exp(mx, xt))));
+    }
+    return bad;
+}
+
 // Lane roles in the m16n8k16 fragments (lane = 4 g + t): A rows g and g+8,
 // k-slots 2t, 2t+1, 2t+8, 2t+9; B column g; D columns 2t, 2t+1.
 struct Lane {
@@ -242,6 +270,7 @@ struct Q8 {
     static constexpr int kXT = 14;
     // the build needs every block's scale before it writes the image
     static constexpr bool kTwoPhase = true;
+    static constexpr bool kSplit = false;
 
     // rowA/rowB: shared address of the item (8 blocks) in rows g / g+8;
     // gi: global item index (block 8 gi).
@@ -278,30 +307,29 @@ struct Q8 {
                 dO[1] = h2f(wb >> 16) * kTwo24;
             }
             const int par = mu >= 9 ? 1 : 0;
-            // byte ^ 0x80 = 128 + code as a binary16 subnormal: (128 + code) 2^-24
-            const uint32_t A0 = vand_xor(wa, 0x00FF00FFu, 0x00800080u);
-            const uint32_t A1 = vand_xor(wb, 0x00FF00FFu, 0x00800080u);
-            const uint32_t A2 = vand_xor(wa >> 8, 0x00FF00FFu, 0x00800080u);
-            const uint32_t A3 = vand_xor(wb >> 8, 0x00FF00FFu, 0x00800080u);
+            // byte ^ 0x80 = 128 + code as a binary16 subnormal, less 128 2^-24:
+            // the signed code as the subnormal code 2^-24
+            const uint32_t A0 = vhsub2(vand_xor(wa, 0x00FF00FFu, 0x00800080u), 0x00800080u);
+            const uint32_t A1 = vhsub2(vand_xor(wb, 0x00FF00FFu, 0x00800080u), 0x00800080u);
+            const uint32_t A2 = vhsub2(vand_xor(wa >> 8, 0x00FF00FFu, 0x00800080u), 0x00800080u);
+            const uint32_t A3 = vhsub2(vand_xor(wb >> 8, 0x00FF00FFu, 0x00800080u), 0x00800080u);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const uint2 bv = lds64(bb[nt][par] + 32 * mu);
                 mma_f16(D[nt][mu & 1], A0, A1, A2, A3, bv.x, bv.y);
             }
         }
-        // D = 2^-24 sum (128 + code) a with a = x 2^s (s per token and block);
-        // y += 2^(24-s) d (D - 2^-17 X), X = sum a, for columns 2t (even
-        // block) and 2t+1 (odd block)
+        // D = 2^-24 sum code a with a = x 2^s (s per token and block):
+        // y += 2^(24-s) d D for columns 2t (even block) and 2t+1 (odd block)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            const uint4 xv = lds128(sb + p.off_xs + nt * p.xs_tok + 16 * (4 * gi + t));
-            const float X[2] = {__uint_as_float(xv.x), __uint_as_float(xv.y)};
-            const float iv[2] = {__uint_as_float(xv.z), __uint_as_float(xv.w)};
+            const uint2 xv = lds64(sb + p.off_xs + nt * p.xs_tok + 8 * (4 * gi + t));
+            const float iv[2] = {__uint_as_float(xv.x), __uint_as_float(xv.y)};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int r = e >> 1, odd = e & 1;
                 const float Ds = D[nt][0][e] + D[nt][1][e];
-                acc[2 * nt + r] = fmaf((odd ? dO[r] : dE[r]) * iv[odd], Ds - X[odd], acc[2 * nt + r]);
+                acc[2 * nt + r] = fmaf((odd ? dO[r] : dE[r]) * iv[odd], Ds, acc[2 * nt + r]);
             }
         }
     }
@@ -320,41 +348,10 @@ struct Q8 {
     }
 
     // Phase 1, one thread per (token, block): the block's scale 2^s from its
-    // largest |x|, then X = 2^-17 (= 128 2^-24) times the sum of the block's
-    // 32 binary16 operands and 2^-s, stored as {X_even, X_odd, 2^-s_even,
-    // 2^-s_odd} per block pair.  Returns whether this thread met a
-    // non-finite activation.
+    // largest |x|, stored as 2^-s (4 bytes per block, in block order).
+    // Returns whether this thread met a non-finite activation.
     static __device__ bool build_scales(const SP& p, uint32_t sb, int64_t xoff) {
-        bool bad = false;
-        for (int e = threadIdx.x; e < p.m * p.nblk; e += kCW * 32) {
-            const int tok = e / p.nblk, blk = e % p.nblk;
-            const uint32_t xs = xaddr(p, sb, tok, 32 * blk);
-            uint4 v[4];
-            uint32_t mx = 0;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                v[c] = lds128(xs + 16 * c);
-                mx = absmax8_bf16(mx, v[c]);
-            }
-            mx = max(mx & 0xFFFFu, mx >> 16);
-            bad |= mx >= 0x7F80u;
-            const int se = xscale_exp(mx, kXT);
-            const float S = exp2_int(se);
-            float X = 0.f;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint32_t wv[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    X += __half2float(hx(bf16lo_to_f32(wv[q]), S));
-                    X += __half2float(hx(bf16hi_to_f32(wv[q]), S));
-                }
-            }
-            const uint32_t xo = sb + p.off_xs + tok * p.xs_tok + 16 * (blk >> 1) + 4 * (blk & 1);
-            sts32(xo, __float_as_uint(X * 7.62939453125e-06f));
-            sts32(xo + 8, __float_as_uint(exp2_int(-se)));
-        }
-        return bad;
+        return block_scales(p, sb, kXT);
     }
     // Phase 2: image entry (item, mu, t') = binary16 of the scaled activations
     // of the 4 raw bytes at offset 272 item + 68 t' + 4 mu of a row, as
@@ -372,12 +369,137 @@ struct Q8 {
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
                 const int R = R0 + b, blk = R / 34, o = R - 34 * blk;
-                const uint32_t ib = lds32(sb + p.off_xs + tok * p.xs_tok + 16 * (blk >> 1) + 4 * (blk & 1) + 8);
+                const uint32_t ib = lds32(sb + p.off_xs + tok * p.xs_tok + 4 * blk);
                 const float S = __uint_as_float(0x7F000000u - ib);
                 h[b] = o >= 2 ? hx(xval(p, sb, tok, 32 * blk + o - 2), S) : __float2half_rn(0.f);
             }
             sts64(sb + p.off_img + tok * p.img_tok + it * kItemImg + mu * 32 + tt * 8, hpair(h[0], h[2]),
                   hpair(h[1], h[3]));
+        }
+        return false;
+    }
+};
+
+// ===========================================================================
+// q4_0
+// ===========================================================================
+// q4_0 (18 bytes per 32 values): fp16 d, then 16 bytes whose low nibbles are
+// values 0..15 and high nibbles values 16..31; y = d (code - 8).  Item = 16
+// rows x 8 blocks (144 bytes of a row).  Lane t owns blocks 2t and 2t+1 (36
+// bytes, word aligned) and feeds two MMAs per word: the low nibbles as
+// binary16 subnormals less 8 2^-24 ((code - 8) 2^-24, exact) against x, the
+// high nibbles in place less 128 2^-24 (16 (code - 8) 2^-24) against x/16.
+// Words 0..4 hold the even block (its d in bytes 0..1, the odd block's d in
+// bytes 18..19: zero activations), words 5..8 the odd block, so MMA column
+// 2t + parity collects exactly lane t's block of that parity.
+template <int NT>
+struct Q40 {
+    static constexpr int kVPB = 32, kBPB = 18;
+    static constexpr int kItemBlocks = 8;
+    static constexpr uint32_t kItemImg = 18 * 32;   // 9 words x (low, high) per item and token
+    static constexpr uint32_t kZero = kItemImg;
+    static constexpr int kAccPerLane = 2 * NT;
+    static constexpr int kXT = 14;
+    static constexpr bool kTwoPhase = true;
+    static constexpr bool kSplit = false;
+
+    static __device__ __forceinline__ void item(const SP& p, uint32_t sb, const Lane& L, uint32_t rowA,
+                                                uint32_t rowB, int gi, float (&acc)[2 * NT]) {
+        const int t = L.t;
+        const bool act = (L.g >> 1) == t;
+        uint32_t bb[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const uint32_t img = sb + p.off_img + nt * p.img_tok + gi * kItemImg + 8 * t;
+            const uint32_t zero = sb + p.off_zero + 8 * t;
+            bb[nt][0] = (act && (L.g & 1) == 0) ? img : zero;
+            bb[nt][1] = (act && (L.g & 1) == 1) ? img : zero;
+        }
+        float D[NT][2][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) D[nt][c][e] = 0.f;
+        const uint32_t a0 = rowA + 36 * t, b0 = rowB + 36 * t;
+        float dE[2], dO[2];
+#pragma unroll
+        for (int mu = 0; mu < 9; ++mu) {
+            const uint32_t wa = lds32(a0 + 4 * mu), wb = lds32(b0 + 4 * mu);
+            if (mu == 0) {   // the even block's d: bytes 0..1 of the span
+                dE[0] = h2f(wa & 0xffff) * kTwo24;
+                dE[1] = h2f(wb & 0xffff) * kTwo24;
+            }
+            if (mu == 4) {   // the odd block's d: bytes 18..19
+                dO[0] = h2f(wa >> 16) * kTwo24;
+                dO[1] = h2f(wb >> 16) * kTwo24;
+            }
+            const int par = mu >= 5 ? 1 : 0;
+            const uint32_t wa8 = wa >> 8, wb8 = wb >> 8;
+            // low nibbles as subnormals (c - 8) 2^-24, high nibbles in place:
+            // 16 (c - 8) 2^-24
+            const uint32_t L0 = vhsub2(vand_or(wa, 0x000F000Fu, 0u), 0x00080008u);
+            const uint32_t L1 = vhsub2(vand_or(wb, 0x000F000Fu, 0u), 0x00080008u);
+            const uint32_t L2 = vhsub2(vand_or(wa8, 0x000F000Fu, 0u), 0x00080008u);
+            const uint32_t L3 = vhsub2(vand_or(wb8, 0x000F000Fu, 0u), 0x00080008u);
+            const uint32_t H0 = vhsub2(vand_or(wa, 0x00F000F0u, 0u), 0x00800080u);
+            const uint32_t H1 = vhsub2(vand_or(wb, 0x00F000F0u, 0u), 0x00800080u);
+            const uint32_t H2 = vhsub2(vand_or(wa8, 0x00F000F0u, 0u), 0x00800080u);
+            const uint32_t H3 = vhsub2(vand_or(wb8, 0x00F000F0u, 0u), 0x00800080u);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const uint2 bl = lds64(bb[nt][par] + 64 * mu), bh = lds64(bb[nt][par] + 64 * mu + 32);
+                mma_f16(D[nt][mu & 1], L0, L1, L2, L3, bl.x, bl.y);
+                mma_f16(D[nt][mu & 1], H0, H1, H2, H3, bh.x, bh.y);
+            }
+        }
+        // D = 2^-24 sum (c - 8) a (a = x 2^s, the high half against
+        // x 2^s / 16): y += 2^(24-s) d D
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const uint2 xv = lds64(sb + p.off_xs + nt * p.xs_tok + 8 * (4 * gi + t));
+            const float iv[2] = {__uint_as_float(xv.x), __uint_as_float(xv.y)};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = e >> 1, odd = e & 1;
+                const float Ds = D[nt][0][e] + D[nt][1][e];
+                acc[2 * nt + r] = fmaf((odd ? dO[r] : dE[r]) * iv[odd], Ds, acc[2 * nt + r]);
+            }
+        }
+    }
+
+    static __device__ __forceinline__ void store_part(const SP& p, const Lane& L, float (&acc)[2 * NT], float* part) {
+        Q8<NT>::store_part(p, L, acc, part);
+    }
+
+    // Phase 1: the block scales (stored as 2^-s per block).
+    static __device__ bool build_scales(const SP& p, uint32_t sb, int64_t xoff) {
+        return block_scales(p, sb, kXT);
+    }
+    // Phase 2: image entries (item, mu, low / high, t') = binary16 of the
+    // scaled activations of the 4 raw bytes at offset 144 item + 36 t' + 4 mu
+    // of a row, as (byte0, byte2 | byte1, byte3): the low nibble's value
+    // (x 2^s) or the high nibble's (x 2^s / 16); d bytes get 0.
+    static __device__ bool build(const SP& p, uint32_t sb, int64_t xoff) {
+        const int items = p.nblk / 8;
+        const int per_tok = items * 9 * 4;
+        for (int e = threadIdx.x; e < p.m * per_tok; e += kCW * 32) {
+            const int tok = e / per_tok, rem = e % per_tok;
+            const int it = rem / 36, mu = (rem % 36) >> 2, tt = rem & 3;
+            const int R0 = it * 144 + 36 * tt + 4 * mu;
+            __half lo[4], hi[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int R = R0 + b, blk = R / 18, o = R - 18 * blk;
+                const uint32_t ib = lds32(sb + p.off_xs + tok * p.xs_tok + 4 * blk);
+                const float S = __uint_as_float(0x7F000000u - ib);
+                lo[b] = o >= 2 ? hx(xval(p, sb, tok, 32 * blk + o - 2), S) : __float2half_rn(0.f);
+                hi[b] = o >= 2 ? hx(xval(p, sb, tok, 32 * blk + 14 + o), S * 0.0625f) : __float2half_rn(0.f);
+            }
+            const uint32_t dst = sb + p.off_img + tok * p.img_tok + it * kItemImg + mu * 64 + tt * 8;
+            sts64(dst, hpair(lo[0], lo[2]), hpair(lo[1], lo[3]));
+            sts64(dst + 32, hpair(hi[0], hi[2]), hpair(hi[1], hi[3]));
         }
         return false;
     }
@@ -404,6 +526,7 @@ struct Q6 {
     // normal binary16 numbers down to 2^-22 of the run's largest magnitude
     static constexpr int kXT = 14;
     static constexpr bool kTwoPhase = false;
+    static constexpr bool kSplit = false;
 
     // Word at shared address a: 4-byte aligned (MODE 0), 2 bytes past a
     // 4-byte boundary (MODE 1), or either, per thread (MODE 2: rows at their
@@ -422,8 +545,8 @@ struct Q6 {
     // sub-blocks j = 8h + 2q + lh.  Its 6-bit codes come from nibble q >> 1 of
     // ql[64h + 32 (q & 1) + l] and bits 2q of qh[32h + l].  For each pass
     // qp = q & 1 and word k the lane feeds two MMAs: the low nibbles (q = qp,
-    // 1024 + c6, activations x/16) into column 2t and the high nibbles
-    // (q = qp + 2, 1024 + 16 c6, x/256) into column 2t + 1.  The four lanes of
+    // c6 - 32 as a subnormal, activations x/16) into column 2t and the high
+    // nibbles (q = qp + 2, 16 (c6 - 32), x/256) into column 2t + 1.  The four lanes of
     // a row read their words in the order (k + t) mod 4, which spreads them over
     // all 32 banks; the activation image follows the same order.
     template <int ODD>
@@ -476,16 +599,17 @@ struct Q6 {
                 const uint32_t wa8 = wa >> 8, wb8 = wb >> 8;
                 const uint32_t sa02 = ha[k] << sh, sa13 = ha[k] >> (8 - sh);
                 const uint32_t sb02 = hb[k] << sh, sb13 = hb[k] >> (8 - sh);
-                // low nibble + field qp -> c6 as a subnormal (c6 2^-24)
-                const uint32_t L0 = vbitsel(wa, vand_or(sa02, 0x00300030u, 0u), 0x000F000Fu);
-                const uint32_t L1 = vbitsel(wb, vand_or(sb02, 0x00300030u, 0u), 0x000F000Fu);
-                const uint32_t L2 = vbitsel(wa8, vand_or(sa13, 0x00300030u, 0u), 0x000F000Fu);
-                const uint32_t L3 = vbitsel(wb8, vand_or(sb13, 0x00300030u, 0u), 0x000F000Fu);
-                // high nibble + field qp + 2 -> 16 c6 as a subnormal
-                const uint32_t H0 = vbitsel(wa, vand_or(sa02, 0x03000300u, 0u), 0x00F000F0u);
-                const uint32_t H1 = vbitsel(wb, vand_or(sb02, 0x03000300u, 0u), 0x00F000F0u);
-                const uint32_t H2 = vbitsel(wa8, vand_or(sa13, 0x03000300u, 0u), 0x00F000F0u);
-                const uint32_t H3 = vbitsel(wb8, vand_or(sb13, 0x03000300u, 0u), 0x00F000F0u);
+                // low nibble + field qp -> c6 as a subnormal (c6 2^-24), less
+                // 32 2^-24: the centred code, exact
+                const uint32_t L0 = vhsub2(vbitsel(wa, vand_or(sa02, 0x00300030u, 0u), 0x000F000Fu), 0x00200020u);
+                const uint32_t L1 = vhsub2(vbitsel(wb, vand_or(sb02, 0x00300030u, 0u), 0x000F000Fu), 0x00200020u);
+                const uint32_t L2 = vhsub2(vbitsel(wa8, vand_or(sa13, 0x00300030u, 0u), 0x000F000Fu), 0x00200020u);
+                const uint32_t L3 = vhsub2(vbitsel(wb8, vand_or(sb13, 0x00300030u, 0u), 0x000F000Fu), 0x00200020u);
+                // high nibble + field qp + 2 -> 16 c6 as a subnormal, less 512 2^-24
+                const uint32_t H0 = vhsub2(vbitsel(wa, vand_or(sa02, 0x03000300u, 0u), 0x00F000F0u), 0x02000200u);
+                const uint32_t H1 = vhsub2(vbitsel(wb, vand_or(sb02, 0x03000300u, 0u), 0x00F000F0u), 0x02000200u);
+                const uint32_t H2 = vhsub2(vbitsel(wa8, vand_or(sa13, 0x03000300u, 0u), 0x00F000F0u), 0x02000200u);
+                const uint32_t H3 = vhsub2(vbitsel(wb8, vand_or(sb13, 0x03000300u, 0u), 0x00F000F0u), 0x02000200u);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const uint2 bl = lds64(bb[nt][0] + 32 * (8 * qp + k));
@@ -494,22 +618,19 @@ struct Q6 {
                     mma_f16(D[k & 1][nt], H0, H1, H2, H3, bh.x, bh.y);
                 }
             }
-            // column 2t: D = 2^-24 sum c a with a = x 2^s/16, column 2t + 1:
-            // D = 2^-24 sum 16 c a with a = x 2^s/256 (s per 16-value run);
-            // both are 2^-24 2^s sum c x / 16, and sum (c - 32) x =
-            // 16 2^24 2^-s (D - X) with X the stored offset sum (2^-19 sum a,
-            // resp. 2^-15 sum a): y += 2^28 d sc_j 2^-s (D - X)
+            // column 2t: D = 2^-24 sum (c - 32) a with a = x 2^s/16, column
+            // 2t + 1: D = 2^-24 sum 16 (c - 32) a with a = x 2^s/256 (s per
+            // 16-value run); both are 2^-24 2^s sum (c - 32) x / 16:
+            // y += 2^28 d sc_j 2^-s D
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                const uint4 xv = lds128(sb + p.off_xs + nt * p.xs_tok + ((gb * 4 + t) * 2 + qp) * 16);
-                const float X[2] = {__uint_as_float(xv.x), __uint_as_float(xv.y)};
-                const float iv[2] = {__uint_as_float(xv.z), __uint_as_float(xv.w)};
+                const uint2 xv = lds64(sb + p.off_xs + nt * p.xs_tok + ((gb * 4 + t) * 2 + qp) * 8);
+                const float iv[2] = {__uint_as_float(xv.x), __uint_as_float(xv.y)};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int r = e >> 1, c = e & 1;
                     const float Ds = D[0][nt][e] + D[1][nt][e];
-                    acc[2 * nt + r] =
-                        fmaf(__fmul_rn(d16[r], sc[r][qp + 2 * c]) * iv[c], Ds - X[c], acc[2 * nt + r]);
+                    acc[2 * nt + r] = fmaf(__fmul_rn(d16[r], sc[r][qp + 2 * c]) * iv[c], Ds, acc[2 * nt + r]);
                 }
             }
         }
@@ -534,11 +655,9 @@ struct Q6 {
     // s): q = qp + 2s, values v = 128h + 32q + 16 lh + l, l = 0..15.  Its
     // scale 2^e puts the run's largest |x| at 2^14; image entry (block,
     // E = 8 qp + 4 s + k, t') = binary16 of x[v] 2^e / 16 (s = 0) or / 256
-    // (s = 1) for l = 4 ((k + t') mod 4) + {0, 2 | 1, 3}; the run's
-    // {X_s=0, X_s=1, 2^-e_s=0, 2^-e_s=1} per (block, t', qp), X = the sum of
-    // the 16 binary16 operands times 2^-19 (s = 0) or 2^-15 (s = 1): 32 2^-24
-    // and 32 16 2^-24, the code offset in the MMA's units.  Returns whether
-    // this thread met a non-finite activation.
+    // (s = 1) for l = 4 ((k + t') mod 4) + {0, 2 | 1, 3}; the runs'
+    // {2^-e_s=0, 2^-e_s=1} per (block, t', qp).  Returns whether this thread
+    // met a non-finite activation.
     static __device__ bool build(const SP& p, uint32_t sb, int64_t xoff) {
         bool bad = false;
         const int per_tok = p.nblk * 16;
@@ -556,32 +675,36 @@ struct Q6 {
             const float sc = exp2_int(se) * (sl ? 0.00390625f : 0.0625f);
             const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
             __half hv[16];
-            float X = 0.f;
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 hv[2 * u] = hx(bf16lo_to_f32(wv[u]), sc);
                 hv[2 * u + 1] = hx(bf16hi_to_f32(wv[u]), sc);
-                X += __half2float(hv[2 * u]) + __half2float(hv[2 * u + 1]);
             }
             const uint32_t img = sb + p.off_img + tok * p.img_tok + blk * kBlkImg + (8 * qp + 4 * sl) * 32 + tt * 8;
             // values 4g .. 4g+3 go to entry k = (g - t') mod 4
 #pragma unroll
             for (int g = 0; g < 4; ++g)
                 sts64(img + ((g - tt) & 3) * 32, hpair(hv[4 * g], hv[4 * g + 2]), hpair(hv[4 * g + 1], hv[4 * g + 3]));
-            const uint32_t xo = sb + p.off_xs + tok * p.xs_tok + ((blk * 4 + tt) * 2 + qp) * 16 + 4 * sl;
-            sts32(xo, __float_as_uint(X * (sl ? 3.0517578125e-05f : 1.9073486328125e-06f)));   // 2^-15, 2^-19
-            sts32(xo + 8, __float_as_uint(exp2_int(-se)));
+            sts32(sb + p.off_xs + tok * p.xs_tok + ((blk * 4 + tt) * 2 + qp) * 8 + 4 * sl,
+                  __float_as_uint(exp2_int(-se)));
         }
         return bad;
     }
 };
 
 // ===========================================================================
-// q4_K
+// q4_K (and q5_K: FIVE)
 // ===========================================================================
-template <int NT>
+// q5_K (176 B) has q4_K's header (d, dmin, packed 6-bit scales and mins), then
+// qh[32], then the 4-bit codes at byte 48: value 64c + l takes bit 2c of
+// qh[l] as its fifth bit, value 64c + 32 + l bit 2c + 1; q = 0..31.  The
+// image, the scales and the min term are q4_K's; only the code assembly
+// differs: 1024 + q (low) and 1024 + 16 q (high) still hold q sc exactly
+// after the scale FMA (q sc <= 1953 < 2048).
+template <int NT, bool FIVE = false>
 struct Q4 {
-    static constexpr int kVPB = 256, kBPB = 144;
+    static constexpr int kVPB = 256, kBPB = FIVE ? 176 : 144;
+    static constexpr bool kSplit = true;   // the K-split (cluster) kernel serves it
     static constexpr int kItemBlocks = 1;
     static constexpr uint32_t kBlkImg = 544;
     static constexpr uint32_t kZero = kBlkImg;
@@ -601,8 +724,21 @@ struct Q4 {
             bb[nt] = tok < p.m ? sb + p.off_img + tok * p.img_tok + gb * kBlkImg + 8 * t : sb + p.off_zero + 8 * t;
         }
         const uint4 hA = lds128(rowA), hB = lds128(rowB);
-        const uint4 qA0 = lds128(rowA + 16 + 32 * t), qA1 = lds128(rowA + 32 + 32 * t);
-        const uint4 qB0 = lds128(rowB + 16 + 32 * t), qB1 = lds128(rowB + 32 + 32 * t);
+        constexpr uint32_t kQs = FIVE ? 48 : 16;   // first code byte
+        const uint4 qA0 = lds128(rowA + kQs + 32 * t), qA1 = lds128(rowA + kQs + 16 + 32 * t);
+        const uint4 qB0 = lds128(rowB + kQs + 32 * t), qB1 = lds128(rowB + kQs + 16 + 32 * t);
+        uint32_t fA[8], fB[8];   // q5_K: qh[4u .. 4u+3] >> 2t (the lane's two bits at bits 0, 1 of each byte)
+        if constexpr (FIVE) {
+            const uint4 hA0 = lds128(rowA + 16), hA1 = lds128(rowA + 32);
+            const uint4 hB0 = lds128(rowB + 16), hB1 = lds128(rowB + 32);
+            const uint32_t ha[8] = {hA0.x, hA0.y, hA0.z, hA0.w, hA1.x, hA1.y, hA1.z, hA1.w};
+            const uint32_t hb[8] = {hB0.x, hB0.y, hB0.z, hB0.w, hB1.x, hB1.y, hB1.z, hB1.w};
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                fA[u] = ha[u] >> (2 * t);
+                fB[u] = hb[u] >> (2 * t);
+            }
+        }
         // 6-bit scale/min codes of sub-blocks 2t, 2t+1 as (code_2t, code_2t+1)
         // in bits 0..5 / 16..21.  t < 2: sc = s[j] & 63, m = s[j+4] & 63;
         // t >= 2 (j >= 4): sc = (s[j+4] & 15) | (s[j-4] >> 6) << 4,
@@ -646,16 +782,33 @@ struct Q4 {
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const uint32_t a = wA[u], b = wB[u], a8 = a >> 8, b8 = b >> 8;
-            // low nibbles: (1024 + q) sc - 1024 sc = q sc exactly
-            const uint32_t a0 = vhfma2(vand_or(a, 0x000F000Fu, kH1024), S_lo[0], B_lo[0]);
-            const uint32_t a1 = vhfma2(vand_or(b, 0x000F000Fu, kH1024), S_lo[1], B_lo[1]);
-            const uint32_t a2 = vhfma2(vand_or(a8, 0x000F000Fu, kH1024), S_lo[0], B_lo[0]);
-            const uint32_t a3 = vhfma2(vand_or(b8, 0x000F000Fu, kH1024), S_lo[1], B_lo[1]);
-            // high nibbles: (1024 + 16 q) sc / 16 - 64 sc = q sc exactly
-            const uint32_t c0 = vhfma2(vand_or(a, 0x00F000F0u, kH1024), S_hi[0], B_hi[0]);
-            const uint32_t c1 = vhfma2(vand_or(b, 0x00F000F0u, kH1024), S_hi[1], B_hi[1]);
-            const uint32_t c2 = vhfma2(vand_or(a8, 0x00F000F0u, kH1024), S_hi[0], B_hi[0]);
-            const uint32_t c3 = vhfma2(vand_or(b8, 0x00F000F0u, kH1024), S_hi[1], B_hi[1]);
+            uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
+            if constexpr (FIVE) {
+                // fifth bit: bit 0 (low codes) / bit 1 (high codes) of each
+                // byte of f moved to bit 4 / bit 8 of its 16-bit lane
+                const uint32_t fa = fA[u], fb = fB[u];
+                // low nibbles: 1024 + nib + 16 h, times sc, minus 1024 sc -> q sc exactly
+                a0 = vhfma2(vbitsel(a, vand_or(fa << 4, 0x00100010u, kH1024), 0x000F000Fu), S_lo[0], B_lo[0]);
+                a1 = vhfma2(vbitsel(b, vand_or(fb << 4, 0x00100010u, kH1024), 0x000F000Fu), S_lo[1], B_lo[1]);
+                a2 = vhfma2(vbitsel(a8, vand_or(fa >> 4, 0x00100010u, kH1024), 0x000F000Fu), S_lo[0], B_lo[0]);
+                a3 = vhfma2(vbitsel(b8, vand_or(fb >> 4, 0x00100010u, kH1024), 0x000F000Fu), S_lo[1], B_lo[1]);
+                // high nibbles: 1024 + 16 nib + 256 h = 1024 + 16 q, times sc / 16, minus 64 sc
+                c0 = vhfma2(vbitsel(a, vand_or(fa << 7, 0x01000100u, kH1024), 0x00F000F0u), S_hi[0], B_hi[0]);
+                c1 = vhfma2(vbitsel(b, vand_or(fb << 7, 0x01000100u, kH1024), 0x00F000F0u), S_hi[1], B_hi[1]);
+                c2 = vhfma2(vbitsel(a8, vand_or(fa >> 1, 0x01000100u, kH1024), 0x00F000F0u), S_hi[0], B_hi[0]);
+                c3 = vhfma2(vbitsel(b8, vand_or(fb >> 1, 0x01000100u, kH1024), 0x00F000F0u), S_hi[1], B_hi[1]);
+            } else {
+                // low nibbles: (1024 + q) sc - 1024 sc = q sc exactly
+                a0 = vhfma2(vand_or(a, 0x000F000Fu, kH1024), S_lo[0], B_lo[0]);
+                a1 = vhfma2(vand_or(b, 0x000F000Fu, kH1024), S_lo[1], B_lo[1]);
+                a2 = vhfma2(vand_or(a8, 0x000F000Fu, kH1024), S_lo[0], B_lo[0]);
+                a3 = vhfma2(vand_or(b8, 0x000F000Fu, kH1024), S_lo[1], B_lo[1]);
+                // high nibbles: (1024 + 16 q) sc / 16 - 64 sc = q sc exactly
+                c0 = vhfma2(vand_or(a, 0x00F000F0u, kH1024), S_hi[0], B_hi[0]);
+                c1 = vhfma2(vand_or(b, 0x00F000F0u, kH1024), S_hi[1], B_hi[1]);
+                c2 = vhfma2(vand_or(a8, 0x00F000F0u, kH1024), S_hi[0], B_hi[0]);
+                c3 = vhfma2(vand_or(b8, 0x00F000F0u, kH1024), S_hi[1], B_hi[1]);
+            }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const uint2 bl = lds64(bb[nt] + u * 32);
@@ -1219,7 +1372,7 @@ int resident_ctas(int ks, uint32_t smem) {
     if (cache[dev][slot]) return cache[dev][slot];
     const int sms = device_sm_count();
     int n = sms;
-    if constexpr (C::kBPB != 144) {
+    if constexpr (!C::kSplit) {
         if (ks > 1) return 0;
     } else if (ks > 1) {
         // the query needs the launch's shared-memory size to be allowed
@@ -1308,7 +1461,7 @@ int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m,
         // q4_K can build its image from global memory when the raw copy would
         // crowd out the weight stages (not in gather mode, whose x rows are
         // gathered by the copy)
-        p.x_global = (C::kBPB == 144 && p.off_part + xraw + red + 2u * kRows * 2048u > optin) ? 1 : 0;
+        p.x_global = (C::kSplit && p.off_part + xraw + red + 2u * kRows * 2048u > optin) ? 1 : 0;
         if (p.x_global && ga) return 0;
         if (p.x_global) xraw = 0;
         p.off_red = align16(p.off_part + (part > xraw ? part : xraw));
@@ -1403,7 +1556,7 @@ int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m,
         return KQ_OK;
     }
     auto kernel = qmv_stream_kernel<C, false>;
-    if constexpr (C::kBPB == 144) {   // the K split is built for q4_K only
+    if constexpr (C::kSplit) {   // the K split is built for q4_K and q5_K
         if (ks > 1) kernel = qmv_stream_kernel<C, true>;
     } else if (ks > 1) {
         return KQ_ERR_UNSUPPORTED;
@@ -1426,6 +1579,33 @@ int set_stream_wait_limit(uint64_t ns) {
     return record_cuda(cudaMemcpyToSymbol(g_wait_ns, &v, sizeof(v)));
 }
 
+namespace {
+// q4_K and q5_K (FIVE) on the staged kernel.  From M = 4 the activation
+// image of a whole row crowds out the weight stages (and from M = 8 it no
+// longer fits): K is then split over a cluster of 4 (else 2) CTAs, each
+// covering a slice of at least 7 blocks.  Below M = 4 the split's cluster
+// reduction costs more than it saves (measured).
+template <bool FIVE>
+int launch_q4family(const void* w, int64_t n, int64_t k, const uint16_t* x, int m, float* y, cudaStream_t s) {
+    const int nblk = static_cast<int>(k / 256);
+    int ks = 1;
+    if (m >= 4) {
+        if (nblk % 4 == 0 && nblk / 4 >= 7) ks = 4;
+        else if (nblk % 2 == 0 && nblk / 2 >= 7) ks = 2;
+    }
+    for (;;) {
+        // per-token image stride 32 bytes past a multiple of 128: the 8
+        // tokens of an MMA's B fragment then read disjoint banks
+        uint32_t it = (nblk / ks) * Q4<1, FIVE>::kBlkImg;
+        it += (32u - it % 128u + 128u) % 128u;
+        const int rc = m <= 8 ? launch_stream<Q4<1, FIVE>>(w, n, k, x, m, y, s, it, q4_inv_tok(nblk / ks, m), ks)
+                              : launch_stream<Q4<2, FIVE>>(w, n, k, x, m, y, s, it, q4_inv_tok(nblk / ks, m), ks);
+        if (rc != KQ_ERR_UNSUPPORTED || ks == 1) return rc;
+        ks = 1;
+    }
+}
+}  // namespace
+
 // Staged qmv for the shapes it covers; KQ_ERR_UNSUPPORTED otherwise (the
 // caller then takes the general kernel).
 int launch_qmv_stream(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int m, float* y,
@@ -1434,37 +1614,22 @@ int launch_qmv_stream(int type, const void* w, int64_t n, int64_t k, const uint1
     case KQ_Q8_0: {
         const int nblk = static_cast<int>(k / 32);
         if (m > 2 || nblk % 8 != 0) return KQ_ERR_UNSUPPORTED;
-        const uint32_t it = (nblk / 8) * Q8<1>::kItemImg, xt = nblk * 8;
+        const uint32_t it = (nblk / 8) * Q8<1>::kItemImg, xt = nblk * 4;
         return m == 1 ? launch_stream<Q8<1>>(w, n, k, x, m, y, s, it, xt) : launch_stream<Q8<2>>(w, n, k, x, m, y, s, it, xt);
     }
     case KQ_Q6_K: {
         const int nblk = static_cast<int>(k / 256);
         if (m > 2 || nblk % 8 != 0) return KQ_ERR_UNSUPPORTED;
-        const uint32_t it = nblk * Q6<1>::kBlkImg, xt = nblk * 32 * 4;
+        const uint32_t it = nblk * Q6<1>::kBlkImg, xt = nblk * 16 * 4;
         return m == 1 ? launch_stream<Q6<1>>(w, n, k, x, m, y, s, it, xt) : launch_stream<Q6<2>>(w, n, k, x, m, y, s, it, xt);
     }
-    case KQ_Q4_K: {
-        // From M = 4 the activation image of a whole row crowds out the
-        // weight stages (and from M = 8 it no longer fits): K is then split
-        // over a cluster of 4 (else 2) CTAs, each covering a slice of at least
-        // 7 blocks.  Below M = 4 the split's cluster reduction costs more than
-        // it saves (measured).
-        const int nblk = static_cast<int>(k / 256);
-        int ks = 1;
-        if (m >= 4) {
-            if (nblk % 4 == 0 && nblk / 4 >= 7) ks = 4;
-            else if (nblk % 2 == 0 && nblk / 2 >= 7) ks = 2;
-        }
-        for (;;) {
-            // per-token image stride 32 bytes past a multiple of 128: the 8
-            // tokens of an MMA's B fragment then read disjoint banks
-            uint32_t it = (nblk / ks) * Q4<1>::kBlkImg;
-            it += (32u - it % 128u + 128u) % 128u;
-            const int rc = m <= 8 ? launch_stream<Q4<1>>(w, n, k, x, m, y, s, it, q4_inv_tok(nblk / ks, m), ks)
-                                  : launch_stream<Q4<2>>(w, n, k, x, m, y, s, it, q4_inv_tok(nblk / ks, m), ks);
-            if (rc != KQ_ERR_UNSUPPORTED || ks == 1) return rc;
-            ks = 1;
-        }
+    case KQ_Q4_K: return launch_q4family<false>(w, n, k, x, m, y, s);
+    case KQ_Q5_K: return launch_q4family<true>(w, n, k, x, m, y, s);
+    case KQ_Q4_0: {
+        const int nblk = static_cast<int>(k / 32);
+        if (m > 2 || nblk % 8 != 0) return KQ_ERR_UNSUPPORTED;
+        const uint32_t it = (nblk / 8) * Q40<1>::kItemImg, xt = nblk * 4;
+        return m == 1 ? launch_stream<Q40<1>>(w, n, k, x, m, y, s, it, xt) : launch_stream<Q40<2>>(w, n, k, x, m, y, s, it, xt);
     }
     default: return KQ_ERR_UNSUPPORTED;
     }
@@ -1477,30 +1642,42 @@ int launch_gather_qmv(int type, const void* w_bank, const void* w_bank2, int act
                       int64_t n, int64_t k, const uint16_t* x, int xdiv, const int32_t* ids, int pairs, int m_cap,
                       float* y, int32_t* err_flag, cudaStream_t s) {
     GatherArgs ga{ids, err_flag, pairs, xdiv, n_experts, w_bank2, act, limit};
-    const int nblk = static_cast<int>(k / (type == KQ_Q8_0 ? 32 : 256));
+    const int nblk = static_cast<int>(k / (type == KQ_Q8_0 || type == KQ_Q4_0 ? 32 : 256));
     int rc = KQ_ERR_UNSUPPORTED;
     switch (type) {
     case KQ_Q8_0: {
         if (nblk % 8 != 0) return KQ_ERR_UNSUPPORTED;
-        const uint32_t it = (nblk / 8) * Q8<1>::kItemImg, xt = nblk * 8;
+        const uint32_t it = (nblk / 8) * Q8<1>::kItemImg, xt = nblk * 4;
         rc = m_cap >= 2 ? launch_stream<Q8<2>>(w_bank, n, k, x, 2, y, s, it, xt, 1, &ga) : KQ_ERR_UNSUPPORTED;
         if (rc == KQ_ERR_UNSUPPORTED) rc = launch_stream<Q8<1>>(w_bank, n, k, x, 1, y, s, it, xt, 1, &ga);
         return rc;
     }
     case KQ_Q6_K: {   // any k % 256 == 0 (rows that are not a 16-byte multiple included)
-        const uint32_t it = nblk * Q6<1>::kBlkImg, xt = nblk * 32 * 4;
+        const uint32_t it = nblk * Q6<1>::kBlkImg, xt = nblk * 16 * 4;
         rc = m_cap >= 2 ? launch_stream<Q6<2>>(w_bank, n, k, x, 2, y, s, it, xt, 1, &ga) : KQ_ERR_UNSUPPORTED;
         if (rc == KQ_ERR_UNSUPPORTED) rc = launch_stream<Q6<1>>(w_bank, n, k, x, 1, y, s, it, xt, 1, &ga);
         return rc;
     }
-    case KQ_Q4_K: {
+    case KQ_Q4_K:
+    case KQ_Q5_K: {
         uint32_t it = nblk * Q4<1>::kBlkImg;
         it += (32u - it % 128u + 128u) % 128u;
         for (int m = m_cap < 16 ? m_cap : 16; m >= 1; --m) {
-            rc = m <= 8 ? launch_stream<Q4<1>>(w_bank, n, k, x, m, y, s, it, q4_inv_tok(nblk, m), 1, &ga)
-                        : launch_stream<Q4<2>>(w_bank, n, k, x, m, y, s, it, q4_inv_tok(nblk, m), 1, &ga);
+            if (type == KQ_Q4_K)
+                rc = m <= 8 ? launch_stream<Q4<1>>(w_bank, n, k, x, m, y, s, it, q4_inv_tok(nblk, m), 1, &ga)
+                            : launch_stream<Q4<2>>(w_bank, n, k, x, m, y, s, it, q4_inv_tok(nblk, m), 1, &ga);
+            else
+                rc = m <= 8 ? launch_stream<Q4<1, true>>(w_bank, n, k, x, m, y, s, it, q4_inv_tok(nblk, m), 1, &ga)
+                            : launch_stream<Q4<2, true>>(w_bank, n, k, x, m, y, s, it, q4_inv_tok(nblk, m), 1, &ga);
             if (rc != KQ_ERR_UNSUPPORTED) return rc;
         }
+        return rc;
+    }
+    case KQ_Q4_0: {
+        if (nblk % 8 != 0) return KQ_ERR_UNSUPPORTED;
+        const uint32_t it = (nblk / 8) * Q40<1>::kItemImg, xt = nblk * 4;
+        rc = m_cap >= 2 ? launch_stream<Q40<2>>(w_bank, n, k, x, 2, y, s, it, xt, 1, &ga) : KQ_ERR_UNSUPPORTED;
+        if (rc == KQ_ERR_UNSUPPORTED) rc = launch_stream<Q40<1>>(w_bank, n, k, x, 1, y, s, it, xt, 1, &ga);
         return rc;
     }
     default: return KQ_ERR_UNSUPPORTED;

@@ -18,17 +18,23 @@
  *  - W is the codec's wire bytes for an [n, k] matrix, row-major, rows
  *    contiguous: row r starts at byte r * row_bytes with
  *    row_bytes = (k / values_per_block) * bytes_per_block.  This is the
- *    "transpose=True" layout of the mlx-kquant `quantized_matmul` op
- *    (bindings.cpp docstring: "uint8 K-quant wire bytes (laid out [N, K] when
- *    transpose=True)") and of the README's "x @ dequant(w).T".
+ *    layout the mlx-kquant `quantized_matmul` op takes with transpose=True
+ *    (bindings.cpp docstring: the weight operand is uint8 wire bytes, N rows
+ *    of K values in that mode), the README's product x @ dequant(w).T.
  *  - Activations x are bfloat16 [m, k] row-major (passed as uint16_t bit
- *    patterns), any finite value.  The decode kernels of q4_K, q6_K and q8_0
- *    (kq_qmv, kq_gather_qmv, kq_moe_glu_gather) scale each activation row by
- *    a power of two taken from its largest magnitude, round it to binary16
+ *    patterns), any finite value.  The tensor-core decode kernels
+ *    (kq_qmv, kq_gather_qmv, kq_moe_glu_gather) scale each run of
+ *    activations (a block, a 16-value run of q6_K, or a row slice) by a
+ *    power of two taken from its largest magnitude, round it to binary16
  *    and apply the inverse scale to the fp32 sums, so their relative error
- *    does not depend on the magnitude of x; a non-finite activation sets
- *    KQ_DEV_X_RANGE (its outputs are then NaN or infinite).  qmm/gather use
- *    bf16 as is, and the q5_K / q4_0 qmv widens it to fp32 exactly.
+ *    does not depend on the magnitude of x.  Codes enter the MMA centred on
+ *    their format's offset (q8_0 code, q4_0 code - 8, q6_K code - 32,
+ *    exactly), so a weight that decodes to 0 contributes exactly 0 however
+ *    large its activation.  Within one run, values below about 2^-29 of the
+ *    run's largest magnitude fall into binary16's subnormal range and lose
+ *    relative precision.  A non-finite activation sets KQ_DEV_X_RANGE (its
+ *    outputs are then NaN or infinite).  qmm/gather use bf16 as is, and the
+ *    exact fp32 kernel (q4_0 at m >= 3) widens it to fp32 exactly.
  *  - Outputs y are fp32 [m, n] row-major.
  *  - Return value: a kq_status.  A non-zero status means nothing was enqueued
  *    (argument errors) or that the CUDA launch failed (KQ_ERR_CUDA; the
@@ -39,8 +45,8 @@
  *    slower copy paths; kq_qmm / kq_gather_qmm need k % 256 == 0
  *    (KQ_ERR_UNSUPPORTED otherwise).
  *  - `k` must be a multiple of the codec's values_per_block, as the reference
- *    requires ("last dim a multiple of the codec's bytes_per_block",
- *    bindings.cpp `dequantize`); otherwise KQ_ERR_INVALID_ARG.
+ *    requires (bindings.cpp `dequantize`: the last dimension holds whole
+ *    blocks); otherwise KQ_ERR_INVALID_ARG.
  */
 #ifndef KQ_H
 #define KQ_H
@@ -115,9 +121,9 @@ int kq_set_wait_limit(int64_t ns);
 
 /*
  * kq_dequantize - decode wire bytes to fp32, bit-exactly (all five codecs).
- * mlx-kquant bindings.cpp, `dequantize` ("Dequantize GGUF K-quant wire bytes
- * to a float array"); hanzo-ml quantized/mod.rs, `QTensor::dequantize`
- * (to_float into f32).
+ * mlx-kquant bindings.cpp, `dequantize` (wire bytes in, a float array out);
+ * hanzo-ml quantized/mod.rs, `QTensor::dequantize` (decodes to f32 through
+ * its to_float routine).
  *   w    [n_rows, row_bytes] wire bytes
  *   out  [n_rows, k] fp32; element (r, c) = decode of value c of row r,
  *        computed in fp32 as (d*sc)*q - (dmin*m) (q4_K, q5_K), (d*sc)*q
@@ -128,9 +134,9 @@ int kq_dequantize(int type, const void* w, int64_t n_rows, int64_t k, float* out
 
 /*
  * kq_quantize - encode fp32 weights into wire bytes (the step before the
- * products).  mlx-kquant bindings.cpp, `quantize` ("Encode a float weight
- * tensor into GGUF K-quant wire bytes"; last dim a multiple of the codec's
- * block); hanzo-ml quantized/mod.rs `QTensor::quantize`.
+ * products).  mlx-kquant bindings.cpp, `quantize` (float weights in, wire
+ * bytes out; the last dimension holds whole blocks); hanzo-ml
+ * quantized/mod.rs `QTensor::quantize`.
  *   w    [n_rows, k] fp32, finite (scales must stay in binary16 range)
  *   out  [n_rows, row_bytes] wire bytes
  * The pages give no encoding search; this one is fixed step by step in fp32:
@@ -146,8 +152,11 @@ int kq_quantize(int type, const float* w, int64_t n_rows, int64_t k, void* out, 
 
 /*
  * kq_qmv - decode-shaped product y = x . W^T for 1 <= m <= 16 rows of x.
- * (q5_K and q4_0 take a plainer kernel: every weight decoded exactly to
- * fp32 and multiplied by the activations with fp32 FMAs; k % 256 == 0.)
+ * All five codecs take the staged tensor-core kernel (q8_0, q6_K, q4_0 for
+ * m <= 2; q4_K, q5_K for every m).  q8_0 and q6_K at m >= 3 take the
+ * general tensor-core kernel; q4_0 at m >= 3 takes a plainer one (every
+ * weight decoded exactly to fp32 and multiplied by the activations with
+ * fp32 FMAs).  q4_0 needs k % 256 == 0.
  * mlx-kquant bindings.cpp, `quantized_matmul` (x @ dequant(w), transpose=True);
  * README "How it works": small row counts take a weight-read-amortizing
  * kernel (`verify_qmv`).  Every weight byte is read once for all m rows.
@@ -176,8 +185,8 @@ int kq_qmm(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int
  * kq_moe_sort - group routed (token, slot) pairs by expert for a sorted MoE
  * prefill: a stable counting sort by expert id, plus the row gather of x.
  * mlx-kquant README "Performance" (sorted MoE prefill batches route to a
- * per-expert-segment GEMM) and bindings.cpp `gather_qmm_seg` ("rows
- * pre-sorted by expert").
+ * per-expert-segment GEMM) and bindings.cpp `gather_qmm_seg` (its rows come
+ * in already grouped by expert).
  *   topk_ids    [n_tokens, top_k] int32 expert ids, each in [0, n_experts)
  *   x           [n_tokens, k] bf16 (may be NULL when x_sorted is NULL)
  *   sorted_ids  [n_tokens*top_k] uint32 out: expert id of sorted row r
@@ -237,18 +246,19 @@ int kq_gather_qmm(int type, const void* w_bank, int32_t n_experts, int64_t n, in
  * kq_gather_qmv - decode-shaped MoE product with one output row per
  * (token, slot) pair: y[p, :] = x[row(p), :] . dequant(W[ids[p]])^T for the
  * p = token*top_k + slot pairs of ids [n_tokens, top_k].
- * mlx-kquant bindings.cpp, `gather_qmv_kq` ("gathered matvec for K-quant
- * expert stacks (the MoE down projection); one activation row per expert
- * slot": x [T, R, K], w (n_experts, N, bytes_per_row), indices [T, R],
- * output [T, R, N]).  With x_per_token != 0 x holds one row per token,
+ * mlx-kquant bindings.cpp, `gather_qmv_kq` (a matvec over a stack of
+ * expert weight matrices, as in the MoE down projection, with its own
+ * activation row for every expert slot: x [T, R, K], w (n_experts, N,
+ * bytes_per_row), indices [T, R], output [T, R, N]).  With x_per_token != 0 x holds one row per token,
  * row(p) = p / top_k, which is the gate/up product of `moe_glu_gather_kq`
  * before its GLU; else row(p) = p.
  *   w_bank [n_experts, n, row_bytes], x [n_tokens*top_k or n_tokens, k] bf16,
  *   ids [n_tokens*top_k] int32, y [n_tokens*top_k, n] fp32.
  * No host round trip: the pairs are grouped by expert on the device and each
  * routed expert's weights are read once for all of its pairs (in batches of
- * up to 2 (q8_0, q6_K) or 16 (q4_K) activation rows; an expert with more
- * pairs than a batch is streamed once per batch).  Arithmetic as kq_qmv.
+ * up to 2 (q8_0, q6_K, q4_0) or 16 (q4_K, q5_K) activation rows; an expert
+ * with more pairs than a batch is streamed once per batch).  Arithmetic as
+ * kq_qmv.  All five codecs.
  * Limits: 1 <= n_experts <= 256, 1 <= n_tokens*top_k <= 8192; k % 256 == 0,
  * else KQ_ERR_UNSUPPORTED (q6_K rows that are not a 16-byte multiple, k / 256
  * not a multiple of 8, take a slower copy path: each row is staged from the
@@ -270,9 +280,9 @@ int kq_gather_qmv(int type, const void* w_bank, int32_t n_experts, int64_t n, in
  * kq_moe_glu_gather - decode MoE gate/up products and their GLU in one
  * dispatch: out[p, :] = act(x[t, :] . dequant(Wg[e])^T, x[t, :] . dequant(Wu[e])^T)
  * for the pairs p = t*top_k + s of ids [n_tokens, top_k], e = ids[p].
- * mlx-kquant bindings.cpp, `moe_glu_gather_kq` ("gate and up expert matvecs
- * share each activation load and the GLU epilogue act(g) * u is applied in
- * the same dispatch"; act 'silu' (default), 'gelu' (tanh approx),
+ * mlx-kquant bindings.cpp, `moe_glu_gather_kq` (the gate and up matvecs of
+ * an expert load each activation once, and act(g) * u is applied before the
+ * dispatch ends; act 'silu' (default), 'gelu' (tanh approx),
  * 'silu_limit' (requires limit > 0); x [T, K], gate_w and up_w
  * (n_experts, N, bytes_per_row), indices [T, R], output [T, R, N]).
  * Each routed expert's gate and up rows are streamed once; every CTA takes

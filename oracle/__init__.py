@@ -15,7 +15,7 @@ and states the MoE semantics in plain numpy:
 * ``moe_sort``     stable sort of (token, slot) pairs by expert id; x rows
                    gathered into expert-sorted order (mlx-kquant README,
                    "Performance": sorted MoE prefill batches; bindings.cpp
-                   ``gather_qmm_seg``: "rows pre-sorted by expert").
+                   ``gather_qmm_seg``, whose rows come grouped by expert).
 * ``tile_map``     (expert, row_start, num_rows) tiles of at most 64 rows,
                    only the last tile of a segment partial (bindings.cpp,
                    ``expert_tile_map``).
@@ -26,16 +26,16 @@ and states the MoE semantics in plain numpy:
                    quantized matmul per expert).
 * ``gather_qmv``   decode-shaped MoE product, one output row per (token,
                    slot) pair: y[p] = x[row(p)] @ dequant(w[ids[p]]).T
-                   (bindings.cpp, ``gather_qmv_kq``: "one activation row per
-                   expert slot", x [T, R, K], indices [T, R], output
+                   (bindings.cpp, ``gather_qmv_kq``: an activation row of
+                   its own for each expert slot, x [T, R, K], indices [T, R], output
                    [T, R, N]; with one activation row per token the same
                    product feeds the gate/up projections of
                    ``moe_glu_gather_kq``).
 * ``moe_glu_gather`` act(x W_g^T) * (x W_u^T) per pair from the fp64 gate
                    and up products, act silu, gelu (tanh form) or silu with
                    a limit (bindings.cpp, ``moe_glu_gather_kq``).
-* ``quantize``     float -> wire bytes (bindings.cpp, ``quantize``: encode a
-                   float weight tensor into GGUF K-quant wire bytes): q8_0 by
+* ``quantize``     float -> wire bytes (bindings.cpp, ``quantize``: float
+                   weights in, wire bytes out): q8_0 by
                    ggml's absmax rule, q4_K / q6_K by min/max and absmax
                    scales in fixed fp32 steps (see kq_oracle.c).
 * ``inverse_order`` / ``gather_mix``  unsort and score mix of expert-sorted

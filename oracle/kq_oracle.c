@@ -9,9 +9,9 @@
  * floating-point operation below is rounded exactly where it is written.
  *
  * What it computes, and where that is stated:
- *  - dequantize: wire bytes -> float ("dequantize" op docstring, mlx-kquant
- *    bindings.cpp; "QTensor::dequantize -> to_float into f32", hanzo-ml
- *    quantized/mod.rs).  Block sizes: mlx-kquant README, "Codec reference"
+ *  - dequantize: wire bytes -> float (the `dequantize` op docstring,
+ *    mlx-kquant bindings.cpp; QTensor::dequantize, which decodes to f32
+ *    through to_float, hanzo-ml quantized/mod.rs).  Block sizes: mlx-kquant README, "Codec reference"
  *    table (q4_k 256 values / 144 B, q5_k 256 / 176 B, q6_k 256 / 210 B, q8_0
  *    32 / 34 B, q4_0 32 / 18 B).  The
  *    field layout inside a block is not printed on the pages; the pages say
@@ -24,9 +24,9 @@
  *    docstring, transpose=True, mlx-kquant bindings.cpp; README "Using
  *    K-quant ops directly").  The reference value accumulates in fp64; an
  *    fp32 sequential-k variant is provided for timing only.
- *  - quantize: float -> wire bytes ("quantize" op docstring, mlx-kquant
- *    bindings.cpp: encode a float weight tensor into GGUF K-quant wire bytes;
- *    hanzo-ml quantized/mod.rs QTensor::quantize).  The pages give no
+ *  - quantize: float -> wire bytes (the `quantize` op docstring, mlx-kquant
+ *    bindings.cpp: float weights in, wire bytes out; hanzo-ml
+ *    quantized/mod.rs QTensor::quantize).  The pages give no
  *    encoding search.  q8_0 follows ggml's published rule (absmax / 127,
  *    round half away from zero), pinned against gguf.quants.quantize.  q4_K
  *    and q6_K take the plainest reading: per sub-block min/max (q4_K) or

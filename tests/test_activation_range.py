@@ -7,9 +7,11 @@ x: tiny (N(0, sigma^2) down to sigma = 1e-5), large (beyond the binary16
 range), rows of very different magnitude in one batch, and rows where a few
 large entries sit among small ones.  Every call is checked against the fp64
 oracle with the qmv bound (per element 1e-3 * sum |x w| and max-norm 1e-3).
-Shapes reach the staged kernel (M <= 2), the K-split q4_K kernel (M >= 4),
-the general kernel (q8_0 / q6_K at M >= 3; q6_K with 630-byte rows at
-K = 768) and the decode MoE kernels (gather_qmv, moe_glu_gather)."""
+Shapes reach the staged kernel (M <= 2; q4_K / q5_K up to M = 16), the
+K-split q4_K / q5_K kernel (M >= 4), the general kernel (q8_0 / q6_K at
+M >= 3; q6_K with 630-byte rows at K = 768), the exact fp32 kernel (q4_0 at
+M >= 3) and the decode MoE kernels (gather_qmv,
+moe_glu_gather)."""
 import numpy as np
 import pytest
 import torch
@@ -17,17 +19,65 @@ import torch
 import gguf_quant_dequant_q4_b200 as kq
 import oracle
 import synth
-from tests._util import check_qmv, dev_bf16, dev_u8
+from tests._util import check_qmv, dev_bf16, dev_u8, zero_weights_at
 
 pytestmark = pytest.mark.gpu
-CODECS = [kq.Q4_K, kq.Q6_K, kq.Q8_0]
+CODECS = [kq.Q4_K, kq.Q6_K, kq.Q8_0, kq.Q5_K, kq.Q4_0]
 
 
-def run(qtype, n, k, x, seed=0):
-    w = synth.weights(qtype, n, k, seed=seed)
+def run(qtype, n, k, x, seed=0, w=None):
+    w = synth.weights(qtype, n, k, seed=seed) if w is None else w
     y = kq.qmv(dev_bf16(x), dev_u8(w), qtype).cpu().numpy()
     ref, absdot = oracle.matmul(qtype, w, k, x, absdot=True)
     return check_qmv(y, ref, absdot)
+
+
+def outliers_at(m, k, cols, small, big, seed):
+    """N(0, small^2) rows with +-big at the given columns."""
+    x = oracle.bf16_to_f32(synth.activations_scaled([small] * m, k, seed=seed)).copy()
+    sign = np.where(np.random.default_rng(seed).random((m, len(cols))) < 0.5, -1.0, 1.0)
+    x[:, cols] = (big * sign).astype(np.float32)
+    return synth.f32_to_bf16_bits(x)
+
+
+# Large activations where every weight row decodes to an exact zero (the
+# format's code offset): sum |x w| then holds only the small terms, so the
+# large products must cancel exactly.  The codes are centred on the offset
+# in binary16 before the MMA, which makes each such product an exact zero.
+ZERO_COLS = [3, 700, 1333, 2047]
+
+
+@pytest.mark.parametrize("qtype", [kq.Q8_0, kq.Q6_K, kq.Q4_0])
+@pytest.mark.parametrize("m", [1, 2, 3, 7, 16])
+def test_outliers_on_zero_weights(qtype, m):
+    k, n = 2048, 16 * 6 + 5
+    w = zero_weights_at(qtype, synth.weights(qtype, n, k, seed=70), ZERO_COLS)
+    run(qtype, n, k, outliers_at(m, k, ZERO_COLS, 1e-3, 1e4, seed=71 + m), w=w)
+
+
+@pytest.mark.parametrize("qtype", [kq.Q8_0, kq.Q6_K, kq.Q4_0])
+def test_decode_moe_outliers_on_zero_weights(qtype):
+    tokens, top_k, experts, n, k = 3, 2, 4, 150, 2048
+    wg = zero_weights_at(qtype, synth.weights(qtype, n, k, seed=72, experts=experts), ZERO_COLS)
+    wu = zero_weights_at(qtype, synth.weights(qtype, n, k, seed=73, experts=experts), ZERO_COLS)
+    ids = synth.routing(tokens, experts, top_k, seed=74)
+    x = outliers_at(tokens * top_k, k, ZERO_COLS, 1e-3, 1e4, seed=75)
+    y = torch.full((tokens * top_k, n), float("nan"), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kq.gather_qmv(dev_bf16(x), dev_u8(wg), qtype, torch.from_numpy(ids).cuda(), out=y, err=err)
+    assert int(err.item()) == 0
+    ref, a = oracle.gather_qmv(qtype, wg, k, x, ids, absdot=True)
+    check_qmv(y.cpu().numpy(), ref, a)
+    # the gate/up GLU with one activation row per token
+    xt = outliers_at(tokens, k, ZERO_COLS, 1e-3, 1e4, seed=76)
+    out = kq.moe_glu_gather(dev_bf16(xt), dev_u8(wg), dev_u8(wu), qtype, torch.from_numpy(ids).cuda())
+    ref, g, u, ag, au = oracle.moe_glu_gather(qtype, wg, wu, k, xt, ids)
+    dg, du = 1e-3 * ag, 1e-3 * au
+    a = np.abs(oracle.glu(oracle.ACT_SILU, g, np.ones_like(g)))
+    tol = 1.2 * dg * (np.abs(u) + du) + (a + 1.2 * dg) * du + 1e-5 * np.abs(ref) + 1e-300
+    yv = out.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(yv))
+    assert float(np.max(np.abs(yv - ref) / tol)) <= 1.0
 
 
 @pytest.mark.parametrize("qtype", CODECS)
@@ -71,18 +121,20 @@ def test_general_kernel_unaligned_rows(qtype, m):
         run(qtype, 50, 768, x, seed=22)
 
 
+@pytest.mark.parametrize("qtype", [kq.Q4_K, kq.Q5_K])
 @pytest.mark.parametrize("m", [4, 8, 16])
-def test_q4K_split_k_small_and_mixed(m):
-    # K = 7168: the q4_K kernel splits K over a cluster of CTAs, each slice
-    # scaled on its own before the slices are summed
+def test_q4K_split_k_small_and_mixed(qtype, m):
+    # K = 7168: the q4_K / q5_K kernel splits K over a cluster of CTAs, each
+    # slice scaled on its own before the slices are summed
     x = synth.activations_scaled([10.0 ** (-5 + (i % 8)) for i in range(m)], 7168, seed=30 + m)
-    run(kq.Q4_K, 37, 7168, x, seed=31)
+    run(qtype, 37, 7168, x, seed=31)
 
 
-@pytest.mark.parametrize("qtype", [kq.Q5_K, kq.Q4_0])
-def test_exact_kernel_codecs(qtype):
-    x = synth.activations_scaled([1e-5, 1e5, 1.0], 2048, seed=40)
-    run(qtype, 70, 2048, x, seed=41)
+@pytest.mark.parametrize("m", [3, 16])
+def test_exact_kernel_q4_0(m):
+    # q4_0 from M = 3 takes the exact fp32 kernel
+    x = synth.activations_scaled([1e-5, 1e5, 1.0] * (m // 3) + [1e-2] * (m % 3), 2048, seed=40)
+    run(kq.Q4_0, 70, 2048, x, seed=41)
 
 
 @pytest.mark.parametrize("qtype", CODECS)

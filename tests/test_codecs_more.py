@@ -1,6 +1,7 @@
 """q5_K and q4_0 on the GPU vs the CPU oracle: dequantize bit-exact, the
-tensor-core products (qmm, gather) within the qmm bound, and kq_qmv (an exact
-fp32 decode-and-dot kernel for these two codecs) within the qmv bound."""
+tensor-core products (qmm, gather) within the qmm bound, and kq_qmv within
+the qmv bound: the staged tensor-core decode kernel (q5_K up to M = 16,
+q4_0 up to M = 2) and beyond it the exact fp32 decode-and-dot kernel."""
 import numpy as np
 import pytest
 import torch
@@ -44,7 +45,7 @@ def test_qmm_vs_oracle(qtype, m, n):
 
 
 @pytest.mark.parametrize("qtype", CODECS)
-@pytest.mark.parametrize("m", [1, 5, 16])
+@pytest.mark.parametrize("m", [1, 2, 3, 5, 16])
 def test_qmv_vs_oracle(qtype, m):
     n, k = 1000, 4096
     w = synth.weights(qtype, n, k, seed=7)

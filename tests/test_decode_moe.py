@@ -29,7 +29,7 @@ def check_pairs(qtype, w, k, x, ids, y, x_per_token=False, rows=None):
     check_qmv(y[rows], ref[rows], a[rows])
 
 
-@pytest.mark.parametrize("qtype", [kq.Q4_K, kq.Q6_K, kq.Q8_0])
+@pytest.mark.parametrize("qtype", [kq.Q4_K, kq.Q6_K, kq.Q8_0, kq.Q5_K, kq.Q4_0])
 @pytest.mark.parametrize("tokens,top_k,experts,n", [(1, 2, 8, 300), (3, 4, 5, 1000), (16, 2, 4, 520)])
 def test_gather_qmv_vs_oracle(qtype, tokens, top_k, experts, n):
     k = 2048
@@ -41,7 +41,7 @@ def test_gather_qmv_vs_oracle(qtype, tokens, top_k, experts, n):
     check_pairs(qtype, w, k, x, ids, y)
 
 
-@pytest.mark.parametrize("qtype", [kq.Q4_K, kq.Q8_0])
+@pytest.mark.parametrize("qtype", [kq.Q4_K, kq.Q8_0, kq.Q5_K, kq.Q4_0])
 def test_gather_qmv_x_per_token(qtype):
     tokens, top_k, experts, n, k = 4, 2, 6, 257, 4096
     w = synth.weights(qtype, n, k, seed=61, experts=experts)
@@ -52,7 +52,7 @@ def test_gather_qmv_x_per_token(qtype):
     check_pairs(qtype, w, k, x, ids, y, x_per_token=True)
 
 
-@pytest.mark.parametrize("qtype", [kq.Q6_K, kq.Q4_K])
+@pytest.mark.parametrize("qtype", [kq.Q6_K, kq.Q4_K, kq.Q4_0, kq.Q5_K])
 def test_gather_qmv_crowded_expert_and_repeated_ids(qtype):
     # five tokens all route slot 0 to expert 1 (more pairs than one batch of
     # the q6_K kernel), token 2 names expert 3 twice
@@ -174,7 +174,7 @@ def check_glu(y, out, g, u, ag, au, act):
     assert worst <= 1.0, f"error / bound = {worst:.3f}"
 
 
-@pytest.mark.parametrize("qtype", [kq.Q4_K, kq.Q6_K, kq.Q8_0])
+@pytest.mark.parametrize("qtype", [kq.Q4_K, kq.Q6_K, kq.Q8_0, kq.Q5_K, kq.Q4_0])
 @pytest.mark.parametrize("act", [kq.ACT_SILU, kq.ACT_GELU_TANH, kq.ACT_SILU_LIMIT])
 def test_moe_glu_gather_vs_oracle(qtype, act):
     tokens, top_k, experts, n, k = 3, 2, 5, 333, 2048

@@ -10,7 +10,7 @@ import synth
 from tests._util import check_qmv, dev_bf16, dev_u8
 
 pytestmark = pytest.mark.gpu
-CODECS = [kq.Q4_K, kq.Q6_K, kq.Q8_0]
+CODECS = [kq.Q4_K, kq.Q6_K, kq.Q8_0, kq.Q5_K, kq.Q4_0]
 
 
 def run(qtype, n, k, m, seed=0):
@@ -51,11 +51,12 @@ def test_c2_q4K_4096x14336(m):
     run(kq.Q4_K, 4096, 14336, m, seed=synth.SEED_W)
 
 
+@pytest.mark.parametrize("qtype", [kq.Q4_K, kq.Q5_K])
 @pytest.mark.parametrize("m", [7, 9, 16])
-def test_q4K_long_k_many_tokens(m):
+def test_q4K_long_k_many_tokens(qtype, m):
     # an activation image of m x K that does not fit in shared memory at once:
     # the decode kernel walks K in chunks (two images in turn); ragged N
-    run(kq.Q4_K, 200, 8192, m, seed=40 + m)
+    run(qtype, 200, 8192, m, seed=40 + m)
 
 
 # q4_K from M = 4 splits K over a cluster of CTAs (4 CTAs when the slices
@@ -65,8 +66,9 @@ def test_q4K_long_k_many_tokens(m):
 # (n = 2647), and the 2-CTA split (K = 3584: 14 blocks)
 @pytest.mark.parametrize("n,k,m", [(37, 7168, 4), (37, 7168, 12), (2647, 7168, 5), (300, 3584, 8),
                                    (300, 3584, 16)])
-def test_q4K_split_k(n, k, m):
-    run(kq.Q4_K, n, k, m, seed=n + m)
+@pytest.mark.parametrize("qtype", [kq.Q4_K, kq.Q5_K])
+def test_q4K_split_k(qtype, n, k, m):
+    run(qtype, n, k, m, seed=n + m)
 
 
 @pytest.mark.parametrize("qtype", CODECS)
