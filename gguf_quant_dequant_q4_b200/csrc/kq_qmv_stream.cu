@@ -77,9 +77,10 @@ struct SP {
     int m, nblk, g, spr, ns;   // nblk: blocks of the slice
     // x_global 1: build the image from x in global memory (no room for a raw
     // copy); ks: CTAs of a cluster splitting K (q4_K; 1: no split; the token
-    // stride of x is then ks k).  Packed: a larger parameter block was
-    // measured to slow the kernel down.
-    uint32_t x_global : 8, ks : 8;
+    // stride of x is then ks k); strict 1: the wait limit is shorter than the
+    // default, the activation wait tests its phase (see spin_wait).  Packed:
+    // a larger parameter block was measured to slow the kernel down.
+    uint32_t x_global : 8, ks : 8, strict : 1;
     uint32_t rs;   // shared-memory stride of a stage row
     uint32_t off_stage, off_img, img_tok, off_xs, xs_tok, off_zero, off_part, off_xraw;
     uint32_t off_red;   // split: receive slots of the cluster reduction
@@ -154,6 +155,9 @@ __device__ __forceinline__ uint32_t vhfma2(uint32_t a, uint32_t b, uint32_t c) {
 __device__ __forceinline__ void sts64(uint32_t a, uint32_t x, uint32_t y) {
     asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(x), "r"(y));
 }
+__device__ __forceinline__ void sts16(uint32_t a, __half x) {
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(__half_as_ushort(x)));
+}
 __device__ __forceinline__ void sts8(uint32_t a, uint32_t x) {
     asm volatile("st.shared.u8 [%0], %1;" ::"r"(a), "r"(x));
 }
@@ -176,19 +180,24 @@ __device__ __forceinline__ float h2f(uint32_t h) { return __half2float(__ushort_
 // kWaitLimitNs; kq_set_wait_limit shortens it for fault-handling tests).  Read
 // only once a wait has not completed at its first poll.
 __device__ uint64_t g_wait_ns = kWaitLimitNs;
+// Host copy, per device, of whether g_wait_ns is shorter than the default.
+bool g_strict_wait[64];
 __device__ __forceinline__ uint64_t wait_limit() { return *static_cast<volatile uint64_t*>(&g_wait_ns); }
 
 // Bounded spin on an mbarrier phase (no suspend hint: these waits are short
 // and a sleeping warp can wake up late).  False after the time limit, with
-// KQ_DEV_TIMEOUT recorded.  Under a limit shorter than the default (a test's)
-// the time is taken at every poll and a completion seen after the limit
-// counts as run out, so the first wait that is not complete at once runs out.
-__device__ __forceinline__ bool spin_wait(uint64_t* bar, uint32_t parity, int* status) {
-    if (mbar_try_wait(bar, parity)) return true;
+// KQ_DEV_TIMEOUT recorded.  Under a limit shorter than the default (a
+// test's) the time is taken at every poll and a completion seen after the
+// limit counts as run out.  `test_first` (the activation wait, once per CTA,
+// with a short limit): the phase is only tested, never waited on, so that
+// wait runs out unless the copy has already landed.  The per-stage waits
+// keep the plain form: a blocking first poll and no extra work.
+__device__ __forceinline__ bool spin_wait(uint64_t* bar, uint32_t parity, int* status, bool test_first = false) {
+    if (test_first ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns(), limit = wait_limit();
     const bool strict = limit < kWaitLimitNs;
     for (int i = 0;; ++i) {
-        const bool done = mbar_try_wait(bar, parity);
+        const bool done = test_first ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity);
         if (done && !strict) return true;
         if (strict || (i & 255) == 255) {
             if (global_ns() - t0 > limit) {
@@ -202,13 +211,14 @@ __device__ __forceinline__ bool spin_wait(uint64_t* bar, uint32_t parity, int* s
 
 // Bounded wait that lets the warp sleep until the phase completes (the
 // producer: it must not take issue slots from the decoding warps).  `limit`
-// is the time limit (the pipeline's, or kWaitLimitNs for the wind-down).
+// is the time limit (the pipeline's, or kWaitLimitNs for the wind-down); a
+// shorter limit than the default makes the wait strict, as in spin_wait.
 __device__ __forceinline__ bool sleep_wait(uint64_t* bar, uint32_t parity, int* status, uint64_t limit) {
-    if (mbar_try_wait(bar, parity)) return true;
+    const bool strict = limit < kWaitLimitNs;
+    if (strict ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
-    const bool strict = limit < kWaitLimitNs;   // as in spin_wait
     for (;;) {
-        const bool done = mbar_try_wait_sleep(bar, parity);
+        const bool done = strict ? mbar_test_wait(bar, parity) : mbar_try_wait_sleep(bar, parity);
         if (done && !strict) return true;
         if (global_ns() - t0 > limit) {
             if (status) atomicOr(status, KQ_DEV_TIMEOUT);
@@ -231,24 +241,6 @@ __device__ __forceinline__ uint32_t hpair(__half lo, __half hi) {
     return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
 }
 
-// Scales of the 32-value blocks (q8_0, q4_0), one thread per (token, block):
-// 2^s from the block's largest |x| (its scaled values below 2^(xt+1)), stored
-// as 2^-s at 4 bytes per block in block order.  Returns whether this thread
-// met a non-finite activation.
-__device__ __forceinline__ bool block_scales(const SP& p, uint32_t sb, int xt) {
-    bool bad = false;
-    for (int e = threadIdx.x; e < p.m * p.nblk; e += kCW * 32) {
-        const int tok = e / p.nblk, blk = e % p.nblk;
-        const uint32_t xs = xaddr(p, sb, tok, 32 * blk);
-        uint32_t mx = 0;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) mx = absmax8_bf16(mx, lds128(xs + 16 * c));
-        mx = max(mx & 0xFFFFu, mx >> 16);
-        bad |= mx >= 0x7F80u;
-        sts32(sb + p.off_xs + tok * p.xs_tok + 4 * blk, __float_as_uint(exp2_int(-xscale_exp(mx, xt))));
-    }
-    return bad;
-}
 
 // Lane roles in the m16n8k16 fragments (lane = 4 g + t): A rows g and g+8,
 // k-slots 2t, 2t+1, 2t+8, 2t+9; B column g; D columns 2t, 2t+1.
@@ -268,8 +260,6 @@ struct Q8 {
     static constexpr int kAccPerLane = 2 * NT;
     // a block's scaled activations stay below 2^15: far inside binary16
     static constexpr int kXT = 14;
-    // the build needs every block's scale before it writes the image
-    static constexpr bool kTwoPhase = true;
     static constexpr bool kSplit = false;
 
     // rowA/rowB: shared address of the item (8 blocks) in rows g / g+8;
@@ -347,36 +337,50 @@ struct Q8 {
             }
     }
 
-    // Phase 1, one thread per (token, block): the block's scale 2^s from its
-    // largest |x|, stored as 2^-s (4 bytes per block, in block order).
-    // Returns whether this thread met a non-finite activation.
-    static __device__ bool build_scales(const SP& p, uint32_t sb, int64_t xoff) {
-        return block_scales(p, sb, kXT);
-    }
-    // Phase 2: image entry (item, mu, t') = binary16 of the scaled activations
-    // of the 4 raw bytes at offset 272 item + 68 t' + 4 mu of a row, as
-    // (byte0, byte2 | byte1, byte3); scale bytes get 0.  A block's 2^s is read
-    // back from its stored 2^-s (powers of two: the bit patterns of 2^k and
-    // 2^-k add up to 254 << 23).
+    // Image entry (item, mu, t') = binary16 of the scaled activations of the
+    // 4 raw bytes at offset 272 item + 68 t' + 4 mu of a row, as (byte0,
+    // byte2 | byte1, byte3); scale bytes get 0.  Eight neighbouring lanes
+    // share the span of lane t' (blocks b0 = 8 item + 2 t' and b0 + 1), each
+    // with 8 values of one block: they agree on the block's scale 2^s (its
+    // largest |x| at 2^14) by two shuffles, and lane 0 of the block stores
+    // 2^-s (4 bytes per block, in block order).  Every warp runs the same
+    // number of rounds, so the shuffles always see the whole warp.  Returns
+    // whether this thread met a non-finite activation.
     static __device__ bool build(const SP& p, uint32_t sb, int64_t xoff) {
-        const int items = p.nblk / 8;
-        const int per_tok = items * 17 * 4;
-        for (int e = threadIdx.x; e < p.m * per_tok; e += kCW * 32) {
-            const int tok = e / per_tok, rem = e % per_tok;
-            const int it = rem / 68, mu = (rem % 68) >> 2, tt = rem & 3;
-            const int R0 = it * 272 + 68 * tt + 4 * mu;
-            __half h[4];
+        bool bad = false;
+        const int spans = p.nblk / 2, total = p.m * spans * 8;
+        for (int w0 = threadIdx.x & ~31; w0 < total; w0 += kCW * 32) {
+            const int e = w0 + (threadIdx.x & 31);
+            const bool in = e < total;
+            const int sp = e >> 3, tok = sp / spans, s2 = sp - tok * spans;   // s2 = 4 item + t'
+            const int it = s2 >> 2, tt = s2 & 3, odd = (e >> 2) & 1, qq = e & 3;
+            const int blk = 2 * s2 + odd;
+            const uint4 v = in ? lds128(xaddr(p, sb, tok, 32 * blk + 8 * qq)) : make_uint4(0u, 0u, 0u, 0u);
+            uint32_t mx = absmax8_bf16(0u, v);
+            mx = max(mx & 0xFFFFu, mx >> 16);
+            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            bad |= in && mx >= 0x7F80u;
+            const int se = xscale_exp(mx, kXT);
+            const float S = exp2_int(se);
+            if (!in) continue;   // lanes out of range occur in the last round only
+            if (qq == 0) sts32(sb + p.off_xs + tok * p.xs_tok + 4 * blk, __float_as_uint(exp2_int(-se)));
+            // value 8 qq + i of the block is byte j = 8 qq + i + 2 (+ 34) of the span
+            const uint32_t ent = sb + p.off_img + tok * p.img_tok + it * kItemImg + tt * 8;
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const int R = R0 + b, blk = R / 34, o = R - 34 * blk;
-                const uint32_t ib = lds32(sb + p.off_xs + tok * p.xs_tok + 4 * blk);
-                const float S = __uint_as_float(0x7F000000u - ib);
-                h[b] = o >= 2 ? hx(xval(p, sb, tok, 32 * blk + o - 2), S) : __float2half_rn(0.f);
+            for (int i = 0; i < 8; ++i) {
+                const float f = (i & 1) ? bf16hi_to_f32(wv[i >> 1]) : bf16lo_to_f32(wv[i >> 1]);
+                const int j = 8 * qq + i + 2 + 34 * odd, b = j & 3;
+                sts16(ent + (j >> 2) * 32 + 4 * (b & 1) + 2 * (b >> 1), hx(f, S));
             }
-            sts64(sb + p.off_img + tok * p.img_tok + it * kItemImg + mu * 32 + tt * 8, hpair(h[0], h[2]),
-                  hpair(h[1], h[3]));
+            if (qq == 0) {   // the block's scale bytes: span bytes 0, 1 (even) or 34, 35 (odd)
+                const int j0 = 34 * odd, b = j0 & 3;
+                sts16(ent + (j0 >> 2) * 32 + 4 * (b & 1) + 2 * (b >> 1), __float2half_rn(0.f));
+                sts16(ent + ((j0 + 1) >> 2) * 32 + 4 * ((b + 1) & 1) + 2 * ((b + 1) >> 1), __float2half_rn(0.f));
+            }
         }
-        return false;
+        return bad;
     }
 };
 
@@ -400,7 +404,6 @@ struct Q40 {
     static constexpr uint32_t kZero = kItemImg;
     static constexpr int kAccPerLane = 2 * NT;
     static constexpr int kXT = 14;
-    static constexpr bool kTwoPhase = true;
     static constexpr bool kSplit = false;
 
     static __device__ __forceinline__ void item(const SP& p, uint32_t sb, const Lane& L, uint32_t rowA,
@@ -473,35 +476,61 @@ struct Q40 {
         Q8<NT>::store_part(p, L, acc, part);
     }
 
-    // Phase 1: the block scales (stored as 2^-s per block).
-    static __device__ bool build_scales(const SP& p, uint32_t sb, int64_t xoff) {
-        return block_scales(p, sb, kXT);
-    }
-    // Phase 2: image entries (item, mu, low / high, t') = binary16 of the
-    // scaled activations of the 4 raw bytes at offset 144 item + 36 t' + 4 mu
-    // of a row, as (byte0, byte2 | byte1, byte3): the low nibble's value
-    // (x 2^s) or the high nibble's (x 2^s / 16); d bytes get 0.
+    // Image entries (item, mu, low / high, t') = binary16 of the scaled
+    // activations of the 4 raw bytes at offset 144 item + 36 t' + 4 mu of a
+    // row, as (byte0, byte2 | byte1, byte3): the low nibble's value (x 2^s)
+    // or the high nibble's (x 2^s / 16); d bytes get 0.  Eight neighbouring
+    // lanes share the span of lane t' (blocks b0 = 8 item + 2 t' and
+    // b0 + 1), each with 4 code bytes of one block (low values 4 qq + c, high
+    // values 16 + 4 qq + c): they agree on the block's scale 2^s by two
+    // shuffles, and lane 0 of the block stores 2^-s (4 bytes per block, in
+    // block order).  Returns whether this thread met a non-finite activation.
     static __device__ bool build(const SP& p, uint32_t sb, int64_t xoff) {
-        const int items = p.nblk / 8;
-        const int per_tok = items * 9 * 4;
-        for (int e = threadIdx.x; e < p.m * per_tok; e += kCW * 32) {
-            const int tok = e / per_tok, rem = e % per_tok;
-            const int it = rem / 36, mu = (rem % 36) >> 2, tt = rem & 3;
-            const int R0 = it * 144 + 36 * tt + 4 * mu;
-            __half lo[4], hi[4];
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const int R = R0 + b, blk = R / 18, o = R - 18 * blk;
-                const uint32_t ib = lds32(sb + p.off_xs + tok * p.xs_tok + 4 * blk);
-                const float S = __uint_as_float(0x7F000000u - ib);
-                lo[b] = o >= 2 ? hx(xval(p, sb, tok, 32 * blk + o - 2), S) : __float2half_rn(0.f);
-                hi[b] = o >= 2 ? hx(xval(p, sb, tok, 32 * blk + 14 + o), S * 0.0625f) : __float2half_rn(0.f);
+        bool bad = false;
+        const int spans = p.nblk / 2, total = p.m * spans * 8;
+        for (int w0 = threadIdx.x & ~31; w0 < total; w0 += kCW * 32) {
+            const int e = w0 + (threadIdx.x & 31);
+            const bool in = e < total;
+            const int sp = e >> 3, tok = sp / spans, s2 = sp - tok * spans;   // s2 = 4 item + t'
+            const int it = s2 >> 2, tt = s2 & 3, odd = (e >> 2) & 1, qq = e & 3;
+            const int blk = 2 * s2 + odd;
+            uint2 lo = make_uint2(0u, 0u), hi = make_uint2(0u, 0u);
+            if (in) {
+                lo = lds64(xaddr(p, sb, tok, 32 * blk + 4 * qq));
+                hi = lds64(xaddr(p, sb, tok, 32 * blk + 16 + 4 * qq));
             }
-            const uint32_t dst = sb + p.off_img + tok * p.img_tok + it * kItemImg + mu * 64 + tt * 8;
-            sts64(dst, hpair(lo[0], lo[2]), hpair(lo[1], lo[3]));
-            sts64(dst + 32, hpair(hi[0], hi[2]), hpair(hi[1], hi[3]));
+            uint32_t mx = absmax8_bf16(0u, make_uint4(lo.x, lo.y, hi.x, hi.y));
+            mx = max(mx & 0xFFFFu, mx >> 16);
+            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            bad |= in && mx >= 0x7F80u;
+            const int se = xscale_exp(mx, kXT);
+            const float S = exp2_int(se), S16 = S * 0.0625f;
+            if (!in) continue;   // lanes out of range occur in the last round only
+            if (qq == 0) sts32(sb + p.off_xs + tok * p.xs_tok + 4 * blk, __float_as_uint(exp2_int(-se)));
+            // code byte 4 qq + c of the block is byte j = 4 qq + c + 2 (+ 18) of the span
+            const uint32_t ent = sb + p.off_img + tok * p.img_tok + it * kItemImg + tt * 8;
+            const uint32_t lw[2] = {lo.x, lo.y}, hw[2] = {hi.x, hi.y};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int j = 4 * qq + c + 2 + 18 * odd, b = j & 3;
+                const uint32_t a = ent + (j >> 2) * 64 + 4 * (b & 1) + 2 * (b >> 1);
+                const float fl = (c & 1) ? bf16hi_to_f32(lw[c >> 1]) : bf16lo_to_f32(lw[c >> 1]);
+                const float fh = (c & 1) ? bf16hi_to_f32(hw[c >> 1]) : bf16lo_to_f32(hw[c >> 1]);
+                sts16(a, hx(fl, S));
+                sts16(a + 32, hx(fh, S16));
+            }
+            if (qq == 0) {   // the block's d bytes: span bytes 0, 1 (even) or 18, 19 (odd)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int j = 18 * odd + c, b = j & 3;
+                    const uint32_t a = ent + (j >> 2) * 64 + 4 * (b & 1) + 2 * (b >> 1);
+                    sts16(a, __float2half_rn(0.f));
+                    sts16(a + 32, __float2half_rn(0.f));
+                }
+            }
         }
-        return false;
+        return bad;
     }
 };
 
@@ -525,7 +554,6 @@ struct Q6 {
     // a run's scaled activations below 2^15: its x/16 and x/256 operands stay
     // normal binary16 numbers down to 2^-22 of the run's largest magnitude
     static constexpr int kXT = 14;
-    static constexpr bool kTwoPhase = false;
     static constexpr bool kSplit = false;
 
     // Word at shared address a: 4-byte aligned (MODE 0), 2 bytes past a
@@ -674,17 +702,14 @@ struct Q6 {
             const int se = xscale_exp(mx, kXT);
             const float sc = exp2_int(se) * (sl ? 0.00390625f : 0.0625f);
             const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            __half hv[16];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                hv[2 * u] = hx(bf16lo_to_f32(wv[u]), sc);
-                hv[2 * u + 1] = hx(bf16hi_to_f32(wv[u]), sc);
-            }
             const uint32_t img = sb + p.off_img + tok * p.img_tok + blk * kBlkImg + (8 * qp + 4 * sl) * 32 + tt * 8;
-            // values 4g .. 4g+3 go to entry k = (g - t') mod 4
+            // values 4g .. 4g+3 (words 2g, 2g+1) go to entry k = (g - t') mod 4
+            // as binary16 pairs (4g, 4g+2 | 4g+1, 4g+3)
 #pragma unroll
             for (int g = 0; g < 4; ++g)
-                sts64(img + ((g - tt) & 3) * 32, hpair(hv[4 * g], hv[4 * g + 2]), hpair(hv[4 * g + 1], hv[4 * g + 3]));
+                sts64(img + ((g - tt) & 3) * 32,
+                      pack_f16x2(bf16lo_to_f32(wv[2 * g]) * sc, bf16lo_to_f32(wv[2 * g + 1]) * sc),
+                      pack_f16x2(bf16hi_to_f32(wv[2 * g]) * sc, bf16hi_to_f32(wv[2 * g + 1]) * sc));
             sts32(sb + p.off_xs + tok * p.xs_tok + ((blk * 4 + tt) * 2 + qp) * 8 + 4 * sl,
                   __float_as_uint(exp2_int(-se)));
         }
@@ -712,7 +737,6 @@ struct Q4 {
     // a block's scaled activations below 2^10: a sub-block sum X_j (32
     // values) stays below 2^15, inside the binary16 range of its two-part split
     static constexpr int kXT = 9;
-    static constexpr bool kTwoPhase = false;
 
     static __device__ __forceinline__ void item(const SP& p, uint32_t sb, const Lane& L, uint32_t rowA,
                                                 uint32_t rowB, int gb, float (&acc)[4 * NT]) {
@@ -852,61 +876,72 @@ struct Q4 {
     // Image per block and token: MMA (nib, u) of lane t uses the scaled
     // values v = 64t + 32nib + 4u + {0,2 | 1,3}; the last 32 bytes hold (Xhi,
     // Xlo) of sub-blocks 2t and 2t+1, the sums of their binary16 operands.
-    // One thread per 64 values (token, block, t); the four threads of a block
-    // are neighbouring lanes and agree on the block's scale 2^s (largest |x|
-    // at 2^9) by two shuffles; 127 - s (the biased exponent of 2^-s) goes to
-    // the [block][16 tokens] byte table.
+    // Sixteen neighbouring lanes share a (token, block), one per (t, nib,
+    // half uu of u): 16 values each.  They agree on the block's scale 2^s
+    // (largest |x| at 2^9) by four shuffles and add the two halves of a
+    // sub-block sum by one; 127 - s (the biased exponent of 2^-s) goes to the
+    // [block][16 tokens] byte table.  Every warp runs the same number of
+    // rounds, so the shuffles always see the whole warp.
     // Returns whether this thread met a non-finite activation.
     static __device__ bool build(const SP& p, uint32_t sb, int64_t xoff) {
         bool bad = false;
-        const int items = p.m * p.nblk * 4;   // a multiple of 4: a block's lanes are all in or all out
-        for (int it = threadIdx.x; it < items; it += kCW * 32) {
-            const int tok = it / (p.nblk * 4), rem = it % (p.nblk * 4), bl = rem >> 2, t = rem & 3;
-            const uint32_t base = sb + p.off_img + tok * p.img_tok + bl * kBlkImg;
-            const int64_t xi = static_cast<int64_t>(bl) * 256 + 64 * t;
-            const uint32_t xs = xaddr(p, sb, tok, xi);
-            const uint16_t* xg = p.x + static_cast<int64_t>(tok) * p.k * p.ks + xoff + xi;
-            uint4 r[8];
-            uint32_t mx = 0;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                r[c] = p.x_global ? ldg_nc_v4(xg + 8 * c) : lds128(xs + 16 * c);
-                mx = absmax8_bf16(mx, r[c]);
+        const int total = p.m * p.nblk * 16;
+        // the 16 values of lane e: (token, block) e / 16, t, nib, uu from e
+        // mod 16; read a round ahead, so that a round's loads (from global
+        // memory when the image is built from x in place) are in flight while
+        // the previous round converts
+        auto load = [&](int e, uint4 (&r)[2]) {
+            r[0] = r[1] = make_uint4(0u, 0u, 0u, 0u);
+            if (e >= total) return;
+            const int q = e >> 4, tok = q / p.nblk, bl = q - tok * p.nblk;
+            const int64_t xi = static_cast<int64_t>(bl) * 256 + 64 * ((e >> 2) & 3) + 32 * ((e >> 1) & 1) + 16 * (e & 1);
+            if (p.x_global) {
+                const uint16_t* xg = p.x + static_cast<int64_t>(tok) * p.k * p.ks + xoff + xi;
+                r[0] = ldg_nc_v4(xg);
+                r[1] = ldg_nc_v4(xg + 8);
+            } else {
+                const uint32_t xs = xaddr(p, sb, tok, xi);
+                r[0] = lds128(xs);
+                r[1] = lds128(xs + 16);
             }
+        };
+        uint4 nx[2];
+        load((threadIdx.x & ~31) + (threadIdx.x & 31), nx);
+        for (int w0 = threadIdx.x & ~31; w0 < total; w0 += kCW * 32) {
+            const int e = w0 + (threadIdx.x & 31);
+            const bool in = e < total;
+            const int q = e >> 4, tok = q / p.nblk, bl = q - tok * p.nblk;
+            const int uu = e & 1, nib = (e >> 1) & 1, t = (e >> 2) & 3;
+            const uint32_t base = sb + p.off_img + tok * p.img_tok + bl * kBlkImg;
+            const uint4 r[2] = {nx[0], nx[1]};
+            load(e + kCW * 32, nx);
+            uint32_t mx = absmax8_bf16(absmax8_bf16(0u, r[0]), r[1]);
             mx = max(mx & 0xFFFFu, mx >> 16);
-            const unsigned grp = __activemask();
-            mx = max(mx, __shfl_xor_sync(grp, mx, 1));
-            mx = max(mx, __shfl_xor_sync(grp, mx, 2));
-            bad |= mx >= 0x7F80u;
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            bad |= in && mx >= 0x7F80u;
             const int se = xscale_exp(mx, kXT);
             const float S = exp2_int(se);
-            if (t == 0) sts8(sb + p.off_xs + 16 * bl + tok, static_cast<uint32_t>(127 - se));
-            float X[2] = {0.f, 0.f};
+            if (in && (e & 15) == 0) sts8(sb + p.off_xs + 16 * bl + tok, static_cast<uint32_t>(127 - se));
+            float X = 0.f;
+            const uint32_t wv[8] = {r[0].x, r[0].y, r[0].z, r[0].w, r[1].x, r[1].y, r[1].z, r[1].w};
 #pragma unroll
-            for (int nib = 0; nib < 2; ++nib) {
-#pragma unroll
-                for (int uu = 0; uu < 2; ++uu) {
-                    const uint4 r0 = r[4 * nib + 2 * uu], r1 = r[4 * nib + 2 * uu + 1];
-                    const uint32_t wv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int u = 4 * uu + q;
-                        const __half f0 = hx(bf16lo_to_f32(wv[2 * q]), S), f1 = hx(bf16hi_to_f32(wv[2 * q]), S);
-                        const __half f2 = hx(bf16lo_to_f32(wv[2 * q + 1]), S);
-                        const __half f3 = hx(bf16hi_to_f32(wv[2 * q + 1]), S);
-                        X[nib] += (__half2float(f0) + __half2float(f1)) + (__half2float(f2) + __half2float(f3));
-                        sts64(base + (nib * 8 + u) * 32 + t * 8, hpair(f0, f2), hpair(f1, f3));
-                    }
-                }
+            for (int qq = 0; qq < 4; ++qq) {
+                const int u = 4 * uu + qq;
+                // binary16 pairs (v0, v2) and (v1, v3) of the scaled values
+                const uint32_t h02 = pack_f16x2(bf16lo_to_f32(wv[2 * qq]) * S, bf16lo_to_f32(wv[2 * qq + 1]) * S);
+                const uint32_t h13 = pack_f16x2(bf16hi_to_f32(wv[2 * qq]) * S, bf16hi_to_f32(wv[2 * qq + 1]) * S);
+                X = add_f16hi(h13, add_f16hi(h02, add_f16lo(h13, add_f16lo(h02, X))));
+                if (in) sts64(base + (nib * 8 + u) * 32 + t * 8, h02, h13);
             }
-            uint32_t e[2];
-#pragma unroll
-            for (int nib = 0; nib < 2; ++nib) {
-                const __half hi = __float2half_rn(X[nib]);
-                const __half lo = __float2half_rn(X[nib] - __half2float(hi));
-                e[nib] = hpair(hi, lo);
+            // the sub-block sum: this half plus the other (lane e ^ 1), in uu order
+            const float Xo = __shfl_xor_sync(0xffffffffu, X, 1);
+            if (in && uu == 0) {
+                const float Xs = X + Xo;
+                const __half hi = __float2half_rn(Xs);
+                const __half lo = __float2half_rn(Xs - __half2float(hi));
+                sts32(base + 512 + t * 8 + 4 * nib, hpair(hi, lo));
             }
-            sts64(base + 512 + t * 8, e[0], e[1]);
         }
         return bad;
     }
@@ -1187,14 +1222,9 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_stream_kernel(const P p) {
         Lane L;
         L.g = lane >> 2;
         L.t = lane & 3;
-        if (!spin_wait(xbar, 0, p.status)) *abort_flag = 1;
-        // the activation image with its per-block scales (q8_0: the scales
-        // first, the image entries of a block read them)
+        if (!spin_wait(xbar, 0, p.status, p.strict)) *abort_flag = 1;
+        // the activation image with its per-block (or per-run) scales
         bool bad = false;
-        if constexpr (C::kTwoPhase) {
-            if (!*abort_flag) bad = C::build_scales(p, sb, kb0 * C::kVPB);
-            asm volatile("bar.sync 1, %0;" ::"r"(kCW * 32) : "memory");
-        }
         if (!*abort_flag) {
             bad |= C::build(p, sb, kb0 * C::kVPB);
             for (uint32_t o = 4 * tid; o < C::kZero; o += 4 * kCW * 32) sts32(sb + p.off_zero + o, 0u);
@@ -1424,6 +1454,11 @@ int launch_stream(const void* w, int64_t n, int64_t k, const uint16_t* x, int m,
     p.x = x;
     p.y = y;
     p.status = device_status_ptr();
+    {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        p.strict = dev >= 0 && dev < 64 && g_strict_wait[dev] ? 1 : 0;
+    }
     p.n = n;
     p.m = m;
     const int nblk_all = static_cast<int>(k / C::kVPB);
@@ -1576,6 +1611,9 @@ uint32_t q4_inv_tok(int nblk, int m) { return align16(static_cast<uint32_t>(cdiv
 // (ns == 0: the default).
 int set_stream_wait_limit(uint64_t ns) {
     const uint64_t v = ns ? ns : kWaitLimitNs;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64) g_strict_wait[dev] = v < kWaitLimitNs;
     return record_cuda(cudaMemcpyToSymbol(g_wait_ns, &v, sizeof(v)));
 }
 
