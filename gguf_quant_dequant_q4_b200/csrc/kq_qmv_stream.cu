@@ -948,6 +948,180 @@ struct Q4 {
 };
 
 // ===========================================================================
+// q4_K and q5_K at one activation row (column form)
+// ===========================================================================
+// With a single token the 8 MMA columns are free to separate sub-blocks, as in
+// q6_K: lane t's low nibbles (sub-block 2t) go to column 2t, its high nibbles
+// (sub-block 2t+1) to column 2t+1, each B lane of another column reading a
+// zero block.  The codes then enter the MMA as plain binary16 subnormals (q
+// 2^-24; the high nibble in place, 16 q 2^-24, against x/16) and the 6-bit
+// scales and mins are applied once per block in the fp32 epilogue:
+//   y += 2^-s (d sc_2t 2^24 D_2t + d sc_2t+1 2^24 D_2t+1 - dmin (m_2t X_2t + m_2t+1 X_2t+1)),
+// X_j the fp32 sum of sub-block j's binary16 operands as the MMA consumed
+// them (x 2^s, resp. 16 binary16(x 2^s / 16)).  No per-code scale product,
+// no min-term MMA.  q5_K: the fifth bit merged into the code (q <= 31).
+template <bool FIVE = false>
+struct Q4C {
+    static constexpr int kVPB = 256, kBPB = FIVE ? 176 : 144;
+    static constexpr bool kSplit = false;
+    static constexpr int kItemBlocks = 1;
+    // image per block: 16 MMAs x 4 lanes x 8 bytes, then X_2t, X_2t+1 (fp32) per lane
+    static constexpr uint32_t kBlkImg = 544;
+    static constexpr uint32_t kZero = 512;
+    static constexpr int kAccPerLane = 2;
+    // a block's scaled activations below 2^15: far inside binary16
+    static constexpr int kXT = 14;
+
+    static __device__ __forceinline__ void item(const SP& p, uint32_t sb, const Lane& L, uint32_t rowA,
+                                                uint32_t rowB, int gb, float (&acc)[2]) {
+        const int t = L.t;
+        const uint32_t img = sb + p.off_img + gb * kBlkImg;
+        const uint32_t zero = sb + p.off_zero + 8 * t;
+        // B lanes whose column holds lane t's low (2t) or high (2t+1) sub-block
+        const uint32_t blo = L.g == 2 * t ? img + 8 * t : zero;
+        const uint32_t bhi = L.g == 2 * t + 1 ? img + 256 + 8 * t : zero;
+        const uint4 hA = lds128(rowA), hB = lds128(rowB);
+        constexpr uint32_t kQs = FIVE ? 48 : 16;   // first code byte
+        const uint4 qA0 = lds128(rowA + kQs + 32 * t), qA1 = lds128(rowA + kQs + 16 + 32 * t);
+        const uint4 qB0 = lds128(rowB + kQs + 32 * t), qB1 = lds128(rowB + kQs + 16 + 32 * t);
+        uint32_t fA[8], fB[8];   // q5_K: qh[4u .. 4u+3] >> 2t (the lane's two bits at bits 0, 1 of each byte)
+        if constexpr (FIVE) {
+            const uint4 hA0 = lds128(rowA + 16), hA1 = lds128(rowA + 32);
+            const uint4 hB0 = lds128(rowB + 16), hB1 = lds128(rowB + 32);
+            const uint32_t ha[8] = {hA0.x, hA0.y, hA0.z, hA0.w, hA1.x, hA1.y, hA1.z, hA1.w};
+            const uint32_t hb[8] = {hB0.x, hB0.y, hB0.z, hB0.w, hB1.x, hB1.y, hB1.z, hB1.w};
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                fA[u] = ha[u] >> (2 * t);
+                fB[u] = hb[u] >> (2 * t);
+            }
+        }
+        const uint32_t wA[8] = {qA0.x, qA0.y, qA0.z, qA0.w, qA1.x, qA1.y, qA1.z, qA1.w};
+        const uint32_t wB[8] = {qB0.x, qB0.y, qB0.z, qB0.w, qB1.x, qB1.y, qB1.z, qB1.w};
+        float D[4][4];   // four independent MMA chains
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) D[c][e] = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const uint32_t a = wA[u], b = wB[u], a8 = a >> 8, b8 = b >> 8;
+            uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
+            if constexpr (FIVE) {
+                const uint32_t fa = fA[u], fb = fB[u];
+                a0 = vbitsel(a, vand_or(fa << 4, 0x00100010u, 0u), 0x000F000Fu);
+                a1 = vbitsel(b, vand_or(fb << 4, 0x00100010u, 0u), 0x000F000Fu);
+                a2 = vbitsel(a8, vand_or(fa >> 4, 0x00100010u, 0u), 0x000F000Fu);
+                a3 = vbitsel(b8, vand_or(fb >> 4, 0x00100010u, 0u), 0x000F000Fu);
+                c0 = vbitsel(a, vand_or(fa << 7, 0x01000100u, 0u), 0x00F000F0u);
+                c1 = vbitsel(b, vand_or(fb << 7, 0x01000100u, 0u), 0x00F000F0u);
+                c2 = vbitsel(a8, vand_or(fa >> 1, 0x01000100u, 0u), 0x00F000F0u);
+                c3 = vbitsel(b8, vand_or(fb >> 1, 0x01000100u, 0u), 0x00F000F0u);
+            } else {
+                a0 = vand_or(a, 0x000F000Fu, 0u);
+                a1 = vand_or(b, 0x000F000Fu, 0u);
+                a2 = vand_or(a8, 0x000F000Fu, 0u);
+                a3 = vand_or(b8, 0x000F000Fu, 0u);
+                c0 = vand_or(a, 0x00F000F0u, 0u);
+                c1 = vand_or(b, 0x00F000F0u, 0u);
+                c2 = vand_or(a8, 0x00F000F0u, 0u);
+                c3 = vand_or(b8, 0x00F000F0u, 0u);
+            }
+            const uint2 bl = lds64(blo + u * 32);
+            const uint2 bh = lds64(bhi + u * 32);
+            mma_f16(D[u & 3], a0, a1, a2, a3, bl.x, bl.y);
+            mma_f16(D[u & 3], c0, c1, c2, c3, bh.x, bh.y);
+        }
+        // 6-bit scale/min codes of sub-blocks 2t, 2t+1 as (code_2t, code_2t+1)
+        // in bits 0..5 / 16..21.  t < 2: sc = s[j] & 63, m = s[j+4] & 63;
+        // t >= 2 (j >= 4): sc = (s[j+4] & 15) | (s[j-4] >> 6) << 4,
+        // m = (s[j+4] >> 4) | (s[j] >> 6) << 4.
+        const bool lo = t < 2;
+        const uint32_t jj0 = (2 * t) & 3;
+        const uint32_t sel = 0x4040u | jj0 | ((jj0 + 1) << 8);
+        const uint32_t mka = lo ? 0x003F003Fu : 0x000F000Fu, mkb = lo ? 0u : 0x00300030u;
+        const uint2 xv = lds64(img + 512 + 8 * t);   // X_2t, X_2t+1
+        const float X0 = __uint_as_float(xv.x), X1 = __uint_as_float(xv.y);
+        const float iv = __uint_as_float(static_cast<uint32_t>(lds_u16(sb + p.off_xs + 16 * gb) & 0xFFu) << 23);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const uint4 hh = r ? hB : hA;
+            const uint32_t asc = lo ? hh.y : hh.w;
+            const uint32_t am = lo ? hh.z : (hh.w >> 4);
+            const uint32_t scp = (__byte_perm(asc, 0, sel) & mka) | ((__byte_perm(hh.y, 0, sel) >> 2) & mkb);
+            const uint32_t mp = (__byte_perm(am, 0, sel) & mka) | ((__byte_perm(hh.z, 0, sel) >> 2) & mkb);
+            const float d24 = h2f(hh.x & 0xffff) * kTwo24, dm = h2f(hh.x >> 16);
+            const float D0 = (D[0][2 * r] + D[1][2 * r]) + (D[2][2 * r] + D[3][2 * r]);
+            const float D1 = (D[0][2 * r + 1] + D[1][2 * r + 1]) + (D[2][2 * r + 1] + D[3][2 * r + 1]);
+            const float sc0 = static_cast<float>(scp & 0xFFFFu), sc1 = static_cast<float>(scp >> 16);
+            const float m0 = static_cast<float>(mp & 0xFFFFu), m1 = static_cast<float>(mp >> 16);
+            const float v = fmaf(__fmul_rn(d24, sc0), D0, fmaf(__fmul_rn(d24, sc1), D1, -dm * fmaf(m0, X0, m1 * X1)));
+            acc[r] = fmaf(iv, v, acc[r]);
+        }
+    }
+
+    static __device__ __forceinline__ void store_part(const SP& p, const Lane& L, float (&acc)[2], float* part) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            float v = acc[r];
+            v += __shfl_xor_sync(0xffffffffu, v, 1);
+            v += __shfl_xor_sync(0xffffffffu, v, 2);
+            if (L.t == 0) part[(L.g + 8 * r) * p.m] = v;
+        }
+    }
+
+    // Image per (token, block): entry (nib, u, t) = binary16 of lane t's values
+    // 64t + 32nib + 4u + {0,2 | 1,3}, scaled by 2^s (nib 0) or 2^s / 16 (nib
+    // 1, against the high nibble in place), at 256 nib + 32 u + 8 t; then the
+    // fp32 sums X_2t, X_2t+1 at 512 + 8t.  Sixteen neighbouring lanes share a
+    // block, one per (t, nib, half uu of u): they agree on the block's scale
+    // 2^s (largest |x| at 2^14) by four shuffles and add the two halves of a
+    // sub-block sum by one; 127 - s goes to the [block][16 tokens] byte table.
+    // Every warp runs the same number of rounds, so the shuffles always see
+    // the whole warp.  Returns whether this thread met a non-finite activation.
+    static __device__ bool build(const SP& p, uint32_t sb, int64_t xoff) {
+        bool bad = false;
+        const int total = p.m * p.nblk * 16;
+        for (int w0 = threadIdx.x & ~31; w0 < total; w0 += kCW * 32) {
+            const int e = w0 + (threadIdx.x & 31);
+            const bool in = e < total;
+            const int q = e >> 4, tok = q / p.nblk, bl = q - tok * p.nblk;
+            const int uu = e & 1, nib = (e >> 1) & 1, t = (e >> 2) & 3;
+            uint4 r[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+            if (in) {
+                const uint32_t xs = xaddr(p, sb, tok, static_cast<int64_t>(bl) * 256 + 64 * t + 32 * nib + 16 * uu);
+                r[0] = lds128(xs);
+                r[1] = lds128(xs + 16);
+            }
+            uint32_t mx = absmax8_bf16(absmax8_bf16(0u, r[0]), r[1]);
+            mx = max(mx & 0xFFFFu, mx >> 16);
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            bad |= in && mx >= 0x7F80u;
+            const int se = xscale_exp(mx, kXT);
+            const float S = exp2_int(se) * (nib ? 0.0625f : 1.0f);
+            const uint32_t base = sb + p.off_img + tok * p.img_tok + bl * kBlkImg;
+            if (in && (e & 15) == 0) sts8(sb + p.off_xs + 16 * bl + tok, static_cast<uint32_t>(127 - se));
+            float X = 0.f;
+            const uint32_t wv[8] = {r[0].x, r[0].y, r[0].z, r[0].w, r[1].x, r[1].y, r[1].z, r[1].w};
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+                const int u = 4 * uu + qq;
+                const uint32_t h02 = pack_f16x2(bf16lo_to_f32(wv[2 * qq]) * S, bf16lo_to_f32(wv[2 * qq + 1]) * S);
+                const uint32_t h13 = pack_f16x2(bf16hi_to_f32(wv[2 * qq]) * S, bf16hi_to_f32(wv[2 * qq + 1]) * S);
+                X = add_f16hi(h13, add_f16hi(h02, add_f16lo(h13, add_f16lo(h02, X))));
+                if (in) sts64(base + nib * 256 + u * 32 + t * 8, h02, h13);
+            }
+            // the sub-block sum: this half plus the other (lane e ^ 1); the
+            // high sub-block's operands stand for 16 times their value
+            const float Xs = (X + __shfl_xor_sync(0xffffffffu, X, 1)) * (nib ? 16.0f : 1.0f);
+            if (in && uu == 0) sts32(base + 512 + t * 8 + 4 * nib, __float_as_uint(Xs));
+        }
+        return bad;
+    }
+};
+
+// ===========================================================================
 // Kernel
 // ===========================================================================
 // SPLIT: the launch is in clusters of p.ks CTAs that split K (compiled out
@@ -1631,6 +1805,10 @@ int launch_q4family(const void* w, int64_t n, int64_t k, const uint16_t* x, int 
         if (nblk % 4 == 0 && nblk / 4 >= 7) ks = 4;
         else if (nblk % 2 == 0 && nblk / 2 >= 7) ks = 2;
     }
+    if (m == 1) {   // one row: the column form (scales in the epilogue)
+        const int rc = launch_stream<Q4C<FIVE>>(w, n, k, x, 1, y, s, nblk * Q4C<FIVE>::kBlkImg, q4_inv_tok(nblk, 1));
+        if (rc != KQ_ERR_UNSUPPORTED) return rc;
+    }
     for (;;) {
         // per-token image stride 32 bytes past a multiple of 128: the 8
         // tokens of an MMA's B fragment then read disjoint banks
@@ -1701,6 +1879,12 @@ int launch_gather_qmv(int type, const void* w_bank, const void* w_bank2, int act
         uint32_t it = nblk * Q4<1>::kBlkImg;
         it += (32u - it % 128u + 128u) % 128u;
         for (int m = m_cap < 16 ? m_cap : 16; m >= 1; --m) {
+            if (m == 1) {   // one row per virtual expert: the column form
+                const uint32_t it1 = nblk * Q4C<>::kBlkImg;
+                rc = type == KQ_Q4_K ? launch_stream<Q4C<false>>(w_bank, n, k, x, 1, y, s, it1, q4_inv_tok(nblk, 1), 1, &ga)
+                                     : launch_stream<Q4C<true>>(w_bank, n, k, x, 1, y, s, it1, q4_inv_tok(nblk, 1), 1, &ga);
+                if (rc != KQ_ERR_UNSUPPORTED) return rc;
+            }
             if (type == KQ_Q4_K)
                 rc = m <= 8 ? launch_stream<Q4<1>>(w_bank, n, k, x, m, y, s, it, q4_inv_tok(nblk, m), 1, &ga)
                             : launch_stream<Q4<2>>(w_bank, n, k, x, m, y, s, it, q4_inv_tok(nblk, m), 1, &ga);

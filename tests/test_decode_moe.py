@@ -176,8 +176,11 @@ def check_glu(y, out, g, u, ag, au, act):
 
 @pytest.mark.parametrize("qtype", [kq.Q4_K, kq.Q6_K, kq.Q8_0, kq.Q5_K, kq.Q4_0])
 @pytest.mark.parametrize("act", [kq.ACT_SILU, kq.ACT_GELU_TANH, kq.ACT_SILU_LIMIT])
-def test_moe_glu_gather_vs_oracle(qtype, act):
-    tokens, top_k, experts, n, k = 3, 2, 5, 333, 2048
+@pytest.mark.parametrize("tokens", [1, 3])
+def test_moe_glu_gather_vs_oracle(qtype, act, tokens):
+    # one token: every virtual expert has one activation row (the q4_K / q5_K
+    # column form); three: batched rows
+    top_k, experts, n, k = 2, 5, 333, 2048
     wg = synth.weights(qtype, n, k, seed=101, experts=experts)
     wu = synth.weights(qtype, n, k, seed=102, experts=experts)
     ids = synth.routing(tokens, experts, top_k, seed=103)
