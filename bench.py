@@ -72,13 +72,37 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text: str) -> str:
+    """C/CUDA source without its comments and with whitespace collapsed, so that
+    an edit of comments alone keeps a kernel's hash (string literals are kept)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"':
+            j = i + 1
+            while j < n and text[j] != '"':
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash(tag: str | None = None) -> str:
-    """Hash of the kernel sources (of one roofline tag's kernel, or of all)."""
+    """Hash of the kernel sources' code (of one roofline tag's kernel, or of all)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gguf_quant_dequant_q4_b200", "csrc")
     files = KERNEL_SOURCES.get(tag) if tag else None
     for f in sorted(files or os.listdir(csrc)):
-        h.update(open(os.path.join(csrc, f), "rb").read())
+        h.update(_code_only(open(os.path.join(csrc, f), encoding="utf-8", errors="replace").read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -24,9 +24,10 @@
 //    (1024 + code, exactly) and removes the 1024 with the HFMA2 that also
 //    applies its scale; q6_K and q8_0 put the code's bits in the mantissa with
 //    exponent field 0, a subnormal code x 2^-24 (exact; the tensor core keeps
-//    subnormal operands exact), and the codec's own offset (32, 128) is
-//    removed in the fp32 epilogue with a per-sub-block sum of the activation
-//    operands; the 2^24 goes into the per-block scale.
+//    subnormal operands exact), and subtract the codec's own offset from that
+//    subnormal before the MMA (q8_0: 128, q6_K: 2 from its high 2-bit field),
+//    exactly, so that a zero weight contributes exactly zero; the 2^24 goes
+//    into the per-block scale.
 //  * q4_K (per-block scales d, dmin): each lane owns one 64-value group of a
 //    block, so it decodes only its own two 6-bit scale/min pairs; the MMA
 //    chain runs over the whole block and the min term sum_j m_j * X_j is one

@@ -1,52 +1,62 @@
-// kq_qmv for 1 <= m <= 2 (q8_0, q6_K) or m <= 16 (q4_K): y = x . W^T.
+// kq_qmv for 1 <= m <= 2 (q8_0, q6_K, q4_0) or m <= 16 (q4_K, q5_K):
+// y = x . W^T; also the decode MoE products (gather and GLU modes).
 //
 // mlx-kquant bindings.cpp `quantized_matmul` (x @ dequant(w).T) and README
 // "How it works" (small row counts take a kernel that amortizes each weight
-// read over all rows); hanzo-ml quantized/mod.rs (decode multiplies "straight
-// out of the block format").  Block layouts: mlx-kquant README, "Codec
-// reference"; gguf-py constants (q4_K 144 B, q6_K 210 B, q8_0 34 B).
+// read over all rows); hanzo-ml quantized/mod.rs (decode multiplies directly
+// on the packed blocks).  Block layouts: mlx-kquant README, "Codec
+// reference"; gguf-py constants (q4_K 144 B, q5_K 176 B, q6_K 210 B, q8_0
+// 34 B, q4_0 18 B).
 //
 // Streaming.  One CTA per SM owns a balanced contiguous range of rows.  A
 // producer warp streams 16-row stages (whole rows when they fit, else equal
 // row slices) into a ring of shared-memory slots with one 1-D bulk copy per
 // row; big contiguous copies are what keeps HBM busy.  Before the first
 // stage it copies the activation rows, so they land first.  16 consumer
-// warps split every stage into work items and release the slot through an
-// mbarrier; the producer never waits for anything else.
+// warps build the activation image, then split every stage into work items
+// and release the slot through an mbarrier; the producer never waits for
+// anything else.
 //
 // Arithmetic is the exact-integer tensor-core scheme: a lane turns its codes
-// into binary16 integers (OR into the mantissa of 1024), the activations
-// rounded once to binary16 are the B operand of m16n8k16 MMAs, and the tensor
-// core accumulates exact products in fp32; per-block scales are applied in
-// fp32 once a block is complete.  Before that rounding each token's
-// activations are scaled by a power of two that puts its largest magnitude
-// at 2^T (T per codec), and the inverse scale is applied to its fp32 sums, so
-// the relative precision does not depend on the activations' magnitude.  The
-// q8_0 and q6_K codes enter the MMA as binary16 subnormals (the code's bits in
-// the mantissa, exponent field 0: code x 2^-24, exact; the tensor core keeps
-// subnormal operands exact), so the only offset left is the codec's own (128
-// for q8_0's unsigned view of the int8 code, 32 for q6_K), removed in the fp32
-// epilogue with sums of the very binary16 activation operands the MMAs
-// consumed; the 2^24 goes into the per-block scale.  The activation operand of every MMA is
-// precomputed per CTA into a shared-memory image in fragment order (one
-// 8-byte load per MMA); B lanes whose column does not receive a given word
-// read a zero block instead of being masked.  The lane-to-byte mappings:
+// into binary16 integers, the activations rounded once to binary16 are the B
+// operand of m16n8k16 MMAs, and the tensor core accumulates exact products in
+// fp32; per-block scales are applied in fp32 once a block is complete.
+// Before that rounding each run of activations (a block, or a 16-value run of
+// q6_K) is scaled by a power of two that puts its largest magnitude at 2^T
+// (T per codec), and the inverse scale is applied to its fp32 sums, so the
+// relative precision does not depend on the activations' magnitude.  Codes
+// enter the MMA as binary16 subnormals (the code's bits in the mantissa,
+// exponent field 0: code x 2^-24, exact; the tensor core keeps subnormal
+// operands exact), centred on the codec's offset before the MMA (q8_0: 128
+// of the unsigned view of the int8 code, q4_0: 8, q6_K: 32) by one exact
+// sub.f16x2, so a zero weight contributes exactly zero however large its
+// activation; the 2^24 goes into the per-block scale.  q4_K / q5_K at m >= 2
+// multiply their codes by the 6-bit scale exactly in binary16 instead (1024 +
+// code, scaled and the 1024 removed by one HFMA2).  The activation operand of
+// every MMA is precomputed per CTA into a shared-memory image in fragment
+// order (one 8-byte load per MMA); B lanes whose column does not receive a
+// given word read a zero block instead of being masked.  The lane-to-byte
+// mappings:
 //
 //  * q8_0, item = 16 rows x 8 blocks: lane t owns blocks 2t and 2t+1 (68
 //    bytes, word aligned) and feeds one 32-bit word per MMA.  Words 0..8 hold
 //    codes of the even block only (its fp16 scale bytes and the odd block's
 //    get a zero activation), words 9..16 those of the odd block, so MMA
 //    column 2t + parity collects exactly lane t's block of that parity.
+//  * q4_0, item = 16 rows x 8 blocks: as q8_0 with 36-byte spans and two MMAs
+//    per word (low nibbles against x, high nibbles in place against x/16).
 //  * q6_K, item = 16 rows x 1 block: lane t owns a quarter (half h, 16-value
 //    run lh) of the block for all four q; nibble and 2-bit field are merged
 //    into the 6-bit code with two LOP3s; columns 2t, 2t+1 hold its low- and
 //    high-nibble sub-blocks of the current pass.  The four lanes of a row read
 //    their words in a rotated order, which keeps the loads free of bank
 //    conflicts.
-//  * q4_K, item = 16 rows x 1 block: lane t owns values 64t..64t+63 and
-//    multiplies its 4-bit codes by the 6-bit scale exactly in binary16
-//    (q sc <= 945); one column per token; the min term is one more MMA on
-//    (m_j) x (X_j split into two binary16 halves).
+//  * q4_K / q5_K, item = 16 rows x 1 block: lane t owns values 64t..64t+63.
+//    At m >= 2 one column per token, the scale in the operand (q sc <= 945,
+//    <= 1953 with q5_K's fifth bit) and the min term as one more MMA on
+//    (m_j) x (X_j split into two binary16 halves).  At m = 1 (Q4C) the
+//    columns separate lane t's two sub-blocks instead, and scale and min are
+//    applied in the fp32 epilogue.
 //
 // Partial sums of the 16 warps are combined in a fixed order by the last
 // warp to finish a row group: results are bitwise reproducible.

@@ -74,20 +74,23 @@ def test_cpu_sample_is_bounded():
 
 
 def test_traffic_keyed_by_kernel_device_sources(tmp_path, monkeypatch):
-    # the roofline's DRAM traffic is reported only while the sources of the
-    # profiled kernel are the ones the counters were taken on; a host-only
-    # launch header does not count, a change to the kernel's file does
+    # the roofline's DRAM traffic is reported only while the code of the
+    # profiled kernel is the one the counters were taken on; a host-only
+    # launch header and comments do not count, a code change in the kernel's
+    # file does
     csrc = tmp_path / "gguf_quant_dequant_q4_b200" / "csrc"
     csrc.mkdir(parents=True)
     for f in ("kq_qmv_stream.cu", "kq_device.cuh", "kq_launch.h"):
-        (csrc / f).write_text(f"// {f}\n")
+        (csrc / f).write_text(f"// {f}\nint v_{f.split('.')[0]} = 1;\n")
     (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     tag = "qmv_q6_K_m1_14336x4096"
     h = bench.kernel_source_hash(tag)
     (tmp_path / "profiles" / "p.txt").write_text(f"summary\ntraffic {tag} 48223488 {h}\n")
     assert bench.profiled_traffic(tag) == 48223488
-    (csrc / "kq_launch.h").write_text("// a new host declaration\n")
+    (csrc / "kq_launch.h").write_text("// a new host declaration\nint launch(int);\n")
     assert bench.profiled_traffic(tag) == 48223488
-    (csrc / "kq_qmv_stream.cu").write_text("// the kernel changed\n")
+    (csrc / "kq_qmv_stream.cu").write_text("/* reworded */ // comments only\nint v_kq_qmv_stream  =  1;\n")
+    assert bench.profiled_traffic(tag) == 48223488
+    (csrc / "kq_qmv_stream.cu").write_text("// the kernel changed\nint v_kq_qmv_stream = 2;\n")
     assert bench.profiled_traffic(tag) is None
