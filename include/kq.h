@@ -108,14 +108,17 @@ int kq_read_device_status(int32_t* host_status, int clear);
 
 /*
  * kq_set_wait_limit - time limit, in ns, of every pipeline wait of the staged
- * decode kernel (kq_qmv at m <= 2 for q8_0 / q6_K and q4_K shapes it covers,
- * kq_gather_qmv, kq_moe_glu_gather) on the current device; ns <= 0 restores
- * the default of 2 s.  Host call, synchronous.  A wait that runs out sets
- * KQ_DEV_TIMEOUT in the library status word and the kernel winds down
- * (letting its own copies land) without finishing: its outputs are then
- * incomplete.  A short limit exists so that fault-handling tests can make a
- * wait run out on purpose; production code has no reason to call it.
- * No counterpart on the pages (the failure handling of this library).
+ * decode kernel (kq_qmv on the shapes it covers: m <= 2 for q8_0 / q6_K /
+ * q4_0, q4_K / q5_K while their activation image fits; kq_gather_qmv,
+ * kq_moe_glu_gather) on the current device, for launches made after the
+ * call; ns <= 0 restores the default of 2 s.  Host call, synchronous.  A wait
+ * that runs out sets KQ_DEV_TIMEOUT in the library status word and the kernel
+ * winds down (letting its own copies land) without finishing: its outputs
+ * are then incomplete.  Under a limit shorter than the default the first
+ * wait for the activation copy only tests it, so that wait runs out unless
+ * the copy has landed.  A short limit exists so that fault-handling tests
+ * can make a wait run out on purpose; production code has no reason to call
+ * it.  No counterpart on the pages (the failure handling of this library).
  */
 int kq_set_wait_limit(int64_t ns);
 
