@@ -86,3 +86,11 @@ def test_deterministic_and_row_independent(qtype):
     x2[[0, 1, 3, 4, 5]] = synth.activations(5, k, seed=9)
     c = kq.qmv(dev_bf16(x2), w, qtype)
     assert torch.equal(a[2], c[2])
+
+
+@pytest.mark.parametrize("qtype", [kq.Q4_K, kq.Q5_K])
+def test_one_row_long_k_falls_back(qtype):
+    # K = 65536: the one-row column form's activation image and raw copy do
+    # not fit in shared memory, so the call takes the scale-in-operand form
+    # (split over a cluster or with the image built from x in place)
+    run(qtype, 40, 65536, 1, seed=77)
