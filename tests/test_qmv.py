@@ -94,3 +94,13 @@ def test_one_row_long_k_falls_back(qtype):
     # not fit in shared memory, so the call takes the scale-in-operand form
     # (split over a cluster or with the image built from x in place)
     run(qtype, 40, 65536, 1, seed=77)
+
+
+@pytest.mark.parametrize("qtype", [kq.Q8_0, kq.Q6_K])
+@pytest.mark.parametrize("n,k", [(2600, 4096), (2664, 14336), (150, 1024)])
+def test_one_and_two_row_groups(qtype, n, k):
+    # 17 or 18 rows per CTA (1 or 2 rows per CTA at N = 150) leave row groups
+    # of one or two rows in the 16-row tensor-core items; K = 14336 splits
+    # every row over several stages
+    run(qtype, n, k, 1, seed=n + k)
+    run(qtype, n, k, 2, seed=n + k + 1)
