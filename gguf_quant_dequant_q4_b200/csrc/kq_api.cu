@@ -38,12 +38,17 @@ int block_geometry(int type, int* vpb, int* bpb) {
     }
 }
 
-// Common checks of (codec, W, n, k): codec known, k a positive block multiple,
-// n >= 0, W non-null and 16-byte aligned when there is work.
+// Largest k of any call: the kernels count a row's values and blocks in
+// 32-bit integers.
+constexpr int64_t kMaxK = (int64_t(1) << 31) - 1;
+
+// Common checks of (codec, W, n, k): codec known, k a positive block multiple
+// of at most kMaxK values, n >= 0, W non-null and 16-byte aligned when there
+// is work.
 int check_weights(int type, const void* w, int64_t n, int64_t k) {
     int vpb, bpb;
     if (block_geometry(type, &vpb, &bpb)) return KQ_ERR_UNSUPPORTED;
-    if (k <= 0 || k % vpb != 0 || n < 0) return KQ_ERR_INVALID_ARG;
+    if (k <= 0 || k > kMaxK || k % vpb != 0 || n < 0) return KQ_ERR_INVALID_ARG;
     if (n > 0 && !w) return KQ_ERR_INVALID_ARG;
     if (n > 0 && !aligned16(w)) return KQ_ERR_ALIGNMENT;
     return KQ_OK;
@@ -164,7 +169,7 @@ int kq_dequantize(int type, const void* w, int64_t n_rows, int64_t k, float* out
 int kq_quantize(int type, const float* w, int64_t n_rows, int64_t k, void* out, void* stream) {
     int vpb, bpb;
     if (block_geometry(type, &vpb, &bpb)) return KQ_ERR_UNSUPPORTED;
-    if (k <= 0 || k % vpb != 0 || n_rows < 0) return KQ_ERR_INVALID_ARG;
+    if (k <= 0 || k > kMaxK || k % vpb != 0 || n_rows < 0) return KQ_ERR_INVALID_ARG;
     if (n_rows == 0) return KQ_OK;
     if (!w || !out) return KQ_ERR_INVALID_ARG;
     if (!aligned16(w) || !aligned16(out)) return KQ_ERR_ALIGNMENT;
@@ -195,11 +200,12 @@ int kq_moe_sort(const int32_t* topk_ids, int64_t n_tokens, int32_t top_k, int32_
                 int64_t k, uint32_t* sorted_ids, int32_t* sorted_pair, int32_t* inv_order, uint16_t* x_sorted,
                 int32_t* err_flag, void* stream) {
     if (n_tokens < 0 || top_k < 1 || n_experts < 1 || n_experts > 256) return KQ_ERR_INVALID_ARG;
-    if (n_tokens * top_k > (int64_t(1) << 30)) return KQ_ERR_INVALID_ARG;
+    // the token count is bounded first, so that the pair count cannot overflow
+    if (n_tokens > (int64_t(1) << 30) || n_tokens * top_k > (int64_t(1) << 30)) return KQ_ERR_INVALID_ARG;
     if (n_tokens == 0) return KQ_OK;
     if (!topk_ids || !sorted_ids || !sorted_pair) return KQ_ERR_INVALID_ARG;
     if (x_sorted) {
-        if (!x || k <= 0 || k % 8 != 0) return KQ_ERR_INVALID_ARG;
+        if (!x || k <= 0 || k > kMaxK || k % 8 != 0) return KQ_ERR_INVALID_ARG;
         if (!aligned16(x) || !aligned16(x_sorted)) return KQ_ERR_ALIGNMENT;
     }
     return launch_moe_sort(topk_ids, n_tokens, top_k, n_experts, x, k, sorted_ids, sorted_pair, inv_order, x_sorted,

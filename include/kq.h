@@ -46,7 +46,7 @@
  *    (KQ_ERR_UNSUPPORTED otherwise).
  *  - `k` must be a multiple of the codec's values_per_block, as the reference
  *    requires (bindings.cpp `dequantize`: the last dimension holds whole
- *    blocks); otherwise KQ_ERR_INVALID_ARG.
+ *    blocks), and at most 2^31 - 1; otherwise KQ_ERR_INVALID_ARG.
  */
 #ifndef KQ_H
 #define KQ_H
@@ -199,7 +199,9 @@ int kq_qmm(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int
  *               kq_gather_mix takes it); -1 for a pair with a bad id
  *   x_sorted    [n_tokens*top_k, k] bf16 out (nullable): x[sorted_pair/top_k]
  *   err_flag    int32 device word (nullable): KQ_DEV_BAD_EXPERT on bad ids
- * Pairs with equal expert id keep (token, slot) order.  1 <= n_experts <= 256.
+ * Pairs with equal expert id keep (token, slot) order.  1 <= n_experts <= 256,
+ * n_tokens*top_k <= 2^30, and with x_sorted: x non-NULL, k a positive
+ * multiple of 8 (16-byte rows) of at most 2^31 - 1; else KQ_ERR_INVALID_ARG.
  */
 int kq_moe_sort(const int32_t* topk_ids, int64_t n_tokens, int32_t top_k, int32_t n_experts,
                 const uint16_t* x, int64_t k, uint32_t* sorted_ids, int32_t* sorted_pair,

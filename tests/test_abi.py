@@ -66,6 +66,7 @@ def test_matmul_argument_checks(lib, fn):
     assert f(3, A, 16, 256, A, 1, A, None) == UNSUPPORTED            # unknown codec
     assert f(kq.Q4_K, A, 16, 100, A, 1, A, None) == INVALID           # K not a block multiple
     assert f(kq.Q4_K, A, 16, 0, A, 1, A, None) == INVALID
+    assert f(kq.Q4_K, A, 16, 2**31, A, 1, A, None) == INVALID        # K past 32-bit counts
     assert f(kq.Q4_K, A, -1, 256, A, 1, A, None) == INVALID
     assert f(kq.Q4_K, None, 16, 256, A, 1, A, None) == INVALID        # null weights
     assert f(kq.Q4_K, MIS, 16, 256, A, 1, A, None) == ALIGN           # misaligned weights
@@ -83,6 +84,7 @@ def test_quantize_argument_checks(lib):
     assert f(5, A, 4, 256, A, None) == UNSUPPORTED
     assert f(kq.Q4_K, A, 4, 255, A, None) == INVALID
     assert f(kq.Q4_K, A, -1, 256, A, None) == INVALID
+    assert f(kq.Q8_0, A, 4, 2**31, A, None) == INVALID
     assert f(kq.Q4_K, None, 4, 256, A, None) == INVALID
     assert f(kq.Q4_K, A, 4, 256, MIS, None) == ALIGN
     assert f(kq.Q8_0, MIS, 4, 32, A, None) == ALIGN
@@ -95,6 +97,7 @@ def test_dequantize_argument_checks(lib):
     assert f(5, A, 4, 256, A, None) == UNSUPPORTED
     assert f(kq.Q6_K, A, 4, 255, A, None) == INVALID
     assert f(kq.Q6_K, A, 4, 256, None, None) == INVALID
+    assert f(kq.Q8_0, A, 4, 2**36, A, None) == INVALID
     assert f(kq.Q6_K, A, 4, 256, MIS, None) == ALIGN
     assert f(kq.Q6_K, A, 0, 256, None, None) == OK
 
@@ -106,6 +109,8 @@ def test_moe_argument_checks(lib):
     assert s(A, 4, 2, 257, None, 0, A, A, None, None, None, None) == INVALID
     assert s(A, 4, 2, 8, None, 64, A, A, None, A, None, None) == INVALID        # x_sorted without x
     assert s(A, 4, 2, 8, A, 60, A, A, A, A, None, None) == INVALID              # k % 8
+    assert s(A, 2**62, 4, 8, None, 0, A, A, None, None, None, None) == INVALID  # no overflow of the count
+    assert s(A, 4, 2, 8, A, 2**32, A, A, A, A, None, None) == INVALID           # k past 32-bit counts
     assert s(A, 0, 2, 8, None, 0, A, A, A, None, None, None) == OK
     t = lib.kq_expert_tile_map
     assert t(A, 1024, 8, A, 23, A, None, None) == INVALID                 # cap < ceil(1024/64) + 8
