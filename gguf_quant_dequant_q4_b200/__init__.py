@@ -100,6 +100,32 @@ def _need_cuda(*ts):
             raise ValueError("all tensors must be contiguous")
 
 
+def _need(t, what: str, size: int, count: int | None = None, exact: bool = False) -> None:
+    """Tensor ``t`` (if given) holds elements of ``size`` bytes, and at least
+    (or exactly) ``count`` of them: the C ABI takes bare pointers, so a buffer
+    shorter than the call's sizes would be read or written past its end."""
+    if t is None:
+        return
+    if t.element_size() != size:
+        raise TypeError(f"{what}: {size}-byte elements expected, got {t.dtype}")
+    if count is not None and (t.numel() != count if exact else t.numel() < count):
+        raise ValueError(f"{what}: {'exactly' if exact else 'at least'} {count} elements expected, got {t.numel()}")
+
+
+def _whole_blocks(qtype: int, k: int) -> bool:
+    # sizes the library accepts; anything else it rejects with its own status
+    return qtype in _BLOCK and k > 0 and k % _BLOCK[qtype][0] == 0
+
+
+def _need_bank(w, what: str, qtype: int, k: int, dims: int) -> None:
+    """Weight bytes with ``dims`` dimensions whose rows hold ``k`` values."""
+    _need(w, what, 1)
+    if w.dim() != dims:
+        raise ValueError(f"{what}: {dims} dimensions expected, got {w.dim()}")
+    if _whole_blocks(qtype, k) and w.shape[-1] != row_bytes(qtype, k):
+        raise ValueError(f"{what}: rows of {row_bytes(qtype, k)} bytes expected for k = {k}, got {w.shape[-1]}")
+
+
 def block_info(qtype: int) -> tuple[int, int]:
     v, b = _int(), _int()
     _check(lib().kq_block_info(qtype, ctypes.byref(v), ctypes.byref(b)), "kq_block_info")
@@ -134,8 +160,12 @@ def _bf16_bits(x: torch.Tensor) -> torch.Tensor:
 def dequantize(w: torch.Tensor, qtype: int, k: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """fp32 [..., N, K] decode of wire bytes [..., N, row_bytes] (bit-exact)."""
     rows = w.numel() // max(1, w.shape[-1]) if w.dim() else 0
+    _need(w, "w", 1)
+    if w.dim() and _whole_blocks(qtype, k) and w.shape[-1] != row_bytes(qtype, k):
+        raise ValueError(f"w: rows of {row_bytes(qtype, k)} bytes expected for k = {k}, got {w.shape[-1]}")
     if out is None:
         out = torch.empty(*w.shape[:-1], k, dtype=torch.float32, device=w.device)
+    _need(out, "out", 4, rows * k)
     _need_cuda(w, out)
     _check(lib().kq_dequantize(qtype, _ptr(w), rows, k, _ptr(out), _stream(stream)), "kq_dequantize")
     return out
@@ -149,6 +179,8 @@ def quantize(w: torch.Tensor, qtype: int, out: torch.Tensor | None = None, strea
     rows = w.numel() // max(1, k)
     if out is None:
         out = torch.empty(*w.shape[:-1], row_bytes(qtype, k), dtype=torch.uint8, device=w.device)
+    if _whole_blocks(qtype, k):
+        _need(out, "out", 1, rows * row_bytes(qtype, k))
     _need_cuda(w, out)
     _check(lib().kq_quantize(qtype, _ptr(w), rows, k, _ptr(out), _stream(stream)), "kq_quantize")
     return out
@@ -159,8 +191,10 @@ def qmv(x: torch.Tensor, w: torch.Tensor, qtype: int, out: torch.Tensor | None =
     x = _bf16_bits(x)
     m, k = x.shape
     n = w.shape[0]
+    _need_bank(w, "w", qtype, k, 2)
     if out is None:
         out = torch.empty(m, n, dtype=torch.float32, device=x.device)
+    _need(out, "out", 4, m * n)
     _need_cuda(x, w, out)
     _check(lib().kq_qmv(qtype, _ptr(w), n, k, _ptr(x), m, _ptr(out), _stream(stream)), "kq_qmv")
     return out
@@ -171,8 +205,10 @@ def qmm(x: torch.Tensor, w: torch.Tensor, qtype: int, out: torch.Tensor | None =
     x = _bf16_bits(x)
     m, k = x.shape
     n = w.shape[0]
+    _need_bank(w, "w", qtype, k, 2)
     if out is None:
         out = torch.empty(m, n, dtype=torch.float32, device=x.device)
+    _need(out, "out", 4, m * n)
     _need_cuda(x, w, out)
     _check(lib().kq_qmm(qtype, _ptr(w), n, k, _ptr(x), m, _ptr(out), _stream(stream)), "kq_qmm")
     return out
@@ -188,6 +224,8 @@ def moe_sort(topk_ids: torch.Tensor, n_experts: int, x: torch.Tensor | None = No
     plus inv_order (the sorted row of every pair) when with_inverse is set."""
     t, top_k = topk_ids.shape
     rows = t * top_k
+    _need(topk_ids, "topk_ids", 4)
+    _need(err, "err", 4, 1)
     dev = topk_ids.device
     sids = torch.empty(rows, dtype=torch.int32, device=dev)
     pair = torch.empty(rows, dtype=torch.int32, device=dev)
@@ -197,6 +235,7 @@ def moe_sort(topk_ids: torch.Tensor, n_experts: int, x: torch.Tensor | None = No
     if x is not None:
         x = _bf16_bits(x)
         k = x.shape[1]
+        _need(x, "x", 2, t * k)
         xs = torch.empty(rows, k, dtype=x.dtype, device=dev)
     _need_cuda(topk_ids, x, xs, err)
     _check(lib().kq_moe_sort(_ptr(topk_ids), t, top_k, n_experts, _ptr(x), k, _ptr(sids), _ptr(pair), _ptr(inv),
@@ -209,6 +248,8 @@ def expert_tile_map(sorted_ids: torch.Tensor, n_experts: int, cap: int | None = 
     """(map int32 [cap, 3] of (expert, row_start, num_rows), count int32 [1])."""
     rows = sorted_ids.numel()
     cap = map_capacity(rows, n_experts) if cap is None else cap
+    _need(sorted_ids, "sorted_ids", 4)
+    _need(err, "err", 4, 1)
     m = torch.empty(cap, 3, dtype=torch.int32, device=sorted_ids.device)
     c = torch.empty(1, dtype=torch.int32, device=sorted_ids.device)
     _need_cuda(sorted_ids, err)
@@ -224,8 +265,15 @@ def gather_qmm(x_sorted: torch.Tensor, w_bank: torch.Tensor, qtype: int, tile_ma
     x_sorted = _bf16_bits(x_sorted)
     rows, k = x_sorted.shape
     e, n = w_bank.shape[0], w_bank.shape[1]
+    _need_bank(w_bank, "w_bank", qtype, k, 3)
+    _need(tile_map, "tile_map", 4)
+    if tile_map.dim() != 2 or tile_map.shape[1] != 3:
+        raise ValueError(f"tile_map: [cap, 3] expected, got {tuple(tile_map.shape)}")
+    _need(count, "count", 4, 1)
+    _need(err, "err", 4, 1)
     if out is None:
         out = torch.empty(rows, n, dtype=torch.float32, device=x_sorted.device)
+    _need(out, "out", 4, rows * n)
     _need_cuda(x_sorted, w_bank, tile_map, count, out, err)
     _check(lib().kq_gather_qmm(qtype, _ptr(w_bank), e, n, k, _ptr(x_sorted), rows, _ptr(tile_map), _ptr(count),
                                tile_map.shape[0], _ptr(out), _ptr(err), _stream(stream)), "kq_gather_qmm")
@@ -241,8 +289,13 @@ def gather_qmv(x: torch.Tensor, w_bank: torch.Tensor, qtype: int, ids: torch.Ten
     t, top_k = ids.shape
     k = x.shape[-1]
     e, n = w_bank.shape[0], w_bank.shape[1]
+    _need_bank(w_bank, "w_bank", qtype, k, 3)
+    _need(ids, "ids", 4)
+    _need(err, "err", 4, 1)
+    _need(x, "x", 2, (t if x_per_token else t * top_k) * k)
     if out is None:
         out = torch.empty(t * top_k, n, dtype=torch.float32, device=x.device)
+    _need(out, "out", 4, t * top_k * n)
     _need_cuda(x, w_bank, ids, out, err)
     _check(lib().kq_gather_qmv(qtype, _ptr(w_bank), e, n, k, _ptr(x), int(bool(x_per_token)), _ptr(ids), t, top_k,
                                _ptr(out), _ptr(err), _stream(stream)), "kq_gather_qmv")
@@ -254,8 +307,13 @@ def gather_mix(y: torch.Tensor, inv_order: torch.Tensor, scores: torch.Tensor, o
     """out[t] = sum_s scores[t, s] * y[inv_order[t * top_k + s]] (fp32, slots in order)."""
     rows, n = y.shape
     t, top_k = scores.shape
+    _need(y, "y", 4)
+    _need(inv_order, "inv_order", 4, t * top_k)
+    _need(scores, "scores", 4)
+    _need(err, "err", 4, 1)
     if out is None:
         out = torch.empty(t, n, dtype=torch.float32, device=y.device)
+    _need(out, "out", 4, t * n)
     _need_cuda(y, inv_order, scores, out, err)
     _check(lib().kq_gather_mix(_ptr(y), rows, n, _ptr(inv_order), _ptr(scores), t, top_k, _ptr(out), _ptr(err),
                                _stream(stream)), "kq_gather_mix")
@@ -270,8 +328,16 @@ def moe_glu_gather(x: torch.Tensor, gate_bank: torch.Tensor, up_bank: torch.Tens
     t, top_k = ids.shape
     k = x.shape[-1]
     e, n = gate_bank.shape[0], gate_bank.shape[1]
+    _need_bank(gate_bank, "gate_bank", qtype, k, 3)
+    _need_bank(up_bank, "up_bank", qtype, k, 3)
+    if up_bank.shape != gate_bank.shape:
+        raise ValueError(f"up_bank: shape {tuple(gate_bank.shape)} expected, got {tuple(up_bank.shape)}")
+    _need(ids, "ids", 4)
+    _need(err, "err", 4, 1)
+    _need(x, "x", 2, t * k)
     if out is None:
         out = torch.empty(t * top_k, n, dtype=torch.float32, device=x.device)
+    _need(out, "out", 4, t * top_k * n)
     _need_cuda(x, gate_bank, up_bank, ids, out, err)
     _check(lib().kq_moe_glu_gather(qtype, _ptr(gate_bank), _ptr(up_bank), e, n, k, _ptr(x), _ptr(ids), t, top_k,
                                    act, limit, _ptr(out), _ptr(err), _stream(stream)), "kq_moe_glu_gather")
