@@ -93,11 +93,12 @@ def _stream(stream=None) -> int:
 
 
 def _need_cuda(*ts):
-    for t in ts:
-        if t is not None and not t.is_cuda:
-            raise ValueError("all tensors must be CUDA tensors")
-        if t is not None and not t.is_contiguous():
-            raise ValueError("all tensors must be contiguous")
+    # contiguity first: a strided view (say, some rows of every expert of a
+    # bank) would otherwise be walked with the packed stride
+    if any(t is not None and not t.is_contiguous() for t in ts):
+        raise ValueError("all tensors must be contiguous")
+    if any(t is not None and not t.is_cuda for t in ts):
+        raise ValueError("all tensors must be CUDA tensors")
 
 
 def _need(t, what: str, size: int, count: int | None = None, exact: bool = False) -> None:

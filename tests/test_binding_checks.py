@@ -135,3 +135,20 @@ def test_decode_moe_buffers():
         kq.gather_mix(y, i32(t * top_k), torch.zeros(t, top_k, dtype=torch.float64))
     with pytest.raises(ValueError, match="at least 48 elements"):
         kq.gather_mix(y, i32(t * top_k), f32(t, top_k), out=f32(t - 1, n))
+
+
+def test_strided_views_are_refused_and_leading_slices_pass():
+    # a bank sliced along its rows is a strided view: refused, never walked
+    # with the packed stride; a slice of whole experts is contiguous (an offset
+    # pointer) and goes through
+    t, top_k, e, n, k = 2, 2, 6, 16, 256
+    bank = u8(e, n, kq.row_bytes(kq.Q4_K, k))
+    ids = i32(t, top_k)
+    with pytest.raises(ValueError, match="contiguous"):
+        kq.gather_qmv(bf(t * top_k, k), bank[:, : n // 2], kq.Q4_K, ids)
+    with pytest.raises(ValueError, match=CUDA):
+        kq.gather_qmv(bf(t * top_k, k), bank[2:5], kq.Q4_K, ids)
+    with pytest.raises(ValueError, match="contiguous"):
+        kq.qmv(bf(k, 2).t(), bank[0], kq.Q4_K)
+    with pytest.raises(ValueError, match=CUDA):
+        kq.qmv(bf(2, k), bank[0, 4:], kq.Q4_K)

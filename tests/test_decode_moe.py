@@ -209,6 +209,36 @@ def test_moe_glu_gather_full_bank_sampled():
     check_glu(y[:, cols], ref, g, u, ag, au, kq.ACT_SILU)
 
 
+def test_equal_length_banks_and_expert_slices():
+    # q4_K and q4_0 rows of K values are equally long (K/32 * 18 bytes): one
+    # buffer refilled with either codec's bytes is decoded as the codec the
+    # call names (the library keeps no state per weight pointer), and a slice
+    # of whole experts of a bank (an offset pointer) is the bank it views
+    tokens, top_k, experts, n, k = 1, 2, 8, 300, 2048
+    assert kq.row_bytes(kq.Q4_K, k) == kq.row_bytes(kq.Q4_0, k)
+    ids = synth.routing(tokens, experts, top_k, seed=2)
+    x = synth.activations(tokens * top_k, k, seed=3)
+    buf = torch.empty(experts, n, kq.row_bytes(kq.Q4_K, k), dtype=torch.uint8, device="cuda")
+
+    def run(qtype, bank, rid):
+        out = torch.full((tokens * top_k, n), float("nan"), device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        kq.gather_qmv(dev_bf16(x), bank, qtype, torch.from_numpy(rid).cuda(), out=out, err=err)
+        return out.cpu().numpy(), int(err.item())
+
+    for qtype, seed in ((kq.Q4_K, 1), (kq.Q4_0, 1), (kq.Q4_K, 4)):
+        w = synth.weights(qtype, n, k, seed=seed, experts=experts)
+        buf.copy_(torch.from_numpy(w))
+        y, e = run(qtype, buf, ids)
+        assert e == 0
+        check_pairs(qtype, w, k, x, ids, y)
+    # experts 3..7 of the last bank's buffer
+    sub = synth.routing(tokens, experts - 3, top_k, seed=5)
+    y, e = run(kq.Q4_K, buf[3:], sub)
+    assert e == 0
+    check_pairs(kq.Q4_K, w[3:], k, x, sub, y)
+
+
 def test_decode_moe_edge_cases():
     # one pair; zero tokens (nothing enqueued); top-8 mix over the smallest N
     w = synth.weights(kq.Q4_K, 64, 256, seed=1, experts=2)
