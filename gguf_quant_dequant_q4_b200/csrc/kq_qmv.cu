@@ -8,11 +8,14 @@
 // The path is HBM-bound, so the design goal is to spend as few instructions
 // per weight as possible while reading every weight byte exactly once:
 //
-//  * Each CTA owns 16 weight rows and all of K.  Its row segments (several
-//    blocks per row) are streamed into a ring of shared-memory stages by 1-D
-//    bulk async copies (one per row, issued by warp 0, completion counted on
-//    an mbarrier), so many kilobytes per SM are in flight without registers.
-//  * The 8 warps split the blocks of a stage.  A warp decodes its 16 rows into
+//  * One CTA per SM (at most) owns a balanced contiguous range of weight rows,
+//    walked in 16-row groups, and all of K.  Its row segments (several blocks
+//    per row) are streamed into a ring of shared-memory stages by 1-D bulk
+//    async copies (one per row, issued by a producer warp, completion counted
+//    on an mbarrier; rows that are not a 16-byte multiple are staged with
+//    2-byte loads instead), so many kilobytes per SM are in flight without
+//    registers.
+//  * 16 consumer warps split the blocks of a stage.  A warp decodes its 16 rows into
 //    m16n8k16 tensor-core A fragments whose entries are EXACT integers in
 //    binary16: the codes themselves (q6_K, q8_0) or code * 6-bit scale
 //    (q4_K, at most 945).  The activations, rounded once to binary16, are the
@@ -40,8 +43,9 @@
 //    (per super-chunk of K) are multiplied by a power of two that puts their
 //    largest magnitude at 2^T; the warps multiply their partial sums by the
 //    inverse, so the relative precision does not depend on the scale of x.
-//  * Partial sums of the 8 warps are combined in shared memory in a fixed
-//    order: no atomics, bitwise reproducible.
+//  * Partial sums of the 16 consumer warps go to shared memory and a reducer
+//    warp adds them in a fixed order and stores y: no atomics, bitwise
+//    reproducible.
 #include "kq_device.cuh"
 #include "kq_launch.h"
 
