@@ -47,6 +47,14 @@
  *  - `k` must be a multiple of the codec's values_per_block, as the reference
  *    requires (bindings.cpp `dequantize`: the last dimension holds whole
  *    blocks), and at most 2^31 - 1; otherwise KQ_ERR_INVALID_ARG.
+ *  - Environment (read once per process; A/B levers, not needed in use):
+ *    KQ_NO_PDL=1 launches the decode kernels (kq_qmv, kq_gather_qmv,
+ *    kq_moe_glu_gather) without programmatic dependent launch, so a launch
+ *    no longer overlaps its start-up with the end of the previous kernel on
+ *    the stream (the kernels and their results are unchanged);
+ *    KQ_QMM_1SM=1 runs kq_qmm / kq_gather_qmm on single CTAs (128 weight
+ *    rows per unit, MMA M = 128) instead of CTA pairs, a performance lever
+ *    that the test suite does not cover.
  */
 #ifndef KQ_H
 #define KQ_H
