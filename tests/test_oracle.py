@@ -201,9 +201,11 @@ def test_matches_gguf_quants(qtype):
     ref = gguf.quants.dequantize(w, gguf.GGMLQuantizationType(qtype)).astype(np.float32)
     y = oracle.dequantize(qtype, w, k)
     assert np.array_equal(bits(y), bits(ref))
-    # fully random bytes too (any fp16 d, any int8 scale), excluding NaN/inf scales
+    # fully random bytes too (any fp16 d, any int8 scale): where a scale is
+    # NaN or infinite, only the position of the non-finite values is compared
     raw = np.random.default_rng(3).integers(0, 256, size=(64, synth.row_bytes(qtype, 256)), dtype=np.uint8)
-    ref = gguf.quants.dequantize(raw, gguf.GGMLQuantizationType(qtype)).astype(np.float32)
+    with np.errstate(invalid="ignore", over="ignore"):
+        ref = gguf.quants.dequantize(raw, gguf.GGMLQuantizationType(qtype)).astype(np.float32)
     y = oracle.dequantize(qtype, raw, 256)
     fin = np.isfinite(ref)
     assert np.array_equal(np.isfinite(y), fin)
