@@ -322,8 +322,8 @@ int kq_moe_glu_gather(int type, const void* gate_bank, const void* up_bank, int3
  * no fused multiply-add, so results are bit-reproducible.
  *   y [rows, n] fp32 (e.g. kq_gather_qmm's output), inv_order
  *   [n_tokens*top_k] int32 (kq_moe_sort's), scores [n_tokens, top_k] fp32,
- *   out [n_tokens, n] fp32.  n % 4 == 0 and 1 <= top_k <= 64, else
- *   KQ_ERR_INVALID_ARG.
+ *   out [n_tokens, n] fp32.  n % 4 == 0, n <= 67107840 (4 x 256 x 65535)
+ *   and 1 <= top_k <= 64, else KQ_ERR_INVALID_ARG.
  *   err_flag (nullable): KQ_DEV_BAD_RANGE for an inv_order entry outside
  *   [0, rows); that term is left out of the sum.
  */

@@ -147,6 +147,7 @@ def test_decode_moe_argument_checks(lib):
     assert m(A, 8, 6, A, A, 4, 2, A, None, None) == INVALID                      # n % 4
     assert m(A, 8, 8, A, A, 4, 0, A, None, None) == INVALID                      # top_k < 1
     assert m(A, 8, 8, A, A, 4, 65, A, None, None) == INVALID                     # top_k > 64
+    assert m(A, 8, 4 * 256 * 65536, A, A, 4, 2, A, None, None) == INVALID        # past the grid's x extent
     assert m(A, 8, 8, None, A, 4, 2, A, None, None) == INVALID
     assert m(A, 8, 8, A, A, 4, 2, MIS, None, None) == ALIGN
     assert m(MIS, 8, 8, A, A, 4, 2, A, None, None) == ALIGN
