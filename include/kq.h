@@ -188,6 +188,12 @@ int kq_qmv(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int
  * mlx-kquant bindings.cpp `quantized_matmul`; README "Performance"
  * (single-pass matmul on the tensor units).
  *   w [n, row_bytes], x [m, k] bf16, y [m, n] fp32.
+ * k % 256 == 0 (else KQ_ERR_UNSUPPORTED); m, n <= 2^31 - 1 (else
+ * KQ_ERR_INVALID_ARG).  q6_K rows that
+ * are not a 16-byte multiple are read through a flat byte view whose
+ * coordinates are 32-bit: the weight bytes plus two tiles of rows must stay
+ * below 2^31 bytes (else KQ_ERR_UNSUPPORTED; kq_gather_qmm likewise for the
+ * whole bank).
  */
 int kq_qmm(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int64_t m,
            float* y, void* stream);
@@ -238,9 +244,10 @@ int kq_expert_tile_map(const uint32_t* sorted_ids, int64_t rows, int32_t n_exper
  * map, y[r, :] = x_sorted[r, :] . dequant(W[e])^T for start <= r < start + n.
  * mlx-kquant bindings.cpp, `gather_qmm_seg`: "valid tiles never span experts
  * and must cover every x row exactly once (uncovered output rows are left
- * unwritten)"; num_rows <= 64.  Each CTA owns one (expert, 128 weight rows)
- * pair and streams all of that expert's tiles through the tensor cores, so
- * each expert weight tile is decoded once per pass.  Any number of tiles:
+ * unwritten)"; num_rows <= 64.  Each CTA pair owns one (expert, 256 weight
+ * rows) unit at a time and streams up to four of that expert's tiles through
+ * the tensor cores, so each expert weight tile is decoded once per four map
+ * tiles.  Any number of tiles:
  * the map is taken in windows of 1024 slots, one kernel launch per window
  * (ceil(cap / 1024) launches; a window past the device-side count has no
  * work), and an expert's tiles are grouped in map order within a window.
