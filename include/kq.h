@@ -189,11 +189,10 @@ int kq_qmv(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int
  * (single-pass matmul on the tensor units).
  *   w [n, row_bytes], x [m, k] bf16, y [m, n] fp32.
  * k % 256 == 0 (else KQ_ERR_UNSUPPORTED); m, n <= 2^31 - 1 (else
- * KQ_ERR_INVALID_ARG).  q6_K rows that
- * are not a 16-byte multiple are read through a flat byte view whose
- * coordinates are 32-bit: the weight bytes plus two tiles of rows must stay
- * below 2^31 bytes (else KQ_ERR_UNSUPPORTED; kq_gather_qmm likewise for the
- * whole bank).
+ * KQ_ERR_INVALID_ARG).  q6_K rows that are not a 16-byte multiple are read
+ * through a flat byte view whose coordinates are 32-bit: the weight bytes
+ * plus two tiles of rows must stay below 2^31 bytes (else
+ * KQ_ERR_UNSUPPORTED; kq_gather_qmm likewise for the whole bank).
  */
 int kq_qmm(int type, const void* w, int64_t n, int64_t k, const uint16_t* x, int64_t m,
            float* y, void* stream);
