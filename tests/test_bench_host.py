@@ -68,6 +68,19 @@ def test_reference_arm_json(monkeypatch, capsys):
     assert line["metric"] == bench.METRIC
 
 
+def test_reference_arm_other_ranks_do_no_work(monkeypatch, capsys):
+    # under torchrun only rank 0 times the oracle and prints; another rank
+    # returns at once, without a process group or any oracle call
+    def no_call(seconds=10.0):
+        raise AssertionError("rank 1 ran the oracle")
+    monkeypatch.setattr(bench, "cpu_sample", no_call)
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    bench.main(["--impl", "reference", "--steps", "2", "--warmup", "3"])
+    assert capsys.readouterr().out == ""
+
+
 def test_cpu_sample_is_bounded():
     r = bench.cpu_sample(seconds=0.0)       # one pass of the oracle on c1
     assert r["kind"] == "oracle" and r["value"] > 0 and r["cores"] >= 1
